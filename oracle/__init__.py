@@ -1,0 +1,211 @@
+"""CPU oracle for quantized-KV attention -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The CUDA library never calls it, and a
+missing CUDA extension is an error there, never a reason to come here.
+
+Thin ``ctypes`` wrapper around ``liboracle.so`` (built from ``qkv_oracle.cpp``
+by ``oracle/build.py``).  All arrays are numpy; half-precision tensors are
+passed as their raw ``uint16`` bit patterns together with a dtype name.
+
+What each function follows is stated in ``qkv_oracle.cpp``: the MLX
+quantized-KV branch ("add fast::quantized_kv_update": fast.cpp fallback math,
+sdpa_vector.h packing and dequant, quantized.h eps), the MLX CUDA WIP page
+(load_quantized dequant) and llama.cpp PR #25556 (the Q8_0 KV format).
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from dataclasses import dataclass
+from typing import Optional, Sequence
+
+import numpy as np
+
+from . import build as _build
+
+_DT = {"f16": 0, "bf16": 1, "f32": 2}
+_FMT = {"affine": 0, "q8_0": 1}
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = C.CDLL(path)
+        p = C.c_void_p
+        i64 = C.c_int64
+        i32 = C.c_int
+        for name in ("orc_f32_to_f16", "orc_f16_to_f32", "orc_f32_to_bf16", "orc_bf16_to_f32"):
+            getattr(L, name).argtypes = [p, p, i64]
+            getattr(L, name).restype = None
+        L.orc_quantize.argtypes = [i32, p, i32, i64, i32, i32, i32, p, p, p, i32]
+        L.orc_quantize.restype = i32
+        L.orc_dequantize.argtypes = [i32, i32, i32, p, p, p, i64, i32, p]
+        L.orc_dequantize.restype = i32
+        common = [p, i32, i32, i32, i32, i32,
+                  i32, i32, i32, p, p, p,
+                  i32, i32, i32, p, p, p,
+                  i64, i64, C.c_double, i32, p, i32, i64, i64, i64]
+        L.orc_attention.argtypes = common + [i32, i32, p, i64, p, i32]
+        L.orc_attention.restype = i32
+        L.orc_attention_probs.argtypes = common + [i32, i32, i32, p, p]
+        L.orc_attention_probs.restype = i32
+        _lib = L
+    return _lib
+
+
+def _ptr(a: Optional[np.ndarray]):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"], "oracle arrays must be C-contiguous"
+    return a.ctypes.data_as(C.c_void_p)
+
+
+def default_threads() -> int:
+    return max(1, os.cpu_count() or 1)
+
+
+# ----------------------------------------------------------------------------
+# half-precision conversions (IEEE-754, round-to-nearest-even)
+# ----------------------------------------------------------------------------
+def f32_to_f16(x: np.ndarray) -> np.ndarray:
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    y = np.empty(x.shape, np.uint16)
+    lib().orc_f32_to_f16(_ptr(x), _ptr(y), x.size)
+    return y
+
+
+def f16_to_f32(x: np.ndarray) -> np.ndarray:
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    y = np.empty(x.shape, np.float32)
+    lib().orc_f16_to_f32(_ptr(x), _ptr(y), x.size)
+    return y
+
+
+def f32_to_bf16(x: np.ndarray) -> np.ndarray:
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    y = np.empty(x.shape, np.uint16)
+    lib().orc_f32_to_bf16(_ptr(x), _ptr(y), x.size)
+    return y
+
+
+def bf16_to_f32(x: np.ndarray) -> np.ndarray:
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    y = np.empty(x.shape, np.float32)
+    lib().orc_bf16_to_f32(_ptr(x), _ptr(y), x.size)
+    return y
+
+
+def to_f64(x: np.ndarray, dtype: str) -> np.ndarray:
+    """Raw half bits (or float32) -> float64, exactly."""
+    if dtype == "f16":
+        return f16_to_f32(x).astype(np.float64)
+    if dtype == "bf16":
+        return bf16_to_f32(x).astype(np.float64)
+    return np.asarray(x, dtype=np.float32).astype(np.float64)
+
+
+# ----------------------------------------------------------------------------
+# quantized cache
+# ----------------------------------------------------------------------------
+@dataclass
+class QCache:
+    """One of K or V: codes [B,Hkv,Lcap,D*bits/32] uint32, scales (and for the
+    affine format biases) [B,Hkv,Lcap,D/gs] as fp16 bit patterns."""
+    fmt: str
+    bits: int
+    gs: int
+    codes: np.ndarray
+    scales: np.ndarray
+    biases: Optional[np.ndarray]
+
+    @property
+    def Lcap(self) -> int:
+        return self.codes.shape[-2]
+
+
+def quantize(x: np.ndarray, dtype: str, fmt: str = "affine", gs: int = 64,
+             bits: int = 4, nthreads: Optional[int] = None) -> QCache:
+    """Quantize x [..., D] (raw half bits, or float32 for dtype 'f32')."""
+    if fmt == "q8_0":
+        gs, bits = 32, 8
+    x = np.ascontiguousarray(x)
+    D = x.shape[-1]
+    rows = x.size // D
+    codes = np.zeros(x.shape[:-1] + (D * bits // 32,), np.uint32)
+    scales = np.zeros(x.shape[:-1] + (D // gs,), np.uint16)
+    biases = np.zeros_like(scales)
+    rc = lib().orc_quantize(_FMT[fmt], _ptr(x), _DT[dtype], rows, D, gs, bits,
+                            _ptr(codes), _ptr(scales), _ptr(biases),
+                            nthreads or default_threads())
+    if rc:
+        raise ValueError("oracle quantize: unsupported shape/bits")
+    return QCache(fmt, bits, gs, codes, scales, biases if fmt == "affine" else None)
+
+
+def dequantize(c: QCache, D: int) -> np.ndarray:
+    rows = c.codes.size // c.codes.shape[-1]
+    out = np.empty(c.codes.shape[:-1] + (D,), np.float64)
+    lib().orc_dequantize(_FMT[c.fmt], c.bits, c.gs, _ptr(c.codes), _ptr(c.scales),
+                         _ptr(c.biases), rows, D, _ptr(out))
+    return out
+
+
+@dataclass
+class Mask:
+    kind: str = "none"                 # none | causal | additive
+    add: Optional[np.ndarray] = None   # raw bits (f16/bf16) or float32
+    dtype: str = "f32"
+    strides: Sequence[int] = (0, 0, 0)  # element strides over (b, h, query)
+
+
+def _common_args(q64, k: QCache, v: QCache, L, scale, mask: Optional[Mask]):
+    B, Hq, Lq, D = q64.shape
+    Hkv = k.codes.shape[1]
+    mask = mask or Mask()
+    kind = {"none": 0, "causal": 1, "additive": 2}[mask.kind]
+    add = None if mask.add is None else np.ascontiguousarray(mask.add)
+    return [
+        _ptr(q64), B, Hq, Hkv, Lq, D,
+        _FMT[k.fmt], k.bits, k.gs, _ptr(k.codes), _ptr(k.scales), _ptr(k.biases),
+        _FMT[v.fmt], v.bits, v.gs, _ptr(v.codes), _ptr(v.scales), _ptr(v.biases),
+        k.Lcap, L, float(scale), kind, _ptr(add), _DT[mask.dtype],
+        int(mask.strides[0]), int(mask.strides[1]), int(mask.strides[2]),
+    ], add
+
+
+def attention(q: np.ndarray, q_dtype: str, k: QCache, v: QCache, L: int,
+              scale: float, mask: Optional[Mask] = None, mode: str = "two_pass",
+              nsplit: int = 1, rows: Optional[np.ndarray] = None,
+              nthreads: Optional[int] = None) -> np.ndarray:
+    """fp64 attention output [B,Hq,Lq,D].  ``rows`` (flattened (b,h,i) ids)
+    restricts the computation to a subset; other rows are left NaN."""
+    q64 = np.ascontiguousarray(to_f64(q, q_dtype))
+    B, Hq, Lq, D = q64.shape
+    out = np.full((B, Hq, Lq, D), np.nan)
+    args, keep = _common_args(q64, k, v, L, scale, mask)
+    r = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    rc = lib().orc_attention(*args, {"two_pass": 0, "online": 1, "split": 2}[mode],
+                             nsplit, _ptr(r), 0 if r is None else r.size, _ptr(out),
+                             nthreads or default_threads())
+    if rc:
+        raise ValueError("oracle attention: invalid arguments")
+    return out
+
+
+def attention_probs(q: np.ndarray, q_dtype: str, k: QCache, v: QCache, L: int,
+                    scale: float, b: int, h: int, i: int,
+                    mask: Optional[Mask] = None):
+    """Softmax row (length L) and output (length D) of query row (b, h, i)."""
+    q64 = np.ascontiguousarray(to_f64(q, q_dtype))
+    D = q64.shape[-1]
+    probs = np.empty(L, np.float64)
+    o = np.empty(D, np.float64)
+    args, keep = _common_args(q64, k, v, L, scale, mask)
+    rc = lib().orc_attention_probs(*args, b, h, i, _ptr(probs), _ptr(o))
+    if rc:
+        raise ValueError("oracle attention_probs: invalid arguments")
+    return probs, o
