@@ -1,0 +1,539 @@
+#!/usr/bin/env python
+"""Benchmark of the quantized-KV attention hot path on B200.
+
+One step = one decode call (qsdpa_decode) of the workload named by --workload
+(default: B=1, Hq=32, Hkv=8, D=128, L=65536, affine 4-bit groups of 64,
+uniform fp16 inputs, scale 1.0 -- the MLX quantized-SDPA benchmark shape).
+The primary number is HBM throughput in GB/s of ALGORITHMIC bytes (packed K/V
+codes, scales, biases, q and out) per call; microseconds per call are reported
+beside it.  Inputs are synthetic (seeded SplitMix64), quantized on the GPU by
+qkv_quantize_update; the timed calls rotate over enough cache copies that the
+data read in one call is no longer in the 126 MB L2 when it is read again.
+
+--impl reference runs the CPU oracle (the only reference this repository has)
+on a bounded sample of the same workload and reports the same metric.
+
+Launch: python bench.py [--gpus N --steps K --warmup W]; for N > 1 under
+torch.distributed.run, one process per GPU (independent replicas: the path
+has no cross-GPU exchange), rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "quant-KV decode attention µs/call and HBM GB/s (% of peak) at L=64K, 1 B200"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+# ----------------------------------------------------------------------------
+# clocks
+# ----------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.lines = []
+        self.proc = None
+        self.windows = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self, t0, t1):
+        self.windows.append((t0, t1))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        inside = []
+        for t, line in self.lines:
+            if any(a <= t <= b for a, b in self.windows):
+                inside.append(line)
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in inside:
+            parts = [p.strip() for p in line.split(",")]
+            try:
+                sm.append(float(parts[2]))
+                smax.append(float(parts[3]))
+            except (ValueError, IndexError):
+                continue
+            for n, v in zip(names, parts[6:10]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------
+# helpers
+# ----------------------------------------------------------------------------
+def dev16(bits, dtype, device):
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16))
+    return t.view(torch.float16 if dtype == "f16" else torch.bfloat16).to(device)
+
+
+def build_caches(w, inp, ncopies, device):
+    """Quantize the workload's K/V on the GPU into `ncopies` cache copies."""
+    import torch
+    from quantized_kv_attention_split_b200 import qkv
+    fmt = qkv.Q8_0 if w.fmt == "q8_0" else qkv.AFFINE
+    kd_src = dev16(inp.k, w.kv_dtype, device)
+    vd_src = dev16(inp.v, w.kv_dtype, device)
+    caches = []
+    for _ in range(ncopies):
+        kc = qkv.QuantCache.empty(w.B, w.Hkv, w.Lcap, w.D, fmt, w.bits, w.gs, device)
+        vc = qkv.QuantCache.empty(w.B, w.Hkv, w.Lcap, w.D, fmt, w.bits, w.gs, device)
+        qkv.qkv_quantize_update(kd_src, vd_src, kc, vc, 0)
+        caches.append((kc, vc))
+    del kd_src, vd_src
+    torch.cuda.synchronize()
+    return caches
+
+
+def graph_time(step, K, W, sampler=None, min_window_s=0.3):
+    """Device time of exactly K calls of step(i): W eager warm-up calls, then
+    K calls captured in CUDA graphs and replayed between events."""
+    import torch
+    for i in range(W):
+        step(i)
+    torch.cuda.synchronize()
+    chunk = min(K, 256)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    graphs = []
+    with torch.cuda.stream(s):
+        g1 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g1, stream=s):
+            for i in range(chunk):
+                step(i)
+        graphs.append(g1)
+        rem = K % chunk
+        g2 = None
+        if rem:
+            g2 = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g2, stream=s):
+                for i in range(rem):
+                    step(i)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g1.replay()                                   # one untimed replay
+    torch.cuda.synchronize()
+    reps = K // chunk
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if torch.distributed.is_available() and torch.distributed.is_initialized():
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t0 = time.time()
+    start.record()
+    for _ in range(reps):
+        g1.replay()
+    if g2 is not None:
+        g2.replay()
+    end.record()
+    torch.cuda.synchronize()
+    t1 = time.time()
+    ms = start.elapsed_time(end)
+    extra = False
+    if sampler is not None:
+        sampler.mark(t0, t1)
+        if t1 - t0 < min_window_s:
+            # too short for the 50 ms clock sampler: replay the same graph
+            # (untimed) for a while and sample the clocks there as well
+            extra = True
+            n = max(1, int(min_window_s / max(1e-6, ms / 1e3 / max(1, reps))))
+            t2 = time.time()
+            for _ in range(n):
+                g1.replay()
+            torch.cuda.synchronize()
+            sampler.mark(t2, time.time())
+    del graphs
+    return ms / K, extra
+
+
+def oracle_rows_time(w, host_k, host_v, q_bits, nrows_target_s=15.0, max_rows=None):
+    """Time the CPU oracle on a sample of query rows of the workload."""
+    import oracle
+    total_rows = w.B * w.Hq * w.Lq
+    t0 = time.time()
+    oracle.attention(q_bits, w.q_dtype, host_k, host_v, w.L, w.scale,
+                     mask=oracle.Mask("causal") if w.mask == "causal" else None,
+                     rows=np.array([0]), nthreads=1)
+    t_row = max(1e-4, time.time() - t0)
+    threads = oracle.default_threads()
+    nrows = int(min(total_rows, max(threads, nrows_target_s * threads / t_row)))
+    if max_rows:
+        nrows = min(nrows, max_rows)
+    rows = np.linspace(0, total_rows - 1, nrows).astype(np.int64)
+    t0 = time.time()
+    out = oracle.attention(q_bits, w.q_dtype, host_k, host_v, w.L, w.scale,
+                           mask=oracle.Mask("causal") if w.mask == "causal" else None,
+                           rows=rows, nthreads=threads)
+    dt = time.time() - t0
+    return dt, nrows, total_rows, threads, rows, out
+
+
+def host_cache(dc, fmt):
+    import oracle
+    codes = dc.codes.cpu().numpy().view(np.uint32)
+    scales = dc.scales.cpu().numpy().view(np.uint16)
+    biases = None if dc.biases is None else dc.biases.cpu().numpy().view(np.uint16)
+    return oracle.QCache(fmt, dc.bits, dc.group_size, codes, scales, biases)
+
+
+# ----------------------------------------------------------------------------
+# arms
+# ----------------------------------------------------------------------------
+def run_ours(args, rank, world, device):
+    import torch
+    from quantized_kv_attention_split_b200 import qkv, synthetic as S
+
+    qkv.lib()
+    w = S.WORKLOADS[args.workload]
+    hbm_peak, _, peak_kind = peaks()
+    inp = S.make_inputs(w)
+    cache_bytes = w.cache_bytes()
+    io_bytes = 2 * w.B * w.Hq * w.Lq * w.D * 2
+    alg_bytes = cache_bytes + io_bytes
+    ncopies = max(2, math.ceil(3 * 126e6 / cache_bytes))
+    caches = build_caches(w, inp, ncopies, device)
+    qd = dev16(inp.q, w.q_dtype, device)
+    out = torch.empty(w.B, w.Hq, w.Lq, w.D, dtype=torch.float16, device=device)
+    ws = qkv.make_workspace(w.B, w.Hq, w.Hkv, w.Lq, w.D, w.L, device)
+
+    # correctness gate on sampled rows before timing anything
+    qkv.qsdpa_decode(qd, caches[0][0], caches[0][1], w.L, w.scale, out=out, workspace=ws)
+    torch.cuda.synchronize()
+    hk, hv = host_cache(caches[0][0], w.fmt), host_cache(caches[0][1], w.fmt)
+    if rank == 0:
+        import oracle
+        rows = np.array([0, w.Hq // 2, w.Hq - 1])
+        ref = oracle.attention(inp.q, w.q_dtype, hk, hv, w.L, w.scale, rows=rows)
+        got = out.float().cpu().numpy().reshape(-1, w.D)
+        err = float(np.abs(got[rows] - ref.reshape(-1, w.D)[rows]).max())
+        if not err <= 2e-3:
+            print(json.dumps({"error": f"decode output differs from the oracle: {err}"}))
+            sys.exit(1)
+
+    def step(i):
+        kc, vc = caches[i % ncopies]
+        qkv.qsdpa_decode(qd, kc, vc, w.L, w.scale, out=out, workspace=ws)
+
+    sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    sec, extra = graph_time(step, args.steps, args.warmup, sampler)
+    sec /= 1e3
+    if sampler:
+        time.sleep(0.1)
+        sampler.stop()
+
+    # max over ranks
+    t = torch.tensor([sec], device=device, dtype=torch.float64)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    sec = float(t.item())
+    gbs = alg_bytes / sec / 1e9
+
+    # e2e through the public API with host buffers: H2D of q, decode, D2H of out
+    q_host = torch.from_numpy(inp.q.view(np.int16)).view(torch.float16).pin_memory()
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    qe = torch.empty_like(qd)
+    ke = max(20, min(args.steps, 2000))
+    for i in range(5):
+        qe.copy_(q_host, non_blocking=True)
+        step(i)
+        out_host.copy_(out, non_blocking=True)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    e0.record()
+    for i in range(ke):
+        qe.copy_(q_host, non_blocking=True)
+        kc, vc = caches[i % ncopies]
+        qkv.qsdpa_decode(qe, kc, vc, w.L, w.scale, out=out, workspace=ws)
+        out_host.copy_(out, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_sec = e0.elapsed_time(e1) / 1e3 / ke
+    te = torch.tensor([e2e_sec], device=device, dtype=torch.float64)
+    if world > 1:
+        torch.distributed.all_reduce(te, op=torch.distributed.ReduceOp.MAX)
+    e2e_sec = float(te.item())
+
+    result = None
+    if rank == 0:
+        clocks = sampler.summary() if sampler else {}
+        # CPU baseline: the oracle on the host cores, bounded sample of rows
+        dt, nrows, total_rows, threads, _, _ = oracle_rows_time(w, hk, hv, inp.q, 12.0)
+        cpu_gbs = (nrows / total_rows) * alg_bytes / dt / 1e9
+        result = {
+            "metric": METRIC,
+            "value": round(gbs * world, 2),
+            "unit": "GB/s",
+            "us_per_call": round(sec * 1e6, 3),
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": round(sec * 1e3, 6),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "f16",
+            "data": "synthetic (seeded SplitMix64, uniform fp16 q/k/v, K/V quantized on the GPU)",
+            "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
+                       "L": w.L, "Lq": w.Lq, "format": w.fmt, "bits": w.bits,
+                       "group_size": w.gs, "scale": w.scale, "out_dtype": "f16",
+                       "algorithmic_bytes_per_call": alg_bytes,
+                       "l2": f"inputs larger than L2: {ncopies} rotating cache copies "
+                             f"({ncopies * cache_bytes / 1e6:.0f} MB)",
+                       "timing": "CUDA events around CUDA-graph replays of exactly K calls",
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 2), "peak": hbm_peak,
+                         "unit": "GB/s", "frac": round(gbs / hbm_peak, 4),
+                         "peak_source": f"{peak_kind} hbm_gbs",
+                         "traffic": read_traffic(w.name)},
+            "cpu_baseline": {"value": round(cpu_gbs, 4), "unit": "GB/s", "cores": threads,
+                             "kind": "oracle",
+                             "sample": f"{nrows} of {total_rows} query rows over all {w.L} keys "
+                                       f"(fp64 dequantize + attention), scaled to the workload"},
+            "e2e": {"value": round(alg_bytes / e2e_sec / 1e9 * world, 2), "unit": "GB/s",
+                    "us_per_call": round(e2e_sec * 1e6, 3),
+                    "h2d_bytes_per_step": int(qd.numel() * 2),
+                    "d2h_bytes_per_step": int(out.numel() * 2),
+                    "note": "through the Python binding and C ABI, q copied from pinned host "
+                            "memory and the output copied back every call"},
+            "gpu_launches": args.steps,
+            "clocks": {"sm_mhz": clocks.get("sm_mhz"), "sm_max_mhz": clocks.get("sm_max_mhz"),
+                       "reasons": clocks.get("reasons", []), "samples": clocks.get("samples", 0),
+                       "window": "timed region" + (" + untimed replay of the same graph"
+                                                   if extra else "")},
+        }
+        if args.rows:
+            result["rows"] = other_rows(device)
+    del caches
+    return result
+
+
+def read_traffic(workload):
+    """DRAM bytes per launch from the committed ncu summary of this kernel, if
+    it was taken on the current kernel source (else null)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", f"decode_{workload}_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    src = os.path.join(ROOT, "quantized_kv_attention_split_b200", "csrc", "decode_kernel.cuh")
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    kv = {}
+    for line in open(path):
+        if ":" in line and not line.startswith("#"):
+            k, v = line.split(":", 1)
+            kv[k.strip()] = v.strip()
+    if kv.get("kernel_source_sha256_16") != h:
+        return None
+    try:
+        return float(kv["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def other_rows(device):
+    """Secondary rows of the hot path, each timed the same way (device time,
+    rotating copies where the data would fit in L2)."""
+    import torch
+    from quantized_kv_attention_split_b200 import qkv, synthetic as S
+    hbm_peak, _, _ = peaks()
+    rows = {}
+
+    # bulk quantize-and-append: 65536 tokens x 8 heads of K and V, 8-bit affine
+    w = S.WORKLOADS["decode_64k_affine8_update"]
+    inp = S.make_inputs(w, L=w.Lcap)
+    kd_src, vd_src = dev16(inp.k, "f16", device), dev16(inp.v, "f16", device)
+    kc = qkv.QuantCache.empty(w.B, w.Hkv, w.Lcap, w.D, qkv.AFFINE, 8, 64, device)
+    vc = qkv.QuantCache.empty(w.B, w.Hkv, w.Lcap, w.D, qkv.AFFINE, 8, 64, device)
+    sec, _ = graph_time(lambda i: qkv.qkv_quantize_update(kd_src, vd_src, kc, vc, 0), 50, 5)
+    nb = 2 * kd_src.numel() * 2 + w.cache_bytes(w.Lcap)
+    rows["quantize_bulk_65536tok_affine8"] = {
+        "us_per_call": round(sec * 1e3, 2), "GB/s": round(nb / (sec / 1e3) / 1e9, 1),
+        "frac_hbm": round(nb / (sec / 1e3) / 1e9 / hbm_peak, 4), "bytes": nb}
+    # single-token update at offset 65535, then the 8-bit decode over 65536 keys
+    nk, nv = dev16(inp.k[:, :, :1].copy(), "f16", device), dev16(inp.v[:, :, :1].copy(), "f16", device)
+    sec, _ = graph_time(lambda i: qkv.qkv_quantize_update(nk, nv, kc, vc, w.Lcap - 1), 200, 10)
+    rows["update_1tok_affine8"] = {"us_per_call": round(sec * 1e3, 3)}
+    del kd_src, vd_src
+    ncopies = max(2, math.ceil(3 * 126e6 / w.cache_bytes()))
+    copies = [(kc, vc)]
+    for _ in range(ncopies - 1):
+        k2 = qkv.QuantCache(kc.fmt, kc.bits, kc.group_size, kc.codes.clone(), kc.scales.clone(),
+                            kc.biases.clone())
+        v2 = qkv.QuantCache(vc.fmt, vc.bits, vc.group_size, vc.codes.clone(), vc.scales.clone(),
+                            vc.biases.clone())
+        copies.append((k2, v2))
+    q = dev16(S.make_inputs(w).q, "f16", device)
+    out = torch.empty(w.B, w.Hq, 1, w.D, dtype=torch.float16, device=device)
+    ws = qkv.make_workspace(w.B, w.Hq, w.Hkv, 1, w.D, w.L, device)
+
+    def dstep(i):
+        a, b = copies[i % ncopies]
+        qkv.qsdpa_decode(q, a, b, w.L, w.scale, out=out, workspace=ws)
+    sec, _ = graph_time(dstep, 400, 20)
+    nb = w.cache_bytes() + 2 * w.Hq * w.D * 2
+    rows["decode_64k_affine8"] = {"us_per_call": round(sec * 1e3, 3),
+                                  "GB/s": round(nb / (sec / 1e3) / 1e9, 1),
+                                  "frac_hbm": round(nb / (sec / 1e3) / 1e9 / hbm_peak, 4)}
+    del copies, kc, vc
+    torch.cuda.empty_cache()
+
+    for name in ("decode_q8_0_10k", "decode_q8_0_20k"):
+        w = S.WORKLOADS[name]
+        inp = S.make_inputs(w)
+        ncopies = max(2, math.ceil(3 * 126e6 / w.cache_bytes()))
+        caches = build_caches(w, inp, ncopies, device)
+        q = dev16(inp.q, "f16", device)
+        out = torch.empty(w.B, w.Hq, 1, w.D, dtype=torch.float16, device=device)
+        ws = qkv.make_workspace(w.B, w.Hq, w.Hkv, 1, w.D, w.L, device)
+
+        def qstep(i, caches=caches, q=q, out=out, ws=ws, w=w, n=ncopies):
+            a, b = caches[i % n]
+            qkv.qsdpa_decode(q, a, b, w.L, w.scale, out=out, workspace=ws)
+        sec, _ = graph_time(qstep, 400, 20)
+        nb = w.cache_bytes() + 2 * w.Hq * w.D * 2
+        rows[name] = {"us_per_call": round(sec * 1e3, 3), "GB/s": round(nb / (sec / 1e3) / 1e9, 1),
+                      "frac_hbm": round(nb / (sec / 1e3) / 1e9 / hbm_peak, 4)}
+        del caches
+        torch.cuda.empty_cache()
+    return rows
+
+
+def run_reference(args, rank, world):
+    """CPU oracle on a bounded sample of the workload, same metric."""
+    import oracle
+    from quantized_kv_attention_split_b200 import synthetic as S
+    if rank != 0:
+        return None
+    w = S.WORKLOADS[args.workload]
+    inp = S.make_inputs(w)
+    kc = oracle.quantize(inp.k, w.kv_dtype, w.fmt, w.gs, w.bits)
+    vc = oracle.quantize(inp.v, w.kv_dtype, w.fmt, w.gs, w.bits)
+    alg_bytes = w.cache_bytes() + 2 * w.B * w.Hq * w.Lq * w.D * 2
+    total_rows = w.B * w.Hq * w.Lq
+    threads = oracle.default_threads()
+    # size each step so the whole run stays within about two minutes
+    t0 = time.time()
+    oracle.attention(inp.q, w.q_dtype, kc, vc, w.L, w.scale, rows=np.array([0]), nthreads=1)
+    t_row = max(1e-4, time.time() - t0)
+    per_step = 120.0 / max(1, args.steps + args.warmup)
+    nrows = int(min(total_rows, max(1, per_step * threads / t_row)))
+    rows = np.linspace(0, total_rows - 1, nrows).astype(np.int64)
+    for _ in range(args.warmup):
+        oracle.attention(inp.q, w.q_dtype, kc, vc, w.L, w.scale, rows=rows, nthreads=threads)
+    t0 = time.time()
+    for _ in range(args.steps):
+        oracle.attention(inp.q, w.q_dtype, kc, vc, w.L, w.scale, rows=rows, nthreads=threads)
+    dt = (time.time() - t0) / max(1, args.steps)
+    gbs = (nrows / total_rows) * alg_bytes / dt / 1e9
+    sample = f"{nrows} of {total_rows} query rows over all {w.L} keys per step"
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "L": w.L,
+                   "format": w.fmt, "bits": w.bits, "group_size": w.gs},
+        "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": threads,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="decode_64k_affine4")
+    ap.add_argument("--rows", dest="rows", action="store_true", default=True)
+    ap.add_argument("--no-rows", dest="rows", action="store_false")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+
+    import datetime
+    import torch
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+    try:
+        res = run_ours(args, rank, world, device)
+        if rank == 0 and res is not None:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

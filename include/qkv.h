@@ -1,0 +1,148 @@
+/*
+ * qkv.h -- C ABI of libqkv.so: scaled-dot-product attention over a
+ * group-quantized KV cache, and the quantizer that appends tokens to it,
+ * for NVIDIA B200 (sm_100a).
+ *
+ * Sources the operations follow (web pages, by title and section):
+ *  - MLX compare "v0.19.3...quantized-kv-update" ("add
+ *    fast::quantized_kv_update"): mlx/fast.h declarations of
+ *    quantized_scaled_dot_product_attention(q, k, k_scales, k_biases, v,
+ *    v_scales, v_biases, scale, mask, group_size, bits) and kv_update(...);
+ *    mlx/fast.cpp (the fallback defines the math); sdpa_vector.h
+ *    quant_sdpa_vector (packing, dequant, GQA mapping); quantized.h kv_update
+ *    and affine_quantize_impl (eps 1e-7).
+ *  - llama.cpp PR #25556 "Metal: Optimize q8_0 KV": the Q8_0 KV format.
+ *
+ * Conventions shared by every entry point
+ *  - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *    never allocates device memory and never synchronizes: work is enqueued on
+ *    `stream` (a cudaStream_t; NULL = legacy default stream).
+ *  - Half-precision values are passed as their 16-bit patterns.
+ *  - Arguments are validated before anything is launched.  On any error the
+ *    call returns a status other than QKV_OK, launches nothing, and
+ *    qkv_last_error() (per host thread) describes the problem.  Errors
+ *    reported by the CUDA runtime at launch return QKV_ERR_CUDA.
+ *  - No exception crosses this interface and nothing is printed.
+ *
+ * Cache layout (qkv_cache): one struct describes one of K or V.
+ *  - codes  uint32 [B, Hkv, Lcap, D*bits/32], row-major.  Element e of a row
+ *           is stored at bits [(e % (32/bits))*bits, ...+bits) of word
+ *           e / (32/bits): low bits first (the pages' load_keys order).
+ *           Affine codes are unsigned; Q8_0 codes are two's-complement int8.
+ *  - scales fp16 [B, Hkv, Lcap, D/group_size]
+ *  - biases fp16 [B, Hkv, Lcap, D/group_size] (affine only; NULL for Q8_0)
+ *  - dequantized value = scale * code + bias (affine) or scale * code (Q8_0).
+ *  - Lcap is the row capacity per (batch, kv-head); a call uses rows [0, L).
+ *    Lcap must be a multiple of 8 and every pointer 16-byte aligned
+ *    (QKV_ERR_ALIGNMENT otherwise).
+ *  - Supported: affine bits 4 or 8 with group_size 32, 64 or 128; Q8_0
+ *    (bits 8, group_size 32); D in {64, 128, 256} with D % group_size == 0.
+ */
+#ifndef QKV_H_
+#define QKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  QKV_OK = 0,
+  QKV_ERR_INVALID_ARG = 1,   /* bad shape, NULL pointer, out-of-range value   */
+  QKV_ERR_UNSUPPORTED = 2,   /* valid request this build does not implement   */
+  QKV_ERR_ALIGNMENT = 3,     /* pointer or Lcap alignment requirement not met */
+  QKV_ERR_WORKSPACE = 4,     /* workspace missing or smaller than required    */
+  QKV_ERR_CUDA = 5           /* the CUDA runtime reported an error            */
+} qkv_status;
+
+typedef enum { QKV_F16 = 0, QKV_BF16 = 1, QKV_F32 = 2 } qkv_dtype;
+typedef enum { QKV_AFFINE = 0, QKV_Q8_0 = 1 } qkv_format;
+typedef enum { QKV_MASK_NONE = 0, QKV_MASK_CAUSAL = 1, QKV_MASK_ADDITIVE = 2 } qkv_mask_kind;
+
+typedef struct {
+  int fmt;              /* qkv_format                                         */
+  int bits;             /* affine: 4 or 8; Q8_0: 8                            */
+  int group_size;       /* affine: 32, 64 or 128; Q8_0: 32                    */
+  uint32_t* codes;      /* [B, Hkv, Lcap, D*bits/32]                          */
+  uint16_t* scales;     /* fp16 [B, Hkv, Lcap, D/group_size]                  */
+  uint16_t* biases;     /* fp16, same shape; NULL for Q8_0                    */
+  int64_t Lcap;         /* rows per (batch, kv-head); multiple of 8           */
+} qkv_cache;
+
+/* Optional mask (pass NULL for none).
+ *  - QKV_MASK_CAUSAL: query i of Lq sees key j iff j <= L - Lq + i (aligned to
+ *    the bottom-right, i.e. the queries are the last Lq positions).
+ *  - QKV_MASK_ADDITIVE: logit(b,h,i,j) += add[b*stride_b + h*stride_h +
+ *    i*stride_q + j] (element strides; 0 broadcasts), dtype add_dtype; -inf
+ *    hides a key.  The mask is added after `scale` (the pages' fallback adds
+ *    it to q*scale . K^T).
+ * A query row that sees no key returns zeros. */
+typedef struct {
+  int kind;             /* qkv_mask_kind */
+  const void* add;
+  int add_dtype;        /* qkv_dtype */
+  int64_t stride_b, stride_h, stride_q;
+} qkv_mask;
+
+/* Quantize Lnew new tokens per (batch, kv-head) and write them into rows
+ * [offset, offset+Lnew) of the K and V caches, in place (MLX kv_update /
+ * KVUpdate::eval_gpu; the pages copy the whole cache first, this library
+ * updates the caller's buffers in place).
+ *  new_k, new_v: [B, Hkv, Lnew, D] contiguous, dtype in_dtype (f16 or bf16).
+ *  Per group of group_size elements along D (fp32 IEEE, this order):
+ *   affine: mn, mx = min, max; s = (mx-mn)/(2^bits-1); s = max(s, 1e-7);
+ *           scale = fp16_rne(s); bias = fp16_rne(mn);
+ *           code = clamp(rint((x - bias)/scale), 0, 2^bits-1)
+ *   Q8_0:   d = max|x|/127; scale = fp16_rne(d);
+ *           code = scale == 0 ? 0 : clamp(rint(x/scale), -127, 127)
+ *  The result is bit-identical to the CPU oracle.  Requires
+ *  0 <= offset <= Lcap - Lnew.  k and v may use different formats. */
+qkv_status qkv_quantize_update(const void* new_k, const void* new_v, int in_dtype,
+                               int B, int Hkv, int Lnew, int D,
+                               const qkv_cache* k, const qkv_cache* v,
+                               int64_t offset, void* stream);
+
+/* Single-query attention (Lq = 1): out = softmax(q*scale . K^T + mask) V over
+ * keys [0, L) of the dequantized cache (MLX quant_sdpa_vector semantics, plus
+ * GQA, masks and a split over L).
+ *  q:   [B, Hq, 1, D] contiguous, q_dtype f16 or bf16.
+ *  out: [B, Hq, 1, D] contiguous, out_dtype f16, bf16 or f32.
+ *  Hq % Hkv == 0; query head h reads kv-head h / (Hq/Hkv).
+ *  workspace: device scratch of at least qsdpa_workspace_size(...) bytes,
+ *  16-byte aligned, whose first qsdpa_workspace_zero_bytes(...) bytes are
+ *  zero before the first call (the kernel leaves them zero again after every
+ *  call).  Calls that share a workspace must not overlap on the GPU.
+ *  L == 0 writes zeros.  Accuracy: max-abs error vs fp64 <= 2e-3 for f16/bf16
+ *  out, <= 1e-4 for f32 out (values of order one). */
+qkv_status qsdpa_decode(const void* q, int q_dtype, int B, int Hq, int Hkv, int D,
+                        const qkv_cache* k, const qkv_cache* v, int64_t L,
+                        float scale, const qkv_mask* mask, void* out, int out_dtype,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/* Multi-query attention (any Lq >= 1) over keys [0, L) with an optional mask
+ * (the pages' Lq > 1 fallback: quantized_matmul -> softmax -> quantized_matmul,
+ * computed here in one fused pass).  q/out: [B, Hq, Lq, D] contiguous.
+ * Same workspace rules as qsdpa_decode. */
+qkv_status qsdpa_prefill(const void* q, int q_dtype, int B, int Hq, int Hkv, int Lq,
+                         int D, const qkv_cache* k, const qkv_cache* v, int64_t L,
+                         float scale, const qkv_mask* mask, void* out, int out_dtype,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/* Workspace bytes needed by qsdpa_decode (Lq = 1) or qsdpa_prefill for this
+ * problem on the CURRENT device, and how many leading bytes must be zero
+ * before the first call.  0 on invalid arguments. */
+size_t qsdpa_workspace_size(int B, int Hq, int Hkv, int Lq, int D, int64_t L);
+size_t qsdpa_workspace_zero_bytes(int B, int Hq, int Hkv, int Lq, int D, int64_t L);
+
+/* Human-readable text of a status code, and the detail of this host thread's
+ * most recent error (empty string if none). */
+const char* qkv_status_string(int status);
+const char* qkv_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QKV_H_ */

@@ -1,0 +1,224 @@
+// api.cu -- extern "C" entry points of libqkv.so: argument validation, work
+// planning and kernel launch.  Declarations and contracts: include/qkv.h.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "qkv_internal.h"
+
+namespace qkv {
+cudaError_t launch_quantize(const void* new_k, const void* new_v, int in_dtype, int B, int Hkv,
+                            int Lnew, int D, const qkv_cache* k, const qkv_cache* v,
+                            int64_t offset, cudaStream_t stream);
+size_t decode_workspace_bound(int B, int Hq, int Hkv, int D);
+size_t decode_workspace_zero_bytes(int B, int Hq, int Hkv);
+void decode_chunking(int G, int* nc, int* ncg);
+}  // namespace qkv
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+qkv_status fail(qkv_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+qkv_status ok() {
+  g_last_error[0] = '\0';
+  return QKV_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Validates one cache description for head dimension D.
+qkv_status check_cache(const char* name, const qkv_cache* c, int D) {
+  if (c == nullptr) return fail(QKV_ERR_INVALID_ARG, "%s: cache descriptor is NULL", name);
+  if (c->fmt != QKV_AFFINE && c->fmt != QKV_Q8_0)
+    return fail(QKV_ERR_INVALID_ARG, "%s: unknown format %d", name, c->fmt);
+  if (c->fmt == QKV_AFFINE) {
+    if (c->bits != 4 && c->bits != 8)
+      return fail(QKV_ERR_UNSUPPORTED, "%s: affine bits must be 4 or 8 (got %d)", name, c->bits);
+    if (c->group_size != 32 && c->group_size != 64 && c->group_size != 128)
+      return fail(QKV_ERR_UNSUPPORTED, "%s: group_size must be 32, 64 or 128 (got %d)", name,
+                  c->group_size);
+    if (c->biases == nullptr) return fail(QKV_ERR_INVALID_ARG, "%s: affine cache needs biases", name);
+  } else {
+    if (c->bits != 8 || c->group_size != 32)
+      return fail(QKV_ERR_INVALID_ARG, "%s: Q8_0 needs bits 8 and group_size 32", name);
+  }
+  if (D != 64 && D != 128 && D != 256)
+    return fail(QKV_ERR_UNSUPPORTED, "head dimension must be 64, 128 or 256 (got %d)", D);
+  if (D % c->group_size != 0)
+    return fail(QKV_ERR_UNSUPPORTED, "%s: D=%d is not a multiple of group_size=%d", name, D,
+                c->group_size);
+  if (c->codes == nullptr || c->scales == nullptr)
+    return fail(QKV_ERR_INVALID_ARG, "%s: codes and scales must be non-NULL", name);
+  if (c->Lcap <= 0) return fail(QKV_ERR_INVALID_ARG, "%s: Lcap must be positive", name);
+  if (c->Lcap % 8 != 0)
+    return fail(QKV_ERR_ALIGNMENT, "%s: Lcap must be a multiple of 8 (got %lld)", name,
+                (long long)c->Lcap);
+  if (!aligned16(c->codes) || !aligned16(c->scales) ||
+      (c->fmt == QKV_AFFINE && !aligned16(c->biases)))
+    return fail(QKV_ERR_ALIGNMENT, "%s: codes, scales and biases must be 16-byte aligned", name);
+  return QKV_OK;
+}
+
+qkv_status check_dtype(const char* name, int dt, bool allow_f32) {
+  if (dt == QKV_F16 || dt == QKV_BF16 || (allow_f32 && dt == QKV_F32)) return QKV_OK;
+  return fail(QKV_ERR_INVALID_ARG, "%s: unsupported dtype %d", name, dt);
+}
+
+qkv_status attention(const void* q, int q_dtype, int B, int Hq, int Hkv, int Lq, int D,
+                     const qkv_cache* k, const qkv_cache* v, int64_t L, float scale,
+                     const qkv_mask* mask, void* out, int out_dtype, void* workspace,
+                     size_t workspace_bytes, void* stream) {
+  qkv_status st;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Lq <= 0)
+    return fail(QKV_ERR_INVALID_ARG, "B, Hq, Hkv and Lq must be positive");
+  if (Hq % Hkv != 0) return fail(QKV_ERR_INVALID_ARG, "Hq=%d is not a multiple of Hkv=%d", Hq, Hkv);
+  if ((st = check_cache("k", k, D)) != QKV_OK) return st;
+  if ((st = check_cache("v", v, D)) != QKV_OK) return st;
+  if (k->fmt != v->fmt || k->bits != v->bits || k->group_size != v->group_size)
+    return fail(QKV_ERR_UNSUPPORTED, "k and v must use the same format, bits and group_size");
+  if (k->Lcap != v->Lcap) return fail(QKV_ERR_INVALID_ARG, "k and v must have the same Lcap");
+  if (L < 0 || L > k->Lcap) return fail(QKV_ERR_INVALID_ARG, "L=%lld outside [0, Lcap]", (long long)L);
+  if ((st = check_dtype("q", q_dtype, false)) != QKV_OK) return st;
+  if ((st = check_dtype("out", out_dtype, true)) != QKV_OK) return st;
+  if (q == nullptr || out == nullptr) return fail(QKV_ERR_INVALID_ARG, "q and out must be non-NULL");
+  if (!aligned16(q) || !aligned16(out))
+    return fail(QKV_ERR_ALIGNMENT, "q and out must be 16-byte aligned");
+  if (!(scale == scale)) return fail(QKV_ERR_INVALID_ARG, "scale is NaN");
+  int mkind = QKV_MASK_NONE;
+  if (mask != nullptr) {
+    mkind = mask->kind;
+    if (mkind != QKV_MASK_NONE && mkind != QKV_MASK_CAUSAL && mkind != QKV_MASK_ADDITIVE)
+      return fail(QKV_ERR_INVALID_ARG, "unknown mask kind %d", mkind);
+    if (mkind == QKV_MASK_ADDITIVE) {
+      if (mask->add == nullptr) return fail(QKV_ERR_INVALID_ARG, "additive mask pointer is NULL");
+      if ((st = check_dtype("mask", mask->add_dtype, true)) != QKV_OK) return st;
+      if (mask->stride_b < 0 || mask->stride_h < 0 || mask->stride_q < 0)
+        return fail(QKV_ERR_INVALID_ARG, "mask strides must be non-negative");
+    }
+  }
+  if ((int64_t)Hq * Lq > (int64_t)1 << 30)
+    return fail(QKV_ERR_INVALID_ARG, "Hq * Lq too large");
+
+  const size_t elems = (size_t)B * Hq * Lq * D;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (L == 0) {
+    const size_t esz = out_dtype == QKV_F32 ? 4 : 2;
+    if (cudaMemsetAsync(out, 0, elems * esz, s) != cudaSuccess)
+      return fail(QKV_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(cudaGetLastError()));
+    return ok();
+  }
+
+  const int G = Hq / Hkv;
+  const int rows = G * Lq;                 // rows of one kv head: (head, query) pairs
+  qkv::DecodePlan plan;
+  if (!qkv::plan_decode(D, k->bits, k->group_size, k->fmt, out_dtype == QKV_F32, B,
+                        Hkv * rows, Hkv, L, &plan))
+    return fail(QKV_ERR_UNSUPPORTED, "no kernel for D=%d bits=%d group_size=%d", D, k->bits,
+                k->group_size);
+  if (plan.ws_total > 0) {
+    if (workspace == nullptr || workspace_bytes < plan.ws_total)
+      return fail(QKV_ERR_WORKSPACE, "workspace of %zu bytes required (got %zu)", plan.ws_total,
+                  workspace_bytes);
+    if (!aligned16(workspace)) return fail(QKV_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
+  }
+  qkv::DecodeParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.q = q; p.q_dtype = q_dtype; p.out = out; p.out_dtype = out_dtype;
+  p.kc = reinterpret_cast<const uint8_t*>(k->codes); p.ks = k->scales; p.kb = k->biases;
+  p.vc = reinterpret_cast<const uint8_t*>(v->codes); p.vs = v->scales; p.vb = v->biases;
+  p.Lcap = k->Lcap; p.L = L;
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.G = rows; p.Gq = G; p.Lq = Lq;
+  p.scale_log2e = scale * 1.4426950408889634f;
+  p.mask_kind = mkind;
+  if (mkind == QKV_MASK_ADDITIVE) {
+    p.mask = mask->add; p.mask_dtype = mask->add_dtype;
+    p.msb = mask->stride_b; p.msh = mask->stride_h; p.msq = mask->stride_q;
+  }
+  if (mkind == QKV_MASK_CAUSAL && Lq == 1) p.mask_kind = QKV_MASK_NONE;  // all keys visible
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  p.tickets = reinterpret_cast<unsigned*>(ws);
+  p.part_o = reinterpret_cast<float*>(ws + plan.ws_tickets);
+  p.part_ml = reinterpret_cast<float*>(ws + plan.ws_tickets + plan.ws_part_o);
+  cudaError_t e = qkv::launch_decode(D, k->bits, k->group_size, k->fmt, out_dtype == QKV_F32,
+                                     plan, p, s);
+  if (e != cudaSuccess) return fail(QKV_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
+  return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* qkv_status_string(int status) {
+  switch (status) {
+    case QKV_OK: return "ok";
+    case QKV_ERR_INVALID_ARG: return "invalid argument";
+    case QKV_ERR_UNSUPPORTED: return "unsupported";
+    case QKV_ERR_ALIGNMENT: return "alignment";
+    case QKV_ERR_WORKSPACE: return "workspace too small";
+    case QKV_ERR_CUDA: return "CUDA error";
+    default: return "unknown status";
+  }
+}
+
+const char* qkv_last_error(void) { return g_last_error; }
+
+size_t qsdpa_workspace_size(int B, int Hq, int Hkv, int Lq, int D, int64_t L) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Lq <= 0 || Hq % Hkv || L < 0) return 0;
+  if (D != 64 && D != 128 && D != 256) return 0;
+  return qkv::decode_workspace_bound(B, Hq * Lq, Hkv, D);
+}
+
+size_t qsdpa_workspace_zero_bytes(int B, int Hq, int Hkv, int Lq, int D, int64_t L) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Lq <= 0 || Hq % Hkv || L < 0) return 0;
+  (void)D;
+  return qkv::decode_workspace_zero_bytes(B, Hq * Lq, Hkv);
+}
+
+qkv_status qkv_quantize_update(const void* new_k, const void* new_v, int in_dtype, int B, int Hkv,
+                               int Lnew, int D, const qkv_cache* k, const qkv_cache* v,
+                               int64_t offset, void* stream) {
+  qkv_status st;
+  if (B <= 0 || Hkv <= 0 || Lnew < 0) return fail(QKV_ERR_INVALID_ARG, "B, Hkv must be positive, Lnew >= 0");
+  if ((st = check_cache("k", k, D)) != QKV_OK) return st;
+  if ((st = check_cache("v", v, D)) != QKV_OK) return st;
+  if (in_dtype != QKV_F16 && in_dtype != QKV_BF16)
+    return fail(QKV_ERR_INVALID_ARG, "new tokens must be f16 or bf16 (got %d)", in_dtype);
+  if (Lnew == 0) return ok();
+  if (new_k == nullptr || new_v == nullptr)
+    return fail(QKV_ERR_INVALID_ARG, "new_k and new_v must be non-NULL");
+  if (!aligned16(new_k) || !aligned16(new_v))
+    return fail(QKV_ERR_ALIGNMENT, "new_k and new_v must be 16-byte aligned");
+  if (offset < 0 || offset + Lnew > k->Lcap || offset + Lnew > v->Lcap)
+    return fail(QKV_ERR_INVALID_ARG, "offset=%lld with Lnew=%d exceeds Lcap", (long long)offset, Lnew);
+  cudaError_t e = qkv::launch_quantize(new_k, new_v, in_dtype, B, Hkv, Lnew, D, k, v, offset,
+                                       static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(QKV_ERR_CUDA, "quantize launch: %s", cudaGetErrorString(e));
+  return ok();
+}
+
+qkv_status qsdpa_decode(const void* q, int q_dtype, int B, int Hq, int Hkv, int D,
+                        const qkv_cache* k, const qkv_cache* v, int64_t L, float scale,
+                        const qkv_mask* mask, void* out, int out_dtype, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  return attention(q, q_dtype, B, Hq, Hkv, 1, D, k, v, L, scale, mask, out, out_dtype, workspace,
+                   workspace_bytes, stream);
+}
+
+qkv_status qsdpa_prefill(const void* q, int q_dtype, int B, int Hq, int Hkv, int Lq, int D,
+                         const qkv_cache* k, const qkv_cache* v, int64_t L, float scale,
+                         const qkv_mask* mask, void* out, int out_dtype, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  return attention(q, q_dtype, B, Hq, Hkv, Lq, D, k, v, L, scale, mask, out, out_dtype, workspace,
+                   workspace_bytes, stream);
+}
+
+}  // extern "C"

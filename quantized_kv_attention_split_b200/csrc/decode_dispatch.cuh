@@ -1,0 +1,58 @@
+// decode_dispatch.cuh -- compile-time instance table for the decode kernel.
+// Each decode_*.cu translation unit instantiates the kernels of one head
+// dimension; decode_plan.cu picks one at run time.
+#pragma once
+
+#include "decode_kernel.cuh"
+
+namespace qkv {
+
+struct DecodeOps {
+  int (*occupancy)();
+  cudaError_t (*launch)(const DecodePlan&, const DecodeParams&, cudaStream_t);
+  int tk;
+  int nc;
+  size_t smem;
+};
+
+template <int D, int BITS, int GS, bool Q8, int NC, bool F32>
+DecodeOps make_decode_ops() {
+  using I = DecodeInstance<D, BITS, GS, Q8, NC, F32>;
+  return DecodeOps{&I::max_ctas_per_sm, &I::launch, I::C::TK, NC, (size_t)I::C::SMEM};
+}
+
+// Instances of one head dimension; nc in {1, 2, 4}; f32 selects the
+// split-precision value operand used for fp32 output.
+template <int D>
+bool decode_ops_for(int bits, int gs, bool q8, int nc, bool f32, DecodeOps* ops) {
+#define QKV_DEC_NC(BITS, GS, Q8)                                                   \
+  do {                                                                             \
+    if (nc == 1) { *ops = f32 ? make_decode_ops<D, BITS, GS, Q8, 1, true>()        \
+                              : make_decode_ops<D, BITS, GS, Q8, 1, false>(); }    \
+    else if (nc == 2) { *ops = f32 ? make_decode_ops<D, BITS, GS, Q8, 2, true>()   \
+                                   : make_decode_ops<D, BITS, GS, Q8, 2, false>(); } \
+    else { *ops = f32 ? make_decode_ops<D, BITS, GS, Q8, 4, true>()                \
+                      : make_decode_ops<D, BITS, GS, Q8, 4, false>(); }            \
+    return true;                                                                   \
+  } while (0)
+  if (q8) {
+    QKV_DEC_NC(8, 32, true);
+  }
+  if (bits == 4) {
+    if (gs == 32) QKV_DEC_NC(4, 32, false);
+    if (gs == 64) QKV_DEC_NC(4, 64, false);
+    if constexpr (D >= 128) { if (gs == 128) QKV_DEC_NC(4, 128, false); }
+  } else if (bits == 8) {
+    if (gs == 32) QKV_DEC_NC(8, 32, false);
+    if (gs == 64) QKV_DEC_NC(8, 64, false);
+    if constexpr (D >= 128) { if (gs == 128) QKV_DEC_NC(8, 128, false); }
+  }
+#undef QKV_DEC_NC
+  return false;
+}
+
+bool decode_ops_d64(int bits, int gs, bool q8, int nc, bool f32, DecodeOps* ops);
+bool decode_ops_d128(int bits, int gs, bool q8, int nc, bool f32, DecodeOps* ops);
+bool decode_ops_d256(int bits, int gs, bool q8, int nc, bool f32, DecodeOps* ops);
+
+}  // namespace qkv

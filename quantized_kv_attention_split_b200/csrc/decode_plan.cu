@@ -1,0 +1,102 @@
+// decode_plan.cu -- chooses the decode kernel instance and its work split.
+#include <algorithm>
+
+#include "decode_dispatch.cuh"
+
+namespace qkv {
+
+namespace {
+
+// Grid cap per SM used both for planning and for the workspace bound, so that
+// qsdpa_workspace_size() does not depend on the kernel instance.
+constexpr int kMaxCtasPerSm = 2;
+// Upper bound on the bytes of partial results one CTA merges at the end of a
+// unit (the merge is done by a single CTA).
+constexpr double kMergeBytesPerUnit = 160.0 * 1024.0;
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+bool get_ops(int D, int bits, int gs, int fmt, int nc, bool f32, DecodeOps* ops) {
+  const bool q8 = fmt == QKV_Q8_0;
+  if (D == 64) return decode_ops_d64(bits, gs, q8, nc, f32, ops);
+  if (D == 128) return decode_ops_d128(bits, gs, q8, nc, f32, ops);
+  if (D == 256) return decode_ops_d256(bits, gs, q8, nc, f32, ops);
+  return false;
+}
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace
+
+void decode_chunking(int G, int* nc, int* ncg) {
+  const int chunks = (G + 7) / 8;
+  *nc = chunks <= 1 ? 1 : (chunks <= 2 ? 2 : 4);
+  *ncg = (chunks + *nc - 1) / *nc;
+}
+
+size_t decode_workspace_bound(int B, int Hq, int Hkv, int D) {
+  if (B <= 0 || Hkv <= 0 || Hq % Hkv) return 0;
+  int nc, ncg;
+  decode_chunking(Hq / Hkv, &nc, &ncg);
+  const size_t units = (size_t)B * Hkv * ncg;
+  const size_t grid = (size_t)std::max(1, sm_count()) * kMaxCtasPerSm;
+  const size_t hpc = (size_t)nc * 8;
+  return round_up(units * 4, 256) + round_up(2 * grid * hpc * D * 4, 256) +
+         round_up(2 * grid * hpc * 2 * 4, 256);
+}
+
+size_t decode_workspace_zero_bytes(int B, int Hq, int Hkv) {
+  if (B <= 0 || Hkv <= 0 || Hq % Hkv) return 0;
+  int nc, ncg;
+  decode_chunking(Hq / Hkv, &nc, &ncg);
+  return round_up((size_t)B * Hkv * ncg * 4, 256);
+}
+
+bool plan_decode(int D, int bits, int gs, int fmt, int out_f32, int B, int Hq, int Hkv,
+                 int64_t L, DecodePlan* plan) {
+  int nc, ncg;
+  decode_chunking(Hq / Hkv, &nc, &ncg);
+  DecodeOps ops;
+  if (!get_ops(D, bits, gs, fmt, nc, out_f32 != 0, &ops)) return false;
+  const int sms = std::max(1, sm_count());
+  const int occ = std::min(kMaxCtasPerSm, std::max(1, ops.occupancy()));
+  plan->tk = ops.tk;
+  plan->nc = nc;
+  plan->hpc = nc * 8;
+  plan->ncg = ncg;
+  plan->units = (int64_t)B * Hkv * ncg;
+  plan->stages_per_unit = (L + ops.tk - 1) / ops.tk;
+  plan->total_stages = plan->units * plan->stages_per_unit;
+  // One CTA per (SM x resident slot), but no more CTAs per unit than keeps the
+  // final merge of a unit's partial results small.
+  const double part_bytes = (double)plan->hpc * D * 4.0;
+  const int64_t max_parts = std::max<int64_t>(1, (int64_t)(kMergeBytesPerUnit / part_bytes));
+  int64_t grid = (int64_t)sms * occ;
+  grid = std::min<int64_t>(grid, plan->units * max_parts);
+  grid = std::min<int64_t>(grid, plan->total_stages);
+  plan->grid = (int)std::max<int64_t>(1, grid);
+  plan->smem = ops.smem;
+  plan->ws_tickets = round_up((size_t)plan->units * 4, 256);
+  const size_t maxgrid = (size_t)sms * kMaxCtasPerSm;
+  plan->ws_part_o = round_up(2 * maxgrid * plan->hpc * D * 4, 256);
+  plan->ws_part_ml = round_up(2 * maxgrid * plan->hpc * 2 * 4, 256);
+  plan->ws_total = plan->ws_tickets + plan->ws_part_o + plan->ws_part_ml;
+  return true;
+}
+
+cudaError_t launch_decode(int D, int bits, int gs, int fmt, int out_f32, const DecodePlan& plan,
+                          DecodeParams& p, cudaStream_t stream) {
+  DecodeOps ops;
+  if (!get_ops(D, bits, gs, fmt, plan.nc, out_f32 != 0, &ops)) return cudaErrorInvalidValue;
+  p.ncg = plan.ncg;
+  p.stages_per_unit = plan.stages_per_unit;
+  p.total_stages = plan.total_stages;
+  return ops.launch(plan, p, stream);
+}
+
+}  // namespace qkv

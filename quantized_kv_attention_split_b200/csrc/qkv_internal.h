@@ -1,0 +1,70 @@
+// qkv_internal.h -- parameter blocks and launcher declarations shared between
+// the C-ABI front end (api.cu) and the kernel translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/qkv.h"
+
+namespace qkv {
+
+// Everything one decode launch needs (device pointers and sizes).
+struct DecodeParams {
+  const void* q;            // [B, Hq, 1, D]
+  int q_dtype;
+  void* out;                // [B, Hq, 1, D]
+  int out_dtype;
+  const uint8_t* kc;        // K codes, bytes
+  const uint16_t* ks;       // K scales
+  const uint16_t* kb;       // K biases (affine)
+  const uint8_t* vc;
+  const uint16_t* vs;
+  const uint16_t* vb;
+  int64_t Lcap;
+  int64_t L;
+  int B, Hq, Hkv;
+  int G;                    // rows per kv head: (query heads per kv head) * Lq
+  int Gq;                   // query heads per kv head
+  int Lq;                   // queries per head (row r = head * Lq + query)
+  int ncg;                  // row chunk-groups (of up to 32 rows) per kv head
+  float scale_log2e;        // softmax scale times log2(e)
+  // mask: kind 0 none, 1 causal (bottom-right aligned), 2 additive
+  int mask_kind;
+  const void* mask;
+  int mask_dtype;
+  int64_t msb, msh, msq;
+  // work split: units (b, kv-head, chunk-group) x stages of TK keys, divided
+  // evenly over gridDim.x CTAs
+  int64_t stages_per_unit;
+  int64_t total_stages;
+  float* part_o;            // [2 * nCTA][HPC][D]
+  float* part_ml;           // [2 * nCTA][HPC][2]
+  unsigned* tickets;        // [units], zero between calls
+};
+
+struct DecodePlan {
+  int tk;                   // keys per stage
+  int nc;                   // head chunks (of 8) per CTA
+  int hpc;                  // heads per chunk-group slot (nc * 8)
+  int ncg;
+  int64_t units;
+  int64_t stages_per_unit;
+  int64_t total_stages;
+  int grid;
+  size_t smem;
+  size_t ws_tickets;        // bytes (zeroed region)
+  size_t ws_part_o;         // bytes
+  size_t ws_part_ml;        // bytes
+  size_t ws_total;
+};
+
+// Plans a decode launch for the current device; returns false if the shape
+// has no kernel instance.
+bool plan_decode(int D, int bits, int gs, int fmt, int out_f32, int B, int Hq, int Hkv,
+                 int64_t L, DecodePlan* plan);
+cudaError_t launch_decode(int D, int bits, int gs, int fmt, int out_f32,
+                          const DecodePlan& plan, DecodeParams& p, cudaStream_t stream);
+
+}  // namespace qkv

@@ -1,0 +1,202 @@
+"""Python binding of ``libqkv.so`` (argument marshalling only).
+
+The functions keep the names of the C entry points declared in
+``include/qkv.h`` -- :func:`qkv_quantize_update`, :func:`qsdpa_decode`,
+:func:`qsdpa_prefill` -- and take torch CUDA tensors, passing their device
+pointers, sizes and the current CUDA stream to the library.  Every step of the
+computation runs in the library's kernels; there is no fallback: if the
+library is missing or a call fails, a Python exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqkv.so")
+
+F16, BF16, F32 = 0, 1, 2
+AFFINE, Q8_0 = 0, 1
+MASK_NONE, MASK_CAUSAL, MASK_ADDITIVE = 0, 1, 2
+
+_DTYPE = {torch.float16: F16, torch.bfloat16: BF16, torch.float32: F32}
+_STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported", 3: "alignment",
+           4: "workspace too small", 5: "CUDA error"}
+
+
+class _Cache(C.Structure):
+    _fields_ = [("fmt", C.c_int), ("bits", C.c_int), ("group_size", C.c_int),
+                ("codes", C.c_void_p), ("scales", C.c_void_p), ("biases", C.c_void_p),
+                ("Lcap", C.c_int64)]
+
+
+class _Mask(C.Structure):
+    _fields_ = [("kind", C.c_int), ("add", C.c_void_p), ("add_dtype", C.c_int),
+                ("stride_b", C.c_int64), ("stride_h", C.c_int64), ("stride_q", C.c_int64)]
+
+
+class QKVError(RuntimeError):
+    def __init__(self, status: int, detail: str):
+        super().__init__(f"{_STATUS.get(status, status)}: {detail}")
+        self.status = status
+
+
+_lib = None
+
+
+def lib() -> C.CDLL:
+    """Load libqkv.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libqkv.so not found at {LIB_PATH}; build it with "
+                              "`python quantized_kv_attention_split_b200/build.py`")
+        L = C.CDLL(LIB_PATH)
+        p, i32, i64, sz = C.c_void_p, C.c_int, C.c_int64, C.c_size_t
+        cp = C.POINTER(_Cache)
+        mp = C.POINTER(_Mask)
+        L.qkv_quantize_update.argtypes = [p, p, i32, i32, i32, i32, i32, cp, cp, i64, p]
+        L.qkv_quantize_update.restype = i32
+        L.qsdpa_decode.argtypes = [p, i32, i32, i32, i32, i32, cp, cp, i64, C.c_float, mp,
+                                   p, i32, p, sz, p]
+        L.qsdpa_decode.restype = i32
+        L.qsdpa_prefill.argtypes = [p, i32, i32, i32, i32, i32, i32, cp, cp, i64, C.c_float, mp,
+                                    p, i32, p, sz, p]
+        L.qsdpa_prefill.restype = i32
+        L.qsdpa_workspace_size.argtypes = [i32, i32, i32, i32, i32, i64]
+        L.qsdpa_workspace_size.restype = sz
+        L.qsdpa_workspace_zero_bytes.argtypes = [i32, i32, i32, i32, i32, i64]
+        L.qsdpa_workspace_zero_bytes.restype = sz
+        L.qkv_status_string.argtypes = [i32]
+        L.qkv_status_string.restype = C.c_char_p
+        L.qkv_last_error.argtypes = []
+        L.qkv_last_error.restype = C.c_char_p
+        _lib = L
+    return _lib
+
+
+def _check(status: int):
+    if status != 0:
+        raise QKVError(status, lib().qkv_last_error().decode())
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+@dataclass
+class QuantCache:
+    """One of K or V in the library's layout (all tensors on one CUDA device):
+    codes int32 [B,Hkv,Lcap,D*bits/32] (bit patterns of uint32 words), scales
+    and biases float16 [B,Hkv,Lcap,D/group_size] (biases None for Q8_0)."""
+    fmt: int
+    bits: int
+    group_size: int
+    codes: torch.Tensor
+    scales: torch.Tensor
+    biases: Optional[torch.Tensor]
+
+    @property
+    def Lcap(self) -> int:
+        return self.codes.shape[2]
+
+    @staticmethod
+    def empty(B: int, Hkv: int, Lcap: int, D: int, fmt: int = AFFINE, bits: int = 4,
+              group_size: int = 64, device="cuda") -> "QuantCache":
+        if fmt == Q8_0:
+            bits, group_size = 8, 32
+        codes = torch.zeros(B, Hkv, Lcap, D * bits // 32, dtype=torch.int32, device=device)
+        scales = torch.zeros(B, Hkv, Lcap, D // group_size, dtype=torch.float16, device=device)
+        biases = torch.zeros_like(scales) if fmt == AFFINE else None
+        return QuantCache(fmt, bits, group_size, codes, scales, biases)
+
+    def _struct(self) -> _Cache:
+        return _Cache(self.fmt, self.bits, self.group_size, self.codes.data_ptr(),
+                      self.scales.data_ptr(),
+                      self.biases.data_ptr() if self.biases is not None else None,
+                      self.codes.shape[2])
+
+
+def qsdpa_workspace_size(B: int, Hq: int, Hkv: int, Lq: int, D: int, L: int) -> int:
+    return int(lib().qsdpa_workspace_size(B, Hq, Hkv, Lq, D, L))
+
+
+def qsdpa_workspace_zero_bytes(B: int, Hq: int, Hkv: int, Lq: int, D: int, L: int) -> int:
+    return int(lib().qsdpa_workspace_zero_bytes(B, Hq, Hkv, Lq, D, L))
+
+
+def make_workspace(B: int, Hq: int, Hkv: int, Lq: int, D: int, L: int,
+                   device="cuda") -> torch.Tensor:
+    """A zero-initialised workspace of the size the library asks for."""
+    n = qsdpa_workspace_size(B, Hq, Hkv, Lq, D, L)
+    return torch.zeros(max(n, 16), dtype=torch.uint8, device=device)
+
+
+def qkv_quantize_update(new_k: torch.Tensor, new_v: torch.Tensor, k: QuantCache, v: QuantCache,
+                        offset: int, stream=None) -> None:
+    """Quantize new_k/new_v [B,Hkv,Lnew,D] (f16/bf16) into rows
+    [offset, offset+Lnew) of the caches, in place."""
+    assert new_k.is_contiguous() and new_v.is_contiguous()
+    assert new_k.shape == new_v.shape and new_k.dtype == new_v.dtype
+    B, Hkv, Lnew, D = new_k.shape
+    ks, vs = k._struct(), v._struct()
+    _check(lib().qkv_quantize_update(new_k.data_ptr(), new_v.data_ptr(), _DTYPE[new_k.dtype],
+                                     B, Hkv, Lnew, D, C.byref(ks), C.byref(vs), int(offset),
+                                     _stream(stream)))
+
+
+def _mask_struct(mask, causal: bool):
+    if causal:
+        return _Mask(MASK_CAUSAL, None, 0, 0, 0, 0)
+    if mask is None:
+        return None
+    t, strides = mask if isinstance(mask, tuple) else (mask, None)
+    if strides is None:                    # full [B,Hq,Lq,L] (or broadcastable) tensor
+        s = t.stride()
+        strides = (s[0], s[1], s[2]) if t.dim() == 4 else (0, 0, 0)
+    return _Mask(MASK_ADDITIVE, t.data_ptr(), _DTYPE[t.dtype], *[int(x) for x in strides])
+
+
+def _attention(fn, q, k, v, L, scale, mask, causal, out, out_dtype, workspace, stream, decode):
+    assert q.is_contiguous() and q.is_cuda
+    B, Hq, Lq, D = q.shape
+    Hkv = k.codes.shape[1]
+    if out is None:
+        out = torch.empty(B, Hq, Lq, D, dtype=out_dtype or q.dtype, device=q.device)
+    if workspace is None:
+        workspace = make_workspace(B, Hq, Hkv, Lq, D, L, q.device)
+    ks, vs = k._struct(), v._struct()
+    m = _mask_struct(mask, causal)
+    mp = C.byref(m) if m is not None else None
+    common = (C.byref(ks), C.byref(vs), int(L), float(scale), mp, out.data_ptr(),
+              _DTYPE[out.dtype], workspace.data_ptr(), workspace.numel(), _stream(stream))
+    if decode:
+        _check(fn(q.data_ptr(), _DTYPE[q.dtype], B, Hq, Hkv, D, *common))
+    else:
+        _check(fn(q.data_ptr(), _DTYPE[q.dtype], B, Hq, Hkv, Lq, D, *common))
+    return out
+
+
+def qsdpa_decode(q: torch.Tensor, k: QuantCache, v: QuantCache, L: int, scale: float,
+                 mask=None, out: Optional[torch.Tensor] = None, out_dtype=None,
+                 workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """softmax(q*scale . K^T + mask) V for q [B,Hq,1,D] over keys [0, L)."""
+    assert q.shape[2] == 1
+    return _attention(lib().qsdpa_decode, q, k, v, L, scale, mask, False, out, out_dtype,
+                      workspace, stream, True)
+
+
+def qsdpa_prefill(q: torch.Tensor, k: QuantCache, v: QuantCache, L: int, scale: float,
+                  mask=None, causal: bool = False, out: Optional[torch.Tensor] = None,
+                  out_dtype=None, workspace: Optional[torch.Tensor] = None,
+                  stream=None) -> torch.Tensor:
+    """softmax(q*scale . K^T + mask) V for q [B,Hq,Lq,D] over keys [0, L);
+    ``causal`` aligns the Lq queries with the last Lq keys."""
+    return _attention(lib().qsdpa_prefill, q, k, v, L, scale, mask, causal, out, out_dtype,
+                      workspace, stream, False)

@@ -1,0 +1,83 @@
+"""The C-ABI library loads, exports every function include/qkv.h declares,
+and rejects invalid arguments with the documented status codes before any
+CUDA call (these run without a GPU: no compute is launched)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    txt = open(os.path.join(ROOT, "include", "qkv.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(q\w+)\s*\(", txt)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from quantized_kv_attention_split_b200 import qkv
+    return qkv.lib()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert {"qkv_quantize_update", "qsdpa_decode", "qsdpa_prefill"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    assert lib.qkv_status_string(0) == b"ok"
+    assert lib.qkv_status_string(4) == b"workspace too small"
+    assert lib.qkv_status_string(99) == b"unknown status"
+
+
+FAKE = 0x7f0000000000   # 16-byte aligned, never dereferenced: every call below fails validation
+
+
+def _cache(qkv, fmt=0, bits=4, gs=64, Lcap=64, codes=FAKE, scales=FAKE + 4096, biases=FAKE + 8192):
+    return qkv._Cache(fmt, bits, gs, codes, scales, biases, Lcap)
+
+
+def _decode(lib, qkv, k, v, D=128, L=16, q=FAKE, out=FAKE + 65536, qdt=0, odt=0, Hq=8, Hkv=2):
+    return lib.qsdpa_decode(q, qdt, 1, Hq, Hkv, D, C.byref(k), C.byref(v), L, 1.0, None,
+                            out, odt, FAKE + 131072, 1 << 20, None)
+
+
+def test_decode_validation_errors(lib):
+    from quantized_kv_attention_split_b200 import qkv
+    ok = _cache(qkv)
+    assert _decode(lib, qkv, _cache(qkv, bits=5), ok) == 2                 # unsupported bits
+    assert b"bits" in lib.qkv_last_error()
+    assert _decode(lib, qkv, _cache(qkv, gs=48), ok) == 2                  # unsupported group
+    assert _decode(lib, qkv, ok, ok, D=96) == 2                            # unsupported D
+    assert _decode(lib, qkv, _cache(qkv, Lcap=60), _cache(qkv, Lcap=60)) == 3   # Lcap % 8
+    assert _decode(lib, qkv, _cache(qkv, codes=FAKE + 4), ok) == 3         # misaligned codes
+    assert _decode(lib, qkv, ok, ok, q=FAKE + 2) == 3                       # misaligned q
+    assert _decode(lib, qkv, _cache(qkv, biases=0), ok) == 1               # affine without biases
+    assert _decode(lib, qkv, _cache(qkv, fmt=1, bits=4, gs=32), ok) == 1    # bad Q8_0 bits
+    assert _decode(lib, qkv, ok, _cache(qkv, bits=8)) == 2                  # k/v mismatch
+    assert _decode(lib, qkv, ok, ok, L=65) == 1                             # L > Lcap
+    assert _decode(lib, qkv, ok, ok, L=-1) == 1
+    assert _decode(lib, qkv, ok, ok, Hq=6, Hkv=4) == 1                      # Hq % Hkv
+    assert _decode(lib, qkv, ok, ok, qdt=2) == 1                            # q must be 16-bit
+    assert _decode(lib, qkv, ok, ok, odt=7) == 1                            # unknown out dtype
+    assert _decode(lib, qkv, ok, ok, q=0) == 1                              # NULL q
+    m = qkv._Mask(9, None, 0, 0, 0, 0)
+    assert lib.qsdpa_decode(FAKE, 0, 1, 8, 2, 128, C.byref(ok), C.byref(ok), 16, 1.0,
+                            C.byref(m), FAKE, 0, FAKE, 1 << 20, None) == 1  # unknown mask kind
+
+
+def test_quantize_validation_errors(lib):
+    from quantized_kv_attention_split_b200 import qkv
+    ok = _cache(qkv)
+    f = lib.qkv_quantize_update
+    assert f(FAKE, FAKE, 0, 1, 2, 4, 128, C.byref(ok), C.byref(ok), 61, None) == 1  # offset
+    assert f(FAKE, FAKE, 2, 1, 2, 4, 128, C.byref(ok), C.byref(ok), 0, None) == 1   # f32 input
+    assert f(FAKE + 8, FAKE, 0, 1, 2, 4, 128, C.byref(ok), C.byref(ok), 0, None) == 3
+    assert f(0, FAKE, 0, 1, 2, 4, 128, C.byref(ok), C.byref(ok), 0, None) == 1
+    assert f(FAKE, FAKE, 0, 1, 2, 4, 128, C.byref(_cache(qkv, bits=3)), C.byref(ok), 0, None) == 2
+    assert f(FAKE, FAKE, 0, 1, 2, 0, 128, C.byref(ok), C.byref(ok), 0, None) == 0   # nothing to do

@@ -1,0 +1,96 @@
+"""GPU quantize-and-append (qkv_quantize_update) must match the oracle's
+quantizer bit for bit: codes, fp16 scales and fp16 biases, written only to
+rows [offset, offset+Lnew) of each (batch, kv-head)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from helpers import cache_from_dev, to_dev
+from quantized_kv_attention_split_b200 import synthetic as S
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def qkv():
+    from quantized_kv_attention_split_b200 import qkv as m
+    m.lib()
+    return m
+
+
+def _inputs(shape, kind, dtype, seed):
+    rng = np.random.default_rng(seed)
+    if kind == "uniform":
+        x = rng.random(shape, dtype=np.float32)
+    elif kind == "normal":
+        x = rng.standard_normal(shape).astype(np.float32)
+    elif kind == "wide":
+        x = (rng.standard_normal(shape) * 10.0 ** rng.uniform(-4, 3, shape[:-1] + (1,))).astype(
+            np.float32)
+    elif kind == "special":                  # constant groups, zeros, ties
+        x = np.zeros(shape, np.float32)
+        x[..., 1::4, :] = 0.5
+        x[..., 2::4, :] = np.arange(shape[-1]) % 3 - 1.0
+        x[..., 3::4, :] = rng.integers(-4, 5, shape[:-2] + (len(range(3, shape[-2], 4)), shape[-1]))
+    return S.f32_to_half_bits(x, dtype)
+
+
+CASES = [
+    # fmt, bits, gs, D, dtype
+    ("affine", 4, 64, 128, "f16"), ("affine", 4, 32, 64, "f16"), ("affine", 4, 128, 256, "bf16"),
+    ("affine", 8, 64, 128, "bf16"), ("affine", 8, 32, 256, "f16"), ("affine", 8, 128, 128, "f16"),
+    ("q8_0", 8, 32, 256, "f16"), ("q8_0", 8, 32, 64, "bf16"),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "-".join(map(str, c)))
+@pytest.mark.parametrize("kind", ["uniform", "normal", "wide", "special"])
+def test_quantize_update_bit_exact(qkv, case, kind):
+    fmt, bits, gs, D, dtype = case
+    B, Hkv, Lnew, Lcap, offset = 2, 3, 37, 64, 19
+    nk = _inputs((B, Hkv, Lnew, D), kind, dtype, 1)
+    nv = _inputs((B, Hkv, Lnew, D), kind, dtype, 2)
+    from quantized_kv_attention_split_b200.qkv import QuantCache, AFFINE, Q8_0
+    f = Q8_0 if fmt == "q8_0" else AFFINE
+    kd = QuantCache.empty(B, Hkv, Lcap, D, f, bits, gs)
+    vd = QuantCache.empty(B, Hkv, Lcap, D, f, bits, gs)
+    qkv.qkv_quantize_update(to_dev(nk, dtype), to_dev(nv, dtype), kd, vd, offset)
+    torch.cuda.synchronize()
+    for got_d, src in ((kd, nk), (vd, nv)):
+        got = cache_from_dev(got_d, fmt)
+        ref = oracle.quantize(src, dtype, fmt, gs, bits)
+        sl = slice(offset, offset + Lnew)
+        assert np.array_equal(got.codes[:, :, sl], ref.codes)
+        assert np.array_equal(got.scales[:, :, sl], ref.scales)
+        if fmt == "affine":
+            assert np.array_equal(got.biases[:, :, sl], ref.biases)
+        # nothing written outside the target rows
+        assert not got.codes[:, :, :offset].any() and not got.codes[:, :, offset + Lnew:].any()
+        assert not got.scales[:, :, :offset].any() and not got.scales[:, :, offset + Lnew:].any()
+
+
+def test_single_token_update_matches_bulk(qkv):
+    """Appending tokens one at a time gives the same cache as one bulk call."""
+    from quantized_kv_attention_split_b200.qkv import QuantCache
+    B, Hkv, D, Ln = 1, 8, 128, 24
+    nk = _inputs((B, Hkv, Ln, D), "normal", "f16", 5)
+    nv = _inputs((B, Hkv, Ln, D), "normal", "f16", 6)
+    a_k, a_v = QuantCache.empty(B, Hkv, 32, D, bits=8), QuantCache.empty(B, Hkv, 32, D, bits=8)
+    b_k, b_v = QuantCache.empty(B, Hkv, 32, D, bits=8), QuantCache.empty(B, Hkv, 32, D, bits=8)
+    qkv.qkv_quantize_update(to_dev(nk, "f16"), to_dev(nv, "f16"), a_k, a_v, 3)
+    for i in range(Ln):
+        qkv.qkv_quantize_update(to_dev(nk[:, :, i:i + 1].copy(), "f16"),
+                                to_dev(nv[:, :, i:i + 1].copy(), "f16"), b_k, b_v, 3 + i)
+    torch.cuda.synchronize()
+    for x, y in ((a_k, b_k), (a_v, b_v)):
+        assert torch.equal(x.codes, y.codes) and torch.equal(x.scales, y.scales)
+        assert torch.equal(x.biases, y.biases)
+
+
+def test_quantize_rejects_bad_offset(qkv):
+    from quantized_kv_attention_split_b200.qkv import QuantCache
+    kd, vd = QuantCache.empty(1, 1, 16, 64), QuantCache.empty(1, 1, 16, 64)
+    x = torch.zeros(1, 1, 4, 64, dtype=torch.float16, device="cuda")
+    with pytest.raises(qkv.QKVError, match="offset"):
+        qkv.qkv_quantize_update(x, x, kd, vd, 13)
