@@ -130,6 +130,26 @@ qkv_status qsdpa_prefill(const void* q, int q_dtype, int B, int Hq, int Hkv, int
                          float scale, const qkv_mask* mask, void* out, int out_dtype,
                          void* workspace, size_t workspace_bytes, void* stream);
 
+/* Allocation-free variant of qsdpa_decode (the pages have no counterpart:
+ * MLX and llama.cpp allocate their temporaries through their own allocators).
+ * For callers that cannot allocate device memory when they decode -- code
+ * that runs under an allocator which forbids cudaMalloc/cudaFree, services
+ * that fix every buffer before they start, or plug-in interfaces that hand
+ * over only inputs and outputs.  Same arguments and results as qsdpa_decode,
+ * without the workspace: its scratch (tickets and partial results) lives in a
+ * 16 MiB array built into this library, which every GPU that loads the
+ * library keeps until the process exits.  Shapes whose workspace
+ * (qsdpa_workspace_size) exceeds 16 MiB are rejected with QKV_ERR_WORKSPACE.
+ * The first call on a device looks up that device's address of the array;
+ * make that first call before any stream capture.  Every call clears the
+ * tickets it needs and reuses the same array, so calls that may overlap on the
+ * GPU (other streams, other host threads on the same device) race: order them
+ * on one stream. */
+qkv_status qsdpa_decode_noalloc(const void* q, int q_dtype, int B, int Hq, int Hkv, int D,
+                                const qkv_cache* k, const qkv_cache* v, int64_t L,
+                                float scale, const qkv_mask* mask, void* out, int out_dtype,
+                                void* stream);
+
 /* Workspace bytes needed by qsdpa_decode (Lq = 1) or qsdpa_prefill for this
  * problem on the CURRENT device, and how many leading bytes must be zero
  * before the first call.  0 on invalid arguments. */

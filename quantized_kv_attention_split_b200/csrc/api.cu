@@ -222,3 +222,77 @@ qkv_status qsdpa_prefill(const void* q, int q_dtype, int B, int Hq, int Hkv, int
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free decode entry point.
+//
+// Some callers cannot allocate device memory at the point where they decode:
+// code running inside a memory pool that forbids cudaMalloc/cudaFree, hosts
+// that pre-plan every buffer before serving starts, or plug-in interfaces that
+// only hand over input and output pointers.  For them, qsdpa_decode_noalloc
+// runs the same decode kernel as qsdpa_decode but keeps its scratch (the
+// per-unit tickets and the partial results of the split over L) in a
+// fixed-size array that lives in this library's device image.  Every GPU that
+// loads the library holds that array until the process exits.
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = 16u << 20;   // 16 MiB per device
+constexpr int kNoAllocMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+// Device address of the scratch array for the current device.  Taken once per
+// device with that device current (the host-side symbol is only a stand-in and
+// must never be handed to a kernel).
+qkv_status noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(QKV_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kNoAllocMaxDevices)
+    return fail(QKV_ERR_UNSUPPORTED, "device %d beyond the %d devices supported", dev,
+                kNoAllocMaxDevices);
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr)
+      return fail(QKV_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return QKV_OK;
+}
+
+}  // namespace
+
+extern "C" qkv_status qsdpa_decode_noalloc(const void* q, int q_dtype, int B, int Hq, int Hkv,
+                                           int D, const qkv_cache* k, const qkv_cache* v,
+                                           int64_t L, float scale, const qkv_mask* mask,
+                                           void* out, int out_dtype, void* stream) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0)
+    return fail(QKV_ERR_INVALID_ARG, "B, Hq, Hkv must be positive and Hq a multiple of Hkv");
+  const size_t need = qsdpa_workspace_size(B, Hq, Hkv, 1, D, L);
+  if (need == 0) return fail(QKV_ERR_INVALID_ARG, "invalid decode shape (D=%d, L=%lld)", D,
+                             (long long)L);
+  if (need > kNoAllocScratchBytes)
+    return fail(QKV_ERR_WORKSPACE,
+                "qsdpa_decode_noalloc: this shape needs %zu bytes of scratch, more than the "
+                "%zu bytes built into the library; use qsdpa_decode with a caller workspace",
+                need, kNoAllocScratchBytes);
+  void* scratch = nullptr;
+  qkv_status st = noalloc_scratch(&scratch);
+  if (st != QKV_OK) return st;
+  // the tickets at the front must be zero; the previous call left them zero,
+  // but clear them anyway so an interrupted call cannot poison the next one
+  const size_t zero = qsdpa_workspace_zero_bytes(B, Hq, Hkv, 1, D, L);
+  cudaError_t e = cudaMemsetAsync(scratch, 0, zero, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(QKV_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e));
+  return qsdpa_decode(q, q_dtype, B, Hq, Hkv, D, k, v, L, scale, mask, out, out_dtype, scratch,
+                      kNoAllocScratchBytes, stream);
+}

@@ -200,3 +200,30 @@ def qsdpa_prefill(q: torch.Tensor, k: QuantCache, v: QuantCache, L: int, scale: 
     ``causal`` aligns the Lq queries with the last Lq keys."""
     return _attention(lib().qsdpa_prefill, q, k, v, L, scale, mask, causal, out, out_dtype,
                       workspace, stream, False)
+
+
+def qsdpa_decode_noalloc(q: torch.Tensor, k: QuantCache, v: QuantCache, L: int, scale: float,
+                         mask=None, out: Optional[torch.Tensor] = None, out_dtype=None,
+                         stream=None) -> torch.Tensor:
+    """Like :func:`qsdpa_decode` but without a workspace: the library keeps the
+    scratch in a fixed 16 MiB array of its own (for callers that cannot
+    allocate device memory at decode time).  ``out`` should be passed by such
+    callers; it is only allocated here when omitted.  Calls must not overlap
+    on the GPU."""
+    f = lib().qsdpa_decode_noalloc
+    if f.argtypes is None:
+        f.argtypes = [C.c_void_p, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
+                      C.POINTER(_Cache), C.POINTER(_Cache), C.c_int64, C.c_float,
+                      C.POINTER(_Mask), C.c_void_p, C.c_int, C.c_void_p]
+        f.restype = C.c_int
+    assert q.is_contiguous() and q.is_cuda and q.shape[2] == 1
+    B, Hq, _, D = q.shape
+    Hkv = k.codes.shape[1]
+    if out is None:
+        out = torch.empty(B, Hq, 1, D, dtype=out_dtype or q.dtype, device=q.device)
+    ks, vs = k._struct(), v._struct()
+    m = _mask_struct(mask, False)
+    _check(f(q.data_ptr(), _DTYPE[q.dtype], B, Hq, Hkv, D, C.byref(ks), C.byref(vs), int(L),
+             float(scale), C.byref(m) if m is not None else None, out.data_ptr(),
+             _DTYPE[out.dtype], _stream(stream)))
+    return out
