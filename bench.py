@@ -452,7 +452,34 @@ def other_rows(device):
                       "frac_hbm": round(nb / (sec / 1e3) / 1e9 / hbm_peak, 4)}
         del caches
         torch.cuda.empty_cache()
+
+    # prefill: 512 causal queries at depth 20480 over a Q8_0 cache (tcgen05 kernel)
+    w = S.WORKLOADS["prefill_q8_0_512_at_20k"]
+    inp = S.make_inputs(w)
+    caches = build_caches(w, inp, 1, device)
+    q = dev16(inp.q, w.q_dtype, device)
+    out = torch.empty(w.B, w.Hq, w.Lq, w.D, dtype=torch.bfloat16, device=device)
+    ws = qkv.make_workspace(w.B, w.Hq, w.Hkv, w.Lq, w.D, w.L, device)
+    kc, vc = caches[0]
+    sec, _ = graph_time(lambda i: qkv.qsdpa_prefill(q, kc, vc, w.L, w.scale, causal=True, out=out,
+                                                    workspace=ws), 20, 3)
+    flop = prefill_flops(w)
+    _, bf16_peak, _ = peaks()
+    rows[w.name] = {"us_per_call": round(sec * 1e3, 2),
+                    "TFLOP/s": round(flop / (sec / 1e3) / 1e12, 1),
+                    "frac_tensor_peak": round(flop / (sec / 1e3) / 1e12 / bf16_peak, 4),
+                    "flop": flop,
+                    "peak_note": "fp16 operands; measured bf16 dense peak x nominal fp16:bf16 ratio 1"}
+    del caches
+    torch.cuda.empty_cache()
     return rows
+
+
+def prefill_flops(w):
+    """Multiply-adds of Q K^T and P V actually required (causal keys only):
+    4 * D * Hq * sum over queries of visible keys."""
+    vis = sum(min(w.L, w.L - w.Lq + i + 1) for i in range(w.Lq))
+    return 4 * w.D * w.Hq * w.B * vis
 
 
 def run_reference(args, rank, world):

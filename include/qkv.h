@@ -124,7 +124,13 @@ qkv_status qsdpa_decode(const void* q, int q_dtype, int B, int Hq, int Hkv, int 
 /* Multi-query attention (any Lq >= 1) over keys [0, L) with an optional mask
  * (the pages' Lq > 1 fallback: quantized_matmul -> softmax -> quantized_matmul,
  * computed here in one fused pass).  q/out: [B, Hq, Lq, D] contiguous.
- * Same workspace rules as qsdpa_decode. */
+ * Same workspace rules as qsdpa_decode.  With at least 64 (head, query) rows
+ * per kv head and f16/bf16 output the call runs on the tcgen05 tensor-core
+ * kernel (K and V tiles dequantized to fp16, fp32 accumulation in TMEM);
+ * otherwise, and always for f32 output, on the split-K kernel.  The tcgen05
+ * kernel bounds its waits on the tensor core: if one ever times out it sets
+ * the first 32-bit word of the workspace nonzero (the output is then invalid);
+ * that word must be zeroed again before the workspace is reused. */
 qkv_status qsdpa_prefill(const void* q, int q_dtype, int B, int Hq, int Hkv, int Lq,
                          int D, const qkv_cache* k, const qkv_cache* v, int64_t L,
                          float scale, const qkv_mask* mask, void* out, int out_dtype,

@@ -13,11 +13,21 @@ cudaError_t launch_quantize(const void* new_k, const void* new_v, int in_dtype, 
 size_t decode_workspace_bound(int B, int Hq, int Hkv, int D);
 size_t decode_workspace_zero_bytes(int B, int Hq, int Hkv);
 void decode_chunking(int G, int* nc, int* ncg);
+struct PrefillParams;
+}  // namespace qkv
+#include "prefill_kernel.cuh"
+namespace qkv {
+cudaError_t launch_prefill_tc(int D, int bits, int gs, int fmt, PrefillParams& p, cudaStream_t s);
 }  // namespace qkv
 
 namespace {
 
 thread_local char g_last_error[512] = "";
+
+// Multi-query calls with at least this many (head, query) rows per kv head run
+// on the tcgen05 kernel; smaller ones, and fp32 output (whose 1e-4 accuracy
+// needs the split-precision value operand), on the split-K kernel.
+constexpr int kTensorPrefillMinRows = 64;
 
 qkv_status fail(qkv_status st, const char* fmt, ...) {
   va_list ap;
@@ -118,6 +128,30 @@ qkv_status attention(const void* q, int q_dtype, int B, int Hq, int Hkv, int Lq,
 
   const int G = Hq / Hkv;
   const int rows = G * Lq;                 // rows of one kv head: (head, query) pairs
+  if (Lq > 1 && rows >= kTensorPrefillMinRows && out_dtype != QKV_F32) {
+    // many query rows per kv head: the tcgen05 kernel (whole 128-row tiles)
+    const size_t need = qsdpa_workspace_size(B, Hq, Hkv, Lq, D, L);
+    if (workspace == nullptr || workspace_bytes < need)
+      return fail(QKV_ERR_WORKSPACE, "workspace of %zu bytes required (got %zu)", need,
+                  workspace_bytes);
+    qkv::PrefillParams pp;
+    std::memset(&pp, 0, sizeof(pp));
+    pp.q = q; pp.q_dtype = q_dtype; pp.out = out; pp.out_dtype = out_dtype;
+    pp.kc = reinterpret_cast<const uint8_t*>(k->codes); pp.ks = k->scales; pp.kb = k->biases;
+    pp.vc = reinterpret_cast<const uint8_t*>(v->codes); pp.vs = v->scales; pp.vb = v->biases;
+    pp.Lcap = k->Lcap; pp.L = L;
+    pp.B = B; pp.Hq = Hq; pp.Hkv = Hkv; pp.G = G; pp.Lq = Lq;
+    pp.scale_log2e = scale * 1.4426950408889634f;
+    pp.mask_kind = mkind;
+    if (mkind == QKV_MASK_ADDITIVE) {
+      pp.mask = mask->add; pp.mask_dtype = mask->add_dtype;
+      pp.msb = mask->stride_b; pp.msh = mask->stride_h; pp.msq = mask->stride_q;
+    }
+    pp.status = static_cast<unsigned*>(workspace);
+    cudaError_t e = qkv::launch_prefill_tc(D, k->bits, k->group_size, k->fmt, pp, s);
+    if (e != cudaSuccess) return fail(QKV_ERR_CUDA, "prefill launch: %s", cudaGetErrorString(e));
+    return ok();
+  }
   qkv::DecodePlan plan;
   if (!qkv::plan_decode(D, k->bits, k->group_size, k->fmt, out_dtype == QKV_F32, B,
                         Hkv * rows, Hkv, L, &plan))
@@ -145,8 +179,12 @@ qkv_status attention(const void* q, int q_dtype, int B, int Hq, int Hkv, int Lq,
   if (mkind == QKV_MASK_CAUSAL && Lq == 1) p.mask_kind = QKV_MASK_NONE;  // all keys visible
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   p.tickets = reinterpret_cast<unsigned*>(ws);
-  p.part_o = reinterpret_cast<float*>(ws + plan.ws_tickets);
-  p.part_ml = reinterpret_cast<float*>(ws + plan.ws_tickets + plan.ws_part_o);
+  p.tickets1 = reinterpret_cast<unsigned*>(ws + plan.ws_tickets2);
+  uint8_t* parts = ws + plan.ws_tickets;
+  p.part_o = reinterpret_cast<float*>(parts);
+  p.part_ml = reinterpret_cast<float*>(parts + plan.ws_part_o);
+  p.part2_o = reinterpret_cast<float*>(parts + plan.ws_part_o + plan.ws_part_ml);
+  p.part2_ml = reinterpret_cast<float*>(parts + 2 * plan.ws_part_o + plan.ws_part_ml);
   cudaError_t e = qkv::launch_decode(D, k->bits, k->group_size, k->fmt, out_dtype == QKV_F32,
                                      plan, p, s);
   if (e != cudaSuccess) return fail(QKV_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));

@@ -43,7 +43,9 @@ namespace qkv {
 
 constexpr int kDecWarps = 8;
 constexpr int kDecThreads = kDecWarps * 32;
-constexpr int kDecStageBudget = 96 * 1024;
+// 16-key blocks per warp per stage: two, except for 256-byte code rows (a
+// stage of 256 such keys would not fit in shared memory)
+__host__ __device__ constexpr int dec_sub(int D, int bits) { return D * bits / 8 >= 256 ? 1 : 2; }
 
 // XOR coefficients (3 bits each, for line bits 0..3) of the 16-byte-unit
 // swizzle inside each 128-byte line of a staged code tile, found by exhaustive
@@ -62,6 +64,13 @@ __host__ __device__ constexpr uint32_t swizzle_coeffs(int D, int bits, int gs) {
                        : gs == 64 ? swz_pack(2, 4, 2, 0) : swz_pack(4, 2, 4, 0))
                     : (gs == 32 ? swz_pack(0, 2, 4, 2)
                        : gs == 64 ? swz_pack(0, 4, 2, 4) : swz_pack(0, 1, 2, 4)));
+}
+
+// XOR pattern (already shifted to bits 4..6) of 128-byte line `line`.
+template <uint32_t SWZ>
+__host__ __device__ __forceinline__ constexpr int swz_line(int line) {
+  return (((line & 1) ? (SWZ & 7) : 0) ^ ((line & 2) ? ((SWZ >> 3) & 7) : 0) ^
+          ((line & 4) ? ((SWZ >> 6) & 7) : 0) ^ ((line & 8) ? ((SWZ >> 9) & 7) : 0)) << 4;
 }
 
 template <uint32_t SWZ>
@@ -90,15 +99,22 @@ struct DecCfg {
   static constexpr int NMETA = Q8 ? 2 : 4;
   static constexpr int MROW = NG * 2;          // meta bytes per key per array
   static constexpr int WPC = kDecWarps / NC;   // warps per head chunk
-  static constexpr int TK = 16 * WPC;          // keys per stage
+  static constexpr int SUB = dec_sub(D, BITS);   // 16-key blocks per warp per stage
+  static constexpr int TK = 16 * SUB * WPC;      // keys per stage
   static constexpr int CODES = TK * RB;
   static constexpr int META = ((TK * MROW + 127) / 128) * 128;
   static constexpr int META_UNITS = TK * MROW / 16;
   static constexpr int STAGE = 2 * CODES + NMETA * META;
-  static constexpr int NSTAGE = kDecStageBudget / STAGE > 6 ? 6
-                              : (kDecStageBudget / STAGE < 2 ? 2 : kDecStageBudget / STAGE);
-  static constexpr int EPI = kDecWarps * (8 * D + 16) * 4;
-  static constexpr int SMEM = NSTAGE * STAGE > EPI ? NSTAGE * STAGE : EPI;
+  // two CTAs per SM for D <= 128 (one for D = 256): shared-memory budget per CTA
+  // (228 KB per SM holds two CTAs of 108 KB plus their reserved 1 KB each)
+  static constexpr int BUDGET = D <= 128 ? 110592 - NC * 8 * D * 4 : 190 * 1024;
+  static constexpr int NSTAGE = BUDGET / STAGE > 6 ? 6 : (BUDGET / STAGE < 2 ? 2 : BUDGET / STAGE);
+  // epilogue: per-warp partial rows, then the merge scratch (<= 48 parts)
+  static constexpr int EPI = kDecWarps * (8 * D + 16) * 4 + (48 * 32 * 2 + 2 * 32 + 48) * 4;
+  static constexpr int RING = NSTAGE * STAGE > EPI ? NSTAGE * STAGE : EPI;
+  static constexpr int QS_OFF = RING;                 // fp32 query rows of the CTA
+  static constexpr int SMEM = RING + NC * 8 * D * 4;
+  static_assert(SMEM <= 227 * 1024, "shared memory budget");
   static constexpr uint32_t SWZ = swizzle_coeffs(D, BITS, GS);
   static_assert(D % GS == 0, "D must be a multiple of the group size");
   static_assert(NG <= 8, "at most 8 groups per row");
@@ -132,13 +148,129 @@ __device__ __forceinline__ void lds_meta(const uint8_t* p, uint16_t* h) {
   }
 }
 
+constexpr int kMergeGroup = 8;
+
+// Combines n partial results (m, l, o) of one unit, read from the slots
+// slot(0..n-1), by log-sum-exp rescaling.  Writes either the normalized output
+// (out != nullptr; rows hbase.. of the unit starting at element out_base) or
+// a combined partial (dst_ml/dst_o).  The weights are computed once in shared
+// memory so every thread then issues independent loads of the o parts.
+template <int D, int HPC, class SlotFn>
+__device__ __forceinline__ void merge_parts(const float* ml, const float* po, int n, SlotFn slot,
+                                            float* sm, int tid, int hbase, int G,
+                                            float* dst_ml, float* dst_o, void* out, int out_dtype,
+                                            int64_t out_base) {
+  float* w = sm;                                   // [n][HPC] weights (m first)
+  float* lw = sm + n * HPC;                        // [n][HPC] partial sums
+  float* hm = lw + n * HPC;                        // [HPC] max, then combined sum
+  int* sl = reinterpret_cast<int*>(hm + 2 * HPC);  // [n] slots
+  for (int i = tid; i < n; i += kDecThreads) sl[i] = (int)slot(i);
+  __syncthreads();
+  for (int i = tid; i < n * HPC; i += kDecThreads) {
+    const int pp = i / HPC, hl = i - pp * HPC;
+    w[i] = __ldcg(&ml[((int64_t)sl[pp] * HPC + hl) * 2 + 0]);
+    lw[i] = __ldcg(&ml[((int64_t)sl[pp] * HPC + hl) * 2 + 1]);
+  }
+  __syncthreads();
+  for (int hl = tid; hl < HPC; hl += kDecThreads) {
+    float M = -INFINITY;
+    for (int pp = 0; pp < n; ++pp) M = fmaxf(M, w[pp * HPC + hl]);
+    float l = 0.f;
+    for (int pp = 0; pp < n; ++pp) {
+      const float m = w[pp * HPC + hl];
+      const float sc = m == -INFINITY ? 0.f : ex2(m - M);
+      w[pp * HPC + hl] = sc;
+      l = fmaf(sc, lw[pp * HPC + hl], l);
+    }
+    hm[hl] = M;
+    hm[HPC + hl] = l;
+  }
+  __syncthreads();
+  // four consecutive outputs per step, up to 8 parts' loads in flight
+  constexpr int V4 = D / 4;
+  for (int idx = tid; idx < HPC * V4; idx += kDecThreads) {
+    const int hl = idx / V4, e4 = idx - hl * V4;
+    if (hbase + hl >= G) continue;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int p0 = 0; p0 < n; p0 += 8) {
+      float4 o[8];
+      float wv[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int pp = p0 + u;
+        if (pp < n) {
+          o[u] = __ldcg(reinterpret_cast<const float4*>(po + ((int64_t)sl[pp] * HPC + hl) * D) + e4);
+          wv[u] = w[pp * HPC + hl];
+        } else {
+          o[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+          wv[u] = 0.f;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        acc.x = fmaf(wv[u], o[u].x, acc.x);
+        acc.y = fmaf(wv[u], o[u].y, acc.y);
+        acc.z = fmaf(wv[u], o[u].z, acc.z);
+        acc.w = fmaf(wv[u], o[u].w, acc.w);
+      }
+    }
+    const float l = hm[HPC + hl];
+    const int e = e4 * 4;
+    if (out != nullptr) {
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const int64_t oi = out_base + (int64_t)(hbase + hl) * D + e;
+      store_from_float(out, out_dtype, oi, acc.x * inv);
+      store_from_float(out, out_dtype, oi + 1, acc.y * inv);
+      store_from_float(out, out_dtype, oi + 2, acc.z * inv);
+      store_from_float(out, out_dtype, oi + 3, acc.w * inv);
+    } else {
+      *reinterpret_cast<float4*>(dst_o + hl * D + e) = acc;
+      if (e == 0) { dst_ml[hl * 2] = hm[hl]; dst_ml[hl * 2 + 1] = l; }
+    }
+  }
+}
+
+// Raw fp16 bits of group G's scale (or bias) of row r in a staged meta array.
+template <int NG>
+__device__ __forceinline__ uint16_t meta_half(const uint8_t* base, int r, int G) {
+  return reinterpret_cast<const uint16_t*>(base)[r * NG + G];
+}
+
+// Group G's value (as float) of a metadata row held as 32-bit words.
+template <int NG>
+__device__ __forceinline__ float meta_f(const uint32_t* w, int G) {
+  if constexpr (NG == 1) {
+    return half_bits_to_float((uint16_t)w[0]);
+  } else {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[G >> 1]));
+    return (G & 1) ? f.y : f.x;
+  }
+}
+// Group G's 16-bit value of a metadata row held as 32-bit words.
+template <int NG>
+__device__ __forceinline__ uint32_t meta_bits(const uint32_t* w, int G) {
+  if constexpr (NG == 1) return w[0] & 0xffffu;
+  else return (G & 1) ? (w[G >> 1] >> 16) : (w[G >> 1] & 0xffffu);
+}
+// A key's NG metadata halves as 32-bit words.
+template <int NG>
+__device__ __forceinline__ void meta_row(const uint8_t* base, int r, uint32_t* w) {
+  if constexpr (NG == 1) {
+    w[0] = reinterpret_cast<const uint16_t*>(base)[r];
+  } else {
+    lds_words<NG / 2>(base + r * NG * 2, w);
+  }
+}
+
 template <int D, int BITS, int GS, bool Q8, int NC, bool F32OUT>
-__global__ void __launch_bounds__(kDecThreads, 1)
+__global__ void __launch_bounds__(kDecThreads, D <= 128 ? 2 : 1)
 qsdpa_decode_kernel(const DecodeParams p) {
   using C = DecCfg<D, BITS, GS, Q8, NC>;
   constexpr int NG = C::NG, KPG = C::KPG, MT = C::MT, TK = C::TK, NSTAGE = C::NSTAGE;
   constexpr int HPC = NC * 8;
+  constexpr int MW = NG == 1 ? 1 : NG / 2;     // 32-bit words of one key's metadata row
   extern __shared__ __align__(128) uint8_t smem[];
+  float* qst = reinterpret_cast<float*>(smem + C::QS_OFF);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
@@ -159,21 +291,51 @@ qsdpa_decode_kernel(const DecodeParams p) {
     const int hkv = (int)((u / p.ncg) % p.Hkv);
     const int b = (int)(u / ((int64_t)p.ncg * p.Hkv));
     const int64_t row0 = ((int64_t)b * p.Hkv + hkv) * p.Lcap;   // first cache row of this head
-    const int hbase = cg * HPC;                                  // first local head of the CTA
-    const int myhead = hbase + chunk * 8 + g;                    // head whose q this lane loads
-    const bool head_ok = myhead < p.G;
+    const int hbase = cg * HPC;                                  // first local row of the CTA
+
+    // ---------------- query rows -> shared memory (fp32), 16-byte loads --------
+    {
+      const int64_t qbase = (((int64_t)b * p.Hkv + hkv) * p.G + hbase) * D;
+      const int nrows = min(HPC, p.G - hbase);
+      for (int i = tid; i < HPC * D / 8; i += kDecThreads) {
+        const int hl = i / (D / 8), c = i - hl * (D / 8);
+        float v[8];
+        if (hl < nrows) {
+          const uint4 raw = *reinterpret_cast<const uint4*>(
+              reinterpret_cast<const uint16_t*>(p.q) + qbase + (int64_t)hl * D + c * 8);
+          const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            if (p.q_dtype == QKV_F16) {
+              const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
+              v[2 * k] = f.x; v[2 * k + 1] = f.y;
+            } else {
+              v[2 * k] = __uint_as_float(w[k] << 16);
+              v[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) v[k] = 0.f;
+        }
+        float4* dst = reinterpret_cast<float4*>(qst + hl * D + c * 8);
+        dst[0] = make_float4(v[0], v[1], v[2], v[3]);
+        dst[1] = make_float4(v[4], v[5], v[6], v[7]);
+      }
+      __syncthreads();
+    }
 
     // ---------------- query fragments (B operand of the score MMA) ----------
     uint32_t bq[C::KSTEPS][2];
     float qsc[NG][2];
     float scaleK;
     {
-      const int64_t qrow = (((int64_t)b * p.Hkv + hkv) * p.G + myhead) * D;
-      float qv[C::KSTEPS][4];
+      const float* qr = qst + (chunk * 8 + g) * D;
       float qs[NG];
 #pragma unroll
       for (int gg = 0; gg < NG; ++gg) qs[gg] = 0.f;
       float qmax = 0.f;
+      float qv[C::KSTEPS][4];
 #pragma unroll
       for (int s = 0; s < C::KSTEPS; ++s) {
         const int G = s / KPG, ks = s % KPG;
@@ -188,7 +350,7 @@ qsdpa_decode_kernel(const DecodeParams p) {
         }
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          qv[s][i] = head_ok ? load_as_float(p.q, p.q_dtype, qrow + e[i]) : 0.f;
+          qv[s][i] = qr[e[i]];
           qs[G] += qv[s][i];
           qmax = fmaxf(qmax, fabsf(qv[s][i]));
         }
@@ -202,15 +364,11 @@ qsdpa_decode_kernel(const DecodeParams p) {
       const float qscale16 = exp2i(sigma - 4);
 #pragma unroll
       for (int s = 0; s < C::KSTEPS; ++s) {
-        if constexpr (BITS == 4) {
-          bq[s][0] = pack_half2(qv[s][0] * qscale, qv[s][1] * qscale);
-          bq[s][1] = pack_half2(qv[s][2] * qscale16, qv[s][3] * qscale16);
-        } else {
-          bq[s][0] = pack_half2(qv[s][0] * qscale, qv[s][1] * qscale);
-          bq[s][1] = pack_half2(qv[s][2] * qscale, qv[s][3] * qscale);
-        }
+        const float sc2 = BITS == 4 ? qscale16 : qscale;
+        bq[s][0] = pack_half2(qv[s][0] * qscale, qv[s][1] * qscale);
+        bq[s][1] = pack_half2(qv[s][2] * sc2, qv[s][3] * sc2);
       }
-      // group sums: reduce over t, then hand heads 2t, 2t+1 to every lane
+      // group sums: reduce over t, then hand rows 2t, 2t+1 to every lane
 #pragma unroll
       for (int gg = 0; gg < NG; ++gg) {
         qs[gg] += __shfl_xor_sync(~0u, qs[gg], 1);
@@ -225,8 +383,9 @@ qsdpa_decode_kernel(const DecodeParams p) {
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
     float beta[2][NG];
     float O[MT][4];
+    int tau[NG];          // per group: O of that group is kept scaled by 2^tau
 #pragma unroll
-    for (int gg = 0; gg < NG; ++gg) { beta[0][gg] = 0.f; beta[1][gg] = 0.f; }
+    for (int gg = 0; gg < NG; ++gg) { beta[0][gg] = 0.f; beta[1][gg] = 0.f; tau[gg] = 40; }
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) { O[mt][0] = O[mt][1] = O[mt][2] = O[mt][3] = 0.f; }
 
@@ -238,32 +397,58 @@ qsdpa_decode_kernel(const DecodeParams p) {
     const uint8_t* gVb = Q8 ? gVs : reinterpret_cast<const uint8_t*>(p.vb + row0 * NG);
     const int64_t L = p.L;
 
+    // copy plan: 16-byte unit i of a stage is row (i mod CU) / UPR of the K
+    // tile (i < CU) or of the V tile.  When CU is a multiple of the thread
+    // count every unit of a thread lies in a line with the same swizzle.
+    constexpr int CU = TK * C::UPR;
+    constexpr int NU = (2 * CU + kDecThreads - 1) / kDecThreads;
+    const int fx_tid = swz_line<C::SWZ>((tid >> 3) & 15);
+
     auto issue_stage = [&](int stage, int buf) {
-      uint8_t* sb = smem + buf * C::STAGE;
+      const uint32_t sbase = smem_u32(smem + buf * C::STAGE);
       const int64_t key0 = (int64_t)stage * TK;
-      constexpr int CU = TK * C::UPR;
-#pragma unroll 4
-      for (int i = tid; i < 2 * CU; i += kDecThreads) {
-        const int which = i >= CU;
-        const int j = which ? i - CU : i;
-        const int row = j / C::UPR, cu = j - row * C::UPR;
-        const int64_t key = key0 + row;
-        const uint8_t* base = which ? gV : gK;
-        const bool ok = key < L;
-        const uint8_t* src = ok ? base + key * C::RB + cu * 16 : base;
-        const int lin = row * C::RB + cu * 16;
-        cp_async16(smem_u32(sb + which * C::CODES + swz_offset<C::SWZ>(lin)), src, ok ? 16 : 0);
+      const int nvalid = (int)(L - key0 < (int64_t)TK ? L - key0 : (int64_t)TK);      // rows of this stage below L
+      const uint8_t* kb0 = gK + key0 * C::RB;
+      const uint8_t* vb0 = gV + key0 * C::RB;
+#pragma unroll
+      for (int k = 0; k < NU; ++k) {
+        const int i = tid + k * kDecThreads;
+        if ((2 * CU) % kDecThreads == 0 || i < 2 * CU) {
+          const int which = i >= CU, j = which ? i - CU : i;
+          const bool ok = (j / C::UPR) < nvalid;
+          const uint8_t* src = (which ? vb0 : kb0) + (ok ? j * 16 : 0);
+          const int dst = (CU % kDecThreads == 0) ? which * C::CODES + ((j * 16) ^ fx_tid)
+                                                  : which * C::CODES + swz_offset<C::SWZ>(j * 16);
+          cp_async16(sbase + dst, src, ok ? 16 : 0);
+        }
       }
       for (int i = tid; i < C::NMETA * C::META_UNITS; i += kDecThreads) {
         const int arr = i / C::META_UNITS, j = i - arr * C::META_UNITS;
         // affine: K scales, K biases, V scales, V biases; Q8_0: K scales, V scales
         const uint8_t* gm = Q8 ? (arr == 0 ? gKs : gVs)
                                : (arr == 0 ? gKs : arr == 1 ? gKb : arr == 2 ? gVs : gVb);
-        const int64_t kfirst = key0 + (j * 16) / C::MROW;
-        const bool ok = kfirst < L;
-        const uint8_t* src = ok ? gm + key0 * C::MROW + j * 16 : gm;
-        cp_async16(smem_u32(sb + 2 * C::CODES + arr * C::META + j * 16), src, ok ? 16 : 0);
+        const bool ok = (j * 16) / C::MROW < nvalid;
+        const uint8_t* src = gm + (ok ? key0 * C::MROW + j * 16 : 0);
+        cp_async16(sbase + 2 * C::CODES + arr * C::META + j * 16, src, ok ? 16 : 0);
       }
+    };
+
+    // fragment offsets inside a stage (fixed per lane).  The swizzle is
+    // linear in the line bits and a group never straddles a line, so it splits
+    // into a per-row part (computed once here), a per-group constant and, for
+    // the second 16-key block, the constant of a 16-row shift.
+    const int k0 = sub * 16 * C::SUB;
+    auto row_x = [&](int r) { return swz_line<C::SWZ>((r * C::RB) >> 7); };
+    const int xk0 = row_x(k0 + g), xk1 = row_x(k0 + g + 8);
+    const int xva = row_x(k0 + 2 * t), xvb = row_x(k0 + 2 * t + 1);
+    const int xvc = row_x(k0 + 2 * t + 8), xvd = row_x(k0 + 2 * t + 9);
+    auto koff = [&](int r, int x, int st, int G, int part) {
+      return ((r * C::RB + G * C::GB + t * C::NW * 4 + part * 16) ^ x) ^
+             swz_line<C::SWZ>((G * C::GB) >> 7) ^ swz_line<C::SWZ>((st * 16 * C::RB) >> 7);
+    };
+    auto voff = [&](int r, int x, int st, int G) {
+      return ((r * C::RB + G * C::GB + g * C::CB) ^ x) ^ swz_line<C::SWZ>((G * C::GB) >> 7) ^
+             swz_line<C::SWZ>((st * 16 * C::RB) >> 7);
     };
 
     const int nst = s1 - s0;
@@ -283,60 +468,45 @@ qsdpa_decode_kernel(const DecodeParams p) {
       }
       uint8_t* sb = smem + (it % NSTAGE) * C::STAGE;
       const int64_t key0 = (int64_t)(s0 + it) * TK;
-      if (key0 + TK > L) {
+      const int kvalid = (int)(L - key0 < (int64_t)TK ? L - key0 : (int64_t)TK);   // valid keys of this stage
+      if (kvalid < TK) {
         // keys past L: clear their (possibly stale) scales and biases
-        const int first_bad = (int)(L - key0);
         uint16_t* meta = reinterpret_cast<uint16_t*>(sb + 2 * C::CODES);
         for (int i = tid; i < C::NMETA * TK * NG; i += kDecThreads) {
           const int arr = i / (TK * NG), r = i - arr * TK * NG;
-          if (r / NG >= first_bad) meta[arr * (C::META / 2) + r] = 0;
+          if (r / NG >= kvalid) meta[arr * (C::META / 2) + r] = 0;
         }
         __syncthreads();
       }
-
-      const int k0 = sub * 16;
-      const int64_t kg0 = key0 + k0;
-      if (kg0 >= L) continue;                      // warp-uniform: whole block past L
+      if (k0 >= kvalid) continue;                  // warp-uniform: whole block past L
       const uint8_t* sK = sb;
       const uint8_t* sV = sb + C::CODES;
       const uint8_t* sMeta = sb + 2 * C::CODES;
 
-      // metadata of keys k0+g (row 0) and k0+g+8 (row 1)
-      uint16_t ks0[NG], ks1[NG], kb0[NG], kb1[NG], vs0[NG], vs1[NG], vb0[NG], vb1[NG];
-      {
-        const int r0 = k0 + g, r1 = r0 + 8;
-        if constexpr (Q8) {
-          lds_meta<NG>(sMeta + r0 * C::MROW, ks0);
-          lds_meta<NG>(sMeta + r1 * C::MROW, ks1);
-          lds_meta<NG>(sMeta + C::META + r0 * C::MROW, vs0);
-          lds_meta<NG>(sMeta + C::META + r1 * C::MROW, vs1);
-        } else {
-          lds_meta<NG>(sMeta + r0 * C::MROW, ks0);
-          lds_meta<NG>(sMeta + r1 * C::MROW, ks1);
-          lds_meta<NG>(sMeta + C::META + r0 * C::MROW, kb0);
-          lds_meta<NG>(sMeta + C::META + r1 * C::MROW, kb1);
-          lds_meta<NG>(sMeta + 2 * C::META + r0 * C::MROW, vs0);
-          lds_meta<NG>(sMeta + 2 * C::META + r1 * C::MROW, vs1);
-          lds_meta<NG>(sMeta + 3 * C::META + r0 * C::MROW, vb0);
-          lds_meta<NG>(sMeta + 3 * C::META + r1 * C::MROW, vb1);
+      // ---------------- scores S[block][key][row] (base-2 logits) -------------
+      float Sv[C::SUB][4];
+#pragma unroll
+      for (int st = 0; st < C::SUB; ++st) {
+        const int r0 = k0 + 16 * st + g, r1 = r0 + 8;
+        float* Sx = Sv[st];
+        Sx[0] = Sx[1] = Sx[2] = Sx[3] = 0.f;
+        uint32_t ks0[MW], ks1[MW], kb0[MW], kb1[MW];
+        meta_row<NG>(sMeta, r0, ks0);
+        meta_row<NG>(sMeta, r1, ks1);
+        if constexpr (!Q8) {
+          meta_row<NG>(sMeta + C::META, r0, kb0);
+          meta_row<NG>(sMeta + C::META, r1, kb1);
         }
-      }
-
-      // ---------------- scores S[key][head] (base-2 logits) ------------------
-      float S[4] = {0.f, 0.f, 0.f, 0.f};
-      {
-        const int r0 = k0 + g, r1 = r0 + 8;
         int s = 0;
 #pragma unroll
         for (int G = 0; G < NG; ++G) {
           float acc[4] = {0.f, 0.f, 0.f, 0.f};
           uint32_t w0[C::NW], w1[C::NW];
-          const int byte = G * C::GB + t * C::NW * 4;
 #pragma unroll
           for (int part = 0; part < (C::NW + 3) / 4; ++part) {
             constexpr int PW = C::NW < 4 ? C::NW : 4;
-            lds_words<PW>(sK + swz_offset<C::SWZ>(r0 * C::RB + byte + part * 16), w0 + part * 4);
-            lds_words<PW>(sK + swz_offset<C::SWZ>(r1 * C::RB + byte + part * 16), w1 + part * 4);
+            lds_words<PW>(sK + koff(r0, xk0, st, G, part), w0 + part * 4);
+            lds_words<PW>(sK + koff(r1, xk1, st, G, part), w1 + part * 4);
           }
 #pragma unroll
           for (int m = 0; m < C::NW; ++m) {
@@ -359,44 +529,48 @@ qsdpa_decode_kernel(const DecodeParams p) {
               ++s;
             }
           }
-          const float sk0 = half_bits_to_float(ks0[G]), sk1 = half_bits_to_float(ks1[G]);
-          const float bb0 = Q8 ? -128.f * sk0 : half_bits_to_float(kb0[G]);
-          const float bb1 = Q8 ? -128.f * sk1 : half_bits_to_float(kb1[G]);
+          const float sk0 = meta_f<NG>(ks0, G), sk1 = meta_f<NG>(ks1, G);
+          const float bb0 = Q8 ? -128.f * sk0 : meta_f<NG>(kb0, G);
+          const float bb1 = Q8 ? -128.f * sk1 : meta_f<NG>(kb1, G);
           const float c0 = sk0 * scaleK, c1 = sk1 * scaleK;
-          S[0] = fmaf(c0, acc[0], fmaf(bb0, qsc[G][0], S[0]));
-          S[1] = fmaf(c0, acc[1], fmaf(bb0, qsc[G][1], S[1]));
-          S[2] = fmaf(c1, acc[2], fmaf(bb1, qsc[G][0], S[2]));
-          S[3] = fmaf(c1, acc[3], fmaf(bb1, qsc[G][1], S[3]));
+          Sx[0] = fmaf(c0, acc[0], fmaf(bb0, qsc[G][0], Sx[0]));
+          Sx[1] = fmaf(c0, acc[1], fmaf(bb0, qsc[G][1], Sx[1]));
+          Sx[2] = fmaf(c1, acc[2], fmaf(bb1, qsc[G][0], Sx[2]));
+          Sx[3] = fmaf(c1, acc[3], fmaf(bb1, qsc[G][1], Sx[3]));
         }
-      }
-      if (kg0 + 16 > L) {
-        if (kg0 + g >= L) { S[0] = -INFINITY; S[1] = -INFINITY; }
-        if (kg0 + g + 8 >= L) { S[2] = -INFINITY; S[3] = -INFINITY; }
-      }
-      if (p.mask_kind != QKV_MASK_NONE) {
+        const int kr0 = 16 * st + k0 + g;                 // key index within the stage
+        if (kr0 >= kvalid) { Sx[0] = -INFINITY; Sx[1] = -INFINITY; }
+        if (kr0 + 8 >= kvalid) { Sx[2] = -INFINITY; Sx[3] = -INFINITY; }
+        if (p.mask_kind != QKV_MASK_NONE) {
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const int vh = hbase + chunk * 8 + 2 * t + j;     // row = head * Lq + query
-          if (vh < p.G) {
-            const int hr = vh / p.Lq, qi = vh - hr * p.Lq;
+          for (int j = 0; j < 2; ++j) {
+            const int vh = hbase + chunk * 8 + 2 * t + j;     // row = head * Lq + query
+            if (vh < p.G) {
+              const int hr = vh / p.Lq, qi = vh - hr * p.Lq;
 #pragma unroll
-            for (int r = 0; r < 2; ++r) {
-              const int64_t key = kg0 + g + 8 * r;
-              if (key >= L) continue;
-              if (p.mask_kind == QKV_MASK_CAUSAL) {
-                if (key > L - p.Lq + qi) S[2 * r + j] = -INFINITY;
-              } else {
-                const int64_t mi = (int64_t)b * p.msb + ((int64_t)hkv * p.Gq + hr) * p.msh +
-                                   (int64_t)qi * p.msq + key;
-                S[2 * r + j] += kLog2e * load_as_float(p.mask, p.mask_dtype, mi);
+              for (int r = 0; r < 2; ++r) {
+                const int64_t key = key0 + kr0 + 8 * r;
+                if (key >= L) continue;
+                if (p.mask_kind == QKV_MASK_CAUSAL) {
+                  if (key > L - p.Lq + qi) Sx[2 * r + j] = -INFINITY;
+                } else {
+                  const int64_t mi = (int64_t)b * p.msb + ((int64_t)hkv * p.Gq + hr) * p.msh +
+                                     (int64_t)qi * p.msq + key;
+                  Sx[2 * r + j] += kLog2e * load_as_float(p.mask, p.mask_dtype, mi);
+                }
               }
             }
           }
         }
       }
 
-      // ---------------- online softmax ----------------------------------------
-      float t0 = fmaxf(S[0], S[2]), t1 = fmaxf(S[1], S[3]);
+      // ---------------- online softmax over the warp's 32 keys -----------------
+      float t0 = -INFINITY, t1 = -INFINITY;
+#pragma unroll
+      for (int st = 0; st < C::SUB; ++st) {
+        t0 = fmaxf(t0, fmaxf(Sv[st][0], Sv[st][2]));
+        t1 = fmaxf(t1, fmaxf(Sv[st][1], Sv[st][3]));
+      }
 #pragma unroll
       for (int off = 4; off < 32; off <<= 1) {
         t0 = fmaxf(t0, __shfl_xor_sync(~0u, t0, off));
@@ -405,11 +579,18 @@ qsdpa_decode_kernel(const DecodeParams p) {
       const float n0 = fmaxf(m0, t0), n1 = fmaxf(m1, t1);
       const float u0 = n0 == -INFINITY ? 0.f : n0, u1 = n1 == -INFINITY ? 0.f : n1;
       const float al0 = ex2(m0 - u0), al1 = ex2(m1 - u1);
-      const float p0 = ex2(S[0] - u0), p1 = ex2(S[1] - u1);
-      const float p2 = ex2(S[2] - u0), p3 = ex2(S[3] - u1);
+      float P[C::SUB][4];
+#pragma unroll
+      for (int st = 0; st < C::SUB; ++st) {
+        P[st][0] = ex2(Sv[st][0] - u0); P[st][1] = ex2(Sv[st][1] - u1);
+        P[st][2] = ex2(Sv[st][2] - u0); P[st][3] = ex2(Sv[st][3] - u1);
+      }
       m0 = n0; m1 = n1;
-      l0 = fmaf(l0, al0, p0 + p2);
-      l1 = fmaf(l1, al1, p1 + p3);
+      float ps0 = 0.f, ps1 = 0.f;
+#pragma unroll
+      for (int st = 0; st < C::SUB; ++st) { ps0 += P[st][0] + P[st][2]; ps1 += P[st][1] + P[st][3]; }
+      l0 = fmaf(l0, al0, ps0);
+      l1 = fmaf(l1, al1, ps1);
       if (__any_sync(~0u, (al0 != 1.f) || (al1 != 1.f))) {
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt) {
@@ -418,99 +599,121 @@ qsdpa_decode_kernel(const DecodeParams p) {
 #pragma unroll
         for (int G = 0; G < NG; ++G) { beta[0][G] *= al0; beta[1][G] *= al1; }
       }
-      if constexpr (!Q8) {
-#pragma unroll
-        for (int G = 0; G < NG; ++G) {
-          const float vb0f = half_bits_to_float(vb0[G]), vb1f = half_bits_to_float(vb1[G]);
-          beta[0][G] = fmaf(p0, vb0f, fmaf(p2, vb1f, beta[0][G]));
-          beta[1][G] = fmaf(p1, vb0f, fmaf(p3, vb1f, beta[1][G]));
-        }
-      }
 
       // ---------------- values --------------------------------------------------
+      uint32_t vsw[C::SUB][2][MW], vbw[C::SUB][2][MW];
+#pragma unroll
+      for (int st = 0; st < C::SUB; ++st) {
+        const int r0 = k0 + 16 * st + g;
+        meta_row<NG>(sMeta + (Q8 ? 1 : 2) * C::META, r0, vsw[st][0]);
+        meta_row<NG>(sMeta + (Q8 ? 1 : 2) * C::META, r0 + 8, vsw[st][1]);
+        if constexpr (!Q8) {
+          meta_row<NG>(sMeta + 3 * C::META, r0, vbw[st][0]);
+          meta_row<NG>(sMeta + 3 * C::META, r0 + 8, vbw[st][1]);
+        }
+      }
 #pragma unroll
       for (int G = 0; G < NG; ++G) {
-        uint32_t mx = max((uint32_t)vs0[G], (uint32_t)vs1[G]);
+        if constexpr (!Q8) {
 #pragma unroll
-        for (int off = 4; off < 32; off <<= 1) mx = max(mx, __shfl_xor_sync(~0u, mx, off));
-        const int E = (int)((mx >> 10) & 31);
-        const int tau = mx == 0 ? 0 : 14 - (E == 0 ? -15 : E - 15);
-        const float up = exp2i(tau);
-        const float sv0 = half_bits_to_float(vs0[G]) * up, sv1 = half_bits_to_float(vs1[G]) * up;
-        const float x00 = p0 * sv0, x01 = p1 * sv0, x10 = p2 * sv1, x11 = p3 * sv1;
-        const uint32_t top = pack_half2(x00, x01), bot = pack_half2(x10, x11);
-        const uint32_t b0 = movmatrix_trans(top), b1 = movmatrix_trans(bot);
-        uint32_t b0l = 0, b1l = 0;
-        if constexpr (F32OUT) {
-          const float2 ft = unpack_half2(top), fb = unpack_half2(bot);
-          b0l = movmatrix_trans(pack_half2(x00 - ft.x, x01 - ft.y));
-          b1l = movmatrix_trans(pack_half2(x10 - fb.x, x11 - fb.y));
-        }
-        // codes of keys 2t, 2t+1, 2t+8, 2t+9 for this lane's chunk of group G
-        uint32_t wa[C::CW], wb[C::CW], wc[C::CW], wd[C::CW];
-        {
-          const int byte = G * C::GB + g * C::CB;
-          const int ra = k0 + 2 * t;
-          if constexpr (C::CB == 2) {
-            wa[0] = *reinterpret_cast<const uint16_t*>(sV + swz_offset<C::SWZ>(ra * C::RB + byte));
-            wb[0] = *reinterpret_cast<const uint16_t*>(sV + swz_offset<C::SWZ>((ra + 1) * C::RB + byte));
-            wc[0] = *reinterpret_cast<const uint16_t*>(sV + swz_offset<C::SWZ>((ra + 8) * C::RB + byte));
-            wd[0] = *reinterpret_cast<const uint16_t*>(sV + swz_offset<C::SWZ>((ra + 9) * C::RB + byte));
-          } else {
-            lds_words<C::CW>(sV + swz_offset<C::SWZ>(ra * C::RB + byte), wa);
-            lds_words<C::CW>(sV + swz_offset<C::SWZ>((ra + 1) * C::RB + byte), wb);
-            lds_words<C::CW>(sV + swz_offset<C::SWZ>((ra + 8) * C::RB + byte), wc);
-            lds_words<C::CW>(sV + swz_offset<C::SWZ>((ra + 9) * C::RB + byte), wd);
+          for (int st = 0; st < C::SUB; ++st) {
+            const float vb0f = meta_f<NG>(vbw[st][0], G), vb1f = meta_f<NG>(vbw[st][1], G);
+            beta[0][G] = fmaf(P[st][0], vb0f, fmaf(P[st][2], vb1f, beta[0][G]));
+            beta[1][G] = fmaf(P[st][1], vb0f, fmaf(P[st][3], vb1f, beta[1][G]));
           }
-          if constexpr (Q8) {
+        }
+        // keep P * s_v * 2^tau below 2^15: tau only ever decreases (O is
+        // rescaled by the exact power of two when it does)
+        uint32_t mxb = 0;
 #pragma unroll
-            for (int i = 0; i < C::CW; ++i) {
-              wa[i] ^= 0x80808080u; wb[i] ^= 0x80808080u; wc[i] ^= 0x80808080u; wd[i] ^= 0x80808080u;
+        for (int st = 0; st < C::SUB; ++st)
+          mxb = max(mxb, max(meta_bits<NG>(vsw[st][0], G), meta_bits<NG>(vsw[st][1], G)));
+        const int need = 29 - (int)((mxb >> 10) & 31);
+        if (__any_sync(~0u, need < tau[G])) {
+          int nt = need;
+#pragma unroll
+          for (int off = 1; off < 32; off <<= 1) nt = min(nt, __shfl_xor_sync(~0u, nt, off));
+          nt = min(nt, 29);
+          if (nt < tau[G]) {
+            const float f = exp2i(nt - tau[G]);
+#pragma unroll
+            for (int i = 0; i < KPG; ++i) {
+              O[G * KPG + i][0] *= f; O[G * KPG + i][1] *= f;
+              O[G * KPG + i][2] *= f; O[G * KPG + i][3] *= f;
             }
+            tau[G] = nt;
           }
         }
-        // fp32 factor undoing tau and the subnormal code scaling
-        const float f_lo = exp2i((Q8 ? 0 : 24) - tau);
-        const float f_hi = exp2i((Q8 ? 0 : (BITS == 4 ? 20 : 24)) - tau);
+        const float up = exp2i(tau[G]);
 #pragma unroll
-        for (int i = 0; i < KPG; ++i) {
-          uint32_t a[4];
-          if constexpr (BITS == 4) {
-            const int w = i >> 2;
-            const uint32_t sel = ((4u + (i & 3)) << 8) | (uint32_t)(i & 3);
-            const uint32_t xv = prmt(wa[w], wb[w], sel), yv = prmt(wc[w], wd[w], sel);
-            a[0] = xv & 0x000F000Fu; a[1] = xv & 0x00F000F0u;
-            a[2] = yv & 0x000F000Fu; a[3] = yv & 0x00F000F0u;
-          } else {
-            const int w = i >> 1;
-            const uint32_t mA = wa[w] & 0x00FF00FFu, mB = wb[w] & 0x00FF00FFu;
-            const uint32_t nA = wa[w] & 0xFF00FF00u, nB = wb[w] & 0xFF00FF00u;
-            const uint32_t mC = wc[w] & 0x00FF00FFu, mD = wd[w] & 0x00FF00FFu;
-            const uint32_t nC2 = wc[w] & 0xFF00FF00u, nD = wd[w] & 0xFF00FF00u;
-            const uint32_t selm = (i & 1) ? 0x7632u : 0x5410u;
-            const uint32_t seln = (i & 1) ? 0x6723u : 0x4501u;
-            a[0] = prmt(mA, mB, selm); a[1] = prmt(nA, nB, seln);
-            a[2] = prmt(mC, mD, selm); a[3] = prmt(nC2, nD, seln);
+        for (int st = 0; st < C::SUB; ++st) {
+          const float sv0 = meta_f<NG>(vsw[st][0], G) * up, sv1 = meta_f<NG>(vsw[st][1], G) * up;
+          const float x00 = P[st][0] * sv0, x01 = P[st][1] * sv0;
+          const float x10 = P[st][2] * sv1, x11 = P[st][3] * sv1;
+          const uint32_t top = pack_half2(x00, x01), bot = pack_half2(x10, x11);
+          const uint32_t b0 = movmatrix_trans(top), b1 = movmatrix_trans(bot);
+          uint32_t b0l = 0, b1l = 0;
+          if constexpr (F32OUT) {
+            const float2 ft = unpack_half2(top), fb = unpack_half2(bot);
+            b0l = movmatrix_trans(pack_half2(x00 - ft.x, x01 - ft.y));
+            b1l = movmatrix_trans(pack_half2(x10 - fb.x, x11 - fb.y));
+          }
+          // codes of keys 2t, 2t+1, 2t+8, 2t+9 (of this block) for this lane's chunk
+          uint32_t wa[C::CW], wb[C::CW], wc[C::CW], wd[C::CW];
+          {
+            const int ra = k0 + 16 * st + 2 * t;
+            if constexpr (C::CB == 2) {
+              wa[0] = *reinterpret_cast<const uint16_t*>(sV + voff(ra, xva, st, G));
+              wb[0] = *reinterpret_cast<const uint16_t*>(sV + voff(ra + 1, xvb, st, G));
+              wc[0] = *reinterpret_cast<const uint16_t*>(sV + voff(ra + 8, xvc, st, G));
+              wd[0] = *reinterpret_cast<const uint16_t*>(sV + voff(ra + 9, xvd, st, G));
+            } else {
+              lds_words<C::CW>(sV + voff(ra, xva, st, G), wa);
+              lds_words<C::CW>(sV + voff(ra + 1, xvb, st, G), wb);
+              lds_words<C::CW>(sV + voff(ra + 8, xvc, st, G), wc);
+              lds_words<C::CW>(sV + voff(ra + 9, xvd, st, G), wd);
+            }
             if constexpr (Q8) {
-              // exact signed codes: (1024 + u) - 1152 with u = code + 128
-              const __half2 off = __float2half2_rn(1152.f);
 #pragma unroll
-              for (int r = 0; r < 4; ++r) {
-                uint32_t v = a[r] | 0x64006400u;
-                __half2 hv = __hsub2(*reinterpret_cast<__half2*>(&v), off);
-                a[r] = *reinterpret_cast<uint32_t*>(&hv);
+              for (int i = 0; i < C::CW; ++i) {
+                wa[i] ^= 0x80808080u; wb[i] ^= 0x80808080u; wc[i] ^= 0x80808080u; wd[i] ^= 0x80808080u;
               }
             }
           }
-          float d[4];
-          const float z[4] = {0.f, 0.f, 0.f, 0.f};
-          mma_f16(d, a, b0, b1, z);
-          if constexpr (F32OUT) mma_f16(d, a, b0l, b1l, d);
-          const int mt = G * KPG + i;
-          O[mt][0] = fmaf(d[0], f_lo, O[mt][0]);
-          O[mt][1] = fmaf(d[1], f_lo, O[mt][1]);
-          O[mt][2] = fmaf(d[2], f_hi, O[mt][2]);
-          O[mt][3] = fmaf(d[3], f_hi, O[mt][3]);
+#pragma unroll
+          for (int i = 0; i < KPG; ++i) {
+            uint32_t a[4];
+            if constexpr (BITS == 4) {
+              const int w = i >> 2;
+              const uint32_t sel = ((4u + (i & 3)) << 8) | (uint32_t)(i & 3);
+              const uint32_t xv = prmt(wa[w], wb[w], sel), yv = prmt(wc[w], wd[w], sel);
+              a[0] = xv & 0x000F000Fu; a[1] = xv & 0x00F000F0u;
+              a[2] = yv & 0x000F000Fu; a[3] = yv & 0x00F000F0u;
+            } else {
+              const int w = i >> 1;
+              const uint32_t mA = wa[w] & 0x00FF00FFu, mB = wb[w] & 0x00FF00FFu;
+              const uint32_t nA = wa[w] & 0xFF00FF00u, nB = wb[w] & 0xFF00FF00u;
+              const uint32_t mC = wc[w] & 0x00FF00FFu, mD = wd[w] & 0x00FF00FFu;
+              const uint32_t nC2 = wc[w] & 0xFF00FF00u, nD = wd[w] & 0xFF00FF00u;
+              const uint32_t selm = (i & 1) ? 0x7632u : 0x5410u;
+              const uint32_t seln = (i & 1) ? 0x6723u : 0x4501u;
+              a[0] = prmt(mA, mB, selm); a[1] = prmt(nA, nB, seln);
+              a[2] = prmt(mC, mD, selm); a[3] = prmt(nC2, nD, seln);
+              if constexpr (Q8) {
+                // exact signed codes: (1024 + u) - 1152 with u = code + 128
+                const __half2 off = __float2half2_rn(1152.f);
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                  uint32_t v = a[r] | 0x64006400u;
+                  __half2 hv = __hsub2(*reinterpret_cast<__half2*>(&v), off);
+                  a[r] = *reinterpret_cast<uint32_t*>(&hv);
+                }
+              }
+            }
+            const int mt = G * KPG + i;
+            mma_f16(O[mt], a, b0, b1, O[mt]);
+            if constexpr (F32OUT) mma_f16(O[mt], a, b0l, b1l, O[mt]);
+          }
         }
       }
     }
@@ -533,10 +736,14 @@ qsdpa_decode_kernel(const DecodeParams p) {
     for (int mt = 0; mt < MT; ++mt) {
       const int G = mt / KPG, i = mt % KPG;
       const int e = G * GS + g * (GS / 8) + 2 * i;
-      ws[(2 * t) * D + e] = O[mt][0] + beta[0][G];
-      ws[(2 * t + 1) * D + e] = O[mt][1] + beta[1][G];
-      ws[(2 * t) * D + e + 1] = O[mt][2] + beta[0][G];
-      ws[(2 * t + 1) * D + e + 1] = O[mt][3] + beta[1][G];
+      // rows g hold code*2^-24 (Q8_0: exact codes), rows g+8 code*2^-20 for
+      // 4-bit; O of group G carries an extra 2^tau
+      const float f_lo = exp2i((Q8 ? 0 : 24) - tau[G]);
+      const float f_hi = exp2i((Q8 ? 0 : (BITS == 4 ? 20 : 24)) - tau[G]);
+      ws[(2 * t) * D + e] = fmaf(O[mt][0], f_lo, beta[0][G]);
+      ws[(2 * t + 1) * D + e] = fmaf(O[mt][1], f_lo, beta[1][G]);
+      ws[(2 * t) * D + e + 1] = fmaf(O[mt][2], f_hi, beta[0][G]);
+      ws[(2 * t + 1) * D + e + 1] = fmaf(O[mt][3], f_hi, beta[1][G]);
     }
     if (g == 0) {
       ws[8 * D + 2 * t] = m0; ws[8 * D + 2 * t + 1] = m1;
@@ -580,43 +787,68 @@ qsdpa_decode_kernel(const DecodeParams p) {
     }
 
     if (!complete) {
-      // last CTA of this unit to arrive merges all partial results
+      // Merge tree without waiting: the last CTA of each group of kMergeGroup
+      // consecutive parts merges that group into a level-2 partial; the last
+      // group merger of the unit merges the level-2 partials into the output.
+      // (With at most kMergeGroup parts the first level writes the output.)
       __threadfence();
       __syncthreads();
       const int64_t cfirst = ((u * S + 1) * nC - 1) / T;
       const int64_t clast = (((u + 1) * S) * nC - 1) / T;
-      if (tid == 0) {
-        const unsigned nparts = (unsigned)(clast - cfirst + 1);
-        const unsigned prev = atomicAdd(&p.tickets[u], 1u);
-        const int last = prev == nparts - 1;
-        if (last) p.tickets[u] = 0u;
-        s_flag = last;
-      }
-      __syncthreads();
-      if (s_flag) {
-        __threadfence();
-        for (int idx = tid; idx < HPC * D; idx += kDecThreads) {
-          const int hl = idx / D, e = idx - hl * D;
-          const int head = hbase + hl;
-          if (head >= p.G) continue;
-          float M = -INFINITY, l = 0.f, o = 0.f;
-          for (int64_t c = cfirst; c <= clast; ++c) {
-            const int64_t clo = c * T / nC;
-            const int64_t sl = 2 * c + ((clo / S) == u ? 0 : 1);
-            const float mp = __ldcg(&p.part_ml[(sl * HPC + hl) * 2 + 0]);
-            if (mp == -INFINITY) continue;
-            const float lp = __ldcg(&p.part_ml[(sl * HPC + hl) * 2 + 1]);
-            const float op = __ldcg(&p.part_o[(sl * HPC + hl) * D + e]);
-            if (mp > M) {
-              const float sc = ex2(M - mp);     // M = -inf -> 0
-              o *= sc; l *= sc; M = mp;
-            }
-            const float sc = ex2(mp - M);
-            o = fmaf(sc, op, o);
-            l = fmaf(sc, lp, l);
+      const int nparts = (int)(clast - cfirst + 1);
+      const int ngroups = (nparts + kMergeGroup - 1) / kMergeGroup;
+      const int pi = (int)((int64_t)blockIdx.x - cfirst);
+      const int gi = pi / kMergeGroup;
+      auto slot_of = [&](int64_t c) {      // level-1 slot of CTA c for unit u
+        return 2 * c + (((c * T / nC) / S) == u ? 0 : 1);
+      };
+      float* sm = reinterpret_cast<float*>(smem) + kDecWarps * (8 * D + 16);
+      if (ngroups == 1) {
+        if (tid == 0) {
+          const unsigned prev = atomicAdd(&p.tickets[u], 1u);
+          const int last = prev == (unsigned)nparts - 1;
+          if (last) p.tickets[u] = 0u;
+          s_flag = last;
+        }
+        __syncthreads();
+        if (s_flag) {
+          __threadfence();
+          merge_parts<D, HPC>(p.part_ml, p.part_o, nparts, [&](int i) { return slot_of(cfirst + i); },
+                              sm, tid, hbase, p.G, nullptr, nullptr,
+                              p.out, p.out_dtype, (((int64_t)b * p.Hkv + hkv) * p.G) * D);
+        }
+      } else {
+        const int64_t lead = slot_of(cfirst + (int64_t)gi * kMergeGroup);   // group's id
+        const int gsz = min(kMergeGroup, nparts - gi * kMergeGroup);
+        if (tid == 0) {
+          const unsigned prev = atomicAdd(&p.tickets1[lead], 1u);
+          const int last = prev == (unsigned)gsz - 1;
+          if (last) p.tickets1[lead] = 0u;
+          s_flag = last;
+        }
+        __syncthreads();
+        if (s_flag) {
+          __threadfence();
+          const int64_t c0 = cfirst + (int64_t)gi * kMergeGroup;
+          merge_parts<D, HPC>(p.part_ml, p.part_o, gsz, [&](int i) { return slot_of(c0 + i); },
+                              sm, tid, hbase, p.G, p.part2_ml + lead * HPC * 2,
+                              p.part2_o + lead * HPC * D, nullptr, 0, 0);
+          __threadfence();
+          __syncthreads();
+          if (tid == 0) {
+            const unsigned prev = atomicAdd(&p.tickets[u], 1u);
+            const int last = prev == (unsigned)ngroups - 1;
+            if (last) p.tickets[u] = 0u;
+            s_flag = last;
           }
-          const int64_t oi = (((int64_t)b * p.Hkv + hkv) * p.G + head) * D + e;
-          store_from_float(p.out, p.out_dtype, oi, l > 0.f ? o / l : 0.f);
+          __syncthreads();
+          if (s_flag) {
+            __threadfence();
+            merge_parts<D, HPC>(p.part2_ml, p.part2_o, ngroups,
+                                [&](int i) { return slot_of(cfirst + (int64_t)i * kMergeGroup); },
+                                sm, tid, hbase, p.G, nullptr, nullptr,
+                                p.out, p.out_dtype, (((int64_t)b * p.Hkv + hkv) * p.G) * D);
+          }
         }
       }
     }

@@ -8,11 +8,11 @@ namespace qkv {
 namespace {
 
 // Grid cap per SM used both for planning and for the workspace bound, so that
-// qsdpa_workspace_size() does not depend on the kernel instance.
-constexpr int kMaxCtasPerSm = 2;
-// Upper bound on the bytes of partial results one CTA merges at the end of a
-// unit (the merge is done by a single CTA).
-constexpr double kMergeBytesPerUnit = 160.0 * 1024.0;
+// qsdpa_workspace_size() does not depend on the kernel instance: the D <= 128
+// kernels are built for two resident CTAs per SM, the D = 256 ones for one.
+int max_ctas_per_sm(int D) { return D <= 128 ? 2 : 1; }
+// Largest grid: the merge tree's second level then has at most 48 groups of 8.
+constexpr int64_t kMaxGrid = 8 * 48;
 
 int sm_count() {
   int dev = 0, n = 0;
@@ -31,6 +31,10 @@ bool get_ops(int D, int bits, int gs, int fmt, int nc, bool f32, DecodeOps* ops)
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+size_t max_grid(int D) {
+  return (size_t)std::min<int64_t>((int64_t)std::max(1, sm_count()) * max_ctas_per_sm(D), kMaxGrid);
+}
+
 }  // namespace
 
 void decode_chunking(int G, int* nc, int* ncg) {
@@ -39,22 +43,32 @@ void decode_chunking(int G, int* nc, int* ncg) {
   *ncg = (chunks + *nc - 1) / *nc;
 }
 
+// Workspace layout: [unit tickets][group tickets] (both zero between calls),
+// then per-CTA partials (o, then (m, l)), then per-group partials.
+void decode_ws_layout(size_t units, size_t hpc, int D, size_t maxgrid, DecodePlan* plan) {
+  plan->ws_tickets2 = round_up(units * 4, 256);
+  plan->ws_tickets = plan->ws_tickets2 + round_up(2 * maxgrid * 4, 256);
+  plan->ws_part_o = round_up(2 * maxgrid * hpc * D * 4, 256);
+  plan->ws_part_ml = round_up(2 * maxgrid * hpc * 2 * 4, 256);
+  plan->ws_total = plan->ws_tickets + 2 * (plan->ws_part_o + plan->ws_part_ml);
+}
+
 size_t decode_workspace_bound(int B, int Hq, int Hkv, int D) {
   if (B <= 0 || Hkv <= 0 || Hq % Hkv) return 0;
   int nc, ncg;
   decode_chunking(Hq / Hkv, &nc, &ncg);
-  const size_t units = (size_t)B * Hkv * ncg;
-  const size_t grid = (size_t)std::max(1, sm_count()) * kMaxCtasPerSm;
-  const size_t hpc = (size_t)nc * 8;
-  return round_up(units * 4, 256) + round_up(2 * grid * hpc * D * 4, 256) +
-         round_up(2 * grid * hpc * 2 * 4, 256);
+  DecodePlan plan;
+  decode_ws_layout((size_t)B * Hkv * ncg, (size_t)nc * 8, D, max_grid(D), &plan);
+  return plan.ws_total;
 }
 
 size_t decode_workspace_zero_bytes(int B, int Hq, int Hkv) {
   if (B <= 0 || Hkv <= 0 || Hq % Hkv) return 0;
   int nc, ncg;
   decode_chunking(Hq / Hkv, &nc, &ncg);
-  return round_up((size_t)B * Hkv * ncg * 4, 256);
+  DecodePlan plan;
+  decode_ws_layout((size_t)B * Hkv * ncg, (size_t)nc * 8, 64, max_grid(128), &plan);
+  return plan.ws_tickets;
 }
 
 bool plan_decode(int D, int bits, int gs, int fmt, int out_f32, int B, int Hq, int Hkv,
@@ -64,7 +78,7 @@ bool plan_decode(int D, int bits, int gs, int fmt, int out_f32, int B, int Hq, i
   DecodeOps ops;
   if (!get_ops(D, bits, gs, fmt, nc, out_f32 != 0, &ops)) return false;
   const int sms = std::max(1, sm_count());
-  const int occ = std::min(kMaxCtasPerSm, std::max(1, ops.occupancy()));
+  const int occ = std::min(max_ctas_per_sm(D), std::max(1, ops.occupancy()));
   plan->tk = ops.tk;
   plan->nc = nc;
   plan->hpc = nc * 8;
@@ -72,20 +86,13 @@ bool plan_decode(int D, int bits, int gs, int fmt, int out_f32, int B, int Hq, i
   plan->units = (int64_t)B * Hkv * ncg;
   plan->stages_per_unit = (L + ops.tk - 1) / ops.tk;
   plan->total_stages = plan->units * plan->stages_per_unit;
-  // One CTA per (SM x resident slot), but no more CTAs per unit than keeps the
-  // final merge of a unit's partial results small.
-  const double part_bytes = (double)plan->hpc * D * 4.0;
-  const int64_t max_parts = std::max<int64_t>(1, (int64_t)(kMergeBytesPerUnit / part_bytes));
+  // one CTA per (SM x resident slot), each a contiguous equal share of stages
   int64_t grid = (int64_t)sms * occ;
-  grid = std::min<int64_t>(grid, plan->units * max_parts);
   grid = std::min<int64_t>(grid, plan->total_stages);
+  grid = std::min<int64_t>(grid, kMaxGrid);            // merge scratch holds <= 48 groups
   plan->grid = (int)std::max<int64_t>(1, grid);
   plan->smem = ops.smem;
-  plan->ws_tickets = round_up((size_t)plan->units * 4, 256);
-  const size_t maxgrid = (size_t)sms * kMaxCtasPerSm;
-  plan->ws_part_o = round_up(2 * maxgrid * plan->hpc * D * 4, 256);
-  plan->ws_part_ml = round_up(2 * maxgrid * plan->hpc * 2 * 4, 256);
-  plan->ws_total = plan->ws_tickets + plan->ws_part_o + plan->ws_part_ml;
+  decode_ws_layout((size_t)plan->units, (size_t)plan->hpc, D, max_grid(D), plan);
   return true;
 }
 

@@ -39,9 +39,12 @@ struct DecodeParams {
   // evenly over gridDim.x CTAs
   int64_t stages_per_unit;
   int64_t total_stages;
-  float* part_o;            // [2 * nCTA][HPC][D]
+  float* part_o;            // [2 * nCTA][HPC][D]   per-CTA partials
   float* part_ml;           // [2 * nCTA][HPC][2]
+  float* part2_o;           // [2 * nCTA][HPC][D]   per-group partials (merge tree)
+  float* part2_ml;          // [2 * nCTA][HPC][2]
   unsigned* tickets;        // [units], zero between calls
+  unsigned* tickets1;       // [2 * nCTA], zero between calls
 };
 
 struct DecodePlan {
@@ -54,8 +57,9 @@ struct DecodePlan {
   int64_t total_stages;
   int grid;
   size_t smem;
-  size_t ws_tickets;        // bytes (zeroed region)
-  size_t ws_part_o;         // bytes
+  size_t ws_tickets;        // bytes (zeroed region: unit tickets + group tickets)
+  size_t ws_tickets2;       // offset of the group tickets inside the zeroed region
+  size_t ws_part_o;         // bytes of one partial array
   size_t ws_part_ml;        // bytes
   size_t ws_total;
 };

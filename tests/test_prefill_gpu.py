@@ -1,0 +1,101 @@
+"""GPU parity of qsdpa_prefill (multi-query attention) against the oracle.
+Calls with >= 64 (head, query) rows per kv head and 16-bit output run on the
+tcgen05 kernel; smaller ones and fp32 output on the split-K kernel.  Both are
+covered here."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from helpers import TOL, TORCH_DT, cache_to_dev, from_dev, make_problem, max_err, out_err, to_dev
+from quantized_kv_attention_split_b200 import synthetic as S
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def qkv():
+    from quantized_kv_attention_split_b200 import qkv as m
+    m.lib()
+    return m
+
+
+def run_prefill(qkv, q, q_dtype, kc, vc, L, scale, out_dtype, causal=False, mask=None):
+    out = qkv.qsdpa_prefill(to_dev(q, q_dtype), cache_to_dev(kc), cache_to_dev(vc), L, scale,
+                            mask=mask, causal=causal, out_dtype=TORCH_DT[out_dtype])
+    torch.cuda.synchronize()
+    return from_dev(out)
+
+
+CASES = [
+    # B, Hq, Hkv, Lq, D, L, fmt, bits, gs   (rows per kv head = Hq/Hkv * Lq)
+    (1, 8, 2, 32, 128, 300, "q8_0", 8, 32),       # 128 rows, tcgen05
+    (1, 32, 2, 16, 256, 700, "q8_0", 8, 32),      # 256 rows, tcgen05
+    (2, 4, 1, 40, 64, 333, "affine", 4, 64),      # 160 rows (ragged tile)
+    (1, 8, 2, 20, 128, 257, "affine", 8, 64),     # 80 rows
+    (1, 2, 1, 100, 256, 511, "affine", 4, 32),
+    (1, 6, 3, 64, 128, 129, "affine", 4, 128),
+    (1, 4, 1, 8, 128, 200, "affine", 4, 64),      # 32 rows: split-K path
+    (1, 4, 4, 3, 64, 90, "q8_0", 8, 32),          # 3 rows: split-K path
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "-".join(map(str, c)))
+@pytest.mark.parametrize("causal", [False, True])
+def test_prefill_matches_oracle(qkv, case, causal):
+    B, Hq, Hkv, Lq, D, L, fmt, bits, gs = case
+    q, kc, vc = make_problem(B, Hq, Hkv, Lq, D, L, fmt, bits, gs, "normal", q_dtype="bf16",
+                             Lcap=(L // 8 + 3) * 8, seed=5)
+    scale = 1.0 / np.sqrt(D)
+    mask = oracle.Mask("causal") if causal else None
+    ref = oracle.attention(q, "bf16", kc, vc, L, scale, mask=mask)
+    got = run_prefill(qkv, q, "bf16", kc, vc, L, scale, "bf16", causal=causal)
+    assert out_err(got, ref, "bf16") <= 1.0, (max_err(got, ref), out_err(got, ref, "bf16"))
+    got = run_prefill(qkv, q, "bf16", kc, vc, L, scale, "f16", causal=causal)
+    assert max_err(got, ref) <= TOL["f16"], max_err(got, ref)
+    got = run_prefill(qkv, q, "bf16", kc, vc, L, scale, "f32", causal=causal)
+    assert max_err(got, ref) <= TOL["f32"], max_err(got, ref)
+
+
+def test_prefill_additive_mask_and_fp16(qkv):
+    B, Hq, Hkv, Lq, D, L = 1, 16, 2, 16, 128, 400
+    q, kc, vc = make_problem(B, Hq, Hkv, Lq, D, L, "affine", 8, 32, "normal", seed=8)
+    rng = np.random.default_rng(2)
+    m = rng.standard_normal((B, Hq, Lq, L)).astype(np.float32)
+    m[0, 3, 5, :] = -np.inf                       # a fully masked row
+    m[0, 7, :, 100:300] = -np.inf
+    st = (Hq * Lq * L, Lq * L, L)
+    ref = oracle.attention(q, "f16", kc, vc, L, 0.05, mask=oracle.Mask("additive", m, "f32", st))
+    got = run_prefill(qkv, q, "f16", kc, vc, L, 0.05, "f16", mask=torch.from_numpy(m).cuda())
+    assert np.all(got[0, 3, 5] == 0)
+    assert max_err(got, ref) <= TOL["f16"]
+
+
+def test_prefill_lq_greater_than_l_causal(qkv):
+    """Queries before the first key see nothing and return zeros."""
+    B, Hq, Hkv, Lq, D, L = 1, 8, 1, 40, 64, 24
+    q, kc, vc = make_problem(B, Hq, Hkv, Lq, D, L, "q8_0", 8, 32, "normal", seed=9)
+    ref = oracle.attention(q, "f16", kc, vc, L, 0.125, mask=oracle.Mask("causal"))
+    got = run_prefill(qkv, q, "f16", kc, vc, L, 0.125, "f16", causal=True)
+    assert np.all(got[:, :, :Lq - L] == 0)
+    assert max_err(got, ref) <= TOL["f16"]
+
+
+def test_prefill_q8_0_512_at_20k_sampled(qkv):
+    """The 512-query Q8_0 prompt at depth 20480 (Lk = 20992, causal over the
+    last 512), full size, launched as the benchmark launches it; the oracle
+    checks a sample of rows spread over heads and queries."""
+    w = S.WORKLOADS["prefill_q8_0_512_at_20k"]
+    inp = S.make_inputs(w)
+    kc = oracle.quantize(inp.k, w.kv_dtype, "q8_0")
+    vc = oracle.quantize(inp.v, w.kv_dtype, "q8_0")
+    got = run_prefill(qkv, inp.q, w.q_dtype, kc, vc, w.L, w.scale, w.out_dtype, causal=True)
+    rng = np.random.default_rng(0)
+    rows = np.unique(np.concatenate([rng.integers(0, w.Hq * w.Lq, 96),
+                                     [0, w.Lq - 1, w.Hq * w.Lq - 1]]))
+    ref = oracle.attention(inp.q, w.q_dtype, kc, vc, w.L, w.scale, mask=oracle.Mask("causal"),
+                           rows=rows)
+    g = got.reshape(-1, w.D)[rows]
+    r = ref.reshape(-1, w.D)[rows]
+    assert max_err(g, r) <= TOL["bf16"], max_err(g, r)
+    assert out_err(g, r, "bf16") <= 1.0
