@@ -7,25 +7,31 @@
 // one fused pass per tile, for the KV formats of the decode kernel.  The
 // dequantize-tiles-to-16-bit-then-MMA pattern follows the MLX CUDA work-in-
 // progress page (SharedTile::load_quantized feeding the tensor cores); the
-// 5th-generation MMA, TMEM, the warp roles and the layouts are this kernel's.
+// 5th-generation MMA, TMEM residency, the warp roles and the layouts are this
+// kernel's.
 //
 // One CTA owns 128 rows (TMEM lanes) of one kv head; a row is a (query, head)
 // pair, r = query * G + head, so the G heads that share a KV head share every
 // dequantized K/V tile and a tile's rows span few query positions (tight
-// causal bound).  Three warp roles work on 32-key tiles, double-buffered:
-//   * dequant warps (4): cp.async the packed codes and scales of tile t+2 into
-//     a two-slot ring while dequantizing tile t into fp16 K [key][d] and
-//     V [d][key] in the tensor core's K-major swizzled layouts;
-//   * MMA warp (1): S(t) = Q K(t)^T into TMEM (M=128, N=32, K=16 per op), and
-//     once the softmax warps hand over P(t-1), O += P(t-1) V(t-1) (M=128,
-//     N=D); completion is signalled with tcgen05.commit on mbarriers;
-//   * softmax warps (4, one TMEM lane = one row per thread): scale and mask
-//     S, online softmax with a lazily moved maximum (moved only when it grows
-//     by more than 2^8, so the O accumulator in TMEM is rarely rescaled), P as
-//     fp16 into shared memory; finally O / l to the output.
+// causal bound).  Work goes in 32-key tiles through three warp roles:
+//   * dequant warps (8): one thread issues bulk copies (cp.async.bulk, one per
+//     contiguous array) of the packed codes and scales of a tile into a
+//     three-slot ring; all of them turn tile t into fp16 K and V, both stored
+//     [key][d] with 128-byte swizzled rows (K is the K-major B operand of
+//     S = Q K^T, V the MN-major B operand of O += P V), two K slots and three
+//     V slots so dequantization runs ahead of the tensor cores;
+//   * MMA warp (1): S(t) = Q K(t)^T and O += P(t-1) V(t-1) with Q and P read
+//     from TMEM (the A operand), so shared memory only streams K and V;
+//     completion is signalled with tcgen05.commit on mbarriers;
+//   * softmax warps (4, one TMEM lane = one row per thread): stage the
+//     prescaled Q into TMEM, then per tile: scale and mask S, online softmax
+//     with a lazily moved maximum (moved only when it grows by more than 2^8,
+//     so O in TMEM is rarely rescaled), P as fp16 into TMEM; finally O / l to
+//     the output.
 // Every mbarrier wait is bounded: a time-out records an error in the status
 // word and makes every later wait return at once, so all roles finish the
-// tile loop, release TMEM and return.
+// tile loop; before exit the CTA waits (bounded) for its own bulk copies and
+// tensor-core work in flight, then releases TMEM.
 #pragma once
 
 #include "qkv_common.cuh"
@@ -36,9 +42,13 @@ namespace qkv {
 constexpr int kPfBM = 128;        // rows per CTA
 constexpr int kPfBN = 32;         // keys per tile
 constexpr int kPfSoftWarps = 4;
-constexpr int kPfDqWarps = 4;
+constexpr int kPfDqWarps = 8;
+constexpr int kPfDqThreads = 32 * kPfDqWarps;
 constexpr int kPfMmaWarp = kPfSoftWarps + kPfDqWarps;
 constexpr int kPfThreads = 32 * (kPfMmaWarp + 1);
+constexpr int kPfKSlots = 2;      // fp16 K tiles (slot free once S of the tile is done)
+constexpr int kPfVSlots = 3;      // fp16 V tiles (slot free once P V of the tile is done)
+constexpr int kPfRawSlots = 3;    // packed tiles in flight
 constexpr unsigned kPfWaitLimit = 1u << 21;   // try_wait rounds (<= 1 us each) before giving up
 
 struct PrefillParams {
@@ -63,33 +73,50 @@ struct PrefillParams {
   unsigned* status;         // nonzero after a tensor-core wait timed out
 };
 
+// Lane -> chunk map of the dequant warps (a GF(2)-linear map given by the
+// chunk offset each lane bit adds), chosen per layout so that each 8-lane
+// phase of the 16-byte packed-tile reads and of the 16-byte swizzled fp16
+// writes touches eight different bank groups.
+__host__ __device__ constexpr int pf_lane_col(int D, int bits, int b) {
+  return (D == 128 && bits == 4 && b == 1) ? 10
+       : (D == 128 && bits == 8 && b == 2) ? 12
+       : (D == 256 && bits == 4 && b == 1) ? 10
+       : (D == 256 && bits == 4 && b == 2) ? 20
+       : (D == 256 && bits == 8 && b == 2) ? 20
+       : (1 << b);
+}
+
 template <int D, int BITS, int GS, bool Q8>
 struct PfCfg {
   static constexpr int RB = D * BITS / 8;            // bytes per code row
-  static constexpr int UPR = RB / 16;
+  static constexpr int UPR = RB / 16;                // 16-byte chunks per code row
+  static constexpr int CPC = 128 / BITS;             // codes per 16-byte chunk
   static constexpr int NG = D / GS;
-  static constexpr int NMETA = Q8 ? 2 : 4;
+  static constexpr int NMETA = Q8 ? 2 : 4;           // scale (and bias) arrays of K and V
   static constexpr int META_BYTES = ((kPfBN * NG * 2 + 127) / 128) * 128;
-  // operands (1024-byte aligned): Q, K[2], V[2], P[2]
-  static constexpr int Q_OFF = 0;
-  static constexpr int Q_BYTES = kPfBM * D * 2;      // SW128: D/64 blocks of [128][64]
-  static constexpr int K_BYTES = kPfBN * D * 2;      // SW128: D/64 blocks of [32][64]
-  static constexpr int K_OFF = Q_OFF + Q_BYTES;
-  static constexpr int V_BYTES = D * kPfBN * 2;      // SW64: [D][32]
-  static constexpr int V_OFF = K_OFF + 2 * K_BYTES;
-  static constexpr int P_BYTES = kPfBM * kPfBN * 2;  // SW64: [128][32]
-  static constexpr int P_OFF = V_OFF + 2 * V_BYTES;
-  // raw ring slots: K codes, V codes, metadata arrays
-  static constexpr int RAW_BYTES = 2 * kPfBN * RB + NMETA * META_BYTES;
-  static constexpr int RAW_OFF = P_OFF + 2 * P_BYTES;
-  static constexpr int BAR_OFF = RAW_OFF + 2 * RAW_BYTES;
-  static constexpr int SMEM = BAR_OFF + 128 + 1024;  // + barriers, TMEM slot, alignment slack
-  static constexpr int TMEM_COLS = D + 2 * kPfBN <= 128 ? 128 : (D + 2 * kPfBN <= 256 ? 256 : 512);
-  static_assert(D + 2 * kPfBN <= TMEM_COLS, "TMEM budget");
+  // shared memory (1024-byte aligned operand slots)
+  static constexpr int KV_BYTES = kPfBN * D * 2;     // D/64 blocks of [32 keys][128 B]
+  static constexpr int K_OFF = 0;
+  static constexpr int V_OFF = K_OFF + kPfKSlots * KV_BYTES;
+  static constexpr int RAW_CODES = kPfBN * RB;
+  static constexpr int RAW_BYTES = 2 * RAW_CODES + NMETA * META_BYTES;
+  static constexpr int RAW_OFF = V_OFF + kPfVSlots * KV_BYTES;
+  static constexpr int BAR_OFF = RAW_OFF + kPfRawSlots * RAW_BYTES;
+  static constexpr int SMEM = BAR_OFF + 256 + 1024;  // + barriers, TMEM slot, alignment slack
+  // TMEM columns: O, S[2], Q (fp16 pairs), P[2] (fp16 pairs)
+  static constexpr int O_COL = 0;
+  static constexpr int S_COL = D;
+  static constexpr int Q_COL = S_COL + 2 * kPfBN;
+  static constexpr int P_COL = Q_COL + D / 2;
+  static constexpr int COLS = P_COL + 2 * (kPfBN / 2);
+  static constexpr int TMEM_COLS = COLS <= 128 ? 128 : (COLS <= 256 ? 256 : 512);
+  static_assert(COLS <= 512, "TMEM budget");
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
+  static_assert(RAW_BYTES % 128 == 0 && KV_BYTES % 1024 == 0, "slot alignment");
+  static_assert((kPfBN * UPR) % 32 == 0, "whole warps of chunks");
 };
 
-// ---- tcgen05 / mbarrier wrappers -------------------------------------------
+// ---- tcgen05 / mbarrier / bulk-copy wrappers -------------------------------
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
 }
@@ -106,60 +133,81 @@ __device__ __forceinline__ void mbar_arrive(uint32_t addr) {
   asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}\n"
                :: "r"(addr) : "memory");
 }
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t addr, uint32_t bytes) {
+  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}\n"
+               :: "r"(addr), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t addr, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(done) : "r"(addr), "r"(parity), "r"(1000u) : "memory");
+  return done != 0;
+}
 // Bounded wait for the phase with the given parity.  Returns at once (false)
 // if the CTA has already given up; on a time-out it records the error and
 // makes the CTA give up.
 __device__ __forceinline__ bool mbar_wait(uint32_t addr, uint32_t parity, volatile int* abort_flag,
                                           unsigned* status, unsigned code) {
   for (unsigned i = 0; i < kPfWaitLimit; ++i) {
-    uint32_t done;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(done) : "r"(addr), "r"(parity), "r"(1000u) : "memory");
-    if (done) return true;
+    if (mbar_try(addr, parity)) return true;
     if (*abort_flag) return false;
   }
   *abort_flag = 1;
   atomicOr(status, code);
   return false;
 }
+// Bounded wait that ignores an earlier give-up: used before exit for the
+// CTA's own asynchronous work still in flight.
+__device__ __forceinline__ void mbar_drain(uint32_t addr, uint32_t parity, unsigned* status) {
+  for (unsigned i = 0; i < kPfWaitLimit; ++i)
+    if (mbar_try(addr, parity)) return;
+  atomicOr(status, 128u);
+}
+// One contiguous global -> shared copy completing on an mbarrier (no multicast).
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n"
+      :: "r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
+}
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n"
                :: "r"(bar) : "memory");
 }
-// D(tmem) (+)= A(smem desc) * B(smem desc), kind::f16 with fp32 accumulate.
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                       uint32_t idesc, uint32_t accumulate) {
+// D(tmem) (+)= A(tmem) * B(smem desc), kind::f16 with fp32 accumulate.
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}\n"
-      :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate),
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}\n"
+      :: "r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate),
          "r"(0u), "r"(0u), "r"(0u), "r"(0u)
       : "memory");
 }
-// Shared-memory matrix descriptor of a K-major operand with 8-row groups
-// `sbo` bytes apart; swizzle 2 = 128-byte rows (64 16-bit elements), 4 =
-// 64-byte rows (32 elements).
-__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t sbo, uint32_t swizzle) {
+// Shared-memory matrix descriptor with 128-byte swizzled rows: `sbo` = bytes
+// between 8-row groups, `lbo` = bytes between 64-element column blocks (used
+// by MN-major operands only).
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
   uint64_t d = 0;
   d |= (uint64_t)((saddr >> 4) & 0x3fff);          // start address
-  d |= (uint64_t)1 << 16;                          // leading byte offset (unused, 16 B)
+  d |= (uint64_t)((lbo >> 4) & 0x3fff) << 16;      // leading byte offset
   d |= (uint64_t)((sbo >> 4) & 0x3fff) << 32;      // stride byte offset
   d |= (uint64_t)1 << 46;                          // descriptor version (sm_100)
-  d |= (uint64_t)swizzle << 61;
+  d |= (uint64_t)2 << 61;                          // 128-byte swizzle
   return d;
 }
-// Instruction descriptor: f16 x f16 -> f32, both operands K-major, M x N.
-__host__ __device__ constexpr uint32_t f16_idesc(int M, int N) {
-  return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+// Instruction descriptor: f16 x f16 -> f32, A K-major, B K-major (or MN-major
+// with b_mn), M x N.
+__host__ __device__ constexpr uint32_t f16_idesc(int M, int N, bool b_mn) {
+  return (1u << 4) | ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
 }
 
-// 32 consecutive fp32 columns of this thread's TMEM lane (warp-collective).
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
-  uint32_t r[32];
+// 32 consecutive 32-bit columns of this thread's TMEM lane (warp-collective).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
       "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
@@ -169,24 +217,25 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
         "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
         "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* v) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
       "%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n"
-      :: "r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])),
-         "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])),
-         "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
-         "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
-         "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
-         "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])),
-         "r"(__float_as_uint(v[17])), "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])),
-         "r"(__float_as_uint(v[20])), "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])),
-         "r"(__float_as_uint(v[23])), "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])),
-         "r"(__float_as_uint(v[26])), "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])),
-         "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      :: "r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]),
+         "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]),
+         "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]),
+         "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]),
+         "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+      "%13,%14,%15,%16};\n"
+      :: "r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]),
+         "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]),
+         "r"(v[13]), "r"(v[14]), "r"(v[15])
       : "memory");
 }
 __device__ __forceinline__ void tmem_wait_ld() {
@@ -199,142 +248,74 @@ __device__ __forceinline__ void named_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;\n" :: "r"(id), "r"(nthreads) : "memory");
 }
 
-// Byte offset of 16-bit element (row, col) in a K-major operand with
-// 128-byte swizzled rows (64 columns per block, `rows` rows per block).
-__device__ __forceinline__ int sw128_off(int row, int col, int rows) {
+// Byte offset of 16-bit element (row, col) in a tile of 32-row blocks with
+// 128-byte swizzled rows (64 columns per block).
+__device__ __forceinline__ int sw128_off(int row, int col) {
   const int blk = col >> 6, chunk = (col >> 3) & 7;
-  return blk * rows * 128 + row * 128 + ((chunk ^ (row & 7)) << 4) + (col & 7) * 2;
-}
-// Same for 64-byte swizzled rows (32 columns).
-__device__ __forceinline__ int sw64_off(int row, int col) {
-  const int chunk = (col >> 3) & 3;
-  return row * 64 + ((chunk ^ ((row >> 1) & 3)) << 4) + (col & 7) * 2;
+  return blk * kPfBN * 128 + row * 128 + ((chunk ^ (row & 7)) << 4) + (col & 7) * 2;
 }
 
-// Position of head-dimension element e inside a K-major row.  The 4-bit codes
-// of a 32-bit word come out of the mask-and-magic conversion as the pairs
-// (0,4), (1,5), (2,6), (3,7); Q is stored with the same permutation so Q K^T is
-// unchanged.  8-bit codes come out in natural order.
+// Position of head-dimension element e inside a K/V row.  The 4-bit codes of
+// a 32-bit word come out of the mask-and-magic conversion as the pairs (0,4),
+// (1,5), (2,6), (3,7); Q is stored with the same permutation so Q K^T is
+// unchanged, and the output columns of P V are put back in the epilogue.
+// 8-bit codes come out in natural order.
 template <int BITS>
-__device__ __forceinline__ int k_pos(int e) {
+__host__ __device__ constexpr int k_pos(int e) {
   if constexpr (BITS == 4) {
-    const int j = e & 7;
-    return (e & ~7) | ((j & 3) << 1) | (j >> 2);
+    return (e & ~7) | ((e & 3) << 1) | ((e & 7) >> 2);
   } else {
     return e;
   }
 }
 
-// Low bytes of lanes 0/2 of a word -> fp16 pair (1024 + b0, 1024 + b2): the
-// magic exponent 0x64 makes the fp16 value 1024 + byte exactly.
-__device__ __forceinline__ __half2 u8pair_plus1024(uint32_t w) {
-  const uint32_t x = (w & 0x00FF00FFu) | 0x64006400u;
-  return *reinterpret_cast<const __half2*>(&x);
-}
-
-// Raw V rows are stored with their 16-byte units XOR-swizzled by (row / 8)
-// so the transposing reads below (8 rows x 8 word positions per warp) spread
-// over all banks.
-template <int UPR>
-__device__ __forceinline__ int rawv_unit(int row, int unit) {
-  constexpr int M = UPR >= 8 ? 7 : UPR - 1;
-  return unit ^ ((row >> 3) & M);
-}
-
-// Dequantizes one staged tile (raw slot `raw`) into K (fp16 [key][d], SW128)
-// and V (fp16 [d][key], SW64); value = scale * code + bias rounded once.
+// Dequantizes the 32 code rows of one packed tile into fp16 [key][d] with
+// 128-byte swizzled rows; value = scale * code + bias rounded once, rows at or
+// past `nv` (keys past L) are written as zeros.
 template <int D, int BITS, int GS, bool Q8>
-__device__ __forceinline__ void dequant_tile(const uint8_t* raw, uint8_t* kdst, uint8_t* vdst,
-                                             int dq) {
+__device__ __forceinline__ void pf_dequant(const uint8_t* codes, const uint16_t* sc,
+                                           const uint16_t* bi, uint8_t* dst, int nv, int chunk0) {
   using C = PfCfg<D, BITS, GS, Q8>;
-  constexpr int NG = C::NG;
-  constexpr int NT = 32 * kPfDqWarps;
-  const uint8_t* rk = raw;
-  const uint8_t* rv = raw + kPfBN * C::RB;
-  const uint8_t* meta = raw + 2 * kPfBN * C::RB;
-  const uint16_t* mks = reinterpret_cast<const uint16_t*>(meta);
-  const uint16_t* mkb = reinterpret_cast<const uint16_t*>(meta + C::META_BYTES);
-  const uint16_t* mvs = reinterpret_cast<const uint16_t*>(meta + (Q8 ? 1 : 2) * C::META_BYTES);
-  const uint16_t* mvb = reinterpret_cast<const uint16_t*>(meta + 3 * C::META_BYTES);
+  constexpr int NCH = kPfBN * C::UPR;
+  constexpr int ITERS = (NCH + kPfDqThreads - 1) / kPfDqThreads;
   const __half2 off = __float2half2_rn(Q8 ? 1152.f : 1024.f);   // Q8 codes are stored +128
-
-  // K: one 16-byte output chunk (8 elements of one key) per step
-  constexpr int KCH = D / 8;
-  for (int ci = dq; ci < kPfBN * KCH; ci += NT) {
-    const int j = ci / KCH, c = ci - j * KCH;
-    const int G = (c * 8) / GS;
-    const __half2 s2 = __half2half2(__ushort_as_half(mks[j * NG + G]));
-    const __half2 b2 = Q8 ? __float2half2_rn(0.f) : __half2half2(__ushort_as_half(mkb[j * NG + G]));
-    __half2 h[4];
+#pragma unroll
+  for (int it = 0; it < ITERS; ++it) {
+    const int i = chunk0 + it * kPfDqThreads;
+    if (NCH % kPfDqThreads != 0 && i >= NCH) break;   // whole warps drop out together
+    const int key = i / C::UPR, u = i - key * C::UPR;
+    const uint4 w4 = *reinterpret_cast<const uint4*>(codes + i * 16);
+    const int g = (u * C::CPC) / GS;
+    const __half2 s2 = __half2half2(__ushort_as_half(sc[key * C::NG + g]));
+    const __half2 b2 = Q8 ? __float2half2_rn(0.f) : __half2half2(__ushort_as_half(bi[key * C::NG + g]));
+    const bool live = key < nv;
+    const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
     if constexpr (BITS == 8) {
-      const uint2 w = *reinterpret_cast<const uint2*>(rk + j * C::RB + c * 8);
-      const uint32_t w0 = Q8 ? (w.x ^ 0x80808080u) : w.x, w1 = Q8 ? (w.y ^ 0x80808080u) : w.y;
-      h[0] = u8pair_plus1024(prmt(w0, 0u, 0x4140u));
-      h[1] = u8pair_plus1024(prmt(w0, 0u, 0x4342u));
-      h[2] = u8pair_plus1024(prmt(w1, 0u, 0x4140u));
-      h[3] = u8pair_plus1024(prmt(w1, 0u, 0x4342u));
+      uint32_t o[8];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t x = Q8 ? (wv[k] ^ 0x80808080u) : wv[k];
+        const uint32_t h0 = prmt(x, 0x64646464u, 0x4140u);   // (1024 + byte0, 1024 + byte1)
+        const uint32_t h1 = prmt(x, 0x64646464u, 0x4342u);
+        const __half2 v0 = __hfma2(__hsub2(*reinterpret_cast<const __half2*>(&h0), off), s2, b2);
+        const __half2 v1 = __hfma2(__hsub2(*reinterpret_cast<const __half2*>(&h1), off), s2, b2);
+        o[2 * k] = live ? *reinterpret_cast<const uint32_t*>(&v0) : 0u;
+        o[2 * k + 1] = live ? *reinterpret_cast<const uint32_t*>(&v1) : 0u;
+      }
+      *reinterpret_cast<uint4*>(dst + sw128_off(key, u * 16)) = make_uint4(o[0], o[1], o[2], o[3]);
+      *reinterpret_cast<uint4*>(dst + sw128_off(key, u * 16 + 8)) = make_uint4(o[4], o[5], o[6], o[7]);
     } else {
-      const uint32_t w = *reinterpret_cast<const uint32_t*>(rk + j * C::RB + c * 4);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {      // nibbles (k, k+4) -> positions (2k, 2k+1)
-        const uint32_t x = ((w >> (4 * k)) & 0x000F000Fu) | 0x64006400u;
-        h[k] = *reinterpret_cast<const __half2*>(&x);
-      }
-    }
-    uint32_t o[4];
+      for (int k = 0; k < 4; ++k) {      // word k: d = 32u + 8k .. +7, nibbles (j, j+4) -> (2j, 2j+1)
+        uint32_t o[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const __half2 v = __hfma2(__hsub2(h[i], off), s2, b2);
-      o[i] = *reinterpret_cast<const uint32_t*>(&v);
-    }
-    *reinterpret_cast<uint4*>(kdst + sw128_off(j, c * 8, kPfBN)) = make_uint4(o[0], o[1], o[2], o[3]);
-  }
-
-  // V: a task = one 32-bit code word position (EPW dims) x 8 keys, transposed
-  // in registers into EPW output chunks (one per dim) of 8 keys each
-  constexpr int EPW = 32 / BITS;                 // dims per word
-  constexpr int WPR = D / EPW;                   // words per key row
-  constexpr int KB8 = kPfBN / 8;                 // 8-key blocks per tile
-  for (int task = dq; task < WPR * KB8; task += NT) {
-    const int kb8 = task % KB8, wi = task / KB8;
-    const int e0 = wi * EPW, j0 = kb8 * 8;
-    const int G = e0 / GS;
-    uint32_t w[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int r = j0 + i;
-      const int unit = rawv_unit<C::UPR>(r, (wi * 4) >> 4);
-      w[i] = *reinterpret_cast<const uint32_t*>(rv + r * C::RB + unit * 16 + ((wi * 4) & 15));
-      if (Q8) w[i] ^= 0x80808080u;
-    }
-    __half2 s2[4], b2[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      s2[i] = __halves2half2(__ushort_as_half(mvs[(j0 + 2 * i) * NG + G]),
-                             __ushort_as_half(mvs[(j0 + 2 * i + 1) * NG + G]));
-      b2[i] = Q8 ? __float2half2_rn(0.f)
-                 : __halves2half2(__ushort_as_half(mvb[(j0 + 2 * i) * NG + G]),
-                                  __ushort_as_half(mvb[(j0 + 2 * i + 1) * NG + G]));
-    }
-#pragma unroll
-    for (int d = 0; d < EPW; ++d) {
-      uint32_t hv[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        __half2 c;
-        if constexpr (BITS == 8) {
-          // byte d of the words of keys j0+2i and j0+2i+1 -> lanes 0 and 2
-          c = __hsub2(u8pair_plus1024(prmt(w[2 * i], w[2 * i + 1], (uint32_t)(d | ((4 + d) << 8)))), off);
-        } else {
-          const int sh = 4 * d;
-          const uint32_t x = ((w[2 * i] >> sh) & 0xFu) | (((w[2 * i + 1] >> sh) & 0xFu) << 16) |
-                             0x64006400u;
-          c = __hsub2(*reinterpret_cast<const __half2*>(&x), off);
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t x = ((wv[k] >> (4 * j)) & 0x000F000Fu) | 0x64006400u;
+          const __half2 v = __hfma2(__hsub2(*reinterpret_cast<const __half2*>(&x), off), s2, b2);
+          o[j] = live ? *reinterpret_cast<const uint32_t*>(&v) : 0u;
         }
-        const __half2 v = __hfma2(c, s2[i], b2[i]);
-        hv[i] = *reinterpret_cast<const uint32_t*>(&v);
+        *reinterpret_cast<uint4*>(dst + sw128_off(key, u * 32 + 8 * k)) = make_uint4(o[0], o[1], o[2], o[3]);
       }
-      *reinterpret_cast<uint4*>(vdst + sw64_off(e0 + d, j0)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
     }
   }
 }
@@ -347,14 +328,16 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(smem);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // mbarriers: kv_ready[2], s_full[2], p_ready[2], pv_done[2]
   const uint32_t bar0 = sbase + C::BAR_OFF;
-  auto kv_ready = [&](int i) { return bar0 + 8 * i; };
-  auto s_full = [&](int i) { return bar0 + 16 + 8 * i; };
-  auto p_ready = [&](int i) { return bar0 + 32 + 8 * i; };
-  auto pv_done = [&](int i) { return bar0 + 48 + 8 * i; };
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::BAR_OFF + 64);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::BAR_OFF + 68);
+  auto raw_full = [&](int i) { return bar0 + 8 * i; };        // [3] packed tile landed
+  auto k_ready = [&](int i) { return bar0 + 24 + 8 * i; };    // [2] fp16 K written
+  auto v_ready = [&](int i) { return bar0 + 40 + 8 * i; };    // [3] fp16 V written
+  auto s_full = [&](int i) { return bar0 + 64 + 8 * i; };     // [2] S in TMEM
+  auto p_ready = [&](int i) { return bar0 + 80 + 8 * i; };    // [2] P in TMEM
+  auto pv_done = [&](int i) { return bar0 + 96 + 8 * i; };    // [3] P V product done
+  const uint32_t mma_done = bar0 + 120;                       // all tensor-core work done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::BAR_OFF + 128);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::BAR_OFF + 132);
 
   const int mt = blockIdx.x % p.mtiles;
   const int hkv = (blockIdx.x / p.mtiles) % p.Hkv;
@@ -374,24 +357,69 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
   }
   if (tid == 0) {
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(kv_ready(i), 32 * kPfDqWarps);
-      mbar_init(s_full(i), 1);
-      mbar_init(p_ready(i), 32 * kPfSoftWarps);
+    for (int i = 0; i < 3; ++i) {
+      mbar_init(raw_full(i), 1);
+      mbar_init(v_ready(i), kPfDqThreads);
       mbar_init(pv_done(i), 1);
     }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(k_ready(i), kPfDqThreads);
+      mbar_init(s_full(i), 1);
+      mbar_init(p_ready(i), 32 * kPfSoftWarps);
+    }
+    mbar_init(mma_done, 1);
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     *abort_flag = 0;
   }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int64_t row0 = ((int64_t)b * p.Hkv + hkv) * p.Lcap;
 
-  // ---- Q rows -> fp16 (per-row power-of-two prescale), swizzled K-major ----
-  const int r = mt * kPfBM + tid;                 // softmax threads: this thread's row
+  // softmax threads: this thread's row
+  const int r = mt * kPfBM + tid;
   const bool row_ok = tid < kPfBM && r < R;
   const int qi = row_ok ? r / p.G : 0;
   const int hh = row_ok ? r - qi * p.G : 0;
   const int64_t qrow = (((int64_t)b * p.Hq + (int64_t)hkv * p.G + hh) * p.Lq + qi) * D;
+  const uint32_t tmem_row = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+
+  // dequant warps: packed-tile sources
+  const int dq = tid - 32 * kPfSoftWarps;
+  const uint8_t* gK = p.kc + row0 * C::RB;
+  const uint8_t* gV = p.vc + row0 * C::RB;
+  int issued = 0;                                // tiles whose bulk copies were issued
+  auto issue_raw = [&](int t) {                  // one thread: the bulk copies of tile t
+    ++issued;
+    const int slot = t % kPfRawSlots;
+    const int64_t key0 = (int64_t)t * kPfBN;
+    const int nv = L - key0 < kPfBN ? (int)(L - key0) : kPfBN;
+    const int nv8 = (nv + 7) & ~7;               // scale rows in whole 16-byte units
+    const uint32_t cb = (uint32_t)(nv * C::RB), mb = (uint32_t)(nv8 * NG * 2);
+    const uint32_t bar = raw_full(slot);
+    const uint32_t dst = sbase + C::RAW_OFF + slot * C::RAW_BYTES;
+    mbar_arrive_expect_tx(bar, 2 * cb + C::NMETA * mb);
+    bulk_g2s(dst, gK + key0 * C::RB, cb, bar);
+    bulk_g2s(dst + C::RAW_CODES, gV + key0 * C::RB, cb, bar);
+    const int64_t m0 = (row0 + key0) * NG;
+    bulk_g2s(dst + 2 * C::RAW_CODES, p.ks + m0, mb, bar);
+    if (Q8) {
+      bulk_g2s(dst + 2 * C::RAW_CODES + C::META_BYTES, p.vs + m0, mb, bar);
+    } else {
+      bulk_g2s(dst + 2 * C::RAW_CODES + C::META_BYTES, p.kb + m0, mb, bar);
+      bulk_g2s(dst + 2 * C::RAW_CODES + 2 * C::META_BYTES, p.vs + m0, mb, bar);
+      bulk_g2s(dst + 2 * C::RAW_CODES + 3 * C::META_BYTES, p.vb + m0, mb, bar);
+    }
+  };
+  const int n_first = ntiles < kPfRawSlots ? ntiles : kPfRawSlots;
+  if (dq == 0) {
+    for (int t = 0; t < n_first; ++t) issue_raw(t);
+  }
+
+  // ---- Q rows -> fp16 (per-row power-of-two prescale) in TMEM ----------------
   float rowscale = 0.f;
-  if (tid < kPfBM) {
+  if (warp < kPfSoftWarps) {
     float mx = 0.f;
     if (row_ok) {
       for (int e = 0; e < D; e += 8) {
@@ -412,130 +440,106 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
     sigma = max(-96, min(96, sigma));
     const float up = exp2i(sigma);
     rowscale = p.scale_log2e * exp2i(-sigma);
-    uint16_t* qs = reinterpret_cast<uint16_t*>(smem + C::Q_OFF);
-    for (int e = 0; e < D; e += 8) {
-      uint32_t w[4] = {0u, 0u, 0u, 0u};
-      if (row_ok) {
-        const uint4 raw = *reinterpret_cast<const uint4*>(
-            reinterpret_cast<const uint16_t*>(p.q) + qrow + e);
-        w[0] = raw.x; w[1] = raw.y; w[2] = raw.z; w[3] = raw.w;
-      }
+#pragma unroll 1
+    for (int c0 = 0; c0 < D; c0 += 64) {         // 64 elements = 32 TMEM columns
+      uint32_t qw[32];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const uint16_t bits = (uint16_t)(w[k >> 1] >> (16 * (k & 1)));
-        const float v = p.q_dtype == QKV_F16 ? __half2float(__ushort_as_half(bits))
-                                             : __uint_as_float((uint32_t)bits << 16);
-        qs[sw128_off(tid, k_pos<BITS>(e + k), kPfBM) / 2] = __half_as_ushort(__float2half_rn(v * up));
+      for (int e8 = 0; e8 < 64; e8 += 8) {
+        uint32_t w[4] = {0u, 0u, 0u, 0u};
+        if (row_ok) {
+          const uint4 raw = *reinterpret_cast<const uint4*>(
+              reinterpret_cast<const uint16_t*>(p.q) + qrow + c0 + e8);
+          w[0] = raw.x; w[1] = raw.y; w[2] = raw.z; w[3] = raw.w;
+        }
+        float v[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint16_t bits = (uint16_t)(w[k >> 1] >> (16 * (k & 1)));
+          v[k] = (p.q_dtype == QKV_F16 ? __half2float(__ushort_as_half(bits))
+                                       : __uint_as_float((uint32_t)bits << 16)) * up;
+        }
+        float s[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) s[k_pos<BITS>(k)] = v[k];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) qw[e8 / 2 + k] = pack_half2(s[2 * k], s[2 * k + 1]);
       }
+      tmem_st32(tmem_row + C::Q_COL + c0 / 2, qw);
     }
+    tmem_wait_st();
   }
-  fence_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-
-  const int64_t row0 = ((int64_t)b * p.Hkv + hkv) * p.Lcap;
-  constexpr uint32_t kS_COL = D;                   // S[2] after O
 
   if (warp >= kPfSoftWarps && warp < kPfMmaWarp) {
     // ======================= dequant warps =====================================
-    const int dq = tid - 32 * kPfSoftWarps;
-    constexpr int NT = 32 * kPfDqWarps;
-    const uint8_t* gK = p.kc + row0 * C::RB;
-    const uint8_t* gV = p.vc + row0 * C::RB;
-    const uint8_t* gKs = reinterpret_cast<const uint8_t*>(p.ks + row0 * NG);
-    const uint8_t* gKb = Q8 ? gKs : reinterpret_cast<const uint8_t*>(p.kb + row0 * NG);
-    const uint8_t* gVs = reinterpret_cast<const uint8_t*>(p.vs + row0 * NG);
-    const uint8_t* gVb = Q8 ? gVs : reinterpret_cast<const uint8_t*>(p.vb + row0 * NG);
-    auto issue = [&](int t) {
-      const uint32_t slot = sbase + C::RAW_OFF + (t & 1) * C::RAW_BYTES;
-      const int64_t key0 = (int64_t)t * kPfBN;
-      const int64_t nvalid = L - key0;
-      constexpr int CU = kPfBN * C::UPR;
-      for (int i = dq; i < 2 * CU; i += NT) {
-        const int which = i >= CU, j = which ? i - CU : i;
-        const int row = j / C::UPR, unit = j - row * C::UPR;
-        const bool ok = row < nvalid;
-        const uint8_t* src = (which ? gV : gK) + (ok ? (key0 + row) * C::RB + unit * 16 : 0);
-        const int dst = which ? kPfBN * C::RB + row * C::RB + rawv_unit<C::UPR>(row, unit) * 16
-                              : j * 16;
-        cp_async16(slot + dst, src, ok ? 16 : 0);
-      }
-      constexpr int MU = kPfBN * NG * 2 / 16;
-      for (int i = dq; i < C::NMETA * MU; i += NT) {
-        const int arr = i / MU, j = i - arr * MU;
-        const uint8_t* gm = Q8 ? (arr == 0 ? gKs : gVs)
-                               : (arr == 0 ? gKs : arr == 1 ? gKb : arr == 2 ? gVs : gVb);
-        const bool ok = (j * 16) / (NG * 2) < nvalid;
-        cp_async16(slot + 2 * kPfBN * C::RB + arr * C::META_BYTES + j * 16,
-                   ok ? gm + key0 * NG * 2 + j * 16 : gm, ok ? 16 : 0);
-      }
-    };
-    if (ntiles > 0) issue(0);
-    cp_async_commit();
-    if (ntiles > 1) issue(1);
-    cp_async_commit();
+    int cl = 0;
+#pragma unroll
+    for (int bt = 0; bt < 5; ++bt)
+      if ((lane >> bt) & 1) cl ^= pf_lane_col(D, BITS, bt);
+    const int chunk0 = (dq >> 5) * 32 + cl;
     for (int t = 0; t < ntiles; ++t) {
-      const int s = t & 1;
-      cp_async_wait<1>();
-      named_sync(1, NT);
-      uint8_t* raw = smem + C::RAW_OFF + s * C::RAW_BYTES;
-      const int64_t nvalid = L - (int64_t)t * kPfBN;
-      if (nvalid < kPfBN) {          // clear stale scales/biases of keys past L
-        uint16_t* meta = reinterpret_cast<uint16_t*>(raw + 2 * kPfBN * C::RB);
-        for (int i = dq; i < C::NMETA * kPfBN * NG; i += NT) {
-          const int arr = i / (kPfBN * NG), rr = i - arr * kPfBN * NG;
-          if (rr / NG >= nvalid) meta[arr * (C::META_BYTES / 2) + rr] = 0;
-        }
-        named_sync(1, NT);
-      }
-      if (t >= 2) {                  // operand slot s free once P V of tile t-2 is done
-        mbar_wait(pv_done(s), ((t - 2) >> 1) & 1, abort_flag, p.status, 1u);
-        tc_fence_after();
-      }
-      dequant_tile<D, BITS, GS, Q8>(raw, smem + C::K_OFF + s * C::K_BYTES,
-                                    smem + C::V_OFF + s * C::V_BYTES, dq);
+      const int slot = t % kPfRawSlots, ks = t & 1, vs = t % kPfVSlots;
+      const int64_t key0 = (int64_t)t * kPfBN;
+      const int nv = L - key0 < kPfBN ? (int)(L - key0) : kPfBN;
+      mbar_wait(raw_full(slot), (t / kPfRawSlots) & 1, abort_flag, p.status, 1u);
+      const uint8_t* raw = smem + C::RAW_OFF + slot * C::RAW_BYTES;
+      const uint16_t* meta = reinterpret_cast<const uint16_t*>(raw + 2 * C::RAW_CODES);
+      constexpr int MH = C::META_BYTES / 2;      // metadata array stride in halves
+      if (t >= kPfKSlots)                        // K slot free once S of tile t-2 is done
+        mbar_wait(s_full(ks), ((t - 2) >> 1) & 1, abort_flag, p.status, 1u);
+      pf_dequant<D, BITS, GS, Q8>(raw, meta, meta + MH, smem + C::K_OFF + ks * C::KV_BYTES, nv,
+                                  chunk0);
       fence_async_smem();
-      mbar_arrive(kv_ready(s));
-      named_sync(1, NT);             // everyone is done reading raw slot s
-      if (t + 2 < ntiles) issue(t + 2);
-      cp_async_commit();
+      mbar_arrive(k_ready(ks));
+      if (t >= kPfVSlots)                        // V slot free once P V of tile t-3 is done
+        mbar_wait(pv_done(vs), ((t - 3) / 3) & 1, abort_flag, p.status, 1u);
+      pf_dequant<D, BITS, GS, Q8>(raw + C::RAW_CODES, meta + (Q8 ? 1 : 2) * MH,
+                                  meta + 3 * MH, smem + C::V_OFF + vs * C::KV_BYTES, nv, chunk0);
+      fence_async_smem();
+      mbar_arrive(v_ready(vs));
+      named_sync(1, kPfDqThreads);               // every thread is done reading raw slot
+      if (dq == 0 && t + kPfRawSlots < ntiles && !*abort_flag) issue_raw(t + kPfRawSlots);
     }
-    cp_async_wait<0>();
+    if (dq == 0) {                               // own bulk copies still in flight (after a give-up)
+      for (int t = max(0, issued - kPfRawSlots); t < issued; ++t)
+        mbar_drain(raw_full(t % kPfRawSlots), (t / kPfRawSlots) & 1, p.status);
+    }
   } else if (warp == kPfMmaWarp) {
     // ======================= MMA warp ==========================================
-    constexpr uint32_t idesc_s = f16_idesc(kPfBM, kPfBN);
-    constexpr uint32_t idesc_o = f16_idesc(kPfBM, D);
+    constexpr uint32_t idesc_s = f16_idesc(kPfBM, kPfBN, false);
+    constexpr uint32_t idesc_o = f16_idesc(kPfBM, D, true);
     auto issue_s = [&](int t) {
       const int s = t & 1;
-      mbar_wait(kv_ready(s), (t >> 1) & 1, abort_flag, p.status, 2u);
+      mbar_wait(k_ready(s), (t >> 1) & 1, abort_flag, p.status, 2u);
       tc_fence_after();
       if (lane == 0) {
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
-          const int blk = k >> 2, sub = (k & 3) * 32;
-          const uint64_t a = umma_desc(sbase + C::Q_OFF + blk * kPfBM * 128 + sub, 1024, 2);
-          const uint64_t bd = umma_desc(sbase + C::K_OFF + s * C::K_BYTES + blk * kPfBN * 128 + sub,
-                                        1024, 2);
-          tc_mma(tmem + kS_COL + s * kPfBN, a, bd, idesc_s, k > 0 ? 1u : 0u);
+          const uint64_t bd = umma_desc_sw128(
+              sbase + C::K_OFF + s * C::KV_BYTES + (k >> 2) * kPfBN * 128 + (k & 3) * 32, 16, 1024);
+          tc_mma_ts(tmem + C::S_COL + s * kPfBN, tmem + C::Q_COL + k * 8, bd, idesc_s,
+                    k > 0 ? 1u : 0u);
         }
         tc_commit(s_full(s));
       }
       __syncwarp();
     };
     auto issue_pv = [&](int t) {
-      const int s = t & 1;
+      const int s = t & 1, vs = t % kPfVSlots;
+      mbar_wait(v_ready(vs), (t / kPfVSlots) & 1, abort_flag, p.status, 4u);
       mbar_wait(p_ready(s), (t >> 1) & 1, abort_flag, p.status, 4u);
       tc_fence_after();
       if (lane == 0) {
 #pragma unroll
         for (int k = 0; k < kPfBN / 16; ++k) {
-          const uint64_t a = umma_desc(sbase + C::P_OFF + s * C::P_BYTES + k * 32, 512, 4);
-          const uint64_t bd = umma_desc(sbase + C::V_OFF + s * C::V_BYTES + k * 32, 512, 4);
-          tc_mma(tmem, a, bd, idesc_o, (t > 0 || k > 0) ? 1u : 0u);
+          const uint64_t bd = umma_desc_sw128(sbase + C::V_OFF + vs * C::KV_BYTES + k * 16 * 128,
+                                              kPfBN * 128, 1024);
+          tc_mma_ts(tmem + C::O_COL, tmem + C::P_COL + s * (kPfBN / 2) + k * 8, bd, idesc_o,
+                    (t > 0 || k > 0) ? 1u : 0u);
         }
-        tc_commit(pv_done(s));
+        tc_commit(pv_done(vs));
       }
       __syncwarp();
     };
@@ -544,10 +548,16 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
       if (t + 1 < ntiles) issue_s(t + 1);   // overlaps the softmax of tile t
       issue_pv(t);
     }
+    if (lane == 0) {                         // every MMA issued above has completed
+      tc_commit(mma_done);
+      mbar_drain(mma_done, 0, p.status);
+    }
+    __syncwarp();
   } else {
     // ======================= softmax warps (one row per thread) =================
-    const uint32_t tmem_row = tmem + ((uint32_t)(warp * 32) << 16);
     const int64_t causal_lim = L - p.Lq + qi;    // last visible key of this row
+    const bool causal = p.mask_kind == QKV_MASK_CAUSAL;
+    const bool additive = p.mask_kind == QKV_MASK_ADDITIVE;
     float m_used = -INFINITY, lsum = 0.f;
     for (int t = 0; t < ntiles; ++t) {
       const int s = t & 1;
@@ -555,103 +565,128 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
       mbar_wait(s_full(s), (t >> 1) & 1, abort_flag, p.status, 8u);
       tc_fence_after();
       float sv[kPfBN];
-      tmem_ld32(tmem_row + kS_COL + s * kPfBN, sv);
+      tmem_ld32(tmem_row + C::S_COL + s * kPfBN, reinterpret_cast<uint32_t*>(sv));
       tmem_wait_ld();
-      float tmax = -INFINITY;
+      // a tile without masked keys for any row of the warp takes the short path
+      const bool full = __all_sync(~0u, row_ok && !additive && key0 + kPfBN <= kend &&
+                                            (!causal || key0 + kPfBN - 1 <= causal_lim));
+      float tmax;
+      if (full) {
+        float mx = sv[0];
 #pragma unroll
-      for (int j = 0; j < kPfBN; ++j) {
-        const int64_t key = key0 + j;
-        float v = sv[j] * rowscale;
-        bool vis = row_ok && key < kend;
-        if (p.mask_kind == QKV_MASK_CAUSAL) vis = vis && key <= causal_lim;
-        if (vis && p.mask_kind == QKV_MASK_ADDITIVE) {
-          const int64_t mi = (int64_t)b * p.msb + ((int64_t)hkv * p.G + hh) * p.msh +
-                             (int64_t)qi * p.msq + key;
-          v += kLog2e * load_as_float(p.mask, p.mask_dtype, mi);
+        for (int j = 1; j < kPfBN; ++j) mx = fmaxf(mx, sv[j]);
+        tmax = mx * rowscale;
+      } else {
+        tmax = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < kPfBN; ++j) {
+          const int64_t key = key0 + j;
+          bool vis = row_ok && key < kend;
+          if (causal) vis = vis && key <= causal_lim;
+          float v = sv[j] * rowscale;
+          if (vis && additive) {
+            const int64_t mi = (int64_t)b * p.msb + ((int64_t)hkv * p.G + hh) * p.msh +
+                               (int64_t)qi * p.msq + key;
+            v += kLog2e * load_as_float(p.mask, p.mask_dtype, mi);
+          }
+          sv[j] = vis ? v : -INFINITY;
+          tmax = fmaxf(tmax, sv[j]);
         }
-        sv[j] = vis ? v : -INFINITY;
-        tmax = fmaxf(tmax, sv[j]);
       }
       float alpha = 1.f;
-      if (tmax > m_used + 8.f || (m_used == -INFINITY && tmax != -INFINITY)) {
-        alpha = m_used == -INFINITY ? 0.f : ex2(m_used - tmax);
+      if (tmax > m_used + 8.f) {
+        // no earlier key was visible: O and l are still zero, nothing to rescale
+        alpha = m_used == -INFINITY ? 1.f : ex2(m_used - tmax);
         m_used = tmax;
       }
       const float mref = m_used == -INFINITY ? 0.f : m_used;
       // P slot s is free once the P V product of tile t-2 is done; the O
       // rescale needs the product of tile t-1 done (both are rare waits)
-      if (t >= 2) mbar_wait(pv_done(s), ((t - 2) >> 1) & 1, abort_flag, p.status, 16u);
+      if (t >= 2) {
+        mbar_wait(pv_done((t - 2) % kPfVSlots), ((t - 2) / kPfVSlots) & 1, abort_flag, p.status, 16u);
+        tc_fence_after();
+      }
       const bool rescale = t > 0 && __any_sync(~0u, alpha != 1.f);
       if (rescale) {
-        mbar_wait(pv_done(s ^ 1), ((t - 1) >> 1) & 1, abort_flag, p.status, 32u);
+        mbar_wait(pv_done((t - 1) % kPfVSlots), ((t - 1) / kPfVSlots) & 1, abort_flag, p.status, 32u);
         tc_fence_after();
 #pragma unroll 1
         for (int c = 0; c < D; c += 32) {
-          float o[32];
-          tmem_ld32(tmem_row + c, o);
+          uint32_t o[32];
+          tmem_ld32(tmem_row + C::O_COL + c, o);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] *= alpha;
-          tmem_st32(tmem_row + c, o);
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(tmem_row + C::O_COL + c, o);
         }
-        tmem_wait_st();
       }
       float rs = 0.f;
-      uint8_t* ps = smem + C::P_OFF + s * C::P_BYTES;
+      uint32_t pk[kPfBN / 2];
+      if (full) {
+        const float nm = -mref;
 #pragma unroll
-      for (int j = 0; j < kPfBN; j += 8) {
-        uint32_t pk[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float a = ex2(sv[j + 2 * i] - mref), c = ex2(sv[j + 2 * i + 1] - mref);
+        for (int i = 0; i < kPfBN / 2; ++i) {
+          const float a = ex2(fmaf(sv[2 * i], rowscale, nm));
+          const float c = ex2(fmaf(sv[2 * i + 1], rowscale, nm));
           rs += a + c;
           pk[i] = pack_half2(a, c);
         }
-        *reinterpret_cast<uint4*>(ps + sw64_off(tid, j)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < kPfBN / 2; ++i) {
+          const float a = ex2(sv[2 * i] - mref), c = ex2(sv[2 * i + 1] - mref);
+          rs += a + c;
+          pk[i] = pack_half2(a, c);
+        }
       }
+      tmem_st16(tmem_row + C::P_COL + s * (kPfBN / 2), pk);
+      tmem_wait_st();
       lsum = lsum * alpha + rs;
-      fence_async_smem();
       tc_fence_before();
       mbar_arrive(p_ready(s));
     }
     // ---- epilogue: O / l -> out --------------------------------------------
     bool have = ntiles > 0;
     if (have) {
-      have = mbar_wait(pv_done((ntiles - 1) & 1), ((ntiles - 1) >> 1) & 1, abort_flag, p.status, 64u);
+      have = mbar_wait(pv_done((ntiles - 1) % kPfVSlots), ((ntiles - 1) / kPfVSlots) & 1,
+                       abort_flag, p.status, 64u);
       tc_fence_after();
     }
     have = __all_sync(~0u, have) && !*abort_flag;
     const float inv = (lsum > 0.f && have) ? 1.f / lsum : 0.f;
+#pragma unroll 1
     for (int c = 0; c < D; c += 32) {
-      float o[32];
+      uint32_t ob[32];
       if (have) {
-        tmem_ld32(tmem_row + c, o);
+        tmem_ld32(tmem_row + C::O_COL + c, ob);
         tmem_wait_ld();
       } else {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) o[i] = 0.f;
+        for (int i = 0; i < 32; ++i) ob[i] = 0u;
       }
+      float o[32];                               // output order (undo the 4-bit pairing)
+#pragma unroll
+      for (int i = 0; i < 32; ++i) o[i] = __uint_as_float(ob[k_pos<BITS>(i)]) * inv;
       if (row_ok) {
         if (p.out_dtype == QKV_BF16 || p.out_dtype == QKV_F16) {
 #pragma unroll
           for (int i = 0; i < 32; i += 8) {
-            uint32_t pk[4];
+            uint32_t pq[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-              const float a = o[i + 2 * k] * inv, cc = o[i + 2 * k + 1] * inv;
               if (p.out_dtype == QKV_F16) {
-                pk[k] = pack_half2(a, cc);
+                pq[k] = pack_half2(o[i + 2 * k], o[i + 2 * k + 1]);
               } else {
-                const __nv_bfloat162 h2 = __floats2bfloat162_rn(a, cc);
-                pk[k] = *reinterpret_cast<const uint32_t*>(&h2);
+                const __nv_bfloat162 h2 = __floats2bfloat162_rn(o[i + 2 * k], o[i + 2 * k + 1]);
+                pq[k] = *reinterpret_cast<const uint32_t*>(&h2);
               }
             }
             *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.out) + qrow + c + i) =
-                make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                make_uint4(pq[0], pq[1], pq[2], pq[3]);
           }
         } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) store_from_float(p.out, p.out_dtype, qrow + c + i, o[i] * inv);
+          for (int i = 0; i < 32; ++i) store_from_float(p.out, p.out_dtype, qrow + c + i, o[i]);
         }
       }
     }
