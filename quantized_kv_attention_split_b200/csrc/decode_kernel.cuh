@@ -41,11 +41,10 @@
 
 namespace qkv {
 
-constexpr int kDecWarps = 8;
-constexpr int kDecThreads = kDecWarps * 32;
-// 16-key blocks per warp per stage: two, except for 256-byte code rows (a
-// stage of 256 such keys would not fit in shared memory)
-__host__ __device__ constexpr int dec_sub(int D, int bits) { return D * bits / 8 >= 256 ? 1 : 2; }
+// 8 warps per CTA; two CTAs per SM for D <= 128 (independent CTAs overlap
+// each other's stage boundaries), one for D = 256 (more registers per thread).
+__host__ __device__ constexpr int dec_warps(int) { return 8; }
+__host__ __device__ constexpr int dec_ctas_per_sm(int D) { return D <= 128 ? 2 : 1; }
 
 // XOR coefficients (3 bits each, for line bits 0..3) of the 16-byte-unit
 // swizzle inside each 128-byte line of a staged code tile, found by exhaustive
@@ -98,22 +97,26 @@ struct DecCfg {
   static constexpr int CW = CB >= 4 ? CB / 4 : 1;
   static constexpr int NMETA = Q8 ? 2 : 4;
   static constexpr int MROW = NG * 2;          // meta bytes per key per array
-  static constexpr int WPC = kDecWarps / NC;   // warps per head chunk
-  static constexpr int SUB = dec_sub(D, BITS);   // 16-key blocks per warp per stage
+  static constexpr int NWARP = dec_warps(D);
+  static constexpr int NTHR = 32 * NWARP;
+  static constexpr int WPC = NWARP / NC;       // warps per head chunk
+  // ring budget per CTA (228 KB per SM holds two CTAs of 108 KB plus their
+  // reserved 1 KB each)
+  static constexpr int BUDGET = D <= 128 ? 110592 : 224 * 1024;
+  // 16-key blocks per warp per stage: two when three such stages fit, else one
+  static constexpr int STAGE2 = 2 * (32 * WPC) * RB + NMETA * (((32 * WPC * MROW + 127) / 128) * 128);
+  static constexpr int SUB = 3 * STAGE2 <= BUDGET ? 2 : 1;
   static constexpr int TK = 16 * SUB * WPC;      // keys per stage
   static constexpr int CODES = TK * RB;
   static constexpr int META = ((TK * MROW + 127) / 128) * 128;
   static constexpr int META_UNITS = TK * MROW / 16;
   static constexpr int STAGE = 2 * CODES + NMETA * META;
-  // two CTAs per SM for D <= 128 (one for D = 256): shared-memory budget per CTA
-  // (228 KB per SM holds two CTAs of 108 KB plus their reserved 1 KB each)
-  static constexpr int BUDGET = D <= 128 ? 110592 - NC * 8 * D * 4 : 190 * 1024;
   static constexpr int NSTAGE = BUDGET / STAGE > 6 ? 6 : (BUDGET / STAGE < 2 ? 2 : BUDGET / STAGE);
-  // epilogue: per-warp partial rows, then the merge scratch (<= 48 parts)
-  static constexpr int EPI = kDecWarps * (8 * D + 16) * 4 + (48 * 32 * 2 + 2 * 32 + 48) * 4;
+  // epilogue: per-warp partial rows
+  static constexpr int EPI = NWARP * (8 * D + 16) * 4;
   static constexpr int RING = NSTAGE * STAGE > EPI ? NSTAGE * STAGE : EPI;
-  static constexpr int QS_OFF = RING;                 // fp32 query rows of the CTA
-  static constexpr int SMEM = RING + NC * 8 * D * 4;
+  static constexpr int QSB = NC * 8 * D * 4;            // fp32 query rows (in the last ring slot)
+  static constexpr int SMEM = RING > (NSTAGE - 1) * STAGE + QSB ? RING : (NSTAGE - 1) * STAGE + QSB;
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
   static constexpr uint32_t SWZ = swizzle_coeffs(D, BITS, GS);
   static_assert(D % GS == 0, "D must be a multiple of the group size");
@@ -148,84 +151,91 @@ __device__ __forceinline__ void lds_meta(const uint8_t* p, uint16_t* h) {
   }
 }
 
-constexpr int kMergeGroup = 8;
+constexpr int kMergeBatch = 16;   // parts whose loads one merging thread has in flight
+constexpr int kMergeGroup = 8;    // parts per first-level merge when a unit merges in two levels
+constexpr int64_t kMergeFlat = 1 << 15;   // largest parts x rows x D merged by one CTA in one level
 
-// Combines n partial results (m, l, o) of one unit, read from the slots
-// slot(0..n-1), by log-sum-exp rescaling.  Writes either the normalized output
-// (out != nullptr; rows hbase.. of the unit starting at element out_base) or
-// a combined partial (dst_ml/dst_o).  The weights are computed once in shared
-// memory so every thread then issues independent loads of the o parts.
-template <int D, int HPC, class SlotFn>
-__device__ __forceinline__ void merge_parts(const float* ml, const float* po, int n, SlotFn slot,
-                                            float* sm, int tid, int hbase, int G,
-                                            float* dst_ml, float* dst_o, void* out, int out_dtype,
-                                            int64_t out_base) {
-  float* w = sm;                                   // [n][HPC] weights (m first)
-  float* lw = sm + n * HPC;                        // [n][HPC] partial sums
-  float* hm = lw + n * HPC;                        // [HPC] max, then combined sum
-  int* sl = reinterpret_cast<int*>(hm + 2 * HPC);  // [n] slots
-  for (int i = tid; i < n; i += kDecThreads) sl[i] = (int)slot(i);
-  __syncthreads();
-  for (int i = tid; i < n * HPC; i += kDecThreads) {
-    const int pp = i / HPC, hl = i - pp * HPC;
-    w[i] = __ldcg(&ml[((int64_t)sl[pp] * HPC + hl) * 2 + 0]);
-    lw[i] = __ldcg(&ml[((int64_t)sl[pp] * HPC + hl) * 2 + 1]);
-  }
-  __syncthreads();
-  for (int hl = tid; hl < HPC; hl += kDecThreads) {
-    float M = -INFINITY;
-    for (int pp = 0; pp < n; ++pp) M = fmaxf(M, w[pp * HPC + hl]);
-    float l = 0.f;
-    for (int pp = 0; pp < n; ++pp) {
-      const float m = w[pp * HPC + hl];
-      const float sc = m == -INFINITY ? 0.f : ex2(m - M);
-      w[pp * HPC + hl] = sc;
-      l = fmaf(sc, lw[pp * HPC + hl], l);
-    }
-    hm[hl] = M;
-    hm[HPC + hl] = l;
-  }
-  __syncthreads();
-  // four consecutive outputs per step, up to 8 parts' loads in flight
+// Combines n partial results (m, l, o) of one unit by log-sum-exp rescaling.
+// Part i lives in slot 2 * (c0 + i * step), except part 0, which is in slot0.
+// Writes either the nrows normalized rows starting at element out_base
+// (dst_o == nullptr) or one combined partial (dst_ml, dst_o).  A thread owns 4
+// consecutive outputs of one row and every tpi-th part; it loads (m, l) and o
+// of a batch of parts at once and folds them in online, then the tpi threads
+// of an output (adjacent lanes) combine with shuffles: one round trip per
+// batch and no barrier.
+template <int D, int HPC>
+__device__ __noinline__ void merge_unit(const float* ml, const float* po, int n, int64_t slot0,
+                                        int64_t c0, int step, int tid, int nthreads, int nrows,
+                                        void* out, int out_dtype, int64_t out_base, float* dst_ml,
+                                        float* dst_o) {
   constexpr int V4 = D / 4;
-  for (int idx = tid; idx < HPC * V4; idx += kDecThreads) {
-    const int hl = idx / V4, e4 = idx - hl * V4;
-    if (hbase + hl >= G) continue;
+  const int items = nrows * V4;
+  int tpi = 1;
+  while (tpi < 32 && items * tpi * 2 <= nthreads) tpi *= 2;
+  const int ipp = nthreads / tpi;                                 // items per pass
+  const int sub = tid & (tpi - 1);
+  for (int i0 = 0; i0 < items; i0 += ipp) {
+    const int item = i0 + tid / tpi;
+    const bool active = item < items;
+    const int hl = active ? item / V4 : 0, e4 = active ? item - hl * V4 : 0;
+    float M = -INFINITY, Ls = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int p0 = 0; p0 < n; p0 += 8) {
-      float4 o[8];
-      float wv[8];
+    for (int jb = 0; sub + tpi * jb < n; jb += kMergeBatch) {
+      float4 o[kMergeBatch];
+      float2 v[kMergeBatch];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int pp = p0 + u;
-        if (pp < n) {
-          o[u] = __ldcg(reinterpret_cast<const float4*>(po + ((int64_t)sl[pp] * HPC + hl) * D) + e4);
-          wv[u] = w[pp * HPC + hl];
+      for (int k = 0; k < kMergeBatch; ++k) {
+        const int pp = sub + tpi * (jb + k);
+        if (active && pp < n) {
+          const int64_t sx = pp == 0 ? slot0 : 2 * (c0 + (int64_t)pp * step);
+          o[k] = __ldcg(reinterpret_cast<const float4*>(po + (sx * HPC + hl) * D) + e4);
+          v[k] = __ldcg(reinterpret_cast<const float2*>(ml + (sx * HPC + hl) * 2));
         } else {
-          o[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-          wv[u] = 0.f;
+          o[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+          v[k] = make_float2(-INFINITY, 0.f);
         }
       }
+      float Mb = M;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        acc.x = fmaf(wv[u], o[u].x, acc.x);
-        acc.y = fmaf(wv[u], o[u].y, acc.y);
-        acc.z = fmaf(wv[u], o[u].z, acc.z);
-        acc.w = fmaf(wv[u], o[u].w, acc.w);
+      for (int k = 0; k < kMergeBatch; ++k) Mb = fmaxf(Mb, v[k].x);
+      if (Mb != M) {
+        const float f = M == -INFINITY ? 0.f : ex2(M - Mb);
+        Ls *= f; acc.x *= f; acc.y *= f; acc.z *= f; acc.w *= f;
+        M = Mb;
+      }
+#pragma unroll
+      for (int k = 0; k < kMergeBatch; ++k) {
+        const float w = v[k].x == -INFINITY ? 0.f : ex2(v[k].x - M);
+        Ls = fmaf(w, v[k].y, Ls);
+        acc.x = fmaf(w, o[k].x, acc.x);
+        acc.y = fmaf(w, o[k].y, acc.y);
+        acc.z = fmaf(w, o[k].z, acc.z);
+        acc.w = fmaf(w, o[k].w, acc.w);
       }
     }
-    const float l = hm[HPC + hl];
-    const int e = e4 * 4;
-    if (out != nullptr) {
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      const int64_t oi = out_base + (int64_t)(hbase + hl) * D + e;
-      store_from_float(out, out_dtype, oi, acc.x * inv);
-      store_from_float(out, out_dtype, oi + 1, acc.y * inv);
-      store_from_float(out, out_dtype, oi + 2, acc.z * inv);
-      store_from_float(out, out_dtype, oi + 3, acc.w * inv);
-    } else {
-      *reinterpret_cast<float4*>(dst_o + hl * D + e) = acc;
-      if (e == 0) { dst_ml[hl * 2] = hm[hl]; dst_ml[hl * 2 + 1] = l; }
+    for (int off = 1; off < tpi; off <<= 1) {
+      const float M2 = __shfl_xor_sync(~0u, M, off), L2 = __shfl_xor_sync(~0u, Ls, off);
+      const float x2 = __shfl_xor_sync(~0u, acc.x, off), y2 = __shfl_xor_sync(~0u, acc.y, off);
+      const float z2 = __shfl_xor_sync(~0u, acc.z, off), w2 = __shfl_xor_sync(~0u, acc.w, off);
+      const float Mn = fmaxf(M, M2);
+      const float f1 = M == -INFINITY ? 0.f : ex2(M - Mn), f2 = M2 == -INFINITY ? 0.f : ex2(M2 - Mn);
+      Ls = Ls * f1 + L2 * f2;
+      acc.x = acc.x * f1 + x2 * f2; acc.y = acc.y * f1 + y2 * f2;
+      acc.z = acc.z * f1 + z2 * f2; acc.w = acc.w * f1 + w2 * f2;
+      M = Mn;
+    }
+    if (active && sub == 0) {
+      if (dst_o != nullptr) {
+        *reinterpret_cast<float4*>(dst_o + hl * D + e4 * 4) = acc;
+        if (e4 == 0) { dst_ml[hl * 2] = M; dst_ml[hl * 2 + 1] = Ls; }
+      } else {
+        const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+        const int64_t oi = out_base + (int64_t)hl * D + e4 * 4;
+        store_from_float(out, out_dtype, oi, acc.x * inv);
+        store_from_float(out, out_dtype, oi + 1, acc.y * inv);
+        store_from_float(out, out_dtype, oi + 2, acc.z * inv);
+        store_from_float(out, out_dtype, oi + 3, acc.w * inv);
+      }
     }
   }
 }
@@ -263,14 +273,13 @@ __device__ __forceinline__ void meta_row(const uint8_t* base, int r, uint32_t* w
 }
 
 template <int D, int BITS, int GS, bool Q8, int NC, bool F32OUT>
-__global__ void __launch_bounds__(kDecThreads, D <= 128 ? 2 : 1)
+__global__ void __launch_bounds__(32 * dec_warps(D), dec_ctas_per_sm(D))
 qsdpa_decode_kernel(const DecodeParams p) {
   using C = DecCfg<D, BITS, GS, Q8, NC>;
   constexpr int NG = C::NG, KPG = C::KPG, MT = C::MT, TK = C::TK, NSTAGE = C::NSTAGE;
   constexpr int HPC = NC * 8;
   constexpr int MW = NG == 1 ? 1 : NG / 2;     // 32-bit words of one key's metadata row
   extern __shared__ __align__(128) uint8_t smem[];
-  float* qst = reinterpret_cast<float*>(smem + C::QS_OFF);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
@@ -293,37 +302,116 @@ qsdpa_decode_kernel(const DecodeParams p) {
     const int64_t row0 = ((int64_t)b * p.Hkv + hkv) * p.Lcap;   // first cache row of this head
     const int hbase = cg * HPC;                                  // first local row of the CTA
 
-    // ---------------- query rows -> shared memory (fp32), 16-byte loads --------
+    const uint8_t* gK = p.kc + row0 * C::RB;
+    const uint8_t* gV = p.vc + row0 * C::RB;
+    const uint8_t* gKs = reinterpret_cast<const uint8_t*>(p.ks + row0 * NG);
+    const uint8_t* gKb = Q8 ? gKs : reinterpret_cast<const uint8_t*>(p.kb + row0 * NG);
+    const uint8_t* gVs = reinterpret_cast<const uint8_t*>(p.vs + row0 * NG);
+    const uint8_t* gVb = Q8 ? gVs : reinterpret_cast<const uint8_t*>(p.vb + row0 * NG);
+    const int64_t L = p.L;
+
+    // copy plan: 16-byte unit i of a stage is row (i mod CU) / UPR of the K
+    // tile (i < CU) or of the V tile.  When CU is a multiple of the thread
+    // count every unit of a thread lies in a line with the same swizzle.
+    constexpr int CU = TK * C::UPR;
+    constexpr int NU = (2 * CU + C::NTHR - 1) / C::NTHR;
+    const int fx_tid = swz_line<C::SWZ>((tid >> 3) & 15);
+
+    auto issue_stage = [&](int stage, int buf) {
+      const uint32_t sbase = smem_u32(smem + buf * C::STAGE);
+      const int64_t key0 = (int64_t)stage * TK;
+      const int nvalid = (int)(L - key0 < (int64_t)TK ? L - key0 : (int64_t)TK);      // rows of this stage below L
+      const uint8_t* kb0 = gK + key0 * C::RB;
+      const uint8_t* vb0 = gV + key0 * C::RB;
+#pragma unroll
+      for (int k = 0; k < NU; ++k) {
+        const int i = tid + k * C::NTHR;
+        if ((2 * CU) % C::NTHR == 0 || i < 2 * CU) {
+          const int which = i >= CU, j = which ? i - CU : i;
+          const bool ok = (j / C::UPR) < nvalid;
+          const uint8_t* src = (which ? vb0 : kb0) + (ok ? j * 16 : 0);
+          const int dst = (CU % C::NTHR == 0) ? which * C::CODES + ((j * 16) ^ fx_tid)
+                                                  : which * C::CODES + swz_offset<C::SWZ>(j * 16);
+          cp_async16(sbase + dst, src, ok ? 16 : 0);
+        }
+      }
+      for (int i = tid; i < C::NMETA * C::META_UNITS; i += C::NTHR) {
+        const int arr = i / C::META_UNITS, j = i - arr * C::META_UNITS;
+        // affine: K scales, K biases, V scales, V biases; Q8_0: K scales, V scales
+        const uint8_t* gm = Q8 ? (arr == 0 ? gKs : gVs)
+                               : (arr == 0 ? gKs : arr == 1 ? gKb : arr == 2 ? gVs : gVb);
+        const bool ok = (j * 16) / C::MROW < nvalid;
+        const uint8_t* src = gm + (ok ? key0 * C::MROW + j * 16 : 0);
+        cp_async16(sbase + 2 * C::CODES + arr * C::META + j * 16, src, ok ? 16 : 0);
+      }
+    };
+
+    // fragment offsets inside a stage (fixed per lane).  The swizzle is
+    // linear in the line bits and a group never straddles a line, so it splits
+    // into a per-row part (computed once here), a per-group constant and, for
+    // the second 16-key block, the constant of a 16-row shift.
+    const int k0 = sub * 16 * C::SUB;
+    auto row_x = [&](int r) { return swz_line<C::SWZ>((r * C::RB) >> 7); };
+    const int xk0 = row_x(k0 + g), xk1 = row_x(k0 + g + 8);
+    const int xva = row_x(k0 + 2 * t), xvb = row_x(k0 + 2 * t + 1);
+    const int xvc = row_x(k0 + 2 * t + 8), xvd = row_x(k0 + 2 * t + 9);
+    auto koff = [&](int r, int x, int st, int G, int part) {
+      return ((r * C::RB + G * C::GB + t * C::NW * 4 + part * 16) ^ x) ^
+             swz_line<C::SWZ>((G * C::GB) >> 7) ^ swz_line<C::SWZ>((st * 16 * C::RB) >> 7);
+    };
+    auto voff = [&](int r, int x, int st, int G) {
+      return ((r * C::RB + G * C::GB + g * C::CB) ^ x) ^ swz_line<C::SWZ>((G * C::GB) >> 7) ^
+             swz_line<C::SWZ>((st * 16 * C::RB) >> 7);
+    };
+
+    const int nst = s1 - s0;
+    // query rows: their (small) loads go out first, then the copies of the
+    // first stages; the rows are staged as fp32 in the ring's last slot, which
+    // the first NSTAGE-1 stages do not use
+    float* qst = reinterpret_cast<float*>(smem + (NSTAGE - 1) * C::STAGE);
+    constexpr int QCH = HPC * D / 8;                      // 16-byte query chunks
+    constexpr int QPT = (QCH + C::NTHR - 1) / C::NTHR;
+    uint4 qraw[QPT];
     {
       const int64_t qbase = (((int64_t)b * p.Hkv + hkv) * p.G + hbase) * D;
       const int nrows = min(HPC, p.G - hbase);
-      for (int i = tid; i < HPC * D / 8; i += kDecThreads) {
+#pragma unroll
+      for (int k = 0; k < QPT; ++k) {
+        const int i = tid + k * C::NTHR;
         const int hl = i / (D / 8), c = i - hl * (D / 8);
+        qraw[k] = make_uint4(0u, 0u, 0u, 0u);
+        if (i < QCH && hl < nrows)
+          qraw[k] = __ldg(reinterpret_cast<const uint4*>(
+              reinterpret_cast<const uint16_t*>(p.q) + qbase + (int64_t)hl * D + c * 8));
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < NSTAGE - 1; ++i) {
+      if (i < nst) issue_stage(s0 + i, i);
+      cp_async_commit();
+    }
+#pragma unroll
+    for (int k = 0; k < QPT; ++k) {
+      const int i = tid + k * C::NTHR;
+      if (QCH % C::NTHR == 0 || i < QCH) {
+        const uint32_t w[4] = {qraw[k].x, qraw[k].y, qraw[k].z, qraw[k].w};
         float v[8];
-        if (hl < nrows) {
-          const uint4 raw = *reinterpret_cast<const uint4*>(
-              reinterpret_cast<const uint16_t*>(p.q) + qbase + (int64_t)hl * D + c * 8);
-          const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            if (p.q_dtype == QKV_F16) {
-              const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
-              v[2 * k] = f.x; v[2 * k + 1] = f.y;
-            } else {
-              v[2 * k] = __uint_as_float(w[k] << 16);
-              v[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
-            }
+        for (int j = 0; j < 4; ++j) {
+          if (p.q_dtype == QKV_F16) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[j]));
+            v[2 * j] = f.x; v[2 * j + 1] = f.y;
+          } else {
+            v[2 * j] = __uint_as_float(w[j] << 16);
+            v[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
           }
-        } else {
-#pragma unroll
-          for (int k = 0; k < 8; ++k) v[k] = 0.f;
         }
-        float4* dst = reinterpret_cast<float4*>(qst + hl * D + c * 8);
+        float4* dst = reinterpret_cast<float4*>(qst + i * 8);
         dst[0] = make_float4(v[0], v[1], v[2], v[3]);
         dst[1] = make_float4(v[4], v[5], v[6], v[7]);
       }
-      __syncthreads();
     }
+    __syncthreads();
 
     // ---------------- query fragments (B operand of the score MMA) ----------
     uint32_t bq[C::KSTEPS][2];
@@ -389,75 +477,6 @@ qsdpa_decode_kernel(const DecodeParams p) {
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) { O[mt][0] = O[mt][1] = O[mt][2] = O[mt][3] = 0.f; }
 
-    const uint8_t* gK = p.kc + row0 * C::RB;
-    const uint8_t* gV = p.vc + row0 * C::RB;
-    const uint8_t* gKs = reinterpret_cast<const uint8_t*>(p.ks + row0 * NG);
-    const uint8_t* gKb = Q8 ? gKs : reinterpret_cast<const uint8_t*>(p.kb + row0 * NG);
-    const uint8_t* gVs = reinterpret_cast<const uint8_t*>(p.vs + row0 * NG);
-    const uint8_t* gVb = Q8 ? gVs : reinterpret_cast<const uint8_t*>(p.vb + row0 * NG);
-    const int64_t L = p.L;
-
-    // copy plan: 16-byte unit i of a stage is row (i mod CU) / UPR of the K
-    // tile (i < CU) or of the V tile.  When CU is a multiple of the thread
-    // count every unit of a thread lies in a line with the same swizzle.
-    constexpr int CU = TK * C::UPR;
-    constexpr int NU = (2 * CU + kDecThreads - 1) / kDecThreads;
-    const int fx_tid = swz_line<C::SWZ>((tid >> 3) & 15);
-
-    auto issue_stage = [&](int stage, int buf) {
-      const uint32_t sbase = smem_u32(smem + buf * C::STAGE);
-      const int64_t key0 = (int64_t)stage * TK;
-      const int nvalid = (int)(L - key0 < (int64_t)TK ? L - key0 : (int64_t)TK);      // rows of this stage below L
-      const uint8_t* kb0 = gK + key0 * C::RB;
-      const uint8_t* vb0 = gV + key0 * C::RB;
-#pragma unroll
-      for (int k = 0; k < NU; ++k) {
-        const int i = tid + k * kDecThreads;
-        if ((2 * CU) % kDecThreads == 0 || i < 2 * CU) {
-          const int which = i >= CU, j = which ? i - CU : i;
-          const bool ok = (j / C::UPR) < nvalid;
-          const uint8_t* src = (which ? vb0 : kb0) + (ok ? j * 16 : 0);
-          const int dst = (CU % kDecThreads == 0) ? which * C::CODES + ((j * 16) ^ fx_tid)
-                                                  : which * C::CODES + swz_offset<C::SWZ>(j * 16);
-          cp_async16(sbase + dst, src, ok ? 16 : 0);
-        }
-      }
-      for (int i = tid; i < C::NMETA * C::META_UNITS; i += kDecThreads) {
-        const int arr = i / C::META_UNITS, j = i - arr * C::META_UNITS;
-        // affine: K scales, K biases, V scales, V biases; Q8_0: K scales, V scales
-        const uint8_t* gm = Q8 ? (arr == 0 ? gKs : gVs)
-                               : (arr == 0 ? gKs : arr == 1 ? gKb : arr == 2 ? gVs : gVb);
-        const bool ok = (j * 16) / C::MROW < nvalid;
-        const uint8_t* src = gm + (ok ? key0 * C::MROW + j * 16 : 0);
-        cp_async16(sbase + 2 * C::CODES + arr * C::META + j * 16, src, ok ? 16 : 0);
-      }
-    };
-
-    // fragment offsets inside a stage (fixed per lane).  The swizzle is
-    // linear in the line bits and a group never straddles a line, so it splits
-    // into a per-row part (computed once here), a per-group constant and, for
-    // the second 16-key block, the constant of a 16-row shift.
-    const int k0 = sub * 16 * C::SUB;
-    auto row_x = [&](int r) { return swz_line<C::SWZ>((r * C::RB) >> 7); };
-    const int xk0 = row_x(k0 + g), xk1 = row_x(k0 + g + 8);
-    const int xva = row_x(k0 + 2 * t), xvb = row_x(k0 + 2 * t + 1);
-    const int xvc = row_x(k0 + 2 * t + 8), xvd = row_x(k0 + 2 * t + 9);
-    auto koff = [&](int r, int x, int st, int G, int part) {
-      return ((r * C::RB + G * C::GB + t * C::NW * 4 + part * 16) ^ x) ^
-             swz_line<C::SWZ>((G * C::GB) >> 7) ^ swz_line<C::SWZ>((st * 16 * C::RB) >> 7);
-    };
-    auto voff = [&](int r, int x, int st, int G) {
-      return ((r * C::RB + G * C::GB + g * C::CB) ^ x) ^ swz_line<C::SWZ>((G * C::GB) >> 7) ^
-             swz_line<C::SWZ>((st * 16 * C::RB) >> 7);
-    };
-
-    const int nst = s1 - s0;
-#pragma unroll
-    for (int i = 0; i < NSTAGE - 1; ++i) {
-      if (i < nst) issue_stage(s0 + i, i);
-      cp_async_commit();
-    }
-
     for (int it = 0; it < nst; ++it) {
       cp_async_wait<NSTAGE - 2>();
       __syncthreads();
@@ -472,7 +491,7 @@ qsdpa_decode_kernel(const DecodeParams p) {
       if (kvalid < TK) {
         // keys past L: clear their (possibly stale) scales and biases
         uint16_t* meta = reinterpret_cast<uint16_t*>(sb + 2 * C::CODES);
-        for (int i = tid; i < C::NMETA * TK * NG; i += kDecThreads) {
+        for (int i = tid; i < C::NMETA * TK * NG; i += C::NTHR) {
           const int arr = i / (TK * NG), r = i - arr * TK * NG;
           if (r / NG >= kvalid) meta[arr * (C::META / 2) + r] = 0;
         }
@@ -754,7 +773,7 @@ qsdpa_decode_kernel(const DecodeParams p) {
     const bool complete = (s0 == 0) && (s1 == (int)S);
     const int64_t slot = 2 * (int64_t)blockIdx.x + (u == first_unit ? 0 : 1);
     const float* wsf = reinterpret_cast<const float*>(smem);
-    for (int idx = tid; idx < HPC * D; idx += kDecThreads) {
+    for (int idx = tid; idx < HPC * D; idx += C::NTHR) {
       const int hl = idx / D, e = idx - hl * D;       // hl: head within the chunk-group
       const int c = hl >> 3, hh = hl & 7;
       const int head = hbase + hl;
@@ -787,23 +806,23 @@ qsdpa_decode_kernel(const DecodeParams p) {
     }
 
     if (!complete) {
-      // Merge tree without waiting: the last CTA of each group of kMergeGroup
-      // consecutive parts merges that group into a level-2 partial; the last
-      // group merger of the unit merges the level-2 partials into the output.
-      // (With at most kMergeGroup parts the first level writes the output.)
+      // The unit's partials are merged by the last of its CTAs to finish
+      // (atomic ticket), in one level when their volume is small, else in two:
+      // the last CTA of each group of kMergeGroup consecutive CTAs merges the
+      // group into a second-level partial and the last group merger merges
+      // those.  Nobody waits on anybody.
       __threadfence();
       __syncthreads();
       const int64_t cfirst = ((u * S + 1) * nC - 1) / T;
       const int64_t clast = (((u + 1) * S) * nC - 1) / T;
       const int nparts = (int)(clast - cfirst + 1);
-      const int ngroups = (nparts + kMergeGroup - 1) / kMergeGroup;
-      const int pi = (int)((int64_t)blockIdx.x - cfirst);
-      const int gi = pi / kMergeGroup;
-      auto slot_of = [&](int64_t c) {      // level-1 slot of CTA c for unit u
-        return 2 * c + (((c * T / nC) / S) == u ? 0 : 1);
-      };
-      float* sm = reinterpret_cast<float*>(smem) + kDecWarps * (8 * D + 16);
-      if (ngroups == 1) {
+      const int nrows = min(HPC, p.G - hbase);
+      // slot of the unit's first CTA: its second slot if it began in an
+      // earlier unit; every later CTA of the unit began in this one
+      const int64_t slot0 = 2 * cfirst + ((cfirst * T / nC) / S == u ? 0 : 1);
+      auto slot_of = [&](int64_t c) -> int64_t { return c == cfirst ? slot0 : 2 * c; };
+      const int64_t out_base = (((int64_t)b * p.Hkv + hkv) * p.G + hbase) * D;
+      if ((int64_t)nparts * nrows * D <= kMergeFlat) {
         if (tid == 0) {
           const unsigned prev = atomicAdd(&p.tickets[u], 1u);
           const int last = prev == (unsigned)nparts - 1;
@@ -813,12 +832,14 @@ qsdpa_decode_kernel(const DecodeParams p) {
         __syncthreads();
         if (s_flag) {
           __threadfence();
-          merge_parts<D, HPC>(p.part_ml, p.part_o, nparts, [&](int i) { return slot_of(cfirst + i); },
-                              sm, tid, hbase, p.G, nullptr, nullptr,
-                              p.out, p.out_dtype, (((int64_t)b * p.Hkv + hkv) * p.G) * D);
+          merge_unit<D, HPC>(p.part_ml, p.part_o, nparts, slot0, cfirst, 1, tid, C::NTHR, nrows,
+                             p.out, p.out_dtype, out_base, nullptr, nullptr);
         }
       } else {
-        const int64_t lead = slot_of(cfirst + (int64_t)gi * kMergeGroup);   // group's id
+        const int ngroups = (nparts + kMergeGroup - 1) / kMergeGroup;
+        const int gi = (int)((int64_t)blockIdx.x - cfirst) / kMergeGroup;
+        const int64_t c0 = cfirst + (int64_t)gi * kMergeGroup;
+        const int64_t lead = slot_of(c0);                       // the group's second-level slot
         const int gsz = min(kMergeGroup, nparts - gi * kMergeGroup);
         if (tid == 0) {
           const unsigned prev = atomicAdd(&p.tickets1[lead], 1u);
@@ -829,10 +850,8 @@ qsdpa_decode_kernel(const DecodeParams p) {
         __syncthreads();
         if (s_flag) {
           __threadfence();
-          const int64_t c0 = cfirst + (int64_t)gi * kMergeGroup;
-          merge_parts<D, HPC>(p.part_ml, p.part_o, gsz, [&](int i) { return slot_of(c0 + i); },
-                              sm, tid, hbase, p.G, p.part2_ml + lead * HPC * 2,
-                              p.part2_o + lead * HPC * D, nullptr, 0, 0);
+          merge_unit<D, HPC>(p.part_ml, p.part_o, gsz, lead, c0, 1, tid, C::NTHR, nrows,
+                             nullptr, 0, 0, p.part2_ml + lead * HPC * 2, p.part2_o + lead * HPC * D);
           __threadfence();
           __syncthreads();
           if (tid == 0) {
@@ -844,10 +863,8 @@ qsdpa_decode_kernel(const DecodeParams p) {
           __syncthreads();
           if (s_flag) {
             __threadfence();
-            merge_parts<D, HPC>(p.part2_ml, p.part2_o, ngroups,
-                                [&](int i) { return slot_of(cfirst + (int64_t)i * kMergeGroup); },
-                                sm, tid, hbase, p.G, nullptr, nullptr,
-                                p.out, p.out_dtype, (((int64_t)b * p.Hkv + hkv) * p.G) * D);
+            merge_unit<D, HPC>(p.part2_ml, p.part2_o, ngroups, slot0, cfirst, kMergeGroup, tid,
+                               C::NTHR, nrows, p.out, p.out_dtype, out_base, nullptr, nullptr);
           }
         }
       }
@@ -867,7 +884,7 @@ struct DecodeInstance {
       if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
         return 0;
       int n = 0;
-      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, kDecThreads, C::SMEM) != cudaSuccess)
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, C::NTHR, C::SMEM) != cudaSuccess)
         return 0;
       cached = n;
     }
@@ -875,7 +892,7 @@ struct DecodeInstance {
   }
   static cudaError_t launch(const DecodePlan& plan, const DecodeParams& p, cudaStream_t s) {
     auto k = qsdpa_decode_kernel<D, BITS, GS, Q8, NC, F32OUT>;
-    k<<<plan.grid, kDecThreads, C::SMEM, s>>>(p);
+    k<<<plan.grid, C::NTHR, C::SMEM, s>>>(p);
     return cudaGetLastError();
   }
 };

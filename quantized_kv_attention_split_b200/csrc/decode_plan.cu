@@ -8,9 +8,8 @@ namespace qkv {
 namespace {
 
 // Grid cap per SM used both for planning and for the workspace bound, so that
-// qsdpa_workspace_size() does not depend on the kernel instance: the D <= 128
-// kernels are built for two resident CTAs per SM, the D = 256 ones for one.
-int max_ctas_per_sm(int D) { return D <= 128 ? 2 : 1; }
+// qsdpa_workspace_size() does not depend on the kernel instance.
+int max_ctas_per_sm(int D) { return dec_ctas_per_sm(D); }
 // Largest grid: the merge tree's second level then has at most 48 groups of 8.
 constexpr int64_t kMaxGrid = 8 * 48;
 
