@@ -98,7 +98,9 @@ typedef struct {
  *   Q8_0:   d = max|x|/127; scale = fp16_rne(d);
  *           code = scale == 0 ? 0 : clamp(rint(x/scale), -127, 127)
  *  The result is bit-identical to the CPU oracle.  Requires
- *  0 <= offset <= Lcap - Lnew.  k and v may use different formats. */
+ *  0 <= offset <= Lcap - Lnew and B*Hkv <= 65535 (QKV_ERR_UNSUPPORTED
+ *  otherwise).  k and v may use different formats (then K and V are two
+ *  launches, else one). */
 qkv_status qkv_quantize_update(const void* new_k, const void* new_v, int in_dtype,
                                int B, int Hkv, int Lnew, int D,
                                const qkv_cache* k, const qkv_cache* v,

@@ -230,6 +230,8 @@ qkv_status qkv_quantize_update(const void* new_k, const void* new_v, int in_dtyp
   if ((st = check_cache("v", v, D)) != QKV_OK) return st;
   if (in_dtype != QKV_F16 && in_dtype != QKV_BF16)
     return fail(QKV_ERR_INVALID_ARG, "new tokens must be f16 or bf16 (got %d)", in_dtype);
+  if ((int64_t)B * Hkv > 65535)
+    return fail(QKV_ERR_UNSUPPORTED, "B * Hkv must be at most 65535 (got %lld)", (long long)B * Hkv);
   if (Lnew == 0) return ok();
   if (new_k == nullptr || new_v == nullptr)
     return fail(QKV_ERR_INVALID_ARG, "new_k and new_v must be non-NULL");

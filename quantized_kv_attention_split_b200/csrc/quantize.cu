@@ -13,8 +13,9 @@
 // Design: one thread owns 8 consecutive elements (one 16-byte load), the
 // gs/8 lanes of a group reduce min/max with shuffles, each thread packs its 8
 // codes into one (4-bit) or two (8-bit) words and stores them; the first lane
-// of a group stores the fp16 scale (and bias).  K and V are handled by the two
-// halves of the grid's y dimension.
+// of a group stores the fp16 scale (and bias).  Grid: x = blocks of tokens
+// (256 / (D/8) tokens per block), y = (batch, kv head) slab, z = K or V (one
+// launch when both caches have the same format), so no thread divides.
 #include <algorithm>
 
 #include "qkv_common.cuh"
@@ -23,25 +24,39 @@
 namespace qkv {
 
 struct QuantSide {
-  const uint16_t* src;      // [rows, D] fp16/bf16 bits
+  const uint16_t* src;      // [B * Hkv * Lnew, D] fp16/bf16 bits
   uint32_t* codes;          // cache codes base
   uint16_t* scales;
   uint16_t* biases;
-  int fmt, bits, gs;
+  int64_t Lcap;
 };
 
 struct QuantParams {
   QuantSide side[2];
-  int in_dtype;
   int D;
-  int64_t rows;             // B * Hkv * Lnew
+  int row_shift;            // log2(D / 8): threads per token row
   int Lnew;
-  int64_t Lcap, offset;
+  int64_t offset;
 };
 
-__device__ __forceinline__ float load_in(const uint16_t* p, int dtype, int64_t i) {
-  return dtype == QKV_F16 ? __half2float(__ushort_as_half(p[i]))
-                          : __bfloat162float(__ushort_as_bfloat16(p[i]));
+template <bool BF16>
+__device__ __forceinline__ float in_to_float(uint16_t b) {
+  if constexpr (BF16) return __uint_as_float((uint32_t)b << 16);
+  else return __half2float(__ushort_as_half(b));
+}
+
+// rint(RN(d / s)) -- the code decision of the quantizer -- without a division
+// in the common case.  With r = RN(1/s), q0 = RN(d * r) is within 2^-14 of
+// RN(d / s) whenever |q0| < 2^9 (two roundings of relative error 2^-24 each),
+// so both round to the same integer unless q0 lies within 2^-13 of a
+// half-integer; that rare case, and any |q0| >= 2^9 or non-finite value, takes
+// the correctly rounded division, so the result is always identical to it.
+__device__ __forceinline__ int div_rint(float d, float s, float r) {
+  const float q0 = __fmul_rn(d, r);
+  const float n = rintf(q0);
+  if (!(fabsf(q0) < 512.f) || fabsf(fabsf(__fsub_rn(q0, n)) - 0.5f) < 0x1p-13f)
+    return __float2int_rn(__fdiv_rn(d, s));
+  return (int)n;
 }
 
 template <int LANES>
@@ -57,28 +72,30 @@ __device__ __forceinline__ float group_min(float v) {
   return v;
 }
 
-template <int GS, int BITS, bool Q8>
-__device__ __forceinline__ void quantize_item(const QuantParams& p, const QuantSide& s,
-                                              int64_t item, bool active) {
+template <int GS, int BITS, bool Q8, bool BF16>
+__global__ void __launch_bounds__(256) qkv_quantize_kernel(const QuantParams p, int side0) {
   constexpr int LANES = GS / 8;
-  const int per_row = p.D / 8;
-  const int64_t r = item / per_row;
-  const int c8 = (int)(item - r * per_row);        // which 8-element slice of the row
+  const QuantSide& s = (side0 + (int)blockIdx.z) ? p.side[1] : p.side[0];
+  const int per_row = p.D >> 3;
+  const int tok = blockIdx.x * (256 >> p.row_shift) + (threadIdx.x >> p.row_shift);
+  const int c8 = threadIdx.x & (per_row - 1);        // which 8-element slice of the row
+  const bool active = tok < p.Lnew;                 // inactive lanes still join the shuffles
+  const int64_t slab = blockIdx.y;                  // b * Hkv + kv head
+  const int64_t srow = slab * p.Lnew + (active ? tok : 0);
+  const int64_t crow = slab * s.Lcap + p.offset + tok;
   float x[8];
   if (active) {
-    const uint4 raw = *reinterpret_cast<const uint4*>(s.src + r * p.D + c8 * 8);
+    const uint4 raw = __ldg(reinterpret_cast<const uint4*>(s.src + srow * p.D + c8 * 8));
     const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint16_t lo = (uint16_t)(w[i] & 0xffff), hi = (uint16_t)(w[i] >> 16);
-      x[2 * i] = load_in(&lo, p.in_dtype, 0);
-      x[2 * i + 1] = load_in(&hi, p.in_dtype, 0);
+      x[2 * i] = in_to_float<BF16>((uint16_t)(w[i] & 0xffff));
+      x[2 * i + 1] = in_to_float<BF16>((uint16_t)(w[i] >> 16));
     }
   } else {
 #pragma unroll
     for (int i = 0; i < 8; ++i) x[i] = 0.f;
   }
-  const int64_t crow = (r / p.Lnew) * p.Lcap + p.offset + (r % p.Lnew);
   const int grp = (c8 * 8) / GS;
   const bool leader = ((c8 * 8) % GS) == 0;
   const int ng = p.D / GS;
@@ -90,12 +107,13 @@ __device__ __forceinline__ void quantize_item(const QuantParams& p, const QuantS
     const float d = __fdiv_rn(a, 127.f);
     const __half d16 = __float2half_rn(d);
     const float df = __half2float(d16);
+    const float rd = __frcp_rn(df);
     uint32_t w[2] = {0u, 0u};
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       int q = 0;
       if (df != 0.f) {
-        q = __float2int_rn(__fdiv_rn(x[i], df));
+        q = div_rint(x[i], df, rd);
         q = q < -127 ? -127 : (q > 127 ? 127 : q);
       }
       w[i >> 2] |= (uint32_t)(q & 0xff) << ((i & 3) * 8);
@@ -117,10 +135,11 @@ __device__ __forceinline__ void quantize_item(const QuantParams& p, const QuantS
     const __half s16 = __float2half_rn(sc);
     const __half b16 = __float2half_rn(mn);
     const float sf = __half2float(s16), bf = __half2float(b16);
+    const float rs = __frcp_rn(sf);
     uint32_t w[2] = {0u, 0u};
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      int q = __float2int_rn(__fdiv_rn(__fsub_rn(x[i], bf), sf));
+      int q = div_rint(__fsub_rn(x[i], bf), sf, rs);
       q = q < 0 ? 0 : (q > (1 << BITS) - 1 ? (1 << BITS) - 1 : q);
       if constexpr (BITS == 4) w[0] |= (uint32_t)q << (i * 4);
       else w[i >> 2] |= (uint32_t)q << ((i & 3) * 8);
@@ -139,41 +158,27 @@ __device__ __forceinline__ void quantize_item(const QuantParams& p, const QuantS
   }
 }
 
-template <int GS, int BITS, bool Q8>
-__global__ void __launch_bounds__(256) qkv_quantize_kernel(const QuantParams p, int side_idx) {
-  const QuantSide& s = p.side[side_idx];
-  const int64_t items = p.rows * (p.D / 8);
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  // the loop bound is rounded up to whole warps so every lane takes part in
-  // the group shuffles; lanes past the end are inactive
-  const int64_t items_w = (items + 31) / 32 * 32;
-  for (int64_t it = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; it < items_w; it += stride) {
-    quantize_item<GS, BITS, Q8>(p, s, it < items ? it : 0, it < items);
-  }
-}
+namespace {
 
-cudaError_t launch_quantize_side(const QuantParams& p, int side_idx, cudaStream_t stream) {
-  const QuantSide& s = p.side[side_idx];
-  const int64_t items = p.rows * (p.D / 8);
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t want = (items + 255) / 256;
-  const int grid = (int)std::min<int64_t>(want, (int64_t)sms * 16);
-  if (grid <= 0) return cudaSuccess;
+template <bool BF16>
+cudaError_t launch_q(int fmt, int bits, int gs, const QuantParams& p, int side0, int nsides,
+                     dim3 grid, cudaStream_t stream) {
+  grid.z = nsides;
 #define QKV_QLAUNCH(GS, BITS, Q8) \
-  qkv_quantize_kernel<GS, BITS, Q8><<<grid, 256, 0, stream>>>(p, side_idx)
-  if (s.fmt == QKV_Q8_0) QKV_QLAUNCH(32, 8, true);
-  else if (s.bits == 4 && s.gs == 32) QKV_QLAUNCH(32, 4, false);
-  else if (s.bits == 4 && s.gs == 64) QKV_QLAUNCH(64, 4, false);
-  else if (s.bits == 4 && s.gs == 128) QKV_QLAUNCH(128, 4, false);
-  else if (s.bits == 8 && s.gs == 32) QKV_QLAUNCH(32, 8, false);
-  else if (s.bits == 8 && s.gs == 64) QKV_QLAUNCH(64, 8, false);
-  else if (s.bits == 8 && s.gs == 128) QKV_QLAUNCH(128, 8, false);
+  qkv_quantize_kernel<GS, BITS, Q8, BF16><<<grid, 256, 0, stream>>>(p, side0)
+  if (fmt == QKV_Q8_0) QKV_QLAUNCH(32, 8, true);
+  else if (bits == 4 && gs == 32) QKV_QLAUNCH(32, 4, false);
+  else if (bits == 4 && gs == 64) QKV_QLAUNCH(64, 4, false);
+  else if (bits == 4 && gs == 128) QKV_QLAUNCH(128, 4, false);
+  else if (bits == 8 && gs == 32) QKV_QLAUNCH(32, 8, false);
+  else if (bits == 8 && gs == 64) QKV_QLAUNCH(64, 8, false);
+  else if (bits == 8 && gs == 128) QKV_QLAUNCH(128, 8, false);
   else return cudaErrorInvalidValue;
 #undef QKV_QLAUNCH
   return cudaGetLastError();
 }
+
+}  // namespace
 
 cudaError_t launch_quantize(const void* new_k, const void* new_v, int in_dtype, int B, int Hkv,
                             int Lnew, int D, const qkv_cache* k, const qkv_cache* v,
@@ -181,25 +186,36 @@ cudaError_t launch_quantize(const void* new_k, const void* new_v, int in_dtype, 
   QuantParams p;
   const qkv_cache* c[2] = {k, v};
   const void* src[2] = {new_k, new_v};
+  int fmt[2], bits[2], gs[2];
   for (int i = 0; i < 2; ++i) {
     p.side[i].src = static_cast<const uint16_t*>(src[i]);
     p.side[i].codes = c[i]->codes;
     p.side[i].scales = c[i]->scales;
     p.side[i].biases = c[i]->biases;
-    p.side[i].fmt = c[i]->fmt;
-    p.side[i].bits = c[i]->fmt == QKV_Q8_0 ? 8 : c[i]->bits;
-    p.side[i].gs = c[i]->fmt == QKV_Q8_0 ? 32 : c[i]->group_size;
+    p.side[i].Lcap = c[i]->Lcap;
+    fmt[i] = c[i]->fmt;
+    bits[i] = c[i]->fmt == QKV_Q8_0 ? 8 : c[i]->bits;
+    gs[i] = c[i]->fmt == QKV_Q8_0 ? 32 : c[i]->group_size;
   }
-  p.in_dtype = in_dtype;
+  int shift = 0;
+  while ((8 << shift) < D) ++shift;                 // D / 8 = 2^shift threads per token
   p.D = D;
-  p.rows = (int64_t)B * Hkv * Lnew;
+  p.row_shift = shift;
   p.Lnew = Lnew;
-  p.Lcap = k->Lcap;
   p.offset = offset;
-  cudaError_t e = launch_quantize_side(p, 0, stream);
-  if (e != cudaSuccess) return e;
-  p.Lcap = v->Lcap;
-  return launch_quantize_side(p, 1, stream);
+  const int64_t slabs = (int64_t)B * Hkv;
+  if (slabs > 65535 || (8 << shift) != D) return cudaErrorInvalidValue;
+  const int tpb = 256 >> shift;                     // tokens per block
+  dim3 grid((unsigned)((Lnew + tpb - 1) / tpb), (unsigned)slabs, 1);
+  const bool same = fmt[0] == fmt[1] && bits[0] == bits[1] && gs[0] == gs[1];
+  const bool bf16 = in_dtype == QKV_BF16;
+  for (int side0 = 0; side0 < 2; side0 += same ? 2 : 1) {
+    const int n = same ? 2 : 1;
+    cudaError_t e = bf16 ? launch_q<true>(fmt[side0], bits[side0], gs[side0], p, side0, n, grid, stream)
+                         : launch_q<false>(fmt[side0], bits[side0], gs[side0], p, side0, n, grid, stream);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace qkv

@@ -81,3 +81,13 @@ def test_quantize_validation_errors(lib):
     assert f(0, FAKE, 0, 1, 2, 4, 128, C.byref(ok), C.byref(ok), 0, None) == 1
     assert f(FAKE, FAKE, 0, 1, 2, 4, 128, C.byref(_cache(qkv, bits=3)), C.byref(ok), 0, None) == 2
     assert f(FAKE, FAKE, 0, 1, 2, 0, 128, C.byref(ok), C.byref(ok), 0, None) == 0   # nothing to do
+
+
+def test_quantize_rejects_too_many_slabs(lib):
+    """The quantizer's grid holds (batch, kv head) slabs in its y dimension:
+    more than 65535 of them is refused before any launch."""
+    from quantized_kv_attention_split_b200 import qkv
+    ok = _cache(qkv)
+    f = lib.qkv_quantize_update
+    assert f(FAKE, FAKE, 0, 65536, 1, 4, 128, C.byref(ok), C.byref(ok), 0, None) == 2
+    assert b"65535" in lib.qkv_last_error()

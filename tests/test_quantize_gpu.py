@@ -19,8 +19,10 @@ def qkv():
     return m
 
 
-def _inputs(shape, kind, dtype, seed):
+def _inputs(shape, kind, dtype, seed, fmt="affine", bits=4, gs=32):
     rng = np.random.default_rng(seed)
+    if kind == "halfway":                    # codes exactly at and next to x.5
+        return _halfway(shape, dtype, rng, fmt, bits, gs)
     if kind == "uniform":
         x = rng.random(shape, dtype=np.float32)
     elif kind == "normal":
@@ -36,6 +38,29 @@ def _inputs(shape, kind, dtype, seed):
     return S.f32_to_half_bits(x, dtype)
 
 
+def _halfway(shape, dtype, rng, fmt, bits, gs):
+    """Groups whose scale is an exact power of two 2^e (affine: min 0 and max
+    (2^bits - 1) * 2^e; Q8_0: max|x| = 127 * 2^e; all values representable in
+    f16 and bf16), so that (x - bias) / scale is exactly k + 0.5 for the other
+    elements, half of which are then moved one unit in the last place up or
+    down: the quantizer's rounding decision at and right next to every tie."""
+    lead = shape[:-1]
+    ng = shape[-1] // gs
+    e = rng.integers(-8, 5, lead + (ng, 1)).astype(np.float32)
+    top = 127 if fmt == "q8_0" else (1 << bits) - 1
+    k = rng.integers(0, min(top, 127), lead + (ng, gs)).astype(np.float32) + 0.5
+    if fmt == "q8_0":
+        k *= np.where(rng.random(k.shape) < 0.5, -1.0, 1.0)
+    g = k * np.exp2(e)
+    g[..., 0] = top * np.exp2(e[..., 0])
+    if fmt != "q8_0":
+        g[..., 1] = 0.0
+    bits16 = S.f32_to_half_bits(g.reshape(shape), dtype).astype(np.int32)
+    nudge = rng.integers(-1, 2, lead + (ng, gs))
+    nudge[..., :2] = 0
+    return (bits16 + nudge.reshape(shape)).astype(np.uint16)
+
+
 CASES = [
     # fmt, bits, gs, D, dtype
     ("affine", 4, 64, 128, "f16"), ("affine", 4, 32, 64, "f16"), ("affine", 4, 128, 256, "bf16"),
@@ -45,12 +70,12 @@ CASES = [
 
 
 @pytest.mark.parametrize("case", CASES, ids=lambda c: "-".join(map(str, c)))
-@pytest.mark.parametrize("kind", ["uniform", "normal", "wide", "special"])
+@pytest.mark.parametrize("kind", ["uniform", "normal", "wide", "special", "halfway"])
 def test_quantize_update_bit_exact(qkv, case, kind):
     fmt, bits, gs, D, dtype = case
     B, Hkv, Lnew, Lcap, offset = 2, 3, 37, 64, 19
-    nk = _inputs((B, Hkv, Lnew, D), kind, dtype, 1)
-    nv = _inputs((B, Hkv, Lnew, D), kind, dtype, 2)
+    nk = _inputs((B, Hkv, Lnew, D), kind, dtype, 1, fmt, bits, gs)
+    nv = _inputs((B, Hkv, Lnew, D), kind, dtype, 2, fmt, bits, gs)
     from quantized_kv_attention_split_b200.qkv import QuantCache, AFFINE, Q8_0
     f = Q8_0 if fmt == "q8_0" else AFFINE
     kd = QuantCache.empty(B, Hkv, Lcap, D, f, bits, gs)
