@@ -10,12 +10,12 @@
 //           bias = fp16(min); code = clamp(rint((x - bias) / scale))
 //   Q8_0:   scale = fp16(max|x| / 127); code = clamp(rint(x / scale), +-127)
 //
-// Design: one thread owns 8 consecutive elements (one 16-byte load), the
-// gs/8 lanes of a group reduce min/max with shuffles, each thread packs its 8
-// codes into one (4-bit) or two (8-bit) words and stores them; the first lane
-// of a group stores the fp16 scale (and bias).  Grid: x = blocks of tokens
-// (256 / (D/8) tokens per block), y = (batch, kv head) slab, z = K or V (one
-// launch when both caches have the same format), so no thread divides.
+// Design: one thread owns 16 consecutive elements (two 16-byte loads), the
+// gs/16 lanes of a group reduce min/max with shuffles, each thread packs its
+// 16 codes into two (4-bit) or four (8-bit) words and stores them; the first
+// lane of a group stores the fp16 scale (and bias).  Grid: x = blocks of
+// tokens (256 / (D/16) tokens per block), y = (batch, kv head) slab, z = K or
+// V (one launch when both caches have the same format), so no thread divides.
 #include <algorithm>
 
 #include "qkv_common.cuh"
@@ -49,14 +49,14 @@ __device__ __forceinline__ float in_to_float(uint16_t b) {
 // in the common case.  With r = RN(1/s), q0 = RN(d * r) is within 2^-14 of
 // RN(d / s) whenever |q0| < 2^9 (two roundings of relative error 2^-24 each),
 // so both round to the same integer unless q0 lies within 2^-13 of a
-// half-integer; that rare case, and any |q0| >= 2^9 or non-finite value, takes
-// the correctly rounded division, so the result is always identical to it.
-__device__ __forceinline__ int div_rint(float d, float s, float r) {
+// half-integer.  `exact` is set for that rare case and for any |q0| >= 2^9 or
+// non-finite value; the caller then redoes the row with the correctly rounded
+// division, so the result is always identical to it.
+__device__ __forceinline__ int fast_rint_div(float d, float r, bool& exact) {
   const float q0 = __fmul_rn(d, r);
   const float n = rintf(q0);
-  if (!(fabsf(q0) < 512.f) || fabsf(fabsf(__fsub_rn(q0, n)) - 0.5f) < 0x1p-13f)
-    return __float2int_rn(__fdiv_rn(d, s));
-  return (int)n;
+  exact |= !(fabsf(q0) < 512.f) | (fabsf(fabsf(__fsub_rn(q0, n)) - 0.5f) < 0x1p-13f);
+  return (int)fminf(fmaxf(n, -512.f), 512.f);
 }
 
 template <int LANES>
@@ -72,61 +72,61 @@ __device__ __forceinline__ float group_min(float v) {
   return v;
 }
 
+constexpr int kQEpt = 16;   // elements per thread (two 16-byte loads)
+
 template <int GS, int BITS, bool Q8, bool BF16>
 __global__ void __launch_bounds__(256) qkv_quantize_kernel(const QuantParams p, int side0) {
-  constexpr int LANES = GS / 8;
+  constexpr int LANES = GS / kQEpt;                 // threads per group
   const QuantSide& s = (side0 + (int)blockIdx.z) ? p.side[1] : p.side[0];
-  const int per_row = p.D >> 3;
+  const int per_row = p.D / kQEpt;
   const int tok = blockIdx.x * (256 >> p.row_shift) + (threadIdx.x >> p.row_shift);
-  const int c8 = threadIdx.x & (per_row - 1);        // which 8-element slice of the row
+  const int c16 = threadIdx.x & (per_row - 1);      // which 16-element slice of the row
   const bool active = tok < p.Lnew;                 // inactive lanes still join the shuffles
   const int64_t slab = blockIdx.y;                  // b * Hkv + kv head
   const int64_t srow = slab * p.Lnew + (active ? tok : 0);
   const int64_t crow = slab * s.Lcap + p.offset + tok;
-  float x[8];
+  float x[kQEpt];
   if (active) {
-    const uint4 raw = __ldg(reinterpret_cast<const uint4*>(s.src + srow * p.D + c8 * 8));
-    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+    const uint4* src = reinterpret_cast<const uint4*>(s.src + srow * p.D + c16 * kQEpt);
+    const uint4 r0 = __ldg(src), r1 = __ldg(src + 1);
+    const uint32_t w[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 8; ++i) {
       x[2 * i] = in_to_float<BF16>((uint16_t)(w[i] & 0xffff));
       x[2 * i + 1] = in_to_float<BF16>((uint16_t)(w[i] >> 16));
     }
   } else {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) x[i] = 0.f;
+    for (int i = 0; i < kQEpt; ++i) x[i] = 0.f;
   }
-  const int grp = (c8 * 8) / GS;
-  const bool leader = ((c8 * 8) % GS) == 0;
+  const int grp = (c16 * kQEpt) / GS;
+  const bool leader = ((c16 * kQEpt) % GS) == 0;
   const int ng = p.D / GS;
+  int q[kQEpt];
+  uint16_t sbits, bbits = 0;
   if constexpr (Q8) {
     float a = 0.f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(x[i]));
+    for (int i = 0; i < kQEpt; ++i) a = fmaxf(a, fabsf(x[i]));
     a = group_max<LANES>(a);
     const float d = __fdiv_rn(a, 127.f);
     const __half d16 = __float2half_rn(d);
     const float df = __half2float(d16);
+    sbits = __half_as_ushort(d16);
     const float rd = __frcp_rn(df);
-    uint32_t w[2] = {0u, 0u};
+    bool exact = false;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      int q = 0;
-      if (df != 0.f) {
-        q = div_rint(x[i], df, rd);
-        q = q < -127 ? -127 : (q > 127 ? 127 : q);
-      }
-      w[i >> 2] |= (uint32_t)(q & 0xff) << ((i & 3) * 8);
+    for (int i = 0; i < kQEpt; ++i) q[i] = fast_rint_div(x[i], rd, exact);
+    if (exact) {
+#pragma unroll
+      for (int i = 0; i < kQEpt; ++i) q[i] = __float2int_rn(__fdiv_rn(x[i], df));
     }
-    if (active) {
-      uint2* dst = reinterpret_cast<uint2*>(s.codes + crow * (p.D / 4) + c8 * 2);
-      *dst = make_uint2(w[0], w[1]);
-      if (leader) s.scales[crow * ng + grp] = __half_as_ushort(d16);
-    }
+#pragma unroll
+    for (int i = 0; i < kQEpt; ++i) q[i] = df == 0.f ? 0 : (q[i] < -127 ? -127 : (q[i] > 127 ? 127 : q[i]));
   } else {
     float mn = x[0], mx = x[0];
 #pragma unroll
-    for (int i = 1; i < 8; ++i) { mn = fminf(mn, x[i]); mx = fmaxf(mx, x[i]); }
+    for (int i = 1; i < kQEpt; ++i) { mn = fminf(mn, x[i]); mx = fmaxf(mx, x[i]); }
     mn = group_min<LANES>(mn);
     mx = group_max<LANES>(mx);
     constexpr float levels = (float)((1 << BITS) - 1);
@@ -135,25 +135,34 @@ __global__ void __launch_bounds__(256) qkv_quantize_kernel(const QuantParams p, 
     const __half s16 = __float2half_rn(sc);
     const __half b16 = __float2half_rn(mn);
     const float sf = __half2float(s16), bf = __half2float(b16);
+    sbits = __half_as_ushort(s16);
+    bbits = __half_as_ushort(b16);
     const float rs = __frcp_rn(sf);
-    uint32_t w[2] = {0u, 0u};
+    bool exact = false;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      int q = div_rint(__fsub_rn(x[i], bf), sf, rs);
-      q = q < 0 ? 0 : (q > (1 << BITS) - 1 ? (1 << BITS) - 1 : q);
-      if constexpr (BITS == 4) w[0] |= (uint32_t)q << (i * 4);
-      else w[i >> 2] |= (uint32_t)q << ((i & 3) * 8);
+    for (int i = 0; i < kQEpt; ++i) q[i] = fast_rint_div(__fsub_rn(x[i], bf), rs, exact);
+    if (exact) {
+#pragma unroll
+      for (int i = 0; i < kQEpt; ++i) q[i] = __float2int_rn(__fdiv_rn(__fsub_rn(x[i], bf), sf));
     }
-    if (active) {
-      if constexpr (BITS == 4) {
-        s.codes[crow * (p.D / 8) + c8] = w[0];
-      } else {
-        *reinterpret_cast<uint2*>(s.codes + crow * (p.D / 4) + c8 * 2) = make_uint2(w[0], w[1]);
-      }
-      if (leader) {
-        s.scales[crow * ng + grp] = __half_as_ushort(s16);
-        s.biases[crow * ng + grp] = __half_as_ushort(b16);
-      }
+#pragma unroll
+    for (int i = 0; i < kQEpt; ++i) q[i] = q[i] < 0 ? 0 : (q[i] > (1 << BITS) - 1 ? (1 << BITS) - 1 : q[i]);
+  }
+  if (active) {
+    if constexpr (BITS == 4) {
+      uint32_t w[2] = {0u, 0u};
+#pragma unroll
+      for (int i = 0; i < kQEpt; ++i) w[i >> 3] |= (uint32_t)q[i] << ((i & 7) * 4);
+      *reinterpret_cast<uint2*>(s.codes + crow * (p.D / 8) + c16 * 2) = make_uint2(w[0], w[1]);
+    } else {
+      uint32_t w[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+      for (int i = 0; i < kQEpt; ++i) w[i >> 2] |= (uint32_t)(q[i] & 0xff) << ((i & 3) * 8);
+      *reinterpret_cast<uint4*>(s.codes + crow * (p.D / 4) + c16 * 4) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    if (leader) {
+      s.scales[crow * ng + grp] = sbits;
+      if constexpr (!Q8) s.biases[crow * ng + grp] = bbits;
     }
   }
 }
@@ -198,13 +207,13 @@ cudaError_t launch_quantize(const void* new_k, const void* new_v, int in_dtype, 
     gs[i] = c[i]->fmt == QKV_Q8_0 ? 32 : c[i]->group_size;
   }
   int shift = 0;
-  while ((8 << shift) < D) ++shift;                 // D / 8 = 2^shift threads per token
+  while ((kQEpt << shift) < D) ++shift;             // D / 16 = 2^shift threads per token
   p.D = D;
   p.row_shift = shift;
   p.Lnew = Lnew;
   p.offset = offset;
   const int64_t slabs = (int64_t)B * Hkv;
-  if (slabs > 65535 || (8 << shift) != D) return cudaErrorInvalidValue;
+  if (slabs > 65535 || (kQEpt << shift) != D) return cudaErrorInvalidValue;
   const int tpb = 256 >> shift;                     // tokens per block
   dim3 grid((unsigned)((Lnew + tpb - 1) / tpb), (unsigned)slabs, 1);
   const bool same = fmt[0] == fmt[1] && bits[0] == bits[1] && gs[0] == gs[1];
