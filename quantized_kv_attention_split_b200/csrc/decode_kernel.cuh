@@ -317,10 +317,31 @@ qsdpa_decode_kernel(const DecodeParams p) {
     constexpr int NU = (2 * CU + C::NTHR - 1) / C::NTHR;
     const int fx_tid = swz_line<C::SWZ>((tid >> 3) & 15);
 
+    constexpr bool META1 = C::NMETA * C::META_UNITS <= C::NTHR;   // one metadata unit per thread
     auto issue_stage = [&](int stage, int buf) {
       const uint32_t sbase = smem_u32(smem + buf * C::STAGE);
       const int64_t key0 = (int64_t)stage * TK;
       const int nvalid = (int)(L - key0 < (int64_t)TK ? L - key0 : (int64_t)TK);      // rows of this stage below L
+      if (CU % C::NTHR == 0 && META1 && nvalid == TK) {
+        // a full stage: fixed per-thread offsets, no per-unit tests.  Unit
+        // tid + k * NTHR lies k * NTHR * 16 bytes further in both the source
+        // and (the swizzle acts on bits below that) the stage.
+        const uint8_t* ks = gK + key0 * C::RB + tid * 16;
+        const uint8_t* vs = gV + key0 * C::RB + tid * 16;
+        const uint32_t d0 = sbase + ((tid * 16) ^ fx_tid);
+#pragma unroll
+        for (int k = 0; k < CU / C::NTHR; ++k) {
+          cp_async16(d0 + k * C::NTHR * 16, ks + k * C::NTHR * 16, 16);
+          cp_async16(d0 + C::CODES + k * C::NTHR * 16, vs + k * C::NTHR * 16, 16);
+        }
+        if (tid < C::NMETA * C::META_UNITS) {
+          const int marr = tid / C::META_UNITS, mj = tid - marr * C::META_UNITS;
+          const uint8_t* gm = Q8 ? (marr == 0 ? gKs : gVs)
+                                 : (marr == 0 ? gKs : marr == 1 ? gKb : marr == 2 ? gVs : gVb);
+          cp_async16(sbase + 2 * C::CODES + marr * C::META + mj * 16, gm + key0 * C::MROW + mj * 16, 16);
+        }
+        return;
+      }
       const uint8_t* kb0 = gK + key0 * C::RB;
       const uint8_t* vb0 = gV + key0 * C::RB;
 #pragma unroll
@@ -558,8 +579,10 @@ qsdpa_decode_kernel(const DecodeParams p) {
           Sx[3] = fmaf(c1, acc[3], fmaf(bb1, qsc[G][1], Sx[3]));
         }
         const int kr0 = 16 * st + k0 + g;                 // key index within the stage
-        if (kr0 >= kvalid) { Sx[0] = -INFINITY; Sx[1] = -INFINITY; }
-        if (kr0 + 8 >= kvalid) { Sx[2] = -INFINITY; Sx[3] = -INFINITY; }
+        if (kvalid < TK) {                                // only a stage that reaches L
+          if (kr0 >= kvalid) { Sx[0] = -INFINITY; Sx[1] = -INFINITY; }
+          if (kr0 + 8 >= kvalid) { Sx[2] = -INFINITY; Sx[3] = -INFINITY; }
+        }
         if (p.mask_kind != QKV_MASK_NONE) {
 #pragma unroll
           for (int j = 0; j < 2; ++j) {
