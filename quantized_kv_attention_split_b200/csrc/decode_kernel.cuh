@@ -151,7 +151,14 @@ __device__ __forceinline__ void lds_meta(const uint8_t* p, uint16_t* h) {
   }
 }
 
-constexpr int kMergeBatch = 16;   // parts whose loads one merging thread has in flight
+// a / b for non-negative 64-bit values, in 32-bit arithmetic when both fit
+// (the common case; 64-bit division costs several times more instructions).
+__device__ __forceinline__ int64_t udiv64(int64_t a, int64_t b) {
+  if (((uint64_t)a | (uint64_t)b) >> 32 == 0) return (int64_t)((uint32_t)a / (uint32_t)b);
+  return a / b;
+}
+
+constexpr int kMergeBatch = 10;   // parts whose loads one merging thread has in flight
 constexpr int kMergeGroup = 8;    // parts per first-level merge when a unit merges in two levels
 constexpr int64_t kMergeFlat = 1 << 15;   // largest parts x rows x D merged by one CTA in one level
 
@@ -286,19 +293,20 @@ qsdpa_decode_kernel(const DecodeParams p) {
   const int chunk = warp / C::WPC, sub = warp % C::WPC;
   const int64_t S = p.stages_per_unit, T = p.total_stages;
   const int64_t nC = gridDim.x;
-  const int64_t lo = (int64_t)blockIdx.x * T / nC, hi = ((int64_t)blockIdx.x + 1) * T / nC;
-  const int64_t first_unit = lo / S;
+  const int64_t lo = udiv64((int64_t)blockIdx.x * T, nC), hi = udiv64(((int64_t)blockIdx.x + 1) * T, nC);
+  const int64_t first_unit = udiv64(lo, S);
   __shared__ int s_flag;
 
   for (int64_t x = lo; x < hi;) {
-    const int64_t u = x / S;
+    const int64_t u = udiv64(x, S);
     const int s0 = (int)(x - u * S);
     const int s1 = (int)(min(hi, (u + 1) * S) - u * S);
     x = u * S + s1;
 
-    const int cg = (int)(u % p.ncg);
-    const int hkv = (int)((u / p.ncg) % p.Hkv);
-    const int b = (int)(u / ((int64_t)p.ncg * p.Hkv));
+    const int64_t uh = udiv64(u, p.ncg);                 // (batch, kv head)
+    const int cg = (int)(u - uh * p.ncg);
+    const int b = (int)udiv64(uh, p.Hkv);
+    const int hkv = (int)(uh - (int64_t)b * p.Hkv);
     const int64_t row0 = ((int64_t)b * p.Hkv + hkv) * p.Lcap;   // first cache row of this head
     const int hbase = cg * HPC;                                  // first local row of the CTA
 
@@ -836,13 +844,13 @@ qsdpa_decode_kernel(const DecodeParams p) {
       // those.  Nobody waits on anybody.
       __threadfence();
       __syncthreads();
-      const int64_t cfirst = ((u * S + 1) * nC - 1) / T;
-      const int64_t clast = (((u + 1) * S) * nC - 1) / T;
+      const int64_t cfirst = udiv64((u * S + 1) * nC - 1, T);
+      const int64_t clast = udiv64(((u + 1) * S) * nC - 1, T);
       const int nparts = (int)(clast - cfirst + 1);
       const int nrows = min(HPC, p.G - hbase);
       // slot of the unit's first CTA: its second slot if it began in an
       // earlier unit; every later CTA of the unit began in this one
-      const int64_t slot0 = 2 * cfirst + ((cfirst * T / nC) / S == u ? 0 : 1);
+      const int64_t slot0 = 2 * cfirst + (udiv64(udiv64(cfirst * T, nC), S) == u ? 0 : 1);
       auto slot_of = [&](int64_t c) -> int64_t { return c == cfirst ? slot0 : 2 * c; };
       const int64_t out_base = (((int64_t)b * p.Hkv + hkv) * p.G + hbase) * D;
       if ((int64_t)nparts * nrows * D <= kMergeFlat) {
