@@ -44,6 +44,7 @@ namespace qkv {
 // 8 warps per CTA; two CTAs per SM for D <= 128 (independent CTAs overlap
 // each other's stage boundaries), one for D = 256 (more registers per thread).
 __host__ __device__ constexpr int dec_warps(int) { return 8; }
+constexpr int kDecWarpsMax = 8;
 __host__ __device__ constexpr int dec_ctas_per_sm(int D) { return D <= 128 ? 2 : 1; }
 
 // XOR coefficients (3 bits each, for line bits 0..3) of the 16-byte-unit
@@ -400,6 +401,46 @@ qsdpa_decode_kernel(const DecodeParams p) {
     float* qst = reinterpret_cast<float*>(smem + (NSTAGE - 1) * C::STAGE);
     constexpr int QCH = HPC * D / 8;                      // 16-byte query chunks
     constexpr int QPT = (QCH + C::NTHR - 1) / C::NTHR;
+    // Value-scale bound for this CTA's keys of the unit: tau (per group) is
+    // fixed so that P * s_v * 2^tau < 2^15 for every key (P <= 1), i.e.
+    // tau = 29 - the largest exponent field of the group's value scales.  The
+    // scales are loaded here, with the query, before the stages' copies
+    // (which then find them in L2).
+    __shared__ int s_vexp[kDecWarpsMax * 8];
+    int vexp[NG];
+    {
+#pragma unroll
+      for (int gg = 0; gg < NG; ++gg) vexp[gg] = 0;
+      const int64_t klo = (int64_t)s0 * TK;
+      const int64_t khi = (int64_t)s1 * TK < L ? (int64_t)s1 * TK : L;
+      const uint16_t* vsg = p.vs + (row0 + klo) * NG;
+      const int nh = (int)((khi - klo) * NG);      // halves; whole 16-byte units stay in the slab
+      constexpr int VB = 4;                        // 16-byte loads in flight per thread
+      for (int c0 = tid * 8; c0 < nh; c0 += VB * C::NTHR * 8) {
+        uint4 w4[VB];
+#pragma unroll
+        for (int k = 0; k < VB; ++k) {
+          const int c = c0 + k * C::NTHR * 8;
+          w4[k] = c < nh ? __ldg(reinterpret_cast<const uint4*>(vsg + c)) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int k = 0; k < VB; ++k) {
+          const int c = c0 + k * C::NTHR * 8;
+          const uint32_t w[4] = {w4[k].x, w4[k].y, w4[k].z, w4[k].w};
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int e = (int)((w[j >> 1] >> (16 * (j & 1) + 10)) & 31);
+            if (c + j < nh) vexp[j % NG] = max(vexp[j % NG], e);
+          }
+        }
+      }
+#pragma unroll
+      for (int gg = 0; gg < NG; ++gg) {
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) vexp[gg] = max(vexp[gg], __shfl_xor_sync(~0u, vexp[gg], off));
+        if (lane == 0) s_vexp[warp * 8 + gg] = vexp[gg];
+      }
+    }
     uint4 qraw[QPT];
     {
       const int64_t qbase = (((int64_t)b * p.Hkv + hkv) * p.G + hbase) * D;
@@ -500,9 +541,15 @@ qsdpa_decode_kernel(const DecodeParams p) {
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
     float beta[2][NG];
     float O[MT][4];
-    int tau[NG];          // per group: O of that group is kept scaled by 2^tau
+    int tau[NG];          // per group: the value operand carries 2^tau
 #pragma unroll
-    for (int gg = 0; gg < NG; ++gg) { beta[0][gg] = 0.f; beta[1][gg] = 0.f; tau[gg] = 40; }
+    for (int gg = 0; gg < NG; ++gg) {
+      beta[0][gg] = 0.f; beta[1][gg] = 0.f;
+      int e = 0;
+#pragma unroll
+      for (int w = 0; w < C::NWARP; ++w) e = max(e, s_vexp[w * 8 + gg]);
+      tau[gg] = 29 - e;
+    }
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) { O[mt][0] = O[mt][1] = O[mt][2] = O[mt][3] = 0.f; }
 
@@ -670,28 +717,6 @@ qsdpa_decode_kernel(const DecodeParams p) {
             const float vb0f = meta_f<NG>(vbw[st][0], G), vb1f = meta_f<NG>(vbw[st][1], G);
             beta[0][G] = fmaf(P[st][0], vb0f, fmaf(P[st][2], vb1f, beta[0][G]));
             beta[1][G] = fmaf(P[st][1], vb0f, fmaf(P[st][3], vb1f, beta[1][G]));
-          }
-        }
-        // keep P * s_v * 2^tau below 2^15: tau only ever decreases (O is
-        // rescaled by the exact power of two when it does)
-        uint32_t mxb = 0;
-#pragma unroll
-        for (int st = 0; st < C::SUB; ++st)
-          mxb = max(mxb, max(meta_bits<NG>(vsw[st][0], G), meta_bits<NG>(vsw[st][1], G)));
-        const int need = 29 - (int)((mxb >> 10) & 31);
-        if (__any_sync(~0u, need < tau[G])) {
-          int nt = need;
-#pragma unroll
-          for (int off = 1; off < 32; off <<= 1) nt = min(nt, __shfl_xor_sync(~0u, nt, off));
-          nt = min(nt, 29);
-          if (nt < tau[G]) {
-            const float f = exp2i(nt - tau[G]);
-#pragma unroll
-            for (int i = 0; i < KPG; ++i) {
-              O[G * KPG + i][0] *= f; O[G * KPG + i][1] *= f;
-              O[G * KPG + i][2] *= f; O[G * KPG + i][3] *= f;
-            }
-            tau[G] = nt;
           }
         }
         const float up = exp2i(tau[G]);
