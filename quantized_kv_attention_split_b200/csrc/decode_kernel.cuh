@@ -66,6 +66,14 @@ __host__ __device__ constexpr uint32_t swizzle_coeffs(int D, int bits, int gs) {
                        : gs == 64 ? swz_pack(0, 4, 2, 4) : swz_pack(0, 1, 2, 4)));
 }
 
+// XOR coefficients of the value tile's swizzle: the value fragments are read
+// with ldmatrix, 8 key rows x one 16-byte unit per matrix, and these make the
+// 8 rows hit 8 different bank groups (exhaustive search over the same family).
+__host__ __device__ constexpr uint32_t vswizzle_coeffs(int rb) {
+  return rb == 32 ? swz_pack(1, 0, 0, 0) : rb == 64 ? swz_pack(1, 2, 0, 0)
+       : rb == 128 ? swz_pack(1, 2, 4, 0) : swz_pack(0, 1, 2, 4);
+}
+
 // XOR pattern (already shifted to bits 4..6) of 128-byte line `line`.
 template <uint32_t SWZ>
 __host__ __device__ __forceinline__ constexpr int swz_line(int line) {
@@ -119,7 +127,8 @@ struct DecCfg {
   static constexpr int QSB = NC * 8 * D * 4;            // fp32 query rows (in the last ring slot)
   static constexpr int SMEM = RING > (NSTAGE - 1) * STAGE + QSB ? RING : (NSTAGE - 1) * STAGE + QSB;
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
-  static constexpr uint32_t SWZ = swizzle_coeffs(D, BITS, GS);
+  static constexpr uint32_t SWZ = swizzle_coeffs(D, BITS, GS);   // key tile
+  static constexpr uint32_t SWZV = vswizzle_coeffs(RB);          // value tile
   static_assert(D % GS == 0, "D must be a multiple of the group size");
   static_assert(NG <= 8, "at most 8 groups per row");
   static_assert(RB % 16 == 0, "code rows must be whole 16-byte units");
@@ -248,6 +257,17 @@ __device__ __noinline__ void merge_unit(const float* ml, const float* po, int n,
   }
 }
 
+// Transposing shared-memory matrix loads (8x8 of 16-bit elements per matrix).
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1,
+                                              uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr) : "memory");
+}
+__device__ __forceinline__ void ldsm_x2_trans(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];\n"
+               : "=r"(r0), "=r"(r1) : "r"(addr) : "memory");
+}
+
 // Raw fp16 bits of group G's scale (or bias) of row r in a staged meta array.
 template <int NG>
 __device__ __forceinline__ uint16_t meta_half(const uint8_t* base, int r, int G) {
@@ -325,6 +345,7 @@ qsdpa_decode_kernel(const DecodeParams p) {
     constexpr int CU = TK * C::UPR;
     constexpr int NU = (2 * CU + C::NTHR - 1) / C::NTHR;
     const int fx_tid = swz_line<C::SWZ>((tid >> 3) & 15);
+    const int fx_tid_v = swz_line<C::SWZV>((tid >> 3) & 15);
 
     constexpr bool META1 = C::NMETA * C::META_UNITS <= C::NTHR;   // one metadata unit per thread
     auto issue_stage = [&](int stage, int buf) {
@@ -338,10 +359,11 @@ qsdpa_decode_kernel(const DecodeParams p) {
         const uint8_t* ks = gK + key0 * C::RB + tid * 16;
         const uint8_t* vs = gV + key0 * C::RB + tid * 16;
         const uint32_t d0 = sbase + ((tid * 16) ^ fx_tid);
+        const uint32_t d0v = sbase + C::CODES + ((tid * 16) ^ fx_tid_v);
 #pragma unroll
         for (int k = 0; k < CU / C::NTHR; ++k) {
           cp_async16(d0 + k * C::NTHR * 16, ks + k * C::NTHR * 16, 16);
-          cp_async16(d0 + C::CODES + k * C::NTHR * 16, vs + k * C::NTHR * 16, 16);
+          cp_async16(d0v + k * C::NTHR * 16, vs + k * C::NTHR * 16, 16);
         }
         if (tid < C::NMETA * C::META_UNITS) {
           const int marr = tid / C::META_UNITS, mj = tid - marr * C::META_UNITS;
@@ -360,8 +382,10 @@ qsdpa_decode_kernel(const DecodeParams p) {
           const int which = i >= CU, j = which ? i - CU : i;
           const bool ok = (j / C::UPR) < nvalid;
           const uint8_t* src = (which ? vb0 : kb0) + (ok ? j * 16 : 0);
-          const int dst = (CU % C::NTHR == 0) ? which * C::CODES + ((j * 16) ^ fx_tid)
-                                                  : which * C::CODES + swz_offset<C::SWZ>(j * 16);
+          const int dst = (CU % C::NTHR == 0)
+                              ? which * C::CODES + ((j * 16) ^ (which ? fx_tid_v : fx_tid))
+                              : which * C::CODES + (which ? swz_offset<C::SWZV>(j * 16)
+                                                          : swz_offset<C::SWZ>(j * 16));
           cp_async16(sbase + dst, src, ok ? 16 : 0);
         }
       }
@@ -383,15 +407,16 @@ qsdpa_decode_kernel(const DecodeParams p) {
     const int k0 = sub * 16 * C::SUB;
     auto row_x = [&](int r) { return swz_line<C::SWZ>((r * C::RB) >> 7); };
     const int xk0 = row_x(k0 + g), xk1 = row_x(k0 + g + 8);
-    const int xva = row_x(k0 + 2 * t), xvb = row_x(k0 + 2 * t + 1);
-    const int xvc = row_x(k0 + 2 * t + 8), xvd = row_x(k0 + 2 * t + 9);
+    // value fragments: ldmatrix rows.  Lane l addresses row l % 8 of matrix
+    // l / 8; matrices 0/1 hold keys 0-7, 2/3 keys 8-15 of the 16-key block, and
+    // matrices 0/2 the first, 1/3 the second 16-byte unit of a unit pair (x2
+    // loads for 4-bit groups of 32: matrix 0 keys 0-7, matrix 1 keys 8-15).
+    constexpr bool VX2 = BITS == 4 && GS == 32;
+    const int vkey = k0 + (lane & 7) + (VX2 ? ((lane >> 3) & 1) * 8 : ((lane >> 4) & 1) * 8);
+    const int vunit = VX2 ? 0 : ((lane >> 3) & 1);
     auto koff = [&](int r, int x, int st, int G, int part) {
       return ((r * C::RB + G * C::GB + t * C::NW * 4 + part * 16) ^ x) ^
              swz_line<C::SWZ>((G * C::GB) >> 7) ^ swz_line<C::SWZ>((st * 16 * C::RB) >> 7);
-    };
-    auto voff = [&](int r, int x, int st, int G) {
-      return ((r * C::RB + G * C::GB + g * C::CB) ^ x) ^ swz_line<C::SWZ>((G * C::GB) >> 7) ^
-             swz_line<C::SWZ>((st * 16 * C::RB) >> 7);
     };
 
     const int nst = s1 - s0;
@@ -733,61 +758,56 @@ qsdpa_decode_kernel(const DecodeParams p) {
             b0l = movmatrix_trans(pack_half2(x00 - ft.x, x01 - ft.y));
             b1l = movmatrix_trans(pack_half2(x10 - fb.x, x11 - fb.y));
           }
-          // codes of keys 2t, 2t+1, 2t+8, 2t+9 (of this block) for this lane's chunk
-          uint32_t wa[C::CW], wb[C::CW], wc[C::CW], wd[C::CW];
-          {
-            const int ra = k0 + 16 * st + 2 * t;
-            if constexpr (C::CB == 2) {
-              wa[0] = *reinterpret_cast<const uint16_t*>(sV + voff(ra, xva, st, G));
-              wb[0] = *reinterpret_cast<const uint16_t*>(sV + voff(ra + 1, xvb, st, G));
-              wc[0] = *reinterpret_cast<const uint16_t*>(sV + voff(ra + 8, xvc, st, G));
-              wd[0] = *reinterpret_cast<const uint16_t*>(sV + voff(ra + 9, xvd, st, G));
+          // value codes of the block: ldmatrix .trans gives lane (g, t) one
+          // 16-bit unit of keys 2t and 2t+1 (and of 2t+8, 2t+9) per register:
+          // the key pairs of the A operand, one unit (4 or 2 dims) per register
+          constexpr int PAIRS = VX2 ? 1 : (BITS == 4 ? GS / 64 : GS / 32);   // unit pairs per group
+#pragma unroll
+          for (int pr = 0; pr < PAIRS; ++pr) {
+            const int lin = (vkey + 16 * st) * C::RB + G * C::GB + (2 * pr + vunit) * 16;
+            const uint32_t va = smem_u32(sV) + swz_offset<C::SWZV>(lin);
+            uint32_t R[4];
+            if constexpr (VX2) {
+              ldsm_x2_trans(va, R[0], R[2]);
+              R[1] = R[0]; R[3] = R[2];
             } else {
-              lds_words<C::CW>(sV + voff(ra, xva, st, G), wa);
-              lds_words<C::CW>(sV + voff(ra + 1, xvb, st, G), wb);
-              lds_words<C::CW>(sV + voff(ra + 8, xvc, st, G), wc);
-              lds_words<C::CW>(sV + voff(ra + 9, xvd, st, G), wd);
+              ldsm_x4_trans(va, R[0], R[1], R[2], R[3]);
             }
             if constexpr (Q8) {
 #pragma unroll
-              for (int i = 0; i < C::CW; ++i) {
-                wa[i] ^= 0x80808080u; wb[i] ^= 0x80808080u; wc[i] ^= 0x80808080u; wd[i] ^= 0x80808080u;
-              }
+              for (int r = 0; r < 4; ++r) R[r] ^= 0x80808080u;
             }
-          }
+            constexpr int MPP = VX2 ? 2 : (BITS == 4 ? 4 : 2);       // m-tiles per pair
 #pragma unroll
-          for (int i = 0; i < KPG; ++i) {
-            uint32_t a[4];
-            if constexpr (BITS == 4) {
-              const int w = i >> 2;
-              const uint32_t sel = ((4u + (i & 3)) << 8) | (uint32_t)(i & 3);
-              const uint32_t xv = prmt(wa[w], wb[w], sel), yv = prmt(wc[w], wd[w], sel);
-              a[0] = xv & 0x000F000Fu; a[1] = xv & 0x00F000F0u;
-              a[2] = yv & 0x000F000Fu; a[3] = yv & 0x00F000F0u;
-            } else {
-              const int w = i >> 1;
-              const uint32_t mA = wa[w] & 0x00FF00FFu, mB = wb[w] & 0x00FF00FFu;
-              const uint32_t nA = wa[w] & 0xFF00FF00u, nB = wb[w] & 0xFF00FF00u;
-              const uint32_t mC = wc[w] & 0x00FF00FFu, mD = wd[w] & 0x00FF00FFu;
-              const uint32_t nC2 = wc[w] & 0xFF00FF00u, nD = wd[w] & 0xFF00FF00u;
-              const uint32_t selm = (i & 1) ? 0x7632u : 0x5410u;
-              const uint32_t seln = (i & 1) ? 0x6723u : 0x4501u;
-              a[0] = prmt(mA, mB, selm); a[1] = prmt(nA, nB, seln);
-              a[2] = prmt(mC, mD, selm); a[3] = prmt(nC2, nD, seln);
-              if constexpr (Q8) {
-                // exact signed codes: (1024 + u) - 1152 with u = code + 128
-                const __half2 off = __float2half2_rn(1152.f);
+            for (int c = 0; c < MPP; ++c) {
+              uint32_t a[4];
+              if constexpr (BITS == 4) {
+                // nibble c of each unit (x2: nibbles c and c + 2 for the two row halves)
+                const int clo = c, chi = VX2 ? c + 2 : c;
 #pragma unroll
                 for (int r = 0; r < 4; ++r) {
-                  uint32_t v = a[r] | 0x64006400u;
-                  __half2 hv = __hsub2(*reinterpret_cast<__half2*>(&v), off);
-                  a[r] = *reinterpret_cast<uint32_t*>(&hv);
+                  const int cc = (r & 1) ? chi : clo;
+                  const uint32_t y = (cc >= 2) ? (R[r] >> 8) : R[r];
+                  a[r] = y & ((cc & 1) ? 0x00F000F0u : 0x000F000Fu);
+                }
+              } else {
+#pragma unroll
+                for (int r = 0; r < 4; ++r) a[r] = (c ? (R[r] >> 8) : R[r]) & 0x00FF00FFu;
+                if constexpr (Q8) {
+                  // exact signed codes: (1024 + u) - 1152 with u = code + 128
+                  const __half2 off = __float2half2_rn(1152.f);
+#pragma unroll
+                  for (int r = 0; r < 4; ++r) {
+                    uint32_t v = a[r] | 0x64006400u;
+                    __half2 hv = __hsub2(*reinterpret_cast<__half2*>(&v), off);
+                    a[r] = *reinterpret_cast<uint32_t*>(&hv);
+                  }
                 }
               }
+              const int mt = G * KPG + pr * MPP + c;
+              mma_f16(O[mt], a, b0, b1, O[mt]);
+              if constexpr (F32OUT) mma_f16(O[mt], a, b0l, b1l, O[mt]);
             }
-            const int mt = G * KPG + i;
-            mma_f16(O[mt], a, b0, b1, O[mt]);
-            if constexpr (F32OUT) mma_f16(O[mt], a, b0l, b1l, O[mt]);
           }
         }
       }
@@ -810,15 +830,25 @@ qsdpa_decode_kernel(const DecodeParams p) {
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) {
       const int G = mt / KPG, i = mt % KPG;
-      const int e = G * GS + g * (GS / 8) + 2 * i;
-      // rows g hold code*2^-24 (Q8_0: exact codes), rows g+8 code*2^-20 for
-      // 4-bit; O of group G carries an extra 2^tau
-      const float f_lo = exp2i((Q8 ? 0 : 24) - tau[G]);
-      const float f_hi = exp2i((Q8 ? 0 : (BITS == 4 ? 20 : 24)) - tau[G]);
-      ws[(2 * t) * D + e] = fmaf(O[mt][0], f_lo, beta[0][G]);
-      ws[(2 * t + 1) * D + e] = fmaf(O[mt][1], f_lo, beta[1][G]);
-      ws[(2 * t) * D + e + 1] = fmaf(O[mt][2], f_hi, beta[0][G]);
-      ws[(2 * t + 1) * D + e + 1] = fmaf(O[mt][3], f_hi, beta[1][G]);
+      // rows g / g+8 of value m-tile i of group G (the ldmatrix unit layout):
+      //  4-bit, groups >= 64: unit pair i/4, nibble c = i%4 -> dims 64(i/4)+4g+c, +32
+      //  4-bit, groups of 32: nibble c = i -> dims 4g+c and 4g+c+2
+      //  8-bit: unit pair i/2, byte c = i%2 -> dims 32(i/2)+2g+c, +16
+      int dlo, dhi;
+      bool x16 = false;                          // odd nibbles carry code * 2^-20
+      if constexpr (BITS == 4 && GS == 32) {
+        dlo = G * GS + 4 * g + i; dhi = dlo + 2; x16 = (i & 1) != 0;
+      } else if constexpr (BITS == 4) {
+        dlo = G * GS + 64 * (i >> 2) + 4 * g + (i & 3); dhi = dlo + 32; x16 = (i & 1) != 0;
+      } else {
+        dlo = G * GS + 32 * (i >> 1) + 2 * g + (i & 1); dhi = dlo + 16;
+      }
+      // codes entered as code*2^-24 (Q8_0: exact codes); O of group G carries 2^tau
+      const float f = exp2i((Q8 ? 0 : (x16 ? 20 : 24)) - tau[G]);
+      ws[(2 * t) * D + dlo] = fmaf(O[mt][0], f, beta[0][G]);
+      ws[(2 * t + 1) * D + dlo] = fmaf(O[mt][1], f, beta[1][G]);
+      ws[(2 * t) * D + dhi] = fmaf(O[mt][2], f, beta[0][G]);
+      ws[(2 * t + 1) * D + dhi] = fmaf(O[mt][3], f, beta[1][G]);
     }
     if (g == 0) {
       ws[8 * D + 2 * t] = m0; ws[8 * D + 2 * t + 1] = m1;
