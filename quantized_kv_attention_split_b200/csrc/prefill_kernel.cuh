@@ -14,7 +14,7 @@
 // pair, r = query * G + head, so the G heads that share a KV head share every
 // dequantized K/V tile and a tile's rows span few query positions (tight
 // causal bound).  Work goes in 32-key tiles through three warp roles:
-//   * dequant warps (8): one thread issues bulk copies (cp.async.bulk, one per
+//   * dequant warps (11): one thread issues bulk copies (cp.async.bulk, one per
 //     contiguous array) of the packed codes and scales of a tile into a
 //     three-slot ring; all of them turn tile t into fp16 K and V, both stored
 //     [key][d] with 128-byte swizzled rows (K is the K-major B operand of
@@ -40,15 +40,17 @@
 namespace qkv {
 
 constexpr int kPfBM = 128;        // rows per CTA
-constexpr int kPfBN = 32;         // keys per tile
-constexpr int kPfSoftWarps = 4;
-constexpr int kPfDqWarps = 8;
+constexpr int kPfBN = 64;         // keys per tile (S = Q K^T is 128 x 64)
+constexpr int kPfRawKeys = 32;    // keys per packed half tile (one bulk-copy slot)
+constexpr int kPfSoftWarps = 4;   // one thread per row (TMEM lane)
+constexpr int kPfSoftThreads = 32 * kPfSoftWarps;
+constexpr int kPfDqWarps = 11;   // 16 warps in all: 128 registers per thread
 constexpr int kPfDqThreads = 32 * kPfDqWarps;
 constexpr int kPfMmaWarp = kPfSoftWarps + kPfDqWarps;
 constexpr int kPfThreads = 32 * (kPfMmaWarp + 1);
 constexpr int kPfKSlots = 2;      // fp16 K tiles (slot free once S of the tile is done)
-constexpr int kPfVSlots = 3;      // fp16 V tiles (slot free once P V of the tile is done)
-constexpr int kPfRawSlots = 3;    // packed tiles in flight
+constexpr int kPfVSlots = 2;      // fp16 V tiles (slot free once P V of the tile is done)
+constexpr int kPfRawSlots = 4;    // packed half tiles in flight
 constexpr unsigned kPfWaitLimit = 1u << 21;   // try_wait rounds (<= 1 us each) before giving up
 
 struct PrefillParams {
@@ -93,27 +95,26 @@ struct PfCfg {
   static constexpr int CPC = 128 / BITS;             // codes per 16-byte chunk
   static constexpr int NG = D / GS;
   static constexpr int NMETA = Q8 ? 2 : 4;           // scale (and bias) arrays of K and V
-  static constexpr int META_BYTES = ((kPfBN * NG * 2 + 127) / 128) * 128;
+  static constexpr int META_BYTES = ((kPfRawKeys * NG * 2 + 127) / 128) * 128;
   // shared memory (1024-byte aligned operand slots)
-  static constexpr int KV_BYTES = kPfBN * D * 2;     // D/64 blocks of [32 keys][128 B]
+  static constexpr int KV_BYTES = kPfBN * D * 2;     // D/64 blocks of [64 keys][128 B]
   static constexpr int K_OFF = 0;
   static constexpr int V_OFF = K_OFF + kPfKSlots * KV_BYTES;
-  static constexpr int RAW_CODES = kPfBN * RB;
+  static constexpr int RAW_CODES = kPfRawKeys * RB;
   static constexpr int RAW_BYTES = 2 * RAW_CODES + NMETA * META_BYTES;
   static constexpr int RAW_OFF = V_OFF + kPfVSlots * KV_BYTES;
   static constexpr int BAR_OFF = RAW_OFF + kPfRawSlots * RAW_BYTES;
   static constexpr int SMEM = BAR_OFF + 256 + 1024;  // + barriers, TMEM slot, alignment slack
-  // TMEM columns: O, S[2], Q (fp16 pairs), P[2] (fp16 pairs)
+  // TMEM columns: O, S[2] (P of a tile overwrites the first half of its S), Q (fp16 pairs)
   static constexpr int O_COL = 0;
   static constexpr int S_COL = D;
   static constexpr int Q_COL = S_COL + 2 * kPfBN;
-  static constexpr int P_COL = Q_COL + D / 2;
-  static constexpr int COLS = P_COL + 2 * (kPfBN / 2);
+  static constexpr int COLS = Q_COL + D / 2;
   static constexpr int TMEM_COLS = COLS <= 128 ? 128 : (COLS <= 256 ? 256 : 512);
   static_assert(COLS <= 512, "TMEM budget");
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
   static_assert(RAW_BYTES % 128 == 0 && KV_BYTES % 1024 == 0, "slot alignment");
-  static_assert((kPfBN * UPR) % 32 == 0, "whole warps of chunks");
+  static_assert((kPfRawKeys * UPR) % 32 == 0, "whole warps of chunks");
 };
 
 // ---- tcgen05 / mbarrier / bulk-copy wrappers -------------------------------
@@ -248,7 +249,7 @@ __device__ __forceinline__ void named_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;\n" :: "r"(id), "r"(nthreads) : "memory");
 }
 
-// Byte offset of 16-bit element (row, col) in a tile of 32-row blocks with
+// Byte offset of 16-bit element (row, col) in a tile of 64-row blocks with
 // 128-byte swizzled rows (64 columns per block).
 __device__ __forceinline__ int sw128_off(int row, int col) {
   const int blk = col >> 6, chunk = (col >> 3) & 7;
@@ -269,14 +270,15 @@ __host__ __device__ constexpr int k_pos(int e) {
   }
 }
 
-// Dequantizes the 32 code rows of one packed tile into fp16 [key][d] with
-// 128-byte swizzled rows; value = scale * code + bias rounded once, rows at or
-// past `nv` (keys past L) are written as zeros.
+// Dequantizes the 32 code rows of one packed half tile into rows row0h.. of an
+// fp16 [key][d] tile with 128-byte swizzled rows; value = scale * code + bias
+// rounded once, rows at or past `nv` (keys past L) are written as zeros.
 template <int D, int BITS, int GS, bool Q8>
 __device__ __forceinline__ void pf_dequant(const uint8_t* codes, const uint16_t* sc,
-                                           const uint16_t* bi, uint8_t* dst, int nv, int chunk0) {
+                                           const uint16_t* bi, uint8_t* dst, int row0h, int nv,
+                                           int chunk0) {
   using C = PfCfg<D, BITS, GS, Q8>;
-  constexpr int NCH = kPfBN * C::UPR;
+  constexpr int NCH = kPfRawKeys * C::UPR;
   constexpr int ITERS = (NCH + kPfDqThreads - 1) / kPfDqThreads;
   const __half2 off = __float2half2_rn(Q8 ? 1152.f : 1024.f);   // Q8 codes are stored +128
 #pragma unroll
@@ -286,9 +288,11 @@ __device__ __forceinline__ void pf_dequant(const uint8_t* codes, const uint16_t*
     const int key = i / C::UPR, u = i - key * C::UPR;
     const uint4 w4 = *reinterpret_cast<const uint4*>(codes + i * 16);
     const int g = (u * C::CPC) / GS;
-    const __half2 s2 = __half2half2(__ushort_as_half(sc[key * C::NG + g]));
-    const __half2 b2 = Q8 ? __float2half2_rn(0.f) : __half2half2(__ushort_as_half(bi[key * C::NG + g]));
+    // rows at or past nv: scale and bias 0 make every value exactly 0 (codes are finite)
     const bool live = key < nv;
+    const __half2 s2 = __half2half2(__ushort_as_half(live ? sc[key * C::NG + g] : (uint16_t)0));
+    const __half2 b2 = Q8 ? __float2half2_rn(0.f)
+                          : __half2half2(__ushort_as_half(live ? bi[key * C::NG + g] : (uint16_t)0));
     const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
     if constexpr (BITS == 8) {
       uint32_t o[8];
@@ -299,11 +303,11 @@ __device__ __forceinline__ void pf_dequant(const uint8_t* codes, const uint16_t*
         const uint32_t h1 = prmt(x, 0x64646464u, 0x4342u);
         const __half2 v0 = __hfma2(__hsub2(*reinterpret_cast<const __half2*>(&h0), off), s2, b2);
         const __half2 v1 = __hfma2(__hsub2(*reinterpret_cast<const __half2*>(&h1), off), s2, b2);
-        o[2 * k] = live ? *reinterpret_cast<const uint32_t*>(&v0) : 0u;
-        o[2 * k + 1] = live ? *reinterpret_cast<const uint32_t*>(&v1) : 0u;
+        o[2 * k] = *reinterpret_cast<const uint32_t*>(&v0);
+        o[2 * k + 1] = *reinterpret_cast<const uint32_t*>(&v1);
       }
-      *reinterpret_cast<uint4*>(dst + sw128_off(key, u * 16)) = make_uint4(o[0], o[1], o[2], o[3]);
-      *reinterpret_cast<uint4*>(dst + sw128_off(key, u * 16 + 8)) = make_uint4(o[4], o[5], o[6], o[7]);
+      *reinterpret_cast<uint4*>(dst + sw128_off(row0h + key, u * 16)) = make_uint4(o[0], o[1], o[2], o[3]);
+      *reinterpret_cast<uint4*>(dst + sw128_off(row0h + key, u * 16 + 8)) = make_uint4(o[4], o[5], o[6], o[7]);
     } else {
 #pragma unroll
       for (int k = 0; k < 4; ++k) {      // word k: d = 32u + 8k .. +7, nibbles (j, j+4) -> (2j, 2j+1)
@@ -312,9 +316,9 @@ __device__ __forceinline__ void pf_dequant(const uint8_t* codes, const uint16_t*
         for (int j = 0; j < 4; ++j) {
           const uint32_t x = ((wv[k] >> (4 * j)) & 0x000F000Fu) | 0x64006400u;
           const __half2 v = __hfma2(__hsub2(*reinterpret_cast<const __half2*>(&x), off), s2, b2);
-          o[j] = live ? *reinterpret_cast<const uint32_t*>(&v) : 0u;
+          o[j] = *reinterpret_cast<const uint32_t*>(&v);
         }
-        *reinterpret_cast<uint4*>(dst + sw128_off(key, u * 32 + 8 * k)) = make_uint4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<uint4*>(dst + sw128_off(row0h + key, u * 32 + 8 * k)) = make_uint4(o[0], o[1], o[2], o[3]);
       }
     }
   }
@@ -329,13 +333,13 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
   const uint32_t sbase = smem_u32(smem);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t bar0 = sbase + C::BAR_OFF;
-  auto raw_full = [&](int i) { return bar0 + 8 * i; };        // [3] packed tile landed
-  auto k_ready = [&](int i) { return bar0 + 24 + 8 * i; };    // [2] fp16 K written
-  auto v_ready = [&](int i) { return bar0 + 40 + 8 * i; };    // [3] fp16 V written
+  auto raw_full = [&](int i) { return bar0 + 8 * i; };        // [4] packed half tile landed
+  auto k_ready = [&](int i) { return bar0 + 32 + 8 * i; };    // [2] fp16 K written
+  auto v_ready = [&](int i) { return bar0 + 48 + 8 * i; };    // [2] fp16 V written
   auto s_full = [&](int i) { return bar0 + 64 + 8 * i; };     // [2] S in TMEM
   auto p_ready = [&](int i) { return bar0 + 80 + 8 * i; };    // [2] P in TMEM
-  auto pv_done = [&](int i) { return bar0 + 96 + 8 * i; };    // [3] P V product done
-  const uint32_t mma_done = bar0 + 120;                       // all tensor-core work done
+  auto pv_done = [&](int i) { return bar0 + 96 + 8 * i; };    // [2] P V product done
+  const uint32_t mma_done = bar0 + 112;                       // all tensor-core work done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::BAR_OFF + 128);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::BAR_OFF + 132);
 
@@ -350,6 +354,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
     kend = min(L, L - p.Lq + last_row / p.G + 1);
   }
   const int ntiles = kend > 0 ? (int)((kend + kPfBN - 1) / kPfBN) : 0;
+  const int nhalves = kend > 0 ? (int)((kend + kPfRawKeys - 1) / kPfRawKeys) : 0;
 
   if (warp == kPfMmaWarp) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n"
@@ -357,15 +362,13 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
   }
   if (tid == 0) {
-    for (int i = 0; i < 3; ++i) {
-      mbar_init(raw_full(i), 1);
-      mbar_init(v_ready(i), kPfDqThreads);
-      mbar_init(pv_done(i), 1);
-    }
+    for (int i = 0; i < kPfRawSlots; ++i) mbar_init(raw_full(i), 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(k_ready(i), kPfDqThreads);
+      mbar_init(v_ready(i), kPfDqThreads);
       mbar_init(s_full(i), 1);
-      mbar_init(p_ready(i), 32 * kPfSoftWarps);
+      mbar_init(p_ready(i), kPfSoftThreads);
+      mbar_init(pv_done(i), 1);
     }
     mbar_init(mma_done, 1);
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
@@ -377,24 +380,25 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
   const uint32_t tmem = *tmem_slot;
   const int64_t row0 = ((int64_t)b * p.Hkv + hkv) * p.Lcap;
 
-  // softmax threads: this thread's row
-  const int r = mt * kPfBM + tid;
-  const bool row_ok = tid < kPfBM && r < R;
+  // softmax threads: row r = TMEM lane
+  const int quarter = warp & 3;
+  const int r = mt * kPfBM + quarter * 32 + lane;
+  const bool row_ok = warp < kPfSoftWarps && r < R;
   const int qi = row_ok ? r / p.G : 0;
   const int hh = row_ok ? r - qi * p.G : 0;
   const int64_t qrow = (((int64_t)b * p.Hq + (int64_t)hkv * p.G + hh) * p.Lq + qi) * D;
-  const uint32_t tmem_row = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+  const uint32_t tmem_row = tmem + ((uint32_t)(quarter * 32) << 16);
 
-  // dequant warps: packed-tile sources
-  const int dq = tid - 32 * kPfSoftWarps;
+  // dequant warps: packed half-tile sources
+  const int dq = tid - kPfSoftThreads;
   const uint8_t* gK = p.kc + row0 * C::RB;
   const uint8_t* gV = p.vc + row0 * C::RB;
-  int issued = 0;                                // tiles whose bulk copies were issued
-  auto issue_raw = [&](int t) {                  // one thread: the bulk copies of tile t
+  int issued = 0;                                // half tiles whose bulk copies were issued
+  auto issue_raw = [&](int i) {                  // one thread: the bulk copies of half tile i
     ++issued;
-    const int slot = t % kPfRawSlots;
-    const int64_t key0 = (int64_t)t * kPfBN;
-    const int nv = L - key0 < kPfBN ? (int)(L - key0) : kPfBN;
+    const int slot = i % kPfRawSlots;
+    const int64_t key0 = (int64_t)i * kPfRawKeys;
+    const int nv = L - key0 < kPfRawKeys ? (int)(L - key0) : kPfRawKeys;
     const int nv8 = (nv + 7) & ~7;               // scale rows in whole 16-byte units
     const uint32_t cb = (uint32_t)(nv * C::RB), mb = (uint32_t)(nv8 * NG * 2);
     const uint32_t bar = raw_full(slot);
@@ -412,9 +416,8 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
       bulk_g2s(dst + 2 * C::RAW_CODES + 3 * C::META_BYTES, p.vb + m0, mb, bar);
     }
   };
-  const int n_first = ntiles < kPfRawSlots ? ntiles : kPfRawSlots;
   if (dq == 0) {
-    for (int t = 0; t < n_first; ++t) issue_raw(t);
+    for (int i = 0; i < nhalves && i < kPfRawSlots; ++i) issue_raw(i);
   }
 
   // ---- Q rows -> fp16 (per-row power-of-two prescale) in TMEM ----------------
@@ -440,33 +443,35 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
     sigma = max(-96, min(96, sigma));
     const float up = exp2i(sigma);
     rowscale = p.scale_log2e * exp2i(-sigma);
+    {
 #pragma unroll 1
-    for (int c0 = 0; c0 < D; c0 += 64) {         // 64 elements = 32 TMEM columns
-      uint32_t qw[32];
+      for (int c0 = 0; c0 < D; c0 += 64) {       // 64 elements = 32 TMEM columns
+        uint32_t qw[32];
 #pragma unroll
-      for (int e8 = 0; e8 < 64; e8 += 8) {
-        uint32_t w[4] = {0u, 0u, 0u, 0u};
-        if (row_ok) {
-          const uint4 raw = *reinterpret_cast<const uint4*>(
-              reinterpret_cast<const uint16_t*>(p.q) + qrow + c0 + e8);
-          w[0] = raw.x; w[1] = raw.y; w[2] = raw.z; w[3] = raw.w;
+        for (int e8 = 0; e8 < 64; e8 += 8) {
+          uint32_t w[4] = {0u, 0u, 0u, 0u};
+          if (row_ok) {
+            const uint4 raw = *reinterpret_cast<const uint4*>(
+                reinterpret_cast<const uint16_t*>(p.q) + qrow + c0 + e8);
+            w[0] = raw.x; w[1] = raw.y; w[2] = raw.z; w[3] = raw.w;
+          }
+          float v[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const uint16_t bits = (uint16_t)(w[k >> 1] >> (16 * (k & 1)));
+            v[k] = (p.q_dtype == QKV_F16 ? __half2float(__ushort_as_half(bits))
+                                         : __uint_as_float((uint32_t)bits << 16)) * up;
+          }
+          float sq[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) sq[k_pos<BITS>(k)] = v[k];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) qw[e8 / 2 + k] = pack_half2(sq[2 * k], sq[2 * k + 1]);
         }
-        float v[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const uint16_t bits = (uint16_t)(w[k >> 1] >> (16 * (k & 1)));
-          v[k] = (p.q_dtype == QKV_F16 ? __half2float(__ushort_as_half(bits))
-                                       : __uint_as_float((uint32_t)bits << 16)) * up;
-        }
-        float s[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) s[k_pos<BITS>(k)] = v[k];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) qw[e8 / 2 + k] = pack_half2(s[2 * k], s[2 * k + 1]);
+        tmem_st32(tmem_row + C::Q_COL + c0 / 2, qw);
       }
-      tmem_st32(tmem_row + C::Q_COL + c0 / 2, qw);
+      tmem_wait_st();
     }
-    tmem_wait_st();
   }
   tc_fence_before();
   __syncthreads();
@@ -479,32 +484,49 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
     for (int bt = 0; bt < 5; ++bt)
       if ((lane >> bt) & 1) cl ^= pf_lane_col(D, BITS, bt);
     const int chunk0 = (dq >> 5) * 32 + cl;
+    constexpr int MH = C::META_BYTES / 2;        // metadata array stride in halves
+    // one operand tile (K or V) from the tile's two half tiles; a half tile
+    // past the last one is written as zeros (its keys are never visible)
+    auto convert = [&](int t, bool is_v, uint8_t* dst) {
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        const int i = 2 * t + h;
+        const bool present = i < nhalves;
+        const int slot = i % kPfRawSlots;
+        if (present && !is_v)                    // V reuses the half tiles K waited for
+          mbar_wait(raw_full(slot), (i / kPfRawSlots) & 1, abort_flag, p.status, 1u);
+        const uint8_t* raw = smem + C::RAW_OFF + slot * C::RAW_BYTES;
+        const uint16_t* meta = reinterpret_cast<const uint16_t*>(raw + 2 * C::RAW_CODES);
+        const int64_t key0 = (int64_t)i * kPfRawKeys;
+        const int nv = !present ? 0 : (L - key0 < kPfRawKeys ? (int)(L - key0) : kPfRawKeys);
+        if (!is_v)
+          pf_dequant<D, BITS, GS, Q8>(raw, meta, meta + MH, dst, h * kPfRawKeys, nv, chunk0);
+        else
+          pf_dequant<D, BITS, GS, Q8>(raw + C::RAW_CODES, meta + (Q8 ? 1 : 2) * MH, meta + 3 * MH,
+                                      dst, h * kPfRawKeys, nv, chunk0);
+      }
+    };
     for (int t = 0; t < ntiles; ++t) {
-      const int slot = t % kPfRawSlots, ks = t & 1, vs = t % kPfVSlots;
-      const int64_t key0 = (int64_t)t * kPfBN;
-      const int nv = L - key0 < kPfBN ? (int)(L - key0) : kPfBN;
-      mbar_wait(raw_full(slot), (t / kPfRawSlots) & 1, abort_flag, p.status, 1u);
-      const uint8_t* raw = smem + C::RAW_OFF + slot * C::RAW_BYTES;
-      const uint16_t* meta = reinterpret_cast<const uint16_t*>(raw + 2 * C::RAW_CODES);
-      constexpr int MH = C::META_BYTES / 2;      // metadata array stride in halves
+      const int s = t & 1;
       if (t >= kPfKSlots)                        // K slot free once S of tile t-2 is done
-        mbar_wait(s_full(ks), ((t - 2) >> 1) & 1, abort_flag, p.status, 1u);
-      pf_dequant<D, BITS, GS, Q8>(raw, meta, meta + MH, smem + C::K_OFF + ks * C::KV_BYTES, nv,
-                                  chunk0);
+        mbar_wait(s_full(s), ((t - 2) >> 1) & 1, abort_flag, p.status, 1u);
+      convert(t, false, smem + C::K_OFF + s * C::KV_BYTES);
       fence_async_smem();
-      mbar_arrive(k_ready(ks));
-      if (t >= kPfVSlots)                        // V slot free once P V of tile t-3 is done
-        mbar_wait(pv_done(vs), ((t - 3) / 3) & 1, abort_flag, p.status, 1u);
-      pf_dequant<D, BITS, GS, Q8>(raw + C::RAW_CODES, meta + (Q8 ? 1 : 2) * MH,
-                                  meta + 3 * MH, smem + C::V_OFF + vs * C::KV_BYTES, nv, chunk0);
+      mbar_arrive(k_ready(s));
+      if (t >= kPfVSlots)                        // V slot free once P V of tile t-2 is done
+        mbar_wait(pv_done(s), ((t - 2) >> 1) & 1, abort_flag, p.status, 1u);
+      convert(t, true, smem + C::V_OFF + s * C::KV_BYTES);
       fence_async_smem();
-      mbar_arrive(v_ready(vs));
-      named_sync(1, kPfDqThreads);               // every thread is done reading raw slot
-      if (dq == 0 && t + kPfRawSlots < ntiles && !*abort_flag) issue_raw(t + kPfRawSlots);
+      mbar_arrive(v_ready(s));
+      named_sync(1, kPfDqThreads);               // raw slots of half tiles 2t, 2t+1 are free
+      if (dq == 0 && !*abort_flag) {
+        for (int h = 0; h < 2; ++h)
+          if (2 * t + h + kPfRawSlots < nhalves) issue_raw(2 * t + h + kPfRawSlots);
+      }
     }
     if (dq == 0) {                               // own bulk copies still in flight (after a give-up)
-      for (int t = max(0, issued - kPfRawSlots); t < issued; ++t)
-        mbar_drain(raw_full(t % kPfRawSlots), (t / kPfRawSlots) & 1, p.status);
+      for (int i = max(0, issued - kPfRawSlots); i < issued; ++i)
+        mbar_drain(raw_full(i % kPfRawSlots), (i / kPfRawSlots) & 1, p.status);
     }
   } else if (warp == kPfMmaWarp) {
     // ======================= MMA warp ==========================================
@@ -527,28 +549,32 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
       __syncwarp();
     };
     auto issue_pv = [&](int t) {
-      const int s = t & 1, vs = t % kPfVSlots;
-      mbar_wait(v_ready(vs), (t / kPfVSlots) & 1, abort_flag, p.status, 4u);
+      const int s = t & 1;
+      mbar_wait(v_ready(s), (t >> 1) & 1, abort_flag, p.status, 4u);
       mbar_wait(p_ready(s), (t >> 1) & 1, abort_flag, p.status, 4u);
       tc_fence_after();
       if (lane == 0) {
 #pragma unroll
         for (int k = 0; k < kPfBN / 16; ++k) {
-          const uint64_t bd = umma_desc_sw128(sbase + C::V_OFF + vs * C::KV_BYTES + k * 16 * 128,
+          const uint64_t bd = umma_desc_sw128(sbase + C::V_OFF + s * C::KV_BYTES + k * 16 * 128,
                                               kPfBN * 128, 1024);
-          tc_mma_ts(tmem + C::O_COL, tmem + C::P_COL + s * (kPfBN / 2) + k * 8, bd, idesc_o,
+          // P of tile t: fp16 pairs in the first half of its S columns
+          tc_mma_ts(tmem + C::O_COL, tmem + C::S_COL + s * kPfBN + k * 8, bd, idesc_o,
                     (t > 0 || k > 0) ? 1u : 0u);
         }
-        tc_commit(pv_done(vs));
+        tc_commit(pv_done(s));
       }
       __syncwarp();
     };
+    // S(t+2) reuses the columns of S(t) and P(t): it is issued after P V of
+    // tile t, and the tensor core executes one thread's operations in order
     if (ntiles > 0) issue_s(0);
+    if (ntiles > 1) issue_s(1);
     for (int t = 0; t < ntiles; ++t) {
-      if (t + 1 < ntiles) issue_s(t + 1);   // overlaps the softmax of tile t
       issue_pv(t);
+      if (t + 2 < ntiles) issue_s(t + 2);
     }
-    if (lane == 0) {                         // every MMA issued above has completed
+    if (lane == 0) {                             // every MMA issued above has completed
       tc_commit(mma_done);
       mbar_drain(mma_done, 0, p.status);
     }
@@ -566,16 +592,20 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
       tc_fence_after();
       float sv[kPfBN];
       tmem_ld32(tmem_row + C::S_COL + s * kPfBN, reinterpret_cast<uint32_t*>(sv));
+      tmem_ld32(tmem_row + C::S_COL + s * kPfBN + 32, reinterpret_cast<uint32_t*>(sv + 32));
       tmem_wait_ld();
       // a tile without masked keys for any row of the warp takes the short path
       const bool full = __all_sync(~0u, row_ok && !additive && key0 + kPfBN <= kend &&
                                             (!causal || key0 + kPfBN - 1 <= causal_lim));
       float tmax;
       if (full) {
-        float mx = sv[0];
+        float m0 = fmaxf(sv[0], sv[1]), m1 = fmaxf(sv[2], sv[3]);
 #pragma unroll
-        for (int j = 1; j < kPfBN; ++j) mx = fmaxf(mx, sv[j]);
-        tmax = mx * rowscale;
+        for (int j = 4; j < kPfBN; j += 4) {
+          m0 = fmaxf(m0, fmaxf(sv[j], sv[j + 1]));
+          m1 = fmaxf(m1, fmaxf(sv[j + 2], sv[j + 3]));
+        }
+        tmax = fmaxf(m0, m1) * rowscale;
       } else {
         tmax = -INFINITY;
 #pragma unroll
@@ -600,15 +630,9 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
         m_used = tmax;
       }
       const float mref = m_used == -INFINITY ? 0.f : m_used;
-      // P slot s is free once the P V product of tile t-2 is done; the O
-      // rescale needs the product of tile t-1 done (both are rare waits)
-      if (t >= 2) {
-        mbar_wait(pv_done((t - 2) % kPfVSlots), ((t - 2) / kPfVSlots) & 1, abort_flag, p.status, 16u);
-        tc_fence_after();
-      }
       const bool rescale = t > 0 && __any_sync(~0u, alpha != 1.f);
-      if (rescale) {
-        mbar_wait(pv_done((t - 1) % kPfVSlots), ((t - 1) / kPfVSlots) & 1, abort_flag, p.status, 32u);
+      if (rescale) {                             // needs P V of tile t-1 done (rare)
+        mbar_wait(pv_done((t - 1) & 1), ((t - 1) >> 1) & 1, abort_flag, p.status, 32u);
         tc_fence_after();
 #pragma unroll 1
         for (int c = 0; c < D; c += 32) {
@@ -620,36 +644,40 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
           tmem_st32(tmem_row + C::O_COL + c, o);
         }
       }
-      float rs = 0.f;
-      uint32_t pk[kPfBN / 2];
-      if (full) {
-        const float nm = -mref;
+      // P (fp16 pairs) over the first half of this tile's S columns, which
+      // this thread has already read
+      float rs0 = 0.f, rs1 = 0.f;
 #pragma unroll
-        for (int i = 0; i < kPfBN / 2; ++i) {
-          const float a = ex2(fmaf(sv[2 * i], rowscale, nm));
-          const float c = ex2(fmaf(sv[2 * i + 1], rowscale, nm));
-          rs += a + c;
-          pk[i] = pack_half2(a, c);
-        }
-      } else {
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t pk[16];
+        if (full) {
+          const float nm = -mref;
 #pragma unroll
-        for (int i = 0; i < kPfBN / 2; ++i) {
-          const float a = ex2(sv[2 * i] - mref), c = ex2(sv[2 * i + 1] - mref);
-          rs += a + c;
-          pk[i] = pack_half2(a, c);
+          for (int i = 0; i < 16; ++i) {
+            const float a = ex2(fmaf(sv[32 * hf + 2 * i], rowscale, nm));
+            const float c = ex2(fmaf(sv[32 * hf + 2 * i + 1], rowscale, nm));
+            rs0 += a; rs1 += c;
+            pk[i] = pack_half2(a, c);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float a = ex2(sv[32 * hf + 2 * i] - mref), c = ex2(sv[32 * hf + 2 * i + 1] - mref);
+            rs0 += a; rs1 += c;
+            pk[i] = pack_half2(a, c);
+          }
         }
+        tmem_st16(tmem_row + C::S_COL + s * kPfBN + 16 * hf, pk);
       }
-      tmem_st16(tmem_row + C::P_COL + s * (kPfBN / 2), pk);
       tmem_wait_st();
-      lsum = lsum * alpha + rs;
+      lsum = lsum * alpha + (rs0 + rs1);
       tc_fence_before();
       mbar_arrive(p_ready(s));
     }
     // ---- epilogue: O / l -> out --------------------------------------------
     bool have = ntiles > 0;
     if (have) {
-      have = mbar_wait(pv_done((ntiles - 1) % kPfVSlots), ((ntiles - 1) / kPfVSlots) & 1,
-                       abort_flag, p.status, 64u);
+      have = mbar_wait(pv_done((ntiles - 1) & 1), ((ntiles - 1) >> 1) & 1, abort_flag, p.status, 64u);
       tc_fence_after();
     }
     have = __all_sync(~0u, have) && !*abort_flag;
