@@ -14,9 +14,10 @@
 // pair, r = query * G + head, so the G heads that share a KV head share every
 // dequantized K/V tile and a tile's rows span few query positions (tight
 // causal bound).  Work goes in 32-key tiles through three warp roles:
-//   * dequant warps (11): one thread issues bulk copies (cp.async.bulk, one per
-//     contiguous array) of the packed codes and scales of a tile into a
-//     three-slot ring; all of them turn tile t into fp16 K and V, both stored
+//   * producer warp (1): bulk copies (cp.async.bulk, one per contiguous array)
+//     of the packed codes and scales of 32-key half tiles into a four-slot
+//     ring, refilled as soon as the dequant warps release a tile's slots;
+//   * dequant warps (10): turn tile t into fp16 K and V, both stored
 //     [key][d] with 128-byte swizzled rows (K is the K-major B operand of
 //     S = Q K^T, V the MN-major B operand of O += P V), two K slots and three
 //     V slots so dequantization runs ahead of the tensor cores;
@@ -44,10 +45,11 @@ constexpr int kPfBN = 64;         // keys per tile (S = Q K^T is 128 x 64)
 constexpr int kPfRawKeys = 32;    // keys per packed half tile (one bulk-copy slot)
 constexpr int kPfSoftWarps = 4;   // one thread per row (TMEM lane)
 constexpr int kPfSoftThreads = 32 * kPfSoftWarps;
-constexpr int kPfDqWarps = 11;   // 16 warps in all: 128 registers per thread
+constexpr int kPfDqWarps = 10;   // 16 warps in all: 128 registers per thread
 constexpr int kPfDqThreads = 32 * kPfDqWarps;
 constexpr int kPfMmaWarp = kPfSoftWarps + kPfDqWarps;
-constexpr int kPfThreads = 32 * (kPfMmaWarp + 1);
+constexpr int kPfProdWarp = kPfMmaWarp + 1;     // issues the bulk copies
+constexpr int kPfThreads = 32 * (kPfProdWarp + 1);
 constexpr int kPfKSlots = 2;      // fp16 K tiles (slot free once S of the tile is done)
 constexpr int kPfVSlots = 2;      // fp16 V tiles (slot free once P V of the tile is done)
 constexpr int kPfRawSlots = 4;    // packed half tiles in flight
@@ -340,8 +342,9 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
   auto p_ready = [&](int i) { return bar0 + 80 + 8 * i; };    // [2] P in TMEM
   auto pv_done = [&](int i) { return bar0 + 96 + 8 * i; };    // [2] P V product done
   const uint32_t mma_done = bar0 + 112;                       // all tensor-core work done
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::BAR_OFF + 128);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::BAR_OFF + 132);
+  auto raw_free = [&](int i) { return bar0 + 120 + 8 * i; };  // [2] a tile's raw slots released
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::BAR_OFF + 144);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::BAR_OFF + 148);
 
   const int mt = blockIdx.x % p.mtiles;
   const int hkv = (blockIdx.x / p.mtiles) % p.Hkv;
@@ -371,6 +374,8 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
       mbar_init(pv_done(i), 1);
     }
     mbar_init(mma_done, 1);
+    mbar_init(raw_free(0), kPfDqThreads);
+    mbar_init(raw_free(1), kPfDqThreads);
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     *abort_flag = 0;
   }
@@ -394,30 +399,47 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
   const uint8_t* gK = p.kc + row0 * C::RB;
   const uint8_t* gV = p.vc + row0 * C::RB;
   int issued = 0;                                // half tiles whose bulk copies were issued
-  auto issue_raw = [&](int i) {                  // one thread: the bulk copies of half tile i
-    ++issued;
-    const int slot = i % kPfRawSlots;
-    const int64_t key0 = (int64_t)i * kPfRawKeys;
-    const int nv = L - key0 < kPfRawKeys ? (int)(L - key0) : kPfRawKeys;
-    const int nv8 = (nv + 7) & ~7;               // scale rows in whole 16-byte units
-    const uint32_t cb = (uint32_t)(nv * C::RB), mb = (uint32_t)(nv8 * NG * 2);
-    const uint32_t bar = raw_full(slot);
-    const uint32_t dst = sbase + C::RAW_OFF + slot * C::RAW_BYTES;
-    mbar_arrive_expect_tx(bar, 2 * cb + C::NMETA * mb);
-    bulk_g2s(dst, gK + key0 * C::RB, cb, bar);
-    bulk_g2s(dst + C::RAW_CODES, gV + key0 * C::RB, cb, bar);
-    const int64_t m0 = (row0 + key0) * NG;
-    bulk_g2s(dst + 2 * C::RAW_CODES, p.ks + m0, mb, bar);
-    if (Q8) {
-      bulk_g2s(dst + 2 * C::RAW_CODES + C::META_BYTES, p.vs + m0, mb, bar);
-    } else {
-      bulk_g2s(dst + 2 * C::RAW_CODES + C::META_BYTES, p.kb + m0, mb, bar);
-      bulk_g2s(dst + 2 * C::RAW_CODES + 2 * C::META_BYTES, p.vs + m0, mb, bar);
-      bulk_g2s(dst + 2 * C::RAW_CODES + 3 * C::META_BYTES, p.vb + m0, mb, bar);
+  // The bulk copies of half tiles i0 .. i0+n-1 (n <= 2), issued by the 32
+  // lanes of the producer warp: lane 0 first registers the byte counts on
+  // the slots' mbarriers, then every lane issues at most one copy.
+  constexpr int CPH = 2 + C::NMETA;              // copies per half tile
+  auto issue_raw = [&](int i0, int n) {
+    issued += n;
+    if (lane == 0) {
+      for (int k = 0; k < n; ++k) {
+        const int i = i0 + k;
+        const int64_t key0 = (int64_t)i * kPfRawKeys;
+        const int nv = L - key0 < kPfRawKeys ? (int)(L - key0) : kPfRawKeys;
+        const int nv8 = (nv + 7) & ~7;           // scale rows in whole 16-byte units
+        mbar_arrive_expect_tx(raw_full(i % kPfRawSlots),
+                              (uint32_t)(2 * nv * C::RB + C::NMETA * nv8 * NG * 2));
+      }
+    }
+    __syncwarp();
+    if (lane < n * CPH) {
+      const int i = i0 + lane / CPH, which = lane % CPH;
+      const int slot = i % kPfRawSlots;
+      const int64_t key0 = (int64_t)i * kPfRawKeys;
+      const int nv = L - key0 < kPfRawKeys ? (int)(L - key0) : kPfRawKeys;
+      const int nv8 = (nv + 7) & ~7;
+      const uint32_t cb = (uint32_t)(nv * C::RB), mb = (uint32_t)(nv8 * NG * 2);
+      const uint32_t bar = raw_full(slot);
+      const uint32_t dst = sbase + C::RAW_OFF + slot * C::RAW_BYTES;
+      const int64_t m0 = (row0 + key0) * NG;
+      if (which == 0) bulk_g2s(dst, gK + key0 * C::RB, cb, bar);
+      else if (which == 1) bulk_g2s(dst + C::RAW_CODES, gV + key0 * C::RB, cb, bar);
+      else {
+        // metadata arrays in order: K scales, (K biases,) V scales, (V biases)
+        const int arr = which - 2;
+        const uint16_t* src = Q8 ? (arr == 0 ? p.ks : p.vs)
+                                 : (arr == 0 ? p.ks : arr == 1 ? p.kb : arr == 2 ? p.vs : p.vb);
+        bulk_g2s(dst + 2 * C::RAW_CODES + arr * C::META_BYTES, src + m0, mb, bar);
+      }
     }
   };
-  if (dq == 0) {
-    for (int i = 0; i < nhalves && i < kPfRawSlots; ++i) issue_raw(i);
+  if (warp == kPfProdWarp) {
+    const int n0 = nhalves < kPfRawSlots ? nhalves : kPfRawSlots;
+    for (int i0 = 0; i0 < n0; i0 += 2) issue_raw(i0, n0 - i0 < 2 ? n0 - i0 : 2);
   }
 
   // ---- Q rows -> fp16 (per-row power-of-two prescale) in TMEM ----------------
@@ -518,16 +540,23 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
       convert(t, true, smem + C::V_OFF + s * C::KV_BYTES);
       fence_async_smem();
       mbar_arrive(v_ready(s));
-      named_sync(1, kPfDqThreads);               // raw slots of half tiles 2t, 2t+1 are free
-      if (dq == 0 && !*abort_flag) {
-        for (int h = 0; h < 2; ++h)
-          if (2 * t + h + kPfRawSlots < nhalves) issue_raw(2 * t + h + kPfRawSlots);
-      }
+      mbar_arrive(raw_free(s));                  // raw slots of half tiles 2t, 2t+1 are free
     }
-    if (dq == 0) {                               // own bulk copies still in flight (after a give-up)
+  } else if (warp == kPfProdWarp) {
+    // ======================= producer warp =====================================
+    for (int t = 0; t + 2 < ntiles || 2 * t + kPfRawSlots < nhalves; ++t) {
+      const int i0 = 2 * t + kPfRawSlots;
+      if (i0 >= nhalves) break;
+      mbar_wait(raw_free(t & 1), (t >> 1) & 1, abort_flag, p.status, 1u);
+      // warp-uniform decision (issue_raw synchronizes the warp)
+      if (__shfl_sync(~0u, (int)*abort_flag, 0) != 0) break;
+      issue_raw(i0, nhalves - i0 < 2 ? nhalves - i0 : 2);
+    }
+    if (lane == 0) {                             // own bulk copies still in flight (after a give-up)
       for (int i = max(0, issued - kPfRawSlots); i < issued; ++i)
         mbar_drain(raw_full(i % kPfRawSlots), (i / kPfRawSlots) & 1, p.status);
     }
+    __syncwarp();
   } else if (warp == kPfMmaWarp) {
     // ======================= MMA warp ==========================================
     constexpr uint32_t idesc_s = f16_idesc(kPfBM, kPfBN, false);
