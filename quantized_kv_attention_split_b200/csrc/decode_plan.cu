@@ -12,6 +12,9 @@ namespace {
 int max_ctas_per_sm(int D) { return dec_ctas_per_sm(D); }
 // Largest grid: the merge tree's second level then has at most 48 groups of 8.
 constexpr int64_t kMaxGrid = 8 * 48;
+// Partials of at least this many floats count as large (16 rows x D = 256 do).
+constexpr int64_t kBigPartial = 2048;
+constexpr int64_t kBigPartMinStages = 2;
 
 int sm_count() {
   int dev = 0, n = 0;
@@ -89,6 +92,13 @@ bool plan_decode(int D, int bits, int gs, int fmt, int out_f32, int B, int Hq, i
   int64_t grid = (int64_t)sms * occ;
   grid = std::min<int64_t>(grid, plan->total_stages);
   grid = std::min<int64_t>(grid, kMaxGrid);            // merge scratch holds <= 48 groups
+  // A CTA's partial (rows x D fp32) is written, read back and merged; when it
+  // is large (many query rows per KV head, wide heads) give every CTA several
+  // stages, so that partials stay a small fraction of the bytes streamed.
+  if ((int64_t)plan->hpc * D >= kBigPartial) {
+    const int64_t cap = (plan->total_stages + kBigPartMinStages - 1) / kBigPartMinStages;
+    grid = std::min<int64_t>(grid, std::max<int64_t>(1, cap));
+  }
   plan->grid = (int)std::max<int64_t>(1, grid);
   plan->smem = ops.smem;
   decode_ws_layout((size_t)plan->units, (size_t)plan->hpc, D, max_grid(D), plan);
