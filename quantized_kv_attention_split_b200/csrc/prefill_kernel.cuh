@@ -272,55 +272,82 @@ __host__ __device__ constexpr int k_pos(int e) {
   }
 }
 
-// Dequantizes the 32 code rows of one packed half tile into rows row0h.. of an
-// fp16 [key][d] tile with 128-byte swizzled rows; value = scale * code + bias
-// rounded once, rows at or past `nv` (keys past L) are written as zeros.
+// Converts one 16-byte chunk of codes (16 codes of 8 bits or 32 of 4 bits,
+// all in one group) of key row `row`, chunk index u of the row, to fp16 in the
+// 128-byte swizzled [key][d] tile: value = scale * code + bias rounded once.
 template <int D, int BITS, int GS, bool Q8>
-__device__ __forceinline__ void pf_dequant(const uint8_t* codes, const uint16_t* sc,
-                                           const uint16_t* bi, uint8_t* dst, int row0h, int nv,
-                                           int chunk0) {
+__device__ __forceinline__ void pf_convert_chunk(uint4 w4, __half2 s2, __half2 b2, uint8_t* dst,
+                                                 int row, int u) {
+  const __half2 off = __float2half2_rn(Q8 ? 1152.f : 1024.f);   // Q8 codes are stored +128
+  const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
+  if constexpr (BITS == 8) {
+    uint32_t o[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t x = Q8 ? (wv[k] ^ 0x80808080u) : wv[k];
+      const uint32_t h0 = prmt(x, 0x64646464u, 0x4140u);   // (1024 + byte0, 1024 + byte1)
+      const uint32_t h1 = prmt(x, 0x64646464u, 0x4342u);
+      const __half2 v0 = __hfma2(__hsub2(*reinterpret_cast<const __half2*>(&h0), off), s2, b2);
+      const __half2 v1 = __hfma2(__hsub2(*reinterpret_cast<const __half2*>(&h1), off), s2, b2);
+      o[2 * k] = *reinterpret_cast<const uint32_t*>(&v0);
+      o[2 * k + 1] = *reinterpret_cast<const uint32_t*>(&v1);
+    }
+    *reinterpret_cast<uint4*>(dst + sw128_off(row, u * 16)) = make_uint4(o[0], o[1], o[2], o[3]);
+    *reinterpret_cast<uint4*>(dst + sw128_off(row, u * 16 + 8)) = make_uint4(o[4], o[5], o[6], o[7]);
+  } else {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {      // word k: d = 32u + 8k .. +7, nibbles (j, j+4) -> (2j, 2j+1)
+      uint32_t o[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t x = ((wv[k] >> (4 * j)) & 0x000F000Fu) | 0x64006400u;
+        const __half2 v = __hfma2(__hsub2(*reinterpret_cast<const __half2*>(&x), off), s2, b2);
+        o[j] = *reinterpret_cast<const uint32_t*>(&v);
+      }
+      *reinterpret_cast<uint4*>(dst + sw128_off(row, u * 32 + 8 * k)) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
+}
+
+// Dequantizes a 64-key operand tile from its two packed half tiles (raw[h]:
+// codes at +codes_off, scales at +sc_off, biases at +bi_off); rows at or past
+// nv[h] of half h (keys past L) are written as zeros through a zero scale and
+// bias.  Every load of the thread's chunks is issued before any conversion.
+template <int D, int BITS, int GS, bool Q8>
+__device__ __forceinline__ void pf_dequant_tile(const uint8_t* const raw[2], int codes_off,
+                                                int sc_off, int bi_off, uint8_t* dst,
+                                                const int nv[2], int chunk0) {
   using C = PfCfg<D, BITS, GS, Q8>;
   constexpr int NCH = kPfRawKeys * C::UPR;
   constexpr int ITERS = (NCH + kPfDqThreads - 1) / kPfDqThreads;
-  const __half2 off = __float2half2_rn(Q8 ? 1152.f : 1024.f);   // Q8 codes are stored +128
+  uint4 w[2][ITERS];
+  __half2 s2[2][ITERS], b2[2][ITERS];
 #pragma unroll
-  for (int it = 0; it < ITERS; ++it) {
-    const int i = chunk0 + it * kPfDqThreads;
-    if (NCH % kPfDqThreads != 0 && i >= NCH) break;   // whole warps drop out together
-    const int key = i / C::UPR, u = i - key * C::UPR;
-    const uint4 w4 = *reinterpret_cast<const uint4*>(codes + i * 16);
-    const int g = (u * C::CPC) / GS;
-    // rows at or past nv: scale and bias 0 make every value exactly 0 (codes are finite)
-    const bool live = key < nv;
-    const __half2 s2 = __half2half2(__ushort_as_half(live ? sc[key * C::NG + g] : (uint16_t)0));
-    const __half2 b2 = Q8 ? __float2half2_rn(0.f)
-                          : __half2half2(__ushort_as_half(live ? bi[key * C::NG + g] : (uint16_t)0));
-    const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
-    if constexpr (BITS == 8) {
-      uint32_t o[8];
+  for (int h = 0; h < 2; ++h) {
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const uint32_t x = Q8 ? (wv[k] ^ 0x80808080u) : wv[k];
-        const uint32_t h0 = prmt(x, 0x64646464u, 0x4140u);   // (1024 + byte0, 1024 + byte1)
-        const uint32_t h1 = prmt(x, 0x64646464u, 0x4342u);
-        const __half2 v0 = __hfma2(__hsub2(*reinterpret_cast<const __half2*>(&h0), off), s2, b2);
-        const __half2 v1 = __hfma2(__hsub2(*reinterpret_cast<const __half2*>(&h1), off), s2, b2);
-        o[2 * k] = *reinterpret_cast<const uint32_t*>(&v0);
-        o[2 * k + 1] = *reinterpret_cast<const uint32_t*>(&v1);
+    for (int it = 0; it < ITERS; ++it) {
+      const int i = chunk0 + it * kPfDqThreads;
+      if (NCH % kPfDqThreads == 0 || i < NCH) {      // whole warps drop out together
+        const int key = i / C::UPR, u = i - key * C::UPR;
+        const int g = (u * C::CPC) / GS;
+        const bool live = key < nv[h];
+        const uint16_t* sc = reinterpret_cast<const uint16_t*>(raw[h] + sc_off);
+        const uint16_t* bi = reinterpret_cast<const uint16_t*>(raw[h] + bi_off);
+        w[h][it] = *reinterpret_cast<const uint4*>(raw[h] + codes_off + i * 16);
+        s2[h][it] = __half2half2(__ushort_as_half(live ? sc[key * C::NG + g] : (uint16_t)0));
+        b2[h][it] = Q8 ? __float2half2_rn(0.f)
+                       : __half2half2(__ushort_as_half(live ? bi[key * C::NG + g] : (uint16_t)0));
       }
-      *reinterpret_cast<uint4*>(dst + sw128_off(row0h + key, u * 16)) = make_uint4(o[0], o[1], o[2], o[3]);
-      *reinterpret_cast<uint4*>(dst + sw128_off(row0h + key, u * 16 + 8)) = make_uint4(o[4], o[5], o[6], o[7]);
-    } else {
+    }
+  }
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {      // word k: d = 32u + 8k .. +7, nibbles (j, j+4) -> (2j, 2j+1)
-        uint32_t o[4];
+  for (int h = 0; h < 2; ++h) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint32_t x = ((wv[k] >> (4 * j)) & 0x000F000Fu) | 0x64006400u;
-          const __half2 v = __hfma2(__hsub2(*reinterpret_cast<const __half2*>(&x), off), s2, b2);
-          o[j] = *reinterpret_cast<const uint32_t*>(&v);
-        }
-        *reinterpret_cast<uint4*>(dst + sw128_off(row0h + key, u * 32 + 8 * k)) = make_uint4(o[0], o[1], o[2], o[3]);
+    for (int it = 0; it < ITERS; ++it) {
+      const int i = chunk0 + it * kPfDqThreads;
+      if (NCH % kPfDqThreads == 0 || i < NCH) {
+        const int key = i / C::UPR, u = i - key * C::UPR;
+        pf_convert_chunk<D, BITS, GS, Q8>(w[h][it], s2[h][it], b2[h][it], dst, h * kPfRawKeys + key, u);
       }
     }
   }
@@ -506,27 +533,28 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
     for (int bt = 0; bt < 5; ++bt)
       if ((lane >> bt) & 1) cl ^= pf_lane_col(D, BITS, bt);
     const int chunk0 = (dq >> 5) * 32 + cl;
-    constexpr int MH = C::META_BYTES / 2;        // metadata array stride in halves
     // one operand tile (K or V) from the tile's two half tiles; a half tile
     // past the last one is written as zeros (its keys are never visible)
     auto convert = [&](int t, bool is_v, uint8_t* dst) {
-#pragma unroll 1
+      const uint8_t* raw[2];
+      int nv[2];
+#pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int i = 2 * t + h;
         const bool present = i < nhalves;
         const int slot = i % kPfRawSlots;
         if (present && !is_v)                    // V reuses the half tiles K waited for
           mbar_wait(raw_full(slot), (i / kPfRawSlots) & 1, abort_flag, p.status, 1u);
-        const uint8_t* raw = smem + C::RAW_OFF + slot * C::RAW_BYTES;
-        const uint16_t* meta = reinterpret_cast<const uint16_t*>(raw + 2 * C::RAW_CODES);
+        raw[h] = smem + C::RAW_OFF + slot * C::RAW_BYTES;
         const int64_t key0 = (int64_t)i * kPfRawKeys;
-        const int nv = !present ? 0 : (L - key0 < kPfRawKeys ? (int)(L - key0) : kPfRawKeys);
-        if (!is_v)
-          pf_dequant<D, BITS, GS, Q8>(raw, meta, meta + MH, dst, h * kPfRawKeys, nv, chunk0);
-        else
-          pf_dequant<D, BITS, GS, Q8>(raw + C::RAW_CODES, meta + (Q8 ? 1 : 2) * MH, meta + 3 * MH,
-                                      dst, h * kPfRawKeys, nv, chunk0);
+        nv[h] = !present ? 0 : (L - key0 < kPfRawKeys ? (int)(L - key0) : kPfRawKeys);
       }
+      if (!is_v)
+        pf_dequant_tile<D, BITS, GS, Q8>(raw, 0, 2 * C::RAW_CODES, 2 * C::RAW_CODES + C::META_BYTES,
+                                         dst, nv, chunk0);
+      else
+        pf_dequant_tile<D, BITS, GS, Q8>(raw, C::RAW_CODES, 2 * C::RAW_CODES + (Q8 ? 1 : 2) * C::META_BYTES,
+                                         2 * C::RAW_CODES + 3 * C::META_BYTES, dst, nv, chunk0);
     };
     for (int t = 0; t < ntiles; ++t) {
       const int s = t & 1;
