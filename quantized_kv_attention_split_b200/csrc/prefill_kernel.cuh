@@ -309,25 +309,30 @@ __device__ __forceinline__ void pf_convert_chunk(uint4 w4, __half2 s2, __half2 b
   }
 }
 
-// Dequantizes a 64-key operand tile from its two packed half tiles (raw[h]:
-// codes at +codes_off, scales at +sc_off, biases at +bi_off); rows at or past
-// nv[h] of half h (keys past L) are written as zeros through a zero scale and
-// bias.  Every load of the thread's chunks is issued before any conversion.
+// A thread's share of one 64-key operand tile (K or V): its 16-byte code
+// chunks of both packed half tiles with their scale and bias, loaded from the
+// raw ring ahead of the conversion.  raw[h]: the half tile's slot; codes at
+// +codes_off, scales at +sc_off, biases at +bi_off; rows at or past nv[h]
+// (keys past L) get scale and bias 0, hence zeros.
 template <int D, int BITS, int GS, bool Q8>
-__device__ __forceinline__ void pf_dequant_tile(const uint8_t* const raw[2], int codes_off,
-                                                int sc_off, int bi_off, uint8_t* dst,
-                                                const int nv[2], int chunk0) {
+struct PfChunks {
   using C = PfCfg<D, BITS, GS, Q8>;
-  constexpr int NCH = kPfRawKeys * C::UPR;
-  constexpr int ITERS = (NCH + kPfDqThreads - 1) / kPfDqThreads;
+  static constexpr int NCH = kPfRawKeys * C::UPR;
+  static constexpr int ITERS = (NCH + kPfDqThreads - 1) / kPfDqThreads;
   uint4 w[2][ITERS];
   __half2 s2[2][ITERS], b2[2][ITERS];
+
+  __device__ __forceinline__ static bool has(int chunk0, int it) {
+    return NCH % kPfDqThreads == 0 || chunk0 + it * kPfDqThreads < NCH;   // whole warps
+  }
+  __device__ __forceinline__ void load(const uint8_t* const raw[2], int codes_off, int sc_off,
+                                       int bi_off, const int nv[2], int chunk0) {
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
+    for (int h = 0; h < 2; ++h) {
 #pragma unroll
-    for (int it = 0; it < ITERS; ++it) {
-      const int i = chunk0 + it * kPfDqThreads;
-      if (NCH % kPfDqThreads == 0 || i < NCH) {      // whole warps drop out together
+      for (int it = 0; it < ITERS; ++it) {
+        if (!has(chunk0, it)) continue;
+        const int i = chunk0 + it * kPfDqThreads;
         const int key = i / C::UPR, u = i - key * C::UPR;
         const int g = (u * C::CPC) / GS;
         const bool live = key < nv[h];
@@ -340,18 +345,19 @@ __device__ __forceinline__ void pf_dequant_tile(const uint8_t* const raw[2], int
       }
     }
   }
+  __device__ __forceinline__ void store(uint8_t* dst, int chunk0) const {
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
+    for (int h = 0; h < 2; ++h) {
 #pragma unroll
-    for (int it = 0; it < ITERS; ++it) {
-      const int i = chunk0 + it * kPfDqThreads;
-      if (NCH % kPfDqThreads == 0 || i < NCH) {
+      for (int it = 0; it < ITERS; ++it) {
+        if (!has(chunk0, it)) continue;
+        const int i = chunk0 + it * kPfDqThreads;
         const int key = i / C::UPR, u = i - key * C::UPR;
         pf_convert_chunk<D, BITS, GS, Q8>(w[h][it], s2[h][it], b2[h][it], dst, h * kPfRawKeys + key, u);
       }
     }
   }
-}
+};
 
 template <int D, int BITS, int GS, bool Q8>
 __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const PrefillParams p) {
@@ -533,9 +539,10 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
     for (int bt = 0; bt < 5; ++bt)
       if ((lane >> bt) & 1) cl ^= pf_lane_col(D, BITS, bt);
     const int chunk0 = (dq >> 5) * 32 + cl;
-    // one operand tile (K or V) from the tile's two half tiles; a half tile
-    // past the last one is written as zeros (its keys are never visible)
-    auto convert = [&](int t, bool is_v, uint8_t* dst) {
+    // the tile's two packed half tiles; a half tile past the last one gives
+    // zeros (its keys are never visible)
+    for (int t = 0; t < ntiles; ++t) {
+      const int s = t & 1;
       const uint8_t* raw[2];
       int nv[2];
 #pragma unroll
@@ -543,32 +550,27 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
         const int i = 2 * t + h;
         const bool present = i < nhalves;
         const int slot = i % kPfRawSlots;
-        if (present && !is_v)                    // V reuses the half tiles K waited for
-          mbar_wait(raw_full(slot), (i / kPfRawSlots) & 1, abort_flag, p.status, 1u);
+        if (present) mbar_wait(raw_full(slot), (i / kPfRawSlots) & 1, abort_flag, p.status, 1u);
         raw[h] = smem + C::RAW_OFF + slot * C::RAW_BYTES;
         const int64_t key0 = (int64_t)i * kPfRawKeys;
         nv[h] = !present ? 0 : (L - key0 < kPfRawKeys ? (int)(L - key0) : kPfRawKeys);
       }
-      if (!is_v)
-        pf_dequant_tile<D, BITS, GS, Q8>(raw, 0, 2 * C::RAW_CODES, 2 * C::RAW_CODES + C::META_BYTES,
-                                         dst, nv, chunk0);
-      else
-        pf_dequant_tile<D, BITS, GS, Q8>(raw, C::RAW_CODES, 2 * C::RAW_CODES + (Q8 ? 1 : 2) * C::META_BYTES,
-                                         2 * C::RAW_CODES + 3 * C::META_BYTES, dst, nv, chunk0);
-    };
-    for (int t = 0; t < ntiles; ++t) {
-      const int s = t & 1;
+      // K and V chunks of this thread come in together; V converts after K
+      PfChunks<D, BITS, GS, Q8> kch, vch;
+      kch.load(raw, 0, 2 * C::RAW_CODES, 2 * C::RAW_CODES + C::META_BYTES, nv, chunk0);
+      vch.load(raw, C::RAW_CODES, 2 * C::RAW_CODES + (Q8 ? 1 : 2) * C::META_BYTES,
+               2 * C::RAW_CODES + 3 * C::META_BYTES, nv, chunk0);
       if (t >= kPfKSlots)                        // K slot free once S of tile t-2 is done
         mbar_wait(s_full(s), ((t - 2) >> 1) & 1, abort_flag, p.status, 1u);
-      convert(t, false, smem + C::K_OFF + s * C::KV_BYTES);
+      kch.store(smem + C::K_OFF + s * C::KV_BYTES, chunk0);
       fence_async_smem();
       mbar_arrive(k_ready(s));
+      mbar_arrive(raw_free(s));                  // this thread is done with the raw slots
       if (t >= kPfVSlots)                        // V slot free once P V of tile t-2 is done
         mbar_wait(pv_done(s), ((t - 2) >> 1) & 1, abort_flag, p.status, 1u);
-      convert(t, true, smem + C::V_OFF + s * C::KV_BYTES);
+      vch.store(smem + C::V_OFF + s * C::KV_BYTES, chunk0);
       fence_async_smem();
       mbar_arrive(v_ready(s));
-      mbar_arrive(raw_free(s));                  // raw slots of half tiles 2t, 2t+1 are free
     }
   } else if (warp == kPfProdWarp) {
     // ======================= producer warp =====================================
