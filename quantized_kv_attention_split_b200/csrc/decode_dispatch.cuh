@@ -10,15 +10,16 @@ namespace qkv {
 struct DecodeOps {
   int (*occupancy)();
   cudaError_t (*launch)(const DecodePlan&, const DecodeParams&, cudaStream_t);
-  int tk;
+  int tk;      // keys per block
   int nc;
+  int teams;   // teams of warps per CTA, each streaming its own blocks
   size_t smem;
 };
 
 template <int D, int BITS, int GS, bool Q8, int NC, bool F32>
 DecodeOps make_decode_ops() {
   using I = DecodeInstance<D, BITS, GS, Q8, NC, F32>;
-  return DecodeOps{&I::max_ctas_per_sm, &I::launch, I::C::TK, NC, (size_t)I::C::SMEM};
+  return DecodeOps{&I::max_ctas_per_sm, &I::launch, I::C::TK, NC, I::C::NTEAM, (size_t)I::C::SMEM};
 }
 
 // Instances of one head dimension; nc in {1, 2, 4}; f32 selects the

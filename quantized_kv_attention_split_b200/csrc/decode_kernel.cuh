@@ -8,14 +8,18 @@
 //
 // How (B200 design; the Metal kernel on the pages walks every key of one head
 // with one threadgroup and has no split, no GQA sharing and no tensor cores):
-//  * Work: units (batch, kv-head, chunk-group of <=32 query heads) x stages of
-//    TK keys, flattened and cut evenly over the grid, so every SM gets the
-//    same number of stages.  A CTA touches at most two units partially; a
-//    partial result (running max m, sum l, unnormalized o) goes to workspace
-//    and the last CTA of a unit to finish (atomic ticket) merges them
-//    (log-sum-exp rescaling) -- one launch, no waiting.
-//  * Staging: all 256 threads stream codes and scales with 16-byte cp.async
-//    (zero-filled past L) into an NSTAGE-deep shared-memory ring.  Code tiles
+//  * Work: units (batch, kv-head, chunk-group of <=32 query heads) x blocks
+//    of BK (16 or 32) keys, flattened and cut evenly over one CTA per SM.  A
+//    CTA touches at most two units partially; a partial result (running max
+//    m, sum l, unnormalized o) goes to workspace and the last CTA of a unit
+//    to finish (atomic ticket) merges them (log-sum-exp rescaling) -- one
+//    launch, no waiting.  The launch is a programmatic dependent launch: its
+//    set-up overlaps the previous kernel of the stream.
+//  * Teams: the warps of a CTA form teams (one warp per 8-row head chunk).
+//    A team streams its own blocks -- handed out in order through a shared
+//    counter, so fast teams take more -- with 16-byte cp.async (zero-filled
+//    past L) into its own NSTAGE-deep shared-memory ring and meets only its
+//    own warps; there is no CTA-wide barrier until the epilogue.  Code tiles
 //    are XOR-swizzled per 128-byte line so both fragment read patterns below
 //    are bank-conflict-free.
 //  * Scores: one m16n8k16 tensor op per 16 keys x 8 query heads x 16 dims.
@@ -25,15 +29,16 @@
 //    scale and the bias term (bias * sum of q over the group, the identity the
 //    Metal kernel uses with its query_sum) are applied in fp32 afterwards.
 //    Q8_0 codes are offset by 128 (xor 0x80) and corrected the same way.
-//  * Online softmax in base 2 with warp shuffles over the 16 keys.
+//  * Online softmax in base 2 with warp shuffles over the block's keys.
 //  * Values: O^T[e,h] += V^T[e,j] (P[j,h]*s_v[j]*2^tau): V codes are the A
-//    operand (pairs of keys per register, built with byte permutes), the
-//    probabilities times the per-key value scale are the B operand, moved
-//    from the score fragment layout with movmatrix.trans.  tau normalizes each
-//    16-key block so the fp16 operand never over- or underflows; the block
-//    result is folded into fp32 accumulators.  The value bias term
-//    sum_j P[j,h]*b_v[j] is accumulated in fp32.  With fp32 output the B
-//    operand is split into fp16 hi + lo parts (two tensor ops).
+//    operand (transposing ldmatrix loads hand every lane a key pair per
+//    register), the probabilities times the per-key value scale are the B
+//    operand, moved from the score fragment layout with movmatrix.trans.
+//    tau (per warp and group, lowered when a larger value scale appears, with
+//    an exact power-of-two rescale of O) keeps the fp16 operand below 2^15.
+//    The value bias term sum_j P[j,h]*b_v[j] is accumulated in fp32.  With
+//    fp32 output the B operand is split into fp16 hi + lo parts (two tensor
+//    ops).
 #pragma once
 
 #include "qkv_common.cuh"
@@ -41,11 +46,14 @@
 
 namespace qkv {
 
-// 8 warps per CTA; two CTAs per SM for D <= 128 (independent CTAs overlap
-// each other's stage boundaries), one for D = 256 (more registers per thread).
-__host__ __device__ constexpr int dec_warps(int) { return 8; }
-constexpr int kDecWarpsMax = 8;
-__host__ __device__ constexpr int dec_ctas_per_sm(int D) { return D <= 128 ? 2 : 1; }
+// 16 warps per CTA for D <= 128, 8 for D = 256 (about 250 registers per
+// thread); one CTA per SM.  The warps form teams of NC, one warp per 8-row head
+// chunk; every team streams its own blocks of keys through its own
+// shared-memory ring, so the main loop has no CTA-wide barrier and warps that
+// are ahead never wait for warps that are behind.
+__host__ __device__ constexpr int dec_warps(int D) { return D <= 128 ? 16 : 8; }
+constexpr int kDecWarpsMax = 16;
+__host__ __device__ constexpr int dec_ctas_per_sm(int) { return 1; }
 
 // XOR coefficients (3 bits each, for line bits 0..3) of the 16-byte-unit
 // swizzle inside each 128-byte line of a staged code tile, found by exhaustive
@@ -102,31 +110,44 @@ struct DecCfg {
   static constexpr int KPG = GS / 16;          // k-steps per group == V m-tiles per group
   static constexpr int KSTEPS = D / 16;
   static constexpr int MT = D / 16;
-  static constexpr int CB = GS * BITS / 64;    // V chunk bytes per thread per (key, group)
-  static constexpr int CW = CB >= 4 ? CB / 4 : 1;
   static constexpr int NMETA = Q8 ? 2 : 4;
   static constexpr int MROW = NG * 2;          // meta bytes per key per array
   static constexpr int NWARP = dec_warps(D);
   static constexpr int NTHR = 32 * NWARP;
-  static constexpr int WPC = NWARP / NC;       // warps per head chunk
-  // ring budget per CTA (228 KB per SM holds two CTAs of 108 KB plus their
-  // reserved 1 KB each)
-  static constexpr int BUDGET = D <= 128 ? 110592 : 224 * 1024;
-  // 16-key blocks per warp per stage: two when three such stages fit, else one
-  static constexpr int STAGE2 = 2 * (32 * WPC) * RB + NMETA * (((32 * WPC * MROW + 127) / 128) * 128);
-  static constexpr int SUB = 3 * STAGE2 <= BUDGET ? 2 : 1;
-  static constexpr int TK = 16 * SUB * WPC;      // keys per stage
-  static constexpr int CODES = TK * RB;
-  static constexpr int META = ((TK * MROW + 127) / 128) * 128;
-  static constexpr int META_UNITS = TK * MROW / 16;
-  static constexpr int STAGE = 2 * CODES + NMETA * META;
-  static constexpr int NSTAGE = BUDGET / STAGE > 6 ? 6 : (BUDGET / STAGE < 2 ? 2 : BUDGET / STAGE);
-  // epilogue: per-warp partial rows
-  static constexpr int EPI = NWARP * (8 * D + 16) * 4;
-  static constexpr int RING = NSTAGE * STAGE > EPI ? NSTAGE * STAGE : EPI;
-  static constexpr int QSB = NC * 8 * D * 4;            // fp32 query rows (in the last ring slot)
-  static constexpr int SMEM = RING > (NSTAGE - 1) * STAGE + QSB ? RING : (NSTAGE - 1) * STAGE + QSB;
-  static_assert(SMEM <= 227 * 1024, "shared memory budget");
+  static constexpr int NTEAM = NWARP / NC;     // teams; each has one warp per head chunk
+  static constexpr int TTHR = 32 * NC;         // threads per team
+  static constexpr int WPC = NTEAM;            // warps per head chunk
+  static constexpr int QROW = 2 * D + 4;       // staged query row: raw 16-bit values + 4 bytes of padding
+  static constexpr int QSB = ((NC * 8 * QROW + 127) / 128) * 128;
+  // dynamic shared memory of the one CTA of an SM (227 KB less static data)
+  static constexpr int BUDGET = 227 * 1024 - 2048;
+  static constexpr int r16(int x) { return (x + 15) / 16 * 16; }
+  static constexpr int r128(int x) { return (x + 127) / 128 * 128; }
+  static constexpr int stage_bytes(int sub) { return r128(2 * 16 * sub * RB + NMETA * r16(16 * sub * MROW)); }
+  // 16-key sub-blocks per block: two when three such stages per team fit
+  // (D = 256 keeps one: its register budget is spent)
+  static constexpr int SUB = (D <= 128 && NTEAM * 3 * stage_bytes(2) + QSB <= BUDGET) ? 2 : 1;
+  static constexpr int BK = 16 * SUB;          // keys per block
+  static constexpr int TK = BK;
+  static constexpr int CODES = BK * RB;
+  static constexpr int META = r16(BK * MROW);
+  static constexpr int META_UNITS = BK * MROW / 16;
+  static constexpr int KU = BK * UPR;          // 16-byte code units per tile
+  static constexpr int MU = NMETA * META_UNITS;
+  static constexpr int STAGE = stage_bytes(SUB);
+  static constexpr int NS_FIT = (BUDGET - QSB) / (NTEAM * STAGE);
+  static constexpr int NSTAGE = NS_FIT > 6 ? 6 : NS_FIT;
+  static constexpr int TRING = NSTAGE * STAGE;          // one team's ring
+  static constexpr int QOFF = NTEAM * TRING;            // query rows after the rings
+  // epilogue (after every ring is drained): per-warp partial rows, then the
+  // per-(row, warp) combine weights and per-row (m, l)
+  static constexpr int WSW = 8 * D + 16;               // floats per warp
+  static constexpr int EPI_W = NWARP * WSW * 4;
+  static constexpr int EPI = EPI_W + NC * 8 * (NTEAM + 1) * 4 + NC * 8 * 2 * 4;
+  static constexpr int SMEM = QOFF + QSB > EPI ? QOFF + QSB : EPI;
+  static_assert(NSTAGE >= 3, "at least three stages per team");
+  static_assert(SMEM <= BUDGET, "shared memory budget");
+  static_assert(META_UNITS * 16 == BK * MROW, "metadata rows must fill 16-byte units");
   static constexpr uint32_t SWZ = swizzle_coeffs(D, BITS, GS);   // key tile
   static constexpr uint32_t SWZV = vswizzle_coeffs(RB);          // value tile
   static_assert(D % GS == 0, "D must be a multiple of the group size");
@@ -257,6 +278,13 @@ __device__ __noinline__ void merge_unit(const float* ml, const float* po, int n,
   }
 }
 
+// Atomic add with acquire-release semantics at GPU scope.
+__device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned* p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], %2;\n" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
 // Transposing shared-memory matrix loads (8x8 of 16-bit elements per matrix).
 __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1,
                                               uint32_t& r2, uint32_t& r3) {
@@ -301,28 +329,53 @@ __device__ __forceinline__ void meta_row(const uint8_t* base, int r, uint32_t* w
 }
 
 template <int D, int BITS, int GS, bool Q8, int NC, bool F32OUT>
-__global__ void __launch_bounds__(32 * dec_warps(D), dec_ctas_per_sm(D))
-qsdpa_decode_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(32 * dec_warps(D), 1)
+qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
   using C = DecCfg<D, BITS, GS, Q8, NC>;
-  constexpr int NG = C::NG, KPG = C::KPG, MT = C::MT, TK = C::TK, NSTAGE = C::NSTAGE;
+  constexpr int NG = C::NG, KPG = C::KPG, MT = C::MT, BK = C::BK, NSTAGE = C::NSTAGE;
+  constexpr int NTEAM = C::NTEAM, TTHR = C::TTHR;
   constexpr int HPC = NC * 8;
   constexpr int MW = NG == 1 ? 1 : NG / 2;     // 32-bit words of one key's metadata row
   extern __shared__ __align__(128) uint8_t smem[];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
-  const int chunk = warp / C::WPC, sub = warp % C::WPC;
-  const int64_t S = p.stages_per_unit, T = p.total_stages;
+  const int team = warp / NC, chunk = warp - team * NC;
+  const int ttid = tid - team * TTHR;          // thread index within the team
+  uint8_t* const ring = smem + team * C::TRING;
+  uint8_t* const qst = smem + C::QOFF;
+  const int64_t S = p.stages_per_unit, T = p.total_stages;   // blocks of BK keys
   const int64_t nC = gridDim.x;
   const int64_t lo = udiv64((int64_t)blockIdx.x * T, nC), hi = udiv64(((int64_t)blockIdx.x + 1) * T, nC);
   const int64_t first_unit = udiv64(lo, S);
   __shared__ int s_flag;
+  __shared__ int s_next;                 // next block of the segment to hand out
+  __shared__ int s_grab[NTEAM][2];       // a team's next block, double-buffered
 
+  // The launch's parameters sit in constant-bank lines that no SM has cached
+  // yet: touch every line from a different warp so that the misses overlap
+  // instead of following each other through the first instructions.
+  if (lane == 0 && warp * 64 < (int)sizeof(DecodeParams)) {
+    const uint32_t v = reinterpret_cast<const uint32_t*>(&p)[warp * 16];
+    asm volatile("" :: "r"(v));
+  }
+  if (tid == 0) s_next = NTEAM * (NSTAGE - 1);
+  __syncthreads();
+
+  // the threads of one team meet here (one warp: a warp barrier)
+  auto team_sync = [&]() {
+    if constexpr (NC == 1) __syncwarp();
+    else asm volatile("bar.sync %0, %1;\n" :: "r"(1 + team), "n"(TTHR) : "memory");
+  };
+
+  // A CTA's range [lo, hi) of (unit, block) pairs is walked as segments, one
+  // per unit it touches; the teams share a segment's blocks through s_next.
   for (int64_t x = lo; x < hi;) {
     const int64_t u = udiv64(x, S);
     const int s0 = (int)(x - u * S);
     const int s1 = (int)(min(hi, (u + 1) * S) - u * S);
     x = u * S + s1;
+    const int nblk = s1 - s0;
 
     const int64_t uh = udiv64(u, p.ncg);                 // (batch, kv head)
     const int cg = (int)(u - uh * p.ncg);
@@ -331,144 +384,98 @@ qsdpa_decode_kernel(const DecodeParams p) {
     const int64_t row0 = ((int64_t)b * p.Hkv + hkv) * p.Lcap;   // first cache row of this head
     const int hbase = cg * HPC;                                  // first local row of the CTA
 
-    const uint8_t* gK = p.kc + row0 * C::RB;
-    const uint8_t* gV = p.vc + row0 * C::RB;
-    const uint8_t* gKs = reinterpret_cast<const uint8_t*>(p.ks + row0 * NG);
-    const uint8_t* gKb = Q8 ? gKs : reinterpret_cast<const uint8_t*>(p.kb + row0 * NG);
-    const uint8_t* gVs = reinterpret_cast<const uint8_t*>(p.vs + row0 * NG);
-    const uint8_t* gVb = Q8 ? gVs : reinterpret_cast<const uint8_t*>(p.vb + row0 * NG);
     const int64_t L = p.L;
 
-    // copy plan: 16-byte unit i of a stage is row (i mod CU) / UPR of the K
-    // tile (i < CU) or of the V tile.  When CU is a multiple of the thread
-    // count every unit of a thread lies in a line with the same swizzle.
-    constexpr int CU = TK * C::UPR;
-    constexpr int NU = (2 * CU + C::NTHR - 1) / C::NTHR;
-    const int fx_tid = swz_line<C::SWZ>((tid >> 3) & 15);
-    const int fx_tid_v = swz_line<C::SWZV>((tid >> 3) & 15);
-
-    constexpr bool META1 = C::NMETA * C::META_UNITS <= C::NTHR;   // one metadata unit per thread
-    auto issue_stage = [&](int stage, int buf) {
-      const uint32_t sbase = smem_u32(smem + buf * C::STAGE);
-      const int64_t key0 = (int64_t)stage * TK;
-      const int nvalid = (int)(L - key0 < (int64_t)TK ? L - key0 : (int64_t)TK);      // rows of this stage below L
-      if (CU % C::NTHR == 0 && META1 && nvalid == TK) {
-        // a full stage: fixed per-thread offsets, no per-unit tests.  Unit
-        // tid + k * NTHR lies k * NTHR * 16 bytes further in both the source
-        // and (the swizzle acts on bits below that) the stage.
-        const uint8_t* ks = gK + key0 * C::RB + tid * 16;
-        const uint8_t* vs = gV + key0 * C::RB + tid * 16;
-        const uint32_t d0 = sbase + ((tid * 16) ^ fx_tid);
-        const uint32_t d0v = sbase + C::CODES + ((tid * 16) ^ fx_tid_v);
+    // Copy plan of one block (by its team): 16-byte unit i is row i / UPR of
+    // the K tile (i < KU) or of the V tile, then the metadata arrays.  Unit
+    // ttid + k * TTHR of a tile lies in line (ttid / 8) + k * TTHR / 8, and
+    // the swizzle is linear in the line bits, so it splits into a per-thread
+    // part and a per-k constant.
+    const int fx = swz_line<C::SWZ>((ttid >> 3) & 15);
+    const int fxv = swz_line<C::SWZV>((ttid >> 3) & 15);
+    auto issue_block = [&](int blk, int slot) {
+      const uint32_t sbase = smem_u32(ring + slot * C::STAGE);
+      const int64_t key0 = (int64_t)(s0 + blk) * BK;
+      const int nvalid = (int)(L - key0 < (int64_t)BK ? L - key0 : (int64_t)BK);
+      // global addresses are formed from the launch parameters each time
+      // (constant operands) rather than kept live across the loop
+      const int64_t grow = row0 + key0;                        // cache row of the block's first key
+      const uint8_t* kb0 = p.kc + grow * C::RB;
+      const uint8_t* vb0 = p.vc + grow * C::RB;
+      if (C::KU % TTHR == 0 && nvalid == BK) {
+        const uint8_t* ks = kb0 + ttid * 16;
+        const uint8_t* vs = vb0 + ttid * 16;
+        const uint32_t dk = sbase + ((ttid * 16) ^ fx);
+        const uint32_t dv = sbase + C::CODES + ((ttid * 16) ^ fxv);
 #pragma unroll
-        for (int k = 0; k < CU / C::NTHR; ++k) {
-          cp_async16(d0 + k * C::NTHR * 16, ks + k * C::NTHR * 16, 16);
-          cp_async16(d0v + k * C::NTHR * 16, vs + k * C::NTHR * 16, 16);
+        for (int k = 0; k < C::KU / TTHR; ++k) {
+          const int kx = swz_line<C::SWZ>((k * TTHR / 8) & 15);
+          const int kxv = swz_line<C::SWZV>((k * TTHR / 8) & 15);
+          cp_async16((dk ^ kx) + k * TTHR * 16, ks + k * TTHR * 16, 16);
+          cp_async16((dv ^ kxv) + k * TTHR * 16, vs + k * TTHR * 16, 16);
         }
-        if (tid < C::NMETA * C::META_UNITS) {
-          const int marr = tid / C::META_UNITS, mj = tid - marr * C::META_UNITS;
-          const uint8_t* gm = Q8 ? (marr == 0 ? gKs : gVs)
-                                 : (marr == 0 ? gKs : marr == 1 ? gKb : marr == 2 ? gVs : gVb);
-          cp_async16(sbase + 2 * C::CODES + marr * C::META + mj * 16, gm + key0 * C::MROW + mj * 16, 16);
-        }
-        return;
-      }
-      const uint8_t* kb0 = gK + key0 * C::RB;
-      const uint8_t* vb0 = gV + key0 * C::RB;
+      } else {
+        constexpr int NU = (2 * C::KU + TTHR - 1) / TTHR;
 #pragma unroll
-      for (int k = 0; k < NU; ++k) {
-        const int i = tid + k * C::NTHR;
-        if ((2 * CU) % C::NTHR == 0 || i < 2 * CU) {
-          const int which = i >= CU, j = which ? i - CU : i;
-          const bool ok = (j / C::UPR) < nvalid;
-          const uint8_t* src = (which ? vb0 : kb0) + (ok ? j * 16 : 0);
-          const int dst = (CU % C::NTHR == 0)
-                              ? which * C::CODES + ((j * 16) ^ (which ? fx_tid_v : fx_tid))
-                              : which * C::CODES + (which ? swz_offset<C::SWZV>(j * 16)
-                                                          : swz_offset<C::SWZ>(j * 16));
-          cp_async16(sbase + dst, src, ok ? 16 : 0);
+        for (int k = 0; k < NU; ++k) {
+          const int i = ttid + k * TTHR;
+          if ((2 * C::KU) % TTHR == 0 || i < 2 * C::KU) {
+            const int which = i >= C::KU, j = which ? i - C::KU : i;
+            const bool ok = (j / C::UPR) < nvalid;
+            const uint8_t* src = (which ? vb0 : kb0) + (ok ? j * 16 : 0);
+            const int dst = which ? C::CODES + swz_offset<C::SWZV>(j * 16) : swz_offset<C::SWZ>(j * 16);
+            cp_async16(sbase + dst, src, ok ? 16 : 0);
+          }
         }
       }
-      for (int i = tid; i < C::NMETA * C::META_UNITS; i += C::NTHR) {
-        const int arr = i / C::META_UNITS, j = i - arr * C::META_UNITS;
-        // affine: K scales, K biases, V scales, V biases; Q8_0: K scales, V scales
-        const uint8_t* gm = Q8 ? (arr == 0 ? gKs : gVs)
-                               : (arr == 0 ? gKs : arr == 1 ? gKb : arr == 2 ? gVs : gVb);
-        const bool ok = (j * 16) / C::MROW < nvalid;
-        const uint8_t* src = gm + (ok ? key0 * C::MROW + j * 16 : 0);
-        cp_async16(sbase + 2 * C::CODES + arr * C::META + j * 16, src, ok ? 16 : 0);
+      // metadata: affine K scales, K biases, V scales, V biases; Q8_0 K and V scales
+#pragma unroll
+      for (int k = 0; k < (C::MU + TTHR - 1) / TTHR; ++k) {
+        const int i = ttid + k * TTHR;
+        if (C::MU % TTHR == 0 || i < C::MU) {
+          const int arr = i / C::META_UNITS, j = i - arr * C::META_UNITS;
+          const uint16_t* gm = Q8 ? (arr == 0 ? p.ks : p.vs)
+                                  : (arr == 0 ? p.ks : arr == 1 ? p.kb : arr == 2 ? p.vs : p.vb);
+          const bool ok = (j * 16) / C::MROW < nvalid;
+          const uint8_t* src = reinterpret_cast<const uint8_t*>(gm + grow * NG) + (ok ? j * 16 : 0);
+          cp_async16(sbase + 2 * C::CODES + arr * C::META + j * 16, src, ok ? 16 : 0);
+        }
       }
     };
 
-    // fragment offsets inside a stage (fixed per lane).  The swizzle is
-    // linear in the line bits and a group never straddles a line, so it splits
-    // into a per-row part (computed once here), a per-group constant and, for
-    // the second 16-key block, the constant of a 16-row shift.
-    const int k0 = sub * 16 * C::SUB;
+    // fragment offsets inside a tile (fixed per lane).  The swizzle is linear
+    // in the line bits and a group never straddles a line, so it splits into
+    // a per-row part (computed once here), a per-group constant and, for the
+    // second 16-key sub-block, the constant of a 16-row shift.
     auto row_x = [&](int r) { return swz_line<C::SWZ>((r * C::RB) >> 7); };
-    const int xk0 = row_x(k0 + g), xk1 = row_x(k0 + g + 8);
+    const int xk0 = row_x(g), xk1 = row_x(g + 8);
     // value fragments: ldmatrix rows.  Lane l addresses row l % 8 of matrix
     // l / 8; matrices 0/1 hold keys 0-7, 2/3 keys 8-15 of the 16-key block, and
     // matrices 0/2 the first, 1/3 the second 16-byte unit of a unit pair (x2
     // loads for 4-bit groups of 32: matrix 0 keys 0-7, matrix 1 keys 8-15).
     constexpr bool VX2 = BITS == 4 && GS == 32;
-    const int vkey = k0 + (lane & 7) + (VX2 ? ((lane >> 3) & 1) * 8 : ((lane >> 4) & 1) * 8);
+    const int vkey = (lane & 7) + (VX2 ? ((lane >> 3) & 1) * 8 : ((lane >> 4) & 1) * 8);
     const int vunit = VX2 ? 0 : ((lane >> 3) & 1);
     auto koff = [&](int r, int x, int st, int G, int part) {
       return ((r * C::RB + G * C::GB + t * C::NW * 4 + part * 16) ^ x) ^
              swz_line<C::SWZ>((G * C::GB) >> 7) ^ swz_line<C::SWZ>((st * 16 * C::RB) >> 7);
     };
 
-    const int nst = s1 - s0;
-    // query rows: their (small) loads go out first, then the copies of the
-    // first stages; the rows are staged as fp32 in the ring's last slot, which
-    // the first NSTAGE-1 stages do not use
-    float* qst = reinterpret_cast<float*>(smem + (NSTAGE - 1) * C::STAGE);
+    // ---------------- prologue ----------------------------------------------
+    // The query rows go out first, then every team's first NSTAGE-1 blocks,
+    // so that the small loads do not queue behind the copies.  The rows are
+    // staged as raw 16-bit values in rows padded by 4 bytes, which keeps the
+    // fragment reads below free of bank conflicts.
     constexpr int QCH = HPC * D / 8;                      // 16-byte query chunks
     constexpr int QPT = (QCH + C::NTHR - 1) / C::NTHR;
-    // Value-scale bound for this CTA's keys of the unit: tau (per group) is
-    // fixed so that P * s_v * 2^tau < 2^15 for every key (P <= 1), i.e.
-    // tau = 29 - the largest exponent field of the group's value scales.  The
-    // scales are loaded here, with the query, before the stages' copies
-    // (which then find them in L2).
-    __shared__ int s_vexp[kDecWarpsMax * 8];
-    int vexp[NG];
-    {
-#pragma unroll
-      for (int gg = 0; gg < NG; ++gg) vexp[gg] = 0;
-      const int64_t klo = (int64_t)s0 * TK;
-      const int64_t khi = (int64_t)s1 * TK < L ? (int64_t)s1 * TK : L;
-      const uint16_t* vsg = p.vs + (row0 + klo) * NG;
-      const int nh = (int)((khi - klo) * NG);      // halves; whole 16-byte units stay in the slab
-      constexpr int VB = 4;                        // 16-byte loads in flight per thread
-      for (int c0 = tid * 8; c0 < nh; c0 += VB * C::NTHR * 8) {
-        uint4 w4[VB];
-#pragma unroll
-        for (int k = 0; k < VB; ++k) {
-          const int c = c0 + k * C::NTHR * 8;
-          w4[k] = c < nh ? __ldg(reinterpret_cast<const uint4*>(vsg + c)) : make_uint4(0u, 0u, 0u, 0u);
-        }
-#pragma unroll
-        for (int k = 0; k < VB; ++k) {
-          const int c = c0 + k * C::NTHR * 8;
-          const uint32_t w[4] = {w4[k].x, w4[k].y, w4[k].z, w4[k].w};
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int e = (int)((w[j >> 1] >> (16 * (j & 1) + 10)) & 31);
-            if (c + j < nh) vexp[j % NG] = max(vexp[j % NG], e);
-          }
-        }
-      }
-#pragma unroll
-      for (int gg = 0; gg < NG; ++gg) {
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) vexp[gg] = max(vexp[gg], __shfl_xor_sync(~0u, vexp[gg], off));
-        if (lane == 0) s_vexp[warp * 8 + gg] = vexp[gg];
-      }
-    }
+    // Everything above touched only parameters and shared memory; inputs are
+    // read, and the workspace written, only once the previous kernel of the
+    // stream has completed (this launch may start early, overlapping its
+    // set-up with that kernel's tail).
+    grid_dep_wait();
     uint4 qraw[QPT];
     {
-      const int64_t qbase = (((int64_t)b * p.Hkv + hkv) * p.G + hbase) * D;
+      const int64_t qbase = (uh * p.G + hbase) * D;
       const int nrows = min(HPC, p.G - hbase);
 #pragma unroll
       for (int k = 0; k < QPT; ++k) {
@@ -482,38 +489,29 @@ qsdpa_decode_kernel(const DecodeParams p) {
     }
 #pragma unroll
     for (int i = 0; i < NSTAGE - 1; ++i) {
-      if (i < nst) issue_stage(s0 + i, i);
+      const int blk = team + NTEAM * i;
+      if (blk < nblk) issue_block(blk, i);
       cp_async_commit();
     }
 #pragma unroll
     for (int k = 0; k < QPT; ++k) {
       const int i = tid + k * C::NTHR;
       if (QCH % C::NTHR == 0 || i < QCH) {
-        const uint32_t w[4] = {qraw[k].x, qraw[k].y, qraw[k].z, qraw[k].w};
-        float v[8];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          if (p.q_dtype == QKV_F16) {
-            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[j]));
-            v[2 * j] = f.x; v[2 * j + 1] = f.y;
-          } else {
-            v[2 * j] = __uint_as_float(w[j] << 16);
-            v[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
-          }
-        }
-        float4* dst = reinterpret_cast<float4*>(qst + i * 8);
-        dst[0] = make_float4(v[0], v[1], v[2], v[3]);
-        dst[1] = make_float4(v[4], v[5], v[6], v[7]);
+        const int hl = i / (D / 8), c = i - hl * (D / 8);
+        uint32_t* dst = reinterpret_cast<uint32_t*>(qst + hl * C::QROW + c * 16);
+        dst[0] = qraw[k].x; dst[1] = qraw[k].y; dst[2] = qraw[k].z; dst[3] = qraw[k].w;
       }
     }
     __syncthreads();
+    if (ttid == 0) s_grab[team][0] = atomicAdd(&s_next, 1);
 
     // ---------------- query fragments (B operand of the score MMA) ----------
     uint32_t bq[C::KSTEPS][2];
     float qsc[NG][2];
     float scaleK;
     {
-      const float* qr = qst + (chunk * 8 + g) * D;
+      const uint16_t* qr = reinterpret_cast<const uint16_t*>(qst + (chunk * 8 + g) * C::QROW);
+      const bool qf16 = p.q_dtype == QKV_F16;
       float qs[NG];
 #pragma unroll
       for (int gg = 0; gg < NG; ++gg) qs[gg] = 0.f;
@@ -533,7 +531,8 @@ qsdpa_decode_kernel(const DecodeParams p) {
         }
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          qv[s][i] = qr[e[i]];
+          const uint16_t h = qr[e[i]];
+          qv[s][i] = qf16 ? __half2float(__ushort_as_half(h)) : __uint_as_float((uint32_t)h << 16);
           qs[G] += qv[s][i];
           qmax = fmaxf(qmax, fabsf(qv[s][i]));
         }
@@ -566,39 +565,47 @@ qsdpa_decode_kernel(const DecodeParams p) {
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
     float beta[2][NG];
     float O[MT][4];
-    int tau[NG];          // per group: the value operand carries 2^tau
+    // Per group, the value operand carries 2^tau, with tau = 29 - the largest
+    // exponent field of the group's value scales seen so far, so that
+    // P * s_v * 2^tau < 2^15 for every key (P <= 1).  vbound holds those
+    // largest scales (magnitudes, as fp16 bits, two groups per word); tau
+    // only decreases, and O is rescaled by the exact power of two when it does.
+    int tau[NG];
+    uint32_t vbound[MW];
 #pragma unroll
-    for (int gg = 0; gg < NG; ++gg) {
-      beta[0][gg] = 0.f; beta[1][gg] = 0.f;
-      int e = 0;
+    for (int gg = 0; gg < NG; ++gg) { beta[0][gg] = 0.f; beta[1][gg] = 0.f; tau[gg] = 29; }
 #pragma unroll
-      for (int w = 0; w < C::NWARP; ++w) e = max(e, s_vexp[w * 8 + gg]);
-      tau[gg] = 29 - e;
-    }
+    for (int w = 0; w < MW; ++w) vbound[w] = 0u;
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) { O[mt][0] = O[mt][1] = O[mt][2] = O[mt][3] = 0.f; }
 
-    for (int it = 0; it < nst; ++it) {
+
+    // ---------------- main loop: the team's blocks ---------------------------
+    // pend[] holds the blocks in flight, oldest first; blocks are handed out in
+    // increasing order, so once a team sees a block past the segment it has
+    // nothing left.
+    int pend[NSTAGE - 1];
+#pragma unroll
+    for (int i = 0; i < NSTAGE - 1; ++i) pend[i] = team + NTEAM * i;
+    int slot = 0;
+    for (int it = 0; pend[0] < nblk; ++it) {
       cp_async_wait<NSTAGE - 2>();
-      __syncthreads();
+      team_sync();
+      const int cur = pend[0];
+      uint8_t* sb = ring + slot * C::STAGE;
       {
-        const int nx = it + NSTAGE - 1;
-        if (nx < nst) issue_stage(s0 + nx, nx % NSTAGE);
+        // the slot read in the previous iteration takes the next block
+        const int nb = s_grab[team][it & 1];
+        if (ttid == 0) s_grab[team][(it + 1) & 1] = atomicAdd(&s_next, 1);
+        if (nb < nblk) issue_block(nb, slot == 0 ? NSTAGE - 1 : slot - 1);
         cp_async_commit();
+#pragma unroll
+        for (int i = 0; i < NSTAGE - 2; ++i) pend[i] = pend[i + 1];
+        pend[NSTAGE - 2] = nb;
+        slot = slot + 1 == NSTAGE ? 0 : slot + 1;
       }
-      uint8_t* sb = smem + (it % NSTAGE) * C::STAGE;
-      const int64_t key0 = (int64_t)(s0 + it) * TK;
-      const int kvalid = (int)(L - key0 < (int64_t)TK ? L - key0 : (int64_t)TK);   // valid keys of this stage
-      if (kvalid < TK) {
-        // keys past L: clear their (possibly stale) scales and biases
-        uint16_t* meta = reinterpret_cast<uint16_t*>(sb + 2 * C::CODES);
-        for (int i = tid; i < C::NMETA * TK * NG; i += C::NTHR) {
-          const int arr = i / (TK * NG), r = i - arr * TK * NG;
-          if (r / NG >= kvalid) meta[arr * (C::META / 2) + r] = 0;
-        }
-        __syncthreads();
-      }
-      if (k0 >= kvalid) continue;                  // warp-uniform: whole block past L
+      const int64_t key0 = (int64_t)(s0 + cur) * BK;
+      const int kvalid = (int)(L - key0 < (int64_t)BK ? L - key0 : (int64_t)BK);   // valid keys of this block
       const uint8_t* sK = sb;
       const uint8_t* sV = sb + C::CODES;
       const uint8_t* sMeta = sb + 2 * C::CODES;
@@ -607,7 +614,7 @@ qsdpa_decode_kernel(const DecodeParams p) {
       float Sv[C::SUB][4];
 #pragma unroll
       for (int st = 0; st < C::SUB; ++st) {
-        const int r0 = k0 + 16 * st + g, r1 = r0 + 8;
+        const int r0 = 16 * st + g, r1 = r0 + 8;
         float* Sx = Sv[st];
         Sx[0] = Sx[1] = Sx[2] = Sx[3] = 0.f;
         uint32_t ks0[MW], ks1[MW], kb0[MW], kb1[MW];
@@ -658,8 +665,8 @@ qsdpa_decode_kernel(const DecodeParams p) {
           Sx[2] = fmaf(c1, acc[2], fmaf(bb1, qsc[G][0], Sx[2]));
           Sx[3] = fmaf(c1, acc[3], fmaf(bb1, qsc[G][1], Sx[3]));
         }
-        const int kr0 = 16 * st + k0 + g;                 // key index within the stage
-        if (kvalid < TK) {                                // only a stage that reaches L
+        const int kr0 = 16 * st + g;                      // key index within the block
+        if (kvalid < BK) {                                // only a block that reaches L
           if (kr0 >= kvalid) { Sx[0] = -INFINITY; Sx[1] = -INFINITY; }
           if (kr0 + 8 >= kvalid) { Sx[2] = -INFINITY; Sx[3] = -INFINITY; }
         }
@@ -726,12 +733,58 @@ qsdpa_decode_kernel(const DecodeParams p) {
       uint32_t vsw[C::SUB][2][MW], vbw[C::SUB][2][MW];
 #pragma unroll
       for (int st = 0; st < C::SUB; ++st) {
-        const int r0 = k0 + 16 * st + g;
+        const int r0 = 16 * st + g;
         meta_row<NG>(sMeta + (Q8 ? 1 : 2) * C::META, r0, vsw[st][0]);
         meta_row<NG>(sMeta + (Q8 ? 1 : 2) * C::META, r0 + 8, vsw[st][1]);
         if constexpr (!Q8) {
           meta_row<NG>(sMeta + 3 * C::META, r0, vbw[st][0]);
           meta_row<NG>(sMeta + 3 * C::META, r0 + 8, vbw[st][1]);
+        }
+        if (kvalid < BK) {
+          // keys past L: a metadata unit that starts below L is copied whole
+#pragma unroll
+          for (int w = 0; w < MW; ++w) {
+            if (r0 >= kvalid) { vsw[st][0][w] = 0u; vbw[st][0][w] = 0u; }
+            if (r0 + 8 >= kvalid) { vsw[st][1][w] = 0u; vbw[st][1][w] = 0u; }
+          }
+        }
+      }
+      {
+        // largest value scale of the block per group (fp16 bits of non-negative
+        // magnitudes order like the values); a rare warp-wide step when it
+        // exceeds the bound
+        uint32_t vm[MW];
+        bool grow = false;
+#pragma unroll
+        for (int w = 0; w < MW; ++w) {
+          vm[w] = __vmaxu2(vsw[0][0][w] & 0x7fff7fffu, vsw[0][1][w] & 0x7fff7fffu);
+#pragma unroll
+          for (int st = 1; st < C::SUB; ++st)
+            vm[w] = __vmaxu2(vm[w], __vmaxu2(vsw[st][0][w] & 0x7fff7fffu, vsw[st][1][w] & 0x7fff7fffu));
+          grow |= __vmaxu2(vm[w], vbound[w]) != vbound[w];
+        }
+        if (__any_sync(~0u, grow)) {
+#pragma unroll
+          for (int w = 0; w < MW; ++w) {
+            vm[w] = __vmaxu2(vm[w], vbound[w]);
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) vm[w] = __vmaxu2(vm[w], __shfl_xor_sync(~0u, vm[w], off));
+            vbound[w] = vm[w];
+          }
+#pragma unroll
+          for (int G = 0; G < NG; ++G) {
+            const int e = (int)((vbound[G >> 1] >> (16 * (G & 1) + 10)) & 31);
+            const int nt = 29 - e;
+            if (nt < tau[G]) {
+              const float f = exp2i(nt - tau[G]);
+#pragma unroll
+              for (int i = 0; i < KPG; ++i) {
+                O[G * KPG + i][0] *= f; O[G * KPG + i][1] *= f;
+                O[G * KPG + i][2] *= f; O[G * KPG + i][3] *= f;
+              }
+              tau[G] = nt;
+            }
+          }
         }
       }
 #pragma unroll
@@ -812,8 +865,9 @@ qsdpa_decode_kernel(const DecodeParams p) {
         }
       }
     }
-    cp_async_wait<0>();
-    __syncthreads();
+    cp_async_wait<0>();          // only empty groups can still be pending
+    __syncthreads();             // every team is done with its ring
+    grid_dep_launch();           // the next kernel may start its set-up
 
     // ---------------- epilogue: combine the warps of each head chunk ----------
 #pragma unroll
@@ -826,29 +880,19 @@ qsdpa_decode_kernel(const DecodeParams p) {
         beta[1][G] += __shfl_xor_sync(~0u, beta[1][G], off);
       }
     }
-    float* ws = reinterpret_cast<float*>(smem) + warp * (8 * D + 16);
+    // Per warp, its accumulators in fragment order (one float4 per m-tile and
+    // lane, stores free of bank conflicts), then (m, l) of its 8 rows.
+    float* ws = reinterpret_cast<float*>(smem) + warp * C::WSW;
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) {
       const int G = mt / KPG, i = mt % KPG;
-      // rows g / g+8 of value m-tile i of group G (the ldmatrix unit layout):
-      //  4-bit, groups >= 64: unit pair i/4, nibble c = i%4 -> dims 64(i/4)+4g+c, +32
-      //  4-bit, groups of 32: nibble c = i -> dims 4g+c and 4g+c+2
-      //  8-bit: unit pair i/2, byte c = i%2 -> dims 32(i/2)+2g+c, +16
-      int dlo, dhi;
-      bool x16 = false;                          // odd nibbles carry code * 2^-20
-      if constexpr (BITS == 4 && GS == 32) {
-        dlo = G * GS + 4 * g + i; dhi = dlo + 2; x16 = (i & 1) != 0;
-      } else if constexpr (BITS == 4) {
-        dlo = G * GS + 64 * (i >> 2) + 4 * g + (i & 3); dhi = dlo + 32; x16 = (i & 1) != 0;
-      } else {
-        dlo = G * GS + 32 * (i >> 1) + 2 * g + (i & 1); dhi = dlo + 16;
-      }
-      // codes entered as code*2^-24 (Q8_0: exact codes); O of group G carries 2^tau
+      // codes entered as code*2^-24 (odd nibbles: code*2^-20; Q8_0: exact
+      // codes); O of group G carries 2^tau
+      const bool x16 = BITS == 4 && (i & 1) != 0;
       const float f = exp2i((Q8 ? 0 : (x16 ? 20 : 24)) - tau[G]);
-      ws[(2 * t) * D + dlo] = fmaf(O[mt][0], f, beta[0][G]);
-      ws[(2 * t + 1) * D + dlo] = fmaf(O[mt][1], f, beta[1][G]);
-      ws[(2 * t) * D + dhi] = fmaf(O[mt][2], f, beta[0][G]);
-      ws[(2 * t + 1) * D + dhi] = fmaf(O[mt][3], f, beta[1][G]);
+      reinterpret_cast<float4*>(ws)[mt * 32 + lane] =
+          make_float4(fmaf(O[mt][0], f, beta[0][G]), fmaf(O[mt][1], f, beta[1][G]),
+                      fmaf(O[mt][2], f, beta[0][G]), fmaf(O[mt][3], f, beta[1][G]));
     }
     if (g == 0) {
       ws[8 * D + 2 * t] = m0; ws[8 * D + 2 * t + 1] = m1;
@@ -857,105 +901,137 @@ qsdpa_decode_kernel(const DecodeParams p) {
     __syncthreads();
 
     const bool complete = (s0 == 0) && (s1 == (int)S);
-    const int64_t slot = 2 * (int64_t)blockIdx.x + (u == first_unit ? 0 : 1);
     const float* wsf = reinterpret_cast<const float*>(smem);
+    constexpr int WST = NTEAM + 1;                               // padded weight row
+    float* wgt = reinterpret_cast<float*>(smem + C::EPI_W);     // [HPC][WST] combine weights
+    float* rml = wgt + HPC * WST;                                // [HPC][2] (m, l) of the CTA
+    // weights: thread (row R, team k) of the first HPC * NTEAM threads; the
+    // NTEAM teams of a row are adjacent lanes
+    if (tid < HPC * NTEAM) {
+      const int R = tid / NTEAM, k = tid - R * NTEAM;
+      const int c = R >> 3, hh = R & 7;
+      const float* wp = wsf + (k * NC + c) * C::WSW;
+      const float mw = wp[8 * D + hh], lw = wp[8 * D + 8 + hh];
+      float M = mw;
+#pragma unroll
+      for (int off = 1; off < NTEAM; off <<= 1) M = fmaxf(M, __shfl_xor_sync(~0u, M, off));
+      const float w = mw == -INFINITY ? 0.f : ex2(mw - M);
+      float Ls = w * lw;
+#pragma unroll
+      for (int off = 1; off < NTEAM; off <<= 1) Ls += __shfl_xor_sync(~0u, Ls, off);
+      wgt[R * WST + k] = complete ? (Ls > 0.f ? w / Ls : 0.f) : w;
+      if (k == 0) { rml[2 * R] = M; rml[2 * R + 1] = Ls; }
+    }
+    __syncthreads();
+    const int64_t pslot = 2 * (int64_t)blockIdx.x + (u == first_unit ? 0 : 1);
+    // element (chunk c, m-tile mt, lane (gl, tl), j) of the fragment order is
+    // row c*8 + 2*tl + (j & 1) and the dim of m-tile mt's row gl (j < 2) or
+    // gl + 8 (j >= 2):
+    //  4-bit, groups >= 64: unit pair i/4, nibble i%4 -> dims 64(i/4)+4g+i%4, +32
+    //  4-bit, groups of 32: nibble i -> dims 4g+i and 4g+i+2
+    //  8-bit: unit pair i/2, byte i%2 -> dims 32(i/2)+2g+i%2, +16
     for (int idx = tid; idx < HPC * D; idx += C::NTHR) {
-      const int hl = idx / D, e = idx - hl * D;       // hl: head within the chunk-group
-      const int c = hl >> 3, hh = hl & 7;
-      const int head = hbase + hl;
+      const int c = idx / (8 * D), r = idx - c * 8 * D;
+      const int mt = r >> 7, lj = r & 127, gl = lj >> 4, tl = (lj >> 2) & 3, j = lj & 3;
+      const int R = c * 8 + 2 * tl + (j & 1);
+      const int head = hbase + R;
       if (head >= p.G) continue;
-      float M = -INFINITY;
+      const int G = mt / KPG, i = mt % KPG;
+      int dim;
+      if constexpr (BITS == 4 && GS == 32) dim = G * GS + 4 * gl + i + (j >= 2 ? 2 : 0);
+      else if constexpr (BITS == 4) dim = G * GS + 64 * (i >> 2) + 4 * gl + (i & 3) + (j >= 2 ? 32 : 0);
+      else dim = G * GS + 32 * (i >> 1) + 2 * gl + (i & 1) + (j >= 2 ? 16 : 0);
+      float o = 0.f;
 #pragma unroll
-      for (int w = 0; w < C::WPC; ++w) M = fmaxf(M, wsf[(c * C::WPC + w) * (8 * D + 16) + 8 * D + hh]);
-      float o = 0.f, l = 0.f;
-      if (M != -INFINITY) {
-#pragma unroll
-        for (int w = 0; w < C::WPC; ++w) {
-          const float* wp = wsf + (c * C::WPC + w) * (8 * D + 16);
-          const float mw = wp[8 * D + hh];
-          if (mw == -INFINITY) continue;
-          const float sc = ex2(mw - M);
-          o = fmaf(sc, wp[hh * D + e], o);
-          l = fmaf(sc, wp[8 * D + 8 + hh], l);
-        }
-      }
+      for (int k = 0; k < NTEAM; ++k) o = fmaf(wgt[R * WST + k], wsf[(k * NC + c) * C::WSW + r], o);
       if (complete) {
-        const int64_t oi = (((int64_t)b * p.Hkv + hkv) * p.G + head) * D + e;
-        store_from_float(p.out, p.out_dtype, oi, l > 0.f ? o / l : 0.f);
+        const int64_t oi = (uh * p.G + head) * D + dim;
+        store_from_float(p.out, p.out_dtype, oi, o);
       } else {
-        p.part_o[(slot * HPC + hl) * D + e] = o;
-        if (e == 0) {
-          p.part_ml[(slot * HPC + hl) * 2 + 0] = M;
-          p.part_ml[(slot * HPC + hl) * 2 + 1] = l;
+        p.part_o[(pslot * HPC + R) * D + dim] = o;
+        if (dim == 0) {
+          p.part_ml[(pslot * HPC + R) * 2 + 0] = rml[2 * R];
+          p.part_ml[(pslot * HPC + R) * 2 + 1] = rml[2 * R + 1];
         }
       }
     }
+    if (tid == 0) s_next = NTEAM * (NSTAGE - 1);                 // for the next segment
+    __syncthreads();             // the next segment reuses the shared memory
+  }
 
-    if (!complete) {
-      // The unit's partials are merged by the last of its CTAs to finish
-      // (atomic ticket), in one level when their volume is small, else in two:
-      // the last CTA of each group of kMergeGroup consecutive CTAs merges the
-      // group into a second-level partial and the last group merger merges
-      // those.  Nobody waits on anybody.
-      __threadfence();
+  // ---------------- merge of the units this CTA covered partially ------------
+  // Only the first and the last unit of the range can be partial.  A unit's
+  // partials are merged by the last of its CTAs to arrive (atomic ticket), in
+  // one level when their volume is small, else in two: the last CTA of each
+  // group of kMergeGroup consecutive CTAs merges the group into a second-level
+  // partial and the last group merger merges those.  Nobody waits on anybody.
+  // Every thread's partial stores, then the barrier, then one thread's ticket
+  // with acquire-release semantics at GPU scope: the barrier orders the other
+  // threads' stores before that release, and in the CTA that draws the last
+  // ticket the barrier after it orders the acquire before every thread's
+  // reads of the partials.
+  __syncthreads();
+  for (int which = 0; which < 2; ++which) {
+    const int64_t u = which == 0 ? first_unit : udiv64(hi - 1, S);
+    if (which == 1 && u == first_unit) break;
+    const int64_t seg_lo = lo > u * S ? lo : u * S;
+    const int64_t seg_hi = hi < (u + 1) * S ? hi : (u + 1) * S;
+    if (seg_lo == u * S && seg_hi == (u + 1) * S) continue;     // complete: already written
+    const int64_t uh = udiv64(u, p.ncg);
+    const int cg = (int)(u - uh * p.ncg);
+    const int hbase = cg * HPC;
+    const int64_t cfirst = udiv64((u * S + 1) * nC - 1, T);
+    const int64_t clast = udiv64(((u + 1) * S) * nC - 1, T);
+    const int nparts = (int)(clast - cfirst + 1);
+    const int nrows = min(HPC, p.G - hbase);
+    // slot of the unit's first CTA: its second slot if it began in an
+    // earlier unit; every later CTA of the unit began in this one
+    const int64_t slot0 = 2 * cfirst + (udiv64(udiv64(cfirst * T, nC), S) == u ? 0 : 1);
+    auto slot_of = [&](int64_t c) -> int64_t { return c == cfirst ? slot0 : 2 * c; };
+    const int64_t out_base = (uh * p.G + hbase) * D;
+    if ((int64_t)nparts * nrows * D <= kMergeFlat) {
+      if (tid == 0) {
+        const unsigned prev = atom_add_acq_rel_gpu(&p.tickets[u], 1u);
+        const int last = prev == (unsigned)nparts - 1;
+        if (last) p.tickets[u] = 0u;
+        s_flag = last;
+      }
       __syncthreads();
-      const int64_t cfirst = udiv64((u * S + 1) * nC - 1, T);
-      const int64_t clast = udiv64(((u + 1) * S) * nC - 1, T);
-      const int nparts = (int)(clast - cfirst + 1);
-      const int nrows = min(HPC, p.G - hbase);
-      // slot of the unit's first CTA: its second slot if it began in an
-      // earlier unit; every later CTA of the unit began in this one
-      const int64_t slot0 = 2 * cfirst + (udiv64(udiv64(cfirst * T, nC), S) == u ? 0 : 1);
-      auto slot_of = [&](int64_t c) -> int64_t { return c == cfirst ? slot0 : 2 * c; };
-      const int64_t out_base = (((int64_t)b * p.Hkv + hkv) * p.G + hbase) * D;
-      if ((int64_t)nparts * nrows * D <= kMergeFlat) {
+      if (s_flag) {
+        merge_unit<D, HPC>(p.part_ml, p.part_o, nparts, slot0, cfirst, 1, tid, C::NTHR, nrows,
+                           p.out, p.out_dtype, out_base, nullptr, nullptr);
+      }
+    } else {
+      const int ngroups = (nparts + kMergeGroup - 1) / kMergeGroup;
+      const int gi = (int)((int64_t)blockIdx.x - cfirst) / kMergeGroup;
+      const int64_t c0 = cfirst + (int64_t)gi * kMergeGroup;
+      const int64_t lead = slot_of(c0);                       // the group's second-level slot
+      const int gsz = min(kMergeGroup, nparts - gi * kMergeGroup);
+      if (tid == 0) {
+        const unsigned prev = atom_add_acq_rel_gpu(&p.tickets1[lead], 1u);
+        const int last = prev == (unsigned)gsz - 1;
+        if (last) p.tickets1[lead] = 0u;
+        s_flag = last;
+      }
+      __syncthreads();
+      if (s_flag) {
+        merge_unit<D, HPC>(p.part_ml, p.part_o, gsz, lead, c0, 1, tid, C::NTHR, nrows,
+                           nullptr, 0, 0, p.part2_ml + lead * HPC * 2, p.part2_o + lead * HPC * D);
+        __syncthreads();
         if (tid == 0) {
-          const unsigned prev = atomicAdd(&p.tickets[u], 1u);
-          const int last = prev == (unsigned)nparts - 1;
+          const unsigned prev = atom_add_acq_rel_gpu(&p.tickets[u], 1u);
+          const int last = prev == (unsigned)ngroups - 1;
           if (last) p.tickets[u] = 0u;
           s_flag = last;
         }
         __syncthreads();
         if (s_flag) {
-          __threadfence();
-          merge_unit<D, HPC>(p.part_ml, p.part_o, nparts, slot0, cfirst, 1, tid, C::NTHR, nrows,
-                             p.out, p.out_dtype, out_base, nullptr, nullptr);
-        }
-      } else {
-        const int ngroups = (nparts + kMergeGroup - 1) / kMergeGroup;
-        const int gi = (int)((int64_t)blockIdx.x - cfirst) / kMergeGroup;
-        const int64_t c0 = cfirst + (int64_t)gi * kMergeGroup;
-        const int64_t lead = slot_of(c0);                       // the group's second-level slot
-        const int gsz = min(kMergeGroup, nparts - gi * kMergeGroup);
-        if (tid == 0) {
-          const unsigned prev = atomicAdd(&p.tickets1[lead], 1u);
-          const int last = prev == (unsigned)gsz - 1;
-          if (last) p.tickets1[lead] = 0u;
-          s_flag = last;
-        }
-        __syncthreads();
-        if (s_flag) {
-          __threadfence();
-          merge_unit<D, HPC>(p.part_ml, p.part_o, gsz, lead, c0, 1, tid, C::NTHR, nrows,
-                             nullptr, 0, 0, p.part2_ml + lead * HPC * 2, p.part2_o + lead * HPC * D);
-          __threadfence();
-          __syncthreads();
-          if (tid == 0) {
-            const unsigned prev = atomicAdd(&p.tickets[u], 1u);
-            const int last = prev == (unsigned)ngroups - 1;
-            if (last) p.tickets[u] = 0u;
-            s_flag = last;
-          }
-          __syncthreads();
-          if (s_flag) {
-            __threadfence();
-            merge_unit<D, HPC>(p.part2_ml, p.part2_o, ngroups, slot0, cfirst, kMergeGroup, tid,
-                               C::NTHR, nrows, p.out, p.out_dtype, out_base, nullptr, nullptr);
-          }
+          merge_unit<D, HPC>(p.part2_ml, p.part2_o, ngroups, slot0, cfirst, kMergeGroup, tid,
+                             C::NTHR, nrows, p.out, p.out_dtype, out_base, nullptr, nullptr);
         }
       }
     }
-    __syncthreads();
+    __syncthreads();             // s_flag is reused
   }
 }
 
@@ -976,10 +1052,21 @@ struct DecodeInstance {
     }
     return cached;
   }
+  // Launched with programmatic stream serialization: the set-up before the
+  // kernel's grid_dep_wait() overlaps the tail of the previous kernel.
   static cudaError_t launch(const DecodePlan& plan, const DecodeParams& p, cudaStream_t s) {
     auto k = qsdpa_decode_kernel<D, BITS, GS, Q8, NC, F32OUT>;
-    k<<<plan.grid, C::NTHR, C::SMEM, s>>>(p);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)plan.grid);
+    cfg.blockDim = dim3(C::NTHR);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k, p);
   }
 };
 

@@ -14,7 +14,7 @@ int max_ctas_per_sm(int D) { return dec_ctas_per_sm(D); }
 constexpr int64_t kMaxGrid = 8 * 48;
 // Partials of at least this many floats count as large (16 rows x D = 256 do).
 constexpr int64_t kBigPartial = 2048;
-constexpr int64_t kBigPartMinStages = 2;
+constexpr int64_t kBigPartMinStages = 2;   // blocks per team
 
 int sm_count() {
   int dev = 0, n = 0;
@@ -88,16 +88,28 @@ bool plan_decode(int D, int bits, int gs, int fmt, int out_f32, int B, int Hq, i
   plan->units = (int64_t)B * Hkv * ncg;
   plan->stages_per_unit = (L + ops.tk - 1) / ops.tk;
   plan->total_stages = plan->units * plan->stages_per_unit;
-  // one CTA per (SM x resident slot), each a contiguous equal share of stages
-  int64_t grid = (int64_t)sms * occ;
-  grid = std::min<int64_t>(grid, plan->total_stages);
-  grid = std::min<int64_t>(grid, kMaxGrid);            // merge scratch holds <= 48 groups
+  // One CTA per SM, each a contiguous equal share of the (unit, block) range.
+  int64_t cap = (int64_t)sms * occ;
+  cap = std::min<int64_t>(cap, plan->total_stages);
+  cap = std::min<int64_t>(cap, kMaxGrid);              // merge scratch holds <= 48 groups
   // A CTA's partial (rows x D fp32) is written, read back and merged; when it
-  // is large (many query rows per KV head, wide heads) give every CTA several
-  // stages, so that partials stay a small fraction of the bytes streamed.
+  // is large (many query rows per KV head, wide heads) give every team of
+  // every CTA several blocks, so that partials stay a small fraction of the
+  // bytes streamed.
   if ((int64_t)plan->hpc * D >= kBigPartial) {
-    const int64_t cap = (plan->total_stages + kBigPartMinStages - 1) / kBigPartMinStages;
-    grid = std::min<int64_t>(grid, std::max<int64_t>(1, cap));
+    const int64_t per = (int64_t)ops.teams * kBigPartMinStages;
+    cap = std::min<int64_t>(cap, std::max<int64_t>(1, plan->total_stages / per));
+  }
+  int64_t grid = std::max<int64_t>(1, cap);
+  // When the units are few, cut every unit into the same number of pieces (no
+  // CTA then covers parts of two units, which would cost it a second prologue
+  // and epilogue), as long as that leaves at most 15% of the grid idle; no
+  // more pieces than give every team a block (short caches: fewer partials).
+  if (plan->units <= grid) {
+    const int64_t per_unit = std::min<int64_t>(grid / plan->units,
+                                               (plan->stages_per_unit + ops.teams - 1) / ops.teams);
+    if (per_unit * plan->units * 100 >= grid * 85 || per_unit * ops.teams >= plan->stages_per_unit)
+      grid = std::max<int64_t>(1, per_unit) * plan->units;
   }
   plan->grid = (int)std::max<int64_t>(1, grid);
   plan->smem = ops.smem;

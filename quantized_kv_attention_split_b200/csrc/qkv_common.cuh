@@ -83,6 +83,15 @@ __device__ __forceinline__ void store_from_float(void* p, int dtype, int64_t i, 
   else reinterpret_cast<float*>(p)[i] = v;
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start while the previous kernel of the stream is still
+// running; grid_dep_wait() returns once that kernel has completed and its
+// memory operations are visible, and grid_dep_launch() lets the next kernel
+// of the stream start early (it still waits in its own grid_dep_wait()).
+// Both are no-ops for a normal launch.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
 // 2^k as float for integer k in [-126, 127].
 __device__ __forceinline__ float exp2i(int k) {
   return __uint_as_float(static_cast<uint32_t>(k + 127) << 23);
