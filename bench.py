@@ -139,9 +139,45 @@ def build_caches(w, inp, ncopies, device):
     return caches
 
 
-def graph_time(step, K, W, sampler=None, min_window_s=0.3):
+def graph_kernel_nodes(g):
+    """Kernel nodes of a captured CUDA graph (None if it cannot be read)."""
+    try:
+        from cuda.bindings import runtime as rt
+        h = g.raw_cuda_graph()
+        graph = h if isinstance(h, rt.cudaGraph_t) else rt.cudaGraph_t(init_value=int(h))
+        err, _, n = rt.cudaGraphGetNodes(graph, 0)
+        if err != rt.cudaError_t.cudaSuccess:
+            return None
+        err, nodes, n = rt.cudaGraphGetNodes(graph, n)
+        if err != rt.cudaError_t.cudaSuccess:
+            return None
+        kern = 0
+        for nd in nodes[:n]:
+            err, t = rt.cudaGraphNodeGetType(nd)
+            if err == rt.cudaError_t.cudaSuccess and t == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel:
+                kern += 1
+        return kern
+    except Exception:
+        return None
+
+
+LAUNCHES = {}
+
+
+def new_graph():
+    """A CUDA graph whose captured graph stays readable (for counting launches)."""
+    import torch
+    try:
+        return torch.cuda.CUDAGraph(keep_graph=True)
+    except TypeError:
+        return torch.cuda.CUDAGraph()
+
+
+def graph_time(step, K, W, sampler=None, min_window_s=0.3, tag=None):
     """Device time of exactly K calls of step(i): W eager warm-up calls, then
-    K calls captured in CUDA graphs and replayed between events."""
+    K calls captured in CUDA graphs and replayed between events.  With a tag,
+    the kernel launches of the K calls (counted from the captured graphs) are
+    recorded in LAUNCHES[tag]."""
     import torch
     for i in range(W):
         step(i)
@@ -151,7 +187,7 @@ def graph_time(step, K, W, sampler=None, min_window_s=0.3):
     s.wait_stream(torch.cuda.current_stream())
     graphs = []
     with torch.cuda.stream(s):
-        g1 = torch.cuda.CUDAGraph()
+        g1 = new_graph()
         with torch.cuda.graph(g1, stream=s):
             for i in range(chunk):
                 step(i)
@@ -159,12 +195,22 @@ def graph_time(step, K, W, sampler=None, min_window_s=0.3):
         rem = K % chunk
         g2 = None
         if rem:
-            g2 = torch.cuda.CUDAGraph()
+            g2 = new_graph()
             with torch.cuda.graph(g2, stream=s):
                 for i in range(rem):
                     step(i)
     torch.cuda.current_stream().wait_stream(s)
     torch.cuda.synchronize()
+    if tag is not None:
+        n1 = graph_kernel_nodes(g1)
+        n2 = graph_kernel_nodes(g2) if g2 is not None else 0
+        LAUNCHES[tag] = None if n1 is None or n2 is None else n1 * (K // chunk) + n2
+    for g in (g1, g2):
+        if g is not None and hasattr(g, "instantiate"):
+            try:
+                g.instantiate()
+            except RuntimeError:
+                pass                              # already instantiated
     g1.replay()                                   # one untimed replay
     torch.cuda.synchronize()
     reps = K // chunk
@@ -271,7 +317,7 @@ def run_ours(args, rank, world, device):
     if sampler:
         sampler.start()
         time.sleep(0.3)
-    sec, extra = graph_time(step, args.steps, args.warmup, sampler)
+    sec, extra = graph_time(step, args.steps, args.warmup, sampler, tag="main")
     sec /= 1e3
     if sampler:
         time.sleep(0.1)
@@ -353,7 +399,10 @@ def run_ours(args, rank, world, device):
                     "d2h_bytes_per_step": int(out.numel() * 2),
                     "note": "through the Python binding and C ABI, q copied from pinned host "
                             "memory and the output copied back every call"},
-            "gpu_launches": args.steps,
+            "gpu_launches": LAUNCHES.get("main") if LAUNCHES.get("main") is not None else args.steps,
+            "gpu_launches_source": ("kernel nodes of the captured CUDA graphs (decode kernel, plus "
+                                    "the merge kernel when a unit is split over CTAs)"
+                                    if LAUNCHES.get("main") is not None else "one per call (graph not readable)"),
             "clocks": {"sm_mhz": clocks.get("sm_mhz"), "sm_max_mhz": clocks.get("sm_max_mhz"),
                        "reasons": clocks.get("reasons", []), "samples": clocks.get("samples", 0),
                        "window": "timed region" + (" + untimed replay of the same graph"

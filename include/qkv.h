@@ -113,9 +113,12 @@ qkv_status qkv_quantize_update(const void* new_k, const void* new_v, int in_dtyp
  *  out: [B, Hq, 1, D] contiguous, out_dtype f16, bf16 or f32.
  *  Hq % Hkv == 0; query head h reads kv-head h / (Hq/Hkv).
  *  workspace: device scratch of at least qsdpa_workspace_size(...) bytes,
- *  16-byte aligned, whose first qsdpa_workspace_zero_bytes(...) bytes are
- *  zero before the first call (the kernel leaves them zero again after every
- *  call).  Calls that share a workspace must not overlap on the GPU.
+ *  16-byte aligned; decode keeps no state in it between calls.  Calls that
+ *  share a workspace must not overlap on the GPU.  One kernel launch, or two
+ *  when the keys of a (batch, kv-head) are split over several CTAs (the
+ *  second merges their partial results); both are programmatic dependent
+ *  launches, whose set-up may overlap the previous kernel of the stream (they
+ *  read no input and write nothing before that kernel has completed).
  *  L == 0 writes zeros.  Accuracy: max-abs error vs fp64 <= 2e-3 for f16/bf16
  *  out, <= 1e-4 for f32 out (values of order one). */
 qkv_status qsdpa_decode(const void* q, int q_dtype, int B, int Hq, int Hkv, int D,
@@ -126,7 +129,9 @@ qkv_status qsdpa_decode(const void* q, int q_dtype, int B, int Hq, int Hkv, int 
 /* Multi-query attention (any Lq >= 1) over keys [0, L) with an optional mask
  * (the pages' Lq > 1 fallback: quantized_matmul -> softmax -> quantized_matmul,
  * computed here in one fused pass).  q/out: [B, Hq, Lq, D] contiguous.
- * Same workspace rules as qsdpa_decode.  With at least 64 (head, query) rows
+ * Same workspace rules as qsdpa_decode, and the first
+ * qsdpa_workspace_zero_bytes(...) bytes must be zero before the first call
+ * (the kernels leave them zero).  With at least 64 (head, query) rows
  * per kv head and f16/bf16 output the call runs on the tcgen05 tensor-core
  * kernel (K and V tiles dequantized to fp16, fp32 accumulation in TMEM);
  * otherwise, and always for f32 output, on the split-K kernel.  The tcgen05
@@ -144,15 +149,14 @@ qkv_status qsdpa_prefill(const void* q, int q_dtype, int B, int Hq, int Hkv, int
  * that runs under an allocator which forbids cudaMalloc/cudaFree, services
  * that fix every buffer before they start, or plug-in interfaces that hand
  * over only inputs and outputs.  Same arguments and results as qsdpa_decode,
- * without the workspace: its scratch (tickets and partial results) lives in a
- * 16 MiB array built into this library, which every GPU that loads the
+ * without the workspace: its scratch (partial results) lives in a
+ * 8 MiB array built into this library, which every GPU that loads the
  * library keeps until the process exits.  Shapes whose workspace
- * (qsdpa_workspace_size) exceeds 16 MiB are rejected with QKV_ERR_WORKSPACE.
+ * (qsdpa_workspace_size) exceeds 8 MiB are rejected with QKV_ERR_WORKSPACE.
  * The first call on a device looks up that device's address of the array;
- * make that first call before any stream capture.  Every call clears the
- * tickets it needs and reuses the same array, so calls that may overlap on the
- * GPU (other streams, other host threads on the same device) race: order them
- * on one stream. */
+ * make that first call before any stream capture.  Every call reuses the same
+ * array, so calls that may overlap on the GPU (other streams, other host
+ * threads on the same device) race: order them on one stream. */
 qkv_status qsdpa_decode_noalloc(const void* q, int q_dtype, int B, int Hq, int Hkv, int D,
                                 const qkv_cache* k, const qkv_cache* v, int64_t L,
                                 float scale, const qkv_mask* mask, void* out, int out_dtype,
@@ -160,7 +164,7 @@ qkv_status qsdpa_decode_noalloc(const void* q, int q_dtype, int B, int Hq, int H
 
 /* Workspace bytes needed by qsdpa_decode (Lq = 1) or qsdpa_prefill for this
  * problem on the CURRENT device, and how many leading bytes must be zero
- * before the first call.  0 on invalid arguments. */
+ * before the first qsdpa_prefill call.  0 on invalid arguments. */
 size_t qsdpa_workspace_size(int B, int Hq, int Hkv, int Lq, int D, int64_t L);
 size_t qsdpa_workspace_zero_bytes(int B, int Hq, int Hkv, int Lq, int D, int64_t L);
 

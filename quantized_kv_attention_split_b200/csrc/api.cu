@@ -177,14 +177,9 @@ qkv_status attention(const void* q, int q_dtype, int B, int Hq, int Hkv, int Lq,
     p.msb = mask->stride_b; p.msh = mask->stride_h; p.msq = mask->stride_q;
   }
   if (mkind == QKV_MASK_CAUSAL && Lq == 1) p.mask_kind = QKV_MASK_NONE;  // all keys visible
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  p.tickets = reinterpret_cast<unsigned*>(ws);
-  p.tickets1 = reinterpret_cast<unsigned*>(ws + plan.ws_tickets2);
-  uint8_t* parts = ws + plan.ws_tickets;
+  uint8_t* parts = static_cast<uint8_t*>(workspace) + plan.ws_header;
   p.part_o = reinterpret_cast<float*>(parts);
   p.part_ml = reinterpret_cast<float*>(parts + plan.ws_part_o);
-  p.part2_o = reinterpret_cast<float*>(parts + plan.ws_part_o + plan.ws_part_ml);
-  p.part2_ml = reinterpret_cast<float*>(parts + 2 * plan.ws_part_o + plan.ws_part_ml);
   cudaError_t e = qkv::launch_decode(D, k->bits, k->group_size, k->fmt, out_dtype == QKV_F32,
                                      plan, p, s);
   if (e != cudaSuccess) return fail(QKV_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
@@ -271,7 +266,7 @@ qkv_status qsdpa_prefill(const void* q, int q_dtype, int B, int Hq, int Hkv, int
 // that pre-plan every buffer before serving starts, or plug-in interfaces that
 // only hand over input and output pointers.  For them, qsdpa_decode_noalloc
 // runs the same decode kernel as qsdpa_decode but keeps its scratch (the
-// per-unit tickets and the partial results of the split over L) in a
+// partial results of the split over L) in a
 // fixed-size array that lives in this library's device image.  Every GPU that
 // loads the library holds that array until the process exits.
 // ---------------------------------------------------------------------------
@@ -279,7 +274,7 @@ qkv_status qsdpa_prefill(const void* q, int q_dtype, int B, int Hq, int Hkv, int
 
 namespace {
 
-constexpr size_t kNoAllocScratchBytes = 16u << 20;   // 16 MiB per device
+constexpr size_t kNoAllocScratchBytes = 8u << 20;    // 8 MiB per device
 constexpr int kNoAllocMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
@@ -328,11 +323,8 @@ extern "C" qkv_status qsdpa_decode_noalloc(const void* q, int q_dtype, int B, in
   void* scratch = nullptr;
   qkv_status st = noalloc_scratch(&scratch);
   if (st != QKV_OK) return st;
-  // the tickets at the front must be zero; the previous call left them zero,
-  // but clear them anyway so an interrupted call cannot poison the next one
-  const size_t zero = qsdpa_workspace_zero_bytes(B, Hq, Hkv, 1, D, L);
-  cudaError_t e = cudaMemsetAsync(scratch, 0, zero, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return fail(QKV_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e));
+  // decode keeps no state in its scratch between calls (the header that
+  // qsdpa_workspace_zero_bytes covers is the prefill's), so nothing to clear
   return qsdpa_decode(q, q_dtype, B, Hq, Hkv, D, k, v, L, scale, mask, out, out_dtype, scratch,
                       kNoAllocScratchBytes, stream);
 }

@@ -189,102 +189,6 @@ __device__ __forceinline__ int64_t udiv64(int64_t a, int64_t b) {
   return a / b;
 }
 
-constexpr int kMergeBatch = 10;   // parts whose loads one merging thread has in flight
-constexpr int kMergeGroup = 8;    // parts per first-level merge when a unit merges in two levels
-constexpr int64_t kMergeFlat = 1 << 15;   // largest parts x rows x D merged by one CTA in one level
-
-// Combines n partial results (m, l, o) of one unit by log-sum-exp rescaling.
-// Part i lives in slot 2 * (c0 + i * step), except part 0, which is in slot0.
-// Writes either the nrows normalized rows starting at element out_base
-// (dst_o == nullptr) or one combined partial (dst_ml, dst_o).  A thread owns 4
-// consecutive outputs of one row and every tpi-th part; it loads (m, l) and o
-// of a batch of parts at once and folds them in online, then the tpi threads
-// of an output (adjacent lanes) combine with shuffles: one round trip per
-// batch and no barrier.
-template <int D, int HPC>
-__device__ __noinline__ void merge_unit(const float* ml, const float* po, int n, int64_t slot0,
-                                        int64_t c0, int step, int tid, int nthreads, int nrows,
-                                        void* out, int out_dtype, int64_t out_base, float* dst_ml,
-                                        float* dst_o) {
-  constexpr int V4 = D / 4;
-  const int items = nrows * V4;
-  int tpi = 1;
-  while (tpi < 32 && items * tpi * 2 <= nthreads) tpi *= 2;
-  const int ipp = nthreads / tpi;                                 // items per pass
-  const int sub = tid & (tpi - 1);
-  for (int i0 = 0; i0 < items; i0 += ipp) {
-    const int item = i0 + tid / tpi;
-    const bool active = item < items;
-    const int hl = active ? item / V4 : 0, e4 = active ? item - hl * V4 : 0;
-    float M = -INFINITY, Ls = 0.f;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int jb = 0; sub + tpi * jb < n; jb += kMergeBatch) {
-      float4 o[kMergeBatch];
-      float2 v[kMergeBatch];
-#pragma unroll
-      for (int k = 0; k < kMergeBatch; ++k) {
-        const int pp = sub + tpi * (jb + k);
-        if (active && pp < n) {
-          const int64_t sx = pp == 0 ? slot0 : 2 * (c0 + (int64_t)pp * step);
-          o[k] = __ldcg(reinterpret_cast<const float4*>(po + (sx * HPC + hl) * D) + e4);
-          v[k] = __ldcg(reinterpret_cast<const float2*>(ml + (sx * HPC + hl) * 2));
-        } else {
-          o[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-          v[k] = make_float2(-INFINITY, 0.f);
-        }
-      }
-      float Mb = M;
-#pragma unroll
-      for (int k = 0; k < kMergeBatch; ++k) Mb = fmaxf(Mb, v[k].x);
-      if (Mb != M) {
-        const float f = M == -INFINITY ? 0.f : ex2(M - Mb);
-        Ls *= f; acc.x *= f; acc.y *= f; acc.z *= f; acc.w *= f;
-        M = Mb;
-      }
-#pragma unroll
-      for (int k = 0; k < kMergeBatch; ++k) {
-        const float w = v[k].x == -INFINITY ? 0.f : ex2(v[k].x - M);
-        Ls = fmaf(w, v[k].y, Ls);
-        acc.x = fmaf(w, o[k].x, acc.x);
-        acc.y = fmaf(w, o[k].y, acc.y);
-        acc.z = fmaf(w, o[k].z, acc.z);
-        acc.w = fmaf(w, o[k].w, acc.w);
-      }
-    }
-    for (int off = 1; off < tpi; off <<= 1) {
-      const float M2 = __shfl_xor_sync(~0u, M, off), L2 = __shfl_xor_sync(~0u, Ls, off);
-      const float x2 = __shfl_xor_sync(~0u, acc.x, off), y2 = __shfl_xor_sync(~0u, acc.y, off);
-      const float z2 = __shfl_xor_sync(~0u, acc.z, off), w2 = __shfl_xor_sync(~0u, acc.w, off);
-      const float Mn = fmaxf(M, M2);
-      const float f1 = M == -INFINITY ? 0.f : ex2(M - Mn), f2 = M2 == -INFINITY ? 0.f : ex2(M2 - Mn);
-      Ls = Ls * f1 + L2 * f2;
-      acc.x = acc.x * f1 + x2 * f2; acc.y = acc.y * f1 + y2 * f2;
-      acc.z = acc.z * f1 + z2 * f2; acc.w = acc.w * f1 + w2 * f2;
-      M = Mn;
-    }
-    if (active && sub == 0) {
-      if (dst_o != nullptr) {
-        *reinterpret_cast<float4*>(dst_o + hl * D + e4 * 4) = acc;
-        if (e4 == 0) { dst_ml[hl * 2] = M; dst_ml[hl * 2 + 1] = Ls; }
-      } else {
-        const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
-        const int64_t oi = out_base + (int64_t)hl * D + e4 * 4;
-        store_from_float(out, out_dtype, oi, acc.x * inv);
-        store_from_float(out, out_dtype, oi + 1, acc.y * inv);
-        store_from_float(out, out_dtype, oi + 2, acc.z * inv);
-        store_from_float(out, out_dtype, oi + 3, acc.w * inv);
-      }
-    }
-  }
-}
-
-// Atomic add with acquire-release semantics at GPU scope.
-__device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned* p, unsigned v) {
-  unsigned old;
-  asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], %2;\n" : "=r"(old) : "l"(p), "r"(v) : "memory");
-  return old;
-}
-
 // Transposing shared-memory matrix loads (8x8 of 16-bit elements per matrix).
 __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1,
                                               uint32_t& r2, uint32_t& r3) {
@@ -348,7 +252,6 @@ qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
   const int64_t nC = gridDim.x;
   const int64_t lo = udiv64((int64_t)blockIdx.x * T, nC), hi = udiv64(((int64_t)blockIdx.x + 1) * T, nC);
   const int64_t first_unit = udiv64(lo, S);
-  __shared__ int s_flag;
   __shared__ int s_next;                 // next block of the segment to hand out
   __shared__ int s_grab[NTEAM][2];       // a team's next block, double-buffered
 
@@ -959,80 +862,95 @@ qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
     __syncthreads();             // the next segment reuses the shared memory
   }
 
-  // ---------------- merge of the units this CTA covered partially ------------
-  // Only the first and the last unit of the range can be partial.  A unit's
-  // partials are merged by the last of its CTAs to arrive (atomic ticket), in
-  // one level when their volume is small, else in two: the last CTA of each
-  // group of kMergeGroup consecutive CTAs merges the group into a second-level
-  // partial and the last group merger merges those.  Nobody waits on anybody.
-  // Every thread's partial stores, then the barrier, then one thread's ticket
-  // with acquire-release semantics at GPU scope: the barrier orders the other
-  // threads' stores before that release, and in the CTA that draws the last
-  // ticket the barrier after it orders the acquire before every thread's
-  // reads of the partials.
-  __syncthreads();
-  for (int which = 0; which < 2; ++which) {
-    const int64_t u = which == 0 ? first_unit : udiv64(hi - 1, S);
-    if (which == 1 && u == first_unit) break;
-    const int64_t seg_lo = lo > u * S ? lo : u * S;
-    const int64_t seg_hi = hi < (u + 1) * S ? hi : (u + 1) * S;
-    if (seg_lo == u * S && seg_hi == (u + 1) * S) continue;     // complete: already written
-    const int64_t uh = udiv64(u, p.ncg);
-    const int cg = (int)(u - uh * p.ncg);
-    const int hbase = cg * HPC;
-    const int64_t cfirst = udiv64((u * S + 1) * nC - 1, T);
-    const int64_t clast = udiv64(((u + 1) * S) * nC - 1, T);
-    const int nparts = (int)(clast - cfirst + 1);
-    const int nrows = min(HPC, p.G - hbase);
-    // slot of the unit's first CTA: its second slot if it began in an
-    // earlier unit; every later CTA of the unit began in this one
-    const int64_t slot0 = 2 * cfirst + (udiv64(udiv64(cfirst * T, nC), S) == u ? 0 : 1);
-    auto slot_of = [&](int64_t c) -> int64_t { return c == cfirst ? slot0 : 2 * c; };
-    const int64_t out_base = (uh * p.G + hbase) * D;
-    if ((int64_t)nparts * nrows * D <= kMergeFlat) {
-      if (tid == 0) {
-        const unsigned prev = atom_add_acq_rel_gpu(&p.tickets[u], 1u);
-        const int last = prev == (unsigned)nparts - 1;
-        if (last) p.tickets[u] = 0u;
-        s_flag = last;
-      }
-      __syncthreads();
-      if (s_flag) {
-        merge_unit<D, HPC>(p.part_ml, p.part_o, nparts, slot0, cfirst, 1, tid, C::NTHR, nrows,
-                           p.out, p.out_dtype, out_base, nullptr, nullptr);
-      }
-    } else {
-      const int ngroups = (nparts + kMergeGroup - 1) / kMergeGroup;
-      const int gi = (int)((int64_t)blockIdx.x - cfirst) / kMergeGroup;
-      const int64_t c0 = cfirst + (int64_t)gi * kMergeGroup;
-      const int64_t lead = slot_of(c0);                       // the group's second-level slot
-      const int gsz = min(kMergeGroup, nparts - gi * kMergeGroup);
-      if (tid == 0) {
-        const unsigned prev = atom_add_acq_rel_gpu(&p.tickets1[lead], 1u);
-        const int last = prev == (unsigned)gsz - 1;
-        if (last) p.tickets1[lead] = 0u;
-        s_flag = last;
-      }
-      __syncthreads();
-      if (s_flag) {
-        merge_unit<D, HPC>(p.part_ml, p.part_o, gsz, lead, c0, 1, tid, C::NTHR, nrows,
-                           nullptr, 0, 0, p.part2_ml + lead * HPC * 2, p.part2_o + lead * HPC * D);
-        __syncthreads();
-        if (tid == 0) {
-          const unsigned prev = atom_add_acq_rel_gpu(&p.tickets[u], 1u);
-          const int last = prev == (unsigned)ngroups - 1;
-          if (last) p.tickets[u] = 0u;
-          s_flag = last;
-        }
-        __syncthreads();
-        if (s_flag) {
-          merge_unit<D, HPC>(p.part2_ml, p.part2_o, ngroups, slot0, cfirst, kMergeGroup, tid,
-                             C::NTHR, nrows, p.out, p.out_dtype, out_base, nullptr, nullptr);
-        }
+}
+
+// ---------------------------------------------------------------------------
+// Merge of split units: after the decode grid has completed, kMergeLanes
+// adjacent threads per (unit, row, 4 consecutive outputs) fold the unit's
+// partials -- one per CTA that covered part of the unit, every kMergeLanes-th
+// one per thread, loaded in one batch -- by log-sum-exp rescaling, combine
+// across the lanes with shuffles and write the normalized output.  A unit
+// that one CTA covered whole was written by that CTA.
+constexpr int kMergeThreads = 128;
+constexpr int kMergeLanes = 4;
+constexpr int kMergeBatch = 8;   // parts whose loads a thread has in flight
+
+template <int D, int HPC>
+__global__ void __launch_bounds__(kMergeThreads)
+qsdpa_merge_kernel(const __grid_constant__ DecodeParams p, int64_t nC) {
+  grid_dep_wait();               // the decode grid's partials are complete and visible
+  grid_dep_launch();
+  constexpr int V4 = D / 4;
+  const int64_t S = p.stages_per_unit, T = p.total_stages;
+  const int64_t gt = (int64_t)blockIdx.x * kMergeThreads + threadIdx.x;
+  const int sub = (int)(gt & (kMergeLanes - 1));
+  const int64_t item = gt / kMergeLanes;
+  const int64_t u = udiv64(item, HPC * V4);
+  const int r = (int)(item - u * (HPC * V4)), R = r / V4, e4 = r - R * V4;
+  const int64_t uh = udiv64(u, p.ncg);
+  const int head = (int)(u - uh * p.ncg) * HPC + R;
+  bool active = u < udiv64(T, S) && head < p.G;
+  // CTA c covered blocks [c*T/nC, (c+1)*T/nC): the unit's first and last CTA
+  const int64_t cfirst = active ? udiv64((u * S + 1) * nC - 1, T) : 0;
+  const int64_t clast = active ? udiv64((u + 1) * S * nC - 1, T) : 0;
+  const int n = (int)(clast - cfirst + 1);
+  active = active && n > 1;
+  // the first CTA used its second slot if its range began in an earlier unit
+  const int64_t slot0 = 2 * cfirst + (udiv64(udiv64(cfirst * T, nC), S) == u ? 0 : 1);
+  float M = -INFINITY, Ls = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int j0 = 0; active && sub + kMergeLanes * j0 < n; j0 += kMergeBatch) {
+    float4 o[kMergeBatch];
+    float2 v[kMergeBatch];
+#pragma unroll
+    for (int k = 0; k < kMergeBatch; ++k) {
+      const int pp = sub + kMergeLanes * (j0 + k);
+      if (pp < n) {
+        const int64_t sx = pp == 0 ? slot0 : 2 * (cfirst + pp);
+        o[k] = __ldcg(reinterpret_cast<const float4*>(p.part_o + (sx * HPC + R) * D) + e4);
+        v[k] = __ldcg(reinterpret_cast<const float2*>(p.part_ml + (sx * HPC + R) * 2));
+      } else {
+        o[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+        v[k] = make_float2(-INFINITY, 0.f);
       }
     }
-    __syncthreads();             // s_flag is reused
+    float Mb = M;
+#pragma unroll
+    for (int k = 0; k < kMergeBatch; ++k) Mb = fmaxf(Mb, v[k].x);
+    if (Mb != M) {
+      const float f = M == -INFINITY ? 0.f : ex2(M - Mb);
+      Ls *= f; acc.x *= f; acc.y *= f; acc.z *= f; acc.w *= f;
+      M = Mb;
+    }
+#pragma unroll
+    for (int k = 0; k < kMergeBatch; ++k) {
+      const float w = v[k].x == -INFINITY ? 0.f : ex2(v[k].x - M);
+      Ls = fmaf(w, v[k].y, Ls);
+      acc.x = fmaf(w, o[k].x, acc.x);
+      acc.y = fmaf(w, o[k].y, acc.y);
+      acc.z = fmaf(w, o[k].z, acc.z);
+      acc.w = fmaf(w, o[k].w, acc.w);
+    }
   }
+#pragma unroll
+  for (int off = 1; off < kMergeLanes; off <<= 1) {
+    const float M2 = __shfl_xor_sync(~0u, M, off), L2 = __shfl_xor_sync(~0u, Ls, off);
+    const float x2 = __shfl_xor_sync(~0u, acc.x, off), y2 = __shfl_xor_sync(~0u, acc.y, off);
+    const float z2 = __shfl_xor_sync(~0u, acc.z, off), w2 = __shfl_xor_sync(~0u, acc.w, off);
+    const float Mn = fmaxf(M, M2);
+    const float f1 = M == -INFINITY ? 0.f : ex2(M - Mn), f2 = M2 == -INFINITY ? 0.f : ex2(M2 - Mn);
+    Ls = Ls * f1 + L2 * f2;
+    acc.x = acc.x * f1 + x2 * f2; acc.y = acc.y * f1 + y2 * f2;
+    acc.z = acc.z * f1 + z2 * f2; acc.w = acc.w * f1 + w2 * f2;
+    M = Mn;
+  }
+  if (!active || sub != 0) return;
+  const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+  const int64_t oi = (uh * p.G + head) * D + e4 * 4;
+  store_from_float(p.out, p.out_dtype, oi, acc.x * inv);
+  store_from_float(p.out, p.out_dtype, oi + 1, acc.y * inv);
+  store_from_float(p.out, p.out_dtype, oi + 2, acc.z * inv);
+  store_from_float(p.out, p.out_dtype, oi + 3, acc.w * inv);
 }
 
 // Host-side helpers for one instance.
@@ -1052,21 +970,26 @@ struct DecodeInstance {
     }
     return cached;
   }
-  // Launched with programmatic stream serialization: the set-up before the
-  // kernel's grid_dep_wait() overlaps the tail of the previous kernel.
+  // Both kernels are launched with programmatic stream serialization: the
+  // set-up before a kernel's grid_dep_wait() overlaps the previous kernel.
   static cudaError_t launch(const DecodePlan& plan, const DecodeParams& p, cudaStream_t s) {
-    auto k = qsdpa_decode_kernel<D, BITS, GS, Q8, NC, F32OUT>;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)plan.grid);
     cfg.blockDim = dim3(C::NTHR);
     cfg.dynamicSmemBytes = C::SMEM;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, qsdpa_decode_kernel<D, BITS, GS, Q8, NC, F32OUT>, p);
+    if (e != cudaSuccess || !plan.merge) return e;
+    const int64_t threads = plan.units * (NC * 8) * (D / 4) * kMergeLanes;
+    cfg.gridDim = dim3((unsigned)((threads + kMergeThreads - 1) / kMergeThreads));
+    cfg.blockDim = dim3(kMergeThreads);
+    cfg.dynamicSmemBytes = 0;
+    return cudaLaunchKernelEx(&cfg, qsdpa_merge_kernel<D, NC * 8>, p, (int64_t)plan.grid);
   }
 };
 

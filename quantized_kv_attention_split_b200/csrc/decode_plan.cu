@@ -10,7 +10,7 @@ namespace {
 // Grid cap per SM used both for planning and for the workspace bound, so that
 // qsdpa_workspace_size() does not depend on the kernel instance.
 int max_ctas_per_sm(int D) { return dec_ctas_per_sm(D); }
-// Largest grid: the merge tree's second level then has at most 48 groups of 8.
+// Largest grid (the workspace holds two partial slots per CTA).
 constexpr int64_t kMaxGrid = 8 * 48;
 // Partials of at least this many floats count as large (16 rows x D = 256 do).
 constexpr int64_t kBigPartial = 2048;
@@ -45,32 +45,30 @@ void decode_chunking(int G, int* nc, int* ncg) {
   *ncg = (chunks + *nc - 1) / *nc;
 }
 
-// Workspace layout: [unit tickets][group tickets] (both zero between calls),
-// then per-CTA partials (o, then (m, l)), then per-group partials.
-void decode_ws_layout(size_t units, size_t hpc, int D, size_t maxgrid, DecodePlan* plan) {
-  plan->ws_tickets2 = round_up(units * 4, 256);
-  plan->ws_tickets = plan->ws_tickets2 + round_up(2 * maxgrid * 4, 256);
+// Workspace layout: a 256-byte header that is zero between calls (its first
+// word is the prefill's status word; decode leaves it alone), then two
+// partial slots per CTA: o, then (m, l).
+constexpr size_t kWsHeader = 256;
+void decode_ws_layout(size_t hpc, int D, size_t maxgrid, DecodePlan* plan) {
+  plan->ws_header = kWsHeader;
   plan->ws_part_o = round_up(2 * maxgrid * hpc * D * 4, 256);
   plan->ws_part_ml = round_up(2 * maxgrid * hpc * 2 * 4, 256);
-  plan->ws_total = plan->ws_tickets + 2 * (plan->ws_part_o + plan->ws_part_ml);
+  plan->ws_total = plan->ws_header + plan->ws_part_o + plan->ws_part_ml;
 }
 
 size_t decode_workspace_bound(int B, int Hq, int Hkv, int D) {
   if (B <= 0 || Hkv <= 0 || Hq % Hkv) return 0;
   int nc, ncg;
   decode_chunking(Hq / Hkv, &nc, &ncg);
+  (void)ncg;
   DecodePlan plan;
-  decode_ws_layout((size_t)B * Hkv * ncg, (size_t)nc * 8, D, max_grid(D), &plan);
+  decode_ws_layout((size_t)nc * 8, D, max_grid(D), &plan);
   return plan.ws_total;
 }
 
 size_t decode_workspace_zero_bytes(int B, int Hq, int Hkv) {
   if (B <= 0 || Hkv <= 0 || Hq % Hkv) return 0;
-  int nc, ncg;
-  decode_chunking(Hq / Hkv, &nc, &ncg);
-  DecodePlan plan;
-  decode_ws_layout((size_t)B * Hkv * ncg, (size_t)nc * 8, 64, max_grid(128), &plan);
-  return plan.ws_tickets;
+  return kWsHeader;
 }
 
 bool plan_decode(int D, int bits, int gs, int fmt, int out_f32, int B, int Hq, int Hkv,
@@ -91,7 +89,7 @@ bool plan_decode(int D, int bits, int gs, int fmt, int out_f32, int B, int Hq, i
   // One CTA per SM, each a contiguous equal share of the (unit, block) range.
   int64_t cap = (int64_t)sms * occ;
   cap = std::min<int64_t>(cap, plan->total_stages);
-  cap = std::min<int64_t>(cap, kMaxGrid);              // merge scratch holds <= 48 groups
+  cap = std::min<int64_t>(cap, kMaxGrid);              // partial slots in the workspace
   // A CTA's partial (rows x D fp32) is written, read back and merged; when it
   // is large (many query rows per KV head, wide heads) give every team of
   // every CTA several blocks, so that partials stay a small fraction of the
@@ -113,7 +111,12 @@ bool plan_decode(int D, int bits, int gs, int fmt, int out_f32, int B, int Hq, i
   }
   plan->grid = (int)std::max<int64_t>(1, grid);
   plan->smem = ops.smem;
-  decode_ws_layout((size_t)plan->units, (size_t)plan->hpc, D, max_grid(D), plan);
+  // a merge kernel runs after the decode kernel when some unit is split over
+  // several CTAs, i.e. some CTA boundary falls inside a unit
+  plan->merge = false;
+  for (int64_t c = 1; c < plan->grid && !plan->merge; ++c)
+    plan->merge = (c * plan->total_stages / plan->grid) % plan->stages_per_unit != 0;
+  decode_ws_layout((size_t)plan->hpc, D, max_grid(D), plan);
   return true;
 }
 

@@ -35,16 +35,12 @@ struct DecodeParams {
   const void* mask;
   int mask_dtype;
   int64_t msb, msh, msq;
-  // work split: units (b, kv-head, chunk-group) x stages of TK keys, divided
+  // work split: units (b, kv-head, chunk-group) x blocks of TK keys, divided
   // evenly over gridDim.x CTAs
   int64_t stages_per_unit;
   int64_t total_stages;
   float* part_o;            // [2 * nCTA][HPC][D]   per-CTA partials
   float* part_ml;           // [2 * nCTA][HPC][2]
-  float* part2_o;           // [2 * nCTA][HPC][D]   per-group partials (merge tree)
-  float* part2_ml;          // [2 * nCTA][HPC][2]
-  unsigned* tickets;        // [units], zero between calls
-  unsigned* tickets1;       // [2 * nCTA], zero between calls
 };
 
 struct DecodePlan {
@@ -56,9 +52,9 @@ struct DecodePlan {
   int64_t stages_per_unit;
   int64_t total_stages;
   int grid;
+  bool merge;               // some unit is split over several CTAs: merge kernel after
   size_t smem;
-  size_t ws_tickets;        // bytes (zeroed region: unit tickets + group tickets)
-  size_t ws_tickets2;       // offset of the group tickets inside the zeroed region
+  size_t ws_header;         // bytes before the partials (zero between calls)
   size_t ws_part_o;         // bytes of one partial array
   size_t ws_part_ml;        // bytes
   size_t ws_total;

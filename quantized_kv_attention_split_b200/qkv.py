@@ -206,7 +206,7 @@ def qsdpa_decode_noalloc(q: torch.Tensor, k: QuantCache, v: QuantCache, L: int, 
                          mask=None, out: Optional[torch.Tensor] = None, out_dtype=None,
                          stream=None) -> torch.Tensor:
     """Like :func:`qsdpa_decode` but without a workspace: the library keeps the
-    scratch in a fixed 16 MiB array of its own (for callers that cannot
+    scratch in a fixed 8 MiB array of its own (for callers that cannot
     allocate device memory at decode time).  ``out`` should be passed by such
     callers; it is only allocated here when omitted.  Calls must not overlap
     on the GPU."""

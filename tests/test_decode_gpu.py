@@ -133,7 +133,7 @@ def test_workspace_reuse_and_canaries(qkv):
         qkv.qsdpa_decode(qd, kd, vd, L, 1.0, out=out, workspace=ws)
         torch.cuda.synchronize()
         assert max_err(from_dev(out), ref) <= TOL["f16"]
-        assert torch.all(ws[:nz] == 0), "tickets must be back to zero after a call"
+        assert torch.all(ws[:nz] == 0), "the zeroed header must stay zero after a decode"
     assert torch.all(buf[:32] == 7.0) and torch.all(buf[32 + n:] == 7.0)
 
 
