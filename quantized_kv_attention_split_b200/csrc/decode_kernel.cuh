@@ -89,6 +89,13 @@ __host__ __device__ __forceinline__ constexpr int swz_line(int line) {
           ((line & 4) ? ((SWZ >> 6) & 7) : 0) ^ ((line & 8) ? ((SWZ >> 9) & 7) : 0)) << 4;
 }
 
+// Swizzled offset of byte offset `lin` (lin with its unit bits XORed by the
+// pattern of its line); linear over XOR of offsets.
+template <uint32_t SWZ>
+__host__ __device__ __forceinline__ constexpr int swz_xor(int lin) {
+  return lin ^ swz_line<SWZ>((lin >> 7) & 15);
+}
+
 template <uint32_t SWZ>
 __device__ __forceinline__ int swz_offset(int lin) {
   const int line = lin >> 7;
@@ -296,6 +303,16 @@ qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
     // part and a per-k constant.
     const int fx = swz_line<C::SWZ>((ttid >> 3) & 15);
     const int fxv = swz_line<C::SWZV>((ttid >> 3) & 15);
+    // a lane's metadata unit when every lane copies at most one: unit ttid is
+    // 16-byte unit ttid % META_UNITS of array ttid / META_UNITS (lanes past
+    // the last unit copy nothing)
+    const uint8_t* mlane;
+    {
+      const int marr = ttid / C::META_UNITS, mj16 = (ttid - marr * C::META_UNITS) * 16;
+      const uint16_t* arr = Q8 ? (marr == 0 ? p.ks : p.vs)
+                               : (marr == 0 ? p.ks : marr == 1 ? p.kb : marr == 2 ? p.vs : p.vb);
+      mlane = reinterpret_cast<const uint8_t*>(arr) + mj16;
+    }
     auto issue_block = [&](int blk, int slot) {
       const uint32_t sbase = smem_u32(ring + slot * C::STAGE);
       const int64_t key0 = (int64_t)(s0 + blk) * BK;
@@ -332,6 +349,16 @@ qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
         }
       }
       // metadata: affine K scales, K biases, V scales, V biases; Q8_0 K and V scales
+      if constexpr (C::MU <= TTHR) {
+        // one unit per lane: its array and offset were chosen once (mlane)
+        if (C::MU == TTHR || ttid < C::MU) {
+          const int marr = ttid / C::META_UNITS, mj16 = (ttid - marr * C::META_UNITS) * 16;
+          const bool ok = mj16 / C::MROW < nvalid;
+          cp_async16(sbase + 2 * C::CODES + marr * C::META + mj16,
+                     mlane + grow * C::MROW - (ok ? 0 : mj16), ok ? 16 : 0);
+        }
+        return;
+      }
 #pragma unroll
       for (int k = 0; k < (C::MU + TTHR - 1) / TTHR; ++k) {
         const int i = ttid + k * TTHR;
@@ -346,23 +373,24 @@ qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
       }
     };
 
-    // fragment offsets inside a tile (fixed per lane).  The swizzle is linear
-    // in the line bits and a group never straddles a line, so it splits into
-    // a per-row part (computed once here), a per-group constant and, for the
-    // second 16-key sub-block, the constant of a 16-row shift.
-    auto row_x = [&](int r) { return swz_line<C::SWZ>((r * C::RB) >> 7); };
-    const int xk0 = row_x(g), xk1 = row_x(g + 8);
-    // value fragments: ldmatrix rows.  Lane l addresses row l % 8 of matrix
-    // l / 8; matrices 0/1 hold keys 0-7, 2/3 keys 8-15 of the 16-key block, and
-    // matrices 0/2 the first, 1/3 the second 16-byte unit of a unit pair (x2
-    // loads for 4-bit groups of 32: matrix 0 keys 0-7, matrix 1 keys 8-15).
+    // Fragment offsets inside a tile.  A fragment address is a per-lane part
+    // plus a compile-time part (sub-block, group, unit) whose bits do not
+    // overlap, so the sum is an XOR, and the swizzle is linear over XOR: the
+    // swizzled offset is the swizzled lane part XOR the swizzled constant.
+    //  key fragments: row g (or g + 8) of the sub-block, the lane's words t
+    const int kl0 = swz_xor<C::SWZ>(g * C::RB + t * C::NW * 4);
+    const int kl1 = swz_xor<C::SWZ>((g + 8) * C::RB + t * C::NW * 4);
+    auto kconst = [](int st, int G, int part) {
+      return swz_xor<C::SWZ>(st * 16 * C::RB + G * C::GB + part * 16);
+    };
+    //  value fragments: ldmatrix rows.  Lane l addresses row l % 8 of matrix
+    //  l / 8; matrices 0/1 hold keys 0-7, 2/3 keys 8-15 of the 16-key block,
+    //  and matrices 0/2 the first, 1/3 the second 16-byte unit of a unit pair
+    //  (x2 loads for 4-bit groups of 32: matrix 0 keys 0-7, matrix 1 keys 8-15).
     constexpr bool VX2 = BITS == 4 && GS == 32;
     const int vkey = (lane & 7) + (VX2 ? ((lane >> 3) & 1) * 8 : ((lane >> 4) & 1) * 8);
     const int vunit = VX2 ? 0 : ((lane >> 3) & 1);
-    auto koff = [&](int r, int x, int st, int G, int part) {
-      return ((r * C::RB + G * C::GB + t * C::NW * 4 + part * 16) ^ x) ^
-             swz_line<C::SWZ>((G * C::GB) >> 7) ^ swz_line<C::SWZ>((st * 16 * C::RB) >> 7);
-    };
+    const int vl = swz_xor<C::SWZV>(vkey * C::RB + vunit * 16);
 
     // ---------------- prologue ----------------------------------------------
     // The query rows go out first, then every team's first NSTAGE-1 blocks,
@@ -535,8 +563,8 @@ qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
 #pragma unroll
           for (int part = 0; part < (C::NW + 3) / 4; ++part) {
             constexpr int PW = C::NW < 4 ? C::NW : 4;
-            lds_words<PW>(sK + koff(r0, xk0, st, G, part), w0 + part * 4);
-            lds_words<PW>(sK + koff(r1, xk1, st, G, part), w1 + part * 4);
+            lds_words<PW>(sK + (kl0 ^ kconst(st, G, part)), w0 + part * 4);
+            lds_words<PW>(sK + (kl1 ^ kconst(st, G, part)), w1 + part * 4);
           }
 #pragma unroll
           for (int m = 0; m < C::NW; ++m) {
@@ -720,8 +748,7 @@ qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
           constexpr int PAIRS = VX2 ? 1 : (BITS == 4 ? GS / 64 : GS / 32);   // unit pairs per group
 #pragma unroll
           for (int pr = 0; pr < PAIRS; ++pr) {
-            const int lin = (vkey + 16 * st) * C::RB + G * C::GB + (2 * pr + vunit) * 16;
-            const uint32_t va = smem_u32(sV) + swz_offset<C::SWZV>(lin);
+            const uint32_t va = smem_u32(sV) + (vl ^ swz_xor<C::SWZV>(16 * st * C::RB + G * C::GB + 2 * pr * 16));
             uint32_t R[4];
             if constexpr (VX2) {
               ldsm_x2_trans(va, R[0], R[2]);
