@@ -909,21 +909,31 @@ qsdpa_merge_kernel(const __grid_constant__ DecodeParams p, int64_t nC) {
   grid_dep_launch();
   constexpr int V4 = D / 4;
   const int64_t S = p.stages_per_unit, T = p.total_stages;
-  const int64_t gt = (int64_t)blockIdx.x * kMergeThreads + threadIdx.x;
-  const int sub = (int)(gt & (kMergeLanes - 1));
-  const int64_t item = gt / kMergeLanes;
-  const int64_t u = udiv64(item, HPC * V4);
-  const int r = (int)(item - u * (HPC * V4)), R = r / V4, e4 = r - R * V4;
-  const int64_t uh = udiv64(u, p.ncg);
-  const int head = (int)(u - uh * p.ncg) * HPC + R;
-  bool active = u < udiv64(T, S) && head < p.G;
-  // CTA c covered blocks [c*T/nC, (c+1)*T/nC): the unit's first and last CTA
-  const int64_t cfirst = active ? udiv64((u * S + 1) * nC - 1, T) : 0;
-  const int64_t clast = active ? udiv64((u + 1) * S * nC - 1, T) : 0;
-  const int n = (int)(clast - cfirst + 1);
+  const int gt = blockIdx.x * kMergeThreads + threadIdx.x;
+  const int sub = gt & (kMergeLanes - 1);
+  const int item = gt / kMergeLanes;
+  const int u = item / (HPC * V4);
+  const int r = item - u * (HPC * V4), R = r / V4, e4 = r - R * V4;
+  const int uh = p.ncg == 1 ? u : u / p.ncg;
+  const int head = (u - uh * p.ncg) * HPC + R;
+  const int units = (int)udiv64(T, S);
+  bool active = u < units && head < p.G;
+  int64_t cfirst, slot0;
+  int n;
+  if (p.pieces > 0) {
+    // every CTA covered one piece of one unit: CTAs u*pieces ... in order
+    cfirst = (int64_t)u * p.pieces;
+    n = p.pieces;
+    slot0 = 2 * cfirst;
+  } else {
+    // CTA c covered blocks [c*T/nC, (c+1)*T/nC): the unit's first and last CTA
+    cfirst = active ? udiv64(((int64_t)u * S + 1) * nC - 1, T) : 0;
+    const int64_t clast = active ? udiv64(((int64_t)u + 1) * S * nC - 1, T) : 0;
+    n = (int)(clast - cfirst + 1);
+    // the first CTA used its second slot if its range began in an earlier unit
+    slot0 = 2 * cfirst + (udiv64(udiv64(cfirst * T, nC), S) == u ? 0 : 1);
+  }
   active = active && n > 1;
-  // the first CTA used its second slot if its range began in an earlier unit
-  const int64_t slot0 = 2 * cfirst + (udiv64(udiv64(cfirst * T, nC), S) == u ? 0 : 1);
   float M = -INFINITY, Ls = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int j0 = 0; active && sub + kMergeLanes * j0 < n; j0 += kMergeBatch) {
@@ -973,7 +983,7 @@ qsdpa_merge_kernel(const __grid_constant__ DecodeParams p, int64_t nC) {
   }
   if (!active || sub != 0) return;
   const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
-  const int64_t oi = (uh * p.G + head) * D + e4 * 4;
+  const int64_t oi = ((int64_t)uh * p.G + head) * D + e4 * 4;
   store_from_float(p.out, p.out_dtype, oi, acc.x * inv);
   store_from_float(p.out, p.out_dtype, oi + 1, acc.y * inv);
   store_from_float(p.out, p.out_dtype, oi + 2, acc.z * inv);

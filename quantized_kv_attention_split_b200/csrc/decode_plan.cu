@@ -116,6 +116,7 @@ bool plan_decode(int D, int bits, int gs, int fmt, int out_f32, int B, int Hq, i
   plan->merge = false;
   for (int64_t c = 1; c < plan->grid && !plan->merge; ++c)
     plan->merge = (c * plan->total_stages / plan->grid) % plan->stages_per_unit != 0;
+  plan->pieces = plan->grid % plan->units == 0 ? (int)(plan->grid / plan->units) : 0;
   decode_ws_layout((size_t)plan->hpc, D, max_grid(D), plan);
   return true;
 }
@@ -127,6 +128,7 @@ cudaError_t launch_decode(int D, int bits, int gs, int fmt, int out_f32, const D
   p.ncg = plan.ncg;
   p.stages_per_unit = plan.stages_per_unit;
   p.total_stages = plan.total_stages;
+  p.pieces = plan.pieces;
   return ops.launch(plan, p, stream);
 }
 

@@ -39,6 +39,7 @@ struct DecodeParams {
   // evenly over gridDim.x CTAs
   int64_t stages_per_unit;
   int64_t total_stages;
+  int pieces;               // CTAs per unit when every CTA covers one piece of one unit, else 0
   float* part_o;            // [2 * nCTA][HPC][D]   per-CTA partials
   float* part_ml;           // [2 * nCTA][HPC][2]
 };
@@ -52,6 +53,7 @@ struct DecodePlan {
   int64_t stages_per_unit;
   int64_t total_stages;
   int grid;
+  int pieces;               // CTAs per unit when the grid cuts every unit alike, else 0
   bool merge;               // some unit is split over several CTAs: merge kernel after
   size_t smem;
   size_t ws_header;         // bytes before the partials (zero between calls)
