@@ -10,8 +10,9 @@
 //           bias = fp16(min); code = clamp(rint((x - bias) / scale))
 //   Q8_0:   scale = fp16(max|x| / 127); code = clamp(rint(x / scale), +-127)
 //
-// Design: one thread owns 16 consecutive elements (two 16-byte loads), the
-// gs/16 lanes of a group reduce min/max with shuffles, each thread packs its
+// Design: one thread owns 16 consecutive elements (two 16-byte loads) and
+// takes their min / max (or largest magnitude) on the packed 16-bit pairs;
+// the gs/16 lanes of a group reduce with shuffles, each thread packs its
 // 16 codes into two (4-bit) or four (8-bit) words and stores them; the first
 // lane of a group stores the fp16 scale (and bias).  Grid: x = blocks of
 // tokens (256 / (D/16) tokens per block), y = (batch, kv head) slab, z = K or
@@ -39,24 +40,59 @@ struct QuantParams {
   int64_t offset;
 };
 
+// Packed pairs of 16-bit inputs (fp16 or bf16): elementwise min / max
+// (exact: a selection), magnitudes, and the conversion of a pair to fp32.
 template <bool BF16>
-__device__ __forceinline__ float in_to_float(uint16_t b) {
-  if constexpr (BF16) return __uint_as_float((uint32_t)b << 16);
-  else return __half2float(__ushort_as_half(b));
+__device__ __forceinline__ uint32_t pmin(uint32_t a, uint32_t b) {
+  uint32_t r;
+  if constexpr (BF16) {
+    const __nv_bfloat162 v = __hmin2(*reinterpret_cast<const __nv_bfloat162*>(&a),
+                                     *reinterpret_cast<const __nv_bfloat162*>(&b));
+    r = *reinterpret_cast<const uint32_t*>(&v);
+  } else {
+    const __half2 v = __hmin2(*reinterpret_cast<const __half2*>(&a), *reinterpret_cast<const __half2*>(&b));
+    r = *reinterpret_cast<const uint32_t*>(&v);
+  }
+  return r;
+}
+template <bool BF16>
+__device__ __forceinline__ uint32_t pmax(uint32_t a, uint32_t b) {
+  uint32_t r;
+  if constexpr (BF16) {
+    const __nv_bfloat162 v = __hmax2(*reinterpret_cast<const __nv_bfloat162*>(&a),
+                                     *reinterpret_cast<const __nv_bfloat162*>(&b));
+    r = *reinterpret_cast<const uint32_t*>(&v);
+  } else {
+    const __half2 v = __hmax2(*reinterpret_cast<const __half2*>(&a), *reinterpret_cast<const __half2*>(&b));
+    r = *reinterpret_cast<const uint32_t*>(&v);
+  }
+  return r;
+}
+template <bool BF16>
+__device__ __forceinline__ float2 to_f2(uint32_t w) {
+  if constexpr (BF16) return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+  else return __half22float2(*reinterpret_cast<const __half2*>(&w));
 }
 
 // rint(RN(d / s)) -- the code decision of the quantizer -- without a division
-// in the common case.  With r = RN(1/s), q0 = RN(d * r) is within 2^-14 of
-// RN(d / s) whenever |q0| < 2^9 (two roundings of relative error 2^-24 each),
-// so both round to the same integer unless q0 lies within 2^-13 of a
-// half-integer.  `exact` is set for that rare case and for any |q0| >= 2^9 or
-// non-finite value; the caller then redoes the row with the correctly rounded
-// division, so the result is always identical to it.
+// or a conversion instruction in the common case.  With r = RN(1/s),
+// q0 = RN(d * r) is within 2^-14 of RN(d / s) whenever |q0| < 2^9 (two
+// roundings of relative error 2^-24 each), so both round to the same integer
+// unless q0 lies within 2^-13 of a half-integer.  The integer is taken by
+// adding 1.5 * 2^23 (the sum's unit in the last place is 1, so the addition
+// rounds q0 to the nearest integer, ties to even, for |q0| < 2^22) and reading
+// the sum's low bits.  `exact` is set for the rare near-tie and for any
+// |q0| >= 2^9 or non-finite value; the caller then redoes the group's row
+// with the correctly rounded division, so the result is always identical to
+// it.
+constexpr float kRoundMagic = 12582912.f;            // 1.5 * 2^23
+constexpr int kRoundMagicBits = 0x4B400000;
 __device__ __forceinline__ int fast_rint_div(float d, float r, bool& exact) {
   const float q0 = __fmul_rn(d, r);
-  const float n = rintf(q0);
-  exact |= !(fabsf(q0) < 512.f) | (fabsf(fabsf(__fsub_rn(q0, n)) - 0.5f) < 0x1p-13f);
-  return (int)fminf(fmaxf(n, -512.f), 512.f);
+  const float y = __fadd_rn(q0, kRoundMagic);
+  const float n = __fsub_rn(y, kRoundMagic);
+  exact |= !(fabsf(q0) < 512.f) | (fabsf(__fsub_rn(q0, n)) > 0.5f - 0x1p-13f);
+  return __float_as_int(y) - kRoundMagicBits;
 }
 
 template <int LANES>
@@ -75,7 +111,7 @@ __device__ __forceinline__ float group_min(float v) {
 constexpr int kQEpt = 16;   // elements per thread (two 16-byte loads)
 
 template <int GS, int BITS, bool Q8, bool BF16>
-__global__ void __launch_bounds__(256) qkv_quantize_kernel(const QuantParams p, int side0) {
+__global__ void __launch_bounds__(256) qkv_quantize_kernel(const __grid_constant__ QuantParams p, int side0) {
   constexpr int LANES = GS / kQEpt;                 // threads per group
   const QuantSide& s = (side0 + (int)blockIdx.z) ? p.side[1] : p.side[0];
   const int per_row = p.D / kQEpt;
@@ -85,19 +121,21 @@ __global__ void __launch_bounds__(256) qkv_quantize_kernel(const QuantParams p, 
   const int64_t slab = blockIdx.y;                  // b * Hkv + kv head
   const int64_t srow = slab * p.Lnew + (active ? tok : 0);
   const int64_t crow = slab * s.Lcap + p.offset + tok;
-  float x[kQEpt];
+  uint32_t w[8];                                    // 16 raw 16-bit inputs, two per word
   if (active) {
     const uint4* src = reinterpret_cast<const uint4*>(s.src + srow * p.D + c16 * kQEpt);
     const uint4 r0 = __ldg(src), r1 = __ldg(src + 1);
-    const uint32_t w[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      x[2 * i] = in_to_float<BF16>((uint16_t)(w[i] & 0xffff));
-      x[2 * i + 1] = in_to_float<BF16>((uint16_t)(w[i] >> 16));
-    }
+    w[0] = r0.x; w[1] = r0.y; w[2] = r0.z; w[3] = r0.w;
+    w[4] = r1.x; w[5] = r1.y; w[6] = r1.z; w[7] = r1.w;
   } else {
 #pragma unroll
-    for (int i = 0; i < kQEpt; ++i) x[i] = 0.f;
+    for (int i = 0; i < 8; ++i) w[i] = 0u;
+  }
+  float x[kQEpt];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float2 f = to_f2<BF16>(w[i]);
+    x[2 * i] = f.x; x[2 * i + 1] = f.y;
   }
   const int grp = (c16 * kQEpt) / GS;
   const bool leader = ((c16 * kQEpt) % GS) == 0;
@@ -105,10 +143,11 @@ __global__ void __launch_bounds__(256) qkv_quantize_kernel(const QuantParams p, 
   int q[kQEpt];
   uint16_t sbits, bbits = 0;
   if constexpr (Q8) {
-    float a = 0.f;
+    uint32_t a2 = w[0] & 0x7fff7fffu;
 #pragma unroll
-    for (int i = 0; i < kQEpt; ++i) a = fmaxf(a, fabsf(x[i]));
-    a = group_max<LANES>(a);
+    for (int i = 1; i < 8; ++i) a2 = pmax<BF16>(a2, w[i] & 0x7fff7fffu);
+    const float2 af = to_f2<BF16>(a2);
+    const float a = group_max<LANES>(fmaxf(af.x, af.y));
     const float d = __fdiv_rn(a, 127.f);
     const __half d16 = __float2half_rn(d);
     const float df = __half2float(d16);
@@ -122,13 +161,14 @@ __global__ void __launch_bounds__(256) qkv_quantize_kernel(const QuantParams p, 
       for (int i = 0; i < kQEpt; ++i) q[i] = __float2int_rn(__fdiv_rn(x[i], df));
     }
 #pragma unroll
-    for (int i = 0; i < kQEpt; ++i) q[i] = df == 0.f ? 0 : (q[i] < -127 ? -127 : (q[i] > 127 ? 127 : q[i]));
+    for (int i = 0; i < kQEpt; ++i) q[i] = df == 0.f ? 0 : min(max(q[i], -127), 127);
   } else {
-    float mn = x[0], mx = x[0];
+    uint32_t mn2 = w[0], mx2 = w[0];
 #pragma unroll
-    for (int i = 1; i < kQEpt; ++i) { mn = fminf(mn, x[i]); mx = fmaxf(mx, x[i]); }
-    mn = group_min<LANES>(mn);
-    mx = group_max<LANES>(mx);
+    for (int i = 1; i < 8; ++i) { mn2 = pmin<BF16>(mn2, w[i]); mx2 = pmax<BF16>(mx2, w[i]); }
+    const float2 fmn = to_f2<BF16>(mn2), fmx = to_f2<BF16>(mx2);
+    const float mn = group_min<LANES>(fminf(fmn.x, fmn.y));
+    const float mx = group_max<LANES>(fmaxf(fmx.x, fmx.y));
     constexpr float levels = (float)((1 << BITS) - 1);
     float sc = __fdiv_rn(__fsub_rn(mx, mn), levels);
     sc = fmaxf(sc, 1e-7f);
@@ -146,19 +186,28 @@ __global__ void __launch_bounds__(256) qkv_quantize_kernel(const QuantParams p, 
       for (int i = 0; i < kQEpt; ++i) q[i] = __float2int_rn(__fdiv_rn(__fsub_rn(x[i], bf), sf));
     }
 #pragma unroll
-    for (int i = 0; i < kQEpt; ++i) q[i] = q[i] < 0 ? 0 : (q[i] > (1 << BITS) - 1 ? (1 << BITS) - 1 : q[i]);
+    for (int i = 0; i < kQEpt; ++i) q[i] = min(max(q[i], 0), (1 << BITS) - 1);
   }
   if (active) {
     if constexpr (BITS == 4) {
-      uint32_t w[2] = {0u, 0u};
+      // codes in [0, 15]: the sum of shifted codes is their bitwise or
+      uint32_t o[2];
 #pragma unroll
-      for (int i = 0; i < kQEpt; ++i) w[i >> 3] |= (uint32_t)q[i] << ((i & 7) * 4);
-      *reinterpret_cast<uint2*>(s.codes + crow * (p.D / 8) + c16 * 2) = make_uint2(w[0], w[1]);
+      for (int j = 0; j < 2; ++j) {
+        uint32_t v = 0u;
+#pragma unroll
+        for (int i = 7; i >= 0; --i) v = v * 16u + (uint32_t)q[8 * j + i];
+        o[j] = v;
+      }
+      *reinterpret_cast<uint2*>(s.codes + crow * (p.D / 8) + c16 * 2) = make_uint2(o[0], o[1]);
     } else {
-      uint32_t w[4] = {0u, 0u, 0u, 0u};
+      // low bytes of four codes per word (Q8_0 codes are signed)
+      uint32_t o[4];
 #pragma unroll
-      for (int i = 0; i < kQEpt; ++i) w[i >> 2] |= (uint32_t)(q[i] & 0xff) << ((i & 3) * 8);
-      *reinterpret_cast<uint4*>(s.codes + crow * (p.D / 4) + c16 * 4) = make_uint4(w[0], w[1], w[2], w[3]);
+      for (int j = 0; j < 4; ++j)
+        o[j] = __byte_perm(__byte_perm((uint32_t)q[4 * j], (uint32_t)q[4 * j + 1], 0x0040),
+                           __byte_perm((uint32_t)q[4 * j + 2], (uint32_t)q[4 * j + 3], 0x0040), 0x5410);
+      *reinterpret_cast<uint4*>(s.codes + crow * (p.D / 4) + c16 * 4) = make_uint4(o[0], o[1], o[2], o[3]);
     }
     if (leader) {
       s.scales[crow * ng + grp] = sbits;
