@@ -76,22 +76,23 @@ __device__ __forceinline__ float2 to_f2(uint32_t w) {
 
 // rint(RN(d / s)) -- the code decision of the quantizer -- without a division
 // or a conversion instruction in the common case.  With r = RN(1/s),
-// q0 = RN(d * r) is within 2^-14 of RN(d / s) whenever |q0| < 2^9 (two
-// roundings of relative error 2^-24 each), so both round to the same integer
-// unless q0 lies within 2^-13 of a half-integer.  The integer is taken by
-// adding 1.5 * 2^23 (the sum's unit in the last place is 1, so the addition
-// rounds q0 to the nearest integer, ties to even, for |q0| < 2^22) and reading
-// the sum's low bits.  `exact` is set for the rare near-tie and for any
-// |q0| >= 2^9 or non-finite value; the caller then redoes the group's row
-// with the correctly rounded division, so the result is always identical to
-// it.
+// q0 = RN(d * r) differs from RN(d / s) by less than 2^-14 whenever
+// |q0| < 2^9 (two roundings of relative error 2^-24 each), so both round to
+// the same integer unless q0 lies within 2^-13 of a half-integer.  The integer
+// is taken by adding 1.5 * 2^23 (the sum's unit in the last place is 1, so the
+// addition rounds q0 to the nearest integer, ties to even, for |q0| < 2^22)
+// and reading the sum's low bits.  `exact` is set for a near-tie or a
+// non-finite q0; the caller then redoes the row with the correctly rounded
+// division, so the result is always identical to it.  For |q0| >= 2^9 the
+// result may be off, but then both it and the true code lie beyond the code
+// range on the same side (the read-back integer is monotone in q0 and keeps
+// its sign), so the caller's clamp gives the same code.
 constexpr float kRoundMagic = 12582912.f;            // 1.5 * 2^23
 constexpr int kRoundMagicBits = 0x4B400000;
 __device__ __forceinline__ int fast_rint_div(float d, float r, bool& exact) {
   const float q0 = __fmul_rn(d, r);
   const float y = __fadd_rn(q0, kRoundMagic);
-  const float n = __fsub_rn(y, kRoundMagic);
-  exact |= !(fabsf(q0) < 512.f) | (fabsf(__fsub_rn(q0, n)) > 0.5f - 0x1p-13f);
+  exact |= !(fabsf(__fsub_rn(q0, __fsub_rn(y, kRoundMagic))) <= 0.5f - 0x1p-13f);
   return __float_as_int(y) - kRoundMagicBits;
 }
 
@@ -111,7 +112,7 @@ __device__ __forceinline__ float group_min(float v) {
 constexpr int kQEpt = 16;   // elements per thread (two 16-byte loads)
 
 template <int GS, int BITS, bool Q8, bool BF16>
-__global__ void __launch_bounds__(256) qkv_quantize_kernel(const __grid_constant__ QuantParams p, int side0) {
+__global__ void __launch_bounds__(256, 8) qkv_quantize_kernel(const __grid_constant__ QuantParams p, int side0) {
   constexpr int LANES = GS / kQEpt;                 // threads per group
   const QuantSide& s = (side0 + (int)blockIdx.z) ? p.side[1] : p.side[0];
   const int per_row = p.D / kQEpt;
@@ -131,37 +132,23 @@ __global__ void __launch_bounds__(256) qkv_quantize_kernel(const __grid_constant
 #pragma unroll
     for (int i = 0; i < 8; ++i) w[i] = 0u;
   }
-  float x[kQEpt];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const float2 f = to_f2<BF16>(w[i]);
-    x[2 * i] = f.x; x[2 * i + 1] = f.y;
-  }
   const int grp = (c16 * kQEpt) / GS;
   const bool leader = ((c16 * kQEpt) % GS) == 0;
   const int ng = p.D / GS;
-  int q[kQEpt];
+  // per group: the value subtracted (bias; 0 for Q8_0), the fp16 scale as
+  // float, its reciprocal, and the code range
   uint16_t sbits, bbits = 0;
+  float bf = 0.f, sf, rs;
+  constexpr int QLO = Q8 ? -127 : 0, QHI = Q8 ? 127 : (1 << BITS) - 1;
   if constexpr (Q8) {
     uint32_t a2 = w[0] & 0x7fff7fffu;
 #pragma unroll
     for (int i = 1; i < 8; ++i) a2 = pmax<BF16>(a2, w[i] & 0x7fff7fffu);
     const float2 af = to_f2<BF16>(a2);
     const float a = group_max<LANES>(fmaxf(af.x, af.y));
-    const float d = __fdiv_rn(a, 127.f);
-    const __half d16 = __float2half_rn(d);
-    const float df = __half2float(d16);
+    const __half d16 = __float2half_rn(__fdiv_rn(a, 127.f));
+    sf = __half2float(d16);
     sbits = __half_as_ushort(d16);
-    const float rd = __frcp_rn(df);
-    bool exact = false;
-#pragma unroll
-    for (int i = 0; i < kQEpt; ++i) q[i] = fast_rint_div(x[i], rd, exact);
-    if (exact) {
-#pragma unroll
-      for (int i = 0; i < kQEpt; ++i) q[i] = __float2int_rn(__fdiv_rn(x[i], df));
-    }
-#pragma unroll
-    for (int i = 0; i < kQEpt; ++i) q[i] = df == 0.f ? 0 : min(max(q[i], -127), 127);
   } else {
     uint32_t mn2 = w[0], mx2 = w[0];
 #pragma unroll
@@ -170,45 +157,47 @@ __global__ void __launch_bounds__(256) qkv_quantize_kernel(const __grid_constant
     const float mn = group_min<LANES>(fminf(fmn.x, fmn.y));
     const float mx = group_max<LANES>(fmaxf(fmx.x, fmx.y));
     constexpr float levels = (float)((1 << BITS) - 1);
-    float sc = __fdiv_rn(__fsub_rn(mx, mn), levels);
-    sc = fmaxf(sc, 1e-7f);
+    const float sc = fmaxf(__fdiv_rn(__fsub_rn(mx, mn), levels), 1e-7f);
     const __half s16 = __float2half_rn(sc);
     const __half b16 = __float2half_rn(mn);
-    const float sf = __half2float(s16), bf = __half2float(b16);
+    sf = __half2float(s16);
+    bf = __half2float(b16);
     sbits = __half_as_ushort(s16);
     bbits = __half_as_ushort(b16);
-    const float rs = __frcp_rn(sf);
-    bool exact = false;
+  }
+  rs = __frcp_rn(sf);
+  // Codes two at a time straight from the packed inputs, packed as they come;
+  // a second pass with the correctly rounded division in the rare case that
+  // flags it.  Q8_0 with a zero scale gives zero codes.
+  constexpr int CPW = 32 / BITS;                    // codes per output word
+  uint32_t o[kQEpt / CPW];
+  auto emit = [&](int i, int c) {                   // code of element i, clamped
+    c = min(max(c, QLO), QHI);
+    if constexpr (Q8) c = sf == 0.f ? 0 : c;
+    const int sh = (i % CPW) * BITS;
+    const uint32_t u = (uint32_t)c & ((1u << BITS) - 1u);
+    o[i / CPW] = (i % CPW) == 0 ? u : o[i / CPW] | (u << sh);
+  };
+  bool exact = false;
 #pragma unroll
-    for (int i = 0; i < kQEpt; ++i) q[i] = fast_rint_div(__fsub_rn(x[i], bf), rs, exact);
-    if (exact) {
+  for (int i = 0; i < 8; ++i) {
+    const float2 f = to_f2<BF16>(w[i]);
+    emit(2 * i, fast_rint_div(__fsub_rn(f.x, bf), rs, exact));
+    emit(2 * i + 1, fast_rint_div(__fsub_rn(f.y, bf), rs, exact));
+  }
+  if (exact) {
 #pragma unroll
-      for (int i = 0; i < kQEpt; ++i) q[i] = __float2int_rn(__fdiv_rn(__fsub_rn(x[i], bf), sf));
+    for (int i = 0; i < 8; ++i) {
+      const float2 f = to_f2<BF16>(w[i]);
+      emit(2 * i, __float2int_rn(__fdiv_rn(__fsub_rn(f.x, bf), sf)));
+      emit(2 * i + 1, __float2int_rn(__fdiv_rn(__fsub_rn(f.y, bf), sf)));
     }
-#pragma unroll
-    for (int i = 0; i < kQEpt; ++i) q[i] = min(max(q[i], 0), (1 << BITS) - 1);
   }
   if (active) {
-    if constexpr (BITS == 4) {
-      // codes in [0, 15]: the sum of shifted codes is their bitwise or
-      uint32_t o[2];
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        uint32_t v = 0u;
-#pragma unroll
-        for (int i = 7; i >= 0; --i) v = v * 16u + (uint32_t)q[8 * j + i];
-        o[j] = v;
-      }
+    if constexpr (BITS == 4)
       *reinterpret_cast<uint2*>(s.codes + crow * (p.D / 8) + c16 * 2) = make_uint2(o[0], o[1]);
-    } else {
-      // low bytes of four codes per word (Q8_0 codes are signed)
-      uint32_t o[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        o[j] = __byte_perm(__byte_perm((uint32_t)q[4 * j], (uint32_t)q[4 * j + 1], 0x0040),
-                           __byte_perm((uint32_t)q[4 * j + 2], (uint32_t)q[4 * j + 3], 0x0040), 0x5410);
+    else
       *reinterpret_cast<uint4*>(s.codes + crow * (p.D / 4) + c16 * 4) = make_uint4(o[0], o[1], o[2], o[3]);
-    }
     if (leader) {
       s.scales[crow * ng + grp] = sbits;
       if constexpr (!Q8) s.biases[crow * ng + grp] = bbits;
