@@ -35,7 +35,7 @@ struct QuantSide {
 struct QuantParams {
   QuantSide side[2];
   int D;
-  int row_shift;            // log2(D / 8): threads per token row
+  int row_shift;            // log2(D / 32): threads per token row
   int Lnew;
   int64_t offset;
 };
@@ -109,54 +109,61 @@ __device__ __forceinline__ float group_min(float v) {
   return v;
 }
 
-constexpr int kQEpt = 16;   // elements per thread (two 16-byte loads)
+constexpr int kQEpt = 32;   // elements per thread (four 16-byte loads)
+constexpr int kQWords = kQEpt / 2;
 
 template <int GS, int BITS, bool Q8, bool BF16>
-__global__ void __launch_bounds__(256, 8) qkv_quantize_kernel(const __grid_constant__ QuantParams p, int side0) {
+__global__ void __launch_bounds__(256, 6) qkv_quantize_kernel(const __grid_constant__ QuantParams p, int side0) {
   constexpr int LANES = GS / kQEpt;                 // threads per group
   const QuantSide& s = (side0 + (int)blockIdx.z) ? p.side[1] : p.side[0];
   const int per_row = p.D / kQEpt;
   const int tok = blockIdx.x * (256 >> p.row_shift) + (threadIdx.x >> p.row_shift);
-  const int c16 = threadIdx.x & (per_row - 1);      // which 16-element slice of the row
+  const int cs = threadIdx.x & (per_row - 1);       // which 32-element slice of the row
   const bool active = tok < p.Lnew;                 // inactive lanes still join the shuffles
   const int64_t slab = blockIdx.y;                  // b * Hkv + kv head
   const int64_t srow = slab * p.Lnew + (active ? tok : 0);
   const int64_t crow = slab * s.Lcap + p.offset + tok;
-  uint32_t w[8];                                    // 16 raw 16-bit inputs, two per word
+  uint32_t w[kQWords];                              // 32 raw 16-bit inputs, two per word
   if (active) {
-    const uint4* src = reinterpret_cast<const uint4*>(s.src + srow * p.D + c16 * kQEpt);
-    const uint4 r0 = __ldg(src), r1 = __ldg(src + 1);
-    w[0] = r0.x; w[1] = r0.y; w[2] = r0.z; w[3] = r0.w;
-    w[4] = r1.x; w[5] = r1.y; w[6] = r1.z; w[7] = r1.w;
+    const uint4* src = reinterpret_cast<const uint4*>(s.src + srow * p.D + cs * kQEpt);
+#pragma unroll
+    for (int k = 0; k < kQWords / 4; ++k) {
+      const uint4 r = __ldg(src + k);
+      w[4 * k] = r.x; w[4 * k + 1] = r.y; w[4 * k + 2] = r.z; w[4 * k + 3] = r.w;
+    }
   } else {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) w[i] = 0u;
+    for (int i = 0; i < kQWords; ++i) w[i] = 0u;
   }
-  const int grp = (c16 * kQEpt) / GS;
-  const bool leader = ((c16 * kQEpt) % GS) == 0;
+  const int grp = (cs * kQEpt) / GS;
+  const bool leader = ((cs * kQEpt) % GS) == 0;
   const int ng = p.D / GS;
   // per group: the value subtracted (bias; 0 for Q8_0), the fp16 scale as
-  // float, its reciprocal, and the code range
+  // float and its reciprocal; `inside` when every code of the group is known
+  // to fall inside the code range before clamping (then the clamp is skipped)
   uint16_t sbits, bbits = 0;
-  float bf = 0.f, sf, rs;
+  float bf = 0.f, sf;
+  bool inside;
   constexpr int QLO = Q8 ? -127 : 0, QHI = Q8 ? 127 : (1 << BITS) - 1;
   if constexpr (Q8) {
     uint32_t a2 = w[0] & 0x7fff7fffu;
 #pragma unroll
-    for (int i = 1; i < 8; ++i) a2 = pmax<BF16>(a2, w[i] & 0x7fff7fffu);
+    for (int i = 1; i < kQWords; ++i) a2 = pmax<BF16>(a2, w[i] & 0x7fff7fffu);
     const float2 af = to_f2<BF16>(a2);
     const float a = group_max<LANES>(fmaxf(af.x, af.y));
     const __half d16 = __float2half_rn(__fdiv_rn(a, 127.f));
     sf = __half2float(d16);
     sbits = __half_as_ushort(d16);
+    // |x| / d <= a / d; below 127.25 every code lies in [-127, 127]
+    inside = sf > 0.f && a < 127.25f * sf;
   } else {
     uint32_t mn2 = w[0], mx2 = w[0];
 #pragma unroll
-    for (int i = 1; i < 8; ++i) { mn2 = pmin<BF16>(mn2, w[i]); mx2 = pmax<BF16>(mx2, w[i]); }
+    for (int i = 1; i < kQWords; ++i) { mn2 = pmin<BF16>(mn2, w[i]); mx2 = pmax<BF16>(mx2, w[i]); }
     const float2 fmn = to_f2<BF16>(mn2), fmx = to_f2<BF16>(mx2);
     const float mn = group_min<LANES>(fminf(fmn.x, fmn.y));
     const float mx = group_max<LANES>(fmaxf(fmx.x, fmx.y));
-    constexpr float levels = (float)((1 << BITS) - 1);
+    constexpr float levels = (float)QHI;
     const float sc = fmaxf(__fdiv_rn(__fsub_rn(mx, mn), levels), 1e-7f);
     const __half s16 = __float2half_rn(sc);
     const __half b16 = __float2half_rn(mn);
@@ -164,40 +171,58 @@ __global__ void __launch_bounds__(256, 8) qkv_quantize_kernel(const __grid_const
     bf = __half2float(b16);
     sbits = __half_as_ushort(s16);
     bbits = __half_as_ushort(b16);
+    // (x - bias) / scale lies within [(mn - bias) / scale, (mx - bias) / scale];
+    // with margins of a quarter step both ends round into [0, levels]
+    inside = __fsub_rn(mn, bf) > -0.25f * sf && __fsub_rn(mx, bf) < (levels + 0.25f) * sf;
   }
-  rs = __frcp_rn(sf);
+  const float rs = __frcp_rn(sf);
   // Codes two at a time straight from the packed inputs, packed as they come;
   // a second pass with the correctly rounded division in the rare case that
   // flags it.  Q8_0 with a zero scale gives zero codes.
   constexpr int CPW = 32 / BITS;                    // codes per output word
   uint32_t o[kQEpt / CPW];
-  auto emit = [&](int i, int c) {                   // code of element i, clamped
-    c = min(max(c, QLO), QHI);
-    if constexpr (Q8) c = sf == 0.f ? 0 : c;
-    const int sh = (i % CPW) * BITS;
-    const uint32_t u = (uint32_t)c & ((1u << BITS) - 1u);
-    o[i / CPW] = (i % CPW) == 0 ? u : o[i / CPW] | (u << sh);
+  auto emit = [&](int i, int c, bool clamp) {       // code of element i
+    if (clamp) c = min(max(c, QLO), QHI);
+    if constexpr (Q8) {
+      // signed codes: their low bytes, four per word
+      c = sf == 0.f ? 0 : c;
+      const uint32_t sel = (i % 4) == 0 ? 0x3210u : (i % 4) == 1 ? 0x3240u : (i % 4) == 2 ? 0x3410u : 0x4210u;
+      o[i / 4] = (i % 4) == 0 ? (uint32_t)c & 0xffu : __byte_perm(o[i / 4], (uint32_t)c, sel);
+    } else {
+      // codes in [0, levels]: place them by multiplication, no masking
+      const uint32_t u = (uint32_t)c * (1u << ((i % CPW) * BITS));
+      o[i / CPW] = (i % CPW) == 0 ? u : o[i / CPW] + u;
+    }
   };
   bool exact = false;
+  if (__all_sync(~0u, inside)) {
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const float2 f = to_f2<BF16>(w[i]);
-    emit(2 * i, fast_rint_div(__fsub_rn(f.x, bf), rs, exact));
-    emit(2 * i + 1, fast_rint_div(__fsub_rn(f.y, bf), rs, exact));
+    for (int i = 0; i < kQWords; ++i) {
+      const float2 f = to_f2<BF16>(w[i]);
+      emit(2 * i, fast_rint_div(__fsub_rn(f.x, bf), rs, exact), false);
+      emit(2 * i + 1, fast_rint_div(__fsub_rn(f.y, bf), rs, exact), false);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < kQWords; ++i) {
+      const float2 f = to_f2<BF16>(w[i]);
+      emit(2 * i, fast_rint_div(__fsub_rn(f.x, bf), rs, exact), true);
+      emit(2 * i + 1, fast_rint_div(__fsub_rn(f.y, bf), rs, exact), true);
+    }
   }
   if (exact) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < kQWords; ++i) {
       const float2 f = to_f2<BF16>(w[i]);
-      emit(2 * i, __float2int_rn(__fdiv_rn(__fsub_rn(f.x, bf), sf)));
-      emit(2 * i + 1, __float2int_rn(__fdiv_rn(__fsub_rn(f.y, bf), sf)));
+      emit(2 * i, __float2int_rn(__fdiv_rn(__fsub_rn(f.x, bf), sf)), true);
+      emit(2 * i + 1, __float2int_rn(__fdiv_rn(__fsub_rn(f.y, bf), sf)), true);
     }
   }
   if (active) {
-    if constexpr (BITS == 4)
-      *reinterpret_cast<uint2*>(s.codes + crow * (p.D / 8) + c16 * 2) = make_uint2(o[0], o[1]);
-    else
-      *reinterpret_cast<uint4*>(s.codes + crow * (p.D / 4) + c16 * 4) = make_uint4(o[0], o[1], o[2], o[3]);
+    uint4* dst = reinterpret_cast<uint4*>(s.codes + crow * (p.D * BITS / 32) + cs * (kQEpt * BITS / 32));
+#pragma unroll
+    for (int k = 0; k < kQEpt * BITS / 128; ++k)
+      dst[k] = make_uint4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
     if (leader) {
       s.scales[crow * ng + grp] = sbits;
       if constexpr (!Q8) s.biases[crow * ng + grp] = bbits;
@@ -245,7 +270,7 @@ cudaError_t launch_quantize(const void* new_k, const void* new_v, int in_dtype, 
     gs[i] = c[i]->fmt == QKV_Q8_0 ? 32 : c[i]->group_size;
   }
   int shift = 0;
-  while ((kQEpt << shift) < D) ++shift;             // D / 16 = 2^shift threads per token
+  while ((kQEpt << shift) < D) ++shift;             // D / 32 = 2^shift threads per token
   p.D = D;
   p.row_shift = shift;
   p.Lnew = Lnew;
