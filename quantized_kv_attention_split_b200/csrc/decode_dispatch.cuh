@@ -4,8 +4,54 @@
 #pragma once
 
 #include "decode_kernel.cuh"
+#include "decode_merge.cuh"
 
 namespace qkv {
+
+// Host-side helpers for one instance.
+template <int D, int BITS, int GS, bool Q8, int NC, bool F32OUT>
+struct DecodeInstance {
+  using C = DecCfg<D, BITS, GS, Q8, NC>;
+  static int max_ctas_per_sm() {
+    static int cached = -1;
+    if (cached < 0) {
+      auto k = qsdpa_decode_kernel<D, BITS, GS, Q8, NC, F32OUT>;
+      if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
+        return 0;
+      int n = 0;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, C::NTHR, C::SMEM) != cudaSuccess)
+        return 0;
+      cached = n;
+    }
+    return cached;
+  }
+  // Both kernels are launched with programmatic stream serialization: the
+  // set-up before a kernel's grid_dep_wait() overlaps the previous kernel.
+  static cudaError_t launch(const DecodePlan& plan, const DecodeParams& p, cudaStream_t s) {
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)plan.grid);
+    cfg.blockDim = dim3(C::NTHR);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, qsdpa_decode_kernel<D, BITS, GS, Q8, NC, F32OUT>, p);
+    if (e != cudaSuccess || !plan.merge) return e;
+    // parts per unit: at most the CTAs that share one unit
+    const int64_t parts = plan.pieces > 0 ? plan.pieces : (plan.grid + plan.units - 1) / plan.units + 1;
+    int lanes = 1;
+    while (lanes < 4 && lanes * kMergeBatch < parts) lanes *= 2;
+    const int64_t threads = plan.units * (NC * 8) * (D / 4) * lanes;
+    cfg.gridDim = dim3((unsigned)((threads + kMergeThreads - 1) / kMergeThreads));
+    cfg.blockDim = dim3(kMergeThreads);
+    cfg.dynamicSmemBytes = 0;
+    return cudaLaunchKernelEx(&cfg, qsdpa_merge_kernel<D, NC * 8>, p, (int64_t)plan.grid, lanes);
+  }
+};
+
 
 struct DecodeOps {
   int (*occupancy)();

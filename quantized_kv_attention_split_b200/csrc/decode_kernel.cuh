@@ -11,9 +11,9 @@
 //  * Work: units (batch, kv-head, chunk-group of <=32 query heads) x blocks
 //    of BK (16 or 32) keys, flattened and cut evenly over one CTA per SM.  A
 //    CTA touches at most two units partially; a partial result (running max
-//    m, sum l, unnormalized o) goes to workspace and the last CTA of a unit
-//    to finish (atomic ticket) merges them (log-sum-exp rescaling) -- one
-//    launch, no waiting.  The launch is a programmatic dependent launch: its
+//    m, sum l, unnormalized o) goes to workspace and a second kernel
+//    (decode_merge.cuh) merges the partials of split units (log-sum-exp
+//    rescaling).  Both are programmatic dependent launches: a kernel's
 //    set-up overlaps the previous kernel of the stream.
 //  * Teams: the warps of a CTA form teams (one warp per 8-row head chunk).
 //    A team streams its own blocks -- handed out in order through a shared
@@ -890,144 +890,5 @@ qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
   }
 
 }
-
-// ---------------------------------------------------------------------------
-// Merge of split units: after the decode grid has completed, kMergeLanes
-// adjacent threads per (unit, row, 4 consecutive outputs) fold the unit's
-// partials -- one per CTA that covered part of the unit, every kMergeLanes-th
-// one per thread, loaded in one batch -- by log-sum-exp rescaling, combine
-// across the lanes with shuffles and write the normalized output.  A unit
-// that one CTA covered whole was written by that CTA.
-constexpr int kMergeThreads = 128;
-constexpr int kMergeLanes = 4;
-constexpr int kMergeBatch = 8;   // parts whose loads a thread has in flight
-
-template <int D, int HPC>
-__global__ void __launch_bounds__(kMergeThreads)
-qsdpa_merge_kernel(const __grid_constant__ DecodeParams p, int64_t nC) {
-  grid_dep_wait();               // the decode grid's partials are complete and visible
-  grid_dep_launch();
-  constexpr int V4 = D / 4;
-  const int64_t S = p.stages_per_unit, T = p.total_stages;
-  const int gt = blockIdx.x * kMergeThreads + threadIdx.x;
-  const int sub = gt & (kMergeLanes - 1);
-  const int item = gt / kMergeLanes;
-  const int u = item / (HPC * V4);
-  const int r = item - u * (HPC * V4), R = r / V4, e4 = r - R * V4;
-  const int uh = p.ncg == 1 ? u : u / p.ncg;
-  const int head = (u - uh * p.ncg) * HPC + R;
-  const int units = (int)udiv64(T, S);
-  bool active = u < units && head < p.G;
-  int64_t cfirst, slot0;
-  int n;
-  if (p.pieces > 0) {
-    // every CTA covered one piece of one unit: CTAs u*pieces ... in order
-    cfirst = (int64_t)u * p.pieces;
-    n = p.pieces;
-    slot0 = 2 * cfirst;
-  } else {
-    // CTA c covered blocks [c*T/nC, (c+1)*T/nC): the unit's first and last CTA
-    cfirst = active ? udiv64(((int64_t)u * S + 1) * nC - 1, T) : 0;
-    const int64_t clast = active ? udiv64(((int64_t)u + 1) * S * nC - 1, T) : 0;
-    n = (int)(clast - cfirst + 1);
-    // the first CTA used its second slot if its range began in an earlier unit
-    slot0 = 2 * cfirst + (udiv64(udiv64(cfirst * T, nC), S) == u ? 0 : 1);
-  }
-  active = active && n > 1;
-  float M = -INFINITY, Ls = 0.f;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int j0 = 0; active && sub + kMergeLanes * j0 < n; j0 += kMergeBatch) {
-    float4 o[kMergeBatch];
-    float2 v[kMergeBatch];
-#pragma unroll
-    for (int k = 0; k < kMergeBatch; ++k) {
-      const int pp = sub + kMergeLanes * (j0 + k);
-      if (pp < n) {
-        const int64_t sx = pp == 0 ? slot0 : 2 * (cfirst + pp);
-        o[k] = __ldcg(reinterpret_cast<const float4*>(p.part_o + (sx * HPC + R) * D) + e4);
-        v[k] = __ldcg(reinterpret_cast<const float2*>(p.part_ml + (sx * HPC + R) * 2));
-      } else {
-        o[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-        v[k] = make_float2(-INFINITY, 0.f);
-      }
-    }
-    float Mb = M;
-#pragma unroll
-    for (int k = 0; k < kMergeBatch; ++k) Mb = fmaxf(Mb, v[k].x);
-    if (Mb != M) {
-      const float f = M == -INFINITY ? 0.f : ex2(M - Mb);
-      Ls *= f; acc.x *= f; acc.y *= f; acc.z *= f; acc.w *= f;
-      M = Mb;
-    }
-#pragma unroll
-    for (int k = 0; k < kMergeBatch; ++k) {
-      const float w = v[k].x == -INFINITY ? 0.f : ex2(v[k].x - M);
-      Ls = fmaf(w, v[k].y, Ls);
-      acc.x = fmaf(w, o[k].x, acc.x);
-      acc.y = fmaf(w, o[k].y, acc.y);
-      acc.z = fmaf(w, o[k].z, acc.z);
-      acc.w = fmaf(w, o[k].w, acc.w);
-    }
-  }
-#pragma unroll
-  for (int off = 1; off < kMergeLanes; off <<= 1) {
-    const float M2 = __shfl_xor_sync(~0u, M, off), L2 = __shfl_xor_sync(~0u, Ls, off);
-    const float x2 = __shfl_xor_sync(~0u, acc.x, off), y2 = __shfl_xor_sync(~0u, acc.y, off);
-    const float z2 = __shfl_xor_sync(~0u, acc.z, off), w2 = __shfl_xor_sync(~0u, acc.w, off);
-    const float Mn = fmaxf(M, M2);
-    const float f1 = M == -INFINITY ? 0.f : ex2(M - Mn), f2 = M2 == -INFINITY ? 0.f : ex2(M2 - Mn);
-    Ls = Ls * f1 + L2 * f2;
-    acc.x = acc.x * f1 + x2 * f2; acc.y = acc.y * f1 + y2 * f2;
-    acc.z = acc.z * f1 + z2 * f2; acc.w = acc.w * f1 + w2 * f2;
-    M = Mn;
-  }
-  if (!active || sub != 0) return;
-  const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
-  const int64_t oi = ((int64_t)uh * p.G + head) * D + e4 * 4;
-  store_from_float(p.out, p.out_dtype, oi, acc.x * inv);
-  store_from_float(p.out, p.out_dtype, oi + 1, acc.y * inv);
-  store_from_float(p.out, p.out_dtype, oi + 2, acc.z * inv);
-  store_from_float(p.out, p.out_dtype, oi + 3, acc.w * inv);
-}
-
-// Host-side helpers for one instance.
-template <int D, int BITS, int GS, bool Q8, int NC, bool F32OUT>
-struct DecodeInstance {
-  using C = DecCfg<D, BITS, GS, Q8, NC>;
-  static int max_ctas_per_sm() {
-    static int cached = -1;
-    if (cached < 0) {
-      auto k = qsdpa_decode_kernel<D, BITS, GS, Q8, NC, F32OUT>;
-      if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
-        return 0;
-      int n = 0;
-      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, C::NTHR, C::SMEM) != cudaSuccess)
-        return 0;
-      cached = n;
-    }
-    return cached;
-  }
-  // Both kernels are launched with programmatic stream serialization: the
-  // set-up before a kernel's grid_dep_wait() overlaps the previous kernel.
-  static cudaError_t launch(const DecodePlan& plan, const DecodeParams& p, cudaStream_t s) {
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)plan.grid);
-    cfg.blockDim = dim3(C::NTHR);
-    cfg.dynamicSmemBytes = C::SMEM;
-    cfg.stream = s;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, qsdpa_decode_kernel<D, BITS, GS, Q8, NC, F32OUT>, p);
-    if (e != cudaSuccess || !plan.merge) return e;
-    const int64_t threads = plan.units * (NC * 8) * (D / 4) * kMergeLanes;
-    cfg.gridDim = dim3((unsigned)((threads + kMergeThreads - 1) / kMergeThreads));
-    cfg.blockDim = dim3(kMergeThreads);
-    cfg.dynamicSmemBytes = 0;
-    return cudaLaunchKernelEx(&cfg, qsdpa_merge_kernel<D, NC * 8>, p, (int64_t)plan.grid);
-  }
-};
 
 }  // namespace qkv
