@@ -480,6 +480,24 @@ def other_rows(device):
     rows["decode_64k_affine8"] = {"us_per_call": round(sec * 1e3, 3),
                                   "GB/s": round(nb / (sec / 1e3) / 1e9, 1),
                                   "frac_hbm": round(nb / (sec / 1e3) / 1e9 / hbm_peak, 4)}
+    # the decode step with its cache update: the separate calls (update of the
+    # token at row 65535, then decode over 65536 keys) and the fused call
+    def sstep(i):
+        a, b = copies[i % ncopies]
+        qkv.qkv_quantize_update(nk, nv, a, b, w.Lcap - 1)
+        qkv.qsdpa_decode(q, a, b, w.L, w.scale, out=out, workspace=ws)
+
+    def fstep(i):
+        a, b = copies[i % ncopies]
+        qkv.qsdpa_decode_update(q, nk, nv, a, b, w.Lcap - 1, w.scale, out=out, workspace=ws)
+    sec_s, _ = graph_time(sstep, 400, 20)
+    sec_f, _ = graph_time(fstep, 400, 20)
+    rows["update_decode_64k_affine8"] = {
+        "separate_us_per_call": round(sec_s * 1e3, 3), "fused_us_per_call": round(sec_f * 1e3, 3),
+        "fused_GB/s": round(nb / (sec_f / 1e3) / 1e9, 1),
+        "fused_frac_hbm": round(nb / (sec_f / 1e3) / 1e9 / hbm_peak, 4),
+        "note": "update of one token per kv head at row 65535 plus decode over 65536 keys: "
+                "qkv_quantize_update + qsdpa_decode vs qsdpa_decode_update (one decode launch)"}
     del copies, kc, vc
     torch.cuda.empty_cache()
 

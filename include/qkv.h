@@ -126,6 +126,22 @@ qkv_status qsdpa_decode(const void* q, int q_dtype, int B, int Hq, int Hkv, int 
                         float scale, const qkv_mask* mask, void* out, int out_dtype,
                         void* workspace, size_t workspace_bytes, void* stream);
 
+/* Fused decode step (the pages' two calls -- the cache update of the new
+ * token, then single-query attention -- in one decode launch; the pages have
+ * no fused form).  The new token of every (batch, kv head), new_k / new_v
+ * [B, Hkv, 1, D] contiguous in in_dtype (f16 or bf16, 16-byte aligned), is
+ * quantized into cache row L_old exactly as qkv_quantize_update(.., Lnew = 1,
+ * offset = L_old) would write it, and out is qsdpa_decode over the
+ * L_old + 1 keys [0, L_old] that then hold.  Requires L_old + 1 <= Lcap.
+ * Same workspace rules, launches and accuracy as qsdpa_decode; the cache row
+ * is written by the decode kernel, so it must not be read by another kernel
+ * that runs concurrently on the GPU. */
+qkv_status qsdpa_decode_update(const void* q, int q_dtype, const void* new_k, const void* new_v,
+                               int in_dtype, int B, int Hq, int Hkv, int D, const qkv_cache* k,
+                               const qkv_cache* v, int64_t L_old, float scale,
+                               const qkv_mask* mask, void* out, int out_dtype, void* workspace,
+                               size_t workspace_bytes, void* stream);
+
 /* Multi-query attention (any Lq >= 1) over keys [0, L) with an optional mask
  * (the pages' Lq > 1 fallback: quantized_matmul -> softmax -> quantized_matmul,
  * computed here in one fused pass).  q/out: [B, Hq, Lq, D] contiguous.

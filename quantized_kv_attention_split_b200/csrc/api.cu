@@ -82,10 +82,13 @@ qkv_status check_dtype(const char* name, int dt, bool allow_f32) {
   return fail(QKV_ERR_INVALID_ARG, "%s: unsupported dtype %d", name, dt);
 }
 
+// new_k / new_v (non-null only for Lq == 1): fused update -- the new token
+// is quantized into cache row L - 1 by the decode kernel itself.
 qkv_status attention(const void* q, int q_dtype, int B, int Hq, int Hkv, int Lq, int D,
                      const qkv_cache* k, const qkv_cache* v, int64_t L, float scale,
                      const qkv_mask* mask, void* out, int out_dtype, void* workspace,
-                     size_t workspace_bytes, void* stream) {
+                     size_t workspace_bytes, void* stream, const void* new_k = nullptr,
+                     const void* new_v = nullptr, int in_dtype = QKV_F16) {
   qkv_status st;
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Lq <= 0)
     return fail(QKV_ERR_INVALID_ARG, "B, Hq, Hkv and Lq must be positive");
@@ -153,7 +156,8 @@ qkv_status attention(const void* q, int q_dtype, int B, int Hq, int Hkv, int Lq,
     return ok();
   }
   qkv::DecodePlan plan;
-  if (!qkv::plan_decode(D, k->bits, k->group_size, k->fmt, out_dtype == QKV_F32, B,
+  const bool fused = new_k != nullptr;
+  if (!qkv::plan_decode(D, k->bits, k->group_size, k->fmt, out_dtype == QKV_F32, fused, B,
                         Hkv * rows, Hkv, L, &plan))
     return fail(QKV_ERR_UNSUPPORTED, "no kernel for D=%d bits=%d group_size=%d", D, k->bits,
                 k->group_size);
@@ -177,6 +181,11 @@ qkv_status attention(const void* q, int q_dtype, int B, int Hq, int Hkv, int Lq,
     p.msb = mask->stride_b; p.msh = mask->stride_h; p.msq = mask->stride_q;
   }
   if (mkind == QKV_MASK_CAUSAL && Lq == 1) p.mask_kind = QKV_MASK_NONE;  // all keys visible
+  if (fused) {
+    p.new_k = static_cast<const uint16_t*>(new_k);
+    p.new_v = static_cast<const uint16_t*>(new_v);
+    p.new_bf16 = in_dtype == QKV_BF16;
+  }
   uint8_t* parts = static_cast<uint8_t*>(workspace) + plan.ws_header;
   p.part_o = reinterpret_cast<float*>(parts);
   p.part_ml = reinterpret_cast<float*>(parts + plan.ws_part_o);
@@ -246,6 +255,26 @@ qkv_status qsdpa_decode(const void* q, int q_dtype, int B, int Hq, int Hkv, int 
                         size_t workspace_bytes, void* stream) {
   return attention(q, q_dtype, B, Hq, Hkv, 1, D, k, v, L, scale, mask, out, out_dtype, workspace,
                    workspace_bytes, stream);
+}
+
+qkv_status qsdpa_decode_update(const void* q, int q_dtype, const void* new_k, const void* new_v,
+                               int in_dtype, int B, int Hq, int Hkv, int D, const qkv_cache* k,
+                               const qkv_cache* v, int64_t L_old, float scale,
+                               const qkv_mask* mask, void* out, int out_dtype, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  qkv_status st;
+  if ((st = check_cache("k", k, D)) != QKV_OK) return st;
+  if ((st = check_cache("v", v, D)) != QKV_OK) return st;
+  if (in_dtype != QKV_F16 && in_dtype != QKV_BF16)
+    return fail(QKV_ERR_INVALID_ARG, "new tokens must be f16 or bf16 (got %d)", in_dtype);
+  if (new_k == nullptr || new_v == nullptr)
+    return fail(QKV_ERR_INVALID_ARG, "new_k and new_v must be non-NULL");
+  if (!aligned16(new_k) || !aligned16(new_v))
+    return fail(QKV_ERR_ALIGNMENT, "new_k and new_v must be 16-byte aligned");
+  if (L_old < 0 || L_old + 1 > k->Lcap || L_old + 1 > v->Lcap)
+    return fail(QKV_ERR_INVALID_ARG, "L_old=%lld: the new token does not fit Lcap", (long long)L_old);
+  return attention(q, q_dtype, B, Hq, Hkv, 1, D, k, v, L_old + 1, scale, mask, out, out_dtype,
+                   workspace, workspace_bytes, stream, new_k, new_v, in_dtype);
 }
 
 qkv_status qsdpa_prefill(const void* q, int q_dtype, int B, int Hq, int Hkv, int Lq, int D,

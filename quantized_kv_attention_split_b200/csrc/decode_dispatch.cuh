@@ -9,13 +9,13 @@
 namespace qkv {
 
 // Host-side helpers for one instance.
-template <int D, int BITS, int GS, bool Q8, int NC, bool F32OUT>
+template <int D, int BITS, int GS, bool Q8, int NC, bool F32OUT, bool FUSED>
 struct DecodeInstance {
   using C = DecCfg<D, BITS, GS, Q8, NC>;
   static int max_ctas_per_sm() {
     static int cached = -1;
     if (cached < 0) {
-      auto k = qsdpa_decode_kernel<D, BITS, GS, Q8, NC, F32OUT>;
+      auto k = qsdpa_decode_kernel<D, BITS, GS, Q8, NC, F32OUT, FUSED>;
       if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
         return 0;
       int n = 0;
@@ -38,7 +38,7 @@ struct DecodeInstance {
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, qsdpa_decode_kernel<D, BITS, GS, Q8, NC, F32OUT>, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, qsdpa_decode_kernel<D, BITS, GS, Q8, NC, F32OUT, FUSED>, p);
     if (e != cudaSuccess || !plan.merge) return e;
     // parts per unit: at most the CTAs that share one unit
     const int64_t parts = plan.pieces > 0 ? plan.pieces : (plan.grid + plan.units - 1) / plan.units + 1;
@@ -62,24 +62,31 @@ struct DecodeOps {
   size_t smem;
 };
 
-template <int D, int BITS, int GS, bool Q8, int NC, bool F32>
+template <int D, int BITS, int GS, bool Q8, int NC, bool F32, bool FUSED>
 DecodeOps make_decode_ops() {
-  using I = DecodeInstance<D, BITS, GS, Q8, NC, F32>;
+  using I = DecodeInstance<D, BITS, GS, Q8, NC, F32, FUSED>;
   return DecodeOps{&I::max_ctas_per_sm, &I::launch, I::C::TK, NC, I::C::NTEAM, (size_t)I::C::SMEM};
 }
 
-// Instances of one head dimension; nc in {1, 2, 4}; f32 selects the
-// split-precision value operand used for fp32 output.
+// The four variants of one format and chunking: f32 selects the
+// split-precision value operand used for fp32 output, fused the kernel that
+// also quantizes the new token into the cache.
+template <int D, int BITS, int GS, bool Q8, int NC>
+DecodeOps pick_decode_ops(bool f32, bool fused) {
+  if (fused) return f32 ? make_decode_ops<D, BITS, GS, Q8, NC, true, true>()
+                        : make_decode_ops<D, BITS, GS, Q8, NC, false, true>();
+  return f32 ? make_decode_ops<D, BITS, GS, Q8, NC, true, false>()
+             : make_decode_ops<D, BITS, GS, Q8, NC, false, false>();
+}
+
+// Instances of one head dimension; nc in {1, 2, 4}.
 template <int D>
-bool decode_ops_for(int bits, int gs, bool q8, int nc, bool f32, DecodeOps* ops) {
+bool decode_ops_for(int bits, int gs, bool q8, int nc, bool f32, bool fused, DecodeOps* ops) {
 #define QKV_DEC_NC(BITS, GS, Q8)                                                   \
   do {                                                                             \
-    if (nc == 1) { *ops = f32 ? make_decode_ops<D, BITS, GS, Q8, 1, true>()        \
-                              : make_decode_ops<D, BITS, GS, Q8, 1, false>(); }    \
-    else if (nc == 2) { *ops = f32 ? make_decode_ops<D, BITS, GS, Q8, 2, true>()   \
-                                   : make_decode_ops<D, BITS, GS, Q8, 2, false>(); } \
-    else { *ops = f32 ? make_decode_ops<D, BITS, GS, Q8, 4, true>()                \
-                      : make_decode_ops<D, BITS, GS, Q8, 4, false>(); }            \
+    if (nc == 1) *ops = pick_decode_ops<D, BITS, GS, Q8, 1>(f32, fused);           \
+    else if (nc == 2) *ops = pick_decode_ops<D, BITS, GS, Q8, 2>(f32, fused);      \
+    else *ops = pick_decode_ops<D, BITS, GS, Q8, 4>(f32, fused);                   \
     return true;                                                                   \
   } while (0)
   if (q8) {
@@ -98,8 +105,8 @@ bool decode_ops_for(int bits, int gs, bool q8, int nc, bool f32, DecodeOps* ops)
   return false;
 }
 
-bool decode_ops_d64(int bits, int gs, bool q8, int nc, bool f32, DecodeOps* ops);
-bool decode_ops_d128(int bits, int gs, bool q8, int nc, bool f32, DecodeOps* ops);
-bool decode_ops_d256(int bits, int gs, bool q8, int nc, bool f32, DecodeOps* ops);
+bool decode_ops_d64(int bits, int gs, bool q8, int nc, bool f32, bool fused, DecodeOps* ops);
+bool decode_ops_d128(int bits, int gs, bool q8, int nc, bool f32, bool fused, DecodeOps* ops);
+bool decode_ops_d256(int bits, int gs, bool q8, int nc, bool f32, bool fused, DecodeOps* ops);
 
 }  // namespace qkv

@@ -43,6 +43,7 @@
 
 #include "qkv_common.cuh"
 #include "qkv_internal.h"
+#include "quantize_core.cuh"
 
 namespace qkv {
 
@@ -151,7 +152,10 @@ struct DecCfg {
   static constexpr int WSW = 8 * D + 16;               // floats per warp
   static constexpr int EPI_W = NWARP * WSW * 4;
   static constexpr int EPI = EPI_W + NC * 8 * (NTEAM + 1) * 4 + NC * 8 * 2 * 4;
-  static constexpr int SMEM = QOFF + QSB > EPI ? QOFF + QSB : EPI;
+  // fused update: the new token's quantized K and V rows and metadata
+  static constexpr int NEWB = r16(2 * RB + NMETA * MROW);
+  static constexpr int NEWOFF = QOFF + QSB;
+  static constexpr int SMEM = NEWOFF + NEWB > EPI ? NEWOFF + NEWB : EPI;
   static_assert(NSTAGE >= 3, "at least three stages per team");
   static_assert(SMEM <= BUDGET, "shared memory budget");
   static_assert(META_UNITS * 16 == BK * MROW, "metadata rows must fill 16-byte units");
@@ -239,7 +243,7 @@ __device__ __forceinline__ void meta_row(const uint8_t* base, int r, uint32_t* w
   }
 }
 
-template <int D, int BITS, int GS, bool Q8, int NC, bool F32OUT>
+template <int D, int BITS, int GS, bool Q8, int NC, bool F32OUT, bool FUSED>
 __global__ void __launch_bounds__(32 * dec_warps(D), 1)
 qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
   using C = DecCfg<D, BITS, GS, Q8, NC>;
@@ -404,6 +408,60 @@ qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
     // stream has completed (this launch may start early, overlapping its
     // set-up with that kernel's tail).
     grid_dep_wait();
+    // Fused update: the CTA whose segment holds the unit's last block (key
+    // L - 1, the new token) quantizes the new K and V rows of its kv head with
+    // the quantizer's own arithmetic, writes them to the cache and keeps a copy
+    // for the team that gets that block (its copy of the row may predate the
+    // write).  Warp 0: lanes [0, D/32) take K's 32-element slices, the next
+    // D/32 lanes V's.
+    const bool newtok = FUSED && s1 == (int)S;
+    uint8_t* const s_new = smem + C::NEWOFF;
+    if constexpr (FUSED) if (newtok && warp == 0) {
+      constexpr int SL = D / kQEpt;
+      const bool isv = lane >= SL, act = lane < 2 * SL;
+      const int cs = isv ? lane - SL : lane;
+      uint32_t w[kQWords];
+#pragma unroll
+      for (int i = 0; i < kQWords; ++i) w[i] = 0u;
+      if (act) {
+        const uint4* src = reinterpret_cast<const uint4*>((isv ? p.new_v : p.new_k) + uh * D + cs * kQEpt);
+#pragma unroll
+        for (int k = 0; k < kQWords / 4; ++k) {
+          const uint4 r = __ldg(src + k);
+          w[4 * k] = r.x; w[4 * k + 1] = r.y; w[4 * k + 2] = r.z; w[4 * k + 3] = r.w;
+        }
+      }
+      constexpr int OW = kQEpt * BITS / 32;                // code words of a slice
+      uint32_t o[OW];
+      uint16_t sbits, bbits;
+      if (p.new_bf16) quantize_slice<GS, BITS, Q8, true>(w, o, sbits, bbits);
+      else quantize_slice<GS, BITS, Q8, false>(w, o, sbits, bbits);
+      if (act) {
+        const int64_t crow = row0 + L - 1;                   // cache row of the new token
+        uint32_t* codes = const_cast<uint32_t*>(reinterpret_cast<const uint32_t*>(isv ? p.vc : p.kc));
+        uint4* dst = reinterpret_cast<uint4*>(codes + crow * (C::RB / 4) + cs * OW);
+        uint4* cpy = reinterpret_cast<uint4*>(s_new + isv * C::RB + cs * OW * 4);
+#pragma unroll
+        for (int k = 0; k < OW / 4; ++k) {
+          dst[k] = make_uint4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
+          cpy[k] = make_uint4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
+        }
+        if ((cs * kQEpt) % GS == 0) {
+          // metadata arrays in stage order: affine K scales, K biases, V
+          // scales, V biases; Q8_0 K scales, V scales
+          const int gq = (cs * kQEpt) / GS;
+          uint16_t* meta = reinterpret_cast<uint16_t*>(s_new + 2 * C::RB);
+          uint16_t* sc = const_cast<uint16_t*>(isv ? p.vs : p.ks);
+          sc[crow * NG + gq] = sbits;
+          meta[(Q8 ? isv : 2 * isv) * NG + gq] = sbits;
+          if constexpr (!Q8) {
+            uint16_t* bi = const_cast<uint16_t*>(isv ? p.vb : p.kb);
+            bi[crow * NG + gq] = bbits;
+            meta[(2 * isv + 1) * NG + gq] = bbits;
+          }
+        }
+      }
+    }
     uint4 qraw[QPT];
     {
       const int64_t qbase = (uh * p.G + hbase) * D;
@@ -537,6 +595,23 @@ qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
       }
       const int64_t key0 = (int64_t)(s0 + cur) * BK;
       const int kvalid = (int)(L - key0 < (int64_t)BK ? L - key0 : (int64_t)BK);   // valid keys of this block
+      if (FUSED && newtok && key0 + kvalid == L) {
+        // the block of the new token: its row takes the freshly quantized codes
+        const int r = kvalid - 1;
+        for (int i = ttid; i < 2 * C::UPR; i += TTHR) {
+          const int which = i >= C::UPR, u = which ? i - C::UPR : i;
+          const uint4 v = *reinterpret_cast<const uint4*>(s_new + which * C::RB + u * 16);
+          const int off = which ? C::CODES + swz_xor<C::SWZV>(r * C::RB + u * 16)
+                                : swz_xor<C::SWZ>(r * C::RB + u * 16);
+          *reinterpret_cast<uint4*>(sb + off) = v;
+        }
+        for (int i = ttid; i < C::NMETA * NG; i += TTHR) {
+          const int arr = i / NG, gq = i - arr * NG;
+          reinterpret_cast<uint16_t*>(sb + 2 * C::CODES + arr * C::META)[r * NG + gq] =
+              reinterpret_cast<const uint16_t*>(s_new + 2 * C::RB)[i];
+        }
+        team_sync();
+      }
       const uint8_t* sK = sb;
       const uint8_t* sV = sb + C::CODES;
       const uint8_t* sMeta = sb + 2 * C::CODES;

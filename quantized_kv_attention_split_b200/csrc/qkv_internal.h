@@ -40,6 +40,11 @@ struct DecodeParams {
   int64_t stages_per_unit;
   int64_t total_stages;
   int pieces;               // CTAs per unit when every CTA covers one piece of one unit, else 0
+  // fused update: the new token of every (batch, kv head), [B * Hkv, D]
+  // fp16/bf16 bits, is quantized into cache row L - 1 (null: plain decode)
+  const uint16_t* new_k;
+  const uint16_t* new_v;
+  int new_bf16;
   float* part_o;            // [2 * nCTA][HPC][D]   per-CTA partials
   float* part_ml;           // [2 * nCTA][HPC][2]
 };
@@ -53,6 +58,7 @@ struct DecodePlan {
   int64_t stages_per_unit;
   int64_t total_stages;
   int grid;
+  bool fused;               // the kernel also quantizes the new token (row L - 1)
   int pieces;               // CTAs per unit when the grid cuts every unit alike, else 0
   bool merge;               // some unit is split over several CTAs: merge kernel after
   size_t smem;
@@ -64,8 +70,8 @@ struct DecodePlan {
 
 // Plans a decode launch for the current device; returns false if the shape
 // has no kernel instance.
-bool plan_decode(int D, int bits, int gs, int fmt, int out_f32, int B, int Hq, int Hkv,
-                 int64_t L, DecodePlan* plan);
+bool plan_decode(int D, int bits, int gs, int fmt, int out_f32, bool fused, int B, int Hq,
+                 int Hkv, int64_t L, DecodePlan* plan);
 cudaError_t launch_decode(int D, int bits, int gs, int fmt, int out_f32,
                           const DecodePlan& plan, DecodeParams& p, cudaStream_t stream);
 

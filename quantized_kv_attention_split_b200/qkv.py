@@ -67,6 +67,9 @@ def lib() -> C.CDLL:
         L.qsdpa_prefill.argtypes = [p, i32, i32, i32, i32, i32, i32, cp, cp, i64, C.c_float, mp,
                                     p, i32, p, sz, p]
         L.qsdpa_prefill.restype = i32
+        L.qsdpa_decode_update.argtypes = [p, i32, p, p, i32, i32, i32, i32, i32, cp, cp, i64,
+                                          C.c_float, mp, p, i32, p, sz, p]
+        L.qsdpa_decode_update.restype = i32
         L.qsdpa_workspace_size.argtypes = [i32, i32, i32, i32, i32, i64]
         L.qsdpa_workspace_size.restype = sz
         L.qsdpa_workspace_zero_bytes.argtypes = [i32, i32, i32, i32, i32, i64]
@@ -190,6 +193,33 @@ def qsdpa_decode(q: torch.Tensor, k: QuantCache, v: QuantCache, L: int, scale: f
     assert q.shape[2] == 1
     return _attention(lib().qsdpa_decode, q, k, v, L, scale, mask, False, out, out_dtype,
                       workspace, stream, True)
+
+
+def qsdpa_decode_update(q: torch.Tensor, new_k: torch.Tensor, new_v: torch.Tensor,
+                        k: QuantCache, v: QuantCache, L_old: int, scale: float, mask=None,
+                        out: Optional[torch.Tensor] = None, out_dtype=None,
+                        workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """One fused decode step: quantize new_k/new_v [B,Hkv,1,D] (f16/bf16) into
+    cache row L_old, in place, and return softmax(q*scale . K^T + mask) V for
+    q [B,Hq,1,D] over the L_old + 1 keys [0, L_old]."""
+    assert q.is_contiguous() and q.is_cuda and q.shape[2] == 1
+    assert new_k.is_contiguous() and new_v.is_contiguous()
+    assert new_k.shape == new_v.shape and new_k.dtype == new_v.dtype and new_k.shape[2] == 1
+    B, Hq, _, D = q.shape
+    Hkv = k.codes.shape[1]
+    if out is None:
+        out = torch.empty(B, Hq, 1, D, dtype=out_dtype or q.dtype, device=q.device)
+    if workspace is None:
+        workspace = make_workspace(B, Hq, Hkv, 1, D, L_old + 1, q.device)
+    ks, vs = k._struct(), v._struct()
+    m = _mask_struct(mask, False)
+    mp = C.byref(m) if m is not None else None
+    _check(lib().qsdpa_decode_update(q.data_ptr(), _DTYPE[q.dtype], new_k.data_ptr(),
+                                     new_v.data_ptr(), _DTYPE[new_k.dtype], B, Hq, Hkv, D,
+                                     C.byref(ks), C.byref(vs), int(L_old), float(scale), mp,
+                                     out.data_ptr(), _DTYPE[out.dtype], workspace.data_ptr(),
+                                     workspace.numel(), _stream(stream)))
+    return out
 
 
 def qsdpa_prefill(q: torch.Tensor, k: QuantCache, v: QuantCache, L: int, scale: float,
