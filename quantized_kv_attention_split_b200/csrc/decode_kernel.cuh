@@ -134,7 +134,9 @@ struct DecCfg {
   static constexpr int stage_bytes(int sub) { return r128(2 * 16 * sub * RB + NMETA * r16(16 * sub * MROW)); }
   // 16-key sub-blocks per block: two when three such stages per team fit
   // (D = 256 keeps one: its register budget is spent)
-  static constexpr int SUB = (D <= 128 && NTEAM * 3 * stage_bytes(2) + QSB <= BUDGET) ? 2 : 1;
+  // fused update: the new token's raw K and V rows (16-bit inputs)
+  static constexpr int NEWB = 4 * D;
+  static constexpr int SUB = (D <= 128 && NTEAM * 3 * stage_bytes(2) + QSB + NEWB <= BUDGET) ? 2 : 1;
   static constexpr int BK = 16 * SUB;          // keys per block
   static constexpr int TK = BK;
   static constexpr int CODES = BK * RB;
@@ -143,7 +145,7 @@ struct DecCfg {
   static constexpr int KU = BK * UPR;          // 16-byte code units per tile
   static constexpr int MU = NMETA * META_UNITS;
   static constexpr int STAGE = stage_bytes(SUB);
-  static constexpr int NS_FIT = (BUDGET - QSB) / (NTEAM * STAGE);
+  static constexpr int NS_FIT = (BUDGET - QSB - NEWB) / (NTEAM * STAGE);
   static constexpr int NSTAGE = NS_FIT > 6 ? 6 : NS_FIT;
   static constexpr int TRING = NSTAGE * STAGE;          // one team's ring
   static constexpr int QOFF = NTEAM * TRING;            // query rows after the rings
@@ -152,8 +154,6 @@ struct DecCfg {
   static constexpr int WSW = 8 * D + 16;               // floats per warp
   static constexpr int EPI_W = NWARP * WSW * 4;
   static constexpr int EPI = EPI_W + NC * 8 * (NTEAM + 1) * 4 + NC * 8 * 2 * 4;
-  // fused update: the new token's quantized K and V rows and metadata
-  static constexpr int NEWB = r16(2 * RB + NMETA * MROW);
   static constexpr int NEWOFF = QOFF + QSB;
   static constexpr int SMEM = NEWOFF + NEWB > EPI ? NEWOFF + NEWB : EPI;
   static_assert(NSTAGE >= 3, "at least three stages per team");
@@ -243,6 +243,58 @@ __device__ __forceinline__ void meta_row(const uint8_t* base, int r, uint32_t* w
   }
 }
 
+// Fused update, by one warp of the team that got the block of key L - 1:
+// quantize the new token's K and V rows (raw 16-bit values staged at s_new)
+// with the quantizer's arithmetic -- lanes [0, D/32) take K's 32-element
+// slices, the next D/32 lanes V's -- write codes and metadata to cache row
+// crow and into row r of the staged block at sb.  Out of line: it runs once
+// per unit and keeps its registers out of the main loop.
+template <int D, int BITS, int GS, bool Q8>
+__device__ __noinline__ void fused_quantize_patch(const DecodeParams& p, const uint8_t* s_new,
+                                                  uint8_t* sb, int64_t crow, int r, int lane) {
+  using C = DecCfg<D, BITS, GS, Q8, 1>;
+  constexpr int NG = C::NG;
+  constexpr int SL = D / kQEpt;
+  constexpr int OW = kQEpt * BITS / 32;                // code words of a slice
+  const bool isv = lane >= SL, act = lane < 2 * SL;
+  const int cs = isv ? lane - SL : lane;
+  uint32_t w[kQWords];
+#pragma unroll
+  for (int k = 0; k < kQWords / 4; ++k) {
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (act) v = *reinterpret_cast<const uint4*>(s_new + isv * 2 * D + cs * 64 + k * 16);
+    w[4 * k] = v.x; w[4 * k + 1] = v.y; w[4 * k + 2] = v.z; w[4 * k + 3] = v.w;
+  }
+  uint32_t o[OW];
+  uint16_t sbits, bbits;
+  if (p.new_bf16) quantize_slice<GS, BITS, Q8, true>(w, o, sbits, bbits);
+  else quantize_slice<GS, BITS, Q8, false>(w, o, sbits, bbits);
+  if (!act) return;
+  uint32_t* codes = const_cast<uint32_t*>(reinterpret_cast<const uint32_t*>(isv ? p.vc : p.kc));
+  uint4* dst = reinterpret_cast<uint4*>(codes + crow * (C::RB / 4) + cs * OW);
+#pragma unroll
+  for (int k = 0; k < OW / 4; ++k) {
+    const uint4 v = make_uint4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
+    dst[k] = v;
+    // the slice's 16-byte units in the staged (swizzled) row
+    const int lin = r * C::RB + cs * OW * 4 + k * 16;
+    *reinterpret_cast<uint4*>(sb + (isv ? C::CODES + swz_xor<C::SWZV>(lin) : swz_xor<C::SWZ>(lin))) = v;
+  }
+  if ((cs * kQEpt) % GS == 0) {
+    // metadata arrays in stage order: affine K scales, K biases, V scales, V
+    // biases; Q8_0 K scales, V scales
+    const int gq = (cs * kQEpt) / GS;
+    uint16_t* sc = const_cast<uint16_t*>(isv ? p.vs : p.ks);
+    sc[crow * NG + gq] = sbits;
+    reinterpret_cast<uint16_t*>(sb + 2 * C::CODES + (Q8 ? isv : 2 * isv) * C::META)[r * NG + gq] = sbits;
+    if constexpr (!Q8) {
+      uint16_t* bi = const_cast<uint16_t*>(isv ? p.vb : p.kb);
+      bi[crow * NG + gq] = bbits;
+      reinterpret_cast<uint16_t*>(sb + 2 * C::CODES + (2 * isv + 1) * C::META)[r * NG + gq] = bbits;
+    }
+  }
+}
+
 template <int D, int BITS, int GS, bool Q8, int NC, bool F32OUT, bool FUSED>
 __global__ void __launch_bounds__(32 * dec_warps(D), 1)
 qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
@@ -299,6 +351,13 @@ qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
     const int hbase = cg * HPC;                                  // first local row of the CTA
 
     const int64_t L = p.L;
+    // Fused update: the segment that holds the unit's last block (key L - 1,
+    // the new token) has the team that gets that block fetch the new K and V
+    // rows with the block's copies, quantize them with the quantizer's own
+    // arithmetic, write them to the cache and patch its staged copy of the row
+    // (which may predate that write); see fused_quantize_patch.
+    const bool newtok = FUSED && s1 == (int)S;
+    uint8_t* const s_new = smem + C::NEWOFF;
 
     // Copy plan of one block (by its team): 16-byte unit i is row i / UPR of
     // the K tile (i < KU) or of the V tile, then the metadata arrays.  Unit
@@ -353,6 +412,16 @@ qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
         }
       }
       // metadata: affine K scales, K biases, V scales, V biases; Q8_0 K and V scales
+      if constexpr (FUSED) {
+        if (newtok && blk == nblk - 1) {
+          // the new token's raw K and V rows (D 16-bit values each), 4D bytes
+          for (int i = ttid; i < D / 4; i += TTHR) {
+            const int isv = i >= D / 8, j = isv ? i - D / 8 : i;
+            cp_async16(smem_u32(s_new) + i * 16,
+                       reinterpret_cast<const uint8_t*>((isv ? p.new_v : p.new_k) + uh * D) + j * 16, 16);
+          }
+        }
+      }
       if constexpr (C::MU <= TTHR) {
         // one unit per lane: its array and offset were chosen once (mlane)
         if (C::MU == TTHR || ttid < C::MU) {
@@ -408,60 +477,6 @@ qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
     // stream has completed (this launch may start early, overlapping its
     // set-up with that kernel's tail).
     grid_dep_wait();
-    // Fused update: the CTA whose segment holds the unit's last block (key
-    // L - 1, the new token) quantizes the new K and V rows of its kv head with
-    // the quantizer's own arithmetic, writes them to the cache and keeps a copy
-    // for the team that gets that block (its copy of the row may predate the
-    // write).  Warp 0: lanes [0, D/32) take K's 32-element slices, the next
-    // D/32 lanes V's.
-    const bool newtok = FUSED && s1 == (int)S;
-    uint8_t* const s_new = smem + C::NEWOFF;
-    if constexpr (FUSED) if (newtok && warp == 0) {
-      constexpr int SL = D / kQEpt;
-      const bool isv = lane >= SL, act = lane < 2 * SL;
-      const int cs = isv ? lane - SL : lane;
-      uint32_t w[kQWords];
-#pragma unroll
-      for (int i = 0; i < kQWords; ++i) w[i] = 0u;
-      if (act) {
-        const uint4* src = reinterpret_cast<const uint4*>((isv ? p.new_v : p.new_k) + uh * D + cs * kQEpt);
-#pragma unroll
-        for (int k = 0; k < kQWords / 4; ++k) {
-          const uint4 r = __ldg(src + k);
-          w[4 * k] = r.x; w[4 * k + 1] = r.y; w[4 * k + 2] = r.z; w[4 * k + 3] = r.w;
-        }
-      }
-      constexpr int OW = kQEpt * BITS / 32;                // code words of a slice
-      uint32_t o[OW];
-      uint16_t sbits, bbits;
-      if (p.new_bf16) quantize_slice<GS, BITS, Q8, true>(w, o, sbits, bbits);
-      else quantize_slice<GS, BITS, Q8, false>(w, o, sbits, bbits);
-      if (act) {
-        const int64_t crow = row0 + L - 1;                   // cache row of the new token
-        uint32_t* codes = const_cast<uint32_t*>(reinterpret_cast<const uint32_t*>(isv ? p.vc : p.kc));
-        uint4* dst = reinterpret_cast<uint4*>(codes + crow * (C::RB / 4) + cs * OW);
-        uint4* cpy = reinterpret_cast<uint4*>(s_new + isv * C::RB + cs * OW * 4);
-#pragma unroll
-        for (int k = 0; k < OW / 4; ++k) {
-          dst[k] = make_uint4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
-          cpy[k] = make_uint4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
-        }
-        if ((cs * kQEpt) % GS == 0) {
-          // metadata arrays in stage order: affine K scales, K biases, V
-          // scales, V biases; Q8_0 K scales, V scales
-          const int gq = (cs * kQEpt) / GS;
-          uint16_t* meta = reinterpret_cast<uint16_t*>(s_new + 2 * C::RB);
-          uint16_t* sc = const_cast<uint16_t*>(isv ? p.vs : p.ks);
-          sc[crow * NG + gq] = sbits;
-          meta[(Q8 ? isv : 2 * isv) * NG + gq] = sbits;
-          if constexpr (!Q8) {
-            uint16_t* bi = const_cast<uint16_t*>(isv ? p.vb : p.kb);
-            bi[crow * NG + gq] = bbits;
-            meta[(2 * isv + 1) * NG + gq] = bbits;
-          }
-        }
-      }
-    }
     uint4 qraw[QPT];
     {
       const int64_t qbase = (uh * p.G + hbase) * D;
@@ -595,22 +610,12 @@ qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
       }
       const int64_t key0 = (int64_t)(s0 + cur) * BK;
       const int kvalid = (int)(L - key0 < (int64_t)BK ? L - key0 : (int64_t)BK);   // valid keys of this block
-      if (FUSED && newtok && key0 + kvalid == L) {
-        // the block of the new token: its row takes the freshly quantized codes
-        const int r = kvalid - 1;
-        for (int i = ttid; i < 2 * C::UPR; i += TTHR) {
-          const int which = i >= C::UPR, u = which ? i - C::UPR : i;
-          const uint4 v = *reinterpret_cast<const uint4*>(s_new + which * C::RB + u * 16);
-          const int off = which ? C::CODES + swz_xor<C::SWZV>(r * C::RB + u * 16)
-                                : swz_xor<C::SWZ>(r * C::RB + u * 16);
-          *reinterpret_cast<uint4*>(sb + off) = v;
+      if constexpr (FUSED) {
+        if (newtok && key0 + kvalid == L) {
+          if (chunk == 0)
+            fused_quantize_patch<D, BITS, GS, Q8>(p, s_new, sb, row0 + L - 1, kvalid - 1, lane);
+          team_sync();
         }
-        for (int i = ttid; i < C::NMETA * NG; i += TTHR) {
-          const int arr = i / NG, gq = i - arr * NG;
-          reinterpret_cast<uint16_t*>(sb + 2 * C::CODES + arr * C::META)[r * NG + gq] =
-              reinterpret_cast<const uint16_t*>(s_new + 2 * C::RB)[i];
-        }
-        team_sync();
       }
       const uint8_t* sK = sb;
       const uint8_t* sV = sb + C::CODES;
