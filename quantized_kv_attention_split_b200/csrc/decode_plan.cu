@@ -15,6 +15,10 @@ constexpr int64_t kMaxGrid = 8 * 48;
 // Partials of at least this many floats count as large (16 rows x D = 256 do).
 constexpr int64_t kBigPartial = 2048;
 constexpr int64_t kBigPartMinStages = 2;   // blocks per team
+// With large partials, at most this many CTAs share a unit: the merge reads
+// every partial, and beyond this the longer merge costs more than the shorter
+// loop gains (Q8_0, D = 256, 16 rows, 10K and 20K keys: best at 48 of 24..74).
+constexpr int64_t kBigPartMaxPieces = 48;
 
 int sm_count() {
   int dev = 0, n = 0;
@@ -105,9 +109,14 @@ bool plan_decode(int D, int bits, int gs, int fmt, int out_f32, bool fused, int 
   // and epilogue), as long as that leaves at most 15% of the grid idle; no
   // more pieces than give every team a block (short caches: fewer partials).
   if (plan->units <= grid) {
-    const int64_t per_unit = std::min<int64_t>(grid / plan->units,
-                                               (plan->stages_per_unit + ops.teams - 1) / ops.teams);
-    if (per_unit * plan->units * 100 >= grid * 85 || per_unit * ops.teams >= plan->stages_per_unit)
+    int64_t per_unit = std::min<int64_t>(grid / plan->units,
+                                         (plan->stages_per_unit + ops.teams - 1) / ops.teams);
+    bool capped = false;
+    if ((int64_t)plan->hpc * D >= kBigPartial && per_unit > kBigPartMaxPieces) {
+      per_unit = kBigPartMaxPieces;
+      capped = true;
+    }
+    if (capped || per_unit * plan->units * 100 >= grid * 85 || per_unit * ops.teams >= plan->stages_per_unit)
       grid = std::max<int64_t>(1, per_unit) * plan->units;
   }
   plan->grid = (int)std::max<int64_t>(1, grid);
