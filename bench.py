@@ -537,7 +537,59 @@ def other_rows(device):
                     "frac_tensor_peak": round(flop / (sec / 1e3) / 1e12 / bf16_peak, 4),
                     "flop": flop,
                     "peak_note": "fp16 operands; measured bf16 dense peak x nominal fp16:bf16 ratio 1"}
+    # A/B: materialize the cache as fp16 (qkv_dequantize), then dense attention
+    # through torch's scaled_dot_product_attention (a library kernel), against
+    # the fused prefill above
+    try:
+        from torch.nn.attention.bias import causal_lower_right
+        kd = torch.empty(w.B, w.Hkv, w.L, w.D, dtype=torch.float16, device=device)
+        vd = torch.empty_like(kd)
+        qh = q.to(torch.float16)
+        cmask = causal_lower_right(w.Lq, w.L)
+
+        def mstep(i):
+            qkv.qkv_dequantize(kc, w.L, out=kd)
+            qkv.qkv_dequantize(vc, w.L, out=vd)
+            torch.nn.functional.scaled_dot_product_attention(qh, kd, vd, attn_mask=cmask,
+                                                             scale=w.scale, enable_gqa=True)
+        sec_m, _ = graph_time(mstep, 20, 3)
+        sec_d, _ = graph_time(lambda i: (qkv.qkv_dequantize(kc, w.L, out=kd),
+                                         qkv.qkv_dequantize(vc, w.L, out=vd)), 20, 3)
+        rows["materialize_" + w.name] = {
+            "us_per_call": round(sec_m * 1e3, 2), "dequantize_us": round(sec_d * 1e3, 2),
+            "TFLOP/s": round(flop / (sec_m / 1e3) / 1e12, 1),
+            "note": "qkv_dequantize of K and V to fp16, then torch scaled_dot_product_attention "
+                    "(causal, lower-right aligned, GQA); compare prefill_q8_0_512_at_20k"}
+        del kd, vd
+    except Exception as e:                       # the library attention may be unavailable
+        rows["materialize_" + w.name] = {"unavailable": f"{type(e).__name__}: {e}"[:200]}
     del caches
+    torch.cuda.empty_cache()
+
+    # A/B for the main decode workload: materialize K and V (65536 keys), then
+    # dense attention for the one query, against the fused decode (bench value)
+    try:
+        w = S.WORKLOADS["decode_64k_affine4"]
+        inp = S.make_inputs(w)
+        kc, vc = build_caches(w, inp, 1, device)[0]
+        q = dev16(inp.q, "f16", device)
+        kd = torch.empty(w.B, w.Hkv, w.L, w.D, dtype=torch.float16, device=device)
+        vd = torch.empty_like(kd)
+
+        def dstep2(i):
+            qkv.qkv_dequantize(kc, w.L, out=kd)
+            qkv.qkv_dequantize(vc, w.L, out=vd)
+            torch.nn.functional.scaled_dot_product_attention(q, kd, vd, scale=w.scale,
+                                                             enable_gqa=True)
+        sec_m, _ = graph_time(dstep2, 200, 10)
+        nb = w.cache_bytes() + 2 * w.Hq * w.D * 2
+        rows["materialize_" + w.name] = {
+            "us_per_call": round(sec_m * 1e3, 3), "GB/s": round(nb / (sec_m / 1e3) / 1e9, 1),
+            "note": "qkv_dequantize of K and V to fp16 (268 MB written), then torch "
+                    "scaled_dot_product_attention (GQA); compare the bench value"}
+        del kd, vd, kc, vc
+    except Exception as e:
+        rows["materialize_decode_64k_affine4"] = {"unavailable": f"{type(e).__name__}: {e}"[:200]}
     torch.cuda.empty_cache()
     return rows
 

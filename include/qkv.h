@@ -159,6 +159,16 @@ qkv_status qsdpa_prefill(const void* q, int q_dtype, int B, int Hq, int Hkv, int
                          float scale, const qkv_mask* mask, void* out, int out_dtype,
                          void* workspace, size_t workspace_bytes, void* stream);
 
+/* Rows [0, L) of one quantized cache materialized as fp16:
+ * out[b, h, j, e] = fp16(scale * code + bias) (Q8_0: scale * code), the
+ * correctly rounded value of the exact dequantization.  The prompt path of
+ * llama.cpp #25556 converts a Q8_0 cache to fp16 and runs dense attention on
+ * it; this is that conversion, for comparisons of "materialize, then dense
+ * attention" with the fused kernels.  out: [B, Hkv, L, D] contiguous fp16,
+ * 16-byte aligned, caller-owned.  One launch. */
+qkv_status qkv_dequantize(const qkv_cache* c, int B, int Hkv, int D, int64_t L, void* out,
+                          void* stream);
+
 /* Allocation-free variant of qsdpa_decode (the pages have no counterpart:
  * MLX and llama.cpp allocate their temporaries through their own allocators).
  * For callers that cannot allocate device memory when they decode -- code

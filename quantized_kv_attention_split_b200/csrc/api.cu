@@ -249,6 +249,22 @@ qkv_status qkv_quantize_update(const void* new_k, const void* new_v, int in_dtyp
   return ok();
 }
 
+qkv_status qkv_dequantize(const qkv_cache* c, int B, int Hkv, int D, int64_t L, void* out,
+                          void* stream) {
+  qkv_status st;
+  if ((st = check_cache("cache", c, D)) != QKV_OK) return st;
+  if (B <= 0 || Hkv <= 0) return fail(QKV_ERR_INVALID_ARG, "B and Hkv must be positive");
+  if ((int64_t)B * Hkv > 65535)
+    return fail(QKV_ERR_UNSUPPORTED, "B * Hkv must be at most 65535 (got %lld)", (long long)B * Hkv);
+  if (L < 0 || L > c->Lcap) return fail(QKV_ERR_INVALID_ARG, "L=%lld outside [0, Lcap]", (long long)L);
+  if (L == 0) return ok();
+  if (out == nullptr) return fail(QKV_ERR_INVALID_ARG, "out must be non-NULL");
+  if (!aligned16(out)) return fail(QKV_ERR_ALIGNMENT, "out must be 16-byte aligned");
+  cudaError_t e = qkv::launch_dequantize(c, B, Hkv, D, L, out, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(QKV_ERR_CUDA, "dequantize launch: %s", cudaGetErrorString(e));
+  return ok();
+}
+
 qkv_status qsdpa_decode(const void* q, int q_dtype, int B, int Hq, int Hkv, int D,
                         const qkv_cache* k, const qkv_cache* v, int64_t L, float scale,
                         const qkv_mask* mask, void* out, int out_dtype, void* workspace,

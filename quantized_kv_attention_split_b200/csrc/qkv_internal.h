@@ -75,4 +75,8 @@ bool plan_decode(int D, int bits, int gs, int fmt, int out_f32, bool fused, int 
 cudaError_t launch_decode(int D, int bits, int gs, int fmt, int out_f32,
                           const DecodePlan& plan, DecodeParams& p, cudaStream_t stream);
 
+// Rows [0, L) of a cache as fp16 [B * Hkv, L, D] (dequantize.cu).
+cudaError_t launch_dequantize(const qkv_cache* c, int B, int Hkv, int D, int64_t L, void* out,
+                              cudaStream_t stream);
+
 }  // namespace qkv

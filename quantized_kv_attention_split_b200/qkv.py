@@ -70,6 +70,8 @@ def lib() -> C.CDLL:
         L.qsdpa_decode_update.argtypes = [p, i32, p, p, i32, i32, i32, i32, i32, cp, cp, i64,
                                           C.c_float, mp, p, i32, p, sz, p]
         L.qsdpa_decode_update.restype = i32
+        L.qkv_dequantize.argtypes = [cp, i32, i32, i32, i64, p, p]
+        L.qkv_dequantize.restype = i32
         L.qsdpa_workspace_size.argtypes = [i32, i32, i32, i32, i32, i64]
         L.qsdpa_workspace_size.restype = sz
         L.qsdpa_workspace_zero_bytes.argtypes = [i32, i32, i32, i32, i32, i64]
@@ -152,6 +154,20 @@ def qkv_quantize_update(new_k: torch.Tensor, new_v: torch.Tensor, k: QuantCache,
     _check(lib().qkv_quantize_update(new_k.data_ptr(), new_v.data_ptr(), _DTYPE[new_k.dtype],
                                      B, Hkv, Lnew, D, C.byref(ks), C.byref(vs), int(offset),
                                      _stream(stream)))
+
+
+def qkv_dequantize(c: QuantCache, L: int, out: Optional[torch.Tensor] = None,
+                   stream=None) -> torch.Tensor:
+    """Rows [0, L) of a cache as fp16 [B, Hkv, L, D]: the correctly rounded
+    scale * code + bias (for "materialize, then dense attention")."""
+    B, Hkv = c.codes.shape[0], c.codes.shape[1]
+    D = c.codes.shape[3] * 32 // c.bits
+    if out is None:
+        out = torch.empty(B, Hkv, L, D, dtype=torch.float16, device=c.codes.device)
+    assert out.is_contiguous() and out.dtype == torch.float16 and tuple(out.shape) == (B, Hkv, L, D)
+    cs = c._struct()
+    _check(lib().qkv_dequantize(C.byref(cs), B, Hkv, D, int(L), out.data_ptr(), _stream(stream)))
+    return out
 
 
 def _mask_struct(mask, causal: bool):
