@@ -91,3 +91,34 @@ def test_quantize_rejects_too_many_slabs(lib):
     f = lib.qkv_quantize_update
     assert f(FAKE, FAKE, 0, 65536, 1, 4, 128, C.byref(ok), C.byref(ok), 0, None) == 2
     assert b"65535" in lib.qkv_last_error()
+
+
+def test_decode_update_validation_errors(lib):
+    """The fused decode step validates the new-token arguments and the cache
+    room before any launch."""
+    from quantized_kv_attention_split_b200 import qkv
+    ok = _cache(qkv)
+    f = lib.qsdpa_decode_update
+
+    def call(nk=FAKE + 1024, nv=FAKE + 2048, idt=0, L_old=16, k=ok):
+        return f(FAKE, 0, nk, nv, idt, 1, 8, 2, 128, C.byref(k), C.byref(ok), L_old, 1.0, None,
+                 FAKE + 65536, 0, FAKE + 131072, 1 << 20, None)
+    assert call(L_old=64) == 1                     # no room for the new token (Lcap 64)
+    assert b"Lcap" in lib.qkv_last_error()
+    assert call(L_old=-1) == 1
+    assert call(idt=2) == 1                        # new tokens must be 16-bit
+    assert call(nk=0) == 1                         # NULL new_k
+    assert call(nv=FAKE + 2056) == 3               # misaligned new_v
+    assert call(k=_cache(qkv, bits=5)) == 2        # unsupported format
+
+
+def test_dequantize_validation_errors(lib):
+    from quantized_kv_attention_split_b200 import qkv
+    ok = _cache(qkv)
+    f = lib.qkv_dequantize
+    assert f(C.byref(ok), 1, 2, 128, 65, FAKE, None) == 1                    # L > Lcap
+    assert f(C.byref(ok), 1, 2, 128, 16, 0, None) == 1                       # NULL out
+    assert f(C.byref(ok), 1, 2, 128, 16, FAKE + 8, None) == 3                # misaligned out
+    assert f(C.byref(ok), 70000, 1, 128, 16, FAKE, None) == 2                # slabs > 65535
+    assert f(C.byref(_cache(qkv, gs=48)), 1, 2, 128, 16, FAKE, None) == 2    # unsupported group
+    assert f(C.byref(ok), 1, 2, 128, 0, FAKE, None) == 0                     # nothing to do
