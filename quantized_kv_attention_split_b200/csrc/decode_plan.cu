@@ -20,10 +20,16 @@ constexpr int64_t kBigPartMinStages = 2;   // blocks per team
 // loop gains (Q8_0, D = 256, 16 rows, 10K and 20K keys: best at 48 of 24..74).
 constexpr int64_t kBigPartMaxPieces = 48;
 
+// SM count of the current device, queried once per device (every decode call
+// plans its grid with it).
 int sm_count() {
+  constexpr int kMaxDevices = 64;
+  static int cached[kMaxDevices] = {};
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev >= 0 && dev < kMaxDevices && cached[dev] > 0) return cached[dev];
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (dev >= 0 && dev < kMaxDevices) cached[dev] = n;
   return n;
 }
 
