@@ -569,15 +569,15 @@ qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
     float beta[2][NG];
     float O[MT][4];
-    // Per group, the value operand carries 2^tau, with tau = 29 - the largest
+    // Per group, the value operand carries 2^tau, with tau = 21 - the largest
     // exponent field of the group's value scales seen so far, so that
-    // P * s_v * 2^tau < 2^15 for every key (P <= 1).  vbound holds those
+    // P * s_v * 2^tau < 2^15 for every key (P <= 2^8, the lazy max below).  vbound holds those
     // largest scales (magnitudes, as fp16 bits, two groups per word); tau
     // only decreases, and O is rescaled by the exact power of two when it does.
     int tau[NG];
     uint32_t vbound[MW];
 #pragma unroll
-    for (int gg = 0; gg < NG; ++gg) { beta[0][gg] = 0.f; beta[1][gg] = 0.f; tau[gg] = 29; }
+    for (int gg = 0; gg < NG; ++gg) { beta[0][gg] = 0.f; beta[1][gg] = 0.f; tau[gg] = 21; }
 #pragma unroll
     for (int w = 0; w < MW; ++w) vbound[w] = 0u;
 #pragma unroll
@@ -704,34 +704,27 @@ qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
         }
       }
 
-      // ---------------- online softmax over the warp's 32 keys -----------------
+      // ---------------- online softmax over the warp's keys ---------------------
+      // The running max moves lazily: only when a score exceeds it by more
+      // than 8 (base 2) does the warp agree on a new per-row max and rescale;
+      // otherwise P = 2^(S - m) <= 2^8, which tau leaves room for.
       float t0 = -INFINITY, t1 = -INFINITY;
 #pragma unroll
       for (int st = 0; st < C::SUB; ++st) {
         t0 = fmaxf(t0, fmaxf(Sv[st][0], Sv[st][2]));
         t1 = fmaxf(t1, fmaxf(Sv[st][1], Sv[st][3]));
       }
+      if (__any_sync(~0u, (t0 > m0 + 8.f) || (t1 > m1 + 8.f))) {
 #pragma unroll
-      for (int off = 4; off < 32; off <<= 1) {
-        t0 = fmaxf(t0, __shfl_xor_sync(~0u, t0, off));
-        t1 = fmaxf(t1, __shfl_xor_sync(~0u, t1, off));
-      }
-      const float n0 = fmaxf(m0, t0), n1 = fmaxf(m1, t1);
-      const float u0 = n0 == -INFINITY ? 0.f : n0, u1 = n1 == -INFINITY ? 0.f : n1;
-      const float al0 = ex2(m0 - u0), al1 = ex2(m1 - u1);
-      float P[C::SUB][4];
-#pragma unroll
-      for (int st = 0; st < C::SUB; ++st) {
-        P[st][0] = ex2(Sv[st][0] - u0); P[st][1] = ex2(Sv[st][1] - u1);
-        P[st][2] = ex2(Sv[st][2] - u0); P[st][3] = ex2(Sv[st][3] - u1);
-      }
-      m0 = n0; m1 = n1;
-      float ps0 = 0.f, ps1 = 0.f;
-#pragma unroll
-      for (int st = 0; st < C::SUB; ++st) { ps0 += P[st][0] + P[st][2]; ps1 += P[st][1] + P[st][3]; }
-      l0 = fmaf(l0, al0, ps0);
-      l1 = fmaf(l1, al1, ps1);
-      if (__any_sync(~0u, (al0 != 1.f) || (al1 != 1.f))) {
+        for (int off = 4; off < 32; off <<= 1) {
+          t0 = fmaxf(t0, __shfl_xor_sync(~0u, t0, off));
+          t1 = fmaxf(t1, __shfl_xor_sync(~0u, t1, off));
+        }
+        const float n0 = fmaxf(m0, t0), n1 = fmaxf(m1, t1);
+        const float al0 = ex2(m0 - (n0 == -INFINITY ? 0.f : n0));
+        const float al1 = ex2(m1 - (n1 == -INFINITY ? 0.f : n1));
+        m0 = n0; m1 = n1;
+        l0 *= al0; l1 *= al1;
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt) {
           O[mt][0] *= al0; O[mt][1] *= al1; O[mt][2] *= al0; O[mt][3] *= al1;
@@ -739,6 +732,18 @@ qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
 #pragma unroll
         for (int G = 0; G < NG; ++G) { beta[0][G] *= al0; beta[1][G] *= al1; }
       }
+      const float u0 = m0 == -INFINITY ? 0.f : m0, u1 = m1 == -INFINITY ? 0.f : m1;
+      float P[C::SUB][4];
+#pragma unroll
+      for (int st = 0; st < C::SUB; ++st) {
+        P[st][0] = ex2(Sv[st][0] - u0); P[st][1] = ex2(Sv[st][1] - u1);
+        P[st][2] = ex2(Sv[st][2] - u0); P[st][3] = ex2(Sv[st][3] - u1);
+      }
+      float ps0 = 0.f, ps1 = 0.f;
+#pragma unroll
+      for (int st = 0; st < C::SUB; ++st) { ps0 += P[st][0] + P[st][2]; ps1 += P[st][1] + P[st][3]; }
+      l0 += ps0;
+      l1 += ps1;
 
       // ---------------- values --------------------------------------------------
       uint32_t vsw[C::SUB][2][MW], vbw[C::SUB][2][MW];
@@ -785,7 +790,7 @@ qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
 #pragma unroll
           for (int G = 0; G < NG; ++G) {
             const int e = (int)((vbound[G >> 1] >> (16 * (G & 1) + 10)) & 31);
-            const int nt = 29 - e;
+            const int nt = 21 - e;
             if (nt < tau[G]) {
               const float f = exp2i(nt - tau[G]);
 #pragma unroll
