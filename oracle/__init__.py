@@ -48,7 +48,8 @@ def lib():
         common = [p, i32, i32, i32, i32, i32,
                   i32, i32, i32, p, p, p,
                   i32, i32, i32, p, p, p,
-                  i64, i64, C.c_double, i32, p, i32, i64, i64, i64]
+                  i64, i64, C.c_double, i32, p, i32, i64, i64, i64,
+                  C.c_double, p, p]
         L.orc_attention.argtypes = common + [i32, i32, p, i64, p, i32]
         L.orc_attention.restype = i32
         L.orc_attention_probs.argtypes = common + [i32, i32, i32, p, p]
@@ -162,31 +163,48 @@ class Mask:
     strides: Sequence[int] = (0, 0, 0)  # element strides over (b, h, query)
 
 
-def _common_args(q64, k: QCache, v: QCache, L, scale, mask: Optional[Mask]):
+@dataclass
+class Ext:
+    """Attention extensions (see qkv_oracle.cpp): logit softcap (0 = off),
+    per-head sink logits [Hq] and per-head additive-mask slopes [Hq] (ALiBi)."""
+    softcap: float = 0.0
+    sinks: Optional[np.ndarray] = None
+    slopes: Optional[np.ndarray] = None
+
+
+def _common_args(q64, k: QCache, v: QCache, L, scale, mask: Optional[Mask],
+                 ext: Optional[Ext] = None):
     B, Hq, Lq, D = q64.shape
     Hkv = k.codes.shape[1]
     mask = mask or Mask()
+    ext = ext or Ext()
     kind = {"none": 0, "causal": 1, "additive": 2}[mask.kind]
     add = None if mask.add is None else np.ascontiguousarray(mask.add)
+    sinks = None if ext.sinks is None else np.ascontiguousarray(ext.sinks, dtype=np.float64)
+    slopes = None if ext.slopes is None else np.ascontiguousarray(ext.slopes, dtype=np.float64)
+    for a in (sinks, slopes):
+        if a is not None and a.size != Hq:
+            raise ValueError("sinks and slopes hold one value per query head")
     return [
         _ptr(q64), B, Hq, Hkv, Lq, D,
         _FMT[k.fmt], k.bits, k.gs, _ptr(k.codes), _ptr(k.scales), _ptr(k.biases),
         _FMT[v.fmt], v.bits, v.gs, _ptr(v.codes), _ptr(v.scales), _ptr(v.biases),
         k.Lcap, L, float(scale), kind, _ptr(add), _DT[mask.dtype],
         int(mask.strides[0]), int(mask.strides[1]), int(mask.strides[2]),
-    ], add
+        float(ext.softcap), _ptr(sinks), _ptr(slopes),
+    ], (add, sinks, slopes)
 
 
 def attention(q: np.ndarray, q_dtype: str, k: QCache, v: QCache, L: int,
               scale: float, mask: Optional[Mask] = None, mode: str = "two_pass",
               nsplit: int = 1, rows: Optional[np.ndarray] = None,
-              nthreads: Optional[int] = None) -> np.ndarray:
+              nthreads: Optional[int] = None, ext: Optional[Ext] = None) -> np.ndarray:
     """fp64 attention output [B,Hq,Lq,D].  ``rows`` (flattened (b,h,i) ids)
     restricts the computation to a subset; other rows are left NaN."""
     q64 = np.ascontiguousarray(to_f64(q, q_dtype))
     B, Hq, Lq, D = q64.shape
     out = np.full((B, Hq, Lq, D), np.nan)
-    args, keep = _common_args(q64, k, v, L, scale, mask)
+    args, keep = _common_args(q64, k, v, L, scale, mask, ext)
     r = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
     rc = lib().orc_attention(*args, {"two_pass": 0, "online": 1, "split": 2}[mode],
                              nsplit, _ptr(r), 0 if r is None else r.size, _ptr(out),
@@ -198,13 +216,13 @@ def attention(q: np.ndarray, q_dtype: str, k: QCache, v: QCache, L: int,
 
 def attention_probs(q: np.ndarray, q_dtype: str, k: QCache, v: QCache, L: int,
                     scale: float, b: int, h: int, i: int,
-                    mask: Optional[Mask] = None):
+                    mask: Optional[Mask] = None, ext: Optional[Ext] = None):
     """Softmax row (length L) and output (length D) of query row (b, h, i)."""
     q64 = np.ascontiguousarray(to_f64(q, q_dtype))
     D = q64.shape[-1]
     probs = np.empty(L, np.float64)
     o = np.empty(D, np.float64)
-    args, keep = _common_args(q64, k, v, L, scale, mask)
+    args, keep = _common_args(q64, k, v, L, scale, mask, ext)
     rc = lib().orc_attention_probs(*args, b, h, i, _ptr(probs), _ptr(o))
     if rc:
         raise ValueError("oracle attention_probs: invalid arguments")

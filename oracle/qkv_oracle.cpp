@@ -42,6 +42,17 @@
 //    (query i of Lq sees key j iff j <= L - Lq + i); a row with no visible key
 //    returns zeros.
 //  * attention math in fp64 after exact dequantization.
+//  * extensions that the llama.cpp PR's test coverage lists (sinks, ALiBi,
+//    logit softcap; the pages give no formula for them), in their usual
+//    definitions:
+//      - logit softcap c > 0: the scaled logit x = scale*q.k becomes
+//        c*tanh(x/c), before the mask is added;
+//      - ALiBi as a per-head slope on the additive mask: head h adds
+//        slope[h]*mask (a -inf entry hides the key whatever the slope);
+//      - attention sink: a per-head logit sink[h] that joins the softmax
+//        denominator (exp(sink - M)) with no value row, so the weights of
+//        the keys sum to less than 1; a row with no visible key still
+//        returns zeros.
 
 #include <cmath>
 #include <cstdint>
@@ -233,6 +244,9 @@ struct Problem {
   int64_t L;
   double scale;
   Mask mask;
+  double softcap;       // 0: off
+  const double* sinks;  // [Hq] or null
+  const double* slopes; // [Hq] or null (additive mask multiplier)
 };
 
 // Logit of key j for query row (b,h,i); returns false if the key is invisible.
@@ -241,13 +255,14 @@ bool logit(const Problem& p, int b, int h, int i, int64_t j,
   const double* qr = p.q + (((int64_t)b * p.Hq + h) * p.Lq + i) * p.D;
   double s = 0.0;
   for (int e = 0; e < p.D; ++e) s += (qr[e] * p.scale) * kh[e];
+  if (p.softcap > 0.0) s = p.softcap * std::tanh(s / p.softcap);
   if (p.mask.kind == 1) {
     if (j > p.L - p.Lq + i) return false;
   } else if (p.mask.kind == 2) {
     const int64_t idx = b * p.mask.sb + h * p.mask.sh + i * p.mask.sq + j;
     const double m = (double)load_elem(p.mask.add, p.mask.add_dtype, idx);
     if (std::isinf(m) && m < 0) return false;
-    s += m;
+    s += (p.slopes ? p.slopes[h] : 1.0) * m;
   }
   *out = s;
   return true;
@@ -271,6 +286,10 @@ void attend_two_pass(const Problem& p, int b, int h, int i, double* o,
   if (probs) for (int64_t j = 0; j < p.L; ++j) probs[j] = 0.0;
   if (!(mx > -std::numeric_limits<double>::infinity())) return;  // none visible
   double l = 0.0;
+  if (p.sinks) {                                             // the sink joins the max and the sum
+    mx = std::max(mx, p.sinks[h]);
+    l += std::exp(p.sinks[h] - mx);
+  }
   for (int64_t j = 0; j < p.L; ++j) if (vis[j]) { s[j] = std::exp(s[j] - mx); l += s[j]; }
   const int64_t vbase = ((int64_t)b * p.Hkv + kvh) * p.v.Lcap;
   for (int64_t j = 0; j < p.L; ++j) {
@@ -308,6 +327,19 @@ void attend_online_range(const Problem& p, int b, int h, int i, int64_t j0,
   *l_out = l;
 }
 
+// Final normalization of an online/merged (m, l, o): o / l, with the head's
+// sink (if any) folded into the denominator; no visible key gives zeros.
+void finish_row(const Problem& p, int h, double m, double l, double* o) {
+  if (!(l > 0.0)) { for (int e = 0; e < p.D; ++e) o[e] = 0.0; return; }
+  double w = 1.0;
+  if (p.sinks) {
+    const double M = std::max(m, p.sinks[h]);
+    w = std::exp(m - M);
+    l = l * w + std::exp(p.sinks[h] - M);
+  }
+  for (int e = 0; e < p.D; ++e) o[e] = o[e] * w / l;
+}
+
 // Split form: partition keys into `nsplit` contiguous chunks, run the online
 // form on each, then merge the partial (m, l, o) by log-sum-exp rescaling.
 void attend_split(const Problem& p, int b, int h, int i, int nsplit, double* o) {
@@ -328,7 +360,7 @@ void attend_split(const Problem& p, int b, int h, int i, int nsplit, double* o) 
     l += w * ls[sidx];
     for (int e = 0; e < p.D; ++e) o[e] += w * os[(size_t)sidx * p.D + e];
   }
-  for (int e = 0; e < p.D; ++e) o[e] /= l;
+  finish_row(p, h, M, l, o);
 }
 
 template <class F>
@@ -417,7 +449,8 @@ int orc_attention(const double* q, int B, int Hq, int Hkv, int Lq, int D,
                   const uint16_t* vscales, const uint16_t* vbiases,
                   int64_t Lcap, int64_t L, double scale, int mask_kind,
                   const void* mask_add, int mask_dtype, int64_t msb,
-                  int64_t msh, int64_t msq, int mode, int nsplit,
+                  int64_t msh, int64_t msq, double softcap,
+                  const double* sinks, const double* slopes, int mode, int nsplit,
                   const int64_t* rows, int64_t nrows, double* out,
                   int nthreads) {
   if (Hkv <= 0 || Hq % Hkv != 0 || L < 0 || L > Lcap) return 1;
@@ -430,6 +463,7 @@ int orc_attention(const double* q, int B, int Hq, int Hkv, int Lq, int D,
   p.L = L; p.scale = scale;
   p.mask.kind = mask_kind; p.mask.add = mask_add; p.mask.add_dtype = mask_dtype;
   p.mask.sb = msb; p.mask.sh = msh; p.mask.sq = msq;
+  p.softcap = softcap; p.sinks = sinks; p.slopes = slopes;
   const int64_t total = rows ? nrows : (int64_t)B * Hq * Lq;
   parallel_rows(total, nthreads, [&](int64_t r) {
     const int64_t id = rows ? rows[r] : r;
@@ -442,7 +476,7 @@ int orc_attention(const double* q, int B, int Hq, int Hkv, int Lq, int D,
     } else if (mode == 1) {
       double m, l;
       attend_online_range(p, b, h, i, 0, L, &m, &l, o);
-      for (int e = 0; e < D; ++e) o[e] = (l > 0.0) ? o[e] / l : 0.0;
+      finish_row(p, h, m, l, o);
     } else {
       attend_split(p, b, h, i, nsplit < 1 ? 1 : nsplit, o);
     }
@@ -458,7 +492,8 @@ int orc_attention_probs(const double* q, int B, int Hq, int Hkv, int Lq, int D,
                         const uint16_t* vscales, const uint16_t* vbiases,
                         int64_t Lcap, int64_t L, double scale, int mask_kind,
                         const void* mask_add, int mask_dtype, int64_t msb,
-                        int64_t msh, int64_t msq, int b, int h, int i,
+                        int64_t msh, int64_t msq, double softcap,
+                        const double* sinks, const double* slopes, int b, int h, int i,
                         double* probs, double* o) {
   if (Hkv <= 0 || Hq % Hkv != 0 || L < 0 || L > Lcap) return 1;
   if (kfmt == 1) { kbits = 8; kgs = 32; }
@@ -470,6 +505,7 @@ int orc_attention_probs(const double* q, int B, int Hq, int Hkv, int Lq, int D,
   p.L = L; p.scale = scale;
   p.mask.kind = mask_kind; p.mask.add = mask_add; p.mask.add_dtype = mask_dtype;
   p.mask.sb = msb; p.mask.sh = msh; p.mask.sq = msq;
+  p.softcap = softcap; p.sinks = sinks; p.slopes = slopes;
   attend_two_pass(p, b, h, i, o, probs);
   return 0;
 }
