@@ -591,6 +591,58 @@ def other_rows(device):
     except Exception as e:
         rows["materialize_decode_64k_affine4"] = {"unavailable": f"{type(e).__name__}: {e}"[:200]}
     torch.cuda.empty_cache()
+
+    # the attention extensions on the main decode workload (the extension
+    # variant of the decode kernel): logit softcap 30 with per-head sinks, and
+    # ALiBi (a broadcast fp32 distance mask with per-head slopes)
+    w = S.WORKLOADS["decode_64k_affine4"]
+    inp = S.make_inputs(w)
+    ncopies = max(3, math.ceil(3 * 126e6 / w.cache_bytes()))
+    caches = build_caches(w, inp, ncopies, device)
+    q = dev16(inp.q, "f16", device)
+    out = torch.empty(w.B, w.Hq, 1, w.D, dtype=torch.float16, device=device)
+    ws = qkv.make_workspace(w.B, w.Hq, w.Hkv, 1, w.D, w.L, device)
+    sinks = torch.linspace(8.0, 12.0, w.Hq, device=device)
+    slopes = torch.tensor([2.0 ** (-8.0 * (h + 1) / w.Hq) for h in range(w.Hq)], device=device)
+    dist = -torch.arange(w.L - 1, -1, -1, dtype=torch.float32, device=device)
+    nb = w.cache_bytes() + 2 * w.Hq * w.D * 2
+
+    def estep(i, **kw):
+        a, b = caches[i % ncopies]
+        qkv.qsdpa_decode(q, a, b, w.L, w.scale, out=out, workspace=ws, **kw)
+    sec_c, _ = graph_time(lambda i: estep(i, softcap=30.0, sinks=sinks), 400, 20)
+    sec_a, _ = graph_time(lambda i: estep(i, mask=(dist, (0, 0, 0)), mask_slopes=slopes), 400, 20)
+    rows["extensions_decode_64k_affine4"] = {
+        "softcap_sinks_us_per_call": round(sec_c * 1e3, 3),
+        "softcap_sinks_frac_hbm": round(nb / (sec_c / 1e3) / 1e9 / hbm_peak, 4),
+        "alibi_us_per_call": round(sec_a * 1e3, 3),
+        "alibi_frac_hbm": round(nb / (sec_a / 1e3) / 1e9 / hbm_peak, 4),
+        "note": "qsdpa_decode_ext on decode_64k_affine4: softcap 30 + per-head sinks; ALiBi as "
+                "a broadcast fp32 distance mask (256 KB) with per-head slopes; compare the "
+                "bench value"}
+    del caches
+    torch.cuda.empty_cache()
+
+    # the same for the prefill workload: softcap 30 + sinks on the tcgen05 kernel
+    w = S.WORKLOADS["prefill_q8_0_512_at_20k"]
+    inp = S.make_inputs(w)
+    kc, vc = build_caches(w, inp, 1, device)[0]
+    q = dev16(inp.q, w.q_dtype, device)
+    out = torch.empty(w.B, w.Hq, w.Lq, w.D, dtype=torch.bfloat16, device=device)
+    ws = qkv.make_workspace(w.B, w.Hq, w.Hkv, w.Lq, w.D, w.L, device)
+    sinks = torch.linspace(8.0, 12.0, w.Hq, device=device)
+    sec, _ = graph_time(lambda i: qkv.qsdpa_prefill(q, kc, vc, w.L, w.scale, causal=True, out=out,
+                                                    workspace=ws, softcap=30.0, sinks=sinks),
+                        20, 3)
+    flop = prefill_flops(w)
+    _, bf16_peak, _ = peaks()
+    rows["extensions_" + w.name] = {
+        "softcap_sinks_us_per_call": round(sec * 1e3, 2),
+        "TFLOP/s": round(flop / (sec / 1e3) / 1e12, 1),
+        "frac_tensor_peak": round(flop / (sec / 1e3) / 1e12 / bf16_peak, 4),
+        "note": "qsdpa_prefill_ext, softcap 30 + per-head sinks; compare prefill_q8_0_512_at_20k"}
+    del kc, vc
+    torch.cuda.empty_cache()
     return rows
 
 

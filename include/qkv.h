@@ -86,6 +86,32 @@ typedef struct {
   int64_t stride_b, stride_h, stride_q;
 } qkv_mask;
 
+/* Optional attention extensions (pass NULL for none).  The llama.cpp PR's
+ * tests cover these variants of flash attention (sinks, ALiBi, logit
+ * softcap); the pages print no formula, so this library takes the usual
+ * definitions (the CPU oracle states the same):
+ *  softcap > 0:  the scaled logit x = scale * q.k becomes softcap*tanh(x/softcap),
+ *                before the mask is added (Gemma-2 style logit capping);
+ *                0 = off.  Must be finite and >= 0.
+ *  mask_slopes:  device fp32 [Hq] or NULL: with an additive mask, query head h
+ *                adds mask_slopes[h] * mask (a -inf entry still hides the key;
+ *                ignored without an additive mask).  ALiBi is this with a mask
+ *                holding minus the query-key distance and the slopes of
+ *                Press et al. (2^(-8(h+1)/Hq) for a power-of-two Hq).
+ *  sinks:        device fp32 [Hq] or NULL: a per-head logit s_h that joins the
+ *                softmax denominator with no value row (gpt-oss style
+ *                attention sinks): out = sum_j e^(x_j - M) v_j /
+ *                (sum_j e^(x_j - M) + e^(s_h - M)), M = max(max_j x_j, s_h).
+ *                A query row with no visible key still returns zeros.
+ * Both arrays must be 4-byte aligned and stay valid until the call's kernels
+ * have run.  They cost the kernels nothing when absent; softcap adds one
+ * exp2 and one division per logit. */
+typedef struct {
+  float softcap;
+  const float* mask_slopes;
+  const float* sinks;
+} qkv_attn_ext;
+
 /* Quantize Lnew new tokens per (batch, kv-head) and write them into rows
  * [offset, offset+Lnew) of the K and V caches, in place (MLX kv_update /
  * KVUpdate::eval_gpu; the pages copy the whole cache first, this library
@@ -158,6 +184,20 @@ qkv_status qsdpa_prefill(const void* q, int q_dtype, int B, int Hq, int Hkv, int
                          int D, const qkv_cache* k, const qkv_cache* v, int64_t L,
                          float scale, const qkv_mask* mask, void* out, int out_dtype,
                          void* workspace, size_t workspace_bytes, void* stream);
+
+/* qsdpa_decode / qsdpa_prefill with the attention extensions above (ext may
+ * be NULL, which is the plain call).  Same arguments, rules and accuracy
+ * otherwise. */
+qkv_status qsdpa_decode_ext(const void* q, int q_dtype, int B, int Hq, int Hkv, int D,
+                            const qkv_cache* k, const qkv_cache* v, int64_t L,
+                            float scale, const qkv_mask* mask, const qkv_attn_ext* ext,
+                            void* out, int out_dtype, void* workspace,
+                            size_t workspace_bytes, void* stream);
+qkv_status qsdpa_prefill_ext(const void* q, int q_dtype, int B, int Hq, int Hkv, int Lq,
+                             int D, const qkv_cache* k, const qkv_cache* v, int64_t L,
+                             float scale, const qkv_mask* mask, const qkv_attn_ext* ext,
+                             void* out, int out_dtype, void* workspace,
+                             size_t workspace_bytes, void* stream);
 
 /* Rows [0, L) of one quantized cache materialized as fp16:
  * out[b, h, j, e] = fp16(scale * code + bias) (Q8_0: scale * code), the

@@ -1,5 +1,6 @@
 // api.cu -- extern "C" entry points of libqkv.so: argument validation, work
 // planning and kernel launch.  Declarations and contracts: include/qkv.h.
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -88,7 +89,8 @@ qkv_status attention(const void* q, int q_dtype, int B, int Hq, int Hkv, int Lq,
                      const qkv_cache* k, const qkv_cache* v, int64_t L, float scale,
                      const qkv_mask* mask, void* out, int out_dtype, void* workspace,
                      size_t workspace_bytes, void* stream, const void* new_k = nullptr,
-                     const void* new_v = nullptr, int in_dtype = QKV_F16) {
+                     const void* new_v = nullptr, int in_dtype = QKV_F16,
+                     const qkv_attn_ext* ext = nullptr) {
   qkv_status st;
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Lq <= 0)
     return fail(QKV_ERR_INVALID_ARG, "B, Hq, Hkv and Lq must be positive");
@@ -119,6 +121,22 @@ qkv_status attention(const void* q, int q_dtype, int B, int Hq, int Hkv, int Lq,
   }
   if ((int64_t)Hq * Lq > (int64_t)1 << 30)
     return fail(QKV_ERR_INVALID_ARG, "Hq * Lq too large");
+  float cap_a = 0.f, cap_k = 0.f;
+  const float* slopes = nullptr;
+  const float* sinks = nullptr;
+  if (ext != nullptr) {
+    if (!(ext->softcap >= 0.f) || std::isinf(ext->softcap))
+      return fail(QKV_ERR_INVALID_ARG, "softcap must be finite and >= 0");
+    if (ext->softcap > 0.f) {
+      cap_a = ext->softcap * 1.4426950408889634f;
+      cap_k = 2.f / ext->softcap;
+    }
+    if ((reinterpret_cast<uintptr_t>(ext->mask_slopes) & 3u) != 0 ||
+        (reinterpret_cast<uintptr_t>(ext->sinks) & 3u) != 0)
+      return fail(QKV_ERR_ALIGNMENT, "mask_slopes and sinks must be 4-byte aligned");
+    if (mkind == QKV_MASK_ADDITIVE) slopes = ext->mask_slopes;
+    sinks = ext->sinks;
+  }
 
   const size_t elems = (size_t)B * Hq * Lq * D;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -150,6 +168,7 @@ qkv_status attention(const void* q, int q_dtype, int B, int Hq, int Hkv, int Lq,
       pp.mask = mask->add; pp.mask_dtype = mask->add_dtype;
       pp.msb = mask->stride_b; pp.msh = mask->stride_h; pp.msq = mask->stride_q;
     }
+    pp.cap_a = cap_a; pp.cap_k = cap_k; pp.slopes = slopes; pp.sinks = sinks;
     pp.status = static_cast<unsigned*>(workspace);
     cudaError_t e = qkv::launch_prefill_tc(D, k->bits, k->group_size, k->fmt, pp, s);
     if (e != cudaSuccess) return fail(QKV_ERR_CUDA, "prefill launch: %s", cudaGetErrorString(e));
@@ -157,7 +176,11 @@ qkv_status attention(const void* q, int q_dtype, int B, int Hq, int Hkv, int Lq,
   }
   qkv::DecodePlan plan;
   const bool fused = new_k != nullptr;
-  if (!qkv::plan_decode(D, k->bits, k->group_size, k->fmt, out_dtype == QKV_F32, fused, B,
+  const bool extended = cap_a > 0.f || slopes != nullptr || sinks != nullptr;
+  if (fused && extended)
+    return fail(QKV_ERR_UNSUPPORTED, "the fused update step takes no attention extensions");
+  const int var = fused ? qkv::kDecFused : extended ? qkv::kDecExt : qkv::kDecPlain;
+  if (!qkv::plan_decode(D, k->bits, k->group_size, k->fmt, out_dtype == QKV_F32, var, B,
                         Hkv * rows, Hkv, L, &plan))
     return fail(QKV_ERR_UNSUPPORTED, "no kernel for D=%d bits=%d group_size=%d", D, k->bits,
                 k->group_size);
@@ -181,6 +204,7 @@ qkv_status attention(const void* q, int q_dtype, int B, int Hq, int Hkv, int Lq,
     p.msb = mask->stride_b; p.msh = mask->stride_h; p.msq = mask->stride_q;
   }
   if (mkind == QKV_MASK_CAUSAL && Lq == 1) p.mask_kind = QKV_MASK_NONE;  // all keys visible
+  p.cap_a = cap_a; p.cap_k = cap_k; p.slopes = slopes; p.sinks = sinks;
   if (fused) {
     p.new_k = static_cast<const uint16_t*>(new_k);
     p.new_v = static_cast<const uint16_t*>(new_v);
@@ -299,6 +323,24 @@ qkv_status qsdpa_prefill(const void* q, int q_dtype, int B, int Hq, int Hkv, int
                          size_t workspace_bytes, void* stream) {
   return attention(q, q_dtype, B, Hq, Hkv, Lq, D, k, v, L, scale, mask, out, out_dtype, workspace,
                    workspace_bytes, stream);
+}
+
+qkv_status qsdpa_decode_ext(const void* q, int q_dtype, int B, int Hq, int Hkv, int D,
+                            const qkv_cache* k, const qkv_cache* v, int64_t L, float scale,
+                            const qkv_mask* mask, const qkv_attn_ext* ext, void* out,
+                            int out_dtype, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  return attention(q, q_dtype, B, Hq, Hkv, 1, D, k, v, L, scale, mask, out, out_dtype, workspace,
+                   workspace_bytes, stream, nullptr, nullptr, QKV_F16, ext);
+}
+
+qkv_status qsdpa_prefill_ext(const void* q, int q_dtype, int B, int Hq, int Hkv, int Lq, int D,
+                             const qkv_cache* k, const qkv_cache* v, int64_t L, float scale,
+                             const qkv_mask* mask, const qkv_attn_ext* ext, void* out,
+                             int out_dtype, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+  return attention(q, q_dtype, B, Hq, Hkv, Lq, D, k, v, L, scale, mask, out, out_dtype, workspace,
+                   workspace_bytes, stream, nullptr, nullptr, QKV_F16, ext);
 }
 
 }  // extern "C"

@@ -2,7 +2,7 @@
 #include "decode_dispatch.cuh"
 
 namespace qkv {
-bool decode_ops_d256(int bits, int gs, bool q8, int nc, bool f32, bool fused, DecodeOps* ops) {
-  return decode_ops_for<256>(bits, gs, q8, nc, f32, fused, ops);
+bool decode_ops_d256(int bits, int gs, bool q8, int nc, bool f32, int var, DecodeOps* ops) {
+  return decode_ops_for<256>(bits, gs, q8, nc, f32, var, ops);
 }
 }  // namespace qkv

@@ -9,13 +9,13 @@
 namespace qkv {
 
 // Host-side helpers for one instance.
-template <int D, int BITS, int GS, bool Q8, int NC, bool F32OUT, bool FUSED>
+template <int D, int BITS, int GS, bool Q8, int NC, bool F32OUT, int VAR>
 struct DecodeInstance {
   using C = DecCfg<D, BITS, GS, Q8, NC>;
   static int max_ctas_per_sm() {
     static int cached = -1;
     if (cached < 0) {
-      auto k = qsdpa_decode_kernel<D, BITS, GS, Q8, NC, F32OUT, FUSED>;
+      auto k = qsdpa_decode_kernel<D, BITS, GS, Q8, NC, F32OUT, VAR>;
       if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
         return 0;
       int n = 0;
@@ -38,7 +38,7 @@ struct DecodeInstance {
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, qsdpa_decode_kernel<D, BITS, GS, Q8, NC, F32OUT, FUSED>, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, qsdpa_decode_kernel<D, BITS, GS, Q8, NC, F32OUT, VAR>, p);
     if (e != cudaSuccess || !plan.merge) return e;
     // parts per unit: at most the CTAs that share one unit
     const int64_t parts = plan.pieces > 0 ? plan.pieces : (plan.grid + plan.units - 1) / plan.units + 1;
@@ -62,31 +62,35 @@ struct DecodeOps {
   size_t smem;
 };
 
-template <int D, int BITS, int GS, bool Q8, int NC, bool F32, bool FUSED>
+template <int D, int BITS, int GS, bool Q8, int NC, bool F32, int VAR>
 DecodeOps make_decode_ops() {
-  using I = DecodeInstance<D, BITS, GS, Q8, NC, F32, FUSED>;
+  using I = DecodeInstance<D, BITS, GS, Q8, NC, F32, VAR>;
   return DecodeOps{&I::max_ctas_per_sm, &I::launch, I::C::TK, NC, I::C::NTEAM, (size_t)I::C::SMEM};
 }
 
-// The four variants of one format and chunking: f32 selects the
-// split-precision value operand used for fp32 output, fused the kernel that
-// also quantizes the new token into the cache.
+// The six variants of one format and chunking: f32 selects the
+// split-precision value operand used for fp32 output; var the plain kernel,
+// the one that also quantizes the new token into the cache, or the one with
+// the attention extensions (kept apart so the others carry none of their
+// registers).
 template <int D, int BITS, int GS, bool Q8, int NC>
-DecodeOps pick_decode_ops(bool f32, bool fused) {
-  if (fused) return f32 ? make_decode_ops<D, BITS, GS, Q8, NC, true, true>()
-                        : make_decode_ops<D, BITS, GS, Q8, NC, false, true>();
-  return f32 ? make_decode_ops<D, BITS, GS, Q8, NC, true, false>()
-             : make_decode_ops<D, BITS, GS, Q8, NC, false, false>();
+DecodeOps pick_decode_ops(bool f32, int var) {
+  if (var == kDecFused) return f32 ? make_decode_ops<D, BITS, GS, Q8, NC, true, kDecFused>()
+                                   : make_decode_ops<D, BITS, GS, Q8, NC, false, kDecFused>();
+  if (var == kDecExt) return f32 ? make_decode_ops<D, BITS, GS, Q8, NC, true, kDecExt>()
+                                 : make_decode_ops<D, BITS, GS, Q8, NC, false, kDecExt>();
+  return f32 ? make_decode_ops<D, BITS, GS, Q8, NC, true, kDecPlain>()
+             : make_decode_ops<D, BITS, GS, Q8, NC, false, kDecPlain>();
 }
 
 // Instances of one head dimension; nc in {1, 2, 4}.
 template <int D>
-bool decode_ops_for(int bits, int gs, bool q8, int nc, bool f32, bool fused, DecodeOps* ops) {
+bool decode_ops_for(int bits, int gs, bool q8, int nc, bool f32, int var, DecodeOps* ops) {
 #define QKV_DEC_NC(BITS, GS, Q8)                                                   \
   do {                                                                             \
-    if (nc == 1) *ops = pick_decode_ops<D, BITS, GS, Q8, 1>(f32, fused);           \
-    else if (nc == 2) *ops = pick_decode_ops<D, BITS, GS, Q8, 2>(f32, fused);      \
-    else *ops = pick_decode_ops<D, BITS, GS, Q8, 4>(f32, fused);                   \
+    if (nc == 1) *ops = pick_decode_ops<D, BITS, GS, Q8, 1>(f32, var);             \
+    else if (nc == 2) *ops = pick_decode_ops<D, BITS, GS, Q8, 2>(f32, var);        \
+    else *ops = pick_decode_ops<D, BITS, GS, Q8, 4>(f32, var);                     \
     return true;                                                                   \
   } while (0)
   if (q8) {
@@ -105,8 +109,8 @@ bool decode_ops_for(int bits, int gs, bool q8, int nc, bool f32, bool fused, Dec
   return false;
 }
 
-bool decode_ops_d64(int bits, int gs, bool q8, int nc, bool f32, bool fused, DecodeOps* ops);
-bool decode_ops_d128(int bits, int gs, bool q8, int nc, bool f32, bool fused, DecodeOps* ops);
-bool decode_ops_d256(int bits, int gs, bool q8, int nc, bool f32, bool fused, DecodeOps* ops);
+bool decode_ops_d64(int bits, int gs, bool q8, int nc, bool f32, int var, DecodeOps* ops);
+bool decode_ops_d128(int bits, int gs, bool q8, int nc, bool f32, int var, DecodeOps* ops);
+bool decode_ops_d256(int bits, int gs, bool q8, int nc, bool f32, int var, DecodeOps* ops);
 
 }  // namespace qkv

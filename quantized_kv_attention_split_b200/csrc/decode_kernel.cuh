@@ -295,9 +295,11 @@ __device__ __noinline__ void fused_quantize_patch(const DecodeParams& p, const u
   }
 }
 
-template <int D, int BITS, int GS, bool Q8, int NC, bool F32OUT, bool FUSED>
+template <int D, int BITS, int GS, bool Q8, int NC, bool F32OUT, int VAR>
 __global__ void __launch_bounds__(32 * dec_warps(D), 1)
 qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
+  constexpr bool FUSED = VAR == kDecFused;     // also quantizes the new token into row L - 1
+  constexpr bool EXT = VAR == kDecExt;         // logit softcap, mask slopes, sinks
   using C = DecCfg<D, BITS, GS, Q8, NC>;
   constexpr int NG = C::NG, KPG = C::KPG, MT = C::MT, BK = C::BK, NSTAGE = C::NSTAGE;
   constexpr int NTEAM = C::NTEAM, TTHR = C::TTHR;
@@ -676,6 +678,10 @@ qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
           Sx[2] = fmaf(c1, acc[2], fmaf(bb1, qsc[G][0], Sx[2]));
           Sx[3] = fmaf(c1, acc[3], fmaf(bb1, qsc[G][1], Sx[3]));
         }
+        if (EXT && p.cap_a > 0.f) {                       // logit softcap (before the mask)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) Sx[i] = softcap_log2(Sx[i], p.cap_a, p.cap_k);
+        }
         const int kr0 = 16 * st + g;                      // key index within the block
         if (kvalid < BK) {                                // only a block that reaches L
           if (kr0 >= kvalid) { Sx[0] = -INFINITY; Sx[1] = -INFINITY; }
@@ -687,6 +693,7 @@ qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
             const int vh = hbase + chunk * 8 + 2 * t + j;     // row = head * Lq + query
             if (vh < p.G) {
               const int hr = vh / p.Lq, qi = vh - hr * p.Lq;
+              const float slope = kLog2e * (EXT && p.slopes != nullptr ? p.slopes[hkv * p.Gq + hr] : 1.f);
 #pragma unroll
               for (int r = 0; r < 2; ++r) {
                 const int64_t key = key0 + kr0 + 8 * r;
@@ -696,7 +703,8 @@ qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
                 } else {
                   const int64_t mi = (int64_t)b * p.msb + ((int64_t)hkv * p.Gq + hr) * p.msh +
                                      (int64_t)qi * p.msq + key;
-                  Sx[2 * r + j] += kLog2e * load_as_float(p.mask, p.mask_dtype, mi);
+                  const float mv = load_as_float(p.mask, p.mask_dtype, mi);
+                  Sx[2 * r + j] = mv == -INFINITY ? -INFINITY : fmaf(slope, mv, Sx[2 * r + j]);
                 }
               }
             }
@@ -934,7 +942,24 @@ qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
       float Ls = w * lw;
 #pragma unroll
       for (int off = 1; off < NTEAM; off <<= 1) Ls += __shfl_xor_sync(~0u, Ls, off);
-      wgt[R * WST + k] = complete ? (Ls > 0.f ? w / Ls : 0.f) : w;
+      float wk = w;
+      if (complete) {
+        // a CTA that covered its whole unit normalizes here; the head's sink
+        // logit (if any) joins the denominator (a split unit's sink is added
+        // by the merge, once)
+        float Lt = Ls;
+        if (EXT && p.sinks != nullptr && hbase + R < p.G) {
+          const float s2 = kLog2e * p.sinks[hkv * p.Gq + (hbase + R) / p.Lq];
+          const float Mn = fmaxf(M, s2);
+          if (Mn != -INFINITY) {
+            const float f = M == -INFINITY ? 0.f : ex2(M - Mn);
+            Lt = Ls * f + ex2(s2 - Mn);
+            wk = w * f;
+          }
+        }
+        wk = (Ls > 0.f && Lt > 0.f) ? wk / Lt : 0.f;
+      }
+      wgt[R * WST + k] = wk;
       if (k == 0) { rml[2 * R] = M; rml[2 * R + 1] = Ls; }
     }
     __syncthreads();

@@ -1,7 +1,8 @@
 // decode_merge.cuh -- second pass of the split-K decode: the log-sum-exp merge
 // of the per-CTA partials (m_i, l_i, o_i) of every split unit,
 //   M = max_i m_i,  l = sum_i l_i 2^(m_i - M),  out = sum_i o_i 2^(m_i - M) / l
-// (base-2 logits), the same rule the online softmax applies within a CTA.
+// (base-2 logits), the same rule the online softmax applies within a CTA; a
+// head's attention-sink logit s, when given, joins as l += 2^(s - M).
 #pragma once
 
 #include "qkv_common.cuh"
@@ -100,7 +101,16 @@ qsdpa_merge_kernel(const __grid_constant__ DecodeParams p, int64_t nC, int lanes
     M = Mn;
   }
   if (!active || sub != 0) return;
-  const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+  float fo = 1.f;
+  if (p.sinks != nullptr && Ls > 0.f) {
+    // the head's sink logit joins the denominator: (M, l) -> (max(M, s), l 2^(M - M') + 2^(s - M'))
+    const int hkv = uh - (uh / p.Hkv) * p.Hkv;
+    const float s2 = kLog2e * p.sinks[hkv * p.Gq + head / p.Lq];
+    const float Mn = fmaxf(M, s2);
+    fo = ex2(M - Mn);
+    Ls = Ls * fo + ex2(s2 - Mn);
+  }
+  const float inv = Ls > 0.f ? fo / Ls : 0.f;
   const int64_t oi = ((int64_t)uh * p.G + head) * D + e4 * 4;
   store_from_float(p.out, p.out_dtype, oi, acc.x * inv);
   store_from_float(p.out, p.out_dtype, oi + 1, acc.y * inv);

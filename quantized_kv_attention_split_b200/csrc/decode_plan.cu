@@ -33,11 +33,11 @@ int sm_count() {
   return n;
 }
 
-bool get_ops(int D, int bits, int gs, int fmt, int nc, bool f32, bool fused, DecodeOps* ops) {
+bool get_ops(int D, int bits, int gs, int fmt, int nc, bool f32, int var, DecodeOps* ops) {
   const bool q8 = fmt == QKV_Q8_0;
-  if (D == 64) return decode_ops_d64(bits, gs, q8, nc, f32, fused, ops);
-  if (D == 128) return decode_ops_d128(bits, gs, q8, nc, f32, fused, ops);
-  if (D == 256) return decode_ops_d256(bits, gs, q8, nc, f32, fused, ops);
+  if (D == 64) return decode_ops_d64(bits, gs, q8, nc, f32, var, ops);
+  if (D == 128) return decode_ops_d128(bits, gs, q8, nc, f32, var, ops);
+  if (D == 256) return decode_ops_d256(bits, gs, q8, nc, f32, var, ops);
   return false;
 }
 
@@ -81,13 +81,13 @@ size_t decode_workspace_zero_bytes(int B, int Hq, int Hkv) {
   return kWsHeader;
 }
 
-bool plan_decode(int D, int bits, int gs, int fmt, int out_f32, bool fused, int B, int Hq,
+bool plan_decode(int D, int bits, int gs, int fmt, int out_f32, int var, int B, int Hq,
                  int Hkv, int64_t L, DecodePlan* plan) {
   int nc, ncg;
   decode_chunking(Hq / Hkv, &nc, &ncg);
   DecodeOps ops;
-  if (!get_ops(D, bits, gs, fmt, nc, out_f32 != 0, fused, &ops)) return false;
-  plan->fused = fused;
+  if (!get_ops(D, bits, gs, fmt, nc, out_f32 != 0, var, &ops)) return false;
+  plan->var = var;
   const int sms = std::max(1, sm_count());
   const int occ = std::min(max_ctas_per_sm(D), std::max(1, ops.occupancy()));
   plan->tk = ops.tk;
@@ -140,7 +140,7 @@ bool plan_decode(int D, int bits, int gs, int fmt, int out_f32, bool fused, int 
 cudaError_t launch_decode(int D, int bits, int gs, int fmt, int out_f32, const DecodePlan& plan,
                           DecodeParams& p, cudaStream_t stream) {
   DecodeOps ops;
-  if (!get_ops(D, bits, gs, fmt, plan.nc, out_f32 != 0, plan.fused, &ops)) return cudaErrorInvalidValue;
+  if (!get_ops(D, bits, gs, fmt, plan.nc, out_f32 != 0, plan.var, &ops)) return cudaErrorInvalidValue;
   p.ncg = plan.ncg;
   p.stages_per_unit = plan.stages_per_unit;
   p.total_stages = plan.total_stages;

@@ -6,10 +6,10 @@ namespace qkv {
 
 namespace {
 
-template <int D, int BITS, int GS, bool Q8>
-cudaError_t launch_pf(const PrefillParams& p, int grid, cudaStream_t s) {
+template <int D, int BITS, int GS, bool Q8, bool EXT>
+cudaError_t launch_pf_v(const PrefillParams& p, int grid, cudaStream_t s) {
   using C = PfCfg<D, BITS, GS, Q8>;
-  auto k = qsdpa_prefill_tc_kernel<D, BITS, GS, Q8>;
+  auto k = qsdpa_prefill_tc_kernel<D, BITS, GS, Q8, EXT>;
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
@@ -18,6 +18,14 @@ cudaError_t launch_pf(const PrefillParams& p, int grid, cudaStream_t s) {
   }
   k<<<grid, kPfThreads, C::SMEM, s>>>(p);
   return cudaGetLastError();
+}
+
+// the extension instance only when an extension is in use
+template <int D, int BITS, int GS, bool Q8>
+cudaError_t launch_pf(const PrefillParams& p, int grid, cudaStream_t s) {
+  if (p.cap_a > 0.f || p.slopes != nullptr || p.sinks != nullptr)
+    return launch_pf_v<D, BITS, GS, Q8, true>(p, grid, s);
+  return launch_pf_v<D, BITS, GS, Q8, false>(p, grid, s);
 }
 
 template <int D>

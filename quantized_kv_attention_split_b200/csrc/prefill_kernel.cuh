@@ -74,6 +74,9 @@ struct PrefillParams {
   const void* mask;
   int mask_dtype;
   int64_t msb, msh, msq;
+  float cap_a, cap_k;       // logit softcap (cap_a == 0: off), as in DecodeParams
+  const float* slopes;      // per-head additive-mask slopes, fp32 [Hq] or null
+  const float* sinks;       // per-head sink logits, fp32 [Hq] or null
   unsigned* status;         // nonzero after a tensor-core wait timed out
 };
 
@@ -359,7 +362,60 @@ struct PfChunks {
   }
 };
 
-template <int D, int BITS, int GS, bool Q8>
+// Adds slope * mask[j] to the base-2 logits sv[j] of one tile row for j < lim
+// (the others are -inf already and read nothing); a -inf mask entry hides the
+// key.  Each thread reads its own row, so the reads go 16 bytes at a time when
+// the row is 16-byte aligned (scalar reads for the row's ragged end and for
+// unaligned rows), without branches around them; they go out 16 elements at a
+// time (the compiler barrier between the groups keeps it from hoisting all of
+// them, which would not fit the registers next to the tile).
+__device__ __forceinline__ void pf_unpack(uint4 r, const float*, float* o) {
+  o[0] = __uint_as_float(r.x); o[1] = __uint_as_float(r.y);
+  o[2] = __uint_as_float(r.z); o[3] = __uint_as_float(r.w);
+}
+__device__ __forceinline__ void pf_unpack(uint4 r, const __half*, float* o) {
+  const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = unpack_half2(w[i]);
+    o[2 * i] = f.x; o[2 * i + 1] = f.y;
+  }
+}
+__device__ __forceinline__ void pf_unpack(uint4 r, const __nv_bfloat16*, float* o) {
+  const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    o[2 * i] = __uint_as_float(w[i] << 16);
+    o[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ void pf_add_mask(float (&sv)[kPfBN], const T* m, int lim, float slope) {
+  constexpr int EPV = 16 / (int)sizeof(T);              // elements per 16-byte read
+  const bool vec = (reinterpret_cast<uintptr_t>(m) & 15u) == 0;
+#pragma unroll
+  for (int c = 0; c < kPfBN; c += 16) {
+#pragma unroll
+    for (int v = c; v < c + 16; v += EPV) {
+      float mv[EPV];
+      if (vec && v + EPV <= lim) {
+        pf_unpack(__ldg(reinterpret_cast<const uint4*>(m + v)), m, mv);
+      } else {
+#pragma unroll
+        for (int e = 0; e < EPV; ++e) mv[e] = v + e < lim ? to_float_ld(m + v + e) : 0.f;
+      }
+#pragma unroll
+      for (int e = 0; e < EPV; ++e)
+        sv[v + e] = mv[e] == -INFINITY ? -INFINITY : fmaf(slope, mv[e], sv[v + e]);
+    }
+    asm volatile("" ::: "memory");
+  }
+}
+
+// EXT: the instance with the attention extensions (logit softcap, additive-mask
+// slopes, sinks); the plain instance carries none of their code.
+template <int D, int BITS, int GS, bool Q8, bool EXT>
 __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const PrefillParams p) {
   using C = PfCfg<D, BITS, GS, Q8>;
   constexpr int NG = C::NG;
@@ -643,6 +699,9 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
     const int64_t causal_lim = L - p.Lq + qi;    // last visible key of this row
     const bool causal = p.mask_kind == QKV_MASK_CAUSAL;
     const bool additive = p.mask_kind == QKV_MASK_ADDITIVE;
+    const bool capped = EXT && p.cap_a > 0.f;    // logit softcap
+    const float slope = kLog2e * (EXT && additive && p.slopes != nullptr && row_ok
+                                      ? p.slopes[hkv * p.G + hh] : 1.f);
     float m_used = -INFINITY, lsum = 0.f;
     for (int t = 0; t < ntiles; ++t) {
       const int s = t & 1;
@@ -654,7 +713,9 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
       tmem_ld32(tmem_row + C::S_COL + s * kPfBN + 32, reinterpret_cast<uint32_t*>(sv + 32));
       tmem_wait_ld();
       // a tile without masked keys for any row of the warp takes the short path
-      const bool full = __all_sync(~0u, row_ok && !additive && key0 + kPfBN <= kend &&
+      // (the tile maximum is taken over the raw products, which needs rowscale >= 0)
+      const bool full = __all_sync(~0u, row_ok && !additive && rowscale >= 0.f &&
+                                            key0 + kPfBN <= kend &&
                                             (!causal || key0 + kPfBN - 1 <= causal_lim));
       float tmax;
       if (full) {
@@ -665,22 +726,33 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
           m1 = fmaxf(m1, fmaxf(sv[j + 2], sv[j + 3]));
         }
         tmax = fmaxf(m0, m1) * rowscale;
+        if (capped) tmax = softcap_log2(tmax, p.cap_a, p.cap_k);   // the cap is increasing
       } else {
-        tmax = -INFINITY;
+        // per-element path: keys j < lim of the tile are visible (below L and the
+        // causal limit); then the additive mask, its loads all issued together
+        int64_t nv = kend - key0;
+        if (causal && causal_lim - key0 + 1 < nv) nv = causal_lim - key0 + 1;
+        const int lim = !row_ok || nv <= 0 ? 0 : nv >= kPfBN ? kPfBN : (int)nv;
 #pragma unroll
         for (int j = 0; j < kPfBN; ++j) {
-          const int64_t key = key0 + j;
-          bool vis = row_ok && key < kend;
-          if (causal) vis = vis && key <= causal_lim;
           float v = sv[j] * rowscale;
-          if (vis && additive) {
-            const int64_t mi = (int64_t)b * p.msb + ((int64_t)hkv * p.G + hh) * p.msh +
-                               (int64_t)qi * p.msq + key;
-            v += kLog2e * load_as_float(p.mask, p.mask_dtype, mi);
-          }
-          sv[j] = vis ? v : -INFINITY;
-          tmax = fmaxf(tmax, sv[j]);
+          if (capped) v = softcap_log2(v, p.cap_a, p.cap_k);
+          sv[j] = j < lim ? v : -INFINITY;
         }
+        if (additive) {
+          const int64_t mrow = (int64_t)b * p.msb + ((int64_t)hkv * p.G + hh) * p.msh +
+                               (int64_t)qi * p.msq + key0;
+          if (p.mask_dtype == QKV_F32)
+            pf_add_mask(sv, reinterpret_cast<const float*>(p.mask) + mrow, lim, slope);
+          else if (p.mask_dtype == QKV_F16)
+            pf_add_mask(sv, reinterpret_cast<const __half*>(p.mask) + mrow, lim, slope);
+          else
+            pf_add_mask(sv, reinterpret_cast<const __nv_bfloat16*>(p.mask) + mrow, lim, slope);
+        }
+        float m0 = sv[0], m1 = sv[1];
+#pragma unroll
+        for (int j = 2; j < kPfBN; j += 2) { m0 = fmaxf(m0, sv[j]); m1 = fmaxf(m1, sv[j + 1]); }
+        tmax = fmaxf(m0, m1);
       }
       float alpha = 1.f;
       if (tmax > m_used + 8.f) {
@@ -709,7 +781,15 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
         uint32_t pk[16];
-        if (full) {
+        if (full && capped) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float a = ex2(softcap_log2(sv[32 * hf + 2 * i] * rowscale, p.cap_a, p.cap_k) - mref);
+            const float c = ex2(softcap_log2(sv[32 * hf + 2 * i + 1] * rowscale, p.cap_a, p.cap_k) - mref);
+            rs0 += a; rs1 += c;
+            pk[i] = pack_half2(a, c);
+          }
+        } else if (full) {
           const float nm = -mref;
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
@@ -740,7 +820,15 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
       tc_fence_after();
     }
     have = __all_sync(~0u, have) && !*abort_flag;
-    const float inv = (lsum > 0.f && have) ? 1.f / lsum : 0.f;
+    float fo = 1.f;
+    if (EXT && p.sinks != nullptr && row_ok && lsum > 0.f) {
+      // the head's sink logit joins the denominator (P, l and O are relative to m_used)
+      const float s2 = kLog2e * p.sinks[hkv * p.G + hh];
+      const float Mn = fmaxf(m_used, s2);
+      fo = ex2(m_used - Mn);
+      lsum = lsum * fo + ex2(s2 - Mn);
+    }
+    const float inv = (lsum > 0.f && have) ? fo / lsum : 0.f;
 #pragma unroll 1
     for (int c = 0; c < D; c += 32) {
       uint32_t ob[32];

@@ -55,6 +55,16 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// Logit softcap applied to a base-2 logit S = log2(e) x: returns
+// log2(e) c tanh(x / c).  From tanh(y) = 1 - 2 / (1 + e^(2y)) with y = x / c:
+// e^(2y) = 2^(S k) for k = 2 / c, so the result is a - 2a / (1 + 2^(S k)) with
+// a = c log2(e).  The exponent is clamped at 64 (the quotient is then below
+// 2^-60 a) so no infinity enters the division; the absolute error is a few
+// units of a * 2^-23, from ex2.approx and the approximate division.
+__device__ __forceinline__ float softcap_log2(float S, float a, float k) {
+  return a - __fdividef(2.f * a, 1.f + ex2(fminf(S * k, 64.f)));
+}
+
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   return __byte_perm(a, b, sel);
 }
@@ -76,6 +86,12 @@ __device__ __forceinline__ float load_as_float(const void* p, int dtype, int64_t
   if (dtype == QKV_F16) return __half2float(reinterpret_cast<const __half*>(p)[i]);
   if (dtype == QKV_BF16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[i]);
   return reinterpret_cast<const float*>(p)[i];
+}
+// Read-only loads of one mask element as fp32.
+__device__ __forceinline__ float to_float_ld(const float* p) { return __ldg(p); }
+__device__ __forceinline__ float to_float_ld(const __half* p) { return __half2float(__ldg(p)); }
+__device__ __forceinline__ float to_float_ld(const __nv_bfloat16* p) {
+  return __bfloat162float(__ldg(p));
 }
 __device__ __forceinline__ void store_from_float(void* p, int dtype, int64_t i, float v) {
   if (dtype == QKV_F16) reinterpret_cast<__half*>(p)[i] = __float2half_rn(v);

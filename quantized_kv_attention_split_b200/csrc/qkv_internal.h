@@ -11,6 +11,11 @@
 namespace qkv {
 
 // Everything one decode launch needs (device pointers and sizes).
+// Decode kernel variants: the plain kernel, the fused update step (also
+// quantizes the new token into cache row L - 1) and the attention extensions
+// (logit softcap, additive-mask slopes, sinks).
+enum : int { kDecPlain = 0, kDecFused = 1, kDecExt = 2 };
+
 struct DecodeParams {
   const void* q;            // [B, Hq, 1, D]
   int q_dtype;
@@ -35,6 +40,12 @@ struct DecodeParams {
   const void* mask;
   int mask_dtype;
   int64_t msb, msh, msq;
+  // extensions: softcap of the base-2 logit S -> cap_a - 2 cap_a / (1 + 2^(S cap_k))
+  // (cap_a = softcap * log2(e), cap_k = 2 / softcap; cap_a == 0: off), per-head
+  // additive-mask slopes and sink logits (fp32 [Hq], may be null)
+  float cap_a, cap_k;
+  const float* slopes;
+  const float* sinks;
   // work split: units (b, kv-head, chunk-group) x blocks of TK keys, divided
   // evenly over gridDim.x CTAs
   int64_t stages_per_unit;
@@ -58,7 +69,7 @@ struct DecodePlan {
   int64_t stages_per_unit;
   int64_t total_stages;
   int grid;
-  bool fused;               // the kernel also quantizes the new token (row L - 1)
+  int var;                  // kDecPlain, kDecFused or kDecExt
   int pieces;               // CTAs per unit when the grid cuts every unit alike, else 0
   bool merge;               // some unit is split over several CTAs: merge kernel after
   size_t smem;
@@ -70,7 +81,7 @@ struct DecodePlan {
 
 // Plans a decode launch for the current device; returns false if the shape
 // has no kernel instance.
-bool plan_decode(int D, int bits, int gs, int fmt, int out_f32, bool fused, int B, int Hq,
+bool plan_decode(int D, int bits, int gs, int fmt, int out_f32, int var, int B, int Hq,
                  int Hkv, int64_t L, DecodePlan* plan);
 cudaError_t launch_decode(int D, int bits, int gs, int fmt, int out_f32,
                           const DecodePlan& plan, DecodeParams& p, cudaStream_t stream);

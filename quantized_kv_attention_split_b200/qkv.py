@@ -39,6 +39,10 @@ class _Mask(C.Structure):
                 ("stride_b", C.c_int64), ("stride_h", C.c_int64), ("stride_q", C.c_int64)]
 
 
+class _Ext(C.Structure):
+    _fields_ = [("softcap", C.c_float), ("mask_slopes", C.c_void_p), ("sinks", C.c_void_p)]
+
+
 class QKVError(RuntimeError):
     def __init__(self, status: int, detail: str):
         super().__init__(f"{_STATUS.get(status, status)}: {detail}")
@@ -67,6 +71,13 @@ def lib() -> C.CDLL:
         L.qsdpa_prefill.argtypes = [p, i32, i32, i32, i32, i32, i32, cp, cp, i64, C.c_float, mp,
                                     p, i32, p, sz, p]
         L.qsdpa_prefill.restype = i32
+        ep = C.POINTER(_Ext)
+        L.qsdpa_decode_ext.argtypes = [p, i32, i32, i32, i32, i32, cp, cp, i64, C.c_float, mp,
+                                       ep, p, i32, p, sz, p]
+        L.qsdpa_decode_ext.restype = i32
+        L.qsdpa_prefill_ext.argtypes = [p, i32, i32, i32, i32, i32, i32, cp, cp, i64, C.c_float,
+                                        mp, ep, p, i32, p, sz, p]
+        L.qsdpa_prefill_ext.restype = i32
         L.qsdpa_decode_update.argtypes = [p, i32, p, p, i32, i32, i32, i32, i32, cp, cp, i64,
                                           C.c_float, mp, p, i32, p, sz, p]
         L.qsdpa_decode_update.restype = i32
@@ -182,7 +193,21 @@ def _mask_struct(mask, causal: bool):
     return _Mask(MASK_ADDITIVE, t.data_ptr(), _DTYPE[t.dtype], *[int(x) for x in strides])
 
 
-def _attention(fn, q, k, v, L, scale, mask, causal, out, out_dtype, workspace, stream, decode):
+def _ext_struct(softcap, sinks, mask_slopes, Hq, device):
+    """qkv_attn_ext for the optional extensions, or None when none is used.
+    sinks / mask_slopes: fp32 CUDA tensors of Hq values."""
+    if not softcap and sinks is None and mask_slopes is None:
+        return None
+    for t in (sinks, mask_slopes):
+        if t is not None:
+            assert t.is_cuda and t.dtype == torch.float32 and t.is_contiguous()
+            assert t.numel() == Hq and t.device == device
+    return _Ext(float(softcap or 0.0), None if mask_slopes is None else mask_slopes.data_ptr(),
+                None if sinks is None else sinks.data_ptr())
+
+
+def _attention(fn, q, k, v, L, scale, mask, causal, out, out_dtype, workspace, stream, decode,
+               ext=None):
     assert q.is_contiguous() and q.is_cuda
     B, Hq, Lq, D = q.shape
     Hkv = k.codes.shape[1]
@@ -193,8 +218,11 @@ def _attention(fn, q, k, v, L, scale, mask, causal, out, out_dtype, workspace, s
     ks, vs = k._struct(), v._struct()
     m = _mask_struct(mask, causal)
     mp = C.byref(m) if m is not None else None
-    common = (C.byref(ks), C.byref(vs), int(L), float(scale), mp, out.data_ptr(),
-              _DTYPE[out.dtype], workspace.data_ptr(), workspace.numel(), _stream(stream))
+    common = (C.byref(ks), C.byref(vs), int(L), float(scale), mp)
+    if ext is not None:
+        common += (C.byref(ext),)
+    common += (out.data_ptr(), _DTYPE[out.dtype], workspace.data_ptr(), workspace.numel(),
+               _stream(stream))
     if decode:
         _check(fn(q.data_ptr(), _DTYPE[q.dtype], B, Hq, Hkv, D, *common))
     else:
@@ -204,11 +232,17 @@ def _attention(fn, q, k, v, L, scale, mask, causal, out, out_dtype, workspace, s
 
 def qsdpa_decode(q: torch.Tensor, k: QuantCache, v: QuantCache, L: int, scale: float,
                  mask=None, out: Optional[torch.Tensor] = None, out_dtype=None,
-                 workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """softmax(q*scale . K^T + mask) V for q [B,Hq,1,D] over keys [0, L)."""
+                 workspace: Optional[torch.Tensor] = None, stream=None, softcap: float = 0.0,
+                 sinks: Optional[torch.Tensor] = None,
+                 mask_slopes: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """softmax(q*scale . K^T + mask) V for q [B,Hq,1,D] over keys [0, L).
+    ``softcap``, ``sinks`` and ``mask_slopes`` are the attention extensions
+    of ``qkv_attn_ext`` (qsdpa_decode_ext)."""
     assert q.shape[2] == 1
-    return _attention(lib().qsdpa_decode, q, k, v, L, scale, mask, False, out, out_dtype,
-                      workspace, stream, True)
+    ext = _ext_struct(softcap, sinks, mask_slopes, q.shape[1], q.device)
+    fn = lib().qsdpa_decode if ext is None else lib().qsdpa_decode_ext
+    return _attention(fn, q, k, v, L, scale, mask, False, out, out_dtype, workspace, stream,
+                      True, ext)
 
 
 def qsdpa_decode_update(q: torch.Tensor, new_k: torch.Tensor, new_v: torch.Tensor,
@@ -241,11 +275,15 @@ def qsdpa_decode_update(q: torch.Tensor, new_k: torch.Tensor, new_v: torch.Tenso
 def qsdpa_prefill(q: torch.Tensor, k: QuantCache, v: QuantCache, L: int, scale: float,
                   mask=None, causal: bool = False, out: Optional[torch.Tensor] = None,
                   out_dtype=None, workspace: Optional[torch.Tensor] = None,
-                  stream=None) -> torch.Tensor:
+                  stream=None, softcap: float = 0.0, sinks: Optional[torch.Tensor] = None,
+                  mask_slopes: Optional[torch.Tensor] = None) -> torch.Tensor:
     """softmax(q*scale . K^T + mask) V for q [B,Hq,Lq,D] over keys [0, L);
-    ``causal`` aligns the Lq queries with the last Lq keys."""
-    return _attention(lib().qsdpa_prefill, q, k, v, L, scale, mask, causal, out, out_dtype,
-                      workspace, stream, False)
+    ``causal`` aligns the Lq queries with the last Lq keys.  ``softcap``,
+    ``sinks`` and ``mask_slopes`` as in :func:`qsdpa_decode`."""
+    ext = _ext_struct(softcap, sinks, mask_slopes, q.shape[1], q.device)
+    fn = lib().qsdpa_prefill if ext is None else lib().qsdpa_prefill_ext
+    return _attention(fn, q, k, v, L, scale, mask, causal, out, out_dtype, workspace, stream,
+                      False, ext)
 
 
 def qsdpa_decode_noalloc(q: torch.Tensor, k: QuantCache, v: QuantCache, L: int, scale: float,

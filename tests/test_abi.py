@@ -122,3 +122,27 @@ def test_dequantize_validation_errors(lib):
     assert f(C.byref(ok), 70000, 1, 128, 16, FAKE, None) == 2                # slabs > 65535
     assert f(C.byref(_cache(qkv, gs=48)), 1, 2, 128, 16, FAKE, None) == 2    # unsupported group
     assert f(C.byref(ok), 1, 2, 128, 0, FAKE, None) == 0                     # nothing to do
+
+
+def test_extension_validation_errors(lib):
+    """qsdpa_decode_ext / qsdpa_prefill_ext reject a negative, infinite or NaN
+    softcap and misaligned extension arrays before any launch."""
+    from quantized_kv_attention_split_b200 import qkv
+    ok = _cache(qkv)
+
+    def dec(ext):
+        return lib.qsdpa_decode_ext(FAKE, 0, 1, 8, 2, 128, C.byref(ok), C.byref(ok), 16, 1.0,
+                                    None, C.byref(ext), FAKE + 65536, 0, FAKE + 131072, 1 << 20,
+                                    None)
+
+    def pre(ext):
+        return lib.qsdpa_prefill_ext(FAKE, 0, 1, 8, 2, 4, 128, C.byref(ok), C.byref(ok), 16, 1.0,
+                                     None, C.byref(ext), FAKE + 65536, 0, FAKE + 131072, 1 << 20,
+                                     None)
+    for f in (dec, pre):
+        assert f(qkv._Ext(-1.0, None, None)) == 1
+        assert b"softcap" in lib.qkv_last_error()
+        assert f(qkv._Ext(float("inf"), None, None)) == 1
+        assert f(qkv._Ext(float("nan"), None, None)) == 1
+        assert f(qkv._Ext(0.0, FAKE + 2, None)) == 3           # misaligned slopes
+        assert f(qkv._Ext(30.0, None, FAKE + 6)) == 3          # misaligned sinks

@@ -212,3 +212,12 @@ def test_decode_q8_0_full(qkv, name):
     assert max_err(got, ref) <= TOL["f16"], max_err(got, ref)
     got32 = run_decode(qkv, inp.q, "f16", kc, vc, w.L, w.scale, "f32")
     assert max_err(got32, ref) <= TOL["f32"], max_err(got32, ref)
+
+
+def test_decode_negative_scale():
+    from quantized_kv_attention_split_b200 import qkv
+    q, kc, vc = make_problem(1, 32, 8, 1, 128, 3000, "affine", 4, 64, "normal", seed=7)
+    ref = oracle.attention(q, "f16", kc, vc, 3000, -0.2)
+    out = qkv.qsdpa_decode(to_dev(q, "f16"), cache_to_dev(kc), cache_to_dev(vc), 3000, -0.2)
+    torch.cuda.synchronize()
+    assert out_err(from_dev(out), ref, "f16") <= 1.0

@@ -99,3 +99,44 @@ def test_prefill_q8_0_512_at_20k_sampled(qkv):
     r = ref.reshape(-1, w.D)[rows]
     assert max_err(g, r) <= TOL["bf16"], max_err(g, r)
     assert out_err(g, r, "bf16") <= 1.0
+
+
+@pytest.mark.parametrize("scale", [-0.09, 0.0])
+def test_prefill_negative_and_zero_scale(qkv, scale):
+    """A negative softmax scale flips which keys dominate; the tcgen05 kernel's
+    shortcut of scaling the tile maximum of the raw products holds only for a
+    non-negative scale, so such tiles take the per-element path.  Zero scale
+    gives the mean of the visible values."""
+    B, Hq, Hkv, Lq, D, L = 1, 8, 2, 64, 128, 500
+    q, kc, vc = make_problem(B, Hq, Hkv, Lq, D, L, "affine", 4, 64, "normal", q_dtype="bf16",
+                             Lcap=512, seed=6)
+    for causal in (False, True):
+        mask = oracle.Mask("causal") if causal else None
+        ref = oracle.attention(q, "bf16", kc, vc, L, scale, mask=mask)
+        got = run_prefill(qkv, q, "bf16", kc, vc, L, scale, "f16", causal=causal)
+        assert max_err(got, ref) <= TOL["f16"], max_err(got, ref)
+
+
+@pytest.mark.parametrize("mdt,L", [("f16", 333), ("bf16", 333), ("f16", 512), ("bf16", 520),
+                                   ("f32", 301)])
+def test_prefill_additive_mask_half_dtypes_and_alignment(qkv, mdt, L):
+    """Additive masks in every dtype, on rows that are 16-byte aligned (read
+    16 bytes at a time) and rows that are not (odd L: element reads), with a
+    -inf band and a ragged last tile; tcgen05 kernel (64 rows per kv head)."""
+    B, Hq, Hkv, Lq, D = 1, 8, 2, 16, 128
+    q, kc, vc = make_problem(B, Hq, Hkv, Lq, D, L, "q8_0", 8, 32, "normal", q_dtype="bf16",
+                             Lcap=(L // 8 + 2) * 8, seed=10)
+    rng = np.random.default_rng(4)
+    m32 = rng.standard_normal((Hq, Lq, L)).astype(np.float32)
+    m32[2, :, 50:130] = -np.inf
+    m32[5, 3, :] = -np.inf
+    if mdt == "f32":
+        mb, mt = m32, torch.from_numpy(m32).cuda()
+    else:
+        mb = S.f32_to_half_bits(m32, mdt)
+        mt = to_dev(mb, mdt)
+    st = (0, Lq * L, L)
+    ref = oracle.attention(q, "bf16", kc, vc, L, 0.06, mask=oracle.Mask("additive", mb, mdt, st))
+    got = run_prefill(qkv, q, "bf16", kc, vc, L, 0.06, "f16", mask=(mt, st))
+    assert np.all(got[0, 5, 3] == 0)
+    assert max_err(got, ref) <= TOL["f16"], max_err(got, ref)
