@@ -179,7 +179,10 @@ qkv_status attention(const void* q, int q_dtype, int B, int Hq, int Hkv, int Lq,
   const bool extended = cap_a > 0.f || slopes != nullptr || sinks != nullptr;
   if (fused && extended)
     return fail(QKV_ERR_UNSUPPORTED, "the fused update step takes no attention extensions");
-  const int var = fused ? qkv::kDecFused : extended ? qkv::kDecExt : qkv::kDecPlain;
+  // additive masks run on the extension variant (the plain one carries no
+  // code for them); the fused variant has its own
+  const int var = fused ? qkv::kDecFused
+                        : (extended || mkind == QKV_MASK_ADDITIVE) ? qkv::kDecExt : qkv::kDecPlain;
   if (!qkv::plan_decode(D, k->bits, k->group_size, k->fmt, out_dtype == QKV_F32, var, B,
                         Hkv * rows, Hkv, L, &plan))
     return fail(QKV_ERR_UNSUPPORTED, "no kernel for D=%d bits=%d group_size=%d", D, k->bits,

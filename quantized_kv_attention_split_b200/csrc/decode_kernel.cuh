@@ -295,11 +295,26 @@ __device__ __noinline__ void fused_quantize_patch(const DecodeParams& p, const u
   }
 }
 
+// Additive-mask values of a lane's row for the keys 16 st + 8 r (relative to
+// m) of one block, st < SUB, r < 2; keys at or past nk read nothing (0).  No
+// branch around the loads, so they are in flight together.
+template <int SUB, typename T>
+__device__ __forceinline__ void dec_mask_vals(const T* m, int nk, float (&mv)[SUB][2]) {
+#pragma unroll
+  for (int st = 0; st < SUB; ++st)
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int k = 16 * st + 8 * r;
+      mv[st][r] = k < nk ? to_float_ld(m + k) : 0.f;
+    }
+}
+
 template <int D, int BITS, int GS, bool Q8, int NC, bool F32OUT, int VAR>
 __global__ void __launch_bounds__(32 * dec_warps(D), 1)
 qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
   constexpr bool FUSED = VAR == kDecFused;     // also quantizes the new token into row L - 1
   constexpr bool EXT = VAR == kDecExt;         // logit softcap, mask slopes, sinks
+  constexpr bool ADDMASK = VAR != kDecPlain;   // additive masks (plain: none, or causal)
   using C = DecCfg<D, BITS, GS, Q8, NC>;
   constexpr int NG = C::NG, KPG = C::KPG, MT = C::MT, BK = C::BK, NSTAGE = C::NSTAGE;
   constexpr int NTEAM = C::NTEAM, TTHR = C::TTHR;
@@ -687,27 +702,43 @@ qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
           if (kr0 >= kvalid) { Sx[0] = -INFINITY; Sx[1] = -INFINITY; }
           if (kr0 + 8 >= kvalid) { Sx[2] = -INFINITY; Sx[3] = -INFINITY; }
         }
-        if (p.mask_kind != QKV_MASK_NONE) {
+      }
+      if (p.mask_kind != QKV_MASK_NONE) {
+        // the lane's rows 2t, 2t+1 of its chunk against keys 16 st + g (+ 8):
+        // per row one division, then the block's mask values read together
 #pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            const int vh = hbase + chunk * 8 + 2 * t + j;     // row = head * Lq + query
-            if (vh < p.G) {
-              const int hr = vh / p.Lq, qi = vh - hr * p.Lq;
-              const float slope = kLog2e * (EXT && p.slopes != nullptr ? p.slopes[hkv * p.Gq + hr] : 1.f);
+        for (int j = 0; j < 2; ++j) {
+          const int vh = hbase + chunk * 8 + 2 * t + j;         // row = head * Lq + query
+          const bool rv = vh < p.G;
+          const int hr = rv ? vh / p.Lq : 0, qi = rv ? vh - hr * p.Lq : 0;
+          // the plain variant is never launched with an additive mask
+          if (!ADDMASK || p.mask_kind == QKV_MASK_CAUSAL) {
+            const int64_t last = L - p.Lq + qi - key0 - g;      // last visible key, block-relative
+#pragma unroll
+            for (int st = 0; st < C::SUB; ++st) {
+              if (16 * st > last) Sv[st][j] = -INFINITY;
+              if (16 * st + 8 > last) Sv[st][2 + j] = -INFINITY;
+            }
+          } else if constexpr (ADDMASK) {
+            const float slope = kLog2e * (EXT && p.slopes != nullptr && rv
+                                              ? p.slopes[hkv * p.Gq + hr] : 1.f);
+            const int64_t mrow = (int64_t)b * p.msb + ((int64_t)hkv * p.Gq + hr) * p.msh +
+                                 (int64_t)qi * p.msq + key0 + g;
+            const int nk = rv ? (int)(L - key0 - g < (int64_t)BK ? L - key0 - g : (int64_t)BK) : 0;
+            float mv[C::SUB][2];
+            if (p.mask_dtype == QKV_F32)
+              dec_mask_vals<C::SUB>(reinterpret_cast<const float*>(p.mask) + mrow, nk, mv);
+            else if (p.mask_dtype == QKV_F16)
+              dec_mask_vals<C::SUB>(reinterpret_cast<const __half*>(p.mask) + mrow, nk, mv);
+            else
+              dec_mask_vals<C::SUB>(reinterpret_cast<const __nv_bfloat16*>(p.mask) + mrow, nk, mv);
+#pragma unroll
+            for (int st = 0; st < C::SUB; ++st)
 #pragma unroll
               for (int r = 0; r < 2; ++r) {
-                const int64_t key = key0 + kr0 + 8 * r;
-                if (key >= L) continue;
-                if (p.mask_kind == QKV_MASK_CAUSAL) {
-                  if (key > L - p.Lq + qi) Sx[2 * r + j] = -INFINITY;
-                } else {
-                  const int64_t mi = (int64_t)b * p.msb + ((int64_t)hkv * p.Gq + hr) * p.msh +
-                                     (int64_t)qi * p.msq + key;
-                  const float mv = load_as_float(p.mask, p.mask_dtype, mi);
-                  Sx[2 * r + j] = mv == -INFINITY ? -INFINITY : fmaf(slope, mv, Sx[2 * r + j]);
-                }
+                float& x = Sv[st][2 * r + j];
+                x = mv[st][r] == -INFINITY ? -INFINITY : fmaf(slope, mv[st][r], x);
               }
-            }
           }
         }
       }

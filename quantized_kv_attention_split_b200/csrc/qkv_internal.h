@@ -11,9 +11,10 @@
 namespace qkv {
 
 // Everything one decode launch needs (device pointers and sizes).
-// Decode kernel variants: the plain kernel, the fused update step (also
-// quantizes the new token into cache row L - 1) and the attention extensions
-// (logit softcap, additive-mask slopes, sinks).
+// Decode kernel variants: the plain kernel (no mask, or causal), the fused
+// update step (also quantizes the new token into cache row L - 1; any mask)
+// and the one for additive masks and the attention extensions (logit softcap,
+// additive-mask slopes, sinks).
 enum : int { kDecPlain = 0, kDecFused = 1, kDecExt = 2 };
 
 struct DecodeParams {
