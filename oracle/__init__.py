@@ -227,3 +227,48 @@ def attention_probs(q: np.ndarray, q_dtype: str, k: QCache, v: QCache, L: int,
     if rc:
         raise ValueError("oracle attention_probs: invalid arguments")
     return probs, o
+
+
+# ----------------------------------------------------------------------------
+# llama.cpp-style interleaved Q8_0 blocks <-> the library's planes
+# ----------------------------------------------------------------------------
+# Reading (the pages name the Q8_0 KV format -- llama.cpp PR #25556: one fp16
+# scale per 32 int8 codes -- but not its bytes): the GGUF Q8_0 block, 34 bytes,
+# the fp16 scale first (little-endian), then the 32 codes in element order as
+# two's-complement bytes.  Plain numpy, element by element in its arithmetic.
+Q8_0_BLOCK_BYTES = 34
+
+
+def q8_0_to_blocks(c: QCache, L: int) -> np.ndarray:
+    """Rows [0, L) of a Q8_0 cache -> blocks uint8 [B, Hkv, L, D/32, 34]."""
+    assert c.fmt == "q8_0"
+    B, Hkv, _, W = c.codes.shape
+    nb = W * 4 // 32
+    words = c.codes[:, :, :L].astype(np.uint64)             # [B,Hkv,L,W]
+    scales = c.scales[:, :, :L].astype(np.uint64)           # [B,Hkv,L,nb]
+    out = np.zeros((B, Hkv, L, nb, Q8_0_BLOCK_BYTES), np.uint8)
+    out[..., 0] = scales & 0xFF
+    out[..., 1] = scales >> 8
+    for e in range(32):                                     # element e of each block
+        for g in range(nb):
+            d = 32 * g + e                                  # element index in the row
+            out[:, :, :, g, 2 + e] = (words[..., d // 4] >> (8 * (d % 4))) & 0xFF
+    return out
+
+
+def q8_0_from_blocks(blocks: np.ndarray, Lcap: Optional[int] = None) -> QCache:
+    """Blocks uint8 [B, Hkv, L, D/32, 34] -> a Q8_0 cache with Lcap rows (rows
+    past L zero)."""
+    B, Hkv, L, nb, nbytes = blocks.shape
+    assert nbytes == Q8_0_BLOCK_BYTES
+    Lcap = Lcap or L
+    D = 32 * nb
+    codes = np.zeros((B, Hkv, Lcap, D // 4), np.uint32)
+    scales = np.zeros((B, Hkv, Lcap, nb), np.uint16)
+    b = blocks.astype(np.uint32)
+    scales[:, :, :L] = b[..., 0] | (b[..., 1] << 8)
+    for g in range(nb):
+        for e in range(32):
+            d = 32 * g + e
+            codes[:, :, :L, d // 4] |= b[:, :, :, g, 2 + e] << (8 * (d % 4))
+    return QCache("q8_0", 8, 32, codes, scales, None)
