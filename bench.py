@@ -517,6 +517,25 @@ def other_rows(device):
         nb = w.cache_bytes() + 2 * w.Hq * w.D * 2
         rows[name] = {"us_per_call": round(sec * 1e3, 3), "GB/s": round(nb / (sec / 1e3) / 1e9, 1),
                       "frac_hbm": round(nb / (sec / 1e3) / 1e9 / hbm_peak, 4)}
+        if name == "decode_q8_0_20k":
+            # llama.cpp-style interleaved blocks <-> planes for this cache (K and V)
+            a, b = caches[0]
+            bk = qkv.qkv_q8_0_to_blocks(a, w.L)
+            bv = qkv.qkv_q8_0_to_blocks(b, w.L)
+            sec_f, _ = graph_time(lambda i: (qkv.qkv_q8_0_from_blocks(bk, a),
+                                             qkv.qkv_q8_0_from_blocks(bv, b)), 200, 10)
+            sec_t, _ = graph_time(lambda i: (qkv.qkv_q8_0_to_blocks(a, w.L, out=bk),
+                                             qkv.qkv_q8_0_to_blocks(b, w.L, out=bv)), 200, 10)
+            moved = 2 * (bk.numel() + w.cache_bytes() // 2)     # read one form, write the other
+            rows["q8_0_blocks_20k"] = {
+                "from_blocks_us": round(sec_f * 1e3, 3), "to_blocks_us": round(sec_t * 1e3, 3),
+                "from_GB/s": round(moved / (sec_f / 1e3) / 1e9, 1),
+                "to_GB/s": round(moved / (sec_t / 1e3) / 1e9, 1),
+                "frac_hbm_from": round(moved / (sec_f / 1e3) / 1e9 / hbm_peak, 4),
+                "note": "K and V of decode_q8_0_20k (2 x 11.1 MB of planes, 2 x 11.1 MB of "
+                        "34-byte blocks): qkv_q8_0_from_blocks / qkv_q8_0_to_blocks; the data "
+                        "fit in L2"}
+            del bk, bv
         del caches
         torch.cuda.empty_cache()
 

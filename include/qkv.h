@@ -209,6 +209,26 @@ qkv_status qsdpa_prefill_ext(const void* q, int q_dtype, int B, int Hq, int Hkv,
 qkv_status qkv_dequantize(const qkv_cache* c, int B, int Hkv, int D, int64_t L, void* out,
                           void* stream);
 
+/* Conversion between llama.cpp-style interleaved Q8_0 blocks and this
+ * library's Q8_0 planes, bit for bit (llama.cpp #25556 keeps its KV cache in
+ * Q8_0 blocks; their byte layout, not shown on the pages, is the GGUF Q8_0
+ * block: 34 bytes, the fp16 scale first (little-endian), then the 32 int8
+ * codes in element order).  A row of D elements (b, kv head, token l) is D/32
+ * consecutive blocks starting at byte b*stride_b + h*stride_h + l*stride_l of
+ * `blocks` (llama.cpp's token-major K cache: stride_l = Hkv*D/32*34,
+ * stride_h = D/32*34).  blocks and the strides must be 2-byte aligned.
+ *  qkv_q8_0_from_blocks: writes tokens [0, L) of the blocks into cache rows
+ *    [offset, offset + L) of dst (a Q8_0 qkv_cache); 0 <= offset, offset + L <= Lcap.
+ *  qkv_q8_0_to_blocks: writes cache rows [offset, offset + L) of src into
+ *    tokens [0, L) of the blocks; destination rows must not overlap.
+ * One launch each; L == 0 does nothing. */
+qkv_status qkv_q8_0_from_blocks(const void* blocks, int B, int Hkv, int D, int64_t L,
+                                int64_t stride_b, int64_t stride_h, int64_t stride_l,
+                                const qkv_cache* dst, int64_t offset, void* stream);
+qkv_status qkv_q8_0_to_blocks(const qkv_cache* src, int B, int Hkv, int D, int64_t offset,
+                              int64_t L, void* blocks, int64_t stride_b, int64_t stride_h,
+                              int64_t stride_l, void* stream);
+
 /* Allocation-free variant of qsdpa_decode (the pages have no counterpart:
  * MLX and llama.cpp allocate their temporaries through their own allocators).
  * For callers that cannot allocate device memory when they decode -- code

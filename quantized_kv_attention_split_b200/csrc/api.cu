@@ -292,6 +292,48 @@ qkv_status qkv_dequantize(const qkv_cache* c, int B, int Hkv, int D, int64_t L, 
   return ok();
 }
 
+namespace {
+qkv_status check_blocks_args(const qkv_cache* c, int B, int Hkv, int D, int64_t offset, int64_t L,
+                             const void* blocks, int64_t sb, int64_t sh, int64_t sl) {
+  qkv_status st;
+  if ((st = check_cache("cache", c, D)) != QKV_OK) return st;
+  if (c->fmt != QKV_Q8_0) return fail(QKV_ERR_UNSUPPORTED, "block conversion is for Q8_0 caches");
+  if (B <= 0 || Hkv <= 0) return fail(QKV_ERR_INVALID_ARG, "B and Hkv must be positive");
+  if (offset < 0 || L < 0 || offset + L > c->Lcap)
+    return fail(QKV_ERR_INVALID_ARG, "rows [%lld, %lld) outside [0, Lcap]", (long long)offset,
+                (long long)(offset + L));
+  if (blocks == nullptr) return fail(QKV_ERR_INVALID_ARG, "blocks must be non-NULL");
+  if (sb < 0 || sh < 0 || sl < 0) return fail(QKV_ERR_INVALID_ARG, "block strides must be non-negative");
+  if ((reinterpret_cast<uintptr_t>(blocks) & 1u) != 0 || ((sb | sh | sl) & 1) != 0)
+    return fail(QKV_ERR_ALIGNMENT, "blocks and their strides must be 2-byte aligned");
+  return QKV_OK;
+}
+}  // namespace
+
+qkv_status qkv_q8_0_from_blocks(const void* blocks, int B, int Hkv, int D, int64_t L,
+                                int64_t stride_b, int64_t stride_h, int64_t stride_l,
+                                const qkv_cache* dst, int64_t offset, void* stream) {
+  qkv_status st = check_blocks_args(dst, B, Hkv, D, offset, L, blocks, stride_b, stride_h, stride_l);
+  if (st != QKV_OK) return st;
+  if (L == 0) return ok();
+  cudaError_t e = qkv::launch_q8_0_blocks(false, blocks, nullptr, dst, B, Hkv, D, offset, L, stride_b,
+                                          stride_h, stride_l, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(QKV_ERR_CUDA, "block conversion launch: %s", cudaGetErrorString(e));
+  return ok();
+}
+
+qkv_status qkv_q8_0_to_blocks(const qkv_cache* src, int B, int Hkv, int D, int64_t offset, int64_t L,
+                              void* blocks, int64_t stride_b, int64_t stride_h, int64_t stride_l,
+                              void* stream) {
+  qkv_status st = check_blocks_args(src, B, Hkv, D, offset, L, blocks, stride_b, stride_h, stride_l);
+  if (st != QKV_OK) return st;
+  if (L == 0) return ok();
+  cudaError_t e = qkv::launch_q8_0_blocks(true, nullptr, blocks, src, B, Hkv, D, offset, L, stride_b,
+                                          stride_h, stride_l, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(QKV_ERR_CUDA, "block conversion launch: %s", cudaGetErrorString(e));
+  return ok();
+}
+
 qkv_status qsdpa_decode(const void* q, int q_dtype, int B, int Hq, int Hkv, int D,
                         const qkv_cache* k, const qkv_cache* v, int64_t L, float scale,
                         const qkv_mask* mask, void* out, int out_dtype, void* workspace,

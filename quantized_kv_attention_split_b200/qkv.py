@@ -81,6 +81,10 @@ def lib() -> C.CDLL:
         L.qsdpa_decode_update.argtypes = [p, i32, p, p, i32, i32, i32, i32, i32, cp, cp, i64,
                                           C.c_float, mp, p, i32, p, sz, p]
         L.qsdpa_decode_update.restype = i32
+        L.qkv_q8_0_from_blocks.argtypes = [p, i32, i32, i32, i64, i64, i64, i64, cp, i64, p]
+        L.qkv_q8_0_from_blocks.restype = i32
+        L.qkv_q8_0_to_blocks.argtypes = [cp, i32, i32, i32, i64, i64, p, i64, i64, i64, p]
+        L.qkv_q8_0_to_blocks.restype = i32
         L.qkv_dequantize.argtypes = [cp, i32, i32, i32, i64, p, p]
         L.qkv_dequantize.restype = i32
         L.qsdpa_workspace_size.argtypes = [i32, i32, i32, i32, i32, i64]
@@ -178,6 +182,51 @@ def qkv_dequantize(c: QuantCache, L: int, out: Optional[torch.Tensor] = None,
     assert out.is_contiguous() and out.dtype == torch.float16 and tuple(out.shape) == (B, Hkv, L, D)
     cs = c._struct()
     _check(lib().qkv_dequantize(C.byref(cs), B, Hkv, D, int(L), out.data_ptr(), _stream(stream)))
+    return out
+
+
+Q8_0_BLOCK_BYTES = 34
+
+
+def _block_strides(blocks: torch.Tensor, strides):
+    """Byte strides (b, kv head, token) of a uint8 block tensor [B,Hkv,L,D/32*34]
+    (or [B,L,Hkv,D/32*34] when given explicitly as `strides`)."""
+    if strides is not None:
+        return tuple(int(x) for x in strides)
+    s = blocks.stride()
+    return s[0], s[1], s[2]
+
+
+def qkv_q8_0_from_blocks(blocks: torch.Tensor, c: QuantCache, offset: int = 0,
+                         L: Optional[int] = None, strides=None, stream=None) -> QuantCache:
+    """Write llama.cpp-style Q8_0 blocks (uint8 CUDA tensor, by default
+    [B, Hkv, L, D/32*34]; other layouts through `strides` = byte strides of
+    (b, kv head, token) and an explicit L) into cache rows [offset, offset+L)."""
+    assert blocks.dtype == torch.uint8 and blocks.is_cuda and c.fmt == Q8_0
+    B, Hkv, D = c.codes.shape[0], c.codes.shape[1], c.codes.shape[3] * 4
+    if L is None:
+        L = blocks.shape[2]
+    sb, sh, sl = _block_strides(blocks, strides)
+    cs = c._struct()
+    _check(lib().qkv_q8_0_from_blocks(blocks.data_ptr(), B, Hkv, D, int(L), sb, sh, sl,
+                                      C.byref(cs), int(offset), _stream(stream)))
+    return c
+
+
+def qkv_q8_0_to_blocks(c: QuantCache, L: int, offset: int = 0,
+                       out: Optional[torch.Tensor] = None, strides=None,
+                       stream=None) -> torch.Tensor:
+    """Cache rows [offset, offset+L) of a Q8_0 cache as llama.cpp-style blocks
+    (uint8, [B, Hkv, L, D/32*34] unless `out` and `strides` say otherwise)."""
+    assert c.fmt == Q8_0
+    B, Hkv, D = c.codes.shape[0], c.codes.shape[1], c.codes.shape[3] * 4
+    if out is None:
+        out = torch.empty(B, Hkv, L, D // 32 * Q8_0_BLOCK_BYTES, dtype=torch.uint8,
+                          device=c.codes.device)
+    sb, sh, sl = _block_strides(out, strides)
+    cs = c._struct()
+    _check(lib().qkv_q8_0_to_blocks(C.byref(cs), B, Hkv, D, int(offset), int(L), out.data_ptr(),
+                                    sb, sh, sl, _stream(stream)))
     return out
 
 

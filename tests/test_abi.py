@@ -146,3 +146,19 @@ def test_extension_validation_errors(lib):
         assert f(qkv._Ext(float("nan"), None, None)) == 1
         assert f(qkv._Ext(0.0, FAKE + 2, None)) == 3           # misaligned slopes
         assert f(qkv._Ext(30.0, None, FAKE + 6)) == 3          # misaligned sinks
+
+
+def test_block_conversion_validation_errors(lib):
+    from quantized_kv_attention_split_b200 import qkv
+    q8 = _cache(qkv, fmt=1, bits=8, gs=32, biases=0)
+    fb, tb = lib.qkv_q8_0_from_blocks, lib.qkv_q8_0_to_blocks
+    st = (64 * 4 * 34, 4 * 34, 2 * 4 * 34)                      # token-major, Hkv 2, D 128
+    assert fb(FAKE, 1, 2, 128, 16, *st, C.byref(_cache(qkv)), 0, None) == 2   # not Q8_0
+    assert fb(FAKE, 1, 2, 128, 16, *st, C.byref(q8), 60, None) == 1           # past Lcap
+    assert b"Lcap" in lib.qkv_last_error()
+    assert fb(FAKE + 1, 1, 2, 128, 16, *st, C.byref(q8), 0, None) == 3        # odd address
+    assert fb(FAKE, 1, 2, 128, 16, 1, 136, 272, C.byref(q8), 0, None) == 3    # odd stride
+    assert fb(0, 1, 2, 128, 16, *st, C.byref(q8), 0, None) == 1               # NULL blocks
+    assert tb(C.byref(q8), 1, 2, 128, -1, 4, FAKE, *st, None) == 1            # negative offset
+    assert tb(C.byref(q8), 1, 2, 96, 0, 4, FAKE, *st, None) == 2              # unsupported D
+    assert tb(C.byref(q8), 1, 2, 128, 0, 0, FAKE, *st, None) == 0             # nothing to do

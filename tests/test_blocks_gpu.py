@@ -1,0 +1,65 @@
+"""llama.cpp-style interleaved Q8_0 blocks <-> the library's Q8_0 planes through
+the C ABI (qkv_q8_0_from_blocks / qkv_q8_0_to_blocks): bit-exact against the
+oracle's conversion, in llama.cpp's token-major layout and head-major, at an
+offset into the cache, and as the input of a decode call."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from helpers import cache_from_dev, cache_to_dev, from_dev, make_problem, out_err, to_dev
+from quantized_kv_attention_split_b200 import synthetic as S
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("shift", [0, 2])
+@pytest.mark.parametrize("B,Hkv,D,L", [(1, 2, 256, 777), (2, 3, 64, 40), (1, 8, 128, 1)])
+def test_blocks_round_trip_token_major(B, Hkv, D, L, shift):
+    """shift 0: 4-byte aligned blocks (moved in pairs, 32-bit words); shift 2:
+    2-byte aligned only (moved block by block, 16-bit units)."""
+    from quantized_kv_attention_split_b200 import qkv
+    x = S.draw(61, "x", (B, Hkv, L, D), "normal", "f16")
+    c = oracle.quantize(x, "f16", "q8_0")
+    blocks = oracle.q8_0_to_blocks(c, L)                       # [B,Hkv,L,nb,34]
+    nb = D // 32
+    # llama.cpp keeps K as [token][kv head][blocks]: token-major bytes
+    tm = np.ascontiguousarray(blocks.transpose(0, 2, 1, 3, 4)).reshape(B, L, Hkv * nb * 34)
+    flat = torch.zeros(tm.size + 16, dtype=torch.uint8, device="cuda")
+    dev = flat[shift:shift + tm.size].view(B, L, Hkv * nb * 34)
+    dev.copy_(torch.from_numpy(tm).cuda())
+    st = (L * Hkv * nb * 34, nb * 34, Hkv * nb * 34)
+    off = 5
+    Lcap = ((off + L) // 8 + 1) * 8
+    dc = qkv.QuantCache.empty(B, Hkv, Lcap, D, qkv.Q8_0)
+    qkv.qkv_q8_0_from_blocks(dev, dc, offset=off, L=L, strides=st)
+    torch.cuda.synchronize()
+    h = cache_from_dev(dc, "q8_0")
+    assert np.array_equal(h.codes[:, :, off:off + L], c.codes)
+    assert np.array_equal(h.scales[:, :, off:off + L], c.scales)
+    assert not h.codes[:, :, :off].any() and not h.codes[:, :, off + L:].any()
+    flat2 = torch.zeros(tm.size + 16, dtype=torch.uint8, device="cuda")
+    back = flat2[shift:shift + tm.size].view(B, L, Hkv * nb * 34)
+    qkv.qkv_q8_0_to_blocks(dc, L, offset=off, out=back, strides=st)
+    torch.cuda.synchronize()
+    assert torch.equal(back, dev)
+    assert not flat2[:shift].any() and not flat2[shift + tm.size:].any()   # nothing written outside
+
+
+def test_blocks_head_major_default_layout_and_decode():
+    """Blocks in the default [B, Hkv, L, D/32*34] layout become a cache that the
+    decode kernel reads like any other."""
+    from quantized_kv_attention_split_b200 import qkv
+    B, Hq, Hkv, D, L = 1, 32, 2, 256, 3000
+    q, kc, vc = make_problem(B, Hq, Hkv, 1, D, L, "q8_0", 8, 32, "normal", seed=62)
+    bk = torch.from_numpy(oracle.q8_0_to_blocks(kc, L).reshape(B, Hkv, L, -1)).cuda()
+    bv = torch.from_numpy(oracle.q8_0_to_blocks(vc, L).reshape(B, Hkv, L, -1)).cuda()
+    dk = qkv.QuantCache.empty(B, Hkv, kc.Lcap, D, qkv.Q8_0)
+    dv = qkv.QuantCache.empty(B, Hkv, kc.Lcap, D, qkv.Q8_0)
+    qkv.qkv_q8_0_from_blocks(bk, dk)
+    qkv.qkv_q8_0_from_blocks(bv, dv)
+    out = qkv.qsdpa_decode(to_dev(q, "f16"), dk, dv, L, 1.0 / 16)
+    torch.cuda.synchronize()
+    ref = oracle.attention(q, "f16", kc, vc, L, 1.0 / 16)
+    assert out_err(from_dev(out), ref, "f16") <= 1.0
+    assert torch.equal(qkv.qkv_q8_0_to_blocks(dk, L), bk)
