@@ -1001,28 +1001,46 @@ qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
     //  4-bit, groups >= 64: unit pair i/4, nibble i%4 -> dims 64(i/4)+4g+i%4, +32
     //  4-bit, groups of 32: nibble i -> dims 4g+i and 4g+i+2
     //  8-bit: unit pair i/2, byte i%2 -> dims 32(i/2)+2g+i%2, +16
-    for (int idx = tid; idx < HPC * D; idx += C::NTHR) {
+    // A thread takes 4 consecutive elements (j = 0..3 of one lane's m-tile):
+    // rows R0 = c*8 + 2*tl and R0 + 1, dims dim and dim + dj; one float4 read
+    // per team and four independent sums.
+    for (int q4 = tid; q4 < HPC * D / 4; q4 += C::NTHR) {
+      const int idx = 4 * q4;
       const int c = idx / (8 * D), r = idx - c * 8 * D;
-      const int mt = r >> 7, lj = r & 127, gl = lj >> 4, tl = (lj >> 2) & 3, j = lj & 3;
-      const int R = c * 8 + 2 * tl + (j & 1);
-      const int head = hbase + R;
+      const int mt = r >> 7, lj = r & 127, gl = lj >> 4, tl = (lj >> 2) & 3;
+      const int R0 = c * 8 + 2 * tl;
+      const int head = hbase + R0;
       if (head >= p.G) continue;
+      const bool v1 = head + 1 < p.G;
       const int G = mt / KPG, i = mt % KPG;
-      int dim;
-      if constexpr (BITS == 4 && GS == 32) dim = G * GS + 4 * gl + i + (j >= 2 ? 2 : 0);
-      else if constexpr (BITS == 4) dim = G * GS + 64 * (i >> 2) + 4 * gl + (i & 3) + (j >= 2 ? 32 : 0);
-      else dim = G * GS + 32 * (i >> 1) + 2 * gl + (i & 1) + (j >= 2 ? 16 : 0);
-      float o = 0.f;
+      int dim, dj;
+      if constexpr (BITS == 4 && GS == 32) { dim = G * GS + 4 * gl + i; dj = 2; }
+      else if constexpr (BITS == 4) { dim = G * GS + 64 * (i >> 2) + 4 * gl + (i & 3); dj = 32; }
+      else { dim = G * GS + 32 * (i >> 1) + 2 * gl + (i & 1); dj = 16; }
+      float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-      for (int k = 0; k < NTEAM; ++k) o = fmaf(wgt[R * WST + k], wsf[(k * NC + c) * C::WSW + r], o);
+      for (int k = 0; k < NTEAM; ++k) {
+        const float4 x = *reinterpret_cast<const float4*>(wsf + (k * NC + c) * C::WSW + r);
+        const float w0 = wgt[R0 * WST + k], w1 = wgt[(R0 + 1) * WST + k];
+        o.x = fmaf(w0, x.x, o.x); o.y = fmaf(w1, x.y, o.y);
+        o.z = fmaf(w0, x.z, o.z); o.w = fmaf(w1, x.w, o.w);
+      }
       if (complete) {
         const int64_t oi = (uh * p.G + head) * D + dim;
-        store_from_float(p.out, p.out_dtype, oi, o);
+        store_from_float(p.out, p.out_dtype, oi, o.x);
+        store_from_float(p.out, p.out_dtype, oi + dj, o.z);
+        if (v1) {
+          store_from_float(p.out, p.out_dtype, oi + D, o.y);
+          store_from_float(p.out, p.out_dtype, oi + D + dj, o.w);
+        }
       } else {
-        p.part_o[(pslot * HPC + R) * D + dim] = o;
+        float* po = p.part_o + (pslot * HPC + R0) * D + dim;
+        po[0] = o.x; po[dj] = o.z;
+        if (v1) { po[D] = o.y; po[D + dj] = o.w; }
         if (dim == 0) {
-          p.part_ml[(pslot * HPC + R) * 2 + 0] = rml[2 * R];
-          p.part_ml[(pslot * HPC + R) * 2 + 1] = rml[2 * R + 1];
+          float* pm = p.part_ml + (pslot * HPC + R0) * 2;
+          pm[0] = rml[2 * R0]; pm[1] = rml[2 * R0 + 1];
+          if (v1) { pm[2] = rml[2 * R0 + 2]; pm[3] = rml[2 * R0 + 3]; }
         }
       }
     }
