@@ -272,3 +272,78 @@ def q8_0_from_blocks(blocks: np.ndarray, Lcap: Optional[int] = None) -> QCache:
             d = 32 * g + e
             codes[:, :, :L, d // 4] |= b[:, :, :, g, 2 + e] << (8 * (d % 4))
     return QCache("q8_0", 8, 32, codes, scales, None)
+
+
+# llama.cpp's other block formats (the PR's follow-up extends its conversion to
+# Q4_0, Q4_1, Q5_0 and Q5_1; their bytes, not on the pages, are the GGUF
+# blocks).  Reading: blocks of 32 elements, little-endian fp16 fields first;
+#   Q4_0: d, qs[16]            x = d * (q - 8)
+#   Q4_1: d, m, qs[16]         x = d * q + m
+#   Q5_0: d, qh[4], qs[16]     x = d * (q - 16)
+#   Q5_1: d, m, qh[4], qs[16]  x = d * q + m
+# element j < 16 is the low nibble of qs[j], element j + 16 its high nibble;
+# Q5's fifth bit of element e is bit e of qh (a little-endian 32-bit word).
+# In the library they become affine caches with groups of 32: 4-bit codes for
+# Q4 (bias -8d for Q4_0), 8-bit codes for Q5 (bias -16d for Q5_0).
+LLAMA_BLOCKS = {  # name: (bytes, has m, has qh, code offset, cache bits)
+    "q4_0": (18, False, False, 8, 4),
+    "q4_1": (20, True, False, 0, 4),
+    "q5_0": (22, False, True, 16, 8),
+    "q5_1": (24, True, True, 0, 8),
+}
+
+
+def _llama_fields(kind: str, blocks: np.ndarray):
+    nbytes, has_m, has_qh, off, _ = LLAMA_BLOCKS[kind]
+    assert blocks.shape[-1] == nbytes
+    b = blocks.astype(np.uint32)
+    d = b[..., 0] | (b[..., 1] << 8)
+    pos = 2
+    m = None
+    if has_m:
+        m = b[..., pos] | (b[..., pos + 1] << 8)
+        pos += 2
+    qh = None
+    if has_qh:
+        qh = b[..., pos] | (b[..., pos + 1] << 8) | (b[..., pos + 2] << 16) | (b[..., pos + 3] << 24)
+        pos += 4
+    q = np.zeros(blocks.shape[:-1] + (32,), np.uint32)
+    for j in range(16):
+        q[..., j] = b[..., pos + j] & 0xF
+        q[..., j + 16] = b[..., pos + j] >> 4
+    if has_qh:
+        for e in range(32):
+            q[..., e] |= ((qh >> e) & 1) << 4
+    return d.astype(np.uint16), None if m is None else m.astype(np.uint16), q, off
+
+
+def llama_block_values(kind: str, blocks: np.ndarray) -> np.ndarray:
+    """Exact values (fp64) of blocks uint8 [..., nb, bytes] -> [..., nb * 32]."""
+    d, m, q, off = _llama_fields(kind, blocks)
+    dv = f16_to_f32(d).astype(np.float64)[..., None]
+    x = dv * (q.astype(np.float64) - off)
+    if m is not None:
+        x = x + f16_to_f32(m).astype(np.float64)[..., None]
+    return x.reshape(blocks.shape[:-2] + (-1,))
+
+
+def llama_blocks_to_cache(kind: str, blocks: np.ndarray, Lcap: Optional[int] = None) -> QCache:
+    """Blocks uint8 [B, Hkv, L, nb, bytes] -> the affine cache (groups of 32)
+    that holds the same values: scale d, bias m (or -off * d, exact in fp16)."""
+    B, Hkv, L, nb, _ = blocks.shape
+    bits = LLAMA_BLOCKS[kind][4]
+    Lcap = Lcap or L
+    D = 32 * nb
+    d, m, q, off = _llama_fields(kind, blocks)
+    if m is None:
+        m = f32_to_f16((-off * f16_to_f32(d).astype(np.float64)).astype(np.float32))
+    codes = np.zeros((B, Hkv, Lcap, D * bits // 32), np.uint32)
+    per = 32 // bits
+    qq = q.reshape(B, Hkv, L, D)
+    for e in range(D):
+        codes[:, :, :L, e // per] |= qq[..., e] << (bits * (e % per))
+    scales = np.zeros((B, Hkv, Lcap, nb), np.uint16)
+    biases = np.zeros((B, Hkv, Lcap, nb), np.uint16)
+    scales[:, :, :L] = d
+    biases[:, :, :L] = m
+    return QCache("affine", bits, 32, codes, scales, biases)

@@ -41,3 +41,38 @@ def test_round_trips(orc):
     rng = np.random.default_rng(0)
     raw = rng.integers(0, 256, (2, 1, 5, 4, 34), dtype=np.uint8)
     assert np.array_equal(orc.q8_0_to_blocks(orc.q8_0_from_blocks(raw, Lcap=8), 5), raw)
+
+
+import pytest
+
+
+@pytest.mark.parametrize("kind", ["q4_0", "q4_1", "q5_0", "q5_1"])
+def test_llama_block_golden_values(orc, kind):
+    g = read_golden("llama_blocks.txt")
+    raw = np.array([int(x, 16) for x in g[kind + "_block"]], np.uint8).reshape(1, 1, 1, 1, -1)
+    want = np.array([float(v) for v in g[kind + "_values"]])
+    assert np.array_equal(orc.llama_block_values(kind, raw).ravel(), want)
+    # the affine cache it becomes holds exactly these values
+    c = orc.llama_blocks_to_cache(kind, raw)
+    assert c.bits == (4 if kind.startswith("q4") else 8) and c.gs == 32
+    assert np.array_equal(orc.dequantize(c, 32).ravel(), want)
+
+
+@pytest.mark.parametrize("kind", ["q4_0", "q4_1", "q5_0", "q5_1"])
+def test_llama_blocks_to_cache_keeps_every_value(orc, kind):
+    nbytes = orc.LLAMA_BLOCKS[kind][0]
+    rng = np.random.default_rng(7)
+    B, Hkv, L, nb = 2, 3, 9, 4
+    raw = rng.integers(0, 256, (B, Hkv, L, nb, nbytes), dtype=np.uint8)
+    # finite fp16 d (and m): drawn values, stored little-endian
+    d = S.f32_to_half_bits(rng.uniform(-3, 3, (B, Hkv, L, nb)).astype(np.float32), "f16")
+    raw[..., 0] = d & 0xFF
+    raw[..., 1] = d >> 8
+    if orc.LLAMA_BLOCKS[kind][1]:
+        m = S.f32_to_half_bits(rng.uniform(-3, 3, (B, Hkv, L, nb)).astype(np.float32), "f16")
+        raw[..., 2] = m & 0xFF
+        raw[..., 3] = m >> 8
+    c = orc.llama_blocks_to_cache(kind, raw, Lcap=16)
+    vals = orc.llama_block_values(kind, raw)
+    assert np.array_equal(orc.dequantize(c, 32 * nb)[:, :, :L], vals)
+    assert not c.codes[:, :, L:].any()
