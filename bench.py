@@ -611,6 +611,30 @@ def other_rows(device):
         rows["materialize_decode_64k_affine4"] = {"unavailable": f"{type(e).__name__}: {e}"[:200]}
     torch.cuda.empty_cache()
 
+    # llama.cpp Q4_0 blocks of the main decode shape (K and V, 65536 tokens,
+    # token-major) into 4-bit affine caches with groups of 32
+    try:
+        w = S.WORKLOADS["decode_64k_affine4"]
+        nbk = w.D // 32
+        blk = torch.randint(0, 256, (w.B, w.L, w.Hkv * nbk * 18), dtype=torch.uint8, device=device)
+        blk.view(w.B, w.L, w.Hkv, nbk, 18)[..., 1] = 0x2C        # finite fp16 scales
+        st = (w.L * w.Hkv * nbk * 18, nbk * 18, w.Hkv * nbk * 18)
+        dk = qkv.QuantCache.empty(w.B, w.Hkv, w.L, w.D, qkv.AFFINE, 4, 32, device)
+        dv = qkv.QuantCache.empty(w.B, w.Hkv, w.L, w.D, qkv.AFFINE, 4, 32, device)
+        sec, _ = graph_time(lambda i: (qkv.qkv_llama_blocks_to_cache("q4_0", blk, dk, L=w.L, strides=st),
+                                       qkv.qkv_llama_blocks_to_cache("q4_0", blk, dv, L=w.L, strides=st)),
+                            100, 5)
+        moved = 2 * (blk.numel() + w.B * w.Hkv * w.L * nbk * 20)
+        rows["llama_q4_0_blocks_64k"] = {
+            "us_per_call": round(sec * 1e3, 3), "GB/s": round(moved / (sec / 1e3) / 1e9, 1),
+            "frac_hbm": round(moved / (sec / 1e3) / 1e9 / hbm_peak, 4),
+            "note": "qkv_llama_blocks_to_cache, Q4_0 blocks (token-major, 2 x 37.7 MB) into K "
+                    "and V 4-bit affine caches with groups of 32 (2 x 41.9 MB)"}
+        del blk, dk, dv
+    except Exception as e:
+        rows["llama_q4_0_blocks_64k"] = {"unavailable": f"{type(e).__name__}: {e}"[:200]}
+    torch.cuda.empty_cache()
+
     # the attention extensions on the main decode workload (the extension
     # variant of the decode kernel): logit softcap 30 with per-head sinks, and
     # ALiBi (a broadcast fp32 distance mask with per-head slopes)

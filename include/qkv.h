@@ -229,6 +229,26 @@ qkv_status qkv_q8_0_to_blocks(const qkv_cache* src, int B, int Hkv, int D, int64
                               int64_t L, void* blocks, int64_t stride_b, int64_t stride_h,
                               int64_t stride_l, void* stream);
 
+/* llama.cpp's other KV block formats into an affine cache with groups of 32
+ * that holds exactly the same values (the PR's follow-up extends its KV
+ * conversion to these types; their bytes, not on the pages, are the GGUF
+ * blocks of 32 elements, little-endian fp16 fields first):
+ *   QKV_BLOCKS_Q4_0  18 bytes: d, qs[16]            x = d (q - 8)   -> 4-bit cache, bias -8d
+ *   QKV_BLOCKS_Q4_1  20 bytes: d, m, qs[16]         x = d q + m     -> 4-bit cache, bias m
+ *   QKV_BLOCKS_Q5_0  22 bytes: d, qh[4], qs[16]     x = d (q - 16)  -> 8-bit cache, bias -16d
+ *   QKV_BLOCKS_Q5_1  24 bytes: d, m, qh[4], qs[16]  x = d q + m     -> 8-bit cache, bias m
+ * (element j < 16 in the low nibble of qs[j], element j + 16 in its high
+ * nibble; the fifth bit of element e is bit e of qh).  dst: affine, group_size
+ * 32, bits 4 for Q4 and 8 for Q5.  Rows, strides, offset and alignment as for
+ * qkv_q8_0_from_blocks (with the block sizes above).  The decode and prefill
+ * calls then read the cache like any affine cache.  One launch. */
+typedef enum { QKV_BLOCKS_Q4_0 = 0, QKV_BLOCKS_Q4_1 = 1, QKV_BLOCKS_Q5_0 = 2,
+               QKV_BLOCKS_Q5_1 = 3 } qkv_block_kind;
+qkv_status qkv_llama_blocks_to_cache(int kind, const void* blocks, int B, int Hkv, int D,
+                                     int64_t L, int64_t stride_b, int64_t stride_h,
+                                     int64_t stride_l, const qkv_cache* dst, int64_t offset,
+                                     void* stream);
+
 /* Allocation-free variant of qsdpa_decode (the pages have no counterpart:
  * MLX and llama.cpp allocate their temporaries through their own allocators).
  * For callers that cannot allocate device memory when they decode -- code

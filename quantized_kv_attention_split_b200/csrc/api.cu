@@ -294,10 +294,15 @@ qkv_status qkv_dequantize(const qkv_cache* c, int B, int Hkv, int D, int64_t L, 
 
 namespace {
 qkv_status check_blocks_args(const qkv_cache* c, int B, int Hkv, int D, int64_t offset, int64_t L,
-                             const void* blocks, int64_t sb, int64_t sh, int64_t sl) {
+                             const void* blocks, int64_t sb, int64_t sh, int64_t sl,
+                             int want_fmt = QKV_Q8_0, int want_bits = 8) {
   qkv_status st;
   if ((st = check_cache("cache", c, D)) != QKV_OK) return st;
-  if (c->fmt != QKV_Q8_0) return fail(QKV_ERR_UNSUPPORTED, "block conversion is for Q8_0 caches");
+  if (want_fmt == QKV_Q8_0 && c->fmt != QKV_Q8_0)
+    return fail(QKV_ERR_UNSUPPORTED, "Q8_0 block conversion needs a Q8_0 cache");
+  if (want_fmt == QKV_AFFINE && (c->fmt != QKV_AFFINE || c->group_size != 32 || c->bits != want_bits))
+    return fail(QKV_ERR_UNSUPPORTED, "these blocks need an affine cache with group_size 32 and %d-bit codes",
+                want_bits);
   if (B <= 0 || Hkv <= 0) return fail(QKV_ERR_INVALID_ARG, "B and Hkv must be positive");
   if (offset < 0 || L < 0 || offset + L > c->Lcap)
     return fail(QKV_ERR_INVALID_ARG, "rows [%lld, %lld) outside [0, Lcap]", (long long)offset,
@@ -318,6 +323,23 @@ qkv_status qkv_q8_0_from_blocks(const void* blocks, int B, int Hkv, int D, int64
   if (L == 0) return ok();
   cudaError_t e = qkv::launch_q8_0_blocks(false, blocks, nullptr, dst, B, Hkv, D, offset, L, stride_b,
                                           stride_h, stride_l, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(QKV_ERR_CUDA, "block conversion launch: %s", cudaGetErrorString(e));
+  return ok();
+}
+
+qkv_status qkv_llama_blocks_to_cache(int kind, const void* blocks, int B, int Hkv, int D,
+                                     int64_t L, int64_t stride_b, int64_t stride_h,
+                                     int64_t stride_l, const qkv_cache* dst, int64_t offset,
+                                     void* stream) {
+  if (kind < QKV_BLOCKS_Q4_0 || kind > QKV_BLOCKS_Q5_1)
+    return fail(QKV_ERR_INVALID_ARG, "unknown block kind %d", kind);
+  const int bits = (kind == QKV_BLOCKS_Q4_0 || kind == QKV_BLOCKS_Q4_1) ? 4 : 8;
+  qkv_status st = check_blocks_args(dst, B, Hkv, D, offset, L, blocks, stride_b, stride_h, stride_l,
+                                    QKV_AFFINE, bits);
+  if (st != QKV_OK) return st;
+  if (L == 0) return ok();
+  cudaError_t e = qkv::launch_llama_blocks(kind, blocks, dst, B, Hkv, D, offset, L, stride_b, stride_h,
+                                           stride_l, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(QKV_ERR_CUDA, "block conversion launch: %s", cudaGetErrorString(e));
   return ok();
 }

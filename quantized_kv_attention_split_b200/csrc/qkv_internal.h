@@ -90,6 +90,9 @@ cudaError_t launch_decode(int D, int bits, int gs, int fmt, int out_f32,
 // Rows [0, L) of a cache as fp16 [B * Hkv, L, D] (dequantize.cu).
 cudaError_t launch_dequantize(const qkv_cache* c, int B, int Hkv, int D, int64_t L, void* out,
                               cudaStream_t stream);
+cudaError_t launch_llama_blocks(int kind, const void* src_blocks, const qkv_cache* c, int B, int Hkv,
+                                int D, int64_t offset, int64_t L, int64_t sb, int64_t sh,
+                                int64_t sl, cudaStream_t stream);
 cudaError_t launch_q8_0_blocks(bool to_blocks, const void* src_blocks, void* dst_blocks,
                                const qkv_cache* c, int B, int Hkv, int D, int64_t offset, int64_t L,
                                int64_t sb, int64_t sh, int64_t sl, cudaStream_t stream);

@@ -85,6 +85,9 @@ def lib() -> C.CDLL:
         L.qkv_q8_0_from_blocks.restype = i32
         L.qkv_q8_0_to_blocks.argtypes = [cp, i32, i32, i32, i64, i64, p, i64, i64, i64, p]
         L.qkv_q8_0_to_blocks.restype = i32
+        L.qkv_llama_blocks_to_cache.argtypes = [i32, p, i32, i32, i32, i64, i64, i64, i64, cp,
+                                                i64, p]
+        L.qkv_llama_blocks_to_cache.restype = i32
         L.qkv_dequantize.argtypes = [cp, i32, i32, i32, i64, p, p]
         L.qkv_dequantize.restype = i32
         L.qsdpa_workspace_size.argtypes = [i32, i32, i32, i32, i32, i64]
@@ -216,6 +219,27 @@ def qkv_q8_0_from_blocks(blocks: torch.Tensor, c: QuantCache, offset: int = 0,
     cs = c._struct()
     _check(lib().qkv_q8_0_from_blocks(blocks.data_ptr(), B, Hkv, D, int(L), sb, sh, sl,
                                       C.byref(cs), int(offset), _stream(stream)))
+    return c
+
+
+LLAMA_BLOCKS = {"q4_0": (0, 18, 4), "q4_1": (1, 20, 4), "q5_0": (2, 22, 8), "q5_1": (3, 24, 8)}
+
+
+def qkv_llama_blocks_to_cache(kind: str, blocks: torch.Tensor, c: QuantCache, offset: int = 0,
+                              L: Optional[int] = None, strides=None, stream=None) -> QuantCache:
+    """Write llama.cpp Q4_0/Q4_1/Q5_0/Q5_1 blocks (uint8 CUDA tensor, by default
+    [B, Hkv, L, D/32*bytes]) into rows [offset, offset+L) of an affine cache with
+    group_size 32 (4-bit codes for Q4, 8-bit for Q5)."""
+    code, nbytes, bits = LLAMA_BLOCKS[kind]
+    assert blocks.dtype == torch.uint8 and blocks.is_cuda and c.fmt == AFFINE
+    B, Hkv = c.codes.shape[0], c.codes.shape[1]
+    D = c.codes.shape[3] * 32 // c.bits
+    if L is None:
+        L = blocks.shape[2]
+    sb, sh, sl = _block_strides(blocks, strides)
+    cs = c._struct()
+    _check(lib().qkv_llama_blocks_to_cache(code, blocks.data_ptr(), B, Hkv, D, int(L), sb, sh, sl,
+                                           C.byref(cs), int(offset), _stream(stream)))
     return c
 
 

@@ -162,3 +162,17 @@ def test_block_conversion_validation_errors(lib):
     assert tb(C.byref(q8), 1, 2, 128, -1, 4, FAKE, *st, None) == 1            # negative offset
     assert tb(C.byref(q8), 1, 2, 96, 0, 4, FAKE, *st, None) == 2              # unsupported D
     assert tb(C.byref(q8), 1, 2, 128, 0, 0, FAKE, *st, None) == 0             # nothing to do
+
+
+def test_llama_blocks_validation_errors(lib):
+    from quantized_kv_attention_split_b200 import qkv
+    f = lib.qkv_llama_blocks_to_cache
+    a4 = _cache(qkv, fmt=0, bits=4, gs=32)
+    a8 = _cache(qkv, fmt=0, bits=8, gs=32)
+    st = (64 * 4 * 18, 4 * 18, 2 * 4 * 18)
+    assert f(9, FAKE, 1, 2, 128, 16, *st, C.byref(a4), 0, None) == 1          # unknown kind
+    assert f(0, FAKE, 1, 2, 128, 16, *st, C.byref(a8), 0, None) == 2          # Q4 into 8-bit
+    assert f(2, FAKE, 1, 2, 128, 16, *st, C.byref(a4), 0, None) == 2          # Q5 into 4-bit
+    assert f(1, FAKE, 1, 2, 128, 16, *st, C.byref(_cache(qkv, gs=64)), 0, None) == 2  # group 64
+    assert f(0, FAKE + 1, 1, 2, 128, 16, *st, C.byref(a4), 0, None) == 3      # odd address
+    assert f(3, FAKE, 1, 2, 128, 70, *st, C.byref(a8), 0, None) == 1          # past Lcap

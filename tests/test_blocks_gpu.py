@@ -63,3 +63,47 @@ def test_blocks_head_major_default_layout_and_decode():
     ref = oracle.attention(q, "f16", kc, vc, L, 1.0 / 16)
     assert out_err(from_dev(out), ref, "f16") <= 1.0
     assert torch.equal(qkv.qkv_q8_0_to_blocks(dk, L), bk)
+
+
+def _random_llama_blocks(kind, B, Hkv, L, nb, seed):
+    nbytes, has_m = oracle.LLAMA_BLOCKS[kind][0], oracle.LLAMA_BLOCKS[kind][1]
+    rng = np.random.default_rng(seed)
+    raw = rng.integers(0, 256, (B, Hkv, L, nb, nbytes), dtype=np.uint8)
+    for lo in ((0, 2) if has_m else (0,)):
+        h = S.f32_to_half_bits(rng.normal(0, 0.05, (B, Hkv, L, nb)).astype(np.float32), "f16")
+        raw[..., lo] = h & 0xFF
+        raw[..., lo + 1] = h >> 8
+    return raw
+
+
+@pytest.mark.parametrize("kind", ["q4_0", "q4_1", "q5_0", "q5_1"])
+def test_llama_blocks_to_cache_matches_oracle_and_decodes(kind):
+    """Random llama.cpp blocks (token-major, at a row offset) become exactly the
+    oracle's affine cache; the decode kernel then matches the oracle on it."""
+    from quantized_kv_attention_split_b200 import qkv
+    B, Hq, Hkv, D, L, off = 1, 16, 2, 128, 1500, 3
+    nb = D // 32
+    nbytes, bits = oracle.LLAMA_BLOCKS[kind][0], oracle.LLAMA_BLOCKS[kind][4]
+    Lcap = ((off + L) // 8 + 1) * 8
+    caches = []
+    for which in (0, 1):
+        raw = _random_llama_blocks(kind, B, Hkv, L, nb, 70 + which)
+        tm = np.ascontiguousarray(raw.transpose(0, 2, 1, 3, 4)).reshape(B, L, Hkv * nb * nbytes)
+        st = (L * Hkv * nb * nbytes, nb * nbytes, Hkv * nb * nbytes)
+        dc = qkv.QuantCache.empty(B, Hkv, Lcap, D, qkv.AFFINE, bits, 32)
+        qkv.qkv_llama_blocks_to_cache(kind, torch.from_numpy(tm).cuda(), dc, offset=off, L=L,
+                                      strides=st)
+        torch.cuda.synchronize()
+        ref = oracle.llama_blocks_to_cache(kind, raw)
+        h = cache_from_dev(dc, "affine")
+        assert np.array_equal(h.codes[:, :, off:off + L], ref.codes)
+        assert np.array_equal(h.scales[:, :, off:off + L], ref.scales)
+        assert np.array_equal(h.biases[:, :, off:off + L], ref.biases)
+        caches.append((dc, h))
+    (dk, hk), (dv, hv) = caches
+    q = S.draw(71, "q", (B, Hq, 1, D), "normal", "f16")
+    L_all = off + L
+    out = qkv.qsdpa_decode(to_dev(q, "f16"), dk, dv, L_all, 0.125)
+    torch.cuda.synchronize()
+    ref = oracle.attention(q, "f16", hk, hv, L_all, 0.125)
+    assert out_err(from_dev(out), ref, "f16") <= 1.0
