@@ -222,6 +222,27 @@ qkv_status attention(const void* q, int q_dtype, int B, int Hq, int Hkv, int Lq,
   return ok();
 }
 
+qkv_status check_blocks_args(const qkv_cache* c, int B, int Hkv, int D, int64_t offset, int64_t L,
+                             const void* blocks, int64_t sb, int64_t sh, int64_t sl,
+                             int want_fmt = QKV_Q8_0, int want_bits = 8) {
+  qkv_status st;
+  if ((st = check_cache("cache", c, D)) != QKV_OK) return st;
+  if (want_fmt == QKV_Q8_0 && c->fmt != QKV_Q8_0)
+    return fail(QKV_ERR_UNSUPPORTED, "Q8_0 block conversion needs a Q8_0 cache");
+  if (want_fmt == QKV_AFFINE && (c->fmt != QKV_AFFINE || c->group_size != 32 || c->bits != want_bits))
+    return fail(QKV_ERR_UNSUPPORTED, "these blocks need an affine cache with group_size 32 and %d-bit codes",
+                want_bits);
+  if (B <= 0 || Hkv <= 0) return fail(QKV_ERR_INVALID_ARG, "B and Hkv must be positive");
+  if (offset < 0 || L < 0 || offset + L > c->Lcap)
+    return fail(QKV_ERR_INVALID_ARG, "rows [%lld, %lld) outside [0, Lcap]", (long long)offset,
+                (long long)(offset + L));
+  if (blocks == nullptr) return fail(QKV_ERR_INVALID_ARG, "blocks must be non-NULL");
+  if (sb < 0 || sh < 0 || sl < 0) return fail(QKV_ERR_INVALID_ARG, "block strides must be non-negative");
+  if ((reinterpret_cast<uintptr_t>(blocks) & 1u) != 0 || ((sb | sh | sl) & 1) != 0)
+    return fail(QKV_ERR_ALIGNMENT, "blocks and their strides must be 2-byte aligned");
+  return QKV_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -292,28 +313,6 @@ qkv_status qkv_dequantize(const qkv_cache* c, int B, int Hkv, int D, int64_t L, 
   return ok();
 }
 
-namespace {
-qkv_status check_blocks_args(const qkv_cache* c, int B, int Hkv, int D, int64_t offset, int64_t L,
-                             const void* blocks, int64_t sb, int64_t sh, int64_t sl,
-                             int want_fmt = QKV_Q8_0, int want_bits = 8) {
-  qkv_status st;
-  if ((st = check_cache("cache", c, D)) != QKV_OK) return st;
-  if (want_fmt == QKV_Q8_0 && c->fmt != QKV_Q8_0)
-    return fail(QKV_ERR_UNSUPPORTED, "Q8_0 block conversion needs a Q8_0 cache");
-  if (want_fmt == QKV_AFFINE && (c->fmt != QKV_AFFINE || c->group_size != 32 || c->bits != want_bits))
-    return fail(QKV_ERR_UNSUPPORTED, "these blocks need an affine cache with group_size 32 and %d-bit codes",
-                want_bits);
-  if (B <= 0 || Hkv <= 0) return fail(QKV_ERR_INVALID_ARG, "B and Hkv must be positive");
-  if (offset < 0 || L < 0 || offset + L > c->Lcap)
-    return fail(QKV_ERR_INVALID_ARG, "rows [%lld, %lld) outside [0, Lcap]", (long long)offset,
-                (long long)(offset + L));
-  if (blocks == nullptr) return fail(QKV_ERR_INVALID_ARG, "blocks must be non-NULL");
-  if (sb < 0 || sh < 0 || sl < 0) return fail(QKV_ERR_INVALID_ARG, "block strides must be non-negative");
-  if ((reinterpret_cast<uintptr_t>(blocks) & 1u) != 0 || ((sb | sh | sl) & 1) != 0)
-    return fail(QKV_ERR_ALIGNMENT, "blocks and their strides must be 2-byte aligned");
-  return QKV_OK;
-}
-}  // namespace
 
 qkv_status qkv_q8_0_from_blocks(const void* blocks, int B, int Hkv, int D, int64_t L,
                                 int64_t stride_b, int64_t stride_h, int64_t stride_l,
