@@ -137,8 +137,3 @@ def test_prefill_extensions_match_oracle(qkv, case):
     plain = oracle.attention(q, "bf16", kc, vc, L, scale, mask=mask_o)
     assert max_err(plain, ref) > 1e-2
 
-
-def test_fused_update_rejects_extensions_in_the_binding(qkv):
-    """The fused update step has no extension arguments; the C entry points
-    that take them are the plain decode and prefill ones."""
-    assert not hasattr(qkv, "qsdpa_decode_update_ext")
