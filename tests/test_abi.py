@@ -176,3 +176,21 @@ def test_llama_blocks_validation_errors(lib):
     assert f(1, FAKE, 1, 2, 128, 16, *st, C.byref(_cache(qkv, gs=64)), 0, None) == 2  # group 64
     assert f(0, FAKE + 1, 1, 2, 128, 16, *st, C.byref(a4), 0, None) == 3      # odd address
     assert f(3, FAKE, 1, 2, 128, 70, *st, C.byref(a8), 0, None) == 1          # past Lcap
+
+
+def test_header_is_plain_c(tmp_path):
+    """include/qkv.h compiles as C99 (no C++ or CUDA types in the boundary),
+    and a C program can take the address of every declared function."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    names = _declared()
+    src = tmp_path / "use_qkv.c"
+    src.write_text('#include "qkv.h"\ntypedef void (*fn_t)(void);\nfn_t fns[] = {\n' +
+                   "".join(f"  (fn_t)&{n},\n" for n in names) + "};\n")
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-pedantic", "-c", str(src),
+                        "-I", os.path.join(ROOT, "include"), "-o", str(tmp_path / "use_qkv.o")],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
