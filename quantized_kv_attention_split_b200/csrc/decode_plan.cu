@@ -17,8 +17,9 @@ constexpr int64_t kBigPartial = 2048;
 constexpr int64_t kBigPartMinStages = 2;   // blocks per team
 // With large partials, at most this many CTAs share a unit: the merge reads
 // every partial, and beyond this the longer merge costs more than the shorter
-// loop gains (Q8_0, D = 256, 16 rows, 10K and 20K keys: best at 48 of 24..74).
-constexpr int64_t kBigPartMaxPieces = 48;
+// loop gains (Q8_0, D = 256, 16 rows, 10K and 20K keys: 64 measured best of
+// 32, 48 and 64 since the epilogue combines four elements per thread).
+constexpr int64_t kBigPartMaxPieces = 64;
 
 // SM count of the current device, queried once per device (every decode call
 // plans its grid with it).
