@@ -10,6 +10,13 @@ beside it.  Inputs are synthetic (seeded SplitMix64), quantized on the GPU by
 qkv_quantize_update; the timed calls rotate over enough cache copies that the
 data read in one call is no longer in the 126 MB L2 when it is read again.
 
+The line's `rows` object times the other rows of the path the same way
+(--no-rows leaves them out): bulk and one-token quantize, the 8-bit decode
+and the fused update + decode, the Q8_0 D=256 decodes, the 512-query prefill,
+the materialize-then-library-attention A/B rows, the attention extensions
+(softcap, sinks, ALiBi) on decode and prefill, and the llama.cpp block
+conversions.
+
 --impl reference runs the CPU oracle (the only reference this repository has)
 on a bounded sample of the same workload and reports the same metric.
 
