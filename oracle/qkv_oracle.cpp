@@ -142,6 +142,31 @@ float load_elem(const void* p, int dtype, int64_t i) {
 }
 
 // ---------------------------------------------------------------------------
+// Code packing.  A row's codes form one little-endian bit stream: element e
+// occupies bits [e*bits, (e+1)*bits), bit i of the stream being bit i%32 of
+// 32-bit word i/32.  For 2, 4 and 8 bits this is "element j of a word at bits
+// [j*bits, (j+1)*bits)" ([MLX-KV] sdpa_vector.h); for 3 and 5 bits it packs 8
+// codes in 3 or 5 bytes and for 6 bits 4 codes in 3 bytes, the pack sizes
+// that [MLX-WIP] mlx/backend/cuda/quantized/quantized_utils.cuh
+// (get_pack_factor, get_bytes_per_pack) states -- reading: within a pack, the
+// same little-endian order (the pages print no 3/5/6-bit pack layout).
+// ---------------------------------------------------------------------------
+void put_code(uint32_t* row, int e, int bits, uint32_t q) {
+  const int64_t pos = (int64_t)e * bits;
+  const int w = (int)(pos / 32), sh = (int)(pos % 32);
+  row[w] |= q << sh;
+  if (sh + bits > 32) row[w + 1] |= q >> (32 - sh);     // the code straddles two words
+}
+
+uint32_t get_code(const uint32_t* row, int e, int bits) {
+  const int64_t pos = (int64_t)e * bits;
+  const int w = (int)(pos / 32), sh = (int)(pos % 32);
+  uint64_t v = row[w] >> sh;
+  if (sh + bits > 32) v |= (uint64_t)row[w + 1] << (32 - sh);
+  return (uint32_t)(v & ((1u << bits) - 1u));
+}
+
+// ---------------------------------------------------------------------------
 // Quantizers ([MLX-KV] quantized.h affine_quantize_impl / kv_update; [LCPP]).
 // ---------------------------------------------------------------------------
 void quantize_affine_group(const float* x, int gs, int bits,
@@ -163,9 +188,7 @@ void quantize_affine_group(const float* x, int gs, int bits,
     int q = (int)r;
     if (q < 0) q = 0;
     if (q > qmax) q = qmax;
-    const int e = first_elem + i;               // element index within the row
-    const int per_word = 32 / bits;
-    codes_row[e / per_word] |= (uint32_t)q << ((e % per_word) * bits);
+    put_code(codes_row, first_elem + i, bits, (uint32_t)q);   // element index within the row
   }
   *scale_out = s16;
   *bias_out = b16;
@@ -212,10 +235,8 @@ void dequant_row(const Cache& c, int D, int64_t row, double* out) {
   const uint32_t* w = c.codes + row * words;
   const uint16_t* sc = c.scales + row * ng;
   const uint16_t* bi = c.fmt == 0 ? c.biases + row * ng : nullptr;
-  const int per_word = 32 / c.bits;
-  const uint32_t mask = (c.bits == 32) ? 0xffffffffu : ((1u << c.bits) - 1u);
   for (int e = 0; e < D; ++e) {
-    const uint32_t field = (w[e / per_word] >> ((e % per_word) * c.bits)) & mask;
+    const uint32_t field = get_code(w, e, c.bits);
     const int g = e / c.gs;
     const double s = (double)half_to_float(sc[g]);
     if (c.fmt == 0) {
@@ -402,12 +423,13 @@ void orc_bf16_to_f32(const uint16_t* x, float* y, int64_t n) {
 
 // --- quantize `rows` rows of D elements (fp16 / bf16 / fp32 input) ----------
 // codes: [rows, D*bits/32] uint32 (zeroed here), scales/biases: [rows, D/gs].
-// fmt 0 = affine (bits 2..8 dividing 32, gs | D), fmt 1 = Q8_0 (gs 32).
+// fmt 0 = affine (bits 2, 3, 4, 5, 6 or 8; gs | D; D*bits a multiple of 32),
+// fmt 1 = Q8_0 (gs 32).
 int orc_quantize(int fmt, const void* x, int in_dtype, int64_t rows, int D,
                  int gs, int bits, uint32_t* codes, uint16_t* scales,
                  uint16_t* biases, int nthreads) {
   if (fmt == 1) { bits = 8; gs = 32; }
-  if (D % gs != 0 || 32 % bits != 0 || (D * bits) % 32 != 0) return 1;
+  if (D % gs != 0 || bits < 2 || bits > 8 || bits == 7 || (D * bits) % 32 != 0) return 1;
   const int words = D * bits / 32, ng = D / gs;
   parallel_rows(rows, nthreads, [&](int64_t r) {
     std::vector<float> xr(D);

@@ -40,6 +40,10 @@ CASES = [
     (1, 6, 3, 2, 64, 19, 19, "affine", 4, 32, 0.3),
     (1, 4, 2, 5, 256, 50, 64, "q8_0", 8, 32, 1.0 / 16),
     (2, 2, 2, 1, 128, 64, 64, "affine", 4, 128, 0.09),
+    (1, 4, 2, 2, 64, 33, 40, "affine", 3, 32, 0.2),     # codes straddle words
+    (1, 2, 1, 1, 128, 21, 24, "affine", 6, 64, 0.1),
+    (1, 2, 1, 3, 64, 17, 24, "affine", 5, 32, 0.3),
+    (1, 2, 2, 1, 64, 12, 16, "affine", 2, 64, 1.0),
 ]
 
 

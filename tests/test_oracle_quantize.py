@@ -82,7 +82,9 @@ def _golden_input(g):
 
 
 @pytest.mark.parametrize("name", ["affine4_ramp.txt", "affine8_bytes.txt",
-                                  "q8_0_block.txt", "affine4_constant.txt"])
+                                  "q8_0_block.txt", "affine4_constant.txt",
+                                  "affine2_ramp.txt", "affine3_ramp.txt",
+                                  "affine5_ramp.txt", "affine6_ramp.txt"])
 def test_golden_packing(orc, name):
     g = read_golden(name)
     x = _golden_input(g)
@@ -102,11 +104,15 @@ def test_golden_packing(orc, name):
 # properties of the quantizers
 # --------------------------------------------------------------------------
 def _unpack(codes, bits, D, signed=False):
-    """Element j of each 32-bit word at bits [j*bits, (j+1)*bits)."""
-    per = 32 // bits
+    """Element e at bits [e*bits, (e+1)*bits) of the row's little-endian bit
+    stream (for 2, 4 and 8 bits: element j of a word at bits [j*bits, ...))."""
     e = np.arange(D)
-    w = codes[..., e // per].astype(np.uint64)
-    f = (w >> ((e % per) * bits).astype(np.uint64)) & np.uint64((1 << bits) - 1)
+    pos = e * bits
+    lo = codes[..., pos // 32].astype(np.uint64)
+    hi_idx = np.minimum(pos // 32 + 1, codes.shape[-1] - 1)
+    hi = codes[..., hi_idx].astype(np.uint64)
+    both = lo | (hi << np.uint64(32))                 # 64-bit window over two words
+    f = (both >> (pos % 32).astype(np.uint64)) & np.uint64((1 << bits) - 1)
     f = f.astype(np.int64)
     if signed:
         f = np.where(f >= 128, f - 256, f)
@@ -127,7 +133,7 @@ def _groups(seed, rows, D, kind, dtype="f16"):
     return S.f32_to_half_bits(x, dtype)
 
 
-@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("bits", [2, 3, 4, 5, 6, 8])
 @pytest.mark.parametrize("gs", [32, 64, 128])
 @pytest.mark.parametrize("kind", ["uniform", "normal", "wide", "offset"])
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
@@ -199,7 +205,7 @@ def test_affine_constant_groups_reconstruct_exactly(orc):
     rng = np.random.default_rng(5)
     vals = rng.standard_normal(32).astype(np.float32)
     x = S.f32_to_half_bits(np.repeat(vals, 64).reshape(32, 64), "f16")
-    for bits in (4, 8):
+    for bits in (2, 3, 4, 5, 6, 8):
         c = orc.quantize(x, "f16", "affine", 64, bits)
         assert np.all(c.codes == 0)
         assert np.array_equal(orc.dequantize(c, 64), orc.to_f64(x, "f16"))
@@ -235,3 +241,22 @@ def test_affine_dot_identity(orc):
         rhs = sum(s[r, g] * (codes[r, g * 64:(g + 1) * 64] @ q[g * 64:(g + 1) * 64])
                   + b[r, g] * q[g * 64:(g + 1) * 64].sum() for g in range(2))
         assert abs(lhs - rhs) <= 1e-12 * max(1.0, abs(lhs))
+
+
+
+@pytest.mark.parametrize("bits", [3, 5, 6])
+def test_odd_widths_pack_as_bit_stream(orc, bits):
+    """3/5/6-bit codes straddle 32-bit words; every code survives the packing
+    and a code's bits never touch its neighbours' (random codes planted through
+    values whose group spans exactly 0..2^bits-1)."""
+    rng = np.random.default_rng(bits)
+    D, gs = 128, 32
+    top = (1 << bits) - 1
+    q = rng.integers(0, top + 1, (16, D))
+    q[:, ::gs] = 0
+    q[:, 1::gs] = top                           # each group spans the full code range
+    x = S.f32_to_half_bits(q.astype(np.float32), "f16")
+    c = orc.quantize(x, "f16", "affine", gs, bits)
+    assert c.codes.shape[-1] == D * bits // 32
+    assert np.array_equal(_unpack(c.codes, bits, D), q)
+    assert np.array_equal(orc.dequantize(c, D), q.astype(np.float64))
