@@ -11,7 +11,9 @@
  *    mlx/fast.cpp (the fallback defines the math); sdpa_vector.h
  *    quant_sdpa_vector (packing, dequant, GQA mapping); quantized.h kv_update
  *    and affine_quantize_impl (eps 1e-7).
- *  - llama.cpp PR #25556 "Metal: Optimize q8_0 KV": the Q8_0 KV format.
+ *  - llama.cpp PR #25556 "Metal: Optimize q8_0 KV": the Q8_0 KV format; its
+ *    merged follow-up: the attention variants its tests cover (sinks, ALiBi,
+ *    logit softcap) and the other KV block types (Q4_0, Q4_1, Q5_0, Q5_1).
  *
  * Conventions shared by every entry point
  *  - All tensor pointers are DEVICE pointers owned by the caller.  The library
