@@ -54,6 +54,11 @@ def lib():
         L.orc_attention.restype = i32
         L.orc_attention_probs.argtypes = common + [i32, i32, i32, p, p]
         L.orc_attention_probs.restype = i32
+        L.orc_attention_kview.argtypes = [p, i32, i32, i32, i32, i32, i32,
+                                          i32, i32, i32, p, p, p,
+                                          i64, i64, C.c_double, i32, p, i32, i64, i64, i64,
+                                          C.c_double, p, p, i32, i32, p, i64, p, i32]
+        L.orc_attention_kview.restype = i32
         _lib = L
     return _lib
 
@@ -211,6 +216,27 @@ def attention(q: np.ndarray, q_dtype: str, k: QCache, v: QCache, L: int,
                              nthreads or default_threads())
     if rc:
         raise ValueError("oracle attention: invalid arguments")
+    return out
+
+
+def attention_kview(q: np.ndarray, q_dtype: str, k: QCache, L: int, scale: float, Dv: int,
+                    mask: Optional[Mask] = None, mode: str = "two_pass", nsplit: int = 1,
+                    rows: Optional[np.ndarray] = None, nthreads: Optional[int] = None,
+                    ext: Optional[Ext] = None) -> np.ndarray:
+    """fp64 attention [B,Hq,Lq,Dv] whose values are the first Dv elements of
+    the key rows (the MLA shape: K rows of Dk, V a view of K)."""
+    q64 = np.ascontiguousarray(to_f64(q, q_dtype))
+    B, Hq, Lq, Dk = q64.shape
+    out = np.full((B, Hq, Lq, Dv), np.nan)
+    args, keep = _common_args(q64, k, k, L, scale, mask, ext)
+    # the common list holds both caches; the view entry takes the key cache once
+    a = args[:5] + [Dk, Dv] + args[6:12] + args[18:]
+    r = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    rc = lib().orc_attention_kview(*a, {"two_pass": 0, "online": 1, "split": 2}[mode], nsplit,
+                                   _ptr(r), 0 if r is None else r.size, _ptr(out),
+                                   nthreads or default_threads())
+    if rc:
+        raise ValueError("oracle attention_kview: invalid arguments")
     return out
 
 

@@ -261,6 +261,7 @@ struct Mask {
 struct Problem {
   const double* q;      // [B,Hq,Lq,D] already converted to fp64
   int B, Hq, Hkv, Lq, D;
+  int Dv;               // output / value width: D, or fewer when V is a view of K's first Dv
   Cache k, v;
   int64_t L;
   double scale;
@@ -303,7 +304,7 @@ void attend_two_pass(const Problem& p, int b, int h, int i, double* o,
     dequant_row(p.k, p.D, base + j, kh.data());
     if (logit(p, b, h, i, j, kh, &s[j])) { vis[j] = 1; mx = std::max(mx, s[j]); }
   }
-  for (int e = 0; e < p.D; ++e) o[e] = 0.0;
+  for (int e = 0; e < p.Dv; ++e) o[e] = 0.0;
   if (probs) for (int64_t j = 0; j < p.L; ++j) probs[j] = 0.0;
   if (!(mx > -std::numeric_limits<double>::infinity())) return;  // none visible
   double l = 0.0;
@@ -318,7 +319,7 @@ void attend_two_pass(const Problem& p, int b, int h, int i, double* o,
     const double pj = s[j] / l;
     if (probs) probs[j] = pj;
     dequant_row(p.v, p.D, vbase + j, vh.data());
-    for (int e = 0; e < p.D; ++e) o[e] += pj * vh[e];
+    for (int e = 0; e < p.Dv; ++e) o[e] += pj * vh[e];
   }
 }
 
@@ -331,7 +332,7 @@ void attend_online_range(const Problem& p, int b, int h, int i, int64_t j0,
   const int64_t vb = ((int64_t)b * p.Hkv + kvh) * p.v.Lcap;
   std::vector<double> kh(p.D), vh(p.D);
   double m = -std::numeric_limits<double>::infinity(), l = 0.0;
-  for (int e = 0; e < p.D; ++e) o[e] = 0.0;
+  for (int e = 0; e < p.Dv; ++e) o[e] = 0.0;
   for (int64_t j = j0; j < j1; ++j) {
     dequant_row(p.k, p.D, kb + j, kh.data());
     double sj;
@@ -341,7 +342,7 @@ void attend_online_range(const Problem& p, int b, int h, int i, int64_t j0,
     const double pj = std::exp(sj - mn);
     dequant_row(p.v, p.D, vb + j, vh.data());
     l = l * alpha + pj;
-    for (int e = 0; e < p.D; ++e) o[e] = o[e] * alpha + pj * vh[e];
+    for (int e = 0; e < p.Dv; ++e) o[e] = o[e] * alpha + pj * vh[e];
     m = mn;
   }
   *m_out = m;
@@ -351,35 +352,35 @@ void attend_online_range(const Problem& p, int b, int h, int i, int64_t j0,
 // Final normalization of an online/merged (m, l, o): o / l, with the head's
 // sink (if any) folded into the denominator; no visible key gives zeros.
 void finish_row(const Problem& p, int h, double m, double l, double* o) {
-  if (!(l > 0.0)) { for (int e = 0; e < p.D; ++e) o[e] = 0.0; return; }
+  if (!(l > 0.0)) { for (int e = 0; e < p.Dv; ++e) o[e] = 0.0; return; }
   double w = 1.0;
   if (p.sinks) {
     const double M = std::max(m, p.sinks[h]);
     w = std::exp(m - M);
     l = l * w + std::exp(p.sinks[h] - M);
   }
-  for (int e = 0; e < p.D; ++e) o[e] = o[e] * w / l;
+  for (int e = 0; e < p.Dv; ++e) o[e] = o[e] * w / l;
 }
 
 // Split form: partition keys into `nsplit` contiguous chunks, run the online
 // form on each, then merge the partial (m, l, o) by log-sum-exp rescaling.
 void attend_split(const Problem& p, int b, int h, int i, int nsplit, double* o) {
   const double ninf = -std::numeric_limits<double>::infinity();
-  std::vector<double> ms(nsplit), ls(nsplit), os((size_t)nsplit * p.D);
+  std::vector<double> ms(nsplit), ls(nsplit), os((size_t)nsplit * p.Dv);
   for (int sidx = 0; sidx < nsplit; ++sidx) {
     const int64_t j0 = p.L * sidx / nsplit, j1 = p.L * (sidx + 1) / nsplit;
-    attend_online_range(p, b, h, i, j0, j1, &ms[sidx], &ls[sidx], &os[(size_t)sidx * p.D]);
+    attend_online_range(p, b, h, i, j0, j1, &ms[sidx], &ls[sidx], &os[(size_t)sidx * p.Dv]);
   }
   double M = ninf;
   for (double m : ms) M = std::max(M, m);
-  for (int e = 0; e < p.D; ++e) o[e] = 0.0;
+  for (int e = 0; e < p.Dv; ++e) o[e] = 0.0;
   if (M == ninf) return;
   double l = 0.0;
   for (int sidx = 0; sidx < nsplit; ++sidx) {
     if (ms[sidx] == ninf) continue;
     const double w = std::exp(ms[sidx] - M);
     l += w * ls[sidx];
-    for (int e = 0; e < p.D; ++e) o[e] += w * os[(size_t)sidx * p.D + e];
+    for (int e = 0; e < p.Dv; ++e) o[e] += w * os[(size_t)sidx * p.Dv + e];
   }
   finish_row(p, h, M, l, o);
 }
@@ -393,6 +394,28 @@ void parallel_rows(int64_t n, int nthreads, F f) {
     ts.emplace_back([&, t]() { for (int64_t r = t; r < n; r += nthreads) f(r); });
   }
   for (auto& th : ts) th.join();
+}
+
+// Every requested row (b, h, i) of the output, in one of the three evaluation
+// orders; row id ((b*Hq)+h)*Lq+i, output rows of p.Dv values.
+void run_rows(const Problem& p, int mode, int nsplit, const int64_t* rows, int64_t total,
+              double* out, int nthreads) {
+  parallel_rows(total, nthreads, [&](int64_t r) {
+    const int64_t id = rows ? rows[r] : r;
+    const int i = (int)(id % p.Lq);
+    const int h = (int)((id / p.Lq) % p.Hq);
+    const int b = (int)(id / ((int64_t)p.Lq * p.Hq));
+    double* o = out + id * p.Dv;
+    if (mode == 0) {
+      attend_two_pass(p, b, h, i, o, nullptr);
+    } else if (mode == 1) {
+      double m, l;
+      attend_online_range(p, b, h, i, 0, p.L, &m, &l, o);
+      finish_row(p, h, m, l, o);
+    } else {
+      attend_split(p, b, h, i, nsplit < 1 ? 1 : nsplit, o);
+    }
+  });
 }
 
 Cache make_cache(int fmt, int bits, int gs, const uint32_t* codes,
@@ -479,7 +502,7 @@ int orc_attention(const double* q, int B, int Hq, int Hkv, int Lq, int D,
   if (kfmt == 1) { kbits = 8; kgs = 32; }
   if (vfmt == 1) { vbits = 8; vgs = 32; }
   Problem p;
-  p.q = q; p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Lq = Lq; p.D = D;
+  p.q = q; p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Lq = Lq; p.D = D; p.Dv = D;
   p.k = make_cache(kfmt, kbits, kgs, kcodes, kscales, kbiases, Lcap);
   p.v = make_cache(vfmt, vbits, vgs, vcodes, vscales, vbiases, Lcap);
   p.L = L; p.scale = scale;
@@ -487,22 +510,34 @@ int orc_attention(const double* q, int B, int Hq, int Hkv, int Lq, int D,
   p.mask.sb = msb; p.mask.sh = msh; p.mask.sq = msq;
   p.softcap = softcap; p.sinks = sinks; p.slopes = slopes;
   const int64_t total = rows ? nrows : (int64_t)B * Hq * Lq;
-  parallel_rows(total, nthreads, [&](int64_t r) {
-    const int64_t id = rows ? rows[r] : r;
-    const int i = (int)(id % Lq);
-    const int h = (int)((id / Lq) % Hq);
-    const int b = (int)(id / ((int64_t)Lq * Hq));
-    double* o = out + id * D;
-    if (mode == 0) {
-      attend_two_pass(p, b, h, i, o, nullptr);
-    } else if (mode == 1) {
-      double m, l;
-      attend_online_range(p, b, h, i, 0, L, &m, &l, o);
-      finish_row(p, h, m, l, o);
-    } else {
-      attend_split(p, b, h, i, nsplit < 1 ? 1 : nsplit, o);
-    }
-  });
+  run_rows(p, mode, nsplit, rows, total, out, nthreads);
+  return 0;
+}
+
+// --- attention whose values are a view of the keys ---------------------------
+// (the MLA shape of the llama.cpp PR's follow-up: K rows of Dk elements, V the
+// first Dv of each K row).  One cache; out: fp64 [B,Hq,Lq,Dv].
+int orc_attention_kview(const double* q, int B, int Hq, int Hkv, int Lq, int Dk, int Dv,
+                        int kfmt, int kbits, int kgs, const uint32_t* kcodes,
+                        const uint16_t* kscales, const uint16_t* kbiases,
+                        int64_t Lcap, int64_t L, double scale, int mask_kind,
+                        const void* mask_add, int mask_dtype, int64_t msb,
+                        int64_t msh, int64_t msq, double softcap,
+                        const double* sinks, const double* slopes, int mode, int nsplit,
+                        const int64_t* rows, int64_t nrows, double* out,
+                        int nthreads) {
+  if (Hkv <= 0 || Hq % Hkv != 0 || L < 0 || L > Lcap || Dv <= 0 || Dv > Dk) return 1;
+  if (kfmt == 1) { kbits = 8; kgs = 32; }
+  Problem p;
+  p.q = q; p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Lq = Lq; p.D = Dk; p.Dv = Dv;
+  p.k = make_cache(kfmt, kbits, kgs, kcodes, kscales, kbiases, Lcap);
+  p.v = p.k;                                            // values: the key rows themselves
+  p.L = L; p.scale = scale;
+  p.mask.kind = mask_kind; p.mask.add = mask_add; p.mask.add_dtype = mask_dtype;
+  p.mask.sb = msb; p.mask.sh = msh; p.mask.sq = msq;
+  p.softcap = softcap; p.sinks = sinks; p.slopes = slopes;
+  const int64_t total = rows ? nrows : (int64_t)B * Hq * Lq;
+  run_rows(p, mode, nsplit, rows, total, out, nthreads);
   return 0;
 }
 
@@ -521,7 +556,7 @@ int orc_attention_probs(const double* q, int B, int Hq, int Hkv, int Lq, int D,
   if (kfmt == 1) { kbits = 8; kgs = 32; }
   if (vfmt == 1) { vbits = 8; vgs = 32; }
   Problem p;
-  p.q = q; p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Lq = Lq; p.D = D;
+  p.q = q; p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Lq = Lq; p.D = D; p.Dv = D;
   p.k = make_cache(kfmt, kbits, kgs, kcodes, kscales, kbiases, Lcap);
   p.v = make_cache(vfmt, vbits, vgs, vcodes, vscales, vbiases, Lcap);
   p.L = L; p.scale = scale;

@@ -168,3 +168,25 @@ def test_row_subset(orc):
     flat = sub.reshape(-1, D)
     assert np.array_equal(flat[rows], full.reshape(-1, D)[rows])
     assert np.isnan(flat[1]).all()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_values_as_a_view_of_the_keys_matches_torch(orc, causal):
+    """MLA shape of the llama.cpp PR's follow-up tests: K rows of 576 (Q8_0),
+    V the first 512 elements of each K row; torch's SDPA in fp64 with V given
+    as that slice (a library routine that takes different K and V widths)."""
+    B, Hq, Hkv, Lq, Dk, Dv, L = 1, 4, 1, 3, 576, 512, 40
+    k = S.draw(91, "k", (B, Hkv, L, Dk), "normal", "f16")
+    q = S.draw(92, "q", (B, Hq, Lq, Dk), "normal", "f16")
+    kc = orc.quantize(k, "f16", "q8_0")
+    K = torch.from_numpy(orc.dequantize(kc, Dk)).repeat_interleave(Hq // Hkv, dim=1)
+    q64 = torch.from_numpy(orc.to_f64(q, "f16"))
+    scale = 1.0 / 24
+    mask = orc.Mask("causal") if causal else None
+    tmask = None
+    if causal:
+        tmask = torch.ones(Lq, L, dtype=torch.bool).tril(diagonal=L - Lq)
+    ref = F.scaled_dot_product_attention(q64, K, K[..., :Dv], attn_mask=tmask, scale=scale).numpy()
+    for mode, ns in (("two_pass", 1), ("online", 1), ("split", 4)):
+        out = orc.attention_kview(q, "f16", kc, L, scale, Dv, mask=mask, mode=mode, nsplit=ns)
+        np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)

@@ -89,3 +89,24 @@ def test_attention_against_exact_arithmetic(orc, fmt, bits, use_mask, softcap, u
             for e in range(D):
                 w = float(want[e])
                 assert abs(got[e] - w) <= 1e-13 * max(1.0, abs(w)), (h, i, e, got[e], w)
+
+
+def test_values_as_a_view_of_the_keys_exact(orc):
+    """The MLA shape (V = the first Dv elements of every K row) on a tiny
+    problem, against the same exact arithmetic."""
+    B, Hq, Hkv, Lq, Dk, Dv, L = 1, 2, 1, 2, 64, 32, 5
+    k = S.draw(83, "k", (B, Hkv, L, Dk), "normal", "f16")
+    q = S.draw(84, "q", (B, Hq, Lq, Dk), "normal", "f16")
+    kc = orc.quantize(k, "f16", "q8_0")
+    Kd = orc.dequantize(kc, Dk)
+    qd = orc.to_f64(q, "f16")
+    out = orc.attention_kview(q, "f16", kc, L, 0.125, Dv, ext=orc.Ext(sinks=np.array([0.3, -2.0])))
+    assert out.shape == (B, Hq, Lq, Dv)
+    K = [[Fraction(float(x)) for x in Kd[0, 0, j]] for j in range(L)]
+    V = [row[:Dv] for row in K]
+    for h in range(Hq):
+        for i in range(Lq):
+            qrow = [Fraction(float(x)) for x in qd[0, h, i]]
+            want = _exact_row(qrow, K, V, Fraction(1, 8), None, 0.0, [0.3, -2.0][h])
+            for e in range(Dv):
+                assert abs(out[0, h, i, e] - float(want[e])) <= 1e-13 * max(1.0, abs(float(want[e])))
