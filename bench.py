@@ -180,11 +180,13 @@ def new_graph():
         return torch.cuda.CUDAGraph()
 
 
-def graph_time(step, K, W, sampler=None, min_window_s=0.3, tag=None):
+def graph_time(step, K, W, sampler=None, min_window_s=0.3, tag=None, sync_ranks=False):
     """Device time of exactly K calls of step(i): W eager warm-up calls, then
     K calls captured in CUDA graphs and replayed between events.  With a tag,
     the kernel launches of the K calls (counted from the captured graphs) are
-    recorded in LAUNCHES[tag]."""
+    recorded in LAUNCHES[tag].  sync_ranks: a barrier over all ranks right
+    before the timed region (only for calls that every rank makes; the
+    secondary rows run on rank 0 alone)."""
     import torch
     for i in range(W):
         step(i)
@@ -222,7 +224,7 @@ def graph_time(step, K, W, sampler=None, min_window_s=0.3, tag=None):
     torch.cuda.synchronize()
     reps = K // chunk
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if torch.distributed.is_available() and torch.distributed.is_initialized():
+    if sync_ranks and torch.distributed.is_available() and torch.distributed.is_initialized():
         torch.distributed.barrier()
     torch.cuda.synchronize()
     t0 = time.time()
@@ -340,7 +342,7 @@ def run_ours(args, rank, world, device):
     if sampler:
         sampler.start()
         time.sleep(0.3)
-    sec, extra = graph_time(step, args.steps, args.warmup, sampler, tag="main")
+    sec, extra = graph_time(step, args.steps, args.warmup, sampler, tag="main", sync_ranks=True)
     sec /= 1e3
     if sampler:
         time.sleep(0.1)
