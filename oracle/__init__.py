@@ -373,3 +373,55 @@ def llama_blocks_to_cache(kind: str, blocks: np.ndarray, Lcap: Optional[int] = N
     scales[:, :, :L] = d
     biases[:, :, :L] = m
     return QCache("affine", bits, 32, codes, scales, biases)
+
+
+def llama_quantize_blocks(kind: str, x: np.ndarray, dtype: str = "f16") -> np.ndarray:
+    """x [..., D] (raw half bits, or float32 for "f32") -> llama.cpp blocks
+    uint8 [..., D/32, bytes] of the given kind.  Reading (the pages show no
+    quantizer for these types): llama.cpp's published reference quantizers,
+    in fp32, block by block of 32 --
+      Q4_0 / Q5_0: m = the element of largest magnitude (first such), d = m / -8
+        (or m / -16), id = 1/d (0 if d == 0), q = min(15 | 31, trunc(x*id + 8.5 | 16.5));
+      Q4_1 / Q5_1: lo, hi = min, max, d = (hi - lo) / 15 (or 31), id = 1/d (0 if
+        d == 0), q = min(15 | 31, trunc((x - lo)*id + 0.5)), m = lo;
+    d (and m) stored as fp16 (round to nearest even), the codes computed with
+    the fp32 d."""
+    nbytes, has_m, has_qh, off, _ = LLAMA_BLOCKS[kind]
+    xf = to_f64(x, dtype).astype(np.float32)
+    D = xf.shape[-1]
+    xb = xf.reshape(xf.shape[:-1] + (D // 32, 32))
+    top = np.float32(2 * off - 1 if not has_m else (15 if kind == "q4_1" else 31))
+    if has_m:
+        lo = xb.min(-1)
+        hi = xb.max(-1)
+        d = ((hi - lo) / top).astype(np.float32)
+        idv = np.where(d != 0, np.float32(1) / np.where(d != 0, d, np.float32(1)), np.float32(0))
+        t = (xb - lo[..., None]) * idv[..., None] + np.float32(0.5)
+        q = np.minimum(np.trunc(t), top).astype(np.uint32)
+    else:
+        amax_i = np.abs(xb).argmax(-1)
+        mval = np.take_along_axis(xb, amax_i[..., None], -1)[..., 0]
+        d = (mval / np.float32(-off)).astype(np.float32)
+        idv = np.where(d != 0, np.float32(1) / np.where(d != 0, d, np.float32(1)), np.float32(0))
+        t = xb * idv[..., None] + np.float32(off + 0.5)
+        q = np.minimum(np.trunc(t), top).astype(np.uint32)
+    out = np.zeros(xb.shape[:-1] + (nbytes,), np.uint8)
+    d16 = f32_to_f16(d.astype(np.float32))
+    out[..., 0] = d16 & 0xFF
+    out[..., 1] = d16 >> 8
+    pos = 2
+    if has_m:
+        m16 = f32_to_f16(lo.astype(np.float32))
+        out[..., 2] = m16 & 0xFF
+        out[..., 3] = m16 >> 8
+        pos = 4
+    if has_qh:
+        qh = np.zeros(q.shape[:-1], np.uint64)
+        for e in range(32):
+            qh |= ((q[..., e].astype(np.uint64) >> 4) & 1) << e
+        for k in range(4):
+            out[..., pos + k] = (qh >> (8 * k)) & 0xFF
+        pos += 4
+    for j in range(16):
+        out[..., pos + j] = (q[..., j] & 0xF) | ((q[..., j + 16] & 0xF) << 4)
+    return out

@@ -76,3 +76,52 @@ def test_llama_blocks_to_cache_keeps_every_value(orc, kind):
     vals = orc.llama_block_values(kind, raw)
     assert np.array_equal(orc.dequantize(c, 32 * nb)[:, :, :L], vals)
     assert not c.codes[:, :, L:].any()
+
+
+@pytest.mark.parametrize("kind", ["q4_0", "q4_1", "q5_0", "q5_1"])
+def test_llama_quantizer_reproduces_the_hand_built_blocks(orc, kind):
+    """Each hand-built block's values quantize back to exactly that block: its
+    scale (and minimum) is what the reference quantizer derives from them, and
+    every value sits on a code."""
+    g = read_golden("llama_blocks.txt")
+    raw = np.array([int(x, 16) for x in g[kind + "_block"]], np.uint8)
+    vals = np.array([float(v) for v in g[kind + "_values"]], np.float32)
+    x = S.f32_to_half_bits(vals, "f16")[None, :]
+    assert np.array_equal(orc.llama_quantize_blocks(kind, x)[0, 0], raw)
+
+
+@pytest.mark.parametrize("kind", ["q4_0", "q4_1", "q5_0", "q5_1"])
+@pytest.mark.parametrize("dist", ["normal", "uniform"])
+def test_llama_quantizer_error_bound(orc, kind, dist):
+    """|x - xhat| <= the step (Q4_0/Q5_0: the code range is clamped on one
+    side, so up to one step; Q4_1/Q5_1: half a step) plus what storing d and m
+    in fp16 moves the levels."""
+    D = 256
+    x = S.draw(95, "x", (40, D), dist, "f16")
+    blocks = orc.llama_quantize_blocks(kind, x)
+    xh = orc.llama_block_values(kind, blocks)
+    xf = orc.to_f64(x, "f16")
+    nbytes, has_m, _, off, _ = orc.LLAMA_BLOCKS[kind]
+    xb = xf.reshape(40, D // 32, 32).astype(np.float32)
+    top = 15 if kind.startswith("q4") else 31
+    if has_m:
+        d = ((xb.max(-1) - xb.min(-1)) / np.float32(top)).astype(np.float64)
+        half = 0.5
+        lo = xb.min(-1).astype(np.float64)
+        m16 = orc.f16_to_f32(blocks[..., 2].astype(np.uint16) | (blocks[..., 3].astype(np.uint16) << 8))
+        shift = np.abs(lo - m16.astype(np.float64))
+        reach = top
+    else:
+        i = np.abs(xb).argmax(-1)
+        d = (np.take_along_axis(xb, i[..., None], -1)[..., 0] / np.float32(-off)).astype(np.float64)
+        # half a step, except where the code would pass the top and is clamped
+        t = xb.astype(np.float64) / np.where(d != 0, d, 1.0)[..., None] + off
+        half = np.where(t + 0.5 >= top + 1, 1.0, 0.5)
+        shift = 0.0
+        reach = max(off, top - off)
+    d16 = orc.f16_to_f32(blocks[..., 0].astype(np.uint16) | (blocks[..., 1].astype(np.uint16) << 8))
+    dd = np.abs(d)[..., None]
+    bound = dd * half * (1 + 2.0 ** -20) + (np.abs(d - d16.astype(np.float64)) * reach)[..., None]
+    bound = bound + (shift[..., None] if has_m else 0.0)
+    err = np.abs(xf - xh).reshape(40, D // 32, 32)
+    assert np.all(err <= bound + 1e-12), (err - bound).max()
