@@ -1,7 +1,11 @@
-"""Pins for the oracle's conversion between llama.cpp-style interleaved Q8_0
-blocks (34 bytes: fp16 scale, then 32 int8 codes) and the library's planes
-(CPU only): a hand-derived block, the dequantized values read straight from
-the block bytes, and round trips."""
+"""Pins for the oracle's llama.cpp block formats (CPU only):
+ * Q8_0 blocks (34 bytes: fp16 scale, then 32 int8 codes) <-> the library's
+   planes: a hand-derived block, the dequantized values read straight from the
+   block bytes, round trips;
+ * Q4_0/Q4_1/Q5_0/Q5_1 blocks: hand-built blocks and their values, the affine
+   caches that hold exactly those values;
+ * the reference quantizers for those blocks: the hand-built blocks are fixed
+   points, and a per-element error bound."""
 import numpy as np
 
 from conftest import read_golden
