@@ -12,6 +12,11 @@ What each function follows is stated in ``qkv_oracle.cpp``: the MLX
 quantized-KV branch ("add fast::quantized_kv_update": fast.cpp fallback math,
 sdpa_vector.h packing and dequant, quantized.h eps), the MLX CUDA WIP page
 (load_quantized dequant) and llama.cpp PR #25556 (the Q8_0 KV format).
+
+Parity unpinned: agreement with MLX's or llama.cpp's own quantizer outputs
+(the pages print no quantizer body and no worked example); the quantizers
+(and the llama.cpp block quantizers below, a reading of the published
+reference ones) are pinned only by what their definitions fix.
 """
 from __future__ import annotations
 

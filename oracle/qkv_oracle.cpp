@@ -42,6 +42,11 @@
 //    (query i of Lq sees key j iff j <= L - Lq + i); a row with no visible key
 //    returns zeros.
 //  * attention math in fp64 after exact dequantization.
+//  * parity unpinned: agreement with MLX's or llama.cpp's OWN quantizer
+//    outputs (their rounding choices) -- the pages print neither the
+//    quantizer bodies nor a worked example; the quantizers here are pinned
+//    only by what their definitions fix (error bound, per-element optimality,
+//    min-max structure, hand-derived fixtures).
 //  * extensions that the llama.cpp PR's test coverage lists (sinks, ALiBi,
 //    logit softcap; the pages give no formula for them), in their usual
 //    definitions:
