@@ -224,6 +224,44 @@ def attention(q: np.ndarray, q_dtype: str, k: QCache, v: QCache, L: int,
     return out
 
 
+def attention_dense(q: np.ndarray, q_dtype: str, k: QCache, v: QCache, L: int, scale: float,
+                    causal: bool = False, heads: Optional[Sequence[int]] = None,
+                    row_block: int = 1024) -> np.ndarray:
+    """fp64 attention [B,Hq,Lq,D] evaluated as the definition reads, with
+    library matrix products as its steps (MLX compare, mlx/fast.cpp fallback of
+    quantized_scaled_dot_product_attention: q*scale, S = q K^T, the causal
+    limit, a max-subtracted ("precise") softmax, then P V), over the cache
+    dequantized once by the C oracle (exact fp64 values).  For checking many
+    rows of a large problem in seconds: no additive mask and no extensions.
+    ``heads``: the query heads to compute (others are left NaN).  A row that
+    sees no key is zero, as in :func:`attention`."""
+    q64 = to_f64(q, q_dtype)
+    B, Hq, Lq, D = q64.shape
+    Hkv = k.codes.shape[1]
+    G = Hq // Hkv
+    out = np.full((B, Hq, Lq, D), np.nan)
+    Kd = dequantize(k, D)[:, :, :L]
+    Vd = dequantize(v, D)[:, :, :L]
+    sel = range(Hq) if heads is None else heads
+    j = np.arange(L)
+    for b in range(B):
+        for h in sel:
+            Kh, Vh = Kd[b, h // G], Vd[b, h // G]               # GQA: kv head h // G
+            for i0 in range(0, Lq, row_block):
+                i1 = min(Lq, i0 + row_block)
+                S = (q64[b, h, i0:i1] * scale) @ Kh.T            # [rows, L]
+                if causal:                                       # query i sees j <= L - Lq + i
+                    lim = L - Lq + np.arange(i0, i1)
+                    S = np.where(j[None, :] <= lim[:, None], S, -np.inf)
+                m = S.max(axis=1, keepdims=True)
+                vis = np.isfinite(m)
+                P = np.exp(S - np.where(vis, m, 0.0))
+                den = P.sum(axis=1, keepdims=True)
+                O = (P @ Vh) / np.where(vis, den, 1.0)
+                out[b, h, i0:i1] = np.where(vis, O, 0.0)
+    return out
+
+
 def attention_kview(q: np.ndarray, q_dtype: str, k: QCache, L: int, scale: float, Dv: int,
                     mask: Optional[Mask] = None, mode: str = "two_pass", nsplit: int = 1,
                     rows: Optional[np.ndarray] = None, nthreads: Optional[int] = None,
@@ -360,7 +398,8 @@ def llama_block_values(kind: str, blocks: np.ndarray) -> np.ndarray:
 
 def llama_blocks_to_cache(kind: str, blocks: np.ndarray, Lcap: Optional[int] = None) -> QCache:
     """Blocks uint8 [B, Hkv, L, nb, bytes] -> the affine cache (groups of 32)
-    that holds the same values: scale d, bias m (or -off * d, exact in fp16)."""
+    that holds the same values: scale d, bias m (or -off * d, exact in fp16
+    while |off * d| <= 65504; beyond, the fp16 bias rounds to +-inf)."""
     B, Hkv, L, nb, _ = blocks.shape
     bits = LLAMA_BLOCKS[kind][4]
     Lcap = Lcap or L

@@ -190,3 +190,34 @@ def test_values_as_a_view_of_the_keys_matches_torch(orc, causal):
     for mode, ns in (("two_pass", 1), ("online", 1), ("split", 4)):
         out = orc.attention_kview(q, "f16", kc, L, scale, Dv, mask=mask, mode=mode, nsplit=ns)
         np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("case", CASES)
+@pytest.mark.parametrize("causal", [False, True])
+def test_dense_form_matches_torch_and_the_loops(orc, case, causal):
+    """The matrix-product form (attention_dense, used to check every row of a
+    large prefill) against torch's SDPA in fp64 and against the oracle's own
+    per-row loops, with and without the bottom-right causal limit."""
+    B, Hq, Hkv, Lq, D, L, Lcap, fmt, bits, gs, scale = case
+    kc, vc = _cache(orc, B, Hkv, L, D, fmt, bits, gs, seed=B * 100 + D + 1, Lcap=Lcap)
+    q = S.draw(19, "q", (B, Hq, Lq, D), "normal", "f16")
+    tmask = torch.ones(Lq, L, dtype=torch.bool).tril(diagonal=L - Lq) if causal else None
+    ref = _torch_ref(orc, q, "f16", kc, vc, L, scale, D, attn_mask=tmask)
+    out = orc.attention_dense(q, "f16", kc, vc, L, scale, causal=causal, row_block=2)
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+    loops = orc.attention(q, "f16", kc, vc, L, scale,
+                          mask=orc.Mask("causal") if causal else None)
+    np.testing.assert_allclose(out, loops, rtol=0, atol=1e-12)
+
+
+def test_dense_form_head_subset_and_rows_with_no_key(orc):
+    """Only the requested heads are computed (the rest stay NaN); causal
+    queries placed before the first key return zeros, as in the loops."""
+    B, Hq, Hkv, Lq, D, L = 1, 4, 2, 7, 64, 5
+    kc, vc = _cache(orc, B, Hkv, L, D, "q8_0", 8, 32, seed=23, Lcap=8)
+    q = S.draw(24, "q", (B, Hq, Lq, D), "normal", "f16")
+    out = orc.attention_dense(q, "f16", kc, vc, L, 0.2, causal=True, heads=[1, 2])
+    assert np.isnan(out[0, 0]).all() and np.isnan(out[0, 3]).all()
+    loops = orc.attention(q, "f16", kc, vc, L, 0.2, mask=orc.Mask("causal"))
+    np.testing.assert_allclose(out[0, 1:3], loops[0, 1:3], rtol=0, atol=1e-12)
+    assert np.all(out[0, 1:3, :Lq - L] == 0)

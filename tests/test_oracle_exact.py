@@ -110,3 +110,32 @@ def test_values_as_a_view_of_the_keys_exact(orc):
             want = _exact_row(qrow, K, V, Fraction(1, 8), None, 0.0, [0.3, -2.0][h])
             for e in range(Dv):
                 assert abs(out[0, h, i, e] - float(want[e])) <= 1e-13 * max(1.0, abs(float(want[e])))
+
+
+@pytest.mark.parametrize("fmt,bits,causal", [("affine", 4, False), ("q8_0", 8, True),
+                                             ("affine", 3, True)])
+def test_dense_form_against_exact_arithmetic(orc, fmt, bits, causal):
+    """The matrix-product form of the oracle (attention_dense) on the same
+    tiny problems, against exact logits and a 60-digit softmax; the causal
+    limit is given to the exact side as -inf mask entries."""
+    B, Hq, Hkv, Lq, D, L = 1, 4, 2, 3, 32, 6
+    k = S.draw(85, "k", (B, Hkv, L, D), "normal", "f16")
+    v = S.draw(85, "v", (B, Hkv, L, D), "normal", "f16")
+    q = S.draw(86, "q", (B, Hq, Lq, D), "normal", "f16")
+    kc = orc.quantize(k, "f16", fmt, 32, bits)
+    vc = orc.quantize(v, "f16", fmt, 32, bits)
+    Kd, Vd, qd = orc.dequantize(kc, D), orc.dequantize(vc, D), orc.to_f64(q, "f16")
+    out = orc.attention_dense(q, "f16", kc, vc, L, 0.5, causal=causal)
+    G = Hq // Hkv
+    for h in range(Hq):
+        K = [[Fraction(float(x)) for x in Kd[0, h // G, j]] for j in range(L)]
+        V = [[Fraction(float(x)) for x in Vd[0, h // G, j]] for j in range(L)]
+        for i in range(Lq):
+            madd = None
+            if causal:
+                madd = np.array([0.0 if j <= L - Lq + i else -np.inf for j in range(L)])
+            qrow = [Fraction(float(x)) for x in qd[0, h, i]]
+            want = _exact_row(qrow, K, V, Fraction(1, 2), madd, 0.0, None)
+            for e in range(D):
+                w = float(want[e])
+                assert abs(out[0, h, i, e] - w) <= 1e-13 * max(1.0, abs(w)), (h, i, e)
