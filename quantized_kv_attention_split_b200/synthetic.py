@@ -184,3 +184,47 @@ def make_inputs(w: Workload, L: Optional[int] = None, seed: Optional[int] = None
         nk = draw(seed, "new_k", (w.B, w.Hkv, w.update_tokens, w.D), w.dist, w.kv_dtype)
         nv = draw(seed, "new_v", (w.B, w.Hkv, w.update_tokens, w.D), w.dist, w.kv_dtype)
     return Inputs(q, k, v, nk, nv)
+
+
+# ----------------------------------------------------------------------------
+# edge-case inputs (structure chosen to drive the kernels' rare paths; values
+# are still seeded draws, rounded once to the half type)
+# ----------------------------------------------------------------------------
+def value_spikes(seed: int, shape, dtype: str, period: int, lo_exp: float, hi_exp: float,
+                 gs: int) -> np.ndarray:
+    """[B, Hkv, L, D] raw half bits: U[0,1) values, and in every `period`-th
+    row (a seeded phase per head) one element of each group of `gs` (a
+    seeded position) replaced by 2^e, e growing linearly from lo_exp at row 0
+    to hi_exp at the last row -- magnitudes that grow along the cache."""
+    B, H, L, D = shape
+    x = uniform01(sub_seed(seed, "vs_base"), B * H * L * D).reshape(B, H, L, D)
+    pick = splitmix64(sub_seed(seed, "vs_pick"), B * H * (1 + D // gs))
+    rows = np.arange(L)
+    e = lo_exp + (hi_exp - lo_exp) * rows / max(1, L - 1)
+    k = 0
+    for b in range(B):
+        for h in range(H):
+            phase = int(pick[k] % np.uint64(period)); k += 1
+            sel = rows[(rows % period) == phase]
+            for g in range(D // gs):
+                col = g * gs + int(pick[k] % np.uint64(gs)); k += 1
+                x[b, h, sel, col] = np.exp2(e[sel])
+    return f32_to_half_bits(x, dtype)
+
+
+def key_levels(seed: int, shape, dtype: str, level: np.ndarray, noise: float = 0.1) -> np.ndarray:
+    """[B, Hkv, L, D] raw half bits: row j of every head is level[j] plus
+    `noise` * U[0,1) per element (with queries of positive entries, a row's
+    logit grows with its level, so `level` shapes the logits along the
+    cache: steps, isolated spikes, ramps)."""
+    B, H, L, D = shape
+    u = uniform01(sub_seed(seed, "kl_noise"), B * H * L * D).reshape(B, H, L, D)
+    x = np.asarray(level, np.float32)[None, None, :, None] + np.float32(noise) * u
+    return f32_to_half_bits(x, dtype)
+
+
+def spike_positions(seed: int, L: int, n: int, lo: int = 0) -> np.ndarray:
+    """n distinct seeded row indices in [lo, L), sorted."""
+    r = splitmix64(sub_seed(seed, "spk"), 4 * n)
+    pos = np.unique((r % np.uint64(L - lo)).astype(np.int64) + lo)
+    return pos[:n]
