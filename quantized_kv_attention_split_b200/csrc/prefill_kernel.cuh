@@ -29,6 +29,15 @@
 //     with a lazily moved maximum (moved only when it grows by more than 2^8,
 //     so O in TMEM is rarely rescaled), P as fp16 into TMEM; finally O / l to
 //     the output.
+// Range: the fp16 tiles hold scale * code + bias, which leaves the fp16 range
+// for caches of large values (bf16 inputs, or fp16 ones near its maximum).
+// Once a tile's packed data has landed, the producer warp bounds the tile's
+// K and V magnitudes from its scales and biases and publishes two powers of
+// two: 2^eK for the tile's K (S of the tile is scaled back by 2^eK in the
+// softmax) and 2^eV for V, the largest needed so far (O in TMEM is rescaled
+// exactly when it grows, and scaled back by 2^eV at the end).  Both are 1
+// (exponent 0) unless a tile's values reach 2^15, so ordinary caches take the
+// unscaled path.
 // Every mbarrier wait is bounded: a time-out records an error in the status
 // word and makes every later wait return at once, so all roles finish the
 // tile loop; before exit the CTA waits (bounded) for its own bulk copies and
@@ -172,6 +181,32 @@ __device__ __forceinline__ void mbar_drain(uint32_t addr, uint32_t parity, unsig
     if (mbar_try(addr, parity)) return;
   atomicOr(status, 128u);
 }
+// Per-tile range exponents, published by the producer warp in a ring of 8
+// words of shared memory: ((t + 1) << 10) | (eK << 5) | eV for tile t.  The
+// tag makes every entry self-identifying (no phase to track); the producer is
+// never more than a few tiles ahead of the slowest reader.  Bounded wait that
+// returns -1 on a give-up (and records a time-out like mbar_wait).
+constexpr int kPfRangeRing = 8;
+__device__ __forceinline__ int pf_range_get(const volatile uint32_t* ring, int t,
+                                            volatile int* abort_flag, unsigned* status) {
+  const uint32_t want = (uint32_t)(t + 1) & 0x3fffffu;
+  for (unsigned i = 0; i < kPfWaitLimit; ++i) {
+    const uint32_t v = ring[t & (kPfRangeRing - 1)];
+    if ((v >> 10) == want) return (int)(v & 1023u);
+    if (*abort_flag) return -1;
+    __nanosleep(32);
+  }
+  *abort_flag = 1;
+  atomicOr(status, 256u);
+  return -1;
+}
+// Exponent e >= 0 such that a tile whose values are bounded by `bound` fits
+// below 2^15 once multiplied by 2^-e (0 for bounds below 2^15).
+__device__ __forceinline__ int pf_range_exp(float bound) {
+  const int ex = (int)((__float_as_uint(bound) >> 23) & 0xff) - 127;   // floor(log2 bound)
+  return min(31, max(0, ex - 14));
+}
+
 // One contiguous global -> shared copy completing on an mbarrier (no multicast).
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile(
@@ -328,8 +363,10 @@ struct PfChunks {
   __device__ __forceinline__ static bool has(int chunk0, int it) {
     return NCH % kPfDqThreads == 0 || chunk0 + it * kPfDqThreads < NCH;   // whole warps
   }
+  // e > 0: scale and bias multiplied by 2^-e (exact power of two), so the
+  // converted values stay below 2^15 (see the range note above)
   __device__ __forceinline__ void load(const uint8_t* const raw[2], int codes_off, int sc_off,
-                                       int bi_off, const int nv[2], int chunk0) {
+                                       int bi_off, const int nv[2], int chunk0, int e) {
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
 #pragma unroll
@@ -346,6 +383,16 @@ struct PfChunks {
         b2[h][it] = Q8 ? __float2half2_rn(0.f)
                        : __half2half2(__ushort_as_half(live ? bi[key * C::NG + g] : (uint16_t)0));
       }
+    }
+    if (e != 0) {
+      const __half2 f = __float2half2_rn(exp2i(-e));
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int it = 0; it < ITERS; ++it) {
+          s2[h][it] = __hmul2(s2[h][it], f);
+          b2[h][it] = __hmul2(b2[h][it], f);
+        }
     }
   }
   __device__ __forceinline__ void store(uint8_t* dst, int chunk0) const {
@@ -434,6 +481,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
   auto raw_free = [&](int i) { return bar0 + 120 + 8 * i; };  // [2] a tile's raw slots released
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::BAR_OFF + 144);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::BAR_OFF + 148);
+  volatile uint32_t* range_ring = reinterpret_cast<volatile uint32_t*>(smem + C::BAR_OFF + 160);
 
   const int mt = blockIdx.x % p.mtiles;
   const int hkv = (blockIdx.x / p.mtiles) % p.Hkv;
@@ -467,6 +515,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
     mbar_init(raw_free(1), kPfDqThreads);
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     *abort_flag = 0;
+    for (int i = 0; i < kPfRangeRing; ++i) range_ring[i] = 0u;
   }
   tc_fence_before();
   __syncthreads();
@@ -611,11 +660,14 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
         const int64_t key0 = (int64_t)i * kPfRawKeys;
         nv[h] = !present ? 0 : (L - key0 < kPfRawKeys ? (int)(L - key0) : kPfRawKeys);
       }
+      // the tile's range exponents (0 and 0 unless its values reach 2^15)
+      const int rg = pf_range_get(range_ring, t, abort_flag, p.status);
+      const int eK = rg < 0 ? 0 : rg >> 5, eV = rg < 0 ? 0 : rg & 31;
       // K and V chunks of this thread come in together; V converts after K
       PfChunks<D, BITS, GS, Q8> kch, vch;
-      kch.load(raw, 0, 2 * C::RAW_CODES, 2 * C::RAW_CODES + C::META_BYTES, nv, chunk0);
+      kch.load(raw, 0, 2 * C::RAW_CODES, 2 * C::RAW_CODES + C::META_BYTES, nv, chunk0, eK);
       vch.load(raw, C::RAW_CODES, 2 * C::RAW_CODES + (Q8 ? 1 : 2) * C::META_BYTES,
-               2 * C::RAW_CODES + 3 * C::META_BYTES, nv, chunk0);
+               2 * C::RAW_CODES + 3 * C::META_BYTES, nv, chunk0, eV);
       if (t >= kPfKSlots)                        // K slot free once S of tile t-2 is done
         mbar_wait(s_full(s), ((t - 2) >> 1) & 1, abort_flag, p.status, 1u);
       kch.store(smem + C::K_OFF + s * C::KV_BYTES, chunk0);
@@ -630,9 +682,43 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
     }
   } else if (warp == kPfProdWarp) {
     // ======================= producer warp =====================================
-    for (int t = 0; t + 2 < ntiles || 2 * t + kPfRawSlots < nhalves; ++t) {
+    // Tile t's range exponents are published before the warp waits for the
+    // tile's raw slots to be released (the dequant warps read them first).
+    constexpr float kCodeMax = Q8 ? 128.f : (float)((1 << BITS) - 1);   // largest |code|
+    int eV = 0;                                  // largest V exponent so far
+    for (int t = 0; t < ntiles; ++t) {
+      float bk = 0.f, bv = 0.f;                  // bounds of |scale * code + bias|
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int i = 2 * t + h;
+        if (i >= nhalves) break;
+        const int slot = i % kPfRawSlots;
+        mbar_wait(raw_full(slot), (i / kPfRawSlots) & 1, abort_flag, p.status, 1u);
+        const int64_t key0 = (int64_t)i * kPfRawKeys;
+        const int nv = L - key0 < kPfRawKeys ? (int)(L - key0) : kPfRawKeys;
+        const uint16_t* m = reinterpret_cast<const uint16_t*>(smem + C::RAW_OFF + slot * C::RAW_BYTES +
+                                                              2 * C::RAW_CODES);
+        constexpr int A = C::META_BYTES / 2;     // halves per metadata array
+        for (int j = lane; j < nv * NG; j += 32) {
+          const float sk = fabsf(half_bits_to_float(m[j]));
+          const float sv = fabsf(half_bits_to_float(m[(Q8 ? 1 : 2) * A + j]));
+          const float ak = Q8 ? 0.f : fabsf(half_bits_to_float(m[A + j]));
+          const float av = Q8 ? 0.f : fabsf(half_bits_to_float(m[3 * A + j]));
+          bk = fmaxf(bk, fmaf(sk, kCodeMax, ak));
+          bv = fmaxf(bv, fmaf(sv, kCodeMax, av));
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        bk = fmaxf(bk, __shfl_xor_sync(~0u, bk, off));
+        bv = fmaxf(bv, __shfl_xor_sync(~0u, bv, off));
+      }
+      eV = max(eV, pf_range_exp(bv));
+      if (lane == 0)
+        range_ring[t & (kPfRangeRing - 1)] =
+            (((uint32_t)(t + 1) & 0x3fffffu) << 10) | ((uint32_t)pf_range_exp(bk) << 5) | (uint32_t)eV;
       const int i0 = 2 * t + kPfRawSlots;
-      if (i0 >= nhalves) break;
+      if (i0 >= nhalves) continue;
       mbar_wait(raw_free(t & 1), (t >> 1) & 1, abort_flag, p.status, 1u);
       // warp-uniform decision (issue_raw synchronizes the warp)
       if (__shfl_sync(~0u, (int)*abort_flag, 0) != 0) break;
@@ -708,6 +794,13 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
       const int64_t key0 = (int64_t)t * kPfBN;
       mbar_wait(s_full(s), (t >> 1) & 1, abort_flag, p.status, 8u);
       tc_fence_after();
+      // S of this tile was computed from K * 2^-eK: scale it back
+      // (the ring still holds tile t - 1's entry: the producer is never more
+      // than a few tiles ahead of this role)
+      const int rg = pf_range_get(range_ring, t, abort_flag, p.status);
+      const int eK = rg < 0 ? 0 : rg >> 5;
+      const int dV = rg < 0 || t == 0 ? 0 : (rg & 31) - (int)(range_ring[(t - 1) & (kPfRangeRing - 1)] & 31u);
+      const float rs = eK == 0 ? rowscale : rowscale * exp2i(eK);
       float sv[kPfBN];
       tmem_ld32(tmem_row + C::S_COL + s * kPfBN, reinterpret_cast<uint32_t*>(sv));
       tmem_ld32(tmem_row + C::S_COL + s * kPfBN + 32, reinterpret_cast<uint32_t*>(sv + 32));
@@ -725,7 +818,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
           m0 = fmaxf(m0, fmaxf(sv[j], sv[j + 1]));
           m1 = fmaxf(m1, fmaxf(sv[j + 2], sv[j + 3]));
         }
-        tmax = fmaxf(m0, m1) * rowscale;
+        tmax = fmaxf(m0, m1) * rs;
         if (capped) tmax = softcap_log2(tmax, p.cap_a, p.cap_k);   // the cap is increasing
       } else {
         // per-element path: keys j < lim of the tile are visible (below L and the
@@ -735,7 +828,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
         const int lim = !row_ok || nv <= 0 ? 0 : nv >= kPfBN ? kPfBN : (int)nv;
 #pragma unroll
         for (int j = 0; j < kPfBN; ++j) {
-          float v = sv[j] * rowscale;
+          float v = sv[j] * rs;
           if (capped) v = softcap_log2(v, p.cap_a, p.cap_k);
           sv[j] = j < lim ? v : -INFINITY;
         }
@@ -761,7 +854,10 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
         m_used = tmax;
       }
       const float mref = m_used == -INFINITY ? 0.f : m_used;
-      const bool rescale = t > 0 && __any_sync(~0u, alpha != 1.f);
+      // O also takes the growth of the V exponent (its P V terms from here on
+      // are computed from V * 2^-eV of this tile)
+      const float alpha_o = dV > 0 ? alpha * exp2i(-dV) : alpha;
+      const bool rescale = t > 0 && __any_sync(~0u, alpha_o != 1.f);
       if (rescale) {                             // needs P V of tile t-1 done (rare)
         mbar_wait(pv_done((t - 1) & 1), ((t - 1) >> 1) & 1, abort_flag, p.status, 32u);
         tc_fence_after();
@@ -771,7 +867,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
           tmem_ld32(tmem_row + C::O_COL + c, o);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha_o);
           tmem_st32(tmem_row + C::O_COL + c, o);
         }
       }
@@ -784,8 +880,8 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
         if (full && capped) {
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float a = ex2(softcap_log2(sv[32 * hf + 2 * i] * rowscale, p.cap_a, p.cap_k) - mref);
-            const float c = ex2(softcap_log2(sv[32 * hf + 2 * i + 1] * rowscale, p.cap_a, p.cap_k) - mref);
+            const float a = ex2(softcap_log2(sv[32 * hf + 2 * i] * rs, p.cap_a, p.cap_k) - mref);
+            const float c = ex2(softcap_log2(sv[32 * hf + 2 * i + 1] * rs, p.cap_a, p.cap_k) - mref);
             rs0 += a; rs1 += c;
             pk[i] = pack_half2(a, c);
           }
@@ -793,8 +889,8 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
           const float nm = -mref;
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float a = ex2(fmaf(sv[32 * hf + 2 * i], rowscale, nm));
-            const float c = ex2(fmaf(sv[32 * hf + 2 * i + 1], rowscale, nm));
+            const float a = ex2(fmaf(sv[32 * hf + 2 * i], rs, nm));
+            const float c = ex2(fmaf(sv[32 * hf + 2 * i + 1], rs, nm));
             rs0 += a; rs1 += c;
             pk[i] = pack_half2(a, c);
           }
@@ -828,7 +924,9 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
       fo = ex2(m_used - Mn);
       lsum = lsum * fo + ex2(s2 - Mn);
     }
-    const float inv = (lsum > 0.f && have) ? fo / lsum : 0.f;
+    // O carries 2^-eV of the last tile (the largest V exponent)
+    const int eVend = ntiles > 0 ? (int)(range_ring[(ntiles - 1) & (kPfRangeRing - 1)] & 31u) : 0;
+    const float inv = (lsum > 0.f && have) ? fo / lsum * exp2i(eVend) : 0.f;
 #pragma unroll 1
     for (int c = 0; c < D; c += 32) {
       uint32_t ob[32];
