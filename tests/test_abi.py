@@ -194,3 +194,34 @@ def test_header_is_plain_c(tmp_path):
                         "-I", os.path.join(ROOT, "include"), "-o", str(tmp_path / "use_qkv.o")],
                        capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
+
+
+def test_noalloc_validation_matches_decode(lib):
+    """qsdpa_decode_noalloc rejects what qsdpa_decode rejects, with the same
+    status, before it looks up its scratch or launches anything."""
+    from quantized_kv_attention_split_b200 import qkv
+    f = lib.qsdpa_decode_noalloc
+    f.argtypes = [C.c_void_p, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
+                  C.POINTER(qkv._Cache), C.POINTER(qkv._Cache), C.c_int64, C.c_float,
+                  C.POINTER(qkv._Mask), C.c_void_p, C.c_int, C.c_void_p]
+    f.restype = C.c_int
+    ok = _cache(qkv)
+
+    def na(k, v, D=128, L=16, Hq=8, Hkv=2):
+        return f(FAKE, 0, 1, Hq, Hkv, D, C.byref(k), C.byref(v), L, 1.0, None, FAKE + 65536, 0,
+                 None)
+    cases = [
+        dict(k=ok, v=ok, D=96),                                   # unsupported D
+        dict(k=_cache(qkv, bits=5), v=ok),                        # unsupported bits
+        dict(k=_cache(qkv, gs=48), v=ok),                         # unsupported group
+        dict(k=_cache(qkv, Lcap=60), v=_cache(qkv, Lcap=60)),     # Lcap alignment
+        dict(k=_cache(qkv, biases=0), v=ok),                      # affine without biases
+        dict(k=ok, v=ok, L=65),                                   # L > Lcap
+        dict(k=ok, v=ok, L=-1),
+        dict(k=ok, v=ok, Hq=6, Hkv=4),                            # Hq % Hkv
+    ]
+    for c in cases:
+        want = _decode(lib, qkv, c["k"], c["v"], D=c.get("D", 128), L=c.get("L", 16),
+                       Hq=c.get("Hq", 8), Hkv=c.get("Hkv", 2))
+        assert want != 0
+        assert na(**c) == want, c

@@ -49,3 +49,19 @@ def test_block_strides():
     assert qkv._block_strides(t, None) == (3 * 5 * 136, 5 * 136, 136)
     assert qkv._block_strides(t, (7, 8, 9)) == (7, 8, 9)
     assert qkv.LLAMA_BLOCKS["q5_1"] == (3, 24, 8) and qkv.Q8_0_BLOCK_BYTES == 34
+
+
+def test_calls_switch_to_the_tensors_device(monkeypatch):
+    """A call whose tensors live on a device that is not the current one runs
+    with that device made current (launch, default stream, workspace size);
+    on the current device nothing is switched."""
+    import contextlib
+
+    class Fake:
+        def __init__(self, dev):
+            self.device = dev
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    assert isinstance(qkv._on(Fake(torch.device("cuda", 0))), contextlib.nullcontext)
+    assert isinstance(qkv._on(Fake(torch.device("cpu"))), contextlib.nullcontext)
+    ctx = qkv._on(Fake(torch.device("cuda", 3)))
+    assert isinstance(ctx, torch.cuda.device) and ctx.idx == 3

@@ -129,3 +129,24 @@ def test_llama_quantizer_error_bound(orc, kind, dist):
     bound = bound + (shift[..., None] if has_m else 0.0)
     err = np.abs(xf - xh).reshape(40, D // 32, 32)
     assert np.all(err <= bound + 1e-12), (err - bound).max()
+
+
+@pytest.mark.parametrize("kind,d_ok,d_over", [("q4_0", 8188.0, 8192.0), ("q5_0", 4094.0, 4096.0)])
+def test_offset_bias_range_limit(orc, kind, d_ok, d_over):
+    """The _0 blocks become affine groups with bias -8d (Q4_0) or -16d (Q5_0),
+    stored in fp16: exact up to |bias| = 65504 (d = 8188 / 4094), and +-inf
+    beyond (d = 8192 / 4096), where the block's own values leave the fp16
+    range.  All codes zero: every value equals the bias."""
+    nbytes, _, _, off, _ = orc.LLAMA_BLOCKS[kind]
+    for d, finite in ((d_ok, True), (d_over, False), (-d_ok, True), (-d_over, False)):
+        raw = np.zeros((1, 1, 1, 1, nbytes), np.uint8)
+        db = int(S.f32_to_half_bits(np.array([d], np.float32), "f16")[0])
+        raw[..., 0], raw[..., 1] = db & 0xFF, db >> 8
+        c = orc.llama_blocks_to_cache(kind, raw)
+        bias = float(orc.f16_to_f32(c.biases.ravel())[0])
+        if finite:
+            assert bias == -off * d and abs(bias) == 65504.0
+            assert np.array_equal(orc.dequantize(c, 32).ravel(), orc.llama_block_values(kind, raw).ravel())
+        else:
+            assert np.isinf(bias) and np.sign(bias) == -np.sign(d)
+            assert np.all(np.abs(orc.llama_block_values(kind, raw)) > 65504)
