@@ -243,7 +243,11 @@ qkv_status qkv_q8_0_to_blocks(const qkv_cache* src, int B, int Hkv, int D, int64
  * nibble; the fifth bit of element e is bit e of qh).  dst: affine, group_size
  * 32, bits 4 for Q4 and 8 for Q5.  Rows, strides, offset and alignment as for
  * qkv_q8_0_from_blocks (with the block sizes above).  The decode and prefill
- * calls then read the cache like any affine cache.  One launch. */
+ * calls then read the cache like any affine cache.  One launch.
+ * Range: the bias -8d (Q4_0) or -16d (Q5_0) is exact in fp16 for |d| <= 8188
+ * (Q4_0) or |d| <= 4094 (Q5_0); a block with a larger d holds values outside
+ * the fp16 range, its bias is stored as +-inf and attention over it returns
+ * non-finite values (the conversion itself reports no error). */
 typedef enum { QKV_BLOCKS_Q4_0 = 0, QKV_BLOCKS_Q4_1 = 1, QKV_BLOCKS_Q5_0 = 2,
                QKV_BLOCKS_Q5_1 = 3 } qkv_block_kind;
 qkv_status qkv_llama_blocks_to_cache(int kind, const void* blocks, int B, int Hkv, int D,

@@ -463,8 +463,15 @@ extern "C" qkv_status qsdpa_decode_noalloc(const void* q, int q_dtype, int B, in
                                            int D, const qkv_cache* k, const qkv_cache* v,
                                            int64_t L, float scale, const qkv_mask* mask,
                                            void* out, int out_dtype, void* stream) {
-  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0)
-    return fail(QKV_ERR_INVALID_ARG, "B, Hq, Hkv must be positive and Hq a multiple of Hkv");
+  // the checks qsdpa_decode makes first, in its order, so that both entry
+  // points return the same status for a shape neither can run
+  if (B <= 0 || Hq <= 0 || Hkv <= 0)
+    return fail(QKV_ERR_INVALID_ARG, "B, Hq, Hkv and Lq must be positive");
+  if (Hq % Hkv != 0) return fail(QKV_ERR_INVALID_ARG, "Hq=%d is not a multiple of Hkv=%d", Hq, Hkv);
+  qkv_status st;
+  if ((st = check_cache("k", k, D)) != QKV_OK) return st;
+  if ((st = check_cache("v", v, D)) != QKV_OK) return st;
+  if (L < 0 || L > k->Lcap) return fail(QKV_ERR_INVALID_ARG, "L=%lld outside [0, Lcap]", (long long)L);
   const size_t need = qsdpa_workspace_size(B, Hq, Hkv, 1, D, L);
   if (need == 0) return fail(QKV_ERR_INVALID_ARG, "invalid decode shape (D=%d, L=%lld)", D,
                              (long long)L);
@@ -474,7 +481,7 @@ extern "C" qkv_status qsdpa_decode_noalloc(const void* q, int q_dtype, int B, in
                 "%zu bytes built into the library; use qsdpa_decode with a caller workspace",
                 need, kNoAllocScratchBytes);
   void* scratch = nullptr;
-  qkv_status st = noalloc_scratch(&scratch);
+  st = noalloc_scratch(&scratch);
   if (st != QKV_OK) return st;
   // decode keeps no state in its scratch between calls (the header that
   // qsdpa_workspace_zero_bytes covers is the prefill's), so nothing to clear

@@ -107,8 +107,10 @@ __global__ void __launch_bounds__(256) qkv_q8_0_to_block_pairs_kernel(const __gr
 // then fp16 m (HAS_M), then the 32 fifth bits qh (HAS_QH, bit e for element
 // e), then qs[16]: element j < 16 in the low nibble of qs[j], element j + 16
 // in the high one) into an affine cache with groups of 32 holding the same
-// values: scale d, bias m or -OFF * d (a power-of-two multiple: exact in
-// fp16), codes BITS wide in the library's packing (element e at bits
+// values: scale d, bias m or -OFF * d (a power-of-two multiple of an fp16
+// value: exact while |OFF * d| <= 65504, i.e. |d| <= 8188 for Q4_0 and 4094
+// for Q5_0; a larger d gives a block whose values leave the fp16 range, and
+// its bias rounds to +-inf), codes BITS wide in the library's packing (element e at bits
 // BITS*(e % (32/BITS)) of word e / (32/BITS)).  One thread per block.
 template <int NBYTES, bool HAS_M, bool HAS_QH, int OFF, int BITS>
 __global__ void __launch_bounds__(256) qkv_llama_blocks_kernel(const __grid_constant__ BlocksParams p) {

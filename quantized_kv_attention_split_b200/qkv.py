@@ -9,6 +9,7 @@ library is missing or a call fails, a Python exception is raised.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes as C
 import os
 from dataclasses import dataclass
@@ -113,6 +114,16 @@ def _stream(stream) -> Optional[int]:
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
 
 
+def _on(t: torch.Tensor):
+    """Context in which t's device is the current one: the library launches on
+    the current device (and the default stream is the current device's), so a
+    call whose tensors live on another device switches to it first."""
+    idx = t.device.index
+    if idx is None or idx == torch.cuda.current_device():
+        return contextlib.nullcontext()
+    return torch.cuda.device(idx)
+
+
 @dataclass
 class QuantCache:
     """One of K or V in the library's layout (all tensors on one CUDA device):
@@ -175,9 +186,10 @@ def qkv_quantize_update(new_k: torch.Tensor, new_v: torch.Tensor, k: QuantCache,
     assert new_k.shape == new_v.shape and new_k.dtype == new_v.dtype
     B, Hkv, Lnew, D = new_k.shape
     ks, vs = k._struct(), v._struct()
-    _check(lib().qkv_quantize_update(new_k.data_ptr(), new_v.data_ptr(), _DTYPE[new_k.dtype],
-                                     B, Hkv, Lnew, D, C.byref(ks), C.byref(vs), int(offset),
-                                     _stream(stream)))
+    with _on(new_k):
+        _check(lib().qkv_quantize_update(new_k.data_ptr(), new_v.data_ptr(), _DTYPE[new_k.dtype],
+                                         B, Hkv, Lnew, D, C.byref(ks), C.byref(vs), int(offset),
+                                         _stream(stream)))
 
 
 def qkv_dequantize(c: QuantCache, L: int, out: Optional[torch.Tensor] = None,
@@ -190,7 +202,9 @@ def qkv_dequantize(c: QuantCache, L: int, out: Optional[torch.Tensor] = None,
         out = torch.empty(B, Hkv, L, D, dtype=torch.float16, device=c.codes.device)
     assert out.is_contiguous() and out.dtype == torch.float16 and tuple(out.shape) == (B, Hkv, L, D)
     cs = c._struct()
-    _check(lib().qkv_dequantize(C.byref(cs), B, Hkv, D, int(L), out.data_ptr(), _stream(stream)))
+    with _on(out):
+        _check(lib().qkv_dequantize(C.byref(cs), B, Hkv, D, int(L), out.data_ptr(),
+                                    _stream(stream)))
     return out
 
 
@@ -217,8 +231,9 @@ def qkv_q8_0_from_blocks(blocks: torch.Tensor, c: QuantCache, offset: int = 0,
         L = blocks.shape[2]
     sb, sh, sl = _block_strides(blocks, strides)
     cs = c._struct()
-    _check(lib().qkv_q8_0_from_blocks(blocks.data_ptr(), B, Hkv, D, int(L), sb, sh, sl,
-                                      C.byref(cs), int(offset), _stream(stream)))
+    with _on(blocks):
+        _check(lib().qkv_q8_0_from_blocks(blocks.data_ptr(), B, Hkv, D, int(L), sb, sh, sl,
+                                          C.byref(cs), int(offset), _stream(stream)))
     return c
 
 
@@ -238,8 +253,9 @@ def qkv_llama_blocks_to_cache(kind: str, blocks: torch.Tensor, c: QuantCache, of
         L = blocks.shape[2]
     sb, sh, sl = _block_strides(blocks, strides)
     cs = c._struct()
-    _check(lib().qkv_llama_blocks_to_cache(code, blocks.data_ptr(), B, Hkv, D, int(L), sb, sh, sl,
-                                           C.byref(cs), int(offset), _stream(stream)))
+    with _on(blocks):
+        _check(lib().qkv_llama_blocks_to_cache(code, blocks.data_ptr(), B, Hkv, D, int(L), sb, sh,
+                                               sl, C.byref(cs), int(offset), _stream(stream)))
     return c
 
 
@@ -255,8 +271,9 @@ def qkv_q8_0_to_blocks(c: QuantCache, L: int, offset: int = 0,
                           device=c.codes.device)
     sb, sh, sl = _block_strides(out, strides)
     cs = c._struct()
-    _check(lib().qkv_q8_0_to_blocks(C.byref(cs), B, Hkv, D, int(offset), int(L), out.data_ptr(),
-                                    sb, sh, sl, _stream(stream)))
+    with _on(out):
+        _check(lib().qkv_q8_0_to_blocks(C.byref(cs), B, Hkv, D, int(offset), int(L),
+                                        out.data_ptr(), sb, sh, sl, _stream(stream)))
     return out
 
 
@@ -293,19 +310,21 @@ def _attention(fn, q, k, v, L, scale, mask, causal, out, out_dtype, workspace, s
     if out is None:
         out = torch.empty(B, Hq, Lq, D, dtype=out_dtype or q.dtype, device=q.device)
     if workspace is None:
-        workspace = make_workspace(B, Hq, Hkv, Lq, D, L, q.device)
+        with _on(q):                       # sized for the device that runs the call
+            workspace = make_workspace(B, Hq, Hkv, Lq, D, L, q.device)
     ks, vs = k._struct(), v._struct()
     m = _mask_struct(mask, causal)
     mp = C.byref(m) if m is not None else None
     common = (C.byref(ks), C.byref(vs), int(L), float(scale), mp)
     if ext is not None:
         common += (C.byref(ext),)
-    common += (out.data_ptr(), _DTYPE[out.dtype], workspace.data_ptr(), workspace.numel(),
-               _stream(stream))
-    if decode:
-        _check(fn(q.data_ptr(), _DTYPE[q.dtype], B, Hq, Hkv, D, *common))
-    else:
-        _check(fn(q.data_ptr(), _DTYPE[q.dtype], B, Hq, Hkv, Lq, D, *common))
+    with _on(q):
+        common += (out.data_ptr(), _DTYPE[out.dtype], workspace.data_ptr(), workspace.numel(),
+                   _stream(stream))
+        if decode:
+            _check(fn(q.data_ptr(), _DTYPE[q.dtype], B, Hq, Hkv, D, *common))
+        else:
+            _check(fn(q.data_ptr(), _DTYPE[q.dtype], B, Hq, Hkv, Lq, D, *common))
     return out
 
 
@@ -339,15 +358,17 @@ def qsdpa_decode_update(q: torch.Tensor, new_k: torch.Tensor, new_v: torch.Tenso
     if out is None:
         out = torch.empty(B, Hq, 1, D, dtype=out_dtype or q.dtype, device=q.device)
     if workspace is None:
-        workspace = make_workspace(B, Hq, Hkv, 1, D, L_old + 1, q.device)
+        with _on(q):
+            workspace = make_workspace(B, Hq, Hkv, 1, D, L_old + 1, q.device)
     ks, vs = k._struct(), v._struct()
     m = _mask_struct(mask, False)
     mp = C.byref(m) if m is not None else None
-    _check(lib().qsdpa_decode_update(q.data_ptr(), _DTYPE[q.dtype], new_k.data_ptr(),
-                                     new_v.data_ptr(), _DTYPE[new_k.dtype], B, Hq, Hkv, D,
-                                     C.byref(ks), C.byref(vs), int(L_old), float(scale), mp,
-                                     out.data_ptr(), _DTYPE[out.dtype], workspace.data_ptr(),
-                                     workspace.numel(), _stream(stream)))
+    with _on(q):
+        _check(lib().qsdpa_decode_update(q.data_ptr(), _DTYPE[q.dtype], new_k.data_ptr(),
+                                         new_v.data_ptr(), _DTYPE[new_k.dtype], B, Hq, Hkv, D,
+                                         C.byref(ks), C.byref(vs), int(L_old), float(scale), mp,
+                                         out.data_ptr(), _DTYPE[out.dtype], workspace.data_ptr(),
+                                         workspace.numel(), _stream(stream)))
     return out
 
 
@@ -386,7 +407,8 @@ def qsdpa_decode_noalloc(q: torch.Tensor, k: QuantCache, v: QuantCache, L: int, 
         out = torch.empty(B, Hq, 1, D, dtype=out_dtype or q.dtype, device=q.device)
     ks, vs = k._struct(), v._struct()
     m = _mask_struct(mask, False)
-    _check(f(q.data_ptr(), _DTYPE[q.dtype], B, Hq, Hkv, D, C.byref(ks), C.byref(vs), int(L),
-             float(scale), C.byref(m) if m is not None else None, out.data_ptr(),
-             _DTYPE[out.dtype], _stream(stream)))
+    with _on(q):
+        _check(f(q.data_ptr(), _DTYPE[q.dtype], B, Hq, Hkv, D, C.byref(ks), C.byref(vs), int(L),
+                 float(scale), C.byref(m) if m is not None else None, out.data_ptr(),
+                 _DTYPE[out.dtype], _stream(stream)))
     return out
