@@ -254,6 +254,28 @@ def graph_time(step, K, W, sampler=None, min_window_s=0.3, tag=None, sync_ranks=
     return ms / K, extra
 
 
+def isolated_time(step, n=20, flush_bytes=512 << 20):
+    """Median device time of single calls that overlap nothing: before each
+    call the L2 is flushed by reading flush_bytes (more than the 126 MB L2;
+    a read leaves clean lines, so the call pays no write-backs) and the
+    stream drains, so the call neither starts early nor finds its data in
+    L2; events bracket the call alone."""
+    import torch
+    buf = torch.ones(flush_bytes // 8, dtype=torch.int64, device="cuda")
+    times = []
+    for i in range(n + 2):
+        buf.sum()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        step(i)
+        e1.record()
+        torch.cuda.synchronize()
+        if i >= 2:
+            times.append(e0.elapsed_time(e1) / 1e3)
+    del buf
+    return statistics.median(times)
+
+
 def oracle_rows_time(w, host_k, host_v, q_bits, nrows_target_s=15.0, max_rows=None):
     """Time the CPU oracle on a sample of query rows of the workload."""
     import oracle
@@ -350,6 +372,8 @@ def run_ours(args, rank, world, device):
 
     sec = max_over_ranks(sec, device, world)
     gbs = alg_bytes / sec / 1e9
+    # one call alone (cold L2, no overlap with a previous call)
+    iso_sec = max_over_ranks(isolated_time(step), device, world)
 
     # e2e through the public API with host buffers: H2D of q, decode, D2H of out
     q_host = torch.from_numpy(inp.q.view(np.int16)).view(torch.float16).pin_memory()
@@ -385,6 +409,7 @@ def run_ours(args, rank, world, device):
             "value": round(replica_rate(alg_bytes, sec, world) / 1e9, 2),
             "unit": "GB/s",
             "us_per_call": round(sec * 1e6, 3),
+            "us_per_call_isolated": round(iso_sec * 1e6, 3),
             "n_gpus": world,
             "steps": args.steps,
             "warmup": args.warmup,
@@ -400,7 +425,10 @@ def run_ours(args, rank, world, device):
                        "algorithmic_bytes_per_call": alg_bytes,
                        "l2": f"inputs larger than L2: {ncopies} rotating cache copies "
                              f"({ncopies * cache_bytes / 1e6:.0f} MB)",
-                       "timing": "CUDA events around CUDA-graph replays of exactly K calls",
+                       "timing": "CUDA events around CUDA-graph replays of exactly K back-to-back "
+                                 "calls (a call may start while the previous one finishes: its "
+                                 "set-up and L2 prefetch overlap that call's tail); "
+                                 "us_per_call_isolated: median of single calls after an L2 flush",
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
             "roofline": {"bound": "hbm", "achieved": round(gbs, 2), "peak": hbm_peak,
                          "unit": "GB/s", "frac": round(gbs / hbm_peak, 4),

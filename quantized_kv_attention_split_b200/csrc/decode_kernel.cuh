@@ -193,12 +193,6 @@ __device__ __forceinline__ void lds_meta(const uint8_t* p, uint16_t* h) {
   }
 }
 
-// a / b for non-negative 64-bit values, in 32-bit arithmetic when both fit
-// (the common case; 64-bit division costs several times more instructions).
-__device__ __forceinline__ int64_t udiv64(int64_t a, int64_t b) {
-  if (((uint64_t)a | (uint64_t)b) >> 32 == 0) return (int64_t)((uint32_t)a / (uint32_t)b);
-  return a / b;
-}
 
 // Transposing shared-memory matrix loads (8x8 of 16-bit elements per matrix).
 __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1,

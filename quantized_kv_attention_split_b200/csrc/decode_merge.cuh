@@ -1,32 +1,29 @@
-// decode_merge.cuh -- second pass of the split-K decode: the log-sum-exp merge
-// of the per-CTA partials (m_i, l_i, o_i) of every split unit,
-//   M = max_i m_i,  l = sum_i l_i 2^(m_i - M),  out = sum_i o_i 2^(m_i - M) / l
-// (base-2 logits), the same rule the online softmax applies within a CTA; a
-// head's attention-sink logit s, when given, joins as l += 2^(s - M).
+// decode_merge.cuh -- second pass of the split-K decode, as its own kernel:
+// the log-sum-exp merge (decode_fold.cuh) of the per-CTA partials of every
+// split unit.
 #pragma once
 
 #include "qkv_common.cuh"
 #include "qkv_internal.h"
-#include "decode_kernel.cuh"
+#include "decode_fold.cuh"
 
 namespace qkv {
 
 // ---------------------------------------------------------------------------
-// Merge of split units: after the decode grid has completed, `lanes` adjacent
-// threads (a power of two up to 4, chosen so that a thread's share of the
-// parts fits one batch of loads) per (unit, row, 4 consecutive outputs) fold
-// the unit's partials -- one per CTA that covered part of the unit, every
-// lanes-th one per thread -- by log-sum-exp rescaling, combine across the
-// lanes with shuffles and write the normalized output.  A unit that one CTA
-// covered whole was written by that CTA.
+// Merge of split units: after the decode grid has completed, `lanes`
+// adjacent threads (a power of two up to 4, chosen so that a thread's share of
+// the parts fits one batch of loads) per (unit, row, 4 consecutive outputs)
+// fold the unit's partials.  A unit that one CTA covered whole was written by
+// that CTA.  (Folding in the decode kernel instead -- the last CTA of a unit,
+// found with an atomic count, folds the others' partials -- measured slower:
+// the count's round trip and the fold sit on the grid's critical path.)
 constexpr int kMergeThreads = 128;
-constexpr int kMergeBatch = 8;   // parts whose loads a thread has in flight
 
 template <int D, int HPC>
 __global__ void __launch_bounds__(kMergeThreads)
 qsdpa_merge_kernel(const __grid_constant__ DecodeParams p, int64_t nC, int lanes) {
+  grid_dep_launch();             // the next kernel may take SMs as this one's CTAs finish
   grid_dep_wait();               // the decode grid's partials are complete and visible
-  grid_dep_launch();
   constexpr int V4 = D / 4;
   const int64_t S = p.stages_per_unit, T = p.total_stages;
   const int gt = blockIdx.x * kMergeThreads + threadIdx.x;
@@ -38,84 +35,11 @@ qsdpa_merge_kernel(const __grid_constant__ DecodeParams p, int64_t nC, int lanes
   const int head = (u - uh * p.ncg) * HPC + R;
   const int units = (int)udiv64(T, S);
   bool active = u < units && head < p.G;
-  int64_t cfirst, slot0;
-  int n;
-  if (p.pieces > 0) {
-    // every CTA covered one piece of one unit: CTAs u*pieces ... in order
-    cfirst = (int64_t)u * p.pieces;
-    n = p.pieces;
-    slot0 = 2 * cfirst;
-  } else {
-    // CTA c covered blocks [c*T/nC, (c+1)*T/nC): the unit's first and last CTA
-    cfirst = active ? udiv64(((int64_t)u * S + 1) * nC - 1, T) : 0;
-    const int64_t clast = active ? udiv64(((int64_t)u + 1) * S * nC - 1, T) : 0;
-    n = (int)(clast - cfirst + 1);
-    // the first CTA used its second slot if its range began in an earlier unit
-    slot0 = 2 * cfirst + (udiv64(udiv64(cfirst * T, nC), S) == u ? 0 : 1);
-  }
-  active = active && n > 1;
-  float M = -INFINITY, Ls = 0.f;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int j0 = 0; active && sub + lanes * j0 < n; j0 += kMergeBatch) {
-    float4 o[kMergeBatch];
-    float2 v[kMergeBatch];
-#pragma unroll
-    for (int k = 0; k < kMergeBatch; ++k) {
-      const int pp = sub + lanes * (j0 + k);
-      if (pp < n) {
-        const int64_t sx = pp == 0 ? slot0 : 2 * (cfirst + pp);
-        o[k] = __ldcg(reinterpret_cast<const float4*>(p.part_o + (sx * HPC + R) * D) + e4);
-        v[k] = __ldcg(reinterpret_cast<const float2*>(p.part_ml + (sx * HPC + R) * 2));
-      } else {
-        o[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-        v[k] = make_float2(-INFINITY, 0.f);
-      }
-    }
-    float Mb = M;
-#pragma unroll
-    for (int k = 0; k < kMergeBatch; ++k) Mb = fmaxf(Mb, v[k].x);
-    if (Mb != M) {
-      const float f = M == -INFINITY ? 0.f : ex2(M - Mb);
-      Ls *= f; acc.x *= f; acc.y *= f; acc.z *= f; acc.w *= f;
-      M = Mb;
-    }
-#pragma unroll
-    for (int k = 0; k < kMergeBatch; ++k) {
-      const float w = v[k].x == -INFINITY ? 0.f : ex2(v[k].x - M);
-      Ls = fmaf(w, v[k].y, Ls);
-      acc.x = fmaf(w, o[k].x, acc.x);
-      acc.y = fmaf(w, o[k].y, acc.y);
-      acc.z = fmaf(w, o[k].z, acc.z);
-      acc.w = fmaf(w, o[k].w, acc.w);
-    }
-  }
-  for (int off = 1; off < lanes; off <<= 1) {
-    const float M2 = __shfl_xor_sync(~0u, M, off), L2 = __shfl_xor_sync(~0u, Ls, off);
-    const float x2 = __shfl_xor_sync(~0u, acc.x, off), y2 = __shfl_xor_sync(~0u, acc.y, off);
-    const float z2 = __shfl_xor_sync(~0u, acc.z, off), w2 = __shfl_xor_sync(~0u, acc.w, off);
-    const float Mn = fmaxf(M, M2);
-    const float f1 = M == -INFINITY ? 0.f : ex2(M - Mn), f2 = M2 == -INFINITY ? 0.f : ex2(M2 - Mn);
-    Ls = Ls * f1 + L2 * f2;
-    acc.x = acc.x * f1 + x2 * f2; acc.y = acc.y * f1 + y2 * f2;
-    acc.z = acc.z * f1 + z2 * f2; acc.w = acc.w * f1 + w2 * f2;
-    M = Mn;
-  }
-  if (!active || sub != 0) return;
-  float fo = 1.f;
-  if (p.sinks != nullptr && Ls > 0.f) {
-    // the head's sink logit joins the denominator: (M, l) -> (max(M, s), l 2^(M - M') + 2^(s - M'))
-    const int hkv = uh - (uh / p.Hkv) * p.Hkv;
-    const float s2 = kLog2e * p.sinks[hkv * p.Gq + head / p.Lq];
-    const float Mn = fmaxf(M, s2);
-    fo = ex2(M - Mn);
-    Ls = Ls * fo + ex2(s2 - Mn);
-  }
-  const float inv = Ls > 0.f ? fo / Ls : 0.f;
-  const int64_t oi = ((int64_t)uh * p.G + head) * D + e4 * 4;
-  store_from_float(p.out, p.out_dtype, oi, acc.x * inv);
-  store_from_float(p.out, p.out_dtype, oi + 1, acc.y * inv);
-  store_from_float(p.out, p.out_dtype, oi + 2, acc.z * inv);
-  store_from_float(p.out, p.out_dtype, oi + 3, acc.w * inv);
+  UnitParts up;
+  up.cfirst = 0; up.slot0 = 0; up.n = 0;
+  if (active) up = unit_parts(p, u, nC);
+  active = active && up.n > 1;
+  merge_item<D, HPC>(p, up, uh, head, R, e4, sub, lanes, active);
 }
 
 }  // namespace qkv

@@ -108,6 +108,13 @@ __device__ __forceinline__ void store_from_float(void* p, int dtype, int64_t i, 
 __device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
 __device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
 
+// a / b for non-negative 64-bit values, in 32-bit arithmetic when both fit
+// (the common case; 64-bit division costs several times more instructions).
+__device__ __forceinline__ int64_t udiv64(int64_t a, int64_t b) {
+  if (((uint64_t)a | (uint64_t)b) >> 32 == 0) return (int64_t)((uint32_t)a / (uint32_t)b);
+  return a / b;
+}
+
 // 2^k as float for integer k in [-126, 127].
 __device__ __forceinline__ float exp2i(int k) {
   return __uint_as_float(static_cast<uint32_t>(k + 127) << 23);

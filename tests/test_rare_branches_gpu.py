@@ -208,7 +208,7 @@ def test_prefill_mixed_magnitudes_along_the_cache(qkv):
     qs = S.f32_to_half_bits(oracle.bf16_to_f32(q) * np.float32(2.0 ** -14), "bf16")
     kc = oracle.quantize(S.f32_to_half_bits(k * f, "bf16"), "bf16", "q8_0")
     vc = oracle.quantize(S.f32_to_half_bits(v * f, "bf16"), "bf16", "q8_0")
-    scale = 0.5
+    scale = 1.0 / np.sqrt(D)
     ref = oracle.attention(qs, "bf16", kc, vc, L_, scale, mask=oracle.Mask("causal"))
     out = qkv.qsdpa_prefill(to_dev(qs, "bf16"), cache_to_dev(kc), cache_to_dev(vc), L_, scale,
                             causal=True, out_dtype=torch.bfloat16)
