@@ -680,6 +680,39 @@ def other_rows(device):
         rows["llama_q4_0_blocks_64k"] = {"unavailable": f"{type(e).__name__}: {e}"[:200]}
     torch.cuda.empty_cache()
 
+    # llama.cpp's reference Q4_0 / Q5_1 quantizers on the GPU: 65536 tokens of
+    # K and V (the main decode shape) into token-major blocks, and one new
+    # token of every head written straight into the affine caches
+    try:
+        w = S.WORKLOADS["decode_64k_affine4"]
+        nbk = w.D // 32
+        inp = S.make_inputs(w)
+        kx, vx = dev16(inp.k, "f16", device), dev16(inp.v, "f16", device)
+        for kind, nbytes, bits in (("q4_0", 18, 4), ("q5_1", 24, 8)):
+            ob = torch.empty(w.B, w.L, w.Hkv * nbk * nbytes, dtype=torch.uint8, device=device)
+            st = (w.L * w.Hkv * nbk * nbytes, nbk * nbytes, w.Hkv * nbk * nbytes)
+            sec, _ = graph_time(lambda i: (qkv.qkv_llama_quantize_blocks(kind, kx, out=ob, strides=st),
+                                           qkv.qkv_llama_quantize_blocks(kind, vx, out=ob, strides=st)),
+                                50, 5)
+            moved = 2 * (kx.numel() * 2 + ob.numel())
+            dk = qkv.QuantCache.empty(w.B, w.Hkv, 64, w.D, qkv.AFFINE, bits, 32, device)
+            dv = qkv.QuantCache.empty(w.B, w.Hkv, 64, w.D, qkv.AFFINE, bits, 32, device)
+            nk, nv = kx[:, :, :1].contiguous(), vx[:, :, :1].contiguous()
+            sec1, _ = graph_time(lambda i: qkv.qkv_llama_quantize_update(kind, nk, nv, dk, dv, 63),
+                                 200, 10)
+            rows[f"llama_{kind}_quantize_64k"] = {
+                "us_per_call": round(sec * 1e3, 3), "GB/s": round(moved / (sec / 1e3) / 1e9, 1),
+                "frac_hbm": round(moved / (sec / 1e3) / 1e9 / hbm_peak, 4),
+                "update_1tok_us": round(sec1 * 1e3, 3),
+                "note": f"qkv_llama_quantize_blocks, K and V of 65536 tokens x 8 heads (2 x 16.8 MB "
+                        f"fp16 in) to token-major {kind} blocks; update_1tok: "
+                        f"qkv_llama_quantize_update of one token per head into the affine caches"}
+            del ob, dk, dv
+        del kx, vx
+    except Exception as e:
+        rows["llama_q4_0_quantize_64k"] = {"unavailable": f"{type(e).__name__}: {e}"[:200]}
+    torch.cuda.empty_cache()
+
     # the attention extensions on the main decode workload (the extension
     # variant of the decode kernel): logit softcap 30 with per-head sinks, and
     # ALiBi (a broadcast fp32 distance mask with per-head slopes)

@@ -255,6 +255,45 @@ qkv_status qkv_llama_blocks_to_cache(int kind, const void* blocks, int B, int Hk
                                      int64_t stride_l, const qkv_cache* dst, int64_t offset,
                                      void* stream);
 
+/* The same block formats written on the GPU (the PR's follow-up keeps the KV
+ * cache in these types, so a cache imported from llama.cpp is extended in its
+ * own format).  The quantizer is llama.cpp's published reference one (not on
+ * the pages), per block of 32 elements in fp32 IEEE operations in this order:
+ *   Q4_0 / Q5_0: m = the element of largest magnitude (the first such),
+ *                d = m / -8 (Q5_0: m / -16), id = d == 0 ? 0 : 1/d,
+ *                q = min(15 (31), trunc(x*id + 8.5 (16.5)))
+ *   Q4_1 / Q5_1: lo, hi = min, max, d = (hi - lo) / 15 (31),
+ *                id = d == 0 ? 0 : 1/d, q = min(15 (31), trunc((x - lo)*id + 0.5)),
+ *                m = lo
+ * with d and m stored as fp16 (round to nearest even) and the codes computed
+ * from the fp32 d; bit-identical to the CPU oracle.
+ *  qkv_llama_quantize_blocks: x [B, Hkv, L, D] contiguous, f16 or bf16,
+ *    16-byte aligned -> the blocks of tokens [0, L), placed by the byte
+ *    strides as for qkv_q8_0_from_blocks (blocks and strides 2-byte aligned;
+ *    offset the blocks pointer to append).  D in {64, 128, 256}.
+ *  qkv_llama_quantize_update: new_k / new_v [B, Hkv, Lnew, D] (f16 or bf16,
+ *    16-byte aligned) quantized the same way and written into rows
+ *    [offset, offset + Lnew) of affine caches with group_size 32 (4-bit codes
+ *    for Q4, 8-bit for Q5) exactly as qkv_llama_blocks_to_cache would import
+ *    the resulting blocks (scale d, bias m, or -8d / -16d rounded to fp16 from
+ *    the fp16 d).  Two launches (K, then V).
+ *  qkv_llama_cache_to_blocks: rows [offset, offset + L) of such an affine
+ *    cache -> blocks (d = scale, m = bias, the codes' low bits).  The blocks
+ *    hold the rows' values exactly for groups that blocks of that kind can
+ *    hold -- codes below 16 (Q4) or 32 (Q5), and for Q4_0 / Q5_0 a bias of
+ *    -8 (-16) times the scale: the groups written by the import and the
+ *    quantizers above.  One launch.
+ * L == 0 / Lnew == 0 do nothing. */
+qkv_status qkv_llama_quantize_blocks(int kind, const void* x, int in_dtype, int B, int Hkv, int D,
+                                     int64_t L, void* blocks, int64_t stride_b, int64_t stride_h,
+                                     int64_t stride_l, void* stream);
+qkv_status qkv_llama_quantize_update(int kind, const void* new_k, const void* new_v, int in_dtype,
+                                     int B, int Hkv, int Lnew, int D, const qkv_cache* k,
+                                     const qkv_cache* v, int64_t offset, void* stream);
+qkv_status qkv_llama_cache_to_blocks(int kind, const qkv_cache* src, int B, int Hkv, int D,
+                                     int64_t offset, int64_t L, void* blocks, int64_t stride_b,
+                                     int64_t stride_h, int64_t stride_l, void* stream);
+
 /* Allocation-free variant of qsdpa_decode (the pages have no counterpart:
  * MLX and llama.cpp allocate their temporaries through their own allocators).
  * For callers that cannot allocate device memory when they decode -- code

@@ -51,8 +51,9 @@ qkv_status check_cache(const char* name, const qkv_cache* c, int D) {
   if (c->fmt != QKV_AFFINE && c->fmt != QKV_Q8_0)
     return fail(QKV_ERR_INVALID_ARG, "%s: unknown format %d", name, c->fmt);
   if (c->fmt == QKV_AFFINE) {
-    if (c->bits != 4 && c->bits != 8)
-      return fail(QKV_ERR_UNSUPPORTED, "%s: affine bits must be 4 or 8 (got %d)", name, c->bits);
+    if (c->bits != 2 && c->bits != 3 && c->bits != 4 && c->bits != 5 && c->bits != 6 && c->bits != 8)
+      return fail(QKV_ERR_UNSUPPORTED, "%s: affine bits must be 2, 3, 4, 5, 6 or 8 (got %d)", name,
+                  c->bits);
     if (c->group_size != 32 && c->group_size != 64 && c->group_size != 128)
       return fail(QKV_ERR_UNSUPPORTED, "%s: group_size must be 32, 64 or 128 (got %d)", name,
                   c->group_size);
@@ -149,7 +150,10 @@ qkv_status attention(const void* q, int q_dtype, int B, int Hq, int Hkv, int Lq,
 
   const int G = Hq / Hkv;
   const int rows = G * Lq;                 // rows of one kv head: (head, query) pairs
-  if (Lq > 1 && rows >= kTensorPrefillMinRows && out_dtype != QKV_F32) {
+  // the tcgen05 kernel dequantizes 4- and 8-bit codes; other widths take the
+  // split-K kernel
+  const bool tc_codes = k->fmt == QKV_Q8_0 || k->bits == 4 || k->bits == 8;
+  if (Lq > 1 && rows >= kTensorPrefillMinRows && out_dtype != QKV_F32 && tc_codes) {
     // many query rows per kv head: the tcgen05 kernel (whole 128-row tiles)
     const size_t need = qsdpa_workspace_size(B, Hq, Hkv, Lq, D, L);
     if (workspace == nullptr || workspace_bytes < need)
@@ -185,8 +189,10 @@ qkv_status attention(const void* q, int q_dtype, int B, int Hq, int Hkv, int Lq,
                         : (extended || mkind == QKV_MASK_ADDITIVE) ? qkv::kDecExt : qkv::kDecPlain;
   if (!qkv::plan_decode(D, k->bits, k->group_size, k->fmt, out_dtype == QKV_F32, var, B,
                         Hkv * rows, Hkv, L, &plan))
-    return fail(QKV_ERR_UNSUPPORTED, "no kernel for D=%d bits=%d group_size=%d", D, k->bits,
-                k->group_size);
+    return fail(QKV_ERR_UNSUPPORTED,
+                "no kernel for D=%d bits=%d group_size=%d%s", D, k->bits, k->group_size,
+                (k->bits == 4 || k->bits == 8 || k->fmt == QKV_Q8_0)
+                    ? "" : " (2/3/5/6-bit codes: no additive mask, extensions or fused update)");
   if (plan.ws_total > 0) {
     if (workspace == nullptr || workspace_bytes < plan.ws_total)
       return fail(QKV_ERR_WORKSPACE, "workspace of %zu bytes required (got %zu)", plan.ws_total,
@@ -340,6 +346,79 @@ qkv_status qkv_llama_blocks_to_cache(int kind, const void* blocks, int B, int Hk
   cudaError_t e = qkv::launch_llama_blocks(kind, blocks, dst, B, Hkv, D, offset, L, stride_b, stride_h,
                                            stride_l, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(QKV_ERR_CUDA, "block conversion launch: %s", cudaGetErrorString(e));
+  return ok();
+}
+
+qkv_status qkv_llama_quantize_blocks(int kind, const void* x, int in_dtype, int B, int Hkv, int D,
+                                     int64_t L, void* blocks, int64_t stride_b, int64_t stride_h,
+                                     int64_t stride_l, void* stream) {
+  if (kind < QKV_BLOCKS_Q4_0 || kind > QKV_BLOCKS_Q5_1)
+    return fail(QKV_ERR_INVALID_ARG, "unknown block kind %d", kind);
+  if (B <= 0 || Hkv <= 0 || L < 0) return fail(QKV_ERR_INVALID_ARG, "B, Hkv must be positive, L >= 0");
+  if (D != 64 && D != 128 && D != 256)
+    return fail(QKV_ERR_UNSUPPORTED, "head dimension must be 64, 128 or 256 (got %d)", D);
+  if (in_dtype != QKV_F16 && in_dtype != QKV_BF16)
+    return fail(QKV_ERR_INVALID_ARG, "x must be f16 or bf16 (got %d)", in_dtype);
+  if (L == 0) return ok();
+  if (x == nullptr || blocks == nullptr) return fail(QKV_ERR_INVALID_ARG, "x and blocks must be non-NULL");
+  if (!aligned16(x)) return fail(QKV_ERR_ALIGNMENT, "x must be 16-byte aligned");
+  if (stride_b < 0 || stride_h < 0 || stride_l < 0)
+    return fail(QKV_ERR_INVALID_ARG, "block strides must be non-negative");
+  if ((reinterpret_cast<uintptr_t>(blocks) & 1u) != 0 || ((stride_b | stride_h | stride_l) & 1) != 0)
+    return fail(QKV_ERR_ALIGNMENT, "blocks and their strides must be 2-byte aligned");
+  cudaError_t e = qkv::launch_llama_quantize(kind, x, in_dtype, B, Hkv, D, L, blocks, stride_b,
+                                             stride_h, stride_l, nullptr, 0,
+                                             static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(QKV_ERR_CUDA, "block quantize launch: %s", cudaGetErrorString(e));
+  return ok();
+}
+
+qkv_status qkv_llama_quantize_update(int kind, const void* new_k, const void* new_v, int in_dtype,
+                                     int B, int Hkv, int Lnew, int D, const qkv_cache* k,
+                                     const qkv_cache* v, int64_t offset, void* stream) {
+  if (kind < QKV_BLOCKS_Q4_0 || kind > QKV_BLOCKS_Q5_1)
+    return fail(QKV_ERR_INVALID_ARG, "unknown block kind %d", kind);
+  const int bits = (kind == QKV_BLOCKS_Q4_0 || kind == QKV_BLOCKS_Q4_1) ? 4 : 8;
+  if (B <= 0 || Hkv <= 0 || Lnew < 0) return fail(QKV_ERR_INVALID_ARG, "B, Hkv must be positive, Lnew >= 0");
+  qkv_status st;
+  for (const qkv_cache* c : {k, v}) {
+    if ((st = check_cache(c == k ? "k" : "v", c, D)) != QKV_OK) return st;
+    if (c->fmt != QKV_AFFINE || c->group_size != 32 || c->bits != bits)
+      return fail(QKV_ERR_UNSUPPORTED,
+                  "these blocks need an affine cache with group_size 32 and %d-bit codes", bits);
+  }
+  if (in_dtype != QKV_F16 && in_dtype != QKV_BF16)
+    return fail(QKV_ERR_INVALID_ARG, "new tokens must be f16 or bf16 (got %d)", in_dtype);
+  if (offset < 0 || offset + Lnew > k->Lcap || offset + Lnew > v->Lcap)
+    return fail(QKV_ERR_INVALID_ARG, "offset=%lld with Lnew=%d exceeds Lcap", (long long)offset, Lnew);
+  if (Lnew == 0) return ok();
+  if (new_k == nullptr || new_v == nullptr)
+    return fail(QKV_ERR_INVALID_ARG, "new_k and new_v must be non-NULL");
+  if (!aligned16(new_k) || !aligned16(new_v))
+    return fail(QKV_ERR_ALIGNMENT, "new_k and new_v must be 16-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = qkv::launch_llama_quantize(kind, new_k, in_dtype, B, Hkv, D, Lnew, nullptr, 0, 0, 0,
+                                             k, offset, s);
+  if (e == cudaSuccess)
+    e = qkv::launch_llama_quantize(kind, new_v, in_dtype, B, Hkv, D, Lnew, nullptr, 0, 0, 0, v,
+                                   offset, s);
+  if (e != cudaSuccess) return fail(QKV_ERR_CUDA, "block quantize launch: %s", cudaGetErrorString(e));
+  return ok();
+}
+
+qkv_status qkv_llama_cache_to_blocks(int kind, const qkv_cache* src, int B, int Hkv, int D,
+                                     int64_t offset, int64_t L, void* blocks, int64_t stride_b,
+                                     int64_t stride_h, int64_t stride_l, void* stream) {
+  if (kind < QKV_BLOCKS_Q4_0 || kind > QKV_BLOCKS_Q5_1)
+    return fail(QKV_ERR_INVALID_ARG, "unknown block kind %d", kind);
+  const int bits = (kind == QKV_BLOCKS_Q4_0 || kind == QKV_BLOCKS_Q4_1) ? 4 : 8;
+  qkv_status st = check_blocks_args(src, B, Hkv, D, offset, L, blocks, stride_b, stride_h, stride_l,
+                                    QKV_AFFINE, bits);
+  if (st != QKV_OK) return st;
+  if (L == 0) return ok();
+  cudaError_t e = qkv::launch_llama_export(kind, src, B, Hkv, D, offset, L, blocks, stride_b,
+                                           stride_h, stride_l, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(QKV_ERR_CUDA, "block export launch: %s", cudaGetErrorString(e));
   return ok();
 }
 

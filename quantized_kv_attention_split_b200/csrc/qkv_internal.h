@@ -93,6 +93,12 @@ cudaError_t launch_dequantize(const qkv_cache* c, int B, int Hkv, int D, int64_t
 cudaError_t launch_llama_blocks(int kind, const void* src_blocks, const qkv_cache* c, int B, int Hkv,
                                 int D, int64_t offset, int64_t L, int64_t sb, int64_t sh,
                                 int64_t sl, cudaStream_t stream);
+cudaError_t launch_llama_quantize(int kind, const void* x, int in_dtype, int B, int Hkv, int D,
+                                  int64_t L, void* blocks, int64_t sb, int64_t sh, int64_t sl,
+                                  const qkv_cache* c, int64_t offset, cudaStream_t stream);
+cudaError_t launch_llama_export(int kind, const qkv_cache* c, int B, int Hkv, int D, int64_t offset,
+                                int64_t L, void* blocks, int64_t sb, int64_t sh, int64_t sl,
+                                cudaStream_t stream);
 cudaError_t launch_q8_0_blocks(bool to_blocks, const void* src_blocks, void* dst_blocks,
                                const qkv_cache* c, int B, int Hkv, int D, int64_t offset, int64_t L,
                                int64_t sb, int64_t sh, int64_t sl, cudaStream_t stream);

@@ -89,6 +89,14 @@ def lib() -> C.CDLL:
         L.qkv_llama_blocks_to_cache.argtypes = [i32, p, i32, i32, i32, i64, i64, i64, i64, cp,
                                                 i64, p]
         L.qkv_llama_blocks_to_cache.restype = i32
+        L.qkv_llama_quantize_blocks.argtypes = [i32, p, i32, i32, i32, i32, i64, p, i64, i64, i64,
+                                                p]
+        L.qkv_llama_quantize_blocks.restype = i32
+        L.qkv_llama_quantize_update.argtypes = [i32, p, p, i32, i32, i32, i32, i32, cp, cp, i64, p]
+        L.qkv_llama_quantize_update.restype = i32
+        L.qkv_llama_cache_to_blocks.argtypes = [i32, cp, i32, i32, i32, i64, i64, p, i64, i64, i64,
+                                                p]
+        L.qkv_llama_cache_to_blocks.restype = i32
         L.qkv_dequantize.argtypes = [cp, i32, i32, i32, i64, p, p]
         L.qkv_dequantize.restype = i32
         L.qsdpa_workspace_size.argtypes = [i32, i32, i32, i32, i32, i64]
@@ -257,6 +265,57 @@ def qkv_llama_blocks_to_cache(kind: str, blocks: torch.Tensor, c: QuantCache, of
         _check(lib().qkv_llama_blocks_to_cache(code, blocks.data_ptr(), B, Hkv, D, int(L), sb, sh,
                                                sl, C.byref(cs), int(offset), _stream(stream)))
     return c
+
+
+def qkv_llama_quantize_blocks(kind: str, x: torch.Tensor, out: Optional[torch.Tensor] = None,
+                              strides=None, stream=None) -> torch.Tensor:
+    """llama.cpp's reference quantizer for Q4_0/Q4_1/Q5_0/Q5_1 on the GPU:
+    x [B, Hkv, L, D] (f16/bf16) -> blocks (uint8, [B, Hkv, L, D/32*bytes]
+    unless `out` and `strides` say otherwise)."""
+    code, nbytes, _ = LLAMA_BLOCKS[kind]
+    assert x.is_contiguous() and x.is_cuda
+    B, Hkv, L, D = x.shape
+    if out is None:
+        out = torch.empty(B, Hkv, L, D // 32 * nbytes, dtype=torch.uint8, device=x.device)
+    sb, sh, sl = _block_strides(out, strides)
+    with _on(x):
+        _check(lib().qkv_llama_quantize_blocks(code, x.data_ptr(), _DTYPE[x.dtype], B, Hkv, D,
+                                               int(L), out.data_ptr(), sb, sh, sl,
+                                               _stream(stream)))
+    return out
+
+
+def qkv_llama_quantize_update(kind: str, new_k: torch.Tensor, new_v: torch.Tensor, k: QuantCache,
+                              v: QuantCache, offset: int, stream=None) -> None:
+    """Quantize new_k/new_v [B, Hkv, Lnew, D] with llama.cpp's reference
+    quantizer of `kind` and write rows [offset, offset+Lnew) of the affine
+    caches (group 32; 4-bit for Q4, 8-bit for Q5) holding the blocks' values."""
+    code, _, _ = LLAMA_BLOCKS[kind]
+    assert new_k.is_contiguous() and new_v.is_contiguous() and new_k.shape == new_v.shape
+    B, Hkv, Lnew, D = new_k.shape
+    ks, vs = k._struct(), v._struct()
+    with _on(new_k):
+        _check(lib().qkv_llama_quantize_update(code, new_k.data_ptr(), new_v.data_ptr(),
+                                               _DTYPE[new_k.dtype], B, Hkv, Lnew, D, C.byref(ks),
+                                               C.byref(vs), int(offset), _stream(stream)))
+
+
+def qkv_llama_cache_to_blocks(kind: str, c: QuantCache, L: int, offset: int = 0,
+                              out: Optional[torch.Tensor] = None, strides=None,
+                              stream=None) -> torch.Tensor:
+    """Rows [offset, offset+L) of an affine cache (group 32) as llama.cpp blocks
+    of `kind` (uint8, [B, Hkv, L, D/32*bytes] unless `out`/`strides` given)."""
+    code, nbytes, _ = LLAMA_BLOCKS[kind]
+    B, Hkv = c.codes.shape[0], c.codes.shape[1]
+    D = c.codes.shape[3] * 32 // c.bits
+    if out is None:
+        out = torch.empty(B, Hkv, L, D // 32 * nbytes, dtype=torch.uint8, device=c.codes.device)
+    sb, sh, sl = _block_strides(out, strides)
+    cs = c._struct()
+    with _on(out):
+        _check(lib().qkv_llama_cache_to_blocks(code, C.byref(cs), B, Hkv, D, int(offset), int(L),
+                                               out.data_ptr(), sb, sh, sl, _stream(stream)))
+    return out
 
 
 def qkv_q8_0_to_blocks(c: QuantCache, L: int, offset: int = 0,

@@ -50,7 +50,7 @@ def _decode(lib, qkv, k, v, D=128, L=16, q=FAKE, out=FAKE + 65536, qdt=0, odt=0,
 def test_decode_validation_errors(lib):
     from quantized_kv_attention_split_b200 import qkv
     ok = _cache(qkv)
-    assert _decode(lib, qkv, _cache(qkv, bits=5), ok) == 2                 # unsupported bits
+    assert _decode(lib, qkv, _cache(qkv, bits=7), ok) == 2                 # unsupported bits
     assert b"bits" in lib.qkv_last_error()
     assert _decode(lib, qkv, _cache(qkv, gs=48), ok) == 2                  # unsupported group
     assert _decode(lib, qkv, ok, ok, D=96) == 2                            # unsupported D
@@ -79,7 +79,7 @@ def test_quantize_validation_errors(lib):
     assert f(FAKE, FAKE, 2, 1, 2, 4, 128, C.byref(ok), C.byref(ok), 0, None) == 1   # f32 input
     assert f(FAKE + 8, FAKE, 0, 1, 2, 4, 128, C.byref(ok), C.byref(ok), 0, None) == 3
     assert f(0, FAKE, 0, 1, 2, 4, 128, C.byref(ok), C.byref(ok), 0, None) == 1
-    assert f(FAKE, FAKE, 0, 1, 2, 4, 128, C.byref(_cache(qkv, bits=3)), C.byref(ok), 0, None) == 2
+    assert f(FAKE, FAKE, 0, 1, 2, 4, 128, C.byref(_cache(qkv, bits=7)), C.byref(ok), 0, None) == 2
     assert f(FAKE, FAKE, 0, 1, 2, 0, 128, C.byref(ok), C.byref(ok), 0, None) == 0   # nothing to do
 
 
@@ -109,7 +109,7 @@ def test_decode_update_validation_errors(lib):
     assert call(idt=2) == 1                        # new tokens must be 16-bit
     assert call(nk=0) == 1                         # NULL new_k
     assert call(nv=FAKE + 2056) == 3               # misaligned new_v
-    assert call(k=_cache(qkv, bits=5)) == 2        # unsupported format
+    assert call(k=_cache(qkv, bits=7)) == 2        # unsupported format
 
 
 def test_dequantize_validation_errors(lib):
@@ -212,7 +212,7 @@ def test_noalloc_validation_matches_decode(lib):
                  None)
     cases = [
         dict(k=ok, v=ok, D=96),                                   # unsupported D
-        dict(k=_cache(qkv, bits=5), v=ok),                        # unsupported bits
+        dict(k=_cache(qkv, bits=7), v=ok),                        # unsupported bits
         dict(k=_cache(qkv, gs=48), v=ok),                         # unsupported group
         dict(k=_cache(qkv, Lcap=60), v=_cache(qkv, Lcap=60)),     # Lcap alignment
         dict(k=_cache(qkv, biases=0), v=ok),                      # affine without biases
@@ -225,3 +225,24 @@ def test_noalloc_validation_matches_decode(lib):
                        Hq=c.get("Hq", 8), Hkv=c.get("Hkv", 2))
         assert want != 0
         assert na(**c) == want, c
+
+
+def test_llama_quantize_and_export_validation_errors(lib):
+    from quantized_kv_attention_split_b200 import qkv
+    a4 = _cache(qkv, fmt=0, bits=4, gs=32)
+    a8 = _cache(qkv, fmt=0, bits=8, gs=32)
+    st = (64 * 4 * 18, 4 * 18, 2 * 4 * 18)
+    qb, qu, ex = lib.qkv_llama_quantize_blocks, lib.qkv_llama_quantize_update, lib.qkv_llama_cache_to_blocks
+    assert qb(7, FAKE, 0, 1, 2, 128, 16, FAKE, *st, None) == 1                # unknown kind
+    assert qb(0, FAKE, 2, 1, 2, 128, 16, FAKE, *st, None) == 1                # f32 input
+    assert qb(0, FAKE, 0, 1, 2, 96, 16, FAKE, *st, None) == 2                 # unsupported D
+    assert qb(0, FAKE + 8, 0, 1, 2, 128, 16, FAKE, *st, None) == 3            # misaligned x
+    assert qb(0, FAKE, 0, 1, 2, 128, 16, FAKE + 1, *st, None) == 3            # odd blocks address
+    assert qb(0, FAKE, 0, 1, 2, 128, 0, FAKE, *st, None) == 0                 # nothing to do
+    assert qu(0, FAKE, FAKE, 0, 1, 2, 4, 128, C.byref(a8), C.byref(a8), 0, None) == 2   # Q4 into 8-bit
+    assert qu(2, FAKE, FAKE, 0, 1, 2, 4, 128, C.byref(a8), C.byref(a8), 61, None) == 1  # past Lcap
+    assert qu(1, FAKE + 8, FAKE, 0, 1, 2, 4, 128, C.byref(a4), C.byref(a4), 0, None) == 3
+    assert qu(3, FAKE, FAKE, 0, 1, 2, 0, 128, C.byref(a8), C.byref(a8), 0, None) == 0
+    assert ex(1, C.byref(a8), 1, 2, 128, 0, 16, FAKE, *st, None) == 2        # Q4 from 8-bit
+    assert ex(2, C.byref(a8), 1, 2, 128, 60, 16, FAKE, *st, None) == 1       # past Lcap
+    assert ex(0, C.byref(a4), 1, 2, 128, 0, 16, FAKE + 1, *st, None) == 3    # odd address

@@ -107,3 +107,87 @@ def test_llama_blocks_to_cache_matches_oracle_and_decodes(kind):
     torch.cuda.synchronize()
     ref = oracle.attention(q, "f16", hk, hv, L_all, 0.125)
     assert out_err(from_dev(out), ref, "f16") <= 1.0
+
+
+# ---------------------------------------------------------------------------
+# Q4_0 / Q4_1 / Q5_0 / Q5_1 written on the GPU
+# ---------------------------------------------------------------------------
+def _block_inputs(B, Hkv, L, D, dtype, seed):
+    """Normal and uniform draws, plus blocks of special structure: all zeros,
+    a constant block, a block whose largest magnitude appears twice with both
+    signs (the first one sets d), and values on the half-way points of the
+    codes of a previous quantization."""
+    x = S.draw(seed, "x", (B, Hkv, L, D), "normal", dtype)
+    u = S.draw(seed, "u", (B, Hkv, L, D), "uniform", dtype)
+    x[:, :, 1::3] = u[:, :, 1::3]
+    f = (oracle.f16_to_f32 if dtype == "f16" else oracle.bf16_to_f32)(x)
+    f[0, 0, 0, :32] = 0.0
+    f[0, 0, 0, 32:64] = 1.5
+    if D >= 128:
+        f[0, 0, 0, 64:96] = np.linspace(-1, 1, 32, dtype=np.float32)
+        f[0, 0, 0, 70], f[0, 0, 0, 90] = -2.0, 2.0
+    if L > 1:
+        f[0, 0, 1, :32] = (np.arange(32, dtype=np.float32) - 8.0) * 0.125 + 0.0625
+    return S.f32_to_half_bits(f, dtype)
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+@pytest.mark.parametrize("kind", ["q4_0", "q4_1", "q5_0", "q5_1"])
+def test_llama_quantize_blocks_bit_exact(kind, dtype):
+    """The GPU reference quantizer writes exactly the oracle's blocks, in
+    llama.cpp's token-major layout (K: [token][kv head][blocks])."""
+    from quantized_kv_attention_split_b200 import qkv
+    B, Hkv, L, D = 2, 3, 57, 128
+    nb, nbytes = D // 32, oracle.LLAMA_BLOCKS[kind][0]
+    x = _block_inputs(B, Hkv, L, D, dtype, 81)
+    want = oracle.llama_quantize_blocks(kind, x, dtype)           # [B,Hkv,L,nb,bytes]
+    out = torch.zeros(B, L, Hkv, nb * nbytes, dtype=torch.uint8, device="cuda")
+    st = (L * Hkv * nb * nbytes, nb * nbytes, Hkv * nb * nbytes)
+    qkv.qkv_llama_quantize_blocks(kind, to_dev(x, dtype), out=out, strides=st)
+    torch.cuda.synchronize()
+    got = out.cpu().numpy().reshape(B, L, Hkv, nb, nbytes).transpose(0, 2, 1, 3, 4)
+    assert np.array_equal(got, want), np.argwhere(got != want)[:5]
+
+
+@pytest.mark.parametrize("kind", ["q4_0", "q4_1", "q5_0", "q5_1"])
+def test_llama_quantize_update_extends_an_imported_cache(kind):
+    """A cache imported from llama.cpp blocks is extended in its own format:
+    new tokens quantized with the same reference quantizer land in the affine
+    cache exactly as the import would write their blocks; the cache then
+    exports back to exactly the blocks (old and new), and decodes like the
+    oracle over all of it."""
+    from quantized_kv_attention_split_b200 import qkv
+    B, Hq, Hkv, D, L0, Lnew = 1, 16, 2, 128, 700, 37
+    nb, nbytes, bits = D // 32, oracle.LLAMA_BLOCKS[kind][0], oracle.LLAMA_BLOCKS[kind][4]
+    Lcap = ((L0 + Lnew) // 8 + 1) * 8
+    dev_caches, all_blocks = [], []
+    for which in (0, 1):
+        old = oracle.llama_quantize_blocks(kind, S.draw(82 + which, "o", (B, Hkv, L0, D), "normal",
+                                                        "f16"))
+        new_x = _block_inputs(B, Hkv, Lnew, D, "f16", 84 + which)
+        new = oracle.llama_quantize_blocks(kind, new_x)
+        dc = qkv.QuantCache.empty(B, Hkv, Lcap, D, qkv.AFFINE, bits, 32)
+        qkv.qkv_llama_blocks_to_cache(kind, torch.from_numpy(
+            np.ascontiguousarray(old.reshape(B, Hkv, L0, nb * nbytes))).cuda(), dc)
+        dev_caches.append((dc, to_dev(new_x, "f16")))
+        all_blocks.append(np.concatenate([old, new], axis=2))
+    (dk, nk), (dv, nv) = dev_caches
+    qkv.qkv_llama_quantize_update(kind, nk, nv, dk, dv, L0)
+    torch.cuda.synchronize()
+    hosts = []
+    for dc, blocks in zip((dk, dv), all_blocks):
+        ref = oracle.llama_blocks_to_cache(kind, blocks)
+        h = cache_from_dev(dc, "affine")
+        L_all = L0 + Lnew
+        assert np.array_equal(h.codes[:, :, :L_all], ref.codes)
+        assert np.array_equal(h.scales[:, :, :L_all], ref.scales)
+        assert np.array_equal(h.biases[:, :, :L_all], ref.biases)
+        back = qkv.qkv_llama_cache_to_blocks(kind, dc, L_all)
+        torch.cuda.synchronize()
+        assert np.array_equal(back.cpu().numpy().reshape(blocks.shape), blocks)
+        hosts.append(h)
+    q = S.draw(86, "q", (B, Hq, 1, D), "normal", "f16")
+    out = qkv.qsdpa_decode(to_dev(q, "f16"), dk, dv, L0 + Lnew, 0.125)
+    torch.cuda.synchronize()
+    ref = oracle.attention(q, "f16", hosts[0], hosts[1], L0 + Lnew, 0.125)
+    assert out_err(from_dev(out), ref, "f16") <= 1.0
