@@ -9,13 +9,13 @@
 namespace qkv {
 
 // Host-side helpers for one instance.
-template <int D, int BITS, int GS, bool Q8, int NC, bool F32OUT, int VAR>
+template <int D, int BITS, int GS, bool Q8, int NC, bool F32OUT, int VAR, int SB = BITS>
 struct DecodeInstance {
-  using C = DecCfg<D, BITS, GS, Q8, NC>;
+  using C = DecCfg<D, BITS, GS, Q8, NC, SB>;
   static int max_ctas_per_sm() {
     static int cached = -1;
     if (cached < 0) {
-      auto k = qsdpa_decode_kernel<D, BITS, GS, Q8, NC, F32OUT, VAR>;
+      auto k = qsdpa_decode_kernel<D, BITS, GS, Q8, NC, F32OUT, VAR, SB>;
       if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
         return 0;
       int n = 0;
@@ -38,7 +38,7 @@ struct DecodeInstance {
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, qsdpa_decode_kernel<D, BITS, GS, Q8, NC, F32OUT, VAR>, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, qsdpa_decode_kernel<D, BITS, GS, Q8, NC, F32OUT, VAR, SB>, p);
     if (e != cudaSuccess || !plan.merge) return e;
     // parts per unit: at most the CTAs that share one unit
     const int64_t parts = plan.pieces > 0 ? plan.pieces : (plan.grid + plan.units - 1) / plan.units + 1;
@@ -62,9 +62,9 @@ struct DecodeOps {
   size_t smem;
 };
 
-template <int D, int BITS, int GS, bool Q8, int NC, bool F32, int VAR>
+template <int D, int BITS, int GS, bool Q8, int NC, bool F32, int VAR, int SB = BITS>
 DecodeOps make_decode_ops() {
-  using I = DecodeInstance<D, BITS, GS, Q8, NC, F32, VAR>;
+  using I = DecodeInstance<D, BITS, GS, Q8, NC, F32, VAR, SB>;
   return DecodeOps{&I::max_ctas_per_sm, &I::launch, I::C::TK, NC, I::C::NTEAM, (size_t)I::C::SMEM};
 }
 
@@ -109,8 +109,40 @@ bool decode_ops_for(int bits, int gs, bool q8, int nc, bool f32, int var, Decode
   return false;
 }
 
+// Affine codes stored 2, 3, 5 or 6 bits wide: the plain kernel (no additive
+// mask, no extensions, no fused update), transcoding each block to 8-bit.
+template <int D>
+bool decode_ops_x_for(int bits, int gs, int nc, bool f32, DecodeOps* ops) {
+#define QKV_DEC_X(SB, GS)                                                                      \
+  do {                                                                                         \
+    if (nc == 1) *ops = f32 ? make_decode_ops<D, 8, GS, false, 1, true, kDecPlain, SB>()       \
+                            : make_decode_ops<D, 8, GS, false, 1, false, kDecPlain, SB>();     \
+    else if (nc == 2) *ops = f32 ? make_decode_ops<D, 8, GS, false, 2, true, kDecPlain, SB>()  \
+                                 : make_decode_ops<D, 8, GS, false, 2, false, kDecPlain, SB>(); \
+    else *ops = f32 ? make_decode_ops<D, 8, GS, false, 4, true, kDecPlain, SB>()               \
+                    : make_decode_ops<D, 8, GS, false, 4, false, kDecPlain, SB>();             \
+    return true;                                                                               \
+  } while (0)
+#define QKV_DEC_XB(SB)                                      \
+  do {                                                      \
+    if (gs == 32) QKV_DEC_X(SB, 32);                        \
+    if (gs == 64) QKV_DEC_X(SB, 64);                        \
+    if constexpr (D >= 128) { if (gs == 128) QKV_DEC_X(SB, 128); } \
+  } while (0)
+  if (bits == 2) QKV_DEC_XB(2);
+  if (bits == 3) QKV_DEC_XB(3);
+  if (bits == 5) QKV_DEC_XB(5);
+  if (bits == 6) QKV_DEC_XB(6);
+#undef QKV_DEC_XB
+#undef QKV_DEC_X
+  return false;
+}
+
 bool decode_ops_d64(int bits, int gs, bool q8, int nc, bool f32, int var, DecodeOps* ops);
 bool decode_ops_d128(int bits, int gs, bool q8, int nc, bool f32, int var, DecodeOps* ops);
 bool decode_ops_d256(int bits, int gs, bool q8, int nc, bool f32, int var, DecodeOps* ops);
+bool decode_ops_x_d64(int bits, int gs, int nc, bool f32, DecodeOps* ops);
+bool decode_ops_x_d128(int bits, int gs, int nc, bool f32, DecodeOps* ops);
+bool decode_ops_x_d256(int bits, int gs, int nc, bool f32, DecodeOps* ops);
 
 }  // namespace qkv

@@ -108,9 +108,16 @@ __device__ __forceinline__ int swz_offset(int lin) {
   return (lin & ~0x7f) | ((((lin >> 4) & 7) ^ f) << 4) | (lin & 15);
 }
 
-template <int D, int BITS, int GS, bool Q8, int NC>
+// SB: the width of the codes as stored in the cache.  BITS (4 or 8) is the
+// width the fragment code computes with; SB != BITS (affine 2, 3, 5 or 6-bit
+// codes, computed as 8-bit) stages each block's packed rows as they are (one
+// little-endian bit stream per row; rows straddle 16-byte units) and the team
+// transcodes them into an 8-bit tile of its own before the block's math.
+template <int D, int BITS, int GS, bool Q8, int NC, int SB = BITS>
 struct DecCfg {
-  static constexpr int RB = D * BITS / 8;      // bytes per code row
+  static constexpr bool XC = SB != BITS;       // transcoded from SB-bit codes
+  static constexpr int RB = D * BITS / 8;      // bytes per code row (compute width)
+  static constexpr int RBS = D * SB / 8;       // bytes per code row as stored
   static constexpr int UPR = RB / 16;          // 16-byte units per row
   static constexpr int NG = D / GS;            // groups per row
   static constexpr int GB = GS * BITS / 8;     // bytes per group per row
@@ -131,23 +138,32 @@ struct DecCfg {
   static constexpr int BUDGET = 227 * 1024 - 2048;
   static constexpr int r16(int x) { return (x + 15) / 16 * 16; }
   static constexpr int r128(int x) { return (x + 127) / 128 * 128; }
-  static constexpr int stage_bytes(int sub) { return r128(2 * 16 * sub * RB + NMETA * r16(16 * sub * MROW)); }
+  // staged codes of one tile (K or V): the compute tile, or the packed rows
+  static constexpr int scodes(int sub) { return XC ? r16(16 * sub * RBS) : 16 * sub * RB; }
+  static constexpr int stage_bytes(int sub) { return r128(2 * scodes(sub) + NMETA * r16(16 * sub * MROW)); }
+  // a team's 8-bit K and V tiles (transcoded blocks only)
+  static constexpr int xtile_bytes(int sub) { return XC ? 2 * 16 * sub * RB : 0; }
   // 16-key sub-blocks per block: two when three such stages per team fit
   // (D = 256 keeps one: its register budget is spent)
   // fused update: the new token's raw K and V rows (16-bit inputs)
   static constexpr int NEWB = 4 * D;
-  static constexpr int SUB = (D <= 128 && NTEAM * 3 * stage_bytes(2) + QSB + NEWB <= BUDGET) ? 2 : 1;
+  static constexpr int SUB = (D <= 128 && NTEAM * (3 * stage_bytes(2) + xtile_bytes(2)) + QSB + NEWB <= BUDGET) ? 2 : 1;
   static constexpr int BK = 16 * SUB;          // keys per block
   static constexpr int TK = BK;
-  static constexpr int CODES = BK * RB;
+  static constexpr int CODES = BK * RB;        // one compute tile
+  static constexpr int SCODES = scodes(SUB);   // one staged tile
+  static constexpr int MOFF = 2 * SCODES;      // metadata arrays in a stage
+  static constexpr int KUS = SCODES / 16;      // 16-byte units of a staged packed tile
+  static constexpr int XT = xtile_bytes(SUB);
   static constexpr int META = r16(BK * MROW);
   static constexpr int META_UNITS = BK * MROW / 16;
   static constexpr int KU = BK * UPR;          // 16-byte code units per tile
   static constexpr int MU = NMETA * META_UNITS;
   static constexpr int STAGE = stage_bytes(SUB);
-  static constexpr int NS_FIT = (BUDGET - QSB - NEWB) / (NTEAM * STAGE);
+  static constexpr int NS_FIT = (BUDGET - QSB - NEWB - NTEAM * XT) / (NTEAM * STAGE);
   static constexpr int NSTAGE = NS_FIT > 6 ? 6 : NS_FIT;
-  static constexpr int TRING = NSTAGE * STAGE;          // one team's ring
+  static constexpr int XTOFF = NSTAGE * STAGE;          // the team's 8-bit tiles after its ring
+  static constexpr int TRING = NSTAGE * STAGE + XT;     // one team's region
   static constexpr int QOFF = NTEAM * TRING;            // query rows after the rings
   // epilogue (after every ring is drained): per-warp partial rows, then the
   // per-(row, warp) combine weights and per-row (m, l)
@@ -156,7 +172,10 @@ struct DecCfg {
   static constexpr int EPI = EPI_W + NC * 8 * (NTEAM + 1) * 4 + NC * 8 * 2 * 4;
   static constexpr int NEWOFF = QOFF + QSB;
   static constexpr int SMEM = NEWOFF + NEWB > EPI ? NEWOFF + NEWB : EPI;
-  static_assert(NSTAGE >= 3, "at least three stages per team");
+  // three stages per team (two for transcoded blocks, whose 8-bit tiles take
+  // the room of the third: the copy of the next block still overlaps the
+  // math of the current one)
+  static_assert(NSTAGE >= (XC ? 2 : 3), "stages per team");
   static_assert(SMEM <= BUDGET, "shared memory budget");
   static_assert(META_UNITS * 16 == BK * MROW, "metadata rows must fill 16-byte units");
   static constexpr uint32_t SWZ = swizzle_coeffs(D, BITS, GS);   // key tile
@@ -303,13 +322,54 @@ __device__ __forceinline__ void dec_mask_vals(const T* m, int nk, float (&mv)[SU
     }
 }
 
-template <int D, int BITS, int GS, bool Q8, int NC, bool F32OUT, int VAR>
+// A team's transcode of one staged block of SB-bit codes (K rows, then V
+// rows SCODES bytes later; each row one little-endian bit stream, element e
+// at bits [e SB, (e + 1) SB)) into its 8-bit K and V tiles at xt, laid out and
+// swizzled exactly as staged 8-bit codes are.  A thread takes 16-code units
+// (one 16-byte unit of the 8-bit tile): two 64-bit windows of the stream, each
+// giving 8 codes.  Reads stay inside the stage (the V rows and the metadata
+// follow the K rows; the metadata follow the V rows).
+template <class C, int D, int SB>
+__device__ __forceinline__ void transcode_block(const uint8_t* raw, uint8_t* xt, int ttid) {
+  constexpr int UPR8 = C::RB / 16;                 // 16-code units per row
+  constexpr int ITEMS = 2 * C::BK * UPR8;
+  constexpr uint32_t MASK = (1u << SB) - 1u;
+  const uint32_t* rw = reinterpret_cast<const uint32_t*>(raw);
+#pragma unroll 2
+  for (int it = ttid; it < ITEMS; it += C::TTHR) {
+    const int which = it >= C::BK * UPR8;
+    const int rem = which ? it - C::BK * UPR8 : it;
+    const int r = rem / UPR8, j = rem - r * UPR8;
+    const uint32_t* base = rw + which * (C::SCODES / 4);
+    const int p0 = (r * D + 16 * j) * SB;           // bit position of the unit's first code
+    uint32_t out[4];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int ph = p0 + 8 * h * SB, wi = ph >> 5, sh = ph & 31;
+      const uint32_t w0 = base[wi], w1 = base[wi + 1], w2 = base[wi + 2];
+      const uint64_t v = ((uint64_t)__funnelshift_r(w1, w2, sh) << 32) | __funnelshift_r(w0, w1, sh);
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        uint32_t o = 0u;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o |= ((uint32_t)(v >> ((4 * k + e) * SB)) & MASK) << (8 * e);
+        out[2 * h + k] = o;
+      }
+    }
+    const int lin = r * C::RB + 16 * j;
+    *reinterpret_cast<uint4*>(xt + (which ? C::CODES + swz_xor<C::SWZV>(lin) : swz_xor<C::SWZ>(lin))) =
+        make_uint4(out[0], out[1], out[2], out[3]);
+  }
+}
+
+template <int D, int BITS, int GS, bool Q8, int NC, bool F32OUT, int VAR, int SB = BITS>
 __global__ void __launch_bounds__(32 * dec_warps(D), 1)
 qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
   constexpr bool FUSED = VAR == kDecFused;     // also quantizes the new token into row L - 1
   constexpr bool EXT = VAR == kDecExt;         // logit softcap, mask slopes, sinks
   constexpr bool ADDMASK = VAR != kDecPlain;   // additive masks (plain: none, or causal)
-  using C = DecCfg<D, BITS, GS, Q8, NC>;
+  using C = DecCfg<D, BITS, GS, Q8, NC, SB>;
+  static_assert(!C::XC || (BITS == 8 && !Q8 && VAR == kDecPlain), "stored widths compute as 8-bit");
   constexpr int NG = C::NG, KPG = C::KPG, MT = C::MT, BK = C::BK, NSTAGE = C::NSTAGE;
   constexpr int NTEAM = C::NTEAM, TTHR = C::TTHR;
   constexpr int HPC = NC * 8;
@@ -396,7 +456,25 @@ qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
       const int64_t grow = row0 + key0;                        // cache row of the block's first key
       const uint8_t* kb0 = p.kc + grow * C::RB;
       const uint8_t* vb0 = p.vc + grow * C::RB;
-      if (C::KU % TTHR == 0 && nvalid == BK) {
+      if constexpr (C::XC) {
+        // packed rows as they are, flat: a 16-byte unit that holds a byte of
+        // a valid row is copied whole (its tail lies below the next multiple
+        // of 8 rows, inside the cache); later units are zero-filled
+        const uint8_t* ks0 = p.kc + grow * C::RBS;
+        const uint8_t* vs0 = p.vc + grow * C::RBS;
+        const int vbytes = nvalid * C::RBS;
+        constexpr int NU = (2 * C::KUS + TTHR - 1) / TTHR;
+#pragma unroll
+        for (int k = 0; k < NU; ++k) {
+          const int i = ttid + k * TTHR;
+          if ((2 * C::KUS) % TTHR == 0 || i < 2 * C::KUS) {
+            const int which = i >= C::KUS, j = which ? i - C::KUS : i;
+            const bool ok = j * 16 < vbytes;
+            cp_async16(sbase + which * C::SCODES + j * 16, (which ? vs0 : ks0) + (ok ? j * 16 : 0),
+                       ok ? 16 : 0);
+          }
+        }
+      } else if (C::KU % TTHR == 0 && nvalid == BK) {
         const uint8_t* ks = kb0 + ttid * 16;
         const uint8_t* vs = vb0 + ttid * 16;
         const uint32_t dk = sbase + ((ttid * 16) ^ fx);
@@ -438,7 +516,7 @@ qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
         if (C::MU == TTHR || ttid < C::MU) {
           const int marr = ttid / C::META_UNITS, mj16 = (ttid - marr * C::META_UNITS) * 16;
           const bool ok = mj16 / C::MROW < nvalid;
-          cp_async16(sbase + 2 * C::CODES + marr * C::META + mj16,
+          cp_async16(sbase + C::MOFF + marr * C::META + mj16,
                      mlane + grow * C::MROW - (ok ? 0 : mj16), ok ? 16 : 0);
         }
         return;
@@ -452,7 +530,7 @@ qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
                                   : (arr == 0 ? p.ks : arr == 1 ? p.kb : arr == 2 ? p.vs : p.vb);
           const bool ok = (j * 16) / C::MROW < nvalid;
           const uint8_t* src = reinterpret_cast<const uint8_t*>(gm + grow * NG) + (ok ? j * 16 : 0);
-          cp_async16(sbase + 2 * C::CODES + arr * C::META + j * 16, src, ok ? 16 : 0);
+          cp_async16(sbase + C::MOFF + arr * C::META + j * 16, src, ok ? 16 : 0);
         }
       }
     };
@@ -630,7 +708,16 @@ qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
       }
       const uint8_t* sK = sb;
       const uint8_t* sV = sb + C::CODES;
-      const uint8_t* sMeta = sb + 2 * C::CODES;
+      const uint8_t* sMeta = sb + C::MOFF;
+      if constexpr (C::XC) {
+        // the team's warps are past the previous block (team_sync above), so
+        // its 8-bit tiles are free
+        uint8_t* xt = ring + C::XTOFF;
+        transcode_block<C, D, SB>(sb, xt, ttid);
+        team_sync();
+        sK = xt;
+        sV = xt + C::CODES;
+      }
 
       // ---------------- scores S[block][key][row] (base-2 logits) -------------
       float Sv[C::SUB][4];

@@ -36,6 +36,14 @@ int sm_count() {
 
 bool get_ops(int D, int bits, int gs, int fmt, int nc, bool f32, int var, DecodeOps* ops) {
   const bool q8 = fmt == QKV_Q8_0;
+  if (!q8 && bits != 4 && bits != 8) {
+    // codes stored 2, 3, 5 or 6 bits wide: the plain kernel only
+    if (var != kDecPlain) return false;
+    if (D == 64) return decode_ops_x_d64(bits, gs, nc, f32, ops);
+    if (D == 128) return decode_ops_x_d128(bits, gs, nc, f32, ops);
+    if (D == 256) return decode_ops_x_d256(bits, gs, nc, f32, ops);
+    return false;
+  }
   if (D == 64) return decode_ops_d64(bits, gs, q8, nc, f32, var, ops);
   if (D == 128) return decode_ops_d128(bits, gs, q8, nc, f32, var, ops);
   if (D == 256) return decode_ops_d256(bits, gs, q8, nc, f32, var, ops);

@@ -1,0 +1,9 @@
+// decode_x_d256.cu -- decode kernel instances for head dimension 256 with affine
+// codes stored 2, 3, 5 or 6 bits wide (transcoded to 8-bit per block).
+#include "decode_dispatch.cuh"
+
+namespace qkv {
+bool decode_ops_x_d256(int bits, int gs, int nc, bool f32, DecodeOps* ops) {
+  return decode_ops_x_for<256>(bits, gs, nc, f32, ops);
+}
+}  // namespace qkv

@@ -39,11 +39,21 @@ __global__ void __launch_bounds__(256) qkv_dequantize_kernel(const __grid_consta
   const double s = (double)half_bits_to_float(p.scales[crow * ng + g]);
   const double b = Q8 ? 0.0 : (double)half_bits_to_float(p.biases[crow * ng + g]);
   uint32_t w[2];
+  uint64_t stream = 0;                              // 2, 3, 5, 6 bits: the chunk's 8 codes
   if constexpr (BITS == 4) {
     w[0] = p.codes[crow * (p.D / 8) + c8];
-  } else {
+  } else if constexpr (BITS == 8) {
     const uint2 v = reinterpret_cast<const uint2*>(p.codes + crow * (p.D / 4))[c8];
     w[0] = v.x; w[1] = v.y;
+  } else {
+    // one little-endian bit stream per row: the chunk's 8 BITS bits from its
+    // (at most three) words, none past the row
+    const uint32_t* row = p.codes + crow * (p.D * BITS / 32);
+    const int pos = c8 * 8 * BITS, wi = pos >> 5, sh = pos & 31;
+    const uint32_t w0 = row[wi];
+    const uint32_t w1 = sh + 8 * BITS > 32 ? row[wi + 1] : 0u;
+    const uint32_t w2 = sh + 8 * BITS > 64 ? row[wi + 2] : 0u;
+    stream = ((uint64_t)__funnelshift_r(w1, w2, sh) << 32) | __funnelshift_r(w0, w1, sh);
   }
   uint32_t o[4];
 #pragma unroll
@@ -54,7 +64,8 @@ __global__ void __launch_bounds__(256) qkv_dequantize_kernel(const __grid_consta
       int code;
       if constexpr (BITS == 4) code = (int)((w[0] >> (4 * (e + k))) & 0xfu);
       else if constexpr (Q8) code = (int)(int8_t)((w[(e + k) >> 2] >> (8 * ((e + k) & 3))) & 0xffu);
-      else code = (int)((w[(e + k) >> 2] >> (8 * ((e + k) & 3))) & 0xffu);
+      else if constexpr (BITS == 8) code = (int)((w[(e + k) >> 2] >> (8 * ((e + k) & 3))) & 0xffu);
+      else code = (int)((stream >> (BITS * (e + k))) & ((1u << BITS) - 1u));
       x[k] = s * (double)code + b;
     }
     const uint32_t lo = __half_as_ushort(__double2half(x[0]));
@@ -90,6 +101,18 @@ cudaError_t launch_dequantize(const qkv_cache* c, int B, int Hkv, int D, int64_t
   else if (bits == 8 && gs == 32) QKV_DQ(8, 32, false);
   else if (bits == 8 && gs == 64) QKV_DQ(8, 64, false);
   else if (bits == 8 && gs == 128) QKV_DQ(8, 128, false);
+  else if (bits == 2 && gs == 32) QKV_DQ(2, 32, false);
+  else if (bits == 2 && gs == 64) QKV_DQ(2, 64, false);
+  else if (bits == 2 && gs == 128) QKV_DQ(2, 128, false);
+  else if (bits == 3 && gs == 32) QKV_DQ(3, 32, false);
+  else if (bits == 3 && gs == 64) QKV_DQ(3, 64, false);
+  else if (bits == 3 && gs == 128) QKV_DQ(3, 128, false);
+  else if (bits == 5 && gs == 32) QKV_DQ(5, 32, false);
+  else if (bits == 5 && gs == 64) QKV_DQ(5, 64, false);
+  else if (bits == 5 && gs == 128) QKV_DQ(5, 128, false);
+  else if (bits == 6 && gs == 32) QKV_DQ(6, 32, false);
+  else if (bits == 6 && gs == 64) QKV_DQ(6, 64, false);
+  else if (bits == 6 && gs == 128) QKV_DQ(6, 128, false);
   else return cudaErrorInvalidValue;
 #undef QKV_DQ
   return cudaGetLastError();

@@ -63,10 +63,20 @@ __global__ void __launch_bounds__(256, 6) qkv_quantize_kernel(const __grid_const
   uint16_t sbits, bbits;
   quantize_slice<GS, BITS, Q8, BF16>(w, o, sbits, bbits);
   if (active) {
-    uint4* dst = reinterpret_cast<uint4*>(s.codes + crow * (p.D * BITS / 32) + cs * (kQEpt * BITS / 32));
+    // the thread's BITS words: 16-byte stores for 4 and 8 bits, 8-byte ones
+    // for 2 and 6 (their offsets are 8-byte aligned), words for 3 and 5
+    uint32_t* dw = s.codes + crow * (p.D * BITS / 32) + cs * (kQEpt * BITS / 32);
+    if constexpr (BITS % 4 == 0) {
 #pragma unroll
-    for (int k = 0; k < kQEpt * BITS / 128; ++k)
-      dst[k] = make_uint4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
+      for (int k = 0; k < BITS / 4; ++k)
+        reinterpret_cast<uint4*>(dw)[k] = make_uint4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
+    } else if constexpr (BITS % 2 == 0) {
+#pragma unroll
+      for (int k = 0; k < BITS / 2; ++k) reinterpret_cast<uint2*>(dw)[k] = make_uint2(o[2 * k], o[2 * k + 1]);
+    } else {
+#pragma unroll
+      for (int k = 0; k < BITS; ++k) dw[k] = o[k];
+    }
     if (leader) {
       s.scales[crow * ng + grp] = sbits;
       if constexpr (!Q8) s.biases[crow * ng + grp] = bbits;
@@ -89,6 +99,18 @@ cudaError_t launch_q(int fmt, int bits, int gs, const QuantParams& p, int side0,
   else if (bits == 8 && gs == 32) QKV_QLAUNCH(32, 8, false);
   else if (bits == 8 && gs == 64) QKV_QLAUNCH(64, 8, false);
   else if (bits == 8 && gs == 128) QKV_QLAUNCH(128, 8, false);
+  else if (bits == 2 && gs == 32) QKV_QLAUNCH(32, 2, false);
+  else if (bits == 2 && gs == 64) QKV_QLAUNCH(64, 2, false);
+  else if (bits == 2 && gs == 128) QKV_QLAUNCH(128, 2, false);
+  else if (bits == 3 && gs == 32) QKV_QLAUNCH(32, 3, false);
+  else if (bits == 3 && gs == 64) QKV_QLAUNCH(64, 3, false);
+  else if (bits == 3 && gs == 128) QKV_QLAUNCH(128, 3, false);
+  else if (bits == 5 && gs == 32) QKV_QLAUNCH(32, 5, false);
+  else if (bits == 5 && gs == 64) QKV_QLAUNCH(64, 5, false);
+  else if (bits == 5 && gs == 128) QKV_QLAUNCH(128, 5, false);
+  else if (bits == 6 && gs == 32) QKV_QLAUNCH(32, 6, false);
+  else if (bits == 6 && gs == 64) QKV_QLAUNCH(64, 6, false);
+  else if (bits == 6 && gs == 128) QKV_QLAUNCH(128, 6, false);
   else return cudaErrorInvalidValue;
 #undef QKV_QLAUNCH
   return cudaGetLastError();

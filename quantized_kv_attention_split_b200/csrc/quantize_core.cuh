@@ -93,7 +93,11 @@ __device__ __forceinline__ float group_min(float v) {
 // of packed 16-bit inputs, zeros for a thread without a row): the GS/32
 // threads of a group (adjacent lanes; every lane of the warp takes part in
 // the shuffles) agree on the group's fp16 scale (and bias), and the thread's
-// codes come out packed, low bits first, in kQEpt * BITS / 32 words.
+// codes come out packed, low bits first, in kQEpt * BITS / 32 = BITS words.
+// For widths that do not divide 32 (3, 5, 6 bits) the row is one
+// little-endian bit stream, element i at bits [i BITS, (i + 1) BITS), so a
+// code may straddle two words; 32 codes fill exactly BITS words, so every
+// code stays inside its thread's words.
 template <int GS, int BITS, bool Q8, bool BF16>
 __device__ __forceinline__ void quantize_slice(const uint32_t (&w)[kQWords], uint32_t* o,
                                                uint16_t& sbits, uint16_t& bbits) {
@@ -140,6 +144,7 @@ __device__ __forceinline__ void quantize_slice(const uint32_t (&w)[kQWords], uin
   // a second pass with the correctly rounded division in the rare case that
   // flags it.  Q8_0 with a zero scale gives zero codes.
   constexpr int CPW = 32 / BITS;                    // codes per output word
+  constexpr bool STREAM = !Q8 && (32 % BITS) != 0;  // codes straddle words
   auto emit = [&](int i, int c, bool clamp) {       // code of element i
     if (clamp) c = min(max(c, QLO), QHI);
     if constexpr (Q8) {
@@ -147,12 +152,24 @@ __device__ __forceinline__ void quantize_slice(const uint32_t (&w)[kQWords], uin
       c = sf == 0.f ? 0 : c;
       const uint32_t sel = (i % 4) == 0 ? 0x3210u : (i % 4) == 1 ? 0x3240u : (i % 4) == 2 ? 0x3410u : 0x4210u;
       o[i / 4] = (i % 4) == 0 ? (uint32_t)c & 0xffu : __byte_perm(o[i / 4], (uint32_t)c, sel);
+    } else if constexpr (STREAM) {
+      // codes in [0, levels] at bit i * BITS of the stream (words zeroed first)
+      const int pos = i * BITS, wd = pos / 32, sh = pos % 32;
+      o[wd] |= (uint32_t)c << sh;
+      if (sh + BITS > 32) o[wd + 1] |= (uint32_t)c >> (32 - sh);
     } else {
       // codes in [0, levels]: place them by multiplication, no masking
       const uint32_t u = (uint32_t)c * (1u << ((i % CPW) * BITS));
       o[i / CPW] = (i % CPW) == 0 ? u : o[i / CPW] + u;
     }
   };
+  auto clear = [&]() {
+    if constexpr (STREAM) {
+#pragma unroll
+      for (int k = 0; k < BITS; ++k) o[k] = 0u;
+    }
+  };
+  clear();
   bool exact = false;
   if (__all_sync(~0u, inside)) {
 #pragma unroll
@@ -170,6 +187,7 @@ __device__ __forceinline__ void quantize_slice(const uint32_t (&w)[kQWords], uin
     }
   }
   if (exact) {
+    clear();
 #pragma unroll
     for (int i = 0; i < kQWords; ++i) {
       const float2 f = to_f2<BF16>(w[i]);

@@ -146,7 +146,7 @@ def test_decode_rejects_bad_arguments(qkv):
                                                                     device="cuda"))
     with pytest.raises(qkv.QKVError, match="L="):
         qkv.qsdpa_decode(qd, kd, vd, 10 ** 6, 1.0)
-    bad = qkv.QuantCache(kd.fmt, 5, kd.group_size, kd.codes, kd.scales, kd.biases)
+    bad = qkv.QuantCache(kd.fmt, 7, kd.group_size, kd.codes, kd.scales, kd.biases)
     with pytest.raises(qkv.QKVError, match="bits"):
         qkv.qsdpa_decode(qd, bad, vd, 64, 1.0)
 

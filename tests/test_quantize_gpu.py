@@ -1,6 +1,8 @@
 """GPU quantize-and-append (qkv_quantize_update) must match the oracle's
 quantizer bit for bit: codes, fp16 scales and fp16 biases, written only to
-rows [offset, offset+Lnew) of each (batch, kv-head)."""
+rows [offset, offset+Lnew) of each (batch, kv-head).  Affine codes of 2, 3, 4,
+5, 6 and 8 bits (3, 5 and 6-bit codes straddle 32-bit words of the row's bit
+stream) and Q8_0."""
 import numpy as np
 import pytest
 import torch
@@ -66,6 +68,10 @@ CASES = [
     ("affine", 4, 64, 128, "f16"), ("affine", 4, 32, 64, "f16"), ("affine", 4, 128, 256, "bf16"),
     ("affine", 8, 64, 128, "bf16"), ("affine", 8, 32, 256, "f16"), ("affine", 8, 128, 128, "f16"),
     ("q8_0", 8, 32, 256, "f16"), ("q8_0", 8, 32, 64, "bf16"),
+    # codes that straddle 32-bit words (3, 5, 6 bits) and 2-bit codes
+    ("affine", 2, 64, 128, "f16"), ("affine", 2, 32, 256, "bf16"), ("affine", 3, 32, 64, "bf16"),
+    ("affine", 3, 128, 256, "f16"), ("affine", 5, 64, 128, "bf16"), ("affine", 5, 32, 64, "f16"),
+    ("affine", 6, 32, 128, "f16"), ("affine", 6, 128, 256, "bf16"),
 ]
 
 
