@@ -419,17 +419,12 @@ def run_ours(args, rank, world, device):
             "vs_baseline": None,
             "dtype": "f16",
             "data": "synthetic (seeded SplitMix64, uniform fp16 q/k/v, K/V quantized on the GPU)",
-            "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
-                       "L": w.L, "Lq": w.Lq, "format": w.fmt, "bits": w.bits,
-                       "group_size": w.gs, "scale": w.scale, "out_dtype": "f16",
-                       "algorithmic_bytes_per_call": alg_bytes,
-                       "l2": f"inputs larger than L2: {ncopies} rotating cache copies "
-                             f"({ncopies * cache_bytes / 1e6:.0f} MB)",
-                       "timing": "CUDA events around CUDA-graph replays of exactly K back-to-back "
-                                 "calls (a call may start while the previous one finishes: its "
-                                 "set-up and L2 prefetch overlap that call's tail); "
-                                 "us_per_call_isolated: median of single calls after an L2 flush",
-                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+            "config": workload_config(w, world),
+            "l2": f"inputs larger than L2: {ncopies} rotating cache copies "
+                  f"({ncopies * cache_bytes / 1e6:.0f} MB)",
+            "timing": "CUDA events around CUDA-graph replays of exactly K back-to-back calls "
+                      "(a call's set-up overlaps the previous kernel's tail); "
+                      "us_per_call_isolated: median of single calls after an L2 flush",
             "roofline": {"bound": "hbm", "achieved": round(gbs, 2), "peak": hbm_peak,
                          "unit": "GB/s", "frac": round(gbs / hbm_peak, 4),
                          "peak_source": f"{peak_kind} hbm_gbs",
@@ -457,6 +452,15 @@ def run_ours(args, rank, world, device):
             result["rows"] = other_rows(device)
     del caches
     return result
+
+
+def workload_config(w, world):
+    """The `config` object of both arms: the workload and its sizes."""
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "L": w.L,
+            "Lq": w.Lq, "format": w.fmt, "bits": w.bits, "group_size": w.gs, "scale": w.scale,
+            "out_dtype": w.out_dtype,
+            "algorithmic_bytes_per_call": w.cache_bytes() + 2 * w.B * w.Hq * w.Lq * w.D * 2,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
 
 
 def read_traffic(workload):
@@ -680,6 +684,41 @@ def other_rows(device):
         rows["llama_q4_0_blocks_64k"] = {"unavailable": f"{type(e).__name__}: {e}"[:200]}
     torch.cuda.empty_cache()
 
+    # affine codes stored 2, 3, 5 and 6 bits wide: decode of the main shape
+    # (L = 65536, 32 query heads over 8 KV heads, D = 128, groups of 64)
+    try:
+        w = S.WORKLOADS["decode_64k_affine4"]
+        inp = S.make_inputs(w)
+        kx, vx = dev16(inp.k, "f16", device), dev16(inp.v, "f16", device)
+        q = dev16(inp.q, "f16", device)
+        out = torch.empty(w.B, w.Hq, 1, w.D, dtype=torch.float16, device=device)
+        ws = qkv.make_workspace(w.B, w.Hq, w.Hkv, 1, w.D, w.L, device)
+        for bits in (2, 3, 5, 6):
+            per_cache = w.B * w.Hkv * w.L * (w.D * bits // 8 + 2 * 2 * (w.D // w.gs))
+            ncopies = max(3, math.ceil(3 * 126e6 / (2 * per_cache)))
+            caches = []
+            for _ in range(ncopies):
+                kc = qkv.QuantCache.empty(w.B, w.Hkv, w.L, w.D, qkv.AFFINE, bits, w.gs, device)
+                vc = qkv.QuantCache.empty(w.B, w.Hkv, w.L, w.D, qkv.AFFINE, bits, w.gs, device)
+                qkv.qkv_quantize_update(kx, vx, kc, vc, 0)
+                caches.append((kc, vc))
+
+            def xstep(i):
+                a, b = caches[i % ncopies]
+                qkv.qsdpa_decode(q, a, b, w.L, w.scale, out=out, workspace=ws)
+            sec, _ = graph_time(xstep, 400, 20)
+            nb = 2 * per_cache + 2 * w.Hq * w.D * 2
+            rows[f"decode_64k_affine{bits}"] = {
+                "us_per_call": round(sec * 1e3, 3), "GB/s": round(nb / (sec / 1e3) / 1e9, 1),
+                "frac_hbm": round(nb / (sec / 1e3) / 1e9 / hbm_peak, 4), "bytes": nb,
+                "note": f"{bits}-bit codes (one bit stream per row), transcoded to 8-bit per "
+                        f"block by the decode kernel; caches written by qkv_quantize_update"}
+            del caches
+        del kx, vx
+    except Exception as e:
+        rows["decode_64k_affine3"] = {"unavailable": f"{type(e).__name__}: {e}"[:200]}
+    torch.cuda.empty_cache()
+
     # llama.cpp's reference Q4_0 / Q5_1 quantizers on the GPU: 65536 tokens of
     # K and V (the main decode shape) into token-major blocks, and one new
     # token of every head written straight into the affine caches
@@ -807,8 +846,7 @@ def run_reference(args, rank, world):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "L": w.L,
-                   "format": w.fmt, "bits": w.bits, "group_size": w.gs},
+        "config": workload_config(w, world),
         "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": threads,
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,

@@ -59,3 +59,15 @@ def test_traffic_is_read_only_for_the_profiled_source(tmp_path, monkeypatch):
     kern.write_text(kern.read_text() + "\n// changed\n")
     assert bench.read_traffic("decode_64k_affine4") is None
     assert bench.read_traffic("no_such_workload") is None
+
+
+def test_reference_arm_reports_the_gpu_arms_config():
+    """Both arms print the same `config` object (workload_config) for the
+    same workload, so their lines compare the same thing."""
+    import types
+    import bench
+    from quantized_kv_attention_split_b200 import synthetic as S
+    args = types.SimpleNamespace(workload="tiny_decode", steps=1, warmup=3, ref_seconds=1.0)
+    line = bench.run_reference(args, 0, 1)
+    assert line["config"] == bench.workload_config(S.WORKLOADS["tiny_decode"], 1)
+    assert line["impl"] == "reference" and line["config"]["workload"] == "tiny_decode"
