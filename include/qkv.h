@@ -294,6 +294,28 @@ qkv_status qkv_llama_cache_to_blocks(int kind, const qkv_cache* src, int B, int 
                                      int64_t offset, int64_t L, void* blocks, int64_t stride_b,
                                      int64_t stride_h, int64_t stride_l, void* stream);
 
+/* Attention whose values are a view of the keys (the "576/512 MLA" shape of
+ * the llama.cpp PR's follow-up tests: K rows of Dk = 576 elements, V = the
+ * first Dv = 512 elements of every K row, so the cache holds K only and one
+ * stream serves both):
+ *   out[b,h,i,:] = softmax_j(q[b,h,i]*scale . Khat[b,h/G,j] (+ causal)) . Khat[b,h/G,j,:512]
+ *  q:   [B, Hq, Lq, 576] contiguous, f16 or bf16.
+ *  out: [B, Hq, Lq, 512] contiguous, f16 or bf16 (fp32 output is refused:
+ *       the kernel dequantizes to fp16 tiles, max-abs error <= 2e-3 for
+ *       values of order one).
+ *  k:   Q8_0, or affine 4- or 8-bit codes in groups of 32 or 64; rows of 576.
+ *  mask: NULL, none or causal (bottom-right); no additive mask.
+ *  workspace: at least qsdpa_kview_workspace_size(...) bytes, 16-byte aligned
+ *  (partial results of the split over L; no state between calls).  One
+ *  launch, or two when the keys of a (batch, kv head, 16-row tile) are split
+ *  over several CTAs (the second is the decode's merge kernel).  Any Lq >= 1
+ *  (decode and prefill).  L == 0 writes zeros. */
+qkv_status qsdpa_attention_kview(const void* q, int q_dtype, int B, int Hq, int Hkv, int Lq, int Dk,
+                                 int Dv, const qkv_cache* k, int64_t L, float scale,
+                                 const qkv_mask* mask, void* out, int out_dtype, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+size_t qsdpa_kview_workspace_size(int B, int Hq, int Hkv, int Lq, int Dk, int Dv, int64_t L);
+
 /* Allocation-free variant of qsdpa_decode (the pages have no counterpart:
  * MLX and llama.cpp allocate their temporaries through their own allocators).
  * For callers that cannot allocate device memory when they decode -- code

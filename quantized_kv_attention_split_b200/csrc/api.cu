@@ -470,6 +470,79 @@ qkv_status qsdpa_prefill(const void* q, int q_dtype, int B, int Hq, int Hkv, int
                    workspace_bytes, stream);
 }
 
+size_t qsdpa_kview_workspace_size(int B, int Hq, int Hkv, int Lq, int Dk, int Dv, int64_t L) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Lq <= 0 || Hq % Hkv || L < 0) return 0;
+  if (Dk != 576 || Dv != 512) return 0;
+  return qkv::kview_workspace_bytes();
+}
+
+qkv_status qsdpa_attention_kview(const void* q, int q_dtype, int B, int Hq, int Hkv, int Lq, int Dk,
+                                 int Dv, const qkv_cache* k, int64_t L, float scale,
+                                 const qkv_mask* mask, void* out, int out_dtype, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Lq <= 0)
+    return fail(QKV_ERR_INVALID_ARG, "B, Hq, Hkv and Lq must be positive");
+  if (Hq % Hkv != 0) return fail(QKV_ERR_INVALID_ARG, "Hq=%d is not a multiple of Hkv=%d", Hq, Hkv);
+  if (Dk != 576 || Dv != 512)
+    return fail(QKV_ERR_UNSUPPORTED, "values as a view of the keys: Dk=576, Dv=512 (got %d/%d)", Dk, Dv);
+  if (k == nullptr) return fail(QKV_ERR_INVALID_ARG, "k: cache descriptor is NULL");
+  if (k->fmt == QKV_Q8_0) {
+    if (k->bits != 8 || k->group_size != 32)
+      return fail(QKV_ERR_INVALID_ARG, "k: Q8_0 needs bits 8 and group_size 32");
+  } else if (k->fmt == QKV_AFFINE) {
+    if ((k->bits != 4 && k->bits != 8) || (k->group_size != 32 && k->group_size != 64))
+      return fail(QKV_ERR_UNSUPPORTED, "k: the view kernel takes affine 4- or 8-bit codes in groups "
+                  "of 32 or 64 (got %d bits, group %d)", k->bits, k->group_size);
+    if (k->biases == nullptr) return fail(QKV_ERR_INVALID_ARG, "k: affine cache needs biases");
+  } else {
+    return fail(QKV_ERR_INVALID_ARG, "k: unknown format %d", k->fmt);
+  }
+  if (k->codes == nullptr || k->scales == nullptr)
+    return fail(QKV_ERR_INVALID_ARG, "k: codes and scales must be non-NULL");
+  if (k->Lcap <= 0 || k->Lcap % 8 != 0)
+    return fail(k->Lcap <= 0 ? QKV_ERR_INVALID_ARG : QKV_ERR_ALIGNMENT,
+                "k: Lcap must be a positive multiple of 8 (got %lld)", (long long)k->Lcap);
+  if (!aligned16(k->codes) || !aligned16(k->scales) || (k->fmt == QKV_AFFINE && !aligned16(k->biases)))
+    return fail(QKV_ERR_ALIGNMENT, "k: codes, scales and biases must be 16-byte aligned");
+  if (L < 0 || L > k->Lcap) return fail(QKV_ERR_INVALID_ARG, "L=%lld outside [0, Lcap]", (long long)L);
+  qkv_status st;
+  if ((st = check_dtype("q", q_dtype, false)) != QKV_OK) return st;
+  if (out_dtype != QKV_F16 && out_dtype != QKV_BF16)
+    return fail(out_dtype == QKV_F32 ? QKV_ERR_UNSUPPORTED : QKV_ERR_INVALID_ARG,
+                "out: f16 or bf16 (the view kernel's tiles are fp16: no fp32-accurate output)");
+  if (q == nullptr || out == nullptr) return fail(QKV_ERR_INVALID_ARG, "q and out must be non-NULL");
+  if (!aligned16(q) || !aligned16(out)) return fail(QKV_ERR_ALIGNMENT, "q and out must be 16-byte aligned");
+  if (!(scale == scale)) return fail(QKV_ERR_INVALID_ARG, "scale is NaN");
+  int mkind = mask == nullptr ? QKV_MASK_NONE : mask->kind;
+  if (mkind == QKV_MASK_ADDITIVE)
+    return fail(QKV_ERR_UNSUPPORTED, "the view kernel takes no additive mask (none or causal)");
+  if (mkind != QKV_MASK_NONE && mkind != QKV_MASK_CAUSAL)
+    return fail(QKV_ERR_INVALID_ARG, "unknown mask kind %d", mkind);
+  if ((int64_t)Hq * Lq > (int64_t)1 << 30) return fail(QKV_ERR_INVALID_ARG, "Hq * Lq too large");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (L == 0) {
+    if (cudaMemsetAsync(out, 0, (size_t)B * Hq * Lq * Dv * 2, s) != cudaSuccess)
+      return fail(QKV_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(cudaGetLastError()));
+    return ok();
+  }
+  const size_t need = qkv::kview_workspace_bytes();
+  if (workspace == nullptr || workspace_bytes < need)
+    return fail(QKV_ERR_WORKSPACE, "workspace of %zu bytes required (got %zu)", need, workspace_bytes);
+  if (!aligned16(workspace)) return fail(QKV_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
+  qkv::DecodeParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.q = q; p.q_dtype = q_dtype; p.out = out; p.out_dtype = out_dtype;
+  p.kc = reinterpret_cast<const uint8_t*>(k->codes); p.ks = k->scales; p.kb = k->biases;
+  p.Lcap = k->Lcap; p.L = L;
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Gq = Hq / Hkv; p.Lq = Lq; p.G = (Hq / Hkv) * Lq;
+  p.scale_log2e = scale * 1.4426950408889634f;
+  p.mask_kind = (mkind == QKV_MASK_CAUSAL && Lq > 1) ? QKV_MASK_CAUSAL : QKV_MASK_NONE;
+  p.part_o = static_cast<float*>(workspace);
+  cudaError_t e = qkv::launch_kview(k->bits, k->group_size, k->fmt, p, s);
+  if (e != cudaSuccess) return fail(QKV_ERR_CUDA, "view attention launch: %s", cudaGetErrorString(e));
+  return ok();
+}
+
 qkv_status qsdpa_decode_ext(const void* q, int q_dtype, int B, int Hq, int Hkv, int D,
                             const qkv_cache* k, const qkv_cache* v, int64_t L, float scale,
                             const qkv_mask* mask, const qkv_attn_ext* ext, void* out,

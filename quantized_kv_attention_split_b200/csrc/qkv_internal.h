@@ -93,6 +93,12 @@ cudaError_t launch_dequantize(const qkv_cache* c, int B, int Hkv, int D, int64_t
 cudaError_t launch_llama_blocks(int kind, const void* src_blocks, const qkv_cache* c, int B, int Hkv,
                                 int D, int64_t offset, int64_t L, int64_t sb, int64_t sh,
                                 int64_t sl, cudaStream_t stream);
+// Attention whose values are the first 512 elements of 576-element keys
+// (kview.cu): plans the split and launches (p: the decode parameters with the
+// key cache, G = rows per kv head, part_o = the workspace).
+cudaError_t launch_kview(int bits, int gs, int fmt, DecodeParams& p, cudaStream_t s);
+size_t kview_workspace_bytes();
+
 cudaError_t launch_llama_quantize(int kind, const void* x, int in_dtype, int B, int Hkv, int D,
                                   int64_t L, void* blocks, int64_t sb, int64_t sh, int64_t sl,
                                   const qkv_cache* c, int64_t offset, cudaStream_t stream);

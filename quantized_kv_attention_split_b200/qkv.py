@@ -97,6 +97,11 @@ def lib() -> C.CDLL:
         L.qkv_llama_cache_to_blocks.argtypes = [i32, cp, i32, i32, i32, i64, i64, p, i64, i64, i64,
                                                 p]
         L.qkv_llama_cache_to_blocks.restype = i32
+        L.qsdpa_attention_kview.argtypes = [p, i32, i32, i32, i32, i32, i32, i32, cp, i64,
+                                            C.c_float, mp, p, i32, p, sz, p]
+        L.qsdpa_attention_kview.restype = i32
+        L.qsdpa_kview_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32, i64]
+        L.qsdpa_kview_workspace_size.restype = sz
         L.qkv_dequantize.argtypes = [cp, i32, i32, i32, i64, p, p]
         L.qkv_dequantize.restype = i32
         L.qsdpa_workspace_size.argtypes = [i32, i32, i32, i32, i32, i64]
@@ -470,4 +475,29 @@ def qsdpa_decode_noalloc(q: torch.Tensor, k: QuantCache, v: QuantCache, L: int, 
         _check(f(q.data_ptr(), _DTYPE[q.dtype], B, Hq, Hkv, D, C.byref(ks), C.byref(vs), int(L),
                  float(scale), C.byref(m) if m is not None else None, out.data_ptr(),
                  _DTYPE[out.dtype], _stream(stream)))
+    return out
+
+
+def qsdpa_attention_kview(q: torch.Tensor, k: QuantCache, L: int, scale: float, Dv: int = 512,
+                          causal: bool = False, out: Optional[torch.Tensor] = None, out_dtype=None,
+                          workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """softmax(q*scale . K^T) V with V the first Dv elements of every key row
+    (K rows of 576, Dv 512): q [B,Hq,Lq,576] -> out [B,Hq,Lq,512]; the cache
+    holds K only.  ``causal`` aligns the Lq queries with the last Lq keys."""
+    assert q.is_contiguous() and q.is_cuda
+    B, Hq, Lq, Dk = q.shape
+    Hkv = k.codes.shape[1]
+    if out is None:
+        out = torch.empty(B, Hq, Lq, Dv, dtype=out_dtype or q.dtype, device=q.device)
+    with _on(q):
+        if workspace is None:
+            n = int(lib().qsdpa_kview_workspace_size(B, Hq, Hkv, Lq, Dk, Dv, int(L)))
+            workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=q.device)
+        ks = k._struct()
+        m = _mask_struct(None, causal)
+        _check(lib().qsdpa_attention_kview(q.data_ptr(), _DTYPE[q.dtype], B, Hq, Hkv, Lq, Dk, Dv,
+                                           C.byref(ks), int(L), float(scale),
+                                           C.byref(m) if m is not None else None, out.data_ptr(),
+                                           _DTYPE[out.dtype], workspace.data_ptr(),
+                                           workspace.numel(), _stream(stream)))
     return out

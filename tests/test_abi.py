@@ -246,3 +246,23 @@ def test_llama_quantize_and_export_validation_errors(lib):
     assert ex(1, C.byref(a8), 1, 2, 128, 0, 16, FAKE, *st, None) == 2        # Q4 from 8-bit
     assert ex(2, C.byref(a8), 1, 2, 128, 60, 16, FAKE, *st, None) == 1       # past Lcap
     assert ex(0, C.byref(a4), 1, 2, 128, 0, 16, FAKE + 1, *st, None) == 3    # odd address
+
+
+def test_kview_validation_errors(lib):
+    from quantized_kv_attention_split_b200 import qkv
+    q8 = _cache(qkv, fmt=1, bits=8, gs=32, biases=0)
+    f = lib.qsdpa_attention_kview
+
+    def call(k=q8, Dk=576, Dv=512, odt=0, L=16, ws=1 << 26, mask=None):
+        return f(FAKE, 0, 1, 16, 1, 1, Dk, Dv, C.byref(k), L, 0.1,
+                 C.byref(mask) if mask is not None else None, FAKE + 65536, odt, FAKE + 131072, ws,
+                 None)
+    assert call(Dk=512) == 2 and call(Dv=256) == 2                          # shapes other than 576/512
+    assert call(k=_cache(qkv, fmt=0, bits=4, gs=128)) == 2                  # group 128
+    assert call(k=_cache(qkv, fmt=0, bits=3, gs=32)) == 2                   # 3-bit codes
+    assert call(odt=2) == 2                                                 # fp32 out
+    assert call(L=65) == 1                                                  # L > Lcap
+    assert call(ws=16) == 4                                                 # workspace too small
+    assert call(mask=qkv._Mask(2, FAKE, 2, 0, 0, 0)) == 2                   # additive mask
+    assert lib.qsdpa_kview_workspace_size(1, 16, 1, 1, 576, 512, 100) > 0
+    assert lib.qsdpa_kview_workspace_size(1, 16, 1, 1, 128, 128, 100) == 0
