@@ -37,8 +37,14 @@
  *  - Lcap is the row capacity per (batch, kv-head); a call uses rows [0, L).
  *    Lcap must be a multiple of 8 and every pointer 16-byte aligned
  *    (QKV_ERR_ALIGNMENT otherwise).
- *  - Supported: affine bits 4 or 8 with group_size 32, 64 or 128; Q8_0
- *    (bits 8, group_size 32); D in {64, 128, 256} with D % group_size == 0.
+ *  - Supported: affine bits 2, 3, 4, 5, 6 or 8 with group_size 32, 64 or
+ *    128; Q8_0 (bits 8, group_size 32); D in {64, 128, 256} with
+ *    D % group_size == 0 (and D = 576 for qsdpa_attention_kview and the
+ *    quantizer).  Codes of 3, 5 and 6 bits straddle words (the rule above
+ *    read as one little-endian bit stream per row: element e at bits
+ *    [e*bits, (e+1)*bits)).  With 2, 3, 5 or 6-bit codes the attention
+ *    calls take no additive mask, no extensions and no fused update
+ *    (QKV_ERR_UNSUPPORTED), and multi-query calls run on the split-K kernel.
  */
 #ifndef QKV_H_
 #define QKV_H_
@@ -125,7 +131,8 @@ typedef struct {
  *           code = clamp(rint((x - bias)/scale), 0, 2^bits-1)
  *   Q8_0:   d = max|x|/127; scale = fp16_rne(d);
  *           code = scale == 0 ? 0 : clamp(rint(x/scale), -127, 127)
- *  The result is bit-identical to the CPU oracle.  Requires
+ *  The result is bit-identical to the CPU oracle.  D is 64, 128, 256 or 576
+ *  (the key rows of qsdpa_attention_kview).  Requires
  *  0 <= offset <= Lcap - Lnew and B*Hkv <= 65535 (QKV_ERR_UNSUPPORTED
  *  otherwise).  k and v may use different formats (then K and V are two
  *  launches, else one). */
@@ -181,7 +188,13 @@ qkv_status qsdpa_decode_update(const void* q, int q_dtype, const void* new_k, co
  * otherwise, and always for f32 output, on the split-K kernel.  The tcgen05
  * kernel bounds its waits on the tensor core: if one ever times out it sets
  * the first 32-bit word of the workspace nonzero (the output is then invalid);
- * that word must be zeroed again before the workspace is reused. */
+ * that word must be zeroed again before the workspace is reused.  Its fp16
+ * tiles hold scale * code + bias: a small kernel first checks every scale and
+ * bias of rows [0, L), and when some value can reach 2^15 the call runs a
+ * second instance of the tcgen05 kernel that scales each tile by a power of
+ * two and undoes it exactly (values up to the largest the fp16 scales and
+ * biases can express are computed correctly); words 1 and 2 of the workspace
+ * carry that decision and are zero again after the call. */
 qkv_status qsdpa_prefill(const void* q, int q_dtype, int B, int Hq, int Hkv, int Lq,
                          int D, const qkv_cache* k, const qkv_cache* v, int64_t L,
                          float scale, const qkv_mask* mask, void* out, int out_dtype,

@@ -45,8 +45,9 @@ qkv_status ok() {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Validates one cache description for head dimension D.
-qkv_status check_cache(const char* name, const qkv_cache* c, int D) {
+// Validates one cache description for head dimension D (kview: also the
+// 576-element key rows of the view attention, which the quantizer writes).
+qkv_status check_cache(const char* name, const qkv_cache* c, int D, bool kview = false) {
   if (c == nullptr) return fail(QKV_ERR_INVALID_ARG, "%s: cache descriptor is NULL", name);
   if (c->fmt != QKV_AFFINE && c->fmt != QKV_Q8_0)
     return fail(QKV_ERR_INVALID_ARG, "%s: unknown format %d", name, c->fmt);
@@ -62,8 +63,9 @@ qkv_status check_cache(const char* name, const qkv_cache* c, int D) {
     if (c->bits != 8 || c->group_size != 32)
       return fail(QKV_ERR_INVALID_ARG, "%s: Q8_0 needs bits 8 and group_size 32", name);
   }
-  if (D != 64 && D != 128 && D != 256)
-    return fail(QKV_ERR_UNSUPPORTED, "head dimension must be 64, 128 or 256 (got %d)", D);
+  if (D != 64 && D != 128 && D != 256 && !(kview && D == 576))
+    return fail(QKV_ERR_UNSUPPORTED, "head dimension must be 64, 128 or 256%s (got %d)",
+                kview ? " (or 576)" : "", D);
   if (D % c->group_size != 0)
     return fail(QKV_ERR_UNSUPPORTED, "%s: D=%d is not a multiple of group_size=%d", name, D,
                 c->group_size);
@@ -174,6 +176,7 @@ qkv_status attention(const void* q, int q_dtype, int B, int Hq, int Hkv, int Lq,
     }
     pp.cap_a = cap_a; pp.cap_k = cap_k; pp.slopes = slopes; pp.sinks = sinks;
     pp.status = static_cast<unsigned*>(workspace);
+    pp.range = static_cast<unsigned*>(workspace) + 1;   // words 1 and 2 of the zeroed header
     cudaError_t e = qkv::launch_prefill_tc(D, k->bits, k->group_size, k->fmt, pp, s);
     if (e != cudaSuccess) return fail(QKV_ERR_CUDA, "prefill launch: %s", cudaGetErrorString(e));
     return ok();
@@ -284,8 +287,8 @@ qkv_status qkv_quantize_update(const void* new_k, const void* new_v, int in_dtyp
                                int64_t offset, void* stream) {
   qkv_status st;
   if (B <= 0 || Hkv <= 0 || Lnew < 0) return fail(QKV_ERR_INVALID_ARG, "B, Hkv must be positive, Lnew >= 0");
-  if ((st = check_cache("k", k, D)) != QKV_OK) return st;
-  if ((st = check_cache("v", v, D)) != QKV_OK) return st;
+  if ((st = check_cache("k", k, D, true)) != QKV_OK) return st;
+  if ((st = check_cache("v", v, D, true)) != QKV_OK) return st;
   if (in_dtype != QKV_F16 && in_dtype != QKV_BF16)
     return fail(QKV_ERR_INVALID_ARG, "new tokens must be f16 or bf16 (got %d)", in_dtype);
   if ((int64_t)B * Hkv > 65535)

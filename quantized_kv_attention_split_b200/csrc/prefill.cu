@@ -1,15 +1,17 @@
 // prefill.cu -- host side of the tcgen05 multi-query kernel: instance table
 // and launch.
+#include <algorithm>
+
 #include "prefill_kernel.cuh"
 
 namespace qkv {
 
 namespace {
 
-template <int D, int BITS, int GS, bool Q8, bool EXT>
-cudaError_t launch_pf_v(const PrefillParams& p, int grid, cudaStream_t s) {
+template <int D, int BITS, int GS, bool Q8, bool EXT, bool RANGE>
+cudaError_t launch_pf_r(const PrefillParams& p, int grid, cudaStream_t s) {
   using C = PfCfg<D, BITS, GS, Q8>;
-  auto k = qsdpa_prefill_tc_kernel<D, BITS, GS, Q8, EXT>;
+  auto k = qsdpa_prefill_tc_kernel<D, BITS, GS, Q8, EXT, RANGE>;
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
@@ -18,6 +20,24 @@ cudaError_t launch_pf_v(const PrefillParams& p, int grid, cudaStream_t s) {
   }
   k<<<grid, kPfThreads, C::SMEM, s>>>(p);
   return cudaGetLastError();
+}
+
+// A call: the range check of the cache's scales and biases, then the kernel
+// and its range-scaled instance (one of the two runs, the other exits at
+// once).
+template <int D, int BITS, int GS, bool Q8, bool EXT>
+cudaError_t launch_pf_v(const PrefillParams& p, int grid, cudaStream_t s) {
+  const int ng = D / GS;
+  const int64_t units = (p.L * ng + 7) / 8;
+  const int64_t slabs = (int64_t)p.B * p.Hkv;
+  if (slabs > 65535) return cudaErrorInvalidValue;
+  const unsigned cx = (unsigned)std::min<int64_t>(std::max<int64_t>(1, (units + 255) / 256), 148);
+  qkv_range_check_kernel<Q8, BITS><<<dim3(cx, (unsigned)slabs), 256, 0, s>>>(p, ng);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  e = launch_pf_r<D, BITS, GS, Q8, EXT, false>(p, grid, s);
+  if (e != cudaSuccess) return e;
+  return launch_pf_r<D, BITS, GS, Q8, EXT, true>(p, grid, s);
 }
 
 // the extension instance only when an extension is in use

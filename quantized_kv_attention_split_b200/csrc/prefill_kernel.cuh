@@ -31,13 +31,18 @@
 //     the output.
 // Range: the fp16 tiles hold scale * code + bias, which leaves the fp16 range
 // for caches of large values (bf16 inputs, or fp16 ones near its maximum).
-// Once a tile's packed data has landed, the producer warp bounds the tile's
-// K and V magnitudes from its scales and biases and publishes two powers of
-// two: 2^eK for the tile's K (S of the tile is scaled back by 2^eK in the
-// softmax) and 2^eV for V, the largest needed so far (O in TMEM is rescaled
-// exactly when it grows, and scaled back by 2^eV at the end).  Both are 1
-// (exponent 0) unless a tile's values reach 2^15, so ordinary caches take the
-// unscaled path.
+// The magnitudes are bounded from the scales and biases (read straight from
+// global memory, off the
+// tiles' critical path).  A call launches a check of every scale and bias in
+// rows [0, L) (qkv_range_check_kernel, ~1 MB for the 512-query prompt at
+// depth 20K), which raises a flag in the workspace when some value can reach
+// 2^15, then two instances of this kernel.  The first (RANGE false) is the
+// kernel described above and runs when the flag is down.  The second (RANGE
+// true) runs when it is up: the producer publishes powers of two per tile,
+// 2^eK for the tile's K (S of the tile is scaled back by 2^eK in the softmax)
+// and 2^eV for V, the largest needed so far (O in TMEM is rescaled exactly
+// when it grows, and scaled back by 2^eV at the end); its last CTA lowers the
+// flag.  The instance that does not run exits at once.
 // Every mbarrier wait is bounded: a time-out records an error in the status
 // word and makes every later wait return at once, so all roles finish the
 // tile loop; before exit the CTA waits (bounded) for its own bulk copies and
@@ -87,6 +92,8 @@ struct PrefillParams {
   const float* slopes;      // per-head additive-mask slopes, fp32 [Hq] or null
   const float* sinks;       // per-head sink logits, fp32 [Hq] or null
   unsigned* status;         // nonzero after a tensor-core wait timed out
+  unsigned* range;          // [2]: a tile reaches 2^15 (set by the first instance),
+                            // CTAs of the second instance done (its last zeroes both)
 };
 
 // Lane -> chunk map of the dequant warps (a GF(2)-linear map given by the
@@ -194,7 +201,7 @@ __device__ __forceinline__ int pf_range_get(const volatile uint32_t* ring, int t
     const uint32_t v = ring[t & (kPfRangeRing - 1)];
     if ((v >> 10) == want) return (int)(v & 1023u);
     if (*abort_flag) return -1;
-    __nanosleep(32);
+    if (i >= 256) __nanosleep(64);             // normally published a tile ahead: rare
   }
   *abort_flag = 1;
   atomicOr(status, 256u);
@@ -461,8 +468,9 @@ __device__ __forceinline__ void pf_add_mask(float (&sv)[kPfBN], const T* m, int 
 }
 
 // EXT: the instance with the attention extensions (logit softcap, additive-mask
-// slopes, sinks); the plain instance carries none of their code.
-template <int D, int BITS, int GS, bool Q8, bool EXT>
+// slopes, sinks); the plain instance carries none of their code.  RANGE: the
+// second instance of a call (see the range note above).
+template <int D, int BITS, int GS, bool Q8, bool EXT, bool RANGE>
 __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const PrefillParams p) {
   using C = PfCfg<D, BITS, GS, Q8>;
   constexpr int NG = C::NG;
@@ -479,6 +487,25 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
   auto pv_done = [&](int i) { return bar0 + 96 + 8 * i; };    // [2] P V product done
   const uint32_t mma_done = bar0 + 112;                       // all tensor-core work done
   auto raw_free = [&](int i) { return bar0 + 120 + 8 * i; };  // [2] a tile's raw slots released
+  {
+    // the range flag was written by the range check kernel, two kernels
+    // earlier in the stream: the first instance runs when it is down, the
+    // second when it is up.  Every CTA of the second instance counts itself
+    // done at exit; the last one lowers the flag and the count for the next
+    // call.
+    __shared__ int s_run;
+    if (tid == 0) s_run = (*reinterpret_cast<volatile unsigned*>(p.range) != 0u) == RANGE;
+    __syncthreads();
+    const bool run = s_run != 0;
+    __syncthreads();
+    if (!run) {
+      if (RANGE && tid == 0 && atomicAdd(p.range + 1, 1u) + 1 == gridDim.x) {
+        p.range[1] = 0u;
+        p.range[0] = 0u;
+      }
+      return;
+    }
+  }
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::BAR_OFF + 144);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::BAR_OFF + 148);
   volatile uint32_t* range_ring = reinterpret_cast<volatile uint32_t*>(smem + C::BAR_OFF + 160);
@@ -660,9 +687,13 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
         const int64_t key0 = (int64_t)i * kPfRawKeys;
         nv[h] = !present ? 0 : (L - key0 < kPfRawKeys ? (int)(L - key0) : kPfRawKeys);
       }
-      // the tile's range exponents (0 and 0 unless its values reach 2^15)
-      const int rg = pf_range_get(range_ring, t, abort_flag, p.status);
-      const int eK = rg < 0 ? 0 : rg >> 5, eV = rg < 0 ? 0 : rg & 31;
+      // the tile's range exponents (second instance only)
+      int eK = 0, eV = 0;
+      if constexpr (RANGE) {
+        const int rg = pf_range_get(range_ring, t, abort_flag, p.status);
+        eK = rg < 0 ? 0 : rg >> 5;
+        eV = rg < 0 ? 0 : rg & 31;
+      }
       // K and V chunks of this thread come in together; V converts after K
       PfChunks<D, BITS, GS, Q8> kch, vch;
       kch.load(raw, 0, 2 * C::RAW_CODES, 2 * C::RAW_CODES + C::META_BYTES, nv, chunk0, eK);
@@ -682,28 +713,61 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
     }
   } else if (warp == kPfProdWarp) {
     // ======================= producer warp =====================================
-    // Tile t's range exponents are published before the warp waits for the
-    // tile's raw slots to be released (the dequant warps read them first).
+    if constexpr (!RANGE) {
+    for (int t = 0; t + 2 < ntiles || 2 * t + kPfRawSlots < nhalves; ++t) {
+      const int i0 = 2 * t + kPfRawSlots;
+      if (i0 >= nhalves) break;
+      mbar_wait(raw_free(t & 1), (t >> 1) & 1, abort_flag, p.status, 1u);
+      // warp-uniform decision (issue_raw synchronizes the warp)
+      if (__shfl_sync(~0u, (int)*abort_flag, 0) != 0) break;
+      issue_raw(i0, nhalves - i0 < 2 ? nhalves - i0 : 2);
+    }
+    } else {
+    // Range exponents: the warp reads tile t + 2's scales (and biases)
+    // straight from global memory while it waits to refill the raw slots of
+    // tile t, and publishes the tile's exponents after that refill -- a tile
+    // and more before the dequant warps need them -- then starts the reads
+    // for tile t + 3.  Tiles 0 and 1 are published before the loop.
     constexpr float kCodeMax = Q8 ? 128.f : (float)((1 << BITS) - 1);   // largest |code|
+    constexpr int U4 = kPfBN * NG * 2 / 16;      // 16-byte units of one metadata array of a tile
+    constexpr int PER = (U4 + 31) / 32;          // per lane
+    uint4 fm[C::NMETA][PER];                     // metadata of the tile in flight
     int eV = 0;                                  // largest V exponent so far
-    for (int t = 0; t < ntiles; ++t) {
+    auto fetch = [&](int t) {
+      const int64_t key0 = (int64_t)t * kPfBN;
+      const int nvt = L - key0 < kPfBN ? (int)(L - key0) : kPfBN;
+#pragma unroll
+      for (int a = 0; a < C::NMETA; ++a) {
+        // arrays in stage order: K scales, (K biases,) V scales, (V biases)
+        const uint16_t* m = Q8 ? (a == 0 ? p.ks : p.vs)
+                               : (a == 0 ? p.ks : a == 1 ? p.kb : a == 2 ? p.vs : p.vb);
+        const uint4* src = reinterpret_cast<const uint4*>(m + (row0 + key0) * NG);
+#pragma unroll
+        for (int k = 0; k < PER; ++k) {
+          const int i = lane + 32 * k;             // unit i holds keys from i * 8 / NG on
+          fm[a][k] = (i < U4 && i * 8 / NG < nvt) ? __ldg(src + i) : make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+    };
+    auto finish = [&](int t) {
+      const int64_t key0 = (int64_t)t * kPfBN;
+      const int nvt = L - key0 < kPfBN ? (int)(L - key0) : kPfBN;
       float bk = 0.f, bv = 0.f;                  // bounds of |scale * code + bias|
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int i = 2 * t + h;
-        if (i >= nhalves) break;
-        const int slot = i % kPfRawSlots;
-        mbar_wait(raw_full(slot), (i / kPfRawSlots) & 1, abort_flag, p.status, 1u);
-        const int64_t key0 = (int64_t)i * kPfRawKeys;
-        const int nv = L - key0 < kPfRawKeys ? (int)(L - key0) : kPfRawKeys;
-        const uint16_t* m = reinterpret_cast<const uint16_t*>(smem + C::RAW_OFF + slot * C::RAW_BYTES +
-                                                              2 * C::RAW_CODES);
-        constexpr int A = C::META_BYTES / 2;     // halves per metadata array
-        for (int j = lane; j < nv * NG; j += 32) {
-          const float sk = fabsf(half_bits_to_float(m[j]));
-          const float sv = fabsf(half_bits_to_float(m[(Q8 ? 1 : 2) * A + j]));
-          const float ak = Q8 ? 0.f : fabsf(half_bits_to_float(m[A + j]));
-          const float av = Q8 ? 0.f : fabsf(half_bits_to_float(m[3 * A + j]));
+      for (int k = 0; k < PER; ++k) {
+        const int i = lane + 32 * k;
+        const uint32_t* ks = reinterpret_cast<const uint32_t*>(&fm[0][k]);
+        const uint32_t* vs = reinterpret_cast<const uint32_t*>(&fm[Q8 ? 1 : 2][k]);
+        const uint32_t* kb = reinterpret_cast<const uint32_t*>(&fm[Q8 ? 0 : 1][k]);
+        const uint32_t* vb = reinterpret_cast<const uint32_t*>(&fm[Q8 ? 1 : 3][k]);
+#pragma unroll
+        for (int h = 0; h < 8; ++h) {
+          if (i >= U4 || (i * 8 + h) / NG >= nvt) continue;
+          const int sh = 16 * (h & 1);
+          const float sk = fabsf(half_bits_to_float((uint16_t)(ks[h >> 1] >> sh)));
+          const float sv = fabsf(half_bits_to_float((uint16_t)(vs[h >> 1] >> sh)));
+          const float ak = Q8 ? 0.f : fabsf(half_bits_to_float((uint16_t)(kb[h >> 1] >> sh)));
+          const float av = Q8 ? 0.f : fabsf(half_bits_to_float((uint16_t)(vb[h >> 1] >> sh)));
           bk = fmaxf(bk, fmaf(sk, kCodeMax, ak));
           bv = fmaxf(bv, fmaf(sv, kCodeMax, av));
         }
@@ -717,12 +781,21 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
       if (lane == 0)
         range_ring[t & (kPfRangeRing - 1)] =
             (((uint32_t)(t + 1) & 0x3fffffu) << 10) | ((uint32_t)pf_range_exp(bk) << 5) | (uint32_t)eV;
+    };
+    for (int t = 0; t < 2 && t < ntiles; ++t) { fetch(t); finish(t); }
+    if (2 < ntiles) fetch(2);
+    for (int t = 0; t < ntiles; ++t) {
       const int i0 = 2 * t + kPfRawSlots;
-      if (i0 >= nhalves) continue;
-      mbar_wait(raw_free(t & 1), (t >> 1) & 1, abort_flag, p.status, 1u);
-      // warp-uniform decision (issue_raw synchronizes the warp)
-      if (__shfl_sync(~0u, (int)*abort_flag, 0) != 0) break;
-      issue_raw(i0, nhalves - i0 < 2 ? nhalves - i0 : 2);
+      if (i0 < nhalves) {
+        mbar_wait(raw_free(t & 1), (t >> 1) & 1, abort_flag, p.status, 1u);
+        // warp-uniform decision (issue_raw synchronizes the warp)
+        if (__shfl_sync(~0u, (int)*abort_flag, 0) != 0) break;
+        issue_raw(i0, nhalves - i0 < 2 ? nhalves - i0 : 2);
+      }
+      // tile t + 2's metadata was fetched before the wait above: no stall here
+      if (t + 2 < ntiles) finish(t + 2);
+      if (t + 3 < ntiles) fetch(t + 3);
+    }
     }
     if (lane == 0) {                             // own bulk copies still in flight (after a give-up)
       for (int i = max(0, issued - kPfRawSlots); i < issued; ++i)
@@ -794,12 +867,15 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
       const int64_t key0 = (int64_t)t * kPfBN;
       mbar_wait(s_full(s), (t >> 1) & 1, abort_flag, p.status, 8u);
       tc_fence_after();
-      // S of this tile was computed from K * 2^-eK: scale it back
-      // (the ring still holds tile t - 1's entry: the producer is never more
-      // than a few tiles ahead of this role)
-      const int rg = pf_range_get(range_ring, t, abort_flag, p.status);
-      const int eK = rg < 0 ? 0 : rg >> 5;
-      const int dV = rg < 0 || t == 0 ? 0 : (rg & 31) - (int)(range_ring[(t - 1) & (kPfRangeRing - 1)] & 31u);
+      // second instance: S of this tile was computed from K * 2^-eK: scale it
+      // back (the ring still holds tile t - 1's entry: the producer is never
+      // more than a few tiles ahead of this role)
+      int eK = 0, dV = 0;
+      if constexpr (RANGE) {
+        const int rg = pf_range_get(range_ring, t, abort_flag, p.status);
+        eK = rg < 0 ? 0 : rg >> 5;
+        dV = rg < 0 || t == 0 ? 0 : (rg & 31) - (int)(range_ring[(t - 1) & (kPfRangeRing - 1)] & 31u);
+      }
       const float rs = eK == 0 ? rowscale : rowscale * exp2i(eK);
       float sv[kPfBN];
       tmem_ld32(tmem_row + C::S_COL + s * kPfBN, reinterpret_cast<uint32_t*>(sv));
@@ -925,7 +1001,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
       lsum = lsum * fo + ex2(s2 - Mn);
     }
     // O carries 2^-eV of the last tile (the largest V exponent)
-    const int eVend = ntiles > 0 ? (int)(range_ring[(ntiles - 1) & (kPfRangeRing - 1)] & 31u) : 0;
+    const int eVend = RANGE && ntiles > 0 ? (int)(range_ring[(ntiles - 1) & (kPfRangeRing - 1)] & 31u) : 0;
     const float inv = (lsum > 0.f && have) ? fo / lsum * exp2i(eVend) : 0.f;
 #pragma unroll 1
     for (int c = 0; c < D; c += 32) {
@@ -972,6 +1048,44 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n"
                  :: "r"(tmem), "r"(C::TMEM_COLS) : "memory");
   }
+  if constexpr (RANGE) {
+    if (tid == 0 && atomicAdd(p.range + 1, 1u) + 1 == gridDim.x) { p.range[1] = 0u; p.range[0] = 0u; }
+  }
+}
+
+// The range check that precedes the prefill kernel's instances: every
+// 16-byte unit of the K and V metadata rows [0, L) of every (batch, kv head)
+// slab (8 fp16 values; the values of rows at or past L ignored); if some
+// |scale| * (largest code) + |bias| reaches 2^15, the flag goes up.
+template <bool Q8, int BITS>
+__global__ void __launch_bounds__(256) qkv_range_check_kernel(const PrefillParams p, int ng) {
+  constexpr float kCodeMax = Q8 ? 128.f : (float)((1 << BITS) - 1);
+  const int64_t units = (p.L * ng + 7) / 8;                   // per slab and array
+  const int64_t slab = blockIdx.y;
+  const int64_t base = slab * p.Lcap * ng;                    // first element of the slab
+  float bound = 0.f;
+  for (int64_t u = (int64_t)blockIdx.x * 256 + threadIdx.x; u < units; u += (int64_t)gridDim.x * 256) {
+    uint4 v[4];
+    const uint16_t* arr[4] = {p.ks, Q8 ? p.ks : p.kb, p.vs, Q8 ? p.vs : p.vb};
+#pragma unroll
+    for (int a = 0; a < 4; ++a) v[a] = __ldg(reinterpret_cast<const uint4*>(arr[a] + base) + u);
+#pragma unroll
+    for (int h = 0; h < 8; ++h) {
+      if ((u * 8 + h) / ng >= p.L) break;
+      const int sh = 16 * (h & 1);
+      const uint32_t* w0 = reinterpret_cast<const uint32_t*>(&v[0]);
+      const uint32_t* w1 = reinterpret_cast<const uint32_t*>(&v[1]);
+      const uint32_t* w2 = reinterpret_cast<const uint32_t*>(&v[2]);
+      const uint32_t* w3 = reinterpret_cast<const uint32_t*>(&v[3]);
+      const float sk = fabsf(half_bits_to_float((uint16_t)(w0[h >> 1] >> sh)));
+      const float sv = fabsf(half_bits_to_float((uint16_t)(w2[h >> 1] >> sh)));
+      const float bk = Q8 ? 0.f : fabsf(half_bits_to_float((uint16_t)(w1[h >> 1] >> sh)));
+      const float bv = Q8 ? 0.f : fabsf(half_bits_to_float((uint16_t)(w3[h >> 1] >> sh)));
+      bound = fmaxf(bound, fmaxf(fmaf(sk, kCodeMax, bk), fmaf(sv, kCodeMax, bv)));
+    }
+  }
+  // NaN counts as out of range too (the scaled path takes it like the rest)
+  if (__any_sync(~0u, !(bound < 32768.f)) && (threadIdx.x & 31) == 0) atomicOr(p.range, 1u);
 }
 
 }  // namespace qkv
