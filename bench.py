@@ -684,6 +684,39 @@ def other_rows(device):
         rows["llama_q4_0_blocks_64k"] = {"unavailable": f"{type(e).__name__}: {e}"[:200]}
     torch.cuda.empty_cache()
 
+    # values as a view of the keys (MLA 576/512): one Q8_0 cache of 576-wide
+    # K rows, 128 query heads over one KV head, 32768 keys, bf16 q and out
+    try:
+        B, Hq, L = 1, 128, 32768
+        xk = torch.randn(B, 1, L, 576, device=device, dtype=torch.float16)
+        per_cache = B * L * (576 + 36)
+        ncopies = max(3, math.ceil(3 * 126e6 / per_cache))
+        caches = []
+        for _ in range(ncopies):
+            kc = qkv.QuantCache.empty(B, 1, L, 576, qkv.Q8_0, 8, 32, device)
+            qkv.qkv_quantize_update(xk, xk, kc, kc, 0)
+            caches.append(kc)
+        del xk
+        qm = torch.randn(B, Hq, 1, 576, device=device, dtype=torch.bfloat16)
+        om = torch.empty(B, Hq, 1, 512, device=device, dtype=torch.bfloat16)
+        wsm = torch.zeros(qkv.lib().qsdpa_kview_workspace_size(B, Hq, 1, 1, 576, 512, L),
+                          dtype=torch.uint8, device=device)
+        sec, _ = graph_time(lambda i: qkv.qsdpa_attention_kview(qm, caches[i % ncopies], L,
+                                                                576 ** -0.5, out=om, workspace=wsm),
+                            400, 20)
+        nb = per_cache + B * Hq * (576 + 512) * 2
+        flops = 2 * B * Hq * L * (576 + 512)
+        rows["kview_mla_q8_0_32k"] = {
+            "us_per_call": round(sec * 1e3, 3), "GB/s": round(nb / (sec / 1e3) / 1e9, 1),
+            "frac_hbm": round(nb / (sec / 1e3) / 1e9 / hbm_peak, 4),
+            "TFLOP/s": round(flops / (sec / 1e3) / 1e12, 1), "bytes": nb,
+            "note": "qsdpa_attention_kview: Q8_0 K rows of 576, V = their first 512, 128 query "
+                    "heads over 1 KV head, L = 32768 (decode)"}
+        del caches
+    except Exception as e:
+        rows["kview_mla_q8_0_32k"] = {"unavailable": f"{type(e).__name__}: {e}"[:200]}
+    torch.cuda.empty_cache()
+
     # affine codes stored 2, 3, 5 and 6 bits wide: decode of the main shape
     # (L = 65536, 32 query heads over 8 KV heads, D = 128, groups of 64)
     try:

@@ -9,7 +9,7 @@
 // codes into words and stores them; the first lane of a group stores the
 // fp16 scale (and bias).  Grid: x = blocks of tokens (256 / (D/32) tokens
 // per block), y = (batch, kv head) slab, z = K or V (one launch when both
-// caches have the same format), so no thread divides.
+// caches have the same format).
 #include <algorithm>
 
 #include "qkv_common.cuh"
@@ -29,7 +29,8 @@ struct QuantSide {
 struct QuantParams {
   QuantSide side[2];
   int D;
-  int row_shift;            // log2(D / 32): threads per token row
+  int per_row;              // D / 32: threads per token row
+  int tpb;                  // tokens per 256-thread block
   int Lnew;
   int64_t offset;
 };
@@ -37,10 +38,12 @@ struct QuantParams {
 template <int GS, int BITS, bool Q8, bool BF16>
 __global__ void __launch_bounds__(256, 6) qkv_quantize_kernel(const __grid_constant__ QuantParams p, int side0) {
   const QuantSide& s = (side0 + (int)blockIdx.z) ? p.side[1] : p.side[0];
-  const int per_row = p.D / kQEpt;
-  const int tok = blockIdx.x * (256 >> p.row_shift) + (threadIdx.x >> p.row_shift);
-  const int cs = threadIdx.x & (per_row - 1);       // which 32-element slice of the row
-  const bool active = tok < p.Lnew;                 // inactive lanes still join the shuffles
+  // rows of D / 32 threads back to back (a row starts on an even lane, so the
+  // 1, 2 or 4 lanes of a group are adjacent and aligned for the shuffles)
+  const int lt = threadIdx.x / p.per_row;           // token within the block
+  const int cs = threadIdx.x - lt * p.per_row;      // which 32-element slice of the row
+  const int tok = blockIdx.x * p.tpb + lt;
+  const bool active = lt < p.tpb && tok < p.Lnew;   // inactive lanes still join the shuffles
   const int64_t slab = blockIdx.y;                  // b * Hkv + kv head
   const int64_t srow = slab * p.Lnew + (active ? tok : 0);
   const int64_t crow = slab * s.Lcap + p.offset + tok;
@@ -135,15 +138,15 @@ cudaError_t launch_quantize(const void* new_k, const void* new_v, int in_dtype, 
     bits[i] = c[i]->fmt == QKV_Q8_0 ? 8 : c[i]->bits;
     gs[i] = c[i]->fmt == QKV_Q8_0 ? 32 : c[i]->group_size;
   }
-  int shift = 0;
-  while ((kQEpt << shift) < D) ++shift;             // D / 32 = 2^shift threads per token
   p.D = D;
-  p.row_shift = shift;
+  p.per_row = D / kQEpt;
   p.Lnew = Lnew;
   p.offset = offset;
   const int64_t slabs = (int64_t)B * Hkv;
-  if (slabs > 65535 || (kQEpt << shift) != D) return cudaErrorInvalidValue;
-  const int tpb = 256 >> shift;                     // tokens per block
+  if (slabs > 65535 || D % kQEpt != 0 || p.per_row > 256 || p.per_row % 2 != 0)
+    return cudaErrorInvalidValue;
+  const int tpb = 256 / p.per_row;                  // tokens per block
+  p.tpb = tpb;
   dim3 grid((unsigned)((Lnew + tpb - 1) / tpb), (unsigned)slabs, 1);
   const bool same = fmt[0] == fmt[1] && bits[0] == bits[1] && gs[0] == gs[1];
   const bool bf16 = in_dtype == QKV_BF16;

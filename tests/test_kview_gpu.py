@@ -77,3 +77,27 @@ def test_kview_refuses_what_it_does_not_build():
     qd, kd = to_dev(q, "bf16"), cache_to_dev(kc)
     with pytest.raises(qkv.QKVError, match="f16 or bf16"):
         qkv.qsdpa_attention_kview(qd, kd, 64, 0.1, out_dtype=torch.float32)
+
+
+@pytest.mark.parametrize("fmt,bits,gs", [("q8_0", 8, 32), ("affine", 4, 64), ("affine", 8, 32)])
+def test_kview_cache_written_by_the_quantizer(fmt, bits, gs):
+    """576-element key rows appended by qkv_quantize_update (rows of 18
+    threads) are bit-identical to the oracle's, and attended over."""
+    from quantized_kv_attention_split_b200 import qkv
+    B, Hq, L, Lcap = 1, 16, 301, 304
+    x = S.draw(7, "k", (B, 1, L, DK), "normal", "bf16")
+    f = qkv.Q8_0 if fmt == "q8_0" else qkv.AFFINE
+    kd = qkv.QuantCache.empty(B, 1, Lcap, DK, f, bits, gs)
+    vd = qkv.QuantCache.empty(B, 1, Lcap, DK, f, bits, gs)
+    qkv.qkv_quantize_update(to_dev(x, "bf16"), to_dev(x, "bf16"), kd, vd, 0)
+    torch.cuda.synchronize()
+    ref_c = oracle.quantize(x, "bf16", fmt, gs, bits)
+    from helpers import cache_from_dev
+    got_c = cache_from_dev(kd, fmt)
+    assert np.array_equal(got_c.codes[:, :, :L], ref_c.codes)
+    assert np.array_equal(got_c.scales[:, :, :L], ref_c.scales)
+    q = S.draw(8, "q", (B, Hq, 1, DK), "normal", "bf16")
+    ref = oracle.attention_kview(q, "bf16", got_c, L, 0.04, DV)
+    out = qkv.qsdpa_attention_kview(to_dev(q, "bf16"), kd, L, 0.04)
+    torch.cuda.synchronize()
+    assert out_err(from_dev(out), ref, "bf16") <= 1.0
