@@ -186,9 +186,13 @@ qkv_status qsdpa_decode_update(const void* q, int q_dtype, const void* new_k, co
  * per kv head and f16/bf16 output the call runs on the tcgen05 tensor-core
  * kernel (K and V tiles dequantized to fp16, fp32 accumulation in TMEM);
  * otherwise, and always for f32 output, on the split-K kernel.  The tcgen05
- * kernel bounds its waits on the tensor core: if one ever times out it sets
- * the first 32-bit word of the workspace nonzero (the output is then invalid);
- * that word must be zeroed again before the workspace is reused.  Its fp16
+ * kernel bounds its waits on the tensor core (200 ms each; the environment
+ * variable QKV_PREFILL_WAIT_NS sets another limit in ns, and
+ * QKV_PREFILL_STALL_HALF=i, a test hook, withholds the copy of the i-th
+ * 32-key block so that a wait runs out): if one ever times out it sets
+ * the first 32-bit word of the workspace nonzero (the output is then invalid)
+ * and the kernel still returns; that word must be zeroed again before the
+ * workspace is reused.  Its fp16
  * tiles hold scale * code + bias: a small kernel first checks every scale and
  * bias of rows [0, L), and when some value can reach 2^15 the call runs a
  * second instance of the tcgen05 kernel that scales each tile by a power of

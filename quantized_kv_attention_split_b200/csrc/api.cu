@@ -3,6 +3,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 
 #include "qkv_internal.h"
@@ -176,6 +177,12 @@ qkv_status attention(const void* q, int q_dtype, int B, int Hq, int Hkv, int Lq,
     }
     pp.cap_a = cap_a; pp.cap_k = cap_k; pp.slopes = slopes; pp.sinks = sinks;
     pp.status = static_cast<unsigned*>(workspace);
+    // time limit of the kernel's waits, and a test hook that withholds the copy
+    // of one half tile so that a wait runs out (environment, read per call)
+    pp.wait_ns = 0;
+    pp.stall_half = -1;
+    if (const char* e = std::getenv("QKV_PREFILL_WAIT_NS")) pp.wait_ns = std::strtoull(e, nullptr, 10);
+    if (const char* e = std::getenv("QKV_PREFILL_STALL_HALF")) pp.stall_half = std::atoi(e);
     pp.range = static_cast<unsigned*>(workspace) + 1;   // words 1 and 2 of the zeroed header
     cudaError_t e = qkv::launch_prefill_tc(D, k->bits, k->group_size, k->fmt, pp, s);
     if (e != cudaSuccess) return fail(QKV_ERR_CUDA, "prefill launch: %s", cudaGetErrorString(e));

@@ -67,7 +67,12 @@ constexpr int kPfThreads = 32 * (kPfProdWarp + 1);
 constexpr int kPfKSlots = 2;      // fp16 K tiles (slot free once S of the tile is done)
 constexpr int kPfVSlots = 2;      // fp16 V tiles (slot free once P V of the tile is done)
 constexpr int kPfRawSlots = 4;    // packed half tiles in flight
-constexpr unsigned kPfWaitLimit = 1u << 21;   // try_wait rounds (<= 1 us each) before giving up
+// A wait on a barrier gives up after this long (ns; PrefillParams.wait_ns
+// overrides it): a tile's waits normally end within microseconds and a whole
+// 512-query prompt at depth 20K takes about half a millisecond, so 200 ms
+// leaves room for a GPU shared with other work while a CTA that can never
+// proceed still reports within a fraction of a second.
+constexpr uint64_t kPfWaitNs = 200000000ull;
 
 struct PrefillParams {
   const void* q;            // [B, Hq, Lq, D]
@@ -92,6 +97,8 @@ struct PrefillParams {
   const float* slopes;      // per-head additive-mask slopes, fp32 [Hq] or null
   const float* sinks;       // per-head sink logits, fp32 [Hq] or null
   unsigned* status;         // nonzero after a tensor-core wait timed out
+  uint64_t wait_ns;         // time limit of a wait (0: kPfWaitNs)
+  int stall_half;           // test hook: the producer never copies this half tile (-1: none)
   unsigned* range;          // [2]: a tile reaches 2^15 (set by the first instance),
                             // CTAs of the second instance done (its last zeroes both)
 };
@@ -168,14 +175,22 @@ __device__ __forceinline__ bool mbar_try(uint32_t addr, uint32_t parity) {
       : "=r"(done) : "r"(addr), "r"(parity), "r"(1000u) : "memory");
   return done != 0;
 }
-// Bounded wait for the phase with the given parity.  Returns at once (false)
-// if the CTA has already given up; on a time-out it records the error and
-// makes the CTA give up.
+__device__ __forceinline__ uint64_t pf_now_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Bounded wait for the phase with the given parity (at most limit_ns of the
+// global timer).  Returns at once (false) if the CTA has already given up; on
+// a time-out it records the error and makes the CTA give up.
 __device__ __forceinline__ bool mbar_wait(uint32_t addr, uint32_t parity, volatile int* abort_flag,
-                                          unsigned* status, unsigned code) {
-  for (unsigned i = 0; i < kPfWaitLimit; ++i) {
+                                          unsigned* status, unsigned code, uint64_t limit_ns) {
+  if (mbar_try(addr, parity)) return true;
+  const uint64_t t0 = pf_now_ns();
+  for (;;) {
     if (mbar_try(addr, parity)) return true;
     if (*abort_flag) return false;
+    if (pf_now_ns() - t0 > limit_ns) break;
   }
   *abort_flag = 1;
   atomicOr(status, code);
@@ -183,9 +198,13 @@ __device__ __forceinline__ bool mbar_wait(uint32_t addr, uint32_t parity, volati
 }
 // Bounded wait that ignores an earlier give-up: used before exit for the
 // CTA's own asynchronous work still in flight.
-__device__ __forceinline__ void mbar_drain(uint32_t addr, uint32_t parity, unsigned* status) {
-  for (unsigned i = 0; i < kPfWaitLimit; ++i)
+__device__ __forceinline__ void mbar_drain(uint32_t addr, uint32_t parity, unsigned* status,
+                                           uint64_t limit_ns) {
+  const uint64_t t0 = pf_now_ns();
+  for (;;) {
     if (mbar_try(addr, parity)) return;
+    if (pf_now_ns() - t0 > limit_ns) break;
+  }
   atomicOr(status, 128u);
 }
 // Per-tile range exponents, published by the producer warp in a ring of 8
@@ -195,13 +214,19 @@ __device__ __forceinline__ void mbar_drain(uint32_t addr, uint32_t parity, unsig
 // returns -1 on a give-up (and records a time-out like mbar_wait).
 constexpr int kPfRangeRing = 8;
 __device__ __forceinline__ int pf_range_get(const volatile uint32_t* ring, int t,
-                                            volatile int* abort_flag, unsigned* status) {
+                                            volatile int* abort_flag, unsigned* status,
+                                            uint64_t limit_ns) {
   const uint32_t want = (uint32_t)(t + 1) & 0x3fffffu;
-  for (unsigned i = 0; i < kPfWaitLimit; ++i) {
+  uint64_t t0 = 0;
+  for (unsigned i = 0;; ++i) {
     const uint32_t v = ring[t & (kPfRangeRing - 1)];
     if ((v >> 10) == want) return (int)(v & 1023u);
     if (*abort_flag) return -1;
-    if (i >= 256) __nanosleep(64);             // normally published a tile ahead: rare
+    if (i == 256) t0 = pf_now_ns();            // normally published a tile ahead: rare
+    if (i >= 256) {
+      __nanosleep(64);
+      if (pf_now_ns() - t0 > limit_ns) break;
+    }
   }
   *abort_flag = 1;
   atomicOr(status, 256u);
@@ -478,6 +503,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(smem);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint64_t wait_ns = p.wait_ns != 0 ? p.wait_ns : kPfWaitNs;
   const uint32_t bar0 = sbase + C::BAR_OFF;
   auto raw_full = [&](int i) { return bar0 + 8 * i; };        // [4] packed half tile landed
   auto k_ready = [&](int i) { return bar0 + 32 + 8 * i; };    // [2] fp16 K written
@@ -573,6 +599,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
     if (lane == 0) {
       for (int k = 0; k < n; ++k) {
         const int i = i0 + k;
+        if (i == p.stall_half) continue;         // test hook: this half tile never lands
         const int64_t key0 = (int64_t)i * kPfRawKeys;
         const int nv = L - key0 < kPfRawKeys ? (int)(L - key0) : kPfRawKeys;
         const int nv8 = (nv + 7) & ~7;           // scale rows in whole 16-byte units
@@ -581,7 +608,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
       }
     }
     __syncwarp();
-    if (lane < n * CPH) {
+    if (lane < n * CPH && i0 + lane / CPH != p.stall_half) {
       const int i = i0 + lane / CPH, which = lane % CPH;
       const int slot = i % kPfRawSlots;
       const int64_t key0 = (int64_t)i * kPfRawKeys;
@@ -682,7 +709,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
         const int i = 2 * t + h;
         const bool present = i < nhalves;
         const int slot = i % kPfRawSlots;
-        if (present) mbar_wait(raw_full(slot), (i / kPfRawSlots) & 1, abort_flag, p.status, 1u);
+        if (present) mbar_wait(raw_full(slot), (i / kPfRawSlots) & 1, abort_flag, p.status, 1u, wait_ns);
         raw[h] = smem + C::RAW_OFF + slot * C::RAW_BYTES;
         const int64_t key0 = (int64_t)i * kPfRawKeys;
         nv[h] = !present ? 0 : (L - key0 < kPfRawKeys ? (int)(L - key0) : kPfRawKeys);
@@ -690,7 +717,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
       // the tile's range exponents (second instance only)
       int eK = 0, eV = 0;
       if constexpr (RANGE) {
-        const int rg = pf_range_get(range_ring, t, abort_flag, p.status);
+        const int rg = pf_range_get(range_ring, t, abort_flag, p.status, wait_ns);
         eK = rg < 0 ? 0 : rg >> 5;
         eV = rg < 0 ? 0 : rg & 31;
       }
@@ -700,13 +727,13 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
       vch.load(raw, C::RAW_CODES, 2 * C::RAW_CODES + (Q8 ? 1 : 2) * C::META_BYTES,
                2 * C::RAW_CODES + 3 * C::META_BYTES, nv, chunk0, eV);
       if (t >= kPfKSlots)                        // K slot free once S of tile t-2 is done
-        mbar_wait(s_full(s), ((t - 2) >> 1) & 1, abort_flag, p.status, 1u);
+        mbar_wait(s_full(s), ((t - 2) >> 1) & 1, abort_flag, p.status, 1u, wait_ns);
       kch.store(smem + C::K_OFF + s * C::KV_BYTES, chunk0);
       fence_async_smem();
       mbar_arrive(k_ready(s));
       mbar_arrive(raw_free(s));                  // this thread is done with the raw slots
       if (t >= kPfVSlots)                        // V slot free once P V of tile t-2 is done
-        mbar_wait(pv_done(s), ((t - 2) >> 1) & 1, abort_flag, p.status, 1u);
+        mbar_wait(pv_done(s), ((t - 2) >> 1) & 1, abort_flag, p.status, 1u, wait_ns);
       vch.store(smem + C::V_OFF + s * C::KV_BYTES, chunk0);
       fence_async_smem();
       mbar_arrive(v_ready(s));
@@ -717,7 +744,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
     for (int t = 0; t + 2 < ntiles || 2 * t + kPfRawSlots < nhalves; ++t) {
       const int i0 = 2 * t + kPfRawSlots;
       if (i0 >= nhalves) break;
-      mbar_wait(raw_free(t & 1), (t >> 1) & 1, abort_flag, p.status, 1u);
+      mbar_wait(raw_free(t & 1), (t >> 1) & 1, abort_flag, p.status, 1u, wait_ns);
       // warp-uniform decision (issue_raw synchronizes the warp)
       if (__shfl_sync(~0u, (int)*abort_flag, 0) != 0) break;
       issue_raw(i0, nhalves - i0 < 2 ? nhalves - i0 : 2);
@@ -787,7 +814,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
     for (int t = 0; t < ntiles; ++t) {
       const int i0 = 2 * t + kPfRawSlots;
       if (i0 < nhalves) {
-        mbar_wait(raw_free(t & 1), (t >> 1) & 1, abort_flag, p.status, 1u);
+        mbar_wait(raw_free(t & 1), (t >> 1) & 1, abort_flag, p.status, 1u, wait_ns);
         // warp-uniform decision (issue_raw synchronizes the warp)
         if (__shfl_sync(~0u, (int)*abort_flag, 0) != 0) break;
         issue_raw(i0, nhalves - i0 < 2 ? nhalves - i0 : 2);
@@ -799,7 +826,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
     }
     if (lane == 0) {                             // own bulk copies still in flight (after a give-up)
       for (int i = max(0, issued - kPfRawSlots); i < issued; ++i)
-        mbar_drain(raw_full(i % kPfRawSlots), (i / kPfRawSlots) & 1, p.status);
+        mbar_drain(raw_full(i % kPfRawSlots), (i / kPfRawSlots) & 1, p.status, wait_ns);
     }
     __syncwarp();
   } else if (warp == kPfMmaWarp) {
@@ -808,7 +835,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
     constexpr uint32_t idesc_o = f16_idesc(kPfBM, D, true);
     auto issue_s = [&](int t) {
       const int s = t & 1;
-      mbar_wait(k_ready(s), (t >> 1) & 1, abort_flag, p.status, 2u);
+      mbar_wait(k_ready(s), (t >> 1) & 1, abort_flag, p.status, 2u, wait_ns);
       tc_fence_after();
       if (lane == 0) {
 #pragma unroll
@@ -824,8 +851,8 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
     };
     auto issue_pv = [&](int t) {
       const int s = t & 1;
-      mbar_wait(v_ready(s), (t >> 1) & 1, abort_flag, p.status, 4u);
-      mbar_wait(p_ready(s), (t >> 1) & 1, abort_flag, p.status, 4u);
+      mbar_wait(v_ready(s), (t >> 1) & 1, abort_flag, p.status, 4u, wait_ns);
+      mbar_wait(p_ready(s), (t >> 1) & 1, abort_flag, p.status, 4u, wait_ns);
       tc_fence_after();
       if (lane == 0) {
 #pragma unroll
@@ -850,7 +877,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
     }
     if (lane == 0) {                             // every MMA issued above has completed
       tc_commit(mma_done);
-      mbar_drain(mma_done, 0, p.status);
+      mbar_drain(mma_done, 0, p.status, wait_ns);
     }
     __syncwarp();
   } else {
@@ -865,14 +892,14 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
     for (int t = 0; t < ntiles; ++t) {
       const int s = t & 1;
       const int64_t key0 = (int64_t)t * kPfBN;
-      mbar_wait(s_full(s), (t >> 1) & 1, abort_flag, p.status, 8u);
+      mbar_wait(s_full(s), (t >> 1) & 1, abort_flag, p.status, 8u, wait_ns);
       tc_fence_after();
       // second instance: S of this tile was computed from K * 2^-eK: scale it
       // back (the ring still holds tile t - 1's entry: the producer is never
       // more than a few tiles ahead of this role)
       int eK = 0, dV = 0;
       if constexpr (RANGE) {
-        const int rg = pf_range_get(range_ring, t, abort_flag, p.status);
+        const int rg = pf_range_get(range_ring, t, abort_flag, p.status, wait_ns);
         eK = rg < 0 ? 0 : rg >> 5;
         dV = rg < 0 || t == 0 ? 0 : (rg & 31) - (int)(range_ring[(t - 1) & (kPfRangeRing - 1)] & 31u);
       }
@@ -935,7 +962,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
       const float alpha_o = dV > 0 ? alpha * exp2i(-dV) : alpha;
       const bool rescale = t > 0 && __any_sync(~0u, alpha_o != 1.f);
       if (rescale) {                             // needs P V of tile t-1 done (rare)
-        mbar_wait(pv_done((t - 1) & 1), ((t - 1) >> 1) & 1, abort_flag, p.status, 32u);
+        mbar_wait(pv_done((t - 1) & 1), ((t - 1) >> 1) & 1, abort_flag, p.status, 32u, wait_ns);
         tc_fence_after();
 #pragma unroll 1
         for (int c = 0; c < D; c += 32) {
@@ -988,7 +1015,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
     // ---- epilogue: O / l -> out --------------------------------------------
     bool have = ntiles > 0;
     if (have) {
-      have = mbar_wait(pv_done((ntiles - 1) & 1), ((ntiles - 1) >> 1) & 1, abort_flag, p.status, 64u);
+      have = mbar_wait(pv_done((ntiles - 1) & 1), ((ntiles - 1) >> 1) & 1, abort_flag, p.status, 64u, wait_ns);
       tc_fence_after();
     }
     have = __all_sync(~0u, have) && !*abort_flag;
