@@ -375,39 +375,53 @@ def run_ours(args, rank, world, device):
     # one call alone (cold L2, no overlap with a previous call)
     iso_sec = max_over_ranks(isolated_time(step), device, world)
 
-    # e2e through the public API with host buffers: H2D of q, decode, D2H of out
+    # e2e through the public API with host buffers: q in pinned host memory,
+    # the output back in pinned host memory.  The library takes such buffers
+    # directly (its kernels read q and write out over the host link), so a
+    # step is one call; the variant with explicit copies (H2D of q into a
+    # device buffer, decode, D2H of the output) is timed beside it.
     q_host = torch.from_numpy(inp.q.view(np.int16)).view(torch.float16).pin_memory()
     out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     qe = torch.empty_like(qd)
     ke = max(20, min(args.steps, 2000))
-    for i in range(5):
+
+    def e2e_step(i):
+        kc, vc = caches[i % ncopies]
+        qkv.qsdpa_decode(q_host, kc, vc, w.L, w.scale, out=out_host, workspace=ws)
+
+    def copy_step(i):
         qe.copy_(q_host, non_blocking=True)
-        step(i)
+        kc, vc = caches[i % ncopies]
+        qkv.qsdpa_decode(qe, kc, vc, w.L, w.scale, out=out, workspace=ws)
         out_host.copy_(out, non_blocking=True)
+
+    for i in range(5):
+        e2e_step(i)
+        copy_step(i)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         torch.distributed.barrier()
     e0.record()
     for i in range(ke):
-        qe.copy_(q_host, non_blocking=True)
-        kc, vc = caches[i % ncopies]
-        qkv.qsdpa_decode(qe, kc, vc, w.L, w.scale, out=out, workspace=ws)
-        out_host.copy_(out, non_blocking=True)
+        e2e_step(i)
     e1.record()
     torch.cuda.synchronize()
     eager_sec = max_over_ranks(e0.elapsed_time(e1) / 1e3 / ke, device, world)
-
     # the same steps recorded once in a CUDA graph and replayed (what a serving
-    # loop does to take the host's per-call cost out): every step still copies
-    # q in from pinned host memory and the output back out
-    def e2e_step(i):
-        qe.copy_(q_host, non_blocking=True)
-        kc, vc = caches[i % ncopies]
-        qkv.qsdpa_decode(qe, kc, vc, w.L, w.scale, out=out, workspace=ws)
-        out_host.copy_(out, non_blocking=True)
+    # loop does to take the host's per-call cost out)
     e2e_ms, _ = graph_time(e2e_step, ke, 5, sync_ranks=True)
     e2e_sec = max_over_ranks(e2e_ms / 1e3, device, world)
+    copy_ms, _ = graph_time(copy_step, ke, 5, sync_ranks=True)
+    copy_sec = max_over_ranks(copy_ms / 1e3, device, world)
+    # the host buffers hold the same result as the device-buffer call
+    ref_out = out.clone()
+    qkv.qsdpa_decode(qd, caches[0][0], caches[0][1], w.L, w.scale, out=ref_out, workspace=ws)
+    e2e_step(0)
+    torch.cuda.synchronize()
+    e2e_diff = (out_host.float() - ref_out.float().cpu()).abs().max().item()
+    if not e2e_diff <= 2e-3:
+        raise SystemExit(f"e2e: host-buffer result differs from the device-buffer call by {e2e_diff}")
 
     result = None
     if rank == 0:
@@ -447,13 +461,17 @@ def run_ours(args, rank, world, device):
             "e2e": {"value": round(replica_rate(alg_bytes, e2e_sec, world) / 1e9, 2), "unit": "GB/s",
                     "us_per_call": round(e2e_sec * 1e6, 3),
                     "eager_us_per_call": round(eager_sec * 1e6, 3),
+                    "copy_engine_us_per_call": round(copy_sec * 1e6, 3),
                     "h2d_bytes_per_step": int(qd.numel() * 2),
                     "d2h_bytes_per_step": int(out.numel() * 2),
-                    "note": "each step: q copied in from pinned host memory, qsdpa_decode through "
-                            "the Python binding and C ABI, the output copied back to pinned host "
-                            "memory; the steps recorded in CUDA graphs and replayed (device time "
-                            "of exactly K steps); eager_us_per_call: the same steps issued one by "
-                            "one from Python (host-bound)"},
+                    "note": "each step: qsdpa_decode through the Python binding and C ABI with q "
+                            "in pinned host memory and the output written to pinned host memory "
+                            "(the kernels move both over the host link); the steps recorded in "
+                            "CUDA graphs and replayed (device time of exactly K steps); "
+                            "eager_us_per_call: the same steps issued one by one from Python "
+                            "(host-bound); copy_engine_us_per_call: explicit cudaMemcpyAsync of q "
+                            "in and of the output out around a call on device buffers, replayed "
+                            "the same way"},
             "gpu_launches": LAUNCHES.get("main") if LAUNCHES.get("main") is not None else args.steps,
             "gpu_launches_source": ("kernel nodes of the captured CUDA graphs (decode kernel, plus "
                                     "the merge kernel when a unit is split over CTAs)"

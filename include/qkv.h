@@ -16,9 +16,18 @@
  *    logit softcap) and the other KV block types (Q4_0, Q4_1, Q5_0, Q5_1).
  *
  * Conventions shared by every entry point
- *  - All tensor pointers are DEVICE pointers owned by the caller.  The library
- *    never allocates device memory and never synchronizes: work is enqueued on
- *    `stream` (a cudaStream_t; NULL = legacy default stream).
+ *  - All tensor pointers are DEVICE pointers owned by the caller, with one
+ *    exception: q and out of the attention calls (qsdpa_decode, _ext,
+ *    _update, _noalloc, qsdpa_prefill, _ext) may instead point to page-locked
+ *    host memory that the device addresses at the same pointer (cudaHostAlloc
+ *    or cudaMallocHost memory, or cudaHostRegister'ed memory, on a host with
+ *    unified addressing).  The split-K kernels then read q and write out over
+ *    the host link themselves, with no separate copy, and a multi-query call
+ *    with such a q or out runs on the split-K kernel.  Any other host address
+ *    (pageable memory) returns QKV_ERR_INVALID_ARG before anything is
+ *    launched.  The library never allocates device memory and never
+ *    synchronizes: work is enqueued on `stream` (a cudaStream_t; NULL =
+ *    legacy default stream).
  *  - Half-precision values are passed as their 16-bit patterns.
  *  - Arguments are validated before anything is launched.  On any error the
  *    call returns a status other than QKV_OK, launches nothing, and
@@ -71,7 +80,7 @@ typedef enum { QKV_MASK_NONE = 0, QKV_MASK_CAUSAL = 1, QKV_MASK_ADDITIVE = 2 } q
 
 typedef struct {
   int fmt;              /* qkv_format                                         */
-  int bits;             /* affine: 4 or 8; Q8_0: 8                            */
+  int bits;             /* affine: 2, 3, 4, 5, 6 or 8; Q8_0: 8                */
   int group_size;       /* affine: 32, 64 or 128; Q8_0: 32                    */
   uint32_t* codes;      /* [B, Hkv, Lcap, D*bits/32]                          */
   uint16_t* scales;     /* fp16 [B, Hkv, Lcap, D/group_size]                  */

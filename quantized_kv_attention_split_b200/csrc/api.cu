@@ -82,6 +82,35 @@ qkv_status check_cache(const char* name, const qkv_cache* c, int D, bool kview =
   return QKV_OK;
 }
 
+// Where q or out of an attention call lives.  Device (or managed) memory, or
+// page-locked host memory that the device reads and writes at the same
+// address (cudaHostAlloc / cudaMallocHost, and cudaHostRegister where the
+// mapping is the identity, as with unified addressing on 64-bit hosts): the
+// split-K kernels then move those bytes over the host link themselves.
+// Anything else -- pageable host memory, an unknown address -- is refused
+// before a launch, since no kernel could touch it.
+enum class Where { kDevice, kHost };
+qkv_status where_is(const char* name, const void* ptr, Where* w) {
+  cudaPointerAttributes a;
+  const cudaError_t e = cudaPointerGetAttributes(&a, ptr);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    if (e == cudaErrorInvalidValue)
+      return fail(QKV_ERR_INVALID_ARG, "%s: not an address the device can use", name);
+    return fail(QKV_ERR_CUDA, "cudaPointerGetAttributes(%s): %s", name, cudaGetErrorString(e));
+  }
+  if (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) {
+    *w = Where::kDevice;
+    return QKV_OK;
+  }
+  if (a.type == cudaMemoryTypeHost && a.devicePointer == ptr) {
+    *w = Where::kHost;
+    return QKV_OK;
+  }
+  return fail(QKV_ERR_INVALID_ARG,
+              "%s must be device memory or page-locked host memory mapped at the same address", name);
+}
+
 qkv_status check_dtype(const char* name, int dt, bool allow_f32) {
   if (dt == QKV_F16 || dt == QKV_BF16 || (allow_f32 && dt == QKV_F32)) return QKV_OK;
   return fail(QKV_ERR_INVALID_ARG, "%s: unsupported dtype %d", name, dt);
@@ -142,6 +171,11 @@ qkv_status attention(const void* q, int q_dtype, int B, int Hq, int Hkv, int Lq,
     sinks = ext->sinks;
   }
 
+  Where q_at, out_at;
+  if ((st = where_is("q", q, &q_at)) != QKV_OK) return st;
+  if ((st = where_is("out", out, &out_at)) != QKV_OK) return st;
+  const bool host_io = q_at == Where::kHost || out_at == Where::kHost;
+
   const size_t elems = (size_t)B * Hq * Lq * D;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (L == 0) {
@@ -153,10 +187,11 @@ qkv_status attention(const void* q, int q_dtype, int B, int Hq, int Hkv, int Lq,
 
   const int G = Hq / Hkv;
   const int rows = G * Lq;                 // rows of one kv head: (head, query) pairs
-  // the tcgen05 kernel dequantizes 4- and 8-bit codes; other widths take the
+  // the tcgen05 kernel dequantizes 4- and 8-bit codes and takes q and out
+  // from device memory; other widths, and q or out in host memory, take the
   // split-K kernel
   const bool tc_codes = k->fmt == QKV_Q8_0 || k->bits == 4 || k->bits == 8;
-  if (Lq > 1 && rows >= kTensorPrefillMinRows && out_dtype != QKV_F32 && tc_codes) {
+  if (Lq > 1 && rows >= kTensorPrefillMinRows && out_dtype != QKV_F32 && tc_codes && !host_io) {
     // many query rows per kv head: the tcgen05 kernel (whole 128-row tiles)
     const size_t need = qsdpa_workspace_size(B, Hq, Hkv, Lq, D, L);
     if (workspace == nullptr || workspace_bytes < need)

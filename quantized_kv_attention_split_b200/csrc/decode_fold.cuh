@@ -107,10 +107,8 @@ __device__ __forceinline__ void merge_item(const DecodeParams& p, const UnitPart
   }
   const float inv = Ls > 0.f ? fo / Ls : 0.f;
   const int64_t oi = (uh * p.G + head) * D + e4 * 4;
-  store_from_float(p.out, p.out_dtype, oi, acc.x * inv);
-  store_from_float(p.out, p.out_dtype, oi + 1, acc.y * inv);
-  store_from_float(p.out, p.out_dtype, oi + 2, acc.z * inv);
-  store_from_float(p.out, p.out_dtype, oi + 3, acc.w * inv);
+  store4_from_float(p.out, p.out_dtype, oi,
+                    make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv));
 }
 
 }  // namespace qkv

@@ -99,6 +99,25 @@ __device__ __forceinline__ void store_from_float(void* p, int dtype, int64_t i, 
   else reinterpret_cast<float*>(p)[i] = v;
 }
 
+// Four consecutive outputs i..i+3 (i a multiple of 4, the buffer 16-byte
+// aligned) in one 8- or 16-byte store: fewer, wider writes, which matters
+// most when out is host memory written over the host link.
+__device__ __forceinline__ void store4_from_float(void* p, int dtype, int64_t i, float4 v) {
+  if (dtype == QKV_F32) {
+    *reinterpret_cast<float4*>(reinterpret_cast<float*>(p) + i) = v;
+    return;
+  }
+  uint2 w;
+  if (dtype == QKV_F16) {
+    const __half2 a = __floats2half2_rn(v.x, v.y), b = __floats2half2_rn(v.z, v.w);
+    w = make_uint2(*reinterpret_cast<const uint32_t*>(&a), *reinterpret_cast<const uint32_t*>(&b));
+  } else {
+    const __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+    w = make_uint2(*reinterpret_cast<const uint32_t*>(&a), *reinterpret_cast<const uint32_t*>(&b));
+  }
+  *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(p) + i) = w;
+}
+
 // Programmatic dependent launch: a kernel launched with programmatic stream
 // serialization may start while the previous kernel of the stream is still
 // running; grid_dep_wait() returns once that kernel has completed and its

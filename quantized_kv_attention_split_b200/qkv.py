@@ -2,8 +2,9 @@
 
 The functions keep the names of the C entry points declared in
 ``include/qkv.h`` -- :func:`qkv_quantize_update`, :func:`qsdpa_decode`,
-:func:`qsdpa_prefill` -- and take torch CUDA tensors, passing their device
-pointers, sizes and the current CUDA stream to the library.  Every step of the
+:func:`qsdpa_prefill` -- and take torch CUDA tensors (q and out of the
+attention calls may also be pinned CPU tensors), passing their pointers,
+sizes and the current CUDA stream to the library.  Every step of the
 computation runs in the library's kernels; there is no fallback: if the
 library is missing or a call fails, a Python exception is raised.
 """
@@ -366,23 +367,30 @@ def _ext_struct(softcap, sinks, mask_slopes, Hq, device):
                 None if sinks is None else sinks.data_ptr())
 
 
+def _io_ok(t: torch.Tensor) -> bool:
+    """q and out of the attention calls: CUDA tensors, or page-locked CPU
+    tensors, which the kernels read and write over the host link."""
+    return t.is_contiguous() and (t.is_cuda or t.is_pinned())
+
+
 def _attention(fn, q, k, v, L, scale, mask, causal, out, out_dtype, workspace, stream, decode,
                ext=None):
-    assert q.is_contiguous() and q.is_cuda
+    assert _io_ok(q) and (out is None or _io_ok(out))
     B, Hq, Lq, D = q.shape
     Hkv = k.codes.shape[1]
+    dev = k.codes.device                   # the device that runs the call
     if out is None:
-        out = torch.empty(B, Hq, Lq, D, dtype=out_dtype or q.dtype, device=q.device)
+        out = torch.empty(B, Hq, Lq, D, dtype=out_dtype or q.dtype, device=dev)
     if workspace is None:
-        with _on(q):                       # sized for the device that runs the call
-            workspace = make_workspace(B, Hq, Hkv, Lq, D, L, q.device)
+        with _on(k.codes):                 # sized for the device that runs the call
+            workspace = make_workspace(B, Hq, Hkv, Lq, D, L, dev)
     ks, vs = k._struct(), v._struct()
     m = _mask_struct(mask, causal)
     mp = C.byref(m) if m is not None else None
     common = (C.byref(ks), C.byref(vs), int(L), float(scale), mp)
     if ext is not None:
         common += (C.byref(ext),)
-    with _on(q):
+    with _on(k.codes):
         common += (out.data_ptr(), _DTYPE[out.dtype], workspace.data_ptr(), workspace.numel(),
                    _stream(stream))
         if decode:
@@ -399,9 +407,13 @@ def qsdpa_decode(q: torch.Tensor, k: QuantCache, v: QuantCache, L: int, scale: f
                  mask_slopes: Optional[torch.Tensor] = None) -> torch.Tensor:
     """softmax(q*scale . K^T + mask) V for q [B,Hq,1,D] over keys [0, L).
     ``softcap``, ``sinks`` and ``mask_slopes`` are the attention extensions
-    of ``qkv_attn_ext`` (qsdpa_decode_ext)."""
+    of ``qkv_attn_ext`` (qsdpa_decode_ext).  ``q`` and ``out`` may be CUDA
+    tensors on the caches' device or page-locked (pinned) CPU tensors: the
+    kernels then read q and write out over the host link, with no separate
+    copy.  The same holds for :func:`qsdpa_prefill`, whose calls with host
+    tensors run on the split-K kernel."""
     assert q.shape[2] == 1
-    ext = _ext_struct(softcap, sinks, mask_slopes, q.shape[1], q.device)
+    ext = _ext_struct(softcap, sinks, mask_slopes, q.shape[1], k.codes.device)
     fn = lib().qsdpa_decode if ext is None else lib().qsdpa_decode_ext
     return _attention(fn, q, k, v, L, scale, mask, False, out, out_dtype, workspace, stream,
                       True, ext)
@@ -444,7 +456,7 @@ def qsdpa_prefill(q: torch.Tensor, k: QuantCache, v: QuantCache, L: int, scale: 
     """softmax(q*scale . K^T + mask) V for q [B,Hq,Lq,D] over keys [0, L);
     ``causal`` aligns the Lq queries with the last Lq keys.  ``softcap``,
     ``sinks`` and ``mask_slopes`` as in :func:`qsdpa_decode`."""
-    ext = _ext_struct(softcap, sinks, mask_slopes, q.shape[1], q.device)
+    ext = _ext_struct(softcap, sinks, mask_slopes, q.shape[1], k.codes.device)
     fn = lib().qsdpa_prefill if ext is None else lib().qsdpa_prefill_ext
     return _attention(fn, q, k, v, L, scale, mask, causal, out, out_dtype, workspace, stream,
                       False, ext)
@@ -464,14 +476,14 @@ def qsdpa_decode_noalloc(q: torch.Tensor, k: QuantCache, v: QuantCache, L: int, 
                       C.POINTER(_Cache), C.POINTER(_Cache), C.c_int64, C.c_float,
                       C.POINTER(_Mask), C.c_void_p, C.c_int, C.c_void_p]
         f.restype = C.c_int
-    assert q.is_contiguous() and q.is_cuda and q.shape[2] == 1
+    assert _io_ok(q) and (out is None or _io_ok(out)) and q.shape[2] == 1
     B, Hq, _, D = q.shape
     Hkv = k.codes.shape[1]
     if out is None:
-        out = torch.empty(B, Hq, 1, D, dtype=out_dtype or q.dtype, device=q.device)
+        out = torch.empty(B, Hq, 1, D, dtype=out_dtype or q.dtype, device=k.codes.device)
     ks, vs = k._struct(), v._struct()
     m = _mask_struct(mask, False)
-    with _on(q):
+    with _on(k.codes):
         _check(f(q.data_ptr(), _DTYPE[q.dtype], B, Hq, Hkv, D, C.byref(ks), C.byref(vs), int(L),
                  float(scale), C.byref(m) if m is not None else None, out.data_ptr(),
                  _DTYPE[out.dtype], _stream(stream)))
