@@ -777,8 +777,9 @@ def other_rows(device):
             rows[f"decode_64k_affine{bits}"] = {
                 "us_per_call": round(sec * 1e3, 3), "GB/s": round(nb / (sec / 1e3) / 1e9, 1),
                 "frac_hbm": round(nb / (sec / 1e3) / 1e9 / hbm_peak, 4), "bytes": nb,
-                "note": f"{bits}-bit codes (one bit stream per row), transcoded to 8-bit per "
-                        f"block by the decode kernel; caches written by qkv_quantize_update"}
+                "note": f"{bits}-bit codes (one bit stream per row), transcoded per block to "
+                        f"{4 if bits < 4 else 8}-bit codes by the decode kernel; caches written "
+                        f"by qkv_quantize_update"}
             del caches
         del kx, vx
     except Exception as e:

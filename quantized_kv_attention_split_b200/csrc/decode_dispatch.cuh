@@ -110,17 +110,19 @@ bool decode_ops_for(int bits, int gs, bool q8, int nc, bool f32, int var, Decode
 }
 
 // Affine codes stored 2, 3, 5 or 6 bits wide: the plain kernel (no additive
-// mask, no extensions, no fused update), transcoding each block to 8-bit.
+// mask, no extensions, no fused update), transcoding each block to the
+// 4-bit tile (2- and 3-bit codes) or the 8-bit tile (5- and 6-bit codes).
 template <int D>
 bool decode_ops_x_for(int bits, int gs, int nc, bool f32, DecodeOps* ops) {
 #define QKV_DEC_X(SB, GS)                                                                      \
   do {                                                                                         \
-    if (nc == 1) *ops = f32 ? make_decode_ops<D, 8, GS, false, 1, true, kDecPlain, SB>()       \
-                            : make_decode_ops<D, 8, GS, false, 1, false, kDecPlain, SB>();     \
-    else if (nc == 2) *ops = f32 ? make_decode_ops<D, 8, GS, false, 2, true, kDecPlain, SB>()  \
-                                 : make_decode_ops<D, 8, GS, false, 2, false, kDecPlain, SB>(); \
-    else *ops = f32 ? make_decode_ops<D, 8, GS, false, 4, true, kDecPlain, SB>()               \
-                    : make_decode_ops<D, 8, GS, false, 4, false, kDecPlain, SB>();             \
+    constexpr int CB = SB < 4 ? 4 : 8;                                                         \
+    if (nc == 1) *ops = f32 ? make_decode_ops<D, CB, GS, false, 1, true, kDecPlain, SB>()      \
+                            : make_decode_ops<D, CB, GS, false, 1, false, kDecPlain, SB>();    \
+    else if (nc == 2) *ops = f32 ? make_decode_ops<D, CB, GS, false, 2, true, kDecPlain, SB>() \
+                                 : make_decode_ops<D, CB, GS, false, 2, false, kDecPlain, SB>(); \
+    else *ops = f32 ? make_decode_ops<D, CB, GS, false, 4, true, kDecPlain, SB>()              \
+                    : make_decode_ops<D, CB, GS, false, 4, false, kDecPlain, SB>();            \
     return true;                                                                               \
   } while (0)
 #define QKV_DEC_XB(SB)                                      \

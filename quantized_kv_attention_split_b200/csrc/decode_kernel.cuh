@@ -109,10 +109,11 @@ __device__ __forceinline__ int swz_offset(int lin) {
 }
 
 // SB: the width of the codes as stored in the cache.  BITS (4 or 8) is the
-// width the fragment code computes with; SB != BITS (affine 2, 3, 5 or 6-bit
-// codes, computed as 8-bit) stages each block's packed rows as they are (one
-// little-endian bit stream per row; rows straddle 16-byte units) and the team
-// transcodes them into an 8-bit tile of its own before the block's math.
+// width the fragment code computes with; SB != BITS (affine 2 or 3-bit codes,
+// computed as 4-bit; 5 or 6-bit codes, computed as 8-bit) stages each block's
+// packed rows as they are (one little-endian bit stream per row; rows
+// straddle 16-byte units) and the team transcodes them into a tile of its own
+// before the block's math.
 template <int D, int BITS, int GS, bool Q8, int NC, int SB = BITS>
 struct DecCfg {
   static constexpr bool XC = SB != BITS;       // transcoded from SB-bit codes
@@ -141,7 +142,7 @@ struct DecCfg {
   // staged codes of one tile (K or V): the compute tile, or the packed rows
   static constexpr int scodes(int sub) { return XC ? r16(16 * sub * RBS) : 16 * sub * RB; }
   static constexpr int stage_bytes(int sub) { return r128(2 * scodes(sub) + NMETA * r16(16 * sub * MROW)); }
-  // a team's 8-bit K and V tiles (transcoded blocks only)
+  // a team's K and V compute tiles (transcoded blocks only)
   static constexpr int xtile_bytes(int sub) { return XC ? 2 * 16 * sub * RB : 0; }
   // 16-key sub-blocks per block: two when three such stages per team fit
   // (D = 256 keeps one: its register budget is spent)
@@ -162,7 +163,7 @@ struct DecCfg {
   static constexpr int STAGE = stage_bytes(SUB);
   static constexpr int NS_FIT = (BUDGET - QSB - NEWB - NTEAM * XT) / (NTEAM * STAGE);
   static constexpr int NSTAGE = NS_FIT > 6 ? 6 : NS_FIT;
-  static constexpr int XTOFF = NSTAGE * STAGE;          // the team's 8-bit tiles after its ring
+  static constexpr int XTOFF = NSTAGE * STAGE;          // the team's compute tiles after its ring
   static constexpr int TRING = NSTAGE * STAGE + XT;     // one team's region
   static constexpr int QOFF = NTEAM * TRING;            // query rows after the rings
   // epilogue (after every ring is drained): per-warp partial rows, then the
@@ -172,7 +173,7 @@ struct DecCfg {
   static constexpr int EPI = EPI_W + NC * 8 * (NTEAM + 1) * 4 + NC * 8 * 2 * 4;
   static constexpr int NEWOFF = QOFF + QSB;
   static constexpr int SMEM = NEWOFF + NEWB > EPI ? NEWOFF + NEWB : EPI;
-  // three stages per team (two for transcoded blocks, whose 8-bit tiles take
+  // three stages per team (two for transcoded blocks, whose compute tiles take
   // the room of the third: the copy of the next block still overlaps the
   // math of the current one)
   static_assert(NSTAGE >= (XC ? 2 : 3), "stages per team");
@@ -322,39 +323,74 @@ __device__ __forceinline__ void dec_mask_vals(const T* m, int nk, float (&mv)[SU
     }
 }
 
+// Masks of the field-spreading step below: N codes form blocks of 2H codes,
+// block b starting at bit 2 H b BITS, each block's codes still packed SB bits
+// apart; LO selects every block's lower H codes, HI its upper H codes.
+__host__ __device__ constexpr uint32_t spread_mask(int N, int H, int SB, int BITS, bool hi) {
+  uint32_t m = 0u;
+  for (int b = 0; b < N / (2 * H); ++b)
+    for (int i = hi ? H * SB : 0; i < (hi ? 2 * H * SB : H * SB); ++i) m |= 1u << (2 * H * b * BITS + i);
+  return m;
+}
+
+// N codes of SB bits packed from bit 0 -> the same codes BITS bits apart
+// (BITS > SB): halving steps, each moving the upper half of every block up
+// into the zero gap above it (two ANDs, a shift and an OR per step).
+template <int N, int SB, int BITS, int H = N / 2>
+__device__ __forceinline__ uint32_t spread_codes(uint32_t f) {
+  if constexpr (H == 0) {
+    return f;
+  } else {
+    constexpr uint32_t LO = spread_mask(N, H, SB, BITS, false), HI = spread_mask(N, H, SB, BITS, true);
+    return spread_codes<N, SB, BITS, H / 2>((f & LO) | ((f & HI) << (H * (BITS - SB))));
+  }
+}
+
 // A team's transcode of one staged block of SB-bit codes (K rows, then V
 // rows SCODES bytes later; each row one little-endian bit stream, element e
-// at bits [e SB, (e + 1) SB)) into its 8-bit K and V tiles at xt, laid out and
-// swizzled exactly as staged 8-bit codes are.  A thread takes 16-code units
-// (one 16-byte unit of the 8-bit tile): two 64-bit windows of the stream, each
-// giving 8 codes.  Reads stay inside the stage (the V rows and the metadata
-// follow the K rows; the metadata follow the V rows).
-template <class C, int D, int SB>
+// at bits [e SB, (e + 1) SB)) into its K and V tiles of BITS-bit codes at xt
+// (4-bit for 2- and 3-bit codes, 8-bit for 5- and 6-bit ones), laid out and
+// swizzled exactly as staged codes of that width are.  A thread takes one
+// 16-byte unit of the tile: U = 128 / BITS codes, whose U SB stream bits
+// start at a word boundary (at bit 16 of a word for odd units of 5-bit
+// codes); each output word is one field of 32 / BITS codes, spread.  Reads
+// stay inside the stage (the V rows and the metadata follow the K rows; the
+// metadata follow the V rows).
+template <class C, int D, int SB, int BITS>
 __device__ __forceinline__ void transcode_block(const uint8_t* raw, uint8_t* xt, int ttid) {
-  constexpr int UPR8 = C::RB / 16;                 // 16-code units per row
-  constexpr int ITEMS = 2 * C::BK * UPR8;
-  constexpr uint32_t MASK = (1u << SB) - 1u;
+  constexpr int U = 128 / BITS;                    // codes per 16-byte unit of the tile
+  constexpr int F = 32 / BITS;                     // codes per output word
+  constexpr int UPR = C::RB / 16;                  // units per row
+  constexpr int ITEMS = 2 * C::BK * UPR;
+  constexpr bool ALIGNED = (U * SB) % 32 == 0;     // every unit starts at a word
+  constexpr int NIN = ALIGNED ? U * SB / 32 : (U * SB + 16 + 31) / 32;   // input words read
+  constexpr uint32_t FMASK = F * SB == 32 ? ~0u : (1u << (F * SB)) - 1u;
+  static_assert((D * SB) % 32 == 0, "rows start at a word");
+  static_assert(ALIGNED || SB == 5, "unaligned units only for 5-bit codes (offset 0 or 16)");
   const uint32_t* rw = reinterpret_cast<const uint32_t*>(raw);
 #pragma unroll 2
   for (int it = ttid; it < ITEMS; it += C::TTHR) {
-    const int which = it >= C::BK * UPR8;
-    const int rem = which ? it - C::BK * UPR8 : it;
-    const int r = rem / UPR8, j = rem - r * UPR8;
-    const uint32_t* base = rw + which * (C::SCODES / 4);
-    const int p0 = (r * D + 16 * j) * SB;           // bit position of the unit's first code
+    const int which = it >= C::BK * UPR;
+    const int rem = which ? it - C::BK * UPR : it;
+    const int r = rem / UPR, j = rem - r * UPR;
+    const int p0 = (r * D + U * j) * SB;           // stream bit of the unit's first code
+    const uint32_t* src = rw + which * (C::SCODES / 4) + (p0 >> 5);
+    uint32_t w[NIN + 1];
+#pragma unroll
+    for (int k = 0; k < NIN; ++k) w[k] = src[k];
+    w[NIN] = 0u;
+    if constexpr (!ALIGNED) {
+      const int sh = p0 & 31;                      // 0 or 16
+#pragma unroll
+      for (int k = 0; k < NIN; ++k) w[k] = __funnelshift_r(w[k], w[k + 1], sh);
+    }
     uint32_t out[4];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int ph = p0 + 8 * h * SB, wi = ph >> 5, sh = ph & 31;
-      const uint32_t w0 = base[wi], w1 = base[wi + 1], w2 = base[wi + 2];
-      const uint64_t v = ((uint64_t)__funnelshift_r(w1, w2, sh) << 32) | __funnelshift_r(w0, w1, sh);
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        uint32_t o = 0u;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) o |= ((uint32_t)(v >> ((4 * k + e) * SB)) & MASK) << (8 * e);
-        out[2 * h + k] = o;
-      }
+    for (int o = 0; o < 4; ++o) {
+      constexpr int FB = F * SB;                   // field bits
+      const int bit = o * FB, wi = bit >> 5, sh = bit & 31;
+      const uint32_t f = (sh == 0 ? w[wi] : __funnelshift_r(w[wi], w[wi + 1], sh)) & FMASK;
+      out[o] = spread_codes<F, SB, BITS>(f);
     }
     const int lin = r * C::RB + 16 * j;
     *reinterpret_cast<uint4*>(xt + (which ? C::CODES + swz_xor<C::SWZV>(lin) : swz_xor<C::SWZ>(lin))) =
@@ -369,7 +405,8 @@ qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
   constexpr bool EXT = VAR == kDecExt;         // logit softcap, mask slopes, sinks
   constexpr bool ADDMASK = VAR != kDecPlain;   // additive masks (plain: none, or causal)
   using C = DecCfg<D, BITS, GS, Q8, NC, SB>;
-  static_assert(!C::XC || (BITS == 8 && !Q8 && VAR == kDecPlain), "stored widths compute as 8-bit");
+  static_assert(!C::XC || (!Q8 && VAR == kDecPlain && ((BITS == 4 && SB < 4) || (BITS == 8 && SB > 4 && SB < 8))),
+                "2- and 3-bit codes compute as 4-bit, 5- and 6-bit codes as 8-bit");
   constexpr int NG = C::NG, KPG = C::KPG, MT = C::MT, BK = C::BK, NSTAGE = C::NSTAGE;
   constexpr int NTEAM = C::NTEAM, TTHR = C::TTHR;
   constexpr int HPC = NC * 8;
@@ -711,9 +748,9 @@ qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
       const uint8_t* sMeta = sb + C::MOFF;
       if constexpr (C::XC) {
         // the team's warps are past the previous block (team_sync above), so
-        // its 8-bit tiles are free
+        // its compute tiles are free
         uint8_t* xt = ring + C::XTOFF;
-        transcode_block<C, D, SB>(sb, xt, ttid);
+        transcode_block<C, D, SB, BITS>(sb, xt, ttid);
         team_sync();
         sK = xt;
         sV = xt + C::CODES;
