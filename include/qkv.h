@@ -333,7 +333,7 @@ qkv_status qkv_llama_cache_to_blocks(int kind, const qkv_cache* src, int B, int 
  *  mask: NULL, none or causal (bottom-right); no additive mask.
  *  workspace: at least qsdpa_kview_workspace_size(...) bytes, 16-byte aligned
  *  (partial results of the split over L; no state between calls).  One
- *  launch, or two when the keys of a (batch, kv head, 16-row tile) are split
+ *  launch, or two when the keys of a (batch, kv head, 64-row tile) are split
  *  over several CTAs (the second is the decode's merge kernel).  Any Lq >= 1
  *  (decode and prefill).  L == 0 writes zeros. */
 qkv_status qsdpa_attention_kview(const void* q, int q_dtype, int B, int Hq, int Hkv, int Lq, int Dk,

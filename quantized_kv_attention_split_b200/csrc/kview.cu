@@ -8,27 +8,31 @@
 //   out[b, h, i, :] = softmax_j(q[b, h, i] * scale . Khat[b, h / G, j] (+ causal))
 //                     . Khat[b, h / G, j, :Dv]
 //
-// Work: units = (batch, kv head, tile of 16 (head, query) rows, row = head *
+// Work: units = (batch, kv head, tile of 64 (head, query) rows, row = head *
 // Lq + query), each split over `pieces` CTAs along L in blocks of 64 keys.
-// A CTA (8 warps):
-//  * stages the packed K rows and their scales (and biases) of each block by
-//    cp.async into a two-slot ring, then all threads dequantize the block once
-//    into an fp16 tile [64 keys][576] (rows padded by 16 bytes, so the
-//    fragment loads below are free of bank conflicts): fp16(scale*code+bias),
-//    one rounding, as the tcgen05 prefill dequantizes its tiles;
+// A CTA (16 warps):
+//  * stages the packed K rows and their scales (and biases) of the next block
+//    by cp.async into one raw slot while it computes on the current one; all
+//    threads dequantize a block once into an fp16 tile [64 keys][576] (rows
+//    padded by 16 bytes, so the fragment loads below are free of bank
+//    conflicts): fp16(scale*code+bias), one rounding, as the tcgen05 prefill
+//    dequantizes its tiles;
 //  * S^T[key][row] = K q^T on the m16n8k16 tensor op: warp w takes keys
-//    16 (w % 4) .. +16 and rows 8 (w / 4) .. +8 over the 36 k-steps, K from
-//    the tile (ldmatrix), q from an fp16 tile prescaled per row by a power of
-//    two (exact for normal values);
+//    16 (w % 4) .. +16 and rows 16 (w / 4) .. +16 over the 36 k-steps (four
+//    independent accumulator chains), K from the tile (ldmatrix), q from an
+//    fp16 tile prescaled per row by a power of two (exact for normal values);
 //  * the block maximum of each row (shuffles, then across the 4 key warps in
 //    shared memory) moves the running maximum; P = 2^(S - m) in fp16 goes to a
 //    [row][key] tile;
-//  * O^T[dim][row] += V^T P: warp w owns dims 64 w .. +64 of all 16 rows, V^T
+//  * O^T[dim][row] += V^T P: warp w owns dims 32 w .. +32 of all 64 rows, V^T
 //    read from the same K tile with the transposing ldmatrix (the view costs
 //    nothing), after rescaling its accumulators by the rows' factors.
-// A CTA that covered its whole unit writes the normalized output; otherwise
-// (m, l, O) go to the workspace in the split-K decode's partial layout and the
-// decode's merge kernel (decode_merge.cuh, 512-wide rows) folds them.
+// One dequantized block thus serves 64 rows (all 64 heads of a kv head's
+// tile), and the tensor ops of both products run 16 and 8 independent chains
+// per warp.  A CTA that covered its whole unit writes the normalized output;
+// otherwise (m, l, O) go to the workspace in the split-K decode's partial
+// layout and the decode's merge kernel (decode_merge.cuh, 512-wide rows)
+// folds them.
 #include <algorithm>
 
 #include "decode_merge.cuh"
@@ -39,11 +43,12 @@ namespace {
 
 constexpr int kKvDk = 576, kKvDv = 512;
 constexpr int kKvBN = 64;                       // keys per block
-constexpr int kKvRows = 16;                     // (head, query) rows per CTA
-constexpr int kKvThreads = 256;
+constexpr int kKvRows = 64;                     // (head, query) rows per CTA
+constexpr int kKvWarps = 16;
+constexpr int kKvThreads = 32 * kKvWarps;
 constexpr int kKvRowBytes = kKvDk * 2 + 16;     // padded fp16 row of the K and q tiles
 constexpr int kKvPRowBytes = kKvBN * 2 + 16;    // padded fp16 row of the P tile
-constexpr int kKvMaxGrid = 8 * 48;              // partial slots in the workspace (two per CTA)
+constexpr int kKvMaxGrid = 160;                 // CTAs whose partials the workspace holds (two slots each)
 
 template <bool Q8, int BITS, int GS>
 struct KvCfg {
@@ -56,10 +61,10 @@ struct KvCfg {
   static constexpr int Q_OFF = 0;
   static constexpr int K_OFF = Q_OFF + kKvRows * kKvRowBytes;
   static constexpr int P_OFF = K_OFF + kKvBN * kKvRowBytes;
-  static constexpr int RED_OFF = P_OFF + kKvRows * kKvPRowBytes;      // [4][16] floats
-  static constexpr int STAT_OFF = RED_OFF + 4 * kKvRows * 4;          // rowscale, m, alpha: [3][16]
+  static constexpr int RED_OFF = P_OFF + kKvRows * kKvPRowBytes;      // [4][64] floats
+  static constexpr int STAT_OFF = RED_OFF + 4 * kKvRows * 4;          // rowscale, m, alpha: [3][64]
   static constexpr int RAW_OFF = (STAT_OFF + 3 * kKvRows * 4 + 127) / 128 * 128;
-  static constexpr int SMEM = RAW_OFF + 2 * RAW;
+  static constexpr int SMEM = RAW_OFF + RAW;    // one raw slot: the next block lands during the math
   static constexpr int CPR = RB / 16;            // 16-byte code chunks per key
   static_assert(CODES % 16 == 0 && META % 16 == 0, "whole 16-byte units");
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
@@ -115,7 +120,8 @@ __global__ void __launch_bounds__(kKvThreads, 1) qsdpa_kview_kernel(const __grid
   uint8_t* const qt = smem + C::Q_OFF;
   uint8_t* const kt = smem + C::K_OFF;
   uint8_t* const pt = smem + C::P_OFF;
-  float* const red = reinterpret_cast<float*>(smem + C::RED_OFF);     // [4 key warps][16 rows]
+  uint8_t* const raw = smem + C::RAW_OFF;
+  float* const red = reinterpret_cast<float*>(smem + C::RED_OFF);     // [4 key warps][64 rows]
   float* const rsc = reinterpret_cast<float*>(smem + C::STAT_OFF);    // per-row logit scale
   float* const rm = rsc + kKvRows;                                    // running maximum
   float* const ral = rm + kKvRows;                                    // this block's factor
@@ -132,10 +138,10 @@ __global__ void __launch_bounds__(kKvThreads, 1) qsdpa_kview_kernel(const __grid
   const int rbase = cg * kKvRows;                        // first (head, query) row of the tile
   const int64_t L = p.L;
 
-  auto issue = [&](int64_t blk, int slot) {
+  auto issue = [&](int64_t blk) {
     const int64_t key0 = blk * kKvBN;
     const int nvalid = (int)min((int64_t)kKvBN, L - key0);
-    const uint32_t dst = smem_u32(smem + C::RAW_OFF + slot * C::RAW);
+    const uint32_t dst = smem_u32(raw);
     const uint8_t* src = p.kc + (row0 + key0) * C::RB;
     const int cbytes = nvalid * C::RB, mbytes = nvalid * C::NG * 2;
     for (int i = tid; i < C::CODES / 16; i += kKvThreads) {
@@ -156,34 +162,33 @@ __global__ void __launch_bounds__(kKvThreads, 1) qsdpa_kview_kernel(const __grid
   };
 
   grid_dep_wait();
-  if (blo < bhi) issue(blo, 0);
-  cp_async_commit();
-  if (blo + 1 < bhi) issue(blo + 1, 1);
+  if (blo < bhi) issue(blo);
   cp_async_commit();
 
   // q rows -> fp16, each row prescaled by a power of two so that its largest
   // magnitude lies in [2^14, 2^15) (exact for normal values); the logit scale
-  // of row r becomes scale log2(e) 2^-sigma_r.  16 threads per row.
+  // of row r becomes scale log2(e) 2^-sigma_r.  8 threads per row.
   {
-    const int r = tid >> 4, sub = tid & 15;             // 16 threads per row
+    constexpr int TPR = kKvThreads / kKvRows;           // threads per row
+    const int r = tid / TPR, sub = tid % TPR;
     const int row = rbase + r;
     const bool ok = row < p.G;
     const int hl = ok ? row / p.Lq : 0, qi = ok ? row - hl * p.Lq : 0;
     const uint16_t* qr = reinterpret_cast<const uint16_t*>(p.q) +
                          (((int64_t)b * p.Hq + (int64_t)hkv * p.Gq + hl) * p.Lq + qi) * kKvDk;
     float mx = 0.f;
-    for (int e = sub * 2; e < kKvDk; e += 32) {
+    for (int e = sub * 2; e < kKvDk; e += 2 * TPR) {
       const uint32_t w = ok ? *reinterpret_cast<const uint32_t*>(qr + e) : 0u;
       const float a = p.q_dtype == QKV_F16 ? half_bits_to_float((uint16_t)(w & 0xffff)) : __uint_as_float(w << 16);
       const float c = p.q_dtype == QKV_F16 ? half_bits_to_float((uint16_t)(w >> 16)) : __uint_as_float(w & 0xffff0000u);
       mx = fmaxf(mx, fmaxf(fabsf(a), fabsf(c)));
     }
 #pragma unroll
-    for (int off = 1; off < 16; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(~0u, mx, off));
+    for (int off = 1; off < TPR; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(~0u, mx, off));
     int sigma = mx > 0.f ? 14 - (int)(((__float_as_uint(mx) >> 23) & 0xff) - 127) : 0;
     sigma = max(-96, min(96, sigma));
     const float up = exp2i(sigma);
-    for (int e = sub * 2; e < kKvDk; e += 32) {
+    for (int e = sub * 2; e < kKvDk; e += 2 * TPR) {
       const uint32_t w = ok ? *reinterpret_cast<const uint32_t*>(qr + e) : 0u;
       const float a = p.q_dtype == QKV_F16 ? half_bits_to_float((uint16_t)(w & 0xffff)) : __uint_as_float(w << 16);
       const float c = p.q_dtype == QKV_F16 ? half_bits_to_float((uint16_t)(w >> 16)) : __uint_as_float(w & 0xffff0000u);
@@ -195,26 +200,24 @@ __global__ void __launch_bounds__(kKvThreads, 1) qsdpa_kview_kernel(const __grid
     }
   }
 
-  // running state: the O^T fragments of dims 64 warp .. +64 (4 m-tiles) of
-  // both 8-row n-tiles; the row sums l (kept by threads 0..15)
-  float O[4][2][4];
+  // running state: the O^T fragments of dims 32 warp .. +32 (2 m-tiles) of
+  // all 8 row n-tiles; the row sums l (kept by threads 0..63)
+  float O[2][8][4];
 #pragma unroll
-  for (int mt = 0; mt < 4; ++mt)
+  for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) O[mt][nt][0] = O[mt][nt][1] = O[mt][nt][2] = O[mt][nt][3] = 0.f;
-  float lsum = 0.f;                                      // row tid (tid < 16)
-  const int km = warp & 3, hn = warp >> 2;               // score tile: keys 16 km, rows 8 hn
+    for (int nt = 0; nt < 8; ++nt) O[mt][nt][0] = O[mt][nt][1] = O[mt][nt][2] = O[mt][nt][3] = 0.f;
+  float lsum = 0.f;                                      // row tid (tid < 64)
+  const int km = warp & 3, rn = warp >> 2;               // score tile: keys 16 km, rows 16 rn
   const uint32_t qbase = smem_u32(qt), kbase = smem_u32(kt), pbase = smem_u32(pt);
 
   for (int64_t blk = blo; blk < bhi; ++blk) {
-    const int slot = (int)((blk - blo) & 1);
     const int64_t key0 = blk * kKvBN;
     const int nvalid = (int)min((int64_t)kKvBN, L - key0);
-    cp_async_wait<1>();
+    cp_async_wait<0>();
     __syncthreads();                                     // block landed; last block's tiles are free
     // ---- dequantize the block into the fp16 K tile --------------------------
     {
-      const uint8_t* raw = smem + C::RAW_OFF + slot * C::RAW;
       const uint16_t* sc = reinterpret_cast<const uint16_t*>(raw + C::CODES);
       const uint16_t* bi = reinterpret_cast<const uint16_t*>(raw + C::CODES + C::META);
       for (int i = tid; i < kKvBN * C::CPR; i += kKvThreads) {
@@ -229,44 +232,60 @@ __global__ void __launch_bounds__(kKvThreads, 1) qsdpa_kview_kernel(const __grid
       }
     }
     __syncthreads();                                     // tile written; raw slot free
-    if (blk + 2 < bhi) issue(blk + 2, slot);
+    if (blk + 1 < bhi) issue(blk + 1);                   // lands during this block's math
     cp_async_commit();
 
-    // ---- scores of keys 16 km .. +16, rows 8 hn .. +8 ------------------------
-    float s[4] = {0.f, 0.f, 0.f, 0.f};
+    // ---- scores of keys 16 km .. +16, rows 16 rn .. +16 ----------------------
+    // two n-tiles of 8 rows, even and odd k-steps in separate accumulators
+    float s[2][2][4];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) s[h][nt][0] = s[h][nt][1] = s[h][nt][2] = s[h][nt][3] = 0.f;
     {
       const uint32_t aaddr = kbase + (16 * km + (lane & 15)) * kKvRowBytes + 8 * (lane >> 4) * 2;
-      const uint32_t baddr = qbase + (8 * hn + (lane & 7)) * kKvRowBytes + 8 * ((lane >> 3) & 1) * 2;
+      const uint32_t baddr = qbase + (16 * rn + 8 * (lane >> 4) + (lane & 7)) * kKvRowBytes +
+                             8 * ((lane >> 3) & 1) * 2;
 #pragma unroll 6
-      for (int ks = 0; ks < kKvDk / 16; ++ks) {
-        uint32_t a[4], b0, b1;
-        ldsm_x4(aaddr + ks * 32, a);
-        ldsm_x2(baddr + ks * 32, b0, b1);
-        mma_f16(s, a, b0, b1, s);
+      for (int ks = 0; ks < kKvDk / 16; ks += 2) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t a[4], bq[4];
+          ldsm_x4(aaddr + (ks + h) * 32, a);
+          ldsm_x4(baddr + (ks + h) * 32, bq);
+          mma_f16(s[h][0], a, bq[0], bq[1], s[h][0]);
+          mma_f16(s[h][1], a, bq[2], bq[3], s[h][1]);
+        }
       }
     }
-    // base-2 logits; keys past L, and past each row's causal limit, are -inf
-    const int r0 = 8 * hn + 2 * t;                        // rows of s[0], s[2] (s[1], s[3]: r0 + 1)
-    float lg[4];
+    // base-2 logits; keys past L, and past each row's causal limit, are -inf.
+    // lg[nt][i]: key 16 km + g + 8 (i >> 1), row 16 rn + 8 nt + 2 t + (i & 1)
+    float lg[2][4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int r = r0 + (i & 1);
-      const int key = 16 * km + g + 8 * (i >> 1);
-      bool vis = key < nvalid;
-      if (p.mask_kind == QKV_MASK_CAUSAL) {
-        const int row = rbase + r;
-        const int qi = row - (row / p.Lq) * p.Lq;
-        vis = vis && key0 + key <= L - p.Lq + qi;
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = 16 * rn + 8 * nt + 2 * t + (i & 1);
+        const int key = 16 * km + g + 8 * (i >> 1);
+        bool vis = key < nvalid;
+        if (p.mask_kind == QKV_MASK_CAUSAL) {
+          const int row = rbase + r;
+          const int qi = row - (row / p.Lq) * p.Lq;
+          vis = vis && key0 + key <= L - p.Lq + qi;
+        }
+        lg[nt][i] = vis ? (s[0][nt][i] + s[1][nt][i]) * rsc[r] : -INFINITY;
       }
-      lg[i] = vis ? s[i] * rsc[r] : -INFINITY;
-    }
-    float m0 = fmaxf(lg[0], lg[2]), m1 = fmaxf(lg[1], lg[3]);
 #pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-      m0 = fmaxf(m0, __shfl_xor_sync(~0u, m0, off));
-      m1 = fmaxf(m1, __shfl_xor_sync(~0u, m1, off));
+    for (int nt = 0; nt < 2; ++nt) {
+      float m0 = fmaxf(lg[nt][0], lg[nt][2]), m1 = fmaxf(lg[nt][1], lg[nt][3]);
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        m0 = fmaxf(m0, __shfl_xor_sync(~0u, m0, off));
+        m1 = fmaxf(m1, __shfl_xor_sync(~0u, m1, off));
+      }
+      const int r0 = 16 * rn + 8 * nt + 2 * t;
+      if (g == 0) { red[km * kKvRows + r0] = m0; red[km * kKvRows + r0 + 1] = m1; }
     }
-    if (g == 0) { red[km * kKvRows + r0] = m0; red[km * kKvRows + r0 + 1] = m1; }
     __syncthreads();
     if (tid < kKvRows) {
       const float bm = fmaxf(fmaxf(red[tid], red[kKvRows + tid]), fmaxf(red[2 * kKvRows + tid], red[3 * kKvRows + tid]));
@@ -276,13 +295,15 @@ __global__ void __launch_bounds__(kKvThreads, 1) qsdpa_kview_kernel(const __grid
     }
     __syncthreads();
     // ---- P = 2^(S - m) in fp16 to the [row][key] tile; partial row sums -----
-    {
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      const int r0 = 16 * rn + 8 * nt + 2 * t;
       const float mr0 = rm[r0], mr1 = rm[r0 + 1];
       float p4[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const float m = (i & 1) ? mr1 : mr0;
-        p4[i] = lg[i] == -INFINITY ? 0.f : ex2(lg[i] - m);
+        p4[i] = lg[nt][i] == -INFINITY ? 0.f : ex2(lg[nt][i] - m);
       }
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -302,33 +323,37 @@ __global__ void __launch_bounds__(kKvThreads, 1) qsdpa_kview_kernel(const __grid
     __syncthreads();
     if (tid < kKvRows)
       lsum = lsum * ral[tid] + ((red[tid] + red[kKvRows + tid]) + (red[2 * kKvRows + tid] + red[3 * kKvRows + tid]));
-    // ---- O^T[dims 64 warp ..][rows] += V^T P, V = the tile's first 512 dims ---
+    // ---- O^T[dims 32 warp ..][rows] += V^T P, V = the tile's first 512 dims ---
     {
-      float al[2][2];
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) { al[nt][0] = ral[8 * nt + 2 * t]; al[nt][1] = ral[8 * nt + 2 * t + 1]; }
+      for (int nt = 0; nt < 8; ++nt) {
+        const float a0 = ral[8 * nt + 2 * t], a1 = ral[8 * nt + 2 * t + 1];
 #pragma unroll
-      for (int mt = 0; mt < 4; ++mt)
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-          O[mt][nt][0] *= al[nt][0]; O[mt][nt][1] *= al[nt][1];
-          O[mt][nt][2] *= al[nt][0]; O[mt][nt][3] *= al[nt][1];
+        for (int mt = 0; mt < 2; ++mt) {
+          O[mt][nt][0] *= a0; O[mt][nt][1] *= a1;
+          O[mt][nt][2] *= a0; O[mt][nt][3] *= a1;
         }
+      }
       const int mi = lane >> 3, mj = lane & 7;           // ldmatrix: matrix, row
 #pragma unroll
       for (int kk = 0; kk < kKvBN / 16; ++kk) {
-        uint32_t bp[2][2];
+        uint32_t a[2][4];
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-          ldsm_x2(pbase + (8 * nt + (lane & 7)) * kKvPRowBytes + (16 * kk + 8 * ((lane >> 3) & 1)) * 2,
-                  bp[nt][0], bp[nt][1]);
+        for (int mt = 0; mt < 2; ++mt) {
+          const int d0 = 32 * warp + 16 * mt;
+          ldsm_x4_t(kbase + (16 * kk + mj + 8 * (mi >> 1)) * kKvRowBytes + (d0 + 8 * (mi & 1)) * 2, a[mt]);
+        }
 #pragma unroll
-        for (int mt = 0; mt < 4; ++mt) {
-          const int d0 = 64 * warp + 16 * mt;
-          uint32_t a[4];
-          ldsm_x4_t(kbase + (16 * kk + mj + 8 * (mi >> 1)) * kKvRowBytes + (d0 + 8 * (mi & 1)) * 2, a);
+        for (int np = 0; np < 4; ++np) {
+          uint32_t bp[4];                                // n-tiles 2 np and 2 np + 1
+          ldsm_x4(pbase + (16 * np + 8 * (lane >> 4) + (lane & 7)) * kKvPRowBytes +
+                      (16 * kk + 8 * ((lane >> 3) & 1)) * 2,
+                  bp);
 #pragma unroll
-          for (int nt = 0; nt < 2; ++nt) mma_f16(O[mt][nt], a, bp[nt][0], bp[nt][1], O[mt][nt]);
+          for (int mt = 0; mt < 2; ++mt) {
+            mma_f16(O[mt][2 * np], a[mt], bp[0], bp[1], O[mt][2 * np]);
+            mma_f16(O[mt][2 * np + 1], a[mt], bp[2], bp[3], O[mt][2 * np + 1]);
+          }
         }
       }
     }
@@ -342,7 +367,7 @@ __global__ void __launch_bounds__(kKvThreads, 1) qsdpa_kview_kernel(const __grid
   const bool complete = p.pieces == 1;
   const int64_t slot = 2 * (int64_t)blockIdx.x;
 #pragma unroll
-  for (int nt = 0; nt < 2; ++nt)
+  for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
       const int r = 8 * nt + 2 * t + j, row = rbase + r;
@@ -350,10 +375,10 @@ __global__ void __launch_bounds__(kKvThreads, 1) qsdpa_kview_kernel(const __grid
       const float l = red[r];
       const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
-      for (int mt = 0; mt < 4; ++mt)
+      for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
         for (int hi = 0; hi < 2; ++hi) {
-          const int dim = 64 * warp + 16 * mt + g + 8 * hi;
+          const int dim = 32 * warp + 16 * mt + g + 8 * hi;
           const float o = O[mt][nt][2 * hi + j];
           if (complete) store_from_float(p.out, p.out_dtype, (uh * p.G + row) * kKvDv + dim, o * inv);
           else p.part_o[(slot * kKvRows + r) * kKvDv + dim] = o;
@@ -429,7 +454,7 @@ cudaError_t launch_kview(int bits, int gs, int fmt, DecodeParams& p, cudaStream_
   p.stages_per_unit = S;
   p.total_stages = units * S;
   p.pieces = (int)pieces;
-  // the merge kernel's partial layout: o [slot][16][512], (m, l) [slot][16][2]
+  // the merge kernel's partial layout: o [slot][64][512], (m, l) [slot][64][2]
   float* part = p.part_o;
   p.part_ml = part + (size_t)2 * kKvMaxGrid * kKvRows * kKvDv;
   const bool q8 = fmt == QKV_Q8_0;

@@ -170,9 +170,9 @@ __device__ __forceinline__ bool mbar_try(uint32_t addr, uint32_t parity) {
   uint32_t done;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(done) : "r"(addr), "r"(parity), "r"(1000u) : "memory");
+      : "=r"(done) : "r"(addr), "r"(parity) : "memory");
   return done != 0;
 }
 __device__ __forceinline__ uint64_t pf_now_ns() {
@@ -505,14 +505,15 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint64_t wait_ns = p.wait_ns != 0 ? p.wait_ns : kPfWaitNs;
   const uint32_t bar0 = sbase + C::BAR_OFF;
-  auto raw_full = [&](int i) { return bar0 + 8 * i; };        // [4] packed half tile landed
-  auto k_ready = [&](int i) { return bar0 + 32 + 8 * i; };    // [2] fp16 K written
-  auto v_ready = [&](int i) { return bar0 + 48 + 8 * i; };    // [2] fp16 V written
-  auto s_full = [&](int i) { return bar0 + 64 + 8 * i; };     // [2] S in TMEM
-  auto p_ready = [&](int i) { return bar0 + 80 + 8 * i; };    // [2] P in TMEM
-  auto pv_done = [&](int i) { return bar0 + 96 + 8 * i; };    // [2] P V product done
-  const uint32_t mma_done = bar0 + 112;                       // all tensor-core work done
-  auto raw_free = [&](int i) { return bar0 + 120 + 8 * i; };  // [2] a tile's raw slots released
+  constexpr uint32_t RO = 8 * kPfRawSlots;                    // barriers after the raw ones
+  auto raw_full = [&](int i) { return bar0 + 8 * i; };        // [raw slots] packed half tile landed
+  auto k_ready = [&](int i) { return bar0 + RO + 8 * i; };    // [2] fp16 K written
+  auto v_ready = [&](int i) { return bar0 + RO + 16 + 8 * i; };   // [2] fp16 V written
+  auto s_full = [&](int i) { return bar0 + RO + 32 + 8 * i; };    // [2] S in TMEM
+  auto p_ready = [&](int i) { return bar0 + RO + 48 + 8 * i; };   // [2] P in TMEM
+  auto pv_done = [&](int i) { return bar0 + RO + 64 + 8 * i; };   // [2] P V product done
+  const uint32_t mma_done = bar0 + RO + 80;                   // all tensor-core work done
+  auto raw_free = [&](int i) { return bar0 + RO + 88 + 8 * i; };  // [2] a tile's raw slots released
   {
     // the range flag was written by the range check kernel, two kernels
     // earlier in the stream: the first instance runs when it is down, the
@@ -532,9 +533,10 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
       return;
     }
   }
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::BAR_OFF + 144);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::BAR_OFF + 148);
-  volatile uint32_t* range_ring = reinterpret_cast<volatile uint32_t*>(smem + C::BAR_OFF + 160);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::BAR_OFF + RO + 112);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::BAR_OFF + RO + 116);
+  volatile uint32_t* range_ring = reinterpret_cast<volatile uint32_t*>(smem + C::BAR_OFF + RO + 128);
+  static_assert(8 * kPfRawSlots + 128 + 4 * kPfRangeRing <= 256, "barrier area");
 
   const int mt = blockIdx.x % p.mtiles;
   const int hkv = (blockIdx.x / p.mtiles) % p.Hkv;
