@@ -2,9 +2,10 @@
 first 512 elements: the "576/512 MLA" shape of the llama.cpp PR's follow-up
 tests) through the C ABI (qsdpa_attention_kview), against the oracle's
 attention_kview, element by element: Q8_0 and affine 4/8-bit caches, decode
-(one query) and multi-query with and without the causal limit, a single
-16-row tile and many (128 query heads over one KV head), ragged L, units
-split over CTAs (merged by the merge kernel) and whole."""
+(one query) and multi-query with and without the causal limit, one 64-row tile partly
+filled and several (128 query heads over one KV head; 96 heads: a ragged
+second tile), ragged L, units split over CTAs (merged by the merge kernel)
+and whole."""
 import numpy as np
 import pytest
 import torch
@@ -28,7 +29,9 @@ def _problem(B, Hq, Hkv, Lq, L, fmt, bits, gs, seed, dist="normal", q_dtype="bf1
 CASES = [
     # B, Hq, Hkv, Lq, L, fmt, bits, gs
     (1, 16, 1, 1, 4099, "q8_0", 8, 32),       # one tile, split over many CTAs
-    (1, 128, 1, 1, 2048, "q8_0", 8, 32),      # 8 tiles (DeepSeek-like head count)
+    (1, 128, 1, 1, 2048, "q8_0", 8, 32),      # 2 tiles (DeepSeek-like head count)
+    (1, 96, 1, 1, 3001, "q8_0", 8, 32),       # a full tile and a half-filled one
+    (1, 64, 1, 2, 700, "affine", 4, 64),      # multi-query: 128 rows, 2 tiles
     (2, 32, 2, 1, 777, "affine", 8, 64),
     (1, 16, 2, 1, 1000, "affine", 4, 32),
     (1, 8, 1, 1, 90, "affine", 4, 64),        # short: one CTA per unit, written whole
