@@ -861,13 +861,27 @@ def other_rows(device):
     sec, _ = graph_time(lambda i: qkv.qsdpa_prefill(q, kc, vc, w.L, w.scale, causal=True, out=out,
                                                     workspace=ws, softcap=30.0, sinks=sinks),
                         20, 3)
+    # ALiBi: per-query distances (fp32 [Lq, L], -inf above the causal
+    # diagonal, broadcast over heads) with per-head slopes
+    qpos = torch.arange(w.L - w.Lq, w.L, device=device).view(-1, 1)
+    dist = (torch.arange(w.L, device=device).view(1, -1) - qpos).float()
+    alibi = torch.where(dist <= 0, dist, torch.full_like(dist, -float("inf"))).contiguous()
+    slopes = torch.tensor([2.0 ** (-8.0 * (h + 1) / w.Hq) for h in range(w.Hq)], device=device)
+    sec_m, _ = graph_time(lambda i: qkv.qsdpa_prefill(q, kc, vc, w.L, w.scale, mask=(alibi, (0, 0, w.L)),
+                                                      out=out, workspace=ws, mask_slopes=slopes),
+                          10, 3)
     flop = prefill_flops(w)
     _, bf16_peak, _ = peaks()
     rows["extensions_" + w.name] = {
         "softcap_sinks_us_per_call": round(sec * 1e3, 2),
         "TFLOP/s": round(flop / (sec / 1e3) / 1e12, 1),
         "frac_tensor_peak": round(flop / (sec / 1e3) / 1e12 / bf16_peak, 4),
-        "note": "qsdpa_prefill_ext, softcap 30 + per-head sinks; compare prefill_q8_0_512_at_20k"}
+        "alibi_mask_us_per_call": round(sec_m * 1e3, 2),
+        "alibi_mask_frac_tensor_peak": round(flop / (sec_m / 1e3) / 1e12 / bf16_peak, 4),
+        "note": "qsdpa_prefill_ext, softcap 30 + per-head sinks; and an ALiBi additive mask (fp32 "
+                "[Lq, L] distances, -inf above the causal diagonal, broadcast over heads) with "
+                "per-head slopes; compare prefill_q8_0_512_at_20k"}
+    del alibi, dist
     del kc, vc
     torch.cuda.empty_cache()
     return rows

@@ -8,10 +8,10 @@ namespace qkv {
 
 namespace {
 
-template <int D, int BITS, int GS, bool Q8, bool EXT, bool RANGE>
+template <int D, int BITS, int GS, bool Q8, int VAR, bool RANGE>
 cudaError_t launch_pf_r(const PrefillParams& p, int grid, cudaStream_t s) {
   using C = PfCfg<D, BITS, GS, Q8>;
-  auto k = qsdpa_prefill_tc_kernel<D, BITS, GS, Q8, EXT, RANGE>;
+  auto k = qsdpa_prefill_tc_kernel<D, BITS, GS, Q8, VAR, RANGE>;
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
@@ -25,7 +25,7 @@ cudaError_t launch_pf_r(const PrefillParams& p, int grid, cudaStream_t s) {
 // A call: the range check of the cache's scales and biases, then the kernel
 // and its range-scaled instance (one of the two runs, the other exits at
 // once).
-template <int D, int BITS, int GS, bool Q8, bool EXT>
+template <int D, int BITS, int GS, bool Q8, int VAR>
 cudaError_t launch_pf_v(const PrefillParams& p, int grid, cudaStream_t s) {
   const int ng = D / GS;
   const int64_t units = (p.L * ng + 7) / 8;
@@ -35,17 +35,20 @@ cudaError_t launch_pf_v(const PrefillParams& p, int grid, cudaStream_t s) {
   qkv_range_check_kernel<Q8, BITS><<<dim3(cx, (unsigned)slabs), 256, 0, s>>>(p, ng);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  e = launch_pf_r<D, BITS, GS, Q8, EXT, false>(p, grid, s);
+  e = launch_pf_r<D, BITS, GS, Q8, VAR, false>(p, grid, s);
   if (e != cudaSuccess) return e;
-  return launch_pf_r<D, BITS, GS, Q8, EXT, true>(p, grid, s);
+  return launch_pf_r<D, BITS, GS, Q8, VAR, true>(p, grid, s);
 }
 
-// the extension instance only when an extension is in use
+// the extension instance only when an extension is in use; additive masks
+// (with or without slopes) and no softcap or sinks: the mask instance
 template <int D, int BITS, int GS, bool Q8>
 cudaError_t launch_pf(const PrefillParams& p, int grid, cudaStream_t s) {
+  if (p.mask_kind == QKV_MASK_ADDITIVE && !(p.cap_a > 0.f) && p.sinks == nullptr)
+    return launch_pf_v<D, BITS, GS, Q8, kPfMask>(p, grid, s);
   if (p.cap_a > 0.f || p.slopes != nullptr || p.sinks != nullptr)
-    return launch_pf_v<D, BITS, GS, Q8, true>(p, grid, s);
-  return launch_pf_v<D, BITS, GS, Q8, false>(p, grid, s);
+    return launch_pf_v<D, BITS, GS, Q8, kPfExt>(p, grid, s);
+  return launch_pf_v<D, BITS, GS, Q8, kPfPlain>(p, grid, s);
 }
 
 template <int D>

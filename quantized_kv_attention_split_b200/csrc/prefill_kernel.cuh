@@ -239,6 +239,14 @@ __device__ __forceinline__ int pf_range_exp(float bound) {
   return min(31, max(0, ex - 14));
 }
 
+// Cache-line prefetches of global memory (no data returned, no fault).
+__device__ __forceinline__ void prefetch_l1(const void* a) {
+  asm volatile("prefetch.global.L1 [%0];\n" :: "l"(a));
+}
+__device__ __forceinline__ void prefetch_l2(const void* a) {
+  asm volatile("prefetch.global.L2 [%0];\n" :: "l"(a));
+}
+
 // One contiguous global -> shared copy completing on an mbarrier (no multicast).
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile(
@@ -469,6 +477,33 @@ __device__ __forceinline__ void pf_unpack(uint4 r, const __nv_bfloat16*, float* 
   }
 }
 
+// The common case of pf_add_mask (mask instance), taken when every key of the
+// tile is visible to every row of the warp and the slope is positive: sv[j]
+// (raw products) becomes rs * sv[j] + slope * mask[j] in two operations, with
+// no per-key selects (a -inf mask entry still gives -inf: slope * -inf is
+// -inf and the products are finite).
+template <typename T>
+__device__ __forceinline__ void pf_scale_add_mask(float (&sv)[kPfBN], const T* m, float rs, float slope) {
+  constexpr int EPV = 16 / (int)sizeof(T);              // elements per 16-byte read
+  const bool vec = (reinterpret_cast<uintptr_t>(m) & 15u) == 0;
+#pragma unroll
+  for (int c = 0; c < kPfBN; c += 16) {
+#pragma unroll
+    for (int v = c; v < c + 16; v += EPV) {
+      float mv[EPV];
+      if (vec) {
+        pf_unpack(__ldg(reinterpret_cast<const uint4*>(m + v)), m, mv);
+      } else {
+#pragma unroll
+        for (int e = 0; e < EPV; ++e) mv[e] = to_float_ld(m + v + e);
+      }
+#pragma unroll
+      for (int e = 0; e < EPV; ++e) sv[v + e] = fmaf(sv[v + e], rs, slope * mv[e]);
+    }
+    asm volatile("" ::: "memory");
+  }
+}
+
 template <typename T>
 __device__ __forceinline__ void pf_add_mask(float (&sv)[kPfBN], const T* m, int lim, float slope) {
   constexpr int EPV = 16 / (int)sizeof(T);              // elements per 16-byte read
@@ -492,11 +527,17 @@ __device__ __forceinline__ void pf_add_mask(float (&sv)[kPfBN], const T* m, int 
   }
 }
 
-// EXT: the instance with the attention extensions (logit softcap, additive-mask
-// slopes, sinks); the plain instance carries none of their code.  RANGE: the
-// second instance of a call (see the range note above).
-template <int D, int BITS, int GS, bool Q8, bool EXT, bool RANGE>
+// VAR: kPfPlain; kPfExt, the instance with the attention extensions (logit
+// softcap, additive-mask slopes, sinks), which the plain instance carries no
+// code for; kPfMask, the one for additive masks (with or without slopes) and
+// no other extension, which reads each tile's mask in one pass with the
+// scaling of S and fetches the next tiles' entries ahead.  RANGE: the second
+// instance of a call (see the range note above).
+enum : int { kPfPlain = 0, kPfExt = 1, kPfMask = 2 };
+template <int D, int BITS, int GS, bool Q8, int VAR, bool RANGE>
 __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const PrefillParams p) {
+  constexpr bool EXT = VAR == kPfExt;
+  constexpr bool AMASK = VAR == kPfMask;
   using C = PfCfg<D, BITS, GS, Q8>;
   constexpr int NG = C::NG;
   extern __shared__ uint8_t smem_raw[];
@@ -888,12 +929,27 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
     const bool causal = p.mask_kind == QKV_MASK_CAUSAL;
     const bool additive = p.mask_kind == QKV_MASK_ADDITIVE;
     const bool capped = EXT && p.cap_a > 0.f;    // logit softcap
-    const float slope = kLog2e * (EXT && additive && p.slopes != nullptr && row_ok
+    const float slope = kLog2e * ((EXT || AMASK) && additive && p.slopes != nullptr && row_ok
                                       ? p.slopes[hkv * p.G + hh] : 1.f);
     float m_used = -INFINITY, lsum = 0.f;
+    // additive mask: this row's entries, mbase + key (elements of esz bytes)
+    const int64_t mbase = (int64_t)b * p.msb + ((int64_t)hkv * p.G + hh) * p.msh + (int64_t)qi * p.msq;
     for (int t = 0; t < ntiles; ++t) {
       const int s = t & 1;
       const int64_t key0 = (int64_t)t * kPfBN;
+      if constexpr (AMASK) {
+        if (additive && row_ok) {
+          // the row's mask entries of the next tile into L1 and of the one
+          // after into L2 while this tile's S is computed (keys below L only,
+          // so every address lies in the row)
+          const int esz = p.mask_dtype == QKV_F32 ? 4 : 2;
+          const char* mr = static_cast<const char*>(p.mask) + (mbase + key0) * esz;
+          if (key0 + kPfBN < kend) prefetch_l1(mr + kPfBN * esz);
+          if (key0 + kPfBN + 128 / esz < kend) prefetch_l1(mr + kPfBN * esz + 128);
+          if (key0 + 2 * kPfBN < kend) prefetch_l2(mr + 2 * kPfBN * esz);
+          if (key0 + 2 * kPfBN + 128 / esz < kend) prefetch_l2(mr + 2 * kPfBN * esz + 128);
+        }
+      }
       mbar_wait(s_full(s), (t >> 1) & 1, abort_flag, p.status, 8u, wait_ns);
       tc_fence_after();
       // second instance: S of this tile was computed from K * 2^-eK: scale it
@@ -931,6 +987,16 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
         int64_t nv = kend - key0;
         if (causal && causal_lim - key0 + 1 < nv) nv = causal_lim - key0 + 1;
         const int lim = !row_ok || nv <= 0 ? 0 : nv >= kPfBN ? kPfBN : (int)nv;
+        if (AMASK && additive && __all_sync(~0u, lim == kPfBN && slope > 0.f)) {
+          // every key visible to every row of the warp: scale and mask in one pass
+          const int64_t mrow = mbase + key0;
+          if (p.mask_dtype == QKV_F32)
+            pf_scale_add_mask(sv, reinterpret_cast<const float*>(p.mask) + mrow, rs, slope);
+          else if (p.mask_dtype == QKV_F16)
+            pf_scale_add_mask(sv, reinterpret_cast<const __half*>(p.mask) + mrow, rs, slope);
+          else
+            pf_scale_add_mask(sv, reinterpret_cast<const __nv_bfloat16*>(p.mask) + mrow, rs, slope);
+        } else {
 #pragma unroll
         for (int j = 0; j < kPfBN; ++j) {
           float v = sv[j] * rs;
@@ -938,14 +1004,14 @@ __global__ void __launch_bounds__(kPfThreads, 1) qsdpa_prefill_tc_kernel(const P
           sv[j] = j < lim ? v : -INFINITY;
         }
         if (additive) {
-          const int64_t mrow = (int64_t)b * p.msb + ((int64_t)hkv * p.G + hh) * p.msh +
-                               (int64_t)qi * p.msq + key0;
+          const int64_t mrow = mbase + key0;
           if (p.mask_dtype == QKV_F32)
             pf_add_mask(sv, reinterpret_cast<const float*>(p.mask) + mrow, lim, slope);
           else if (p.mask_dtype == QKV_F16)
             pf_add_mask(sv, reinterpret_cast<const __half*>(p.mask) + mrow, lim, slope);
           else
             pf_add_mask(sv, reinterpret_cast<const __nv_bfloat16*>(p.mask) + mrow, lim, slope);
+        }
         }
         float m0 = sv[0], m1 = sv[1];
 #pragma unroll

@@ -145,3 +145,43 @@ def test_prefill_additive_mask_half_dtypes_and_alignment(qkv, mdt, L):
     got = run_prefill(qkv, q, "bf16", kc, vc, L, 0.06, "f16", mask=(mt, st))
     assert np.all(got[0, 5, 3] == 0)
     assert max_err(got, ref) <= TOL["f16"], max_err(got, ref)
+
+
+@pytest.mark.parametrize("mdt", ["f32", "bf16"])
+@pytest.mark.parametrize("negative", [False, True])
+def test_prefill_mask_instance_one_pass_and_fallback(qkv, mdt, negative):
+    """Additive masks without softcap or sinks run on the mask instance of the
+    tcgen05 kernel: a tile whose keys are all visible to every row of a warp,
+    with positive slopes, is scaled and masked in one pass (a -inf entry stays
+    -inf through slope * mask); a negative slope in the warp, the ragged last
+    tile and a causal-style -inf band meet the per-key path.  Many tiles (L =
+    1000), a broadcast mask with per-head slopes, a query row hidden
+    entirely (zeros) and scattered -inf keys."""
+    B, Hq, Hkv, Lq, D, L = 1, 16, 2, 16, 128, 1000
+    q, kc, vc = make_problem(B, Hq, Hkv, Lq, D, L, "affine", 4, 64, "normal", q_dtype="bf16",
+                             Lcap=1008, seed=21)
+    rng = np.random.default_rng(7)
+    m32 = (4.0 * rng.standard_normal((Lq, L))).astype(np.float32)
+    m32[:, 300:340] = -np.inf
+    m32[3, :] = -np.inf
+    m32[5, ::7] = -np.inf
+    m32[9, 640:] = -np.inf
+    if mdt == "f32":
+        mb, mt = m32, torch.from_numpy(m32).cuda()
+    else:
+        mb = S.f32_to_half_bits(m32, mdt)
+        mt = to_dev(mb, mdt)
+    slopes = np.linspace(0.25, 1.5, Hq).astype(np.float32)
+    if negative:
+        slopes[1::5] *= -1.0
+    st = (0, 0, L)
+    scale = 1.0 / np.sqrt(D)
+    ref = oracle.attention(q, "bf16", kc, vc, L, scale, mask=oracle.Mask("additive", mb, mdt, st),
+                           ext=oracle.Ext(slopes=slopes.astype(np.float64)))
+    out = qkv.qsdpa_prefill(to_dev(q, "bf16"), cache_to_dev(kc), cache_to_dev(vc), L, scale,
+                            mask=(mt, st), mask_slopes=torch.from_numpy(slopes).cuda(),
+                            out_dtype=torch.float16)
+    torch.cuda.synchronize()
+    got = from_dev(out)
+    assert np.all(got[:, :, 3] == 0)
+    assert max_err(got, ref) <= TOL["f16"], max_err(got, ref)
