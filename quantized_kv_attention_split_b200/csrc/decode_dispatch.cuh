@@ -110,8 +110,10 @@ bool decode_ops_for(int bits, int gs, bool q8, int nc, bool f32, int var, Decode
 }
 
 // Affine codes stored 2, 3, 5 or 6 bits wide: the plain kernel (no additive
-// mask, no extensions, no fused update), transcoding each block to the
-// 4-bit tile (2- and 3-bit codes) or the 8-bit tile (5- and 6-bit codes).
+// mask, no extensions, no fused update); 2-bit codes in groups of 64 or 128
+// computed as they are, the others transcoding each block to the 4-bit tile
+// (2-bit codes in groups of 32, 3-bit codes) or the 8-bit tile (5- and 6-bit
+// codes).
 template <int D>
 bool decode_ops_x_for(int bits, int gs, int nc, bool f32, DecodeOps* ops) {
 #define QKV_DEC_X(SB, GS)                                                                      \
@@ -131,7 +133,24 @@ bool decode_ops_x_for(int bits, int gs, int nc, bool f32, DecodeOps* ops) {
     if (gs == 64) QKV_DEC_X(SB, 64);                        \
     if constexpr (D >= 128) { if (gs == 128) QKV_DEC_X(SB, 128); } \
   } while (0)
-  if (bits == 2) QKV_DEC_XB(2);
+  if (bits == 2) {
+    // groups of 64 or 128: the 2-bit fragments themselves (whole words per
+    // lane); groups of 32: transcoded to 4-bit
+#define QKV_DEC_N2(GS)                                                                         \
+  do {                                                                                         \
+    if (nc == 1) *ops = f32 ? make_decode_ops<D, 2, GS, false, 1, true, kDecPlain>()           \
+                            : make_decode_ops<D, 2, GS, false, 1, false, kDecPlain>();         \
+    else if (nc == 2) *ops = f32 ? make_decode_ops<D, 2, GS, false, 2, true, kDecPlain>()      \
+                                 : make_decode_ops<D, 2, GS, false, 2, false, kDecPlain>();    \
+    else *ops = f32 ? make_decode_ops<D, 2, GS, false, 4, true, kDecPlain>()                   \
+                    : make_decode_ops<D, 2, GS, false, 4, false, kDecPlain>();                 \
+    return true;                                                                               \
+  } while (0)
+    if (gs == 64) QKV_DEC_N2(64);
+    if constexpr (D >= 128) { if (gs == 128) QKV_DEC_N2(128); }
+#undef QKV_DEC_N2
+    QKV_DEC_XB(2);
+  }
   if (bits == 3) QKV_DEC_XB(3);
   if (bits == 5) QKV_DEC_XB(5);
   if (bits == 6) QKV_DEC_XB(6);

@@ -64,7 +64,9 @@ __host__ __device__ constexpr uint32_t swz_pack(int c0, int c1, int c2, int c3) 
   return (uint32_t)(c0 | (c1 << 3) | (c2 << 6) | (c3 << 9));
 }
 __host__ __device__ constexpr uint32_t swizzle_coeffs(int D, int bits, int gs) {
-  return D == 64 ? (bits == 4 ? (gs == 32 ? swz_pack(1, 0, 0, 0) : swz_pack(2, 0, 0, 0))
+  return bits == 2 ? (D == 64 ? swz_pack(0, 0, 0, 0) : D == 128 ? swz_pack(1, 0, 0, 0)
+                      : (gs == 64 ? swz_pack(2, 1, 0, 0) : swz_pack(2, 0, 0, 0)))
+       : D == 64 ? (bits == 4 ? (gs == 32 ? swz_pack(1, 0, 0, 0) : swz_pack(2, 0, 0, 0))
                               : swz_pack(2, 4, 0, 0))
        : D == 128 ? (bits == 4 ? (gs == 32 ? swz_pack(1, 2, 0, 0) : swz_pack(2, 4, 0, 0))
                                : (gs == 32 ? swz_pack(2, 4, 2, 0)
@@ -108,9 +110,11 @@ __device__ __forceinline__ int swz_offset(int lin) {
   return (lin & ~0x7f) | ((((lin >> 4) & 7) ^ f) << 4) | (lin & 15);
 }
 
-// SB: the width of the codes as stored in the cache.  BITS (4 or 8) is the
-// width the fragment code computes with; SB != BITS (affine 2 or 3-bit codes,
-// computed as 4-bit; 5 or 6-bit codes, computed as 8-bit) stages each block's
+// SB: the width of the codes as stored in the cache.  BITS (2, 4 or 8) is the
+// width the fragment code computes with (2: groups of 64 or 128 only, one or
+// two whole words per lane and row); SB != BITS (affine 2-bit codes in groups
+// of 32 and 3-bit codes, computed as 4-bit; 5 or 6-bit codes, computed as
+// 8-bit) stages each block's
 // packed rows as they are (one little-endian bit stream per row; rows
 // straddle 16-byte units) and the team transcodes them into a tile of its own
 // before the block's math.
@@ -407,6 +411,8 @@ qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
   using C = DecCfg<D, BITS, GS, Q8, NC, SB>;
   static_assert(!C::XC || (!Q8 && VAR == kDecPlain && ((BITS == 4 && SB < 4) || (BITS == 8 && SB > 4 && SB < 8))),
                 "2- and 3-bit codes compute as 4-bit, 5- and 6-bit codes as 8-bit");
+  static_assert(BITS != 2 || (!Q8 && VAR == kDecPlain && GS >= 64),
+                "2-bit fragments: affine codes in groups of 64 or 128, plain variant");
   constexpr int NG = C::NG, KPG = C::KPG, MT = C::MT, BK = C::BK, NSTAGE = C::NSTAGE;
   constexpr int NTEAM = C::NTEAM, TTHR = C::TTHR;
   constexpr int HPC = NC * 8;
@@ -586,7 +592,9 @@ qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
     //  l / 8; matrices 0/1 hold keys 0-7, 2/3 keys 8-15 of the 16-key block,
     //  and matrices 0/2 the first, 1/3 the second 16-byte unit of a unit pair
     //  (x2 loads for 4-bit groups of 32: matrix 0 keys 0-7, matrix 1 keys 8-15).
-    constexpr bool VX2 = BITS == 4 && GS == 32;
+    // (x2 loads: a group of one 16-byte unit -- 4-bit codes in groups of 32,
+    // 2-bit codes in groups of 64)
+    constexpr bool VX2 = (BITS == 4 && GS == 32) || (BITS == 2 && GS == 64);
     const int vkey = (lane & 7) + (VX2 ? ((lane >> 3) & 1) * 8 : ((lane >> 4) & 1) * 8);
     const int vunit = VX2 ? 0 : ((lane >> 3) & 1);
     const int vl = swz_xor<C::SWZV>(vkey * C::RB + vunit * 16);
@@ -651,7 +659,13 @@ qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
       for (int s = 0; s < C::KSTEPS; ++s) {
         const int G = s / KPG, ks = s % KPG;
         int e[4];
-        if constexpr (BITS == 4) {
+        if constexpr (BITS == 2) {
+          // word m of the lane's words, code positions (2j, 2j+8) and
+          // (2j+1, 2j+9) (after a shift by 8 for j >= 2)
+          const int m = ks >> 2, j = ks & 3;
+          const int e0 = G * GS + (t * C::NW + m) * 16 + 2 * j;
+          e[0] = e0; e[1] = e0 + 8; e[2] = e0 + 1; e[3] = e0 + 9;
+        } else if constexpr (BITS == 4) {
           const int m = ks >> 1, hi2 = (ks & 1) * 2;
           const int e0 = G * GS + (t * C::NW + m) * 8 + hi2;
           e[0] = e0; e[1] = e0 + 4; e[2] = e0 + 1; e[3] = e0 + 5;
@@ -676,8 +690,16 @@ qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
       const float qscale16 = exp2i(sigma - 4);
 #pragma unroll
       for (int s = 0; s < C::KSTEPS; ++s) {
-        const float sc2 = BITS == 4 ? qscale16 : qscale;
-        bq[s][0] = pack_half2(qv[s][0] * qscale, qv[s][1] * qscale);
+        // the query at a code position that the masked word holds 2^k times
+        // too large carries 2^-k: 4-bit, odd nibbles x16; 2-bit, positions
+        // 2j, 2j+1 of a byte pair x4^(2j mod 4), x4^(2j+1 mod 4)
+        float sc1 = qscale, sc2 = BITS == 4 ? qscale16 : qscale;
+        if constexpr (BITS == 2) {
+          const bool odd = ((s % KPG) & 1) != 0;
+          sc1 = odd ? exp2i(sigma - 4) : qscale;
+          sc2 = odd ? exp2i(sigma - 6) : exp2i(sigma - 2);
+        }
+        bq[s][0] = pack_half2(qv[s][0] * sc1, qv[s][1] * sc1);
         bq[s][1] = pack_half2(qv[s][2] * sc2, qv[s][3] * sc2);
       }
       // group sums: reduce over t, then hand rows 2t, 2t+1 to every lane
@@ -783,7 +805,21 @@ qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
           }
 #pragma unroll
           for (int m = 0; m < C::NW; ++m) {
-            if constexpr (BITS == 4) {
+            if constexpr (BITS == 2) {
+              // 16 codes per word: masks leave code * 4^k * 2^-24 (k = 0..3)
+              // in each half, exact fp16 subnormals; the shifted word gives
+              // the upper 8 positions of each half
+#pragma unroll
+              for (int hb = 0; hb < 2; ++hb) {
+                const uint32_t y0 = hb ? w0[m] >> 8 : w0[m], y1 = hb ? w1[m] >> 8 : w1[m];
+                uint32_t a[4] = {y0 & 0x00030003u, y1 & 0x00030003u, y0 & 0x000C000Cu, y1 & 0x000C000Cu};
+                mma_f16(acc, a, bq[s][0], bq[s][1], acc);
+                ++s;
+                uint32_t a2[4] = {y0 & 0x00300030u, y1 & 0x00300030u, y0 & 0x00C000C0u, y1 & 0x00C000C0u};
+                mma_f16(acc, a2, bq[s][0], bq[s][1], acc);
+                ++s;
+              }
+            } else if constexpr (BITS == 4) {
               uint32_t a[4] = {w0[m] & 0x000F000Fu, w1[m] & 0x000F000Fu,
                                w0[m] & 0x00F000F0u, w1[m] & 0x00F000F0u};
               mma_f16(acc, a, bq[s][0], bq[s][1], acc);
@@ -987,7 +1023,7 @@ qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
           // value codes of the block: ldmatrix .trans gives lane (g, t) one
           // 16-bit unit of keys 2t and 2t+1 (and of 2t+8, 2t+9) per register:
           // the key pairs of the A operand, one unit (4 or 2 dims) per register
-          constexpr int PAIRS = VX2 ? 1 : (BITS == 4 ? GS / 64 : GS / 32);   // unit pairs per group
+          constexpr int PAIRS = VX2 ? 1 : (BITS == 2 ? GS / 128 : BITS == 4 ? GS / 64 : GS / 32);   // unit pairs per group
 #pragma unroll
           for (int pr = 0; pr < PAIRS; ++pr) {
             const uint32_t va = smem_u32(sV) + (vl ^ swz_xor<C::SWZV>(16 * st * C::RB + G * C::GB + 2 * pr * 16));
@@ -1002,11 +1038,22 @@ qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
 #pragma unroll
               for (int r = 0; r < 4; ++r) R[r] ^= 0x80808080u;
             }
-            constexpr int MPP = VX2 ? 2 : (BITS == 4 ? 4 : 2);       // m-tiles per pair
+            constexpr int MPP = BITS == 2 ? (VX2 ? 4 : 8) : VX2 ? 2 : (BITS == 4 ? 4 : 2);   // m-tiles per pair
 #pragma unroll
             for (int c = 0; c < MPP; ++c) {
               uint32_t a[4];
-              if constexpr (BITS == 4) {
+              if constexpr (BITS == 2) {
+                // code position k of each 16-bit unit: mask 3 << 2k leaves
+                // code * 4^k * 2^-24 (k = c mod 4), the upper positions after
+                // a shift by 8 (x2: the second row half; x4: m-tiles 4..7)
+                constexpr uint32_t kM[4] = {0x00030003u, 0x000C000Cu, 0x00300030u, 0x00C000C0u};
+                const uint32_t msk = kM[c & 3];
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                  const bool up = VX2 ? (r & 1) != 0 : c >= 4;
+                  a[r] = (up ? (R[r] >> 8) : R[r]) & msk;
+                }
+              } else if constexpr (BITS == 4) {
                 // nibble c of each unit (x2: nibbles c and c + 2 for the two row halves)
                 const int clo = c, chi = VX2 ? c + 2 : c;
 #pragma unroll
@@ -1061,7 +1108,9 @@ qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
       // codes entered as code*2^-24 (odd nibbles: code*2^-20; Q8_0: exact
       // codes); O of group G carries 2^tau
       const bool x16 = BITS == 4 && (i & 1) != 0;
-      const float f = exp2i((Q8 ? 0 : (x16 ? 20 : 24)) - tau[G]);
+      // 2-bit: m-tile i holds code position i mod 4 of its units, x4^(i mod 4)
+      const int x4 = BITS == 2 ? 2 * (i & 3) : 0;
+      const float f = exp2i((Q8 ? 0 : (x16 ? 20 : 24 - x4)) - tau[G]);
       reinterpret_cast<float4*>(ws)[mt * 32 + lane] =
           make_float4(fmaf(O[mt][0], f, beta[0][G]), fmaf(O[mt][1], f, beta[1][G]),
                       fmaf(O[mt][2], f, beta[0][G]), fmaf(O[mt][3], f, beta[1][G]));
@@ -1132,7 +1181,9 @@ qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
       const bool v1 = head + 1 < p.G;
       const int G = mt / KPG, i = mt % KPG;
       int dim, dj;
-      if constexpr (BITS == 4 && GS == 32) { dim = G * GS + 4 * gl + i; dj = 2; }
+      if constexpr (BITS == 2 && GS == 64) { dim = G * GS + 8 * gl + i; dj = 4; }
+      else if constexpr (BITS == 2) { dim = G * GS + 8 * gl + i; dj = 64; }
+      else if constexpr (BITS == 4 && GS == 32) { dim = G * GS + 4 * gl + i; dj = 2; }
       else if constexpr (BITS == 4) { dim = G * GS + 64 * (i >> 2) + 4 * gl + (i & 3); dj = 32; }
       else { dim = G * GS + 32 * (i >> 1) + 2 * gl + (i & 1); dj = 16; }
       float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
