@@ -609,7 +609,22 @@ qsdpa_decode_kernel(const __grid_constant__ DecodeParams p) {
     // Everything above touched only parameters and shared memory; inputs are
     // read, and the workspace written, only once the previous kernel of the
     // stream has completed (this launch may start early, overlapping its
-    // set-up with that kernel's tail).
+    // set-up with that kernel's tail).  Before waiting, one lane per team
+    // asks L2 for the team's first blocks (a prefetch reads no data into the
+    // CTA and L2 stays coherent with writes of the previous kernel, so it is
+    // safe to issue early): their copies then start from L2.
+    if (lane == 0 && chunk == 0) {
+#pragma unroll
+      for (int i = 0; i < NSTAGE - 1; ++i) {
+        const int blk = team + NTEAM * i;
+        if (blk >= nblk) break;
+        const int64_t key0 = (int64_t)(s0 + blk) * BK;
+        const int rows = (int)(p.Lcap - key0 < (int64_t)BK ? p.Lcap - key0 : (int64_t)BK);   // inside the cache
+        const int64_t grow = row0 + key0;
+        prefetch_l2_bulk(p.kc + grow * C::RBS, (uint32_t)(rows * C::RBS + 15) & ~15u);
+        prefetch_l2_bulk(p.vc + grow * C::RBS, (uint32_t)(rows * C::RBS + 15) & ~15u);
+      }
+    }
     grid_dep_wait();
     uint4 qraw[QPT];
     {

@@ -127,6 +127,12 @@ __device__ __forceinline__ void store4_from_float(void* p, int dtype, int64_t i,
 __device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
 __device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
 
+// Bulk prefetch of [a, a + bytes) into L2 (a 16-byte aligned, bytes a multiple
+// of 16; no data returned, no fault).
+__device__ __forceinline__ void prefetch_l2_bulk(const void* a, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" :: "l"(a), "r"(bytes) : "memory");
+}
+
 // a / b for non-negative 64-bit values, in 32-bit arithmetic when both fit
 // (the common case; 64-bit division costs several times more instructions).
 __device__ __forceinline__ int64_t udiv64(int64_t a, int64_t b) {
